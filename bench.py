@@ -1,0 +1,465 @@
+"""Benchmark of the fused MoE decode step on B200.
+
+Default workload: the large synthetic MoE decoder (16 layers, d_model 4096,
+32/8 heads of 128, 128 experts top-8, expert and shared FFN 1536, vocab
+64000, about 80 GB of bf16 weights) decoding greedily at batch 1 with a
+4095-position prefilled cache.  Each step streams about 7.6 GB, far more than
+the 126 MB L2, so no flush is needed between steps.
+
+One JSON line on rank 0.  ``--impl reference`` times the CPU oracle instead.
+Under torchrun each rank runs an independent replica (the path does not shard).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+NOMINAL_HBM_GBS = 8000.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ---- distributed plumbing (replicas only) -----------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def dist_init(ws, backend):
+    import datetime
+
+    import torch.distributed as dist
+
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+# ---- clocks -----------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---- bytes per step ---------------------------------------------------------------
+def step_bytes(m, B, T, lengths_after, union_per_step):
+    """Algorithmic bytes of one step: every weight read once (routed experts
+    counted once per distinct expert per layer), plus the KV read of each
+    sequence (its length after the append), the KV append, embedding rows and
+    the logits write."""
+    d, hd = m.d_model, m.head_dim
+    qkv = (m.n_q_heads + 2 * m.n_kv_heads) * hd * d
+    wo = d * m.n_q_heads * hd
+    router = m.n_experts * d
+    shared = 3 * m.shared_ffn * d
+    per_layer = 2 * (qkv + wo + router + shared + 2 * d)
+    expert = 3 * m.expert_ffn * d * 2
+    kv_read = sum(2 * m.n_layers * m.n_kv_heads * hd * L * 2 for L in lengths_after)
+    kv_write = 2 * m.n_layers * m.n_kv_heads * hd * B * T * 2
+    lm = (m.vocab * d + d) * 2
+    return (m.n_layers * per_layer + union_per_step * expert + lm + kv_read + kv_write
+            + B * T * d * 2 + B * T * m.vocab * 4)
+
+
+def profile_traffic(kernel_key: str):
+    """DRAM traffic per launch recorded by ncu in profiles/, if the kernel source
+    has not changed since the capture."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "megakernel_traffic.md")
+    src = os.path.join(ROOT, "decode_megakernel_06_b200", "csrc", "mk_kernel.cu")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or m.group(1) != sha:
+        return None
+    t = re.search(rf"{kernel_key}:\s*([0-9.]+)", text)
+    return float(t.group(1)) if t else None
+
+
+# ---- our arm ----------------------------------------------------------------------
+def build_workload(kind, B, device):
+    import torch
+
+    from synthetic import make_context_lengths, make_kv_cache, make_tokens, make_weights, workload
+
+    if kind == "small":
+        wl = workload("small") if B == 1 else workload("small_batch", B)
+    else:
+        wl = workload(kind, B) if kind == "large" else workload(kind)
+    m = wl.model
+    t0 = time.perf_counter()
+    w = make_weights(m, wl.seed, device)
+    torch.cuda.synchronize()
+    gen_s = time.perf_counter() - t0
+    return wl, m, w, gen_s
+
+
+def time_steps(dec, m, k, v, B, T, ctx, steps, warmup, device):
+    """Greedy decode on the device: step s reads the argmax of step s-1."""
+    import torch
+
+    from synthetic import make_tokens
+
+    n = warmup + steps
+    pos = torch.tensor([[ctx[b] + s * T for b in range(B)] for s in range(n)], dtype=torch.int32,
+                       device=device)
+    bufs = [torch.tensor(make_tokens(m.vocab, B * T, 123), dtype=torch.int32, device=device),
+            torch.empty(B * T, dtype=torch.int32, device=device)]
+    logits = torch.empty((B * T, m.vocab), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    for s in range(warmup):
+        rc = dec.step(bufs[s % 2], pos[s], B, T, k, v, logits, bufs[(s + 1) % 2])
+        assert rc == 0, rc
+    assert dec.status() == 0
+    dec.stats(reset=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        s = warmup + i
+        dec.step(bufs[s % 2], pos[s], B, T, k, v, logits, bufs[(s + 1) % 2])
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    st = dec.status()
+    assert st == 0, st
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total = ev[0].elapsed_time(ev[steps])
+    stats = dec.stats(reset=True)
+    return total, per, stats
+
+
+def time_e2e(dec, m, k, v, B, T, ctx, steps, warmup):
+    """Through the host-buffer entry point: H2D tokens/positions, the step, D2H
+    argmax, every step."""
+    import torch
+
+    from synthetic import make_tokens
+
+    th = torch.tensor(make_tokens(m.vocab, B * T, 321), dtype=torch.int32).pin_memory()
+    ph = torch.empty(B, dtype=torch.int32).pin_memory()
+    out = torch.empty(B * T, dtype=torch.int32).pin_memory()
+    for s in range(warmup):
+        ph.copy_(torch.tensor([ctx[b] + s * T for b in range(B)], dtype=torch.int32))
+        assert dec.step_host(th, ph, B, T, k, v, out) == 0
+        th.copy_(out)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(steps):
+        s = warmup + i
+        ph.copy_(torch.tensor([ctx[b] + s * T for b in range(B)], dtype=torch.int32))
+        assert dec.step_host(th, ph, B, T, k, v, out) == 0
+        th.copy_(out)
+    dt = time.perf_counter() - t0
+    return dt, (th.numel() + ph.numel()) * 4, out.numel() * 4
+
+
+def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1):
+    """The CPU oracle as it stands on the same workload: whole decode steps
+    (all layers), weights copied from the device on demand; the copy time is
+    excluded from the compute time and reported beside it."""
+    import numpy as np
+
+    import oracle
+    from oracle import step as ostep
+    from synthetic import bf16_bits, make_tokens
+
+    threads = oracle.set_threads(0)
+    src = ostep.WeightSource(w, cache=False)
+    # only the sequences' live layers of the cache are needed; copy it once
+    kh = bf16_bits(k_dev[:, :B]).copy()
+    vh = bf16_bits(v_dev[:, :B]).copy()
+    toks = make_tokens(m.vocab, B * T, 555)
+    pos = list(ctx)
+    t_total = 0.0
+    fetch_before = 0.0
+    import time as _t
+
+    orig = src._get
+
+    def timed(key, fetch):
+        t0 = _t.perf_counter()
+        a = orig(key, fetch)
+        timed.fetch += _t.perf_counter() - t0
+        return a
+
+    timed.fetch = 0.0
+    src._get = timed
+    for _ in range(n_steps):
+        t0 = _t.perf_counter()
+        r = ostep.decode_step(m, src, kh, vh, toks, pos, B, T)
+        t_total += _t.perf_counter() - t0
+        toks = [int(x) for x in r.argmax]
+        pos = [p + T for p in pos]
+    compute = t_total - timed.fetch
+    return {"compute_s": compute, "fetch_s": timed.fetch, "steps": n_steps, "threads": threads,
+            "tokens": n_steps * B * T}
+
+
+def run_mine(args):
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+    from synthetic import make_context_lengths, make_kv_cache
+
+    ws, rank, local = dist_env()
+    device = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(device)
+    dist_init(ws, "nccl")
+    peaks, peaks_kind = load_peaks()
+    B = args.batch
+    wl, m, w, gen_s = build_workload(args.workload, B, device)
+    T = wl.tokens_per_step
+    bmax = max([B] + ([1, 2, 4, 8] if args.sweep else []))
+    steps_total = args.warmup + args.steps
+    cap_need = max(make_context_lengths(wl)) + (max(steps_total, 30) + 8) * T + 64
+    cap = (cap_need + 63) // 64 * 64
+    k, v = make_kv_cache(m, bmax, cap, wl.seed, device)
+    ctx = make_context_lengths(wl)
+    dec = mk.Decoder(m, w, max_rows=bmax * T, max_seqs=bmax, kv_capacity=cap,
+                     variant=args.variant)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    total_ms, per, stats = time_steps(dec, m, k, v, B, T, ctx, args.steps, args.warmup, device)
+    clk = clocks.stop()
+
+    union_per_step = stats.expert_union_total / max(1, args.steps)
+    lens = [[ctx[b] + (args.warmup + i) * T + T for b in range(B)] for i in range(args.steps)]
+    bytes_steps = [step_bytes(m, B, T, L, union_per_step) for L in lens]
+    alg_bytes = sum(bytes_steps) / len(bytes_steps)
+    ms_per_step = total_ms / args.steps
+    max_total = max_over_ranks(total_ms, device)
+    tokens_all = sum_over_ranks(args.steps * B * T, device)
+    value = tokens_all / (max_total / 1e3)
+    achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    launches = int(stats.kernel_launches)
+
+    # end to end through the host-buffer entry point (fresh positions)
+    e2e_steps = max(3, min(args.steps, 20))
+    dt, bi, bo = time_e2e(dec, m, k, v, B, T, ctx, e2e_steps, 2)
+    e2e = {"value": e2e_steps * B * T / dt, "unit": "tokens/s", "h2d_bytes_per_step": bi,
+           "d2h_bytes_per_step": bo, "steps": e2e_steps}
+
+    sweep = None
+    if args.sweep and ws == 1:
+        sweep = {}
+        for bb in (1, 2, 4, 8):
+            row = {}
+            for var in ("megakernel", "multikernel", "multikernel_graph"):
+                dec.set_variant(var)
+                n = max(5, min(args.steps, 20))
+                ctx_b = make_context_lengths(wl.__class__(wl.name, m, bb, T, wl.context,
+                                                          wl.context_range, wl.steps, wl.seed))
+                tot, _, st = time_steps(dec, m, k, v, bb, T, ctx_b, n, 3, device)
+                u = st.expert_union_total / n
+                Ls = [c + 3 * T + n * T // 2 + T for c in ctx_b]
+                by = step_bytes(m, bb, T, Ls, u)
+                row[var] = {"tok_s": round(n * bb * T / (tot / 1e3), 1),
+                            "ms_per_step": round(tot / n, 4),
+                            "hbm_gbs": round(by / (tot / n / 1e3) / 1e9, 1),
+                            "launches_per_step": st.kernel_launches // n}
+            sweep[f"bs{bb}"] = row
+        dec.set_variant(args.variant)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        o = oracle_sample(m, w, k, v, B, T, ctx, 1)
+        cpu = {"value": round(o["tokens"] / o["compute_s"], 4), "unit": "tokens/s",
+               "cores": o["threads"], "kind": "oracle",
+               "sample": (f"{o['steps']} full decode step(s) of the same workload on the host "
+                          f"(compute {o['compute_s']:.2f} s; weight copy from the device "
+                          f"{o['fetch_s']:.2f} s excluded)")}
+
+    traffic = profile_traffic(f"large_bs{B}_{args.variant}") if args.workload == "large" else None
+    if rank == 0:
+        line = {
+            "metric": "decode tokens/s/GPU at bs 1-8; achieved HBM GB/s vs 8 TB/s peak",
+            "value": round(value, 2), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "ms_per_step_p50": round(statistics.median(per), 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 weights / fp32 math", "data": "synthetic (seeded random weights, N(0,1) KV)",
+            "config": {"workload": wl.name, "model": m.name, "layers": m.n_layers,
+                       "d_model": m.d_model, "experts": f"{m.n_experts} top-{m.top_k}",
+                       "global_batch": B * ws, "tokens_per_step": T,
+                       "context": wl.context, "variant": args.variant, "parallelism": f"replicas x{ws}",
+                       "l2": "inputs larger than L2 (about 7.6 GB streamed per step)"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": f"{peaks_kind} copy bandwidth",
+                         "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "traffic": traffic, "algorithmic_bytes_per_step": int(alg_bytes),
+                         "expert_union_per_step": round(union_per_step, 2)},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "weight_gen_s": round(gen_s, 2),
+        }
+        if sweep is not None:
+            line["batch_sweep"] = sweep
+        print(json.dumps(line), flush=True)
+    dec.close()
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The CPU oracle, as it stands, timed on the host cores (rank 0 only)."""
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import torch
+
+    from synthetic import make_context_lengths, make_kv_cache
+
+    device = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(device)
+    B = args.batch
+    wl, m, w, gen_s = build_workload(args.workload, B, device)
+    T = wl.tokens_per_step
+    ctx = make_context_lengths(wl)
+    cap = (max(ctx) + (args.warmup + args.steps + 2) * T + 63) // 64 * 64
+    k, v = make_kv_cache(m, B, cap, wl.seed, device)
+    for _ in range(args.warmup):
+        oracle_sample(m, w, k, v, B, T, ctx, 1)
+    res = [oracle_sample(m, w, k, v, B, T, ctx, 1) for _ in range(args.steps)]
+    comp = sum(r["compute_s"] for r in res)
+    value = sum(r["tokens"] for r in res) / comp
+    line = {
+        "impl": "reference",
+        "metric": "decode tokens/s/GPU at bs 1-8; achieved HBM GB/s vs 8 TB/s peak",
+        "value": round(value, 4), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(comp / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp32 (bf16 weights)", "data": "synthetic (seeded random weights, N(0,1) KV)",
+        "config": {"workload": wl.name, "model": m.name, "global_batch": B, "tokens_per_step": T,
+                   "context": wl.context, "variant": "cpu oracle"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": res[0]["threads"],
+                         "kind": "oracle",
+                         "sample": "one full decode step per timed step; weight copies from the device excluded"},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default="large", choices=["large", "small", "tiny"])
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--variant", default="megakernel",
+                    choices=["megakernel", "multikernel", "multikernel_graph"])
+    ap.add_argument("--sweep", action=argparse.BooleanOptionalAction, default=True)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mine(args)
+
+
+if __name__ == "__main__":
+    main()

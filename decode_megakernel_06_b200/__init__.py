@@ -1,0 +1,281 @@
+"""Python binding of ``libmk.so``, the fused MoE decode-step library for B200.
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of ``libmk.so``; PyTorch supplies device memory and streams.  The
+ctypes functions carry the names of the C entry points in ``include/mk.h``;
+``Decoder`` is a thin convenience wrapper that takes torch tensors.
+
+There is no fallback: if ``libmk.so`` is missing or fails to load, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmk.so")
+
+MK_OK = 0
+MK_ERR_ARG = -1
+MK_ERR_CAPACITY = -2
+MK_ERR_CUDA = -3
+MK_ERR_LAUNCH = -4
+MK_ERR_TIMEOUT = -5
+MK_ERR_DEVICE_CHECK = -6
+MK_ERR_UNSUPPORTED = -7
+
+MK_MEGAKERNEL = 0
+MK_MULTIKERNEL = 1
+MK_MULTIKERNEL_GRAPH = 2
+VARIANTS = {"megakernel": MK_MEGAKERNEL, "multikernel": MK_MULTIKERNEL,
+            "multikernel_graph": MK_MULTIKERNEL_GRAPH}
+
+MK_FAULT_NONE = 0
+MK_FAULT_UNREACHABLE_WAIT = 1
+
+OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "LMHEAD"]
+
+
+class mk_model_desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_layers", "d_model", "n_q_heads", "n_kv_heads", "head_dim",
+        "n_experts", "top_k", "expert_ffn", "shared_ffn", "vocab")] + [
+        ("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float),
+        ("max_rows", ctypes.c_int32), ("max_seqs", ctypes.c_int32),
+        ("kv_capacity", ctypes.c_int32), ("variant", ctypes.c_int32)]
+
+
+class mk_layer_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "attn_norm", "wqkv", "wo", "ffn_norm", "router", "w_gate", "w_up", "w_down",
+        "ws_gate", "ws_up", "ws_down")]
+
+
+class mk_weights(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
+                ("lm_head", ctypes.c_void_p), ("layers", ctypes.POINTER(mk_layer_weights))]
+
+
+class mk_kv_cache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p)]
+
+
+class mk_stats(ctypes.Structure):
+    _fields_ = [("steps", ctypes.c_uint64), ("expert_union_total", ctypes.c_uint64),
+                ("kernel_launches", ctypes.c_uint64)]
+
+
+class mk_plan_info(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_ops", "n_cta", "warps_per_cta", "rows_per_tile", "mmax", "attn_chunk",
+        "attn_qsplit", "smem_bytes")] + [("scratch_bytes", ctypes.c_int64)]
+
+
+class MkError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"mk error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+_I32P = ctypes.POINTER(ctypes.c_int32)
+
+
+def lib():
+    """Load ``libmk.so``; raise if it is missing (no fallback exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with decode_megakernel_06_b200/build.py")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64
+    sig = {
+        "mk_create": (i32, [ctypes.POINTER(mk_model_desc), ctypes.POINTER(mk_weights), ctypes.POINTER(vp)]),
+        "mk_decode_step": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
+        "mk_decode_step_host": (i32, [vp, _I32P, _I32P, i32, i32, mk_kv_cache, vp, _I32P, vp]),
+        "mk_get_device_status": (i32, [vp, vp]),
+        "mk_last_device_error_op": (i32, [vp]),
+        "mk_last_error": (ctypes.c_char_p, []),
+        "mk_destroy": (None, [vp]),
+        "mk_set_variant": (i32, [vp, i32]),
+        "mk_set_timeout": (i32, [vp, u64]),
+        "mk_set_debug": (i32, [vp, vp, vp, vp]),
+        "mk_debug_inject": (i32, [vp, i32]),
+        "mk_get_stats": (i32, [vp, ctypes.POINTER(mk_stats), i32]),
+        "mk_validate_desc": (i32, [ctypes.POINTER(mk_model_desc)]),
+        "mk_plan_describe": (i32, [ctypes.POINTER(mk_model_desc), i32, i32, i32,
+                                   ctypes.POINTER(mk_plan_info), _I32P, _I32P, _I32P, _I32P, i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def mk_last_error() -> str:
+    return lib().mk_last_error().decode()
+
+
+def _check(rc: int) -> int:
+    if rc != MK_OK:
+        raise MkError(rc, mk_last_error())
+    return rc
+
+
+# ---- same-named wrappers of the C entry points ---------------------------------
+
+def mk_validate_desc(desc: mk_model_desc) -> int:
+    return lib().mk_validate_desc(ctypes.byref(desc))
+
+
+def mk_plan_describe(desc: mk_model_desc, n_sm: int, B: int, T: int):
+    """Returns (rc, mk_plan_info, [(type, layer, dep0, dep1)] per op)."""
+    info = mk_plan_info()
+    n = 7 * desc.n_layers + 2
+    arrs = [(ctypes.c_int32 * n)() for _ in range(4)]
+    rc = lib().mk_plan_describe(ctypes.byref(desc), n_sm, B, T, ctypes.byref(info),
+                                *[ctypes.cast(a, _I32P) for a in arrs], n)
+    ops = list(zip(*[list(a) for a in arrs])) if rc == MK_OK else []
+    return rc, info, ops
+
+
+def mk_create(desc: mk_model_desc, weights: mk_weights) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(lib().mk_create(ctypes.byref(desc), ctypes.byref(weights), ctypes.byref(h)))
+    return h
+
+
+def mk_decode_step(h, tokens: int, positions: int, B: int, T: int, kv: mk_kv_cache,
+                   out_logits: int, out_argmax: int, stream: int) -> int:
+    return lib().mk_decode_step(h, tokens, positions, B, T, kv, out_logits, out_argmax, stream)
+
+
+def mk_decode_step_host(h, tokens_host, positions_host, B: int, T: int, kv: mk_kv_cache,
+                        out_logits: int, out_argmax_host, stream: int) -> int:
+    return lib().mk_decode_step_host(h, tokens_host, positions_host, B, T, kv, out_logits,
+                                     out_argmax_host, stream)
+
+
+def mk_get_device_status(h, stream: int) -> int:
+    return lib().mk_get_device_status(h, stream)
+
+
+def mk_last_device_error_op(h) -> int:
+    return lib().mk_last_device_error_op(h)
+
+
+def mk_destroy(h) -> None:
+    lib().mk_destroy(h)
+
+
+def mk_set_variant(h, variant: int) -> int:
+    return lib().mk_set_variant(h, variant)
+
+
+def mk_set_timeout(h, ns: int) -> int:
+    return lib().mk_set_timeout(h, ns)
+
+
+def mk_set_debug(h, hidden: int, expert_ids: int, expert_w: int) -> int:
+    return lib().mk_set_debug(h, hidden, expert_ids, expert_w)
+
+
+def mk_debug_inject(h, fault: int) -> int:
+    return lib().mk_debug_inject(h, fault)
+
+
+def mk_get_stats(h, reset: bool = False) -> mk_stats:
+    s = mk_stats()
+    _check(lib().mk_get_stats(h, ctypes.byref(s), 1 if reset else 0))
+    return s
+
+
+# ---- convenience wrapper over torch tensors -------------------------------------
+
+def make_desc(model, max_rows: int, max_seqs: int, kv_capacity: int,
+              variant: int = MK_MEGAKERNEL) -> mk_model_desc:
+    """Descriptor from any object with the decoder's dimension attributes."""
+    return mk_model_desc(model.n_layers, model.d_model, model.n_q_heads, model.n_kv_heads,
+                         model.head_dim, model.n_experts, model.top_k, model.expert_ffn,
+                         model.shared_ffn, model.vocab, float(model.rope_theta),
+                         float(model.rms_eps), max_rows, max_seqs, kv_capacity, variant)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+class Decoder:
+    """A handle over torch-resident weights (dict as produced by the synthetic
+    generator: embed, final_norm, lm_head, layers[...])."""
+
+    def __init__(self, model, weights: Dict[str, object], max_rows: int, max_seqs: int,
+                 kv_capacity: int, variant: str = "megakernel"):
+        import torch
+
+        self.model = model
+        self.max_rows, self.max_seqs, self.kv_capacity = max_rows, max_seqs, kv_capacity
+        self.desc = make_desc(model, max_rows, max_seqs, kv_capacity, VARIANTS[variant])
+        layers = (mk_layer_weights * model.n_layers)()
+        for l, lw in enumerate(weights["layers"]):
+            layers[l] = mk_layer_weights(*[_ptr(lw.get(n)) for n in (
+                "attn_norm", "wqkv", "wo", "ffn_norm", "router", "w_gate", "w_up", "w_down",
+                "ws_gate", "ws_up", "ws_down")])
+        self._layers = layers
+        self._weights = weights
+        self.w = mk_weights(_ptr(weights["embed"]), _ptr(weights["final_norm"]),
+                            _ptr(weights["lm_head"]), layers)
+        self.h = mk_create(self.desc, self.w)
+        self._torch = torch
+
+    def close(self):
+        if self.h:
+            mk_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_variant(self, variant: str):
+        _check(mk_set_variant(self.h, VARIANTS[variant]))
+
+    def set_timeout(self, ns: int):
+        _check(mk_set_timeout(self.h, ns))
+
+    def set_debug(self, hidden=None, expert_ids=None, expert_w=None):
+        _check(mk_set_debug(self.h, _ptr(hidden), _ptr(expert_ids), _ptr(expert_w)))
+
+    def inject(self, fault: int):
+        _check(mk_debug_inject(self.h, fault))
+
+    def step(self, tokens, positions, B: int, T: int, k_cache, v_cache, logits, argmax,
+             stream=None) -> int:
+        """Enqueue one step (device tensors); returns the launch status code."""
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
+        return mk_decode_step(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
+                              _ptr(logits), argmax.data_ptr(), s.cuda_stream)
+
+    def step_host(self, tokens_host, positions_host, B: int, T: int, k_cache, v_cache,
+                  argmax_host, logits=None, stream=None) -> int:
+        """Host-buffer step: int32 CPU tensors in/out (pinned is fastest)."""
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
+        cast = lambda t: ctypes.cast(t.data_ptr(), _I32P)  # noqa: E731
+        return mk_decode_step_host(self.h, cast(tokens_host), cast(positions_host), B, T, kv,
+                                   _ptr(logits), cast(argmax_host), s.cuda_stream)
+
+    def status(self, stream=None) -> int:
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        return mk_get_device_status(self.h, s.cuda_stream)
+
+    def stats(self, reset: bool = False) -> mk_stats:
+        return mk_get_stats(self.h, reset)

@@ -1,0 +1,631 @@
+// mk_api.cu -- host side of libmk.so: descriptor validation, the planner,
+// tensor-map encoding, scratch ownership and the launches of the three
+// execution variants.  See include/mk.h for the contract of every entry point.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+
+using namespace mk;
+
+namespace {
+
+thread_local std::string g_err = "ok";
+
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                   \
+  do {                                                                                   \
+    cudaError_t e__ = (expr);                                                            \
+    if (e__ != cudaSuccess)                                                              \
+      return fail(MK_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e__));         \
+  } while (0)
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// ---- driver entry point for tensor-map encoding --------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows][cols] matrix, box [box_cols][box_rows].
+int encode_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+              uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MK_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0)
+    return fail(MK_ERR_ARG, "tensor base %p is not 16-byte aligned", base);
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MK_ERR_CUDA, "cuTensorMapEncodeTiled(rows=%llu, cols=%llu) failed: %d",
+                (unsigned long long)rows, (unsigned long long)cols, (int)r);
+  return MK_OK;
+}
+
+// ---- planning ---------------------------------------------------------------------
+struct Plan {
+  int M, mmax, rows_per_tile, n_hb;
+  int attn_qvp, attn_qsplit, attn_ppt, attn_chunk, attn_nch_max;
+  int n_ops, n_cta, n_warps;
+  size_t smem;
+};
+
+Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
+  Plan p{};
+  p.M = B * T;
+  p.mmax = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
+  p.rows_per_tile = p.mmax <= 4 ? 16 : 8;
+  p.n_hb = ceil_div(d.d_model, p.rows_per_tile);
+  const int G = d.n_q_heads / d.n_kv_heads;
+  p.attn_qvp = (G * T <= 4) ? 4 : 8;
+  p.attn_qsplit = ceil_div(G * T, p.attn_qvp);
+  p.attn_ppt = 2048 / d.head_dim;
+  p.n_cta = n_sm;
+  p.n_warps = n_sm * kWarpsPerCta;
+  // KV chunk: about one work item per warp, a multiple of the tile height, and
+  // few enough chunks per (sequence, kv head, query group) for a two-level merge.
+  long long total = (long long)B * d.n_kv_heads * p.attn_qsplit * d.kv_capacity;
+  int c = (int)((total + p.n_warps - 1) / p.n_warps);
+  c = std::max(c, ceil_div(d.kv_capacity, kMaxChunks));
+  c = std::max(c, p.attn_ppt);
+  c = ceil_div(c, p.attn_ppt) * p.attn_ppt;
+  p.attn_chunk = c;
+  p.attn_nch_max = ceil_div(d.kv_capacity, c);
+  p.n_ops = n_ops_for(d.n_layers);
+  p.smem = step_smem_bytes(p.n_ops);
+  return p;
+}
+
+struct Sizes {
+  size_t attn_o, attn_ml, attn_o1, attn_ml1, attn_cnt;
+};
+
+Sizes scratch_sizes(const mk_model_desc &d, int n_sm) {
+  Sizes s{};
+  for (int B = 1; B <= d.max_seqs; ++B)
+    for (int T = 1; B * T <= d.max_rows; ++T) {
+      Plan p = make_plan(d, n_sm, B, T);
+      size_t ngrp = (size_t)d.max_seqs * d.n_kv_heads * p.attn_qsplit;
+      s.attn_o = std::max(s.attn_o, ngrp * p.attn_nch_max * p.attn_qvp * d.head_dim);
+      s.attn_ml = std::max(s.attn_ml, ngrp * p.attn_qvp * 2 * p.attn_nch_max);
+      s.attn_o1 = std::max(s.attn_o1, ngrp * kL1Fan * p.attn_qvp * d.head_dim);
+      s.attn_ml1 = std::max(s.attn_ml1, ngrp * p.attn_qvp * 2 * kL1Fan);
+      s.attn_cnt = std::max(s.attn_cnt, ngrp * (kL1Fan + 1));
+    }
+  return s;
+}
+
+}  // namespace
+
+struct GraphEntry {
+  uint64_t key[12];
+  cudaGraphExec_t exec;
+};
+
+struct mk_handle {
+  mk_model_desc desc;
+  std::vector<mk_layer_weights> layers;
+  const void *embed, *final_norm, *lm_head;
+  int device, n_sm;
+  // device allocations owned by the handle
+  std::vector<void *> allocs;
+  CUtensorMap *tmaps;
+  const __nv_bfloat16 **norms;
+  float *h, *ss, *qkv, *o, *attn_o, *attn_ml, *attn_o1, *attn_ml1, *router_part, *gu_shared,
+      *gu_routed, *logits;
+  uint32_t *attn_cnt, *counters, *route_flag, *epoch;
+  Routing *routing;
+  ArgmaxPart *am_part;
+  float2 *rope;
+  int *error;
+  unsigned long long *stats_dev;
+  int32_t *io_tokens, *io_positions, *io_argmax;
+  size_t counters_bytes, route_bytes, attn_cnt_bytes;
+  // kv maps, re-encoded when the cache pointers change
+  void *kv_k, *kv_v;
+  CUtensorMap kmap, vmap;
+  // state
+  int variant;
+  unsigned long long timeout_ns;
+  float *dbg_hidden;
+  int32_t *dbg_ids;
+  float *dbg_w;
+  int inject;
+  int last_error_op;
+  mk_stats stats;
+  std::vector<GraphEntry> graphs;
+  cudaStream_t capture_stream;
+};
+
+extern "C" {
+
+MK_API const char *mk_last_error(void) { return g_err.c_str(); }
+
+MK_API int mk_validate_desc(const mk_model_desc *d) {
+  if (!d) return fail(MK_ERR_ARG, "desc is NULL");
+  if (d->n_layers < 1) return fail(MK_ERR_ARG, "n_layers must be >= 1");
+  if (d->d_model < 8 || d->d_model % 8) return fail(MK_ERR_ARG, "d_model must be a positive multiple of 8");
+  if (d->n_q_heads < 1 || d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads)
+    return fail(MK_ERR_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+  if (d->head_dim != 64 && d->head_dim != 128)
+    return fail(MK_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", d->head_dim);
+  if (d->n_experts < 1 || d->n_experts > kMaxExperts)
+    return fail(MK_ERR_UNSUPPORTED, "n_experts must be in [1, %d]", kMaxExperts);
+  if (d->top_k < 1 || d->top_k > d->n_experts || d->top_k > kMaxTopK)
+    return fail(MK_ERR_ARG, "top_k must be in [1, min(%d, n_experts)]", kMaxTopK);
+  if (d->expert_ffn < 16 || d->expert_ffn % 16) return fail(MK_ERR_ARG, "expert_ffn must be a positive multiple of 16");
+  if (d->shared_ffn < 0 || d->shared_ffn % 16) return fail(MK_ERR_ARG, "shared_ffn must be 0 or a multiple of 16");
+  if (d->vocab < 1) return fail(MK_ERR_ARG, "vocab must be >= 1");
+  if (d->max_rows < 1 || d->max_rows > kMaxRows)
+    return fail(MK_ERR_UNSUPPORTED, "max_rows must be in [1, %d]", kMaxRows);
+  if (d->max_seqs < 1 || d->max_seqs > d->max_rows) return fail(MK_ERR_ARG, "max_seqs must be in [1, max_rows]");
+  if (d->kv_capacity < 1) return fail(MK_ERR_ARG, "kv_capacity must be >= 1");
+  if (!(d->rope_theta > 0.f) || !(d->rms_eps >= 0.f)) return fail(MK_ERR_ARG, "rope_theta > 0 and rms_eps >= 0 required");
+  if (d->variant < MK_MEGAKERNEL || d->variant > MK_MULTIKERNEL_GRAPH) return fail(MK_ERR_ARG, "unknown variant %d", d->variant);
+  const long long kv_rows = (long long)d->n_layers * d->max_seqs * d->n_kv_heads * d->kv_capacity;
+  if (kv_rows >= (1ll << 31)) return fail(MK_ERR_UNSUPPORTED, "KV cache too large");
+  if ((long long)d->n_experts * d->expert_ffn >= (1ll << 31) || (long long)d->n_experts * d->d_model >= (1ll << 31))
+    return fail(MK_ERR_UNSUPPORTED, "expert tensors too large");
+  return MK_OK;
+}
+
+MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, int32_t T,
+                            mk_plan_info *info, int32_t *op_types, int32_t *op_layers,
+                            int32_t *op_dep0, int32_t *op_dep1, int32_t cap) {
+  int rc = mk_validate_desc(desc);
+  if (rc) return rc;
+  if (n_sm < 1) return fail(MK_ERR_ARG, "n_sm must be >= 1");
+  if (B < 1 || T < 1 || B > desc->max_seqs || B * T > desc->max_rows)
+    return fail(MK_ERR_CAPACITY, "B=%d T=%d outside max_seqs=%d max_rows=%d", B, T, desc->max_seqs, desc->max_rows);
+  Plan p = make_plan(*desc, n_sm, B, T);
+  if (info) {
+    info->n_ops = p.n_ops;
+    info->n_cta = p.n_cta;
+    info->warps_per_cta = kWarpsPerCta;
+    info->rows_per_tile = p.rows_per_tile;
+    info->mmax = p.mmax;
+    info->attn_chunk = p.attn_chunk;
+    info->attn_qsplit = p.attn_qsplit;
+    info->smem_bytes = (int32_t)p.smem;
+    Sizes s = scratch_sizes(*desc, n_sm);
+    const mk_model_desc &d = *desc;
+    size_t f = (size_t)d.max_rows * d.d_model * 2 + (size_t)d.max_rows * ceil_div(d.d_model, 8) +
+               (size_t)d.max_rows * (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim +
+               (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml + s.attn_o1 +
+               s.attn_ml1 + (size_t)ceil_div(d.d_model, kPanel) * kMaxRows * d.n_experts +
+               (size_t)kMaxRows * 2 * d.shared_ffn +
+               (size_t)std::min(d.n_experts, d.max_rows * d.top_k) * kMaxRows * 2 * d.expert_ffn +
+               (size_t)d.max_rows * d.vocab + (size_t)d.kv_capacity * d.head_dim;
+    info->scratch_bytes = (int64_t)(f * 4 + s.attn_cnt * 4 + (size_t)d.n_layers * sizeof(Routing) +
+                                    (size_t)p.n_warps * kMaxRows * sizeof(ArgmaxPart));
+  }
+  for (int i = 0; i < p.n_ops && i < cap; ++i) {
+    int d0, d1;
+    op_deps(i, desc->n_layers, &d0, &d1);
+    if (op_types) op_types[i] = op_type_of(i, desc->n_layers);
+    if (op_layers) op_layers[i] = op_layer_of(i, desc->n_layers);
+    if (op_dep0) op_dep0[i] = d0;
+    if (op_dep1) op_dep1[i] = d1;
+  }
+  return MK_OK;
+}
+
+MK_API void mk_destroy(mk_handle *h) {
+  if (!h) return;
+  for (auto &g : h->graphs) cudaGraphExecDestroy(g.exec);
+  if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
+  for (void *p : h->allocs) cudaFree(p);
+  delete h;
+}
+
+static int halloc(mk_handle *h, void **out, size_t bytes) {
+  void *p = nullptr;
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(&p, bytes);
+  if (e != cudaSuccess) return fail(MK_ERR_CUDA, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+  h->allocs.push_back(p);
+  e = cudaMemset(p, 0, bytes);
+  if (e != cudaSuccess) return fail(MK_ERR_CUDA, "cudaMemset failed: %s", cudaGetErrorString(e));
+  *out = p;
+  return MK_OK;
+}
+
+#define HALLOC(ptr, bytes)                                                      \
+  do {                                                                          \
+    int rc__ = halloc(h, reinterpret_cast<void **>(&(ptr)), (bytes));           \
+    if (rc__) {                                                                 \
+      std::string keep = g_err;                                                 \
+      mk_destroy(h);                                                            \
+      g_err = keep;                                                             \
+      return rc__;                                                              \
+    }                                                                           \
+  } while (0)
+
+MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle **out) {
+  if (!out) return fail(MK_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  int rc = mk_validate_desc(desc);
+  if (rc) return rc;
+  if (!w || !w->embed || !w->final_norm || !w->lm_head || !w->layers)
+    return fail(MK_ERR_ARG, "weights: embed, final_norm, lm_head and layers are required");
+  const mk_model_desc &d = *desc;
+  for (int l = 0; l < d.n_layers; ++l) {
+    const mk_layer_weights &lw = w->layers[l];
+    if (!lw.attn_norm || !lw.wqkv || !lw.wo || !lw.ffn_norm || !lw.router || !lw.w_gate || !lw.w_up ||
+        !lw.w_down)
+      return fail(MK_ERR_ARG, "layer %d: a required weight pointer is NULL", l);
+    if (d.shared_ffn > 0 && (!lw.ws_gate || !lw.ws_up || !lw.ws_down))
+      return fail(MK_ERR_ARG, "layer %d: shared expert weights are NULL but shared_ffn > 0", l);
+  }
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  int n_sm = 0, coop = 0;
+  CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
+  if (!coop) return fail(MK_ERR_LAUNCH, "device does not support cooperative launches");
+  const size_t smem = step_smem_bytes(n_ops_for(d.n_layers));
+  for (int mm : {1, 2, 4, 8}) {
+    int per = max_cta_per_sm(mm, smem);
+    if (per < 1) return fail(MK_ERR_LAUNCH, "kernel (M<=%d) cannot keep one CTA per SM with %zu B smem", mm, smem);
+  }
+
+  mk_handle *h = new mk_handle();
+  h->desc = d;
+  h->layers.assign(w->layers, w->layers + d.n_layers);
+  h->embed = w->embed;
+  h->final_norm = w->final_norm;
+  h->lm_head = w->lm_head;
+  h->device = dev;
+  h->n_sm = n_sm;
+  h->variant = d.variant;
+  h->timeout_ns = 1000000000ull;
+  h->inject = MK_FAULT_NONE;
+  h->last_error_op = -1;
+
+  const int L = d.n_layers, D = d.d_model, QKVW = (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim;
+  const int n_ops = n_ops_for(L), NW = n_sm * kWarpsPerCta;
+  Sizes s = scratch_sizes(d, n_sm);
+  const int umax = std::min(d.n_experts, d.max_rows * d.top_k);
+  HALLOC(h->tmaps, sizeof(CUtensorMap) * (size_t)(L * MAPS_PER_LAYER + 1));
+  HALLOC(h->norms, sizeof(void *) * 2 * L);
+  HALLOC(h->h, sizeof(float) * (size_t)kMaxRows * D);
+  HALLOC(h->ss, sizeof(float) * (size_t)kMaxRows * ceil_div(D, 8));
+  HALLOC(h->qkv, sizeof(float) * (size_t)kMaxRows * QKVW);
+  HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
+  HALLOC(h->attn_o, sizeof(float) * s.attn_o);
+  HALLOC(h->attn_ml, sizeof(float) * s.attn_ml);
+  HALLOC(h->attn_o1, sizeof(float) * s.attn_o1);
+  HALLOC(h->attn_ml1, sizeof(float) * s.attn_ml1);
+  h->attn_cnt_bytes = sizeof(uint32_t) * s.attn_cnt;
+  HALLOC(h->attn_cnt, h->attn_cnt_bytes);
+  HALLOC(h->router_part, sizeof(float) * (size_t)ceil_div(D, kPanel) * kMaxRows * d.n_experts);
+  HALLOC(h->routing, sizeof(Routing) * (size_t)L);
+  HALLOC(h->gu_shared, sizeof(float) * (size_t)kMaxRows * 2 * std::max(d.shared_ffn, 1));
+  HALLOC(h->gu_routed, sizeof(float) * (size_t)umax * kMaxRows * 2 * d.expert_ffn);
+  HALLOC(h->am_part, sizeof(ArgmaxPart) * (size_t)NW * kMaxRows);
+  HALLOC(h->rope, sizeof(float2) * (size_t)d.kv_capacity * (d.head_dim / 2));
+  h->counters_bytes = sizeof(uint32_t) * (size_t)n_ops * kCounterStride;
+  HALLOC(h->counters, h->counters_bytes);
+  h->route_bytes = sizeof(uint32_t) * (size_t)L * kCounterStride;
+  HALLOC(h->route_flag, h->route_bytes);
+  HALLOC(h->epoch, sizeof(uint32_t) * kCounterStride);
+  HALLOC(h->error, sizeof(int) * kCounterStride);
+  HALLOC(h->stats_dev, sizeof(unsigned long long) * 4);
+  HALLOC(h->logits, sizeof(float) * (size_t)d.max_rows * d.vocab);
+  HALLOC(h->io_tokens, sizeof(int32_t) * kMaxRows);
+  HALLOC(h->io_positions, sizeof(int32_t) * kMaxRows);
+  HALLOC(h->io_argmax, sizeof(int32_t) * kMaxRows);
+
+  // tensor maps of every weight matrix
+  std::vector<CUtensorMap> maps((size_t)L * MAPS_PER_LAYER + 1);
+  std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
+  auto enc = [&](int idx, const void *p, uint64_t rows, uint64_t cols) -> int {
+    return encode_2d(&maps[idx], p, rows, cols, kPanel, kBoxRows);
+  };
+  std::vector<const void *> norm_ptrs(2 * L);
+  for (int l = 0; l < L && rc == MK_OK; ++l) {
+    const mk_layer_weights &lw = w->layers[l];
+    const int b = l * MAPS_PER_LAYER;
+    const uint64_t E = d.n_experts, F = d.expert_ffn, Fs = d.shared_ffn;
+    rc = enc(b + MAP_WQKV, lw.wqkv, QKVW, D);
+    if (!rc) rc = enc(b + MAP_WO, lw.wo, D, (uint64_t)d.n_q_heads * d.head_dim);
+    if (!rc) rc = enc(b + MAP_ROUTER, lw.router, E, D);
+    if (!rc) rc = enc(b + MAP_WGATE, lw.w_gate, E * F, D);
+    if (!rc) rc = enc(b + MAP_WUP, lw.w_up, E * F, D);
+    if (!rc) rc = enc(b + MAP_WDOWN, lw.w_down, E * D, F);
+    if (!rc && Fs > 0) rc = enc(b + MAP_WSGATE, lw.ws_gate, Fs, D);
+    if (!rc && Fs > 0) rc = enc(b + MAP_WSUP, lw.ws_up, Fs, D);
+    if (!rc && Fs > 0) rc = enc(b + MAP_WSDOWN, lw.ws_down, D, Fs);
+    norm_ptrs[2 * l] = lw.attn_norm;
+    norm_ptrs[2 * l + 1] = lw.ffn_norm;
+  }
+  if (!rc) rc = enc(L * MAPS_PER_LAYER, w->lm_head, d.vocab, D);
+  if (rc) {
+    std::string keep = g_err;
+    mk_destroy(h);
+    g_err = keep;
+    return rc;
+  }
+  // rotary table: cos/sin of p * theta^(-2i/hd), angle in double, rounded to float
+  std::vector<float2> rope((size_t)d.kv_capacity * (d.head_dim / 2));
+  for (int p = 0; p < d.kv_capacity; ++p)
+    for (int i = 0; i < d.head_dim / 2; ++i) {
+      double inv_freq = std::pow((double)d.rope_theta, -2.0 * i / (double)d.head_dim);
+      double a = (double)p * inv_freq;
+      rope[(size_t)p * (d.head_dim / 2) + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+    }
+  cudaError_t e = cudaMemcpy(h->tmaps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->norms, norm_ptrs.data(), norm_ptrs.size() * sizeof(void *), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->capture_stream, cudaStreamNonBlocking);
+  if (e != cudaSuccess) {
+    mk_destroy(h);
+    return fail(MK_ERR_CUDA, "mk_create upload failed: %s", cudaGetErrorString(e));
+  }
+  *out = h;
+  g_err = "ok";
+  return MK_OK;
+}
+
+static int reset_sync_state(mk_handle *h, cudaStream_t s) {
+  CUDA_TRY(cudaMemsetAsync(h->counters, 0, h->counters_bytes, s));
+  CUDA_TRY(cudaMemsetAsync(h->route_flag, 0, h->route_bytes, s));
+  CUDA_TRY(cudaMemsetAsync(h->epoch, 0, sizeof(uint32_t) * kCounterStride, s));
+  CUDA_TRY(cudaMemsetAsync(h->attn_cnt, 0, h->attn_cnt_bytes, s));
+  CUDA_TRY(cudaMemsetAsync(h->error, 0, sizeof(int) * kCounterStride, s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  return MK_OK;
+}
+
+static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T,
+                       mk_kv_cache kv, float *logits, int32_t *argmax, Params &p, Plan &pl) {
+  const mk_model_desc &d = h->desc;
+  if (!tokens || !positions || !argmax) return fail(MK_ERR_ARG, "tokens, positions and out_argmax are required");
+  if (!kv.k || !kv.v) return fail(MK_ERR_ARG, "kv.k and kv.v are required");
+  if (B < 1 || T < 1) return fail(MK_ERR_ARG, "B and T must be >= 1");
+  if (B > d.max_seqs || (long long)B * T > d.max_rows)
+    return fail(MK_ERR_CAPACITY, "B=%d T=%d exceeds max_seqs=%d / max_rows=%d", B, T, d.max_seqs, d.max_rows);
+  if (T > d.kv_capacity) return fail(MK_ERR_CAPACITY, "T=%d exceeds kv_capacity=%d", T, d.kv_capacity);
+  if (reinterpret_cast<uintptr_t>(kv.k) % 16 || reinterpret_cast<uintptr_t>(kv.v) % 16)
+    return fail(MK_ERR_ARG, "KV cache pointers must be 16-byte aligned");
+  pl = make_plan(d, h->n_sm, B, T);
+  if (kv.k != h->kv_k || kv.v != h->kv_v) {
+    const uint64_t rows = (uint64_t)d.n_layers * d.max_seqs * d.n_kv_heads * d.kv_capacity;
+    int rc = encode_2d(&h->kmap, kv.k, rows, d.head_dim, d.head_dim, pl.attn_ppt);
+    if (!rc) rc = encode_2d(&h->vmap, kv.v, rows, d.head_dim, d.head_dim, pl.attn_ppt);
+    if (rc) {
+      h->kv_k = h->kv_v = nullptr;
+      return rc;
+    }
+    h->kv_k = kv.k;
+    h->kv_v = kv.v;
+  }
+  std::memset(&p, 0, sizeof p);
+  p.kmap = h->kmap;
+  p.vmap = h->vmap;
+  p.L = d.n_layers; p.d = d.d_model; p.Hq = d.n_q_heads; p.Hkv = d.n_kv_heads; p.hd = d.head_dim;
+  p.E = d.n_experts; p.topk = d.top_k; p.F = d.expert_ffn; p.Fs = d.shared_ffn; p.V = d.vocab;
+  p.Bmax = d.max_seqs; p.cap = d.kv_capacity; p.eps = d.rms_eps;
+  p.B = B; p.T = T; p.M = B * T; p.max_rows = d.max_rows;
+  p.n_cta = pl.n_cta; p.n_warps = pl.n_warps; p.op_begin = 0; p.op_end = pl.n_ops; p.n_ops = pl.n_ops;
+  p.rows_per_tile = pl.rows_per_tile; p.n_hb = pl.n_hb;
+  p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit; p.attn_qvp = pl.attn_qvp;
+  p.attn_ppt = pl.attn_ppt; p.attn_nch_max = pl.attn_nch_max;
+  p.tmaps = h->tmaps; p.norms = h->norms;
+  p.embed = static_cast<const __nv_bfloat16 *>(h->embed);
+  p.final_norm = static_cast<const __nv_bfloat16 *>(h->final_norm);
+  p.kc = static_cast<__nv_bfloat16 *>(kv.k); p.vc = static_cast<__nv_bfloat16 *>(kv.v);
+  p.tokens = tokens; p.positions = positions; p.logits = logits ? logits : h->logits; p.argmax = argmax;
+  p.h = h->h; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
+  p.attn_o = h->attn_o; p.attn_ml = h->attn_ml; p.attn_o1 = h->attn_o1; p.attn_ml1 = h->attn_ml1;
+  p.attn_cnt = h->attn_cnt; p.router_part = h->router_part; p.routing = h->routing;
+  p.gu_shared = h->gu_shared; p.gu_routed = h->gu_routed; p.am_part = h->am_part; p.rope = h->rope;
+  p.counters = h->counters; p.route_flag = h->route_flag; p.epoch = h->epoch; p.error = h->error;
+  p.stats = h->stats_dev;
+  p.dbg_hidden = h->dbg_hidden; p.dbg_ids = h->dbg_ids; p.dbg_w = h->dbg_w;
+  p.timeout_ns = h->timeout_ns;
+  p.inject_op = -1;
+  return MK_OK;
+}
+
+static int launch_variant(mk_handle *h, Params &p, const Plan &pl, cudaStream_t stream, int variant) {
+  if (variant == MK_MEGAKERNEL) {
+    int e = launch_step(p, pl.mmax, true, stream);
+    if (e) return fail(MK_ERR_LAUNCH, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
+    h->stats.kernel_launches += 1;
+    return MK_OK;
+  }
+  for (int op = 0; op < pl.n_ops; ++op) {
+    p.op_begin = op;
+    p.op_end = op + 1;
+    int e = launch_step(p, pl.mmax, false, stream);
+    if (e) return fail(MK_ERR_LAUNCH, "launch of op %d failed: %s", op, cudaGetErrorString((cudaError_t)e));
+  }
+  p.op_begin = 0;
+  p.op_end = pl.n_ops;
+  h->stats.kernel_launches += pl.n_ops;
+  return MK_OK;
+}
+
+static int run_step(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T,
+                    mk_kv_cache kv, float *logits, int32_t *argmax, cudaStream_t stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  Params p;
+  Plan pl;
+  int rc = fill_params(h, tokens, positions, B, T, kv, logits, argmax, p, pl);
+  if (rc) return rc;
+  if (h->inject == MK_FAULT_UNREACHABLE_WAIT) p.inject_op = op_index(0, OP_ATTN);
+  int variant = h->variant;
+  if (variant == MK_MULTIKERNEL_GRAPH && p.inject_op < 0) {
+    uint64_t key[12] = {(uint64_t)B,
+                        (uint64_t)T,
+                        (uint64_t)(uintptr_t)tokens,
+                        (uint64_t)(uintptr_t)positions,
+                        (uint64_t)(uintptr_t)p.logits,
+                        (uint64_t)(uintptr_t)argmax,
+                        (uint64_t)(uintptr_t)kv.k,
+                        (uint64_t)(uintptr_t)kv.v,
+                        (uint64_t)(uintptr_t)h->dbg_hidden,
+                        (uint64_t)(uintptr_t)h->dbg_ids ^ (uint64_t)(uintptr_t)h->dbg_w,
+                        h->timeout_ns,
+                        0};
+    cudaGraphExec_t exec = nullptr;
+    for (auto &g : h->graphs)
+      if (std::memcmp(g.key, key, sizeof key) == 0) exec = g.exec;
+    if (!exec) {
+      CUDA_TRY(cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal));
+      int lrc = launch_variant(h, p, pl, h->capture_stream, MK_MULTIKERNEL);
+      cudaGraph_t graph = nullptr;
+      cudaError_t ce = cudaStreamEndCapture(h->capture_stream, &graph);
+      if (lrc) {
+        if (graph) cudaGraphDestroy(graph);
+        return lrc;
+      }
+      if (ce != cudaSuccess) return fail(MK_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(ce));
+      ce = cudaGraphInstantiate(&exec, graph, 0);
+      cudaGraphDestroy(graph);
+      if (ce != cudaSuccess) return fail(MK_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(ce));
+      if (h->graphs.size() >= 8) {
+        cudaGraphExecDestroy(h->graphs.front().exec);
+        h->graphs.erase(h->graphs.begin());
+      }
+      GraphEntry ge;
+      std::memcpy(ge.key, key, sizeof key);
+      ge.exec = exec;
+      h->graphs.push_back(ge);
+      h->stats.kernel_launches -= pl.n_ops;  // counted again below on replay
+    }
+    CUDA_TRY(cudaGraphLaunch(exec, stream));
+    h->stats.kernel_launches += pl.n_ops;
+  } else {
+    if (variant == MK_MULTIKERNEL_GRAPH) variant = MK_MULTIKERNEL;
+    rc = launch_variant(h, p, pl, stream, variant);
+    if (rc) return rc;
+  }
+  h->inject = MK_FAULT_NONE;
+  h->stats.steps += 1;
+  return MK_OK;
+}
+
+MK_API int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
+                          int32_t T, mk_kv_cache kv, float *out_logits, int32_t *out_argmax,
+                          void *stream) {
+  return run_step(h, tokens, positions, B, T, kv, out_logits, out_argmax, static_cast<cudaStream_t>(stream));
+}
+
+MK_API int mk_get_device_status(mk_handle *h, void *stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUDA_TRY(cudaStreamSynchronize(s));
+  int err[2] = {0, 0};
+  CUDA_TRY(cudaMemcpy(err, h->error, sizeof err, cudaMemcpyDeviceToHost));
+  if (err[0] == 0) {
+    h->last_error_op = -1;
+    return MK_OK;
+  }
+  h->last_error_op = err[1];
+  int rc = reset_sync_state(h, s);
+  if (rc) return rc;
+  if (err[0] == MK_ERR_TIMEOUT) return fail(MK_ERR_TIMEOUT, "device wait timed out in op %d", err[1]);
+  if (err[0] == MK_ERR_DEVICE_CHECK)
+    return fail(MK_ERR_DEVICE_CHECK, "device rejected an input (token id or position) in op %d", err[1]);
+  return fail(err[0], "device error %d in op %d", err[0], err[1]);
+}
+
+MK_API int mk_last_device_error_op(mk_handle *h) { return h ? h->last_error_op : -1; }
+
+MK_API int mk_decode_step_host(mk_handle *h, const int32_t *tokens_host, const int32_t *positions_host,
+                               int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
+                               int32_t *out_argmax_host, void *stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (!tokens_host || !positions_host || !out_argmax_host)
+    return fail(MK_ERR_ARG, "tokens_host, positions_host and out_argmax_host are required");
+  if (B < 1 || T < 1 || B > h->desc.max_seqs || (long long)B * T > h->desc.max_rows)
+    return fail(MK_ERR_CAPACITY, "B=%d T=%d exceeds the handle", B, T);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUDA_TRY(cudaMemcpyAsync(h->io_tokens, tokens_host, sizeof(int32_t) * B * T, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaMemcpyAsync(h->io_positions, positions_host, sizeof(int32_t) * B, cudaMemcpyHostToDevice, s));
+  int rc = run_step(h, h->io_tokens, h->io_positions, B, T, kv, out_logits, h->io_argmax, s);
+  if (rc) return rc;
+  CUDA_TRY(cudaMemcpyAsync(out_argmax_host, h->io_argmax, sizeof(int32_t) * B * T, cudaMemcpyDeviceToHost, s));
+  return mk_get_device_status(h, stream);
+}
+
+MK_API int mk_set_variant(mk_handle *h, int32_t variant) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (variant < MK_MEGAKERNEL || variant > MK_MULTIKERNEL_GRAPH) return fail(MK_ERR_ARG, "unknown variant %d", variant);
+  h->variant = variant;
+  return MK_OK;
+}
+
+MK_API int mk_set_timeout(mk_handle *h, uint64_t timeout_ns) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (timeout_ns == 0) return fail(MK_ERR_ARG, "timeout must be > 0");
+  h->timeout_ns = timeout_ns;
+  return MK_OK;
+}
+
+MK_API int mk_set_debug(mk_handle *h, float *hidden, int32_t *expert_ids, float *expert_w) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  h->dbg_hidden = hidden;
+  h->dbg_ids = expert_ids;
+  h->dbg_w = expert_w;
+  return MK_OK;
+}
+
+MK_API int mk_debug_inject(mk_handle *h, int32_t fault) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (fault != MK_FAULT_NONE && fault != MK_FAULT_UNREACHABLE_WAIT) return fail(MK_ERR_ARG, "unknown fault %d", fault);
+  h->inject = fault;
+  return MK_OK;
+}
+
+MK_API int mk_get_stats(mk_handle *h, mk_stats *out, int32_t reset) {
+  if (!h || !out) return fail(MK_ERR_ARG, "handle and out are required");
+  unsigned long long dev[4] = {0, 0, 0, 0};
+  CUDA_TRY(cudaDeviceSynchronize());
+  CUDA_TRY(cudaMemcpy(dev, h->stats_dev, sizeof dev, cudaMemcpyDeviceToHost));
+  *out = h->stats;
+  out->expert_union_total = dev[0];
+  if (reset) {
+    h->stats = mk_stats{};
+    CUDA_TRY(cudaMemset(h->stats_dev, 0, sizeof dev));
+  }
+  return MK_OK;
+}
+
+}  // extern "C"

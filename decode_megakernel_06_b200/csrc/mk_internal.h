@@ -1,0 +1,132 @@
+// mk_internal.h -- structures shared by the host planner (mk_api.cu) and the
+// persistent decode-step kernel (mk_kernel.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mk {
+
+// ---- geometry ------------------------------------------------------------------
+constexpr int kWarpsPerCta = 8;                     // each warp: producer + consumer
+constexpr int kThreads = kWarpsPerCta * 32;
+constexpr int kSlots = 3;                           // ring slots per warp
+constexpr int kSlotBytes = 8192;                    // one tile: two 4 KB TMA boxes
+constexpr int kPanel = 256;                         // columns per weight box
+constexpr int kBoxRows = 8;                         // rows per weight box
+constexpr int kBoxBytes = kPanel * kBoxRows * 2;    // 4096
+constexpr int kMaxRows = 8;                         // M = B*T cap of this build
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 16;
+constexpr int kL1Fan = 16;                          // attention merge fan-in per level
+constexpr int kMaxChunks = kL1Fan * kL1Fan;         // KV chunks per (seq, kv head, q group)
+constexpr int kCounterStride = 32;                  // uint32s between counters (128 B)
+constexpr int kRouterKChunk = 2 * kPanel;           // router split-K width (512 columns)
+
+// Ops of one step: EMBED, then per layer QKV ATTN OPROJ ROUTER SHARED_GU
+// ROUTED_GU DOWN, then LMHEAD.
+enum OpType : int {
+  OP_EMBED = 0, OP_QKV = 1, OP_ATTN = 2, OP_OPROJ = 3, OP_ROUTER = 4,
+  OP_SHARED_GU = 5, OP_ROUTED_GU = 6, OP_DOWN = 7, OP_LMHEAD = 8
+};
+constexpr int kOpsPerLayer = 7;
+
+__host__ __device__ inline int n_ops_for(int L) { return kOpsPerLayer * L + 2; }
+__host__ __device__ inline int op_type_of(int op, int L) {
+  if (op == 0) return OP_EMBED;
+  if (op == kOpsPerLayer * L + 1) return OP_LMHEAD;
+  return 1 + (op - 1) % kOpsPerLayer;
+}
+__host__ __device__ inline int op_layer_of(int op, int L) {
+  if (op == 0 || op == kOpsPerLayer * L + 1) return -1;
+  return (op - 1) / kOpsPerLayer;
+}
+__host__ __device__ inline int op_index(int layer, int type) {
+  return 1 + kOpsPerLayer * layer + (type - 1);
+}
+// Ops whose completion `op` waits for (-1 = none).
+__host__ __device__ inline void op_deps(int op, int L, int *d0, int *d1) {
+  int t = op_type_of(op, L), l = op_layer_of(op, L);
+  *d0 = -1;
+  *d1 = -1;
+  switch (t) {
+    case OP_EMBED: break;
+    case OP_QKV: *d0 = (l == 0) ? 0 : op_index(l - 1, OP_DOWN); break;
+    case OP_ATTN: *d0 = op_index(l, OP_QKV); break;
+    case OP_OPROJ: *d0 = op_index(l, OP_ATTN); break;
+    case OP_ROUTER:
+    case OP_SHARED_GU:
+    case OP_ROUTED_GU: *d0 = op_index(l, OP_OPROJ); break;  // ROUTED_GU: + routing
+    case OP_DOWN: *d0 = op_index(l, OP_SHARED_GU); *d1 = op_index(l, OP_ROUTED_GU); break;
+    case OP_LMHEAD: *d0 = op_index(L - 1, OP_DOWN); break;
+  }
+}
+
+// Tensor maps per layer, in this order; the lm_head map follows the last layer.
+enum MapSlot : int {
+  MAP_WQKV = 0, MAP_WO, MAP_ROUTER, MAP_WGATE, MAP_WUP, MAP_WDOWN,
+  MAP_WSGATE, MAP_WSUP, MAP_WSDOWN, MAPS_PER_LAYER
+};
+
+// Routing of one layer, written by the last warp to finish the router op.
+struct Routing {
+  int n_union;                           // distinct experts over the M rows
+  int expert[kMaxExperts];               // ascending expert ids, [n_union]
+  uint32_t rowmask[kMaxExperts];         // rows routed to expert[j]
+  float weight[kMaxExperts][kMaxRows];   // renormalised weight of row m (0 if absent)
+};
+
+struct ArgmaxPart {
+  float value;
+  int index;
+};
+
+struct alignas(64) Params {
+  CUtensorMap kmap;   // K cache as 2-D [L*Bmax*Hkv*cap][hd], box [hd][ppt]
+  CUtensorMap vmap;
+  // dims
+  int L, d, Hq, Hkv, hd, E, topk, F, Fs, V, Bmax, cap;
+  float eps;
+  int B, T, M, max_rows;
+  // grid / schedule
+  int n_cta, n_warps, op_begin, op_end, n_ops;
+  int rows_per_tile;   // 16 (tall tiles) or 8 (wide tiles)
+  int n_hb;            // residual row blocks (ceil(d / rows_per_tile))
+  int attn_chunk, attn_qsplit, attn_qvp, attn_ppt, attn_nch_max;
+  // weights
+  const CUtensorMap *tmaps;              // [L][MAPS_PER_LAYER] + lm_head
+  const __nv_bfloat16 *const *norms;     // [L][2]: attn_norm, ffn_norm
+  const __nv_bfloat16 *embed, *final_norm;
+  __nv_bfloat16 *kc, *vc;                // caches (append target)
+  // step io
+  const int *tokens, *positions;
+  float *logits;
+  int *argmax;
+  // scratch
+  float *h, *ss, *qkv, *o;
+  float *attn_o, *attn_ml, *attn_o1, *attn_ml1;
+  uint32_t *attn_cnt;
+  float *router_part;
+  Routing *routing;                      // [L]
+  float *gu_shared, *gu_routed;
+  ArgmaxPart *am_part;
+  const float2 *rope;                    // [cap][hd/2] (cos, sin) of p * theta^(-2i/hd)
+  uint32_t *counters, *route_flag, *epoch;
+  int *error;                            // [0] code, [1] op
+  unsigned long long *stats;             // [0] expert union total
+  // debug
+  float *dbg_hidden;
+  int *dbg_ids;
+  float *dbg_w;
+  unsigned long long timeout_ns;
+  int inject_op;                         // op whose dependency is made unreachable, -1 none
+};
+
+// Launch entry points implemented in mk_kernel.cu.
+int launch_step(const Params &p, int mmax, bool cooperative, cudaStream_t stream);
+size_t step_smem_bytes(int n_ops);
+int max_cta_per_sm(int mmax, size_t smem);
+
+}  // namespace mk

@@ -1,0 +1,231 @@
+/*
+ * mk.h -- C ABI of the fused MoE decode-step library (libmk.so).
+ *
+ * The library runs one decode step of a layered MoE transformer on one B200
+ * as a single persistent kernel: one CTA per SM walks a fixed op schedule,
+ * synchronises through global-memory counters instead of kernel boundaries,
+ * and streams every weight tile through a TMA ring in shared memory that is
+ * filled ahead of the op that consumes it, across op and layer boundaries.
+ * This is the method of the TPU megakernel pages: the whole decode step as
+ * one program, with each weight load decoupled from its consumer so that the
+ * next layer's weights are in flight while the current layer computes
+ * (video "700 tok/s on a 2.8 Trillion Model: The 92-Layer TPU Megakernel",
+ * key technical takeaways; Chinese report "TPU 巨核", section 差距从哪里来;
+ * German report, section "Der Trick").  A one-launch-per-op variant of the
+ * same path (optionally replayed from a CUDA graph) is built in for
+ * comparison: the pages attribute the gap to the idle time between the many
+ * kernels of a stock engine (same sections).
+ *
+ * The step computed, per row m of sequence b at position p (the decoder the
+ * pages fuse: attention, MoE, normalisation and residual -- tpu-megakernels
+ * README, FAQ entry on why a custom megakernel is built):
+ *   h = embed[token]; per layer: x = rms(h) g_attn; q,k,v = Wqkv x; rotary
+ *   embedding (rotate-half, theta) on q and k at p; bf16 k,v appended to the
+ *   cache at p; GQA softmax attention over positions 0..p (causal inside a
+ *   verify block); h += Wo o; y = rms(h) g_ffn; softmax router, top-k
+ *   renormalised; h += sum_k w_e Wd_e(silu(Wg_e y) * Wu_e y) + shared(y);
+ *   finally logits = Wlm (rms(h) g_final) and argmax (lowest index on ties).
+ * Arithmetic is fp32 on bf16 weights and a bf16 KV cache.
+ *
+ * Conventions.  All tensors are row-major.  Weight matrices are [out][in]
+ * bf16 (y = W x).  Expert tensors put the expert index first.  Pointers marked
+ * "device" are CUDA device pointers in the current device's context; the
+ * caller owns every buffer it passes and keeps weights alive until
+ * mk_destroy.  Functions return MK_OK (0) or a negative MK_ERR_* code and
+ * never abort; mk_last_error() returns a thread-local message for the last
+ * failure.  Work is asynchronous on the given stream unless stated otherwise.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MK_API __attribute__((visibility("default")))
+
+/* ---- status codes ---------------------------------------------------------- */
+#define MK_OK 0
+#define MK_ERR_ARG (-1)          /* invalid argument or descriptor              */
+#define MK_ERR_CAPACITY (-2)     /* B, T, B*T or positions exceed the handle    */
+#define MK_ERR_CUDA (-3)         /* a CUDA runtime/driver call failed           */
+#define MK_ERR_LAUNCH (-4)       /* cooperative launch refused / not co-resident */
+#define MK_ERR_TIMEOUT (-5)      /* a bounded device-side wait ran out           */
+#define MK_ERR_DEVICE_CHECK (-6) /* the kernel rejected an input (token id,      */
+                                 /* position) before touching memory with it    */
+#define MK_ERR_UNSUPPORTED (-7)  /* shape outside what this build supports       */
+
+/* ---- execution variants ---------------------------------------------------- */
+#define MK_MEGAKERNEL 0         /* one persistent cooperative launch per step    */
+#define MK_MULTIKERNEL 1        /* one launch per op, no cross-op prefetch       */
+#define MK_MULTIKERNEL_GRAPH 2  /* the per-op launches replayed from a CUDA graph */
+
+/* ---- debug fault injection ---------------------------------------------------- */
+#define MK_FAULT_NONE 0
+#define MK_FAULT_UNREACHABLE_WAIT 1 /* next step: one dependency waits for a count
+                                       that is never reached (bounded wait test) */
+
+/* Model description.  Supported: head_dim in {32, 64, 128, 256};
+ * n_q_heads % n_kv_heads == 0; d_model, n_q_heads*head_dim multiples of 8;
+ * expert_ffn and shared_ffn multiples of 16 (shared_ffn may be 0 = no shared
+ * expert); n_experts <= 256; top_k <= min(16, n_experts);
+ * 1 <= max_rows <= 8; 1 <= max_seqs <= max_rows. */
+typedef struct mk_model_desc {
+  int32_t n_layers, d_model, n_q_heads, n_kv_heads, head_dim;
+  int32_t n_experts, top_k, expert_ffn, shared_ffn, vocab;
+  float rope_theta; /* rotary base, e.g. 1e4                         */
+  float rms_eps;    /* RMSNorm epsilon inside the square root, 1e-6  */
+  int32_t max_rows;     /* cap on rows per step M = B*T              */
+  int32_t max_seqs;     /* cap on sequences B (KV cache batch extent) */
+  int32_t kv_capacity;  /* cache slots per sequence                   */
+  int32_t variant;      /* MK_MEGAKERNEL | MK_MULTIKERNEL | MK_MULTIKERNEL_GRAPH */
+} mk_model_desc;
+
+/* One layer's weights: device pointers to bf16, caller-owned.
+ *   attn_norm, ffn_norm : [d]
+ *   wqkv  : [(Hq + 2 Hkv) hd][d]   rows: Wq (Hq heads), then Wk, then Wv
+ *   wo    : [d][Hq hd]
+ *   router: [E][d]
+ *   w_gate, w_up: [E][F][d];  w_down: [E][d][F]
+ *   ws_gate, ws_up: [Fs][d];  ws_down: [d][Fs]   (NULL when Fs == 0)
+ * Each matrix must start on a 16-byte boundary. */
+typedef struct mk_layer_weights {
+  const void *attn_norm, *wqkv, *wo, *ffn_norm, *router;
+  const void *w_gate, *w_up, *w_down;
+  const void *ws_gate, *ws_up, *ws_down;
+} mk_layer_weights;
+
+/* embed, lm_head: [V][d]; final_norm: [d]; layers: HOST array of n_layers
+ * entries (copied during mk_create). */
+typedef struct mk_weights {
+  const void *embed, *final_norm, *lm_head;
+  const mk_layer_weights *layers;
+} mk_weights;
+
+/* KV cache, device bf16, each [n_layers][max_seqs][Hkv][kv_capacity][hd].
+ * Keys are stored after the rotary embedding.  Caller-owned; written in place
+ * at positions[b] .. positions[b] + T - 1 of every layer. */
+typedef struct mk_kv_cache {
+  void *k, *v;
+} mk_kv_cache;
+
+typedef struct mk_handle mk_handle;
+
+/* Counters kept by a handle (read with mk_get_stats). */
+typedef struct mk_stats {
+  uint64_t steps;              /* decode steps launched                    */
+  uint64_t expert_union_total; /* sum over steps and layers of the number of
+                                  distinct routed experts (device-counted)  */
+  uint64_t kernel_launches;    /* kernels launched by the library           */
+} mk_stats;
+
+/* Schedule summary for a shape (host-only planning; see mk_plan_describe). */
+typedef struct mk_plan_info {
+  int32_t n_ops;           /* ops in one step's schedule                     */
+  int32_t n_cta;           /* CTAs of the persistent grid (= SM count)       */
+  int32_t warps_per_cta;   /* consumer/producer warps per CTA                */
+  int32_t rows_per_tile;   /* weight rows per ring tile (16, or 8 at M > 4)  */
+  int32_t mmax;            /* row capacity of the kernel instance (1,2,4,8)  */
+  int32_t attn_chunk;      /* KV positions per attention work item          */
+  int32_t attn_qsplit;     /* query-vector groups per (sequence, KV head)    */
+  int32_t smem_bytes;      /* dynamic shared memory per CTA                  */
+  int64_t scratch_bytes;   /* device scratch owned by a handle of this shape */
+} mk_plan_info;
+
+#define MK_OP_EMBED 0
+#define MK_OP_QKV 1
+#define MK_OP_ATTN 2
+#define MK_OP_OPROJ 3
+#define MK_OP_ROUTER 4
+#define MK_OP_SHARED_GU 5
+#define MK_OP_ROUTED_GU 6
+#define MK_OP_DOWN 7
+#define MK_OP_LMHEAD 8
+
+/* Create a handle: validates the descriptor, plans the schedule, encodes the
+ * weight tensor maps, allocates scratch on the current device.  No kernel
+ * runs.  `out` receives the handle (NULL on failure). */
+MK_API int mk_create(const mk_model_desc *desc, const mk_weights *weights, mk_handle **out);
+
+/* One decode step of M = B*T rows (row m = b*T + t).
+ *   tokens     : device int32 [B*T], ids in [0, vocab)
+ *   positions  : device int32 [B], cache index of sequence b's first new token;
+ *                0 <= positions[b] and positions[b] + T <= kv_capacity
+ *   B, T       : 1 <= B <= max_seqs, T >= 1, B*T <= max_rows.  T > 1 scores a
+ *                verify block: row t attends positions 0 .. positions[b] + t.
+ *   kv         : the cache (see mk_kv_cache); appended in place
+ *   out_logits : device fp32 [B*T][vocab], or NULL (kept in handle scratch)
+ *   out_argmax : device int32 [B*T] (may alias tokens: read before written)
+ *   stream     : cudaStream_t (NULL = legacy default stream)
+ * Asynchronous.  Invalid token ids or positions are detected on the device:
+ * the step stops and mk_get_device_status reports MK_ERR_DEVICE_CHECK. */
+MK_API int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                          int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
+                          int32_t *out_argmax, void *stream);
+
+/* The same step driven from HOST buffers: copies tokens [B*T] and positions
+ * [B] to the device, runs the step, copies argmax [B*T] back to
+ * out_argmax_host, and waits for the stream.  Logits stay on the device
+ * (out_logits may be NULL).  Returns the device status of the step. */
+MK_API int mk_decode_step_host(mk_handle *h, const int32_t *tokens_host,
+                               const int32_t *positions_host, int32_t B, int32_t T,
+                               mk_kv_cache kv, float *out_logits, int32_t *out_argmax_host,
+                               void *stream);
+
+/* Synchronises `stream`, then returns MK_OK or the first device-side error of
+ * the steps since the last call (MK_ERR_TIMEOUT, MK_ERR_DEVICE_CHECK).  An
+ * error clears the handle's synchronisation state so the next step starts
+ * clean; the failed step's outputs and cache writes are undefined. */
+MK_API int mk_get_device_status(mk_handle *h, void *stream);
+
+/* Device-side detail of the last error returned by mk_get_device_status:
+ * the op index that failed (or -1). */
+MK_API int mk_last_device_error_op(mk_handle *h);
+
+/* Thread-local message for the last failing call (never NULL). */
+MK_API const char *mk_last_error(void);
+
+/* Frees everything the handle owns.  Safe on NULL.  Call after the last step
+ * has finished. */
+MK_API void mk_destroy(mk_handle *h);
+
+/* Switch the execution variant (MK_MEGAKERNEL, MK_MULTIKERNEL,
+ * MK_MULTIKERNEL_GRAPH).  The math is identical across variants. */
+MK_API int mk_set_variant(mk_handle *h, int32_t variant);
+
+/* Bound for every device-side wait, in nanoseconds (default 1e9). */
+MK_API int mk_set_timeout(mk_handle *h, uint64_t timeout_ns);
+
+/* Test/debug outputs, written by every following step (NULL disables):
+ *   hidden     : device fp32 [n_layers + 1][max_rows][d]: the residual stream
+ *                after the embedding and after each layer
+ *   expert_ids : device int32 [n_layers][max_rows][top_k], selection order
+ *   expert_w   : device fp32  [n_layers][max_rows][top_k], renormalised */
+MK_API int mk_set_debug(mk_handle *h, float *hidden, int32_t *expert_ids, float *expert_w);
+
+/* Arm a fault for the next step (MK_FAULT_*). */
+MK_API int mk_debug_inject(mk_handle *h, int32_t fault);
+
+/* Copies the handle's counters; reset != 0 zeroes them afterwards.  Waits for
+ * the device (reads a device counter). */
+MK_API int mk_get_stats(mk_handle *h, mk_stats *out, int32_t reset);
+
+/* Host-only: validate a descriptor without touching the GPU. */
+MK_API int mk_validate_desc(const mk_model_desc *desc);
+
+/* Host-only: plan the step for a shape on a GPU with n_sm SMs and report the
+ * schedule.  If op_types/op_layers/op_dep0/op_dep1 are non-NULL they receive
+ * up to `cap` entries: each op's MK_OP_* type, layer (-1 = none) and the
+ * indices of the ops whose completion it waits for (-1 = none; ROUTED_GU also
+ * waits for its layer's routing, published by the ROUTER op). */
+MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, int32_t T,
+                            mk_plan_info *info, int32_t *op_types, int32_t *op_layers,
+                            int32_t *op_dep0, int32_t *op_dep1, int32_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MK_H */
