@@ -176,7 +176,7 @@ def build_workload(kind, B, device):
     if kind == "small":
         wl = workload("small") if B == 1 else workload("small_batch", B)
     else:
-        wl = workload(kind, B) if kind == "large" else workload(kind)
+        wl = workload(kind, B) if kind in ("large", "profile") else workload(kind)
     m = wl.model
     t0 = time.perf_counter()
     w = make_weights(m, wl.seed, device)
@@ -288,6 +288,37 @@ def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1):
             "tokens": n_steps * B * T}
 
 
+def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr):
+    """One traced step: per op, when the first / last warp started it and when
+    the last warp finished it (microseconds from the step's first op start)."""
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+
+    n_sm = torch.cuda.get_device_properties(device).multi_processor_count
+    rc, info, ops = mk.mk_plan_describe(dec.desc, n_sm, B, T)
+    nw = info.n_cta * info.warps_per_cta
+    buf = torch.zeros((info.n_ops, nw, 2), dtype=torch.int64, device=device)
+    pos = torch.tensor([c for c in ctx], dtype=torch.int32, device=device)
+    tok = torch.zeros(B * T, dtype=torch.int32, device=device)
+    am = torch.empty(B * T, dtype=torch.int32, device=device)
+    dec.set_trace(buf)
+    assert dec.step(tok, pos, B, T, k, v, None, am) == 0
+    assert dec.status() == 0
+    dec.set_trace(None)
+    t = buf.cpu().numpy().astype("float64")
+    t0 = t[:, :, 0][t[:, :, 0] > 0].min()
+    rows = []
+    for i, (typ, layer, d0, d1) in enumerate(ops):
+        s, e = t[i, :, 0] - t0, t[i, :, 1] - t0
+        rows.append((i, mk.OP_NAMES[typ], layer, s.min() / 1e3, s.max() / 1e3, e.max() / 1e3))
+    print(f"{'op':>4} {'name':>10} {'layer':>5} {'first_start':>12} {'last_start':>11} "
+          f"{'last_end':>9} (us)", file=out)
+    for r in rows:
+        print(f"{r[0]:>4} {r[1]:>10} {r[2]:>5} {r[3]:>12.1f} {r[4]:>11.1f} {r[5]:>9.1f}", file=out)
+    return rows
+
+
 def run_mine(args):
     import torch
 
@@ -310,6 +341,11 @@ def run_mine(args):
     ctx = make_context_lengths(wl)
     dec = mk.Decoder(m, w, max_rows=bmax * T, max_seqs=bmax, kv_capacity=cap,
                      variant=args.variant)
+
+    if args.trace:
+        # warm, then one traced step (not part of the timed region)
+        time_steps(dec, m, k, v, B, T, ctx, 1, 3, device)
+        trace_step(dec, m, k, v, B, T, ctx, device)
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -446,12 +482,14 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
-    ap.add_argument("--workload", default="large", choices=["large", "small", "tiny"])
+    ap.add_argument("--workload", default="large", choices=["large", "small", "tiny", "profile"])
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--variant", default="megakernel",
                     choices=["megakernel", "multikernel", "multikernel_graph"])
     ap.add_argument("--sweep", action=argparse.BooleanOptionalAction, default=True)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--trace", action="store_true",
+                    help="print a per-op timeline of one extra step to stderr")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -35,7 +35,8 @@ VARIANTS = {"megakernel": MK_MEGAKERNEL, "multikernel": MK_MULTIKERNEL,
 MK_FAULT_NONE = 0
 MK_FAULT_UNREACHABLE_WAIT = 1
 
-OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "LMHEAD"]
+OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE",
+            "LMHEAD"]
 
 
 class mk_model_desc(ctypes.Structure):
@@ -104,6 +105,7 @@ def lib():
         "mk_set_timeout": (i32, [vp, u64]),
         "mk_set_debug": (i32, [vp, vp, vp, vp]),
         "mk_debug_inject": (i32, [vp, i32]),
+        "mk_set_trace": (i32, [vp, vp]),
         "mk_get_stats": (i32, [vp, ctypes.POINTER(mk_stats), i32]),
         "mk_validate_desc": (i32, [ctypes.POINTER(mk_model_desc)]),
         "mk_plan_describe": (i32, [ctypes.POINTER(mk_model_desc), i32, i32, i32,
@@ -136,7 +138,7 @@ def mk_validate_desc(desc: mk_model_desc) -> int:
 def mk_plan_describe(desc: mk_model_desc, n_sm: int, B: int, T: int):
     """Returns (rc, mk_plan_info, [(type, layer, dep0, dep1)] per op)."""
     info = mk_plan_info()
-    n = 7 * desc.n_layers + 2
+    n = 8 * desc.n_layers + 2
     arrs = [(ctypes.c_int32 * n)() for _ in range(4)]
     rc = lib().mk_plan_describe(ctypes.byref(desc), n_sm, B, T, ctypes.byref(info),
                                 *[ctypes.cast(a, _I32P) for a in arrs], n)
@@ -183,6 +185,10 @@ def mk_set_timeout(h, ns: int) -> int:
 
 def mk_set_debug(h, hidden: int, expert_ids: int, expert_w: int) -> int:
     return lib().mk_set_debug(h, hidden, expert_ids, expert_w)
+
+
+def mk_set_trace(h, trace: int) -> int:
+    return lib().mk_set_trace(h, trace)
 
 
 def mk_debug_inject(h, fault: int) -> int:
@@ -252,6 +258,9 @@ class Decoder:
 
     def set_debug(self, hidden=None, expert_ids=None, expert_w=None):
         _check(mk_set_debug(self.h, _ptr(hidden), _ptr(expert_ids), _ptr(expert_w)))
+
+    def set_trace(self, trace=None):
+        _check(mk_set_trace(self.h, _ptr(trace)))
 
     def inject(self, fault: int):
         _check(mk_debug_inject(self.h, fault))

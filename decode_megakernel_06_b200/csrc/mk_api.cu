@@ -80,7 +80,7 @@ int encode_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, 
 struct Plan {
   int M, mmax, rows_per_tile, n_hb;
   int attn_qvp, attn_qsplit, attn_ppt, attn_chunk, attn_nch_max;
-  int n_ops, n_cta, n_warps;
+  int n_ops, n_cta, n_warps, xs_floats;
   size_t smem;
 };
 
@@ -88,8 +88,8 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   Plan p{};
   p.M = B * T;
   p.mmax = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
-  p.rows_per_tile = p.mmax <= 4 ? 16 : 8;
-  p.n_hb = ceil_div(d.d_model, p.rows_per_tile);
+  p.rows_per_tile = kRows;
+  p.n_hb = ceil_div(d.d_model, kRows);
   const int G = d.n_q_heads / d.n_kv_heads;
   p.attn_qvp = (G * T <= 4) ? 4 : 8;
   p.attn_qsplit = ceil_div(G * T, p.attn_qvp);
@@ -106,7 +106,8 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.attn_chunk = c;
   p.attn_nch_max = ceil_div(d.kv_capacity, c);
   p.n_ops = n_ops_for(d.n_layers);
-  p.smem = step_smem_bytes(p.n_ops);
+  p.xs_floats = kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), 4) * 4 : 0;
+  p.smem = step_smem_bytes(p.n_ops, p.xs_floats);
   return p;
 }
 
@@ -145,8 +146,8 @@ struct mk_handle {
   std::vector<void *> allocs;
   CUtensorMap *tmaps;
   const __nv_bfloat16 **norms;
-  float *h, *ss, *qkv, *o, *attn_o, *attn_ml, *attn_o1, *attn_ml1, *router_part, *gu_shared,
-      *gu_routed, *logits;
+  float *h, *ss, *qkv, *o, *attn_o, *attn_ml, *attn_o1, *attn_ml1, *router_part, *act_shared,
+      *act_routed, *y_part, *logits;
   uint32_t *attn_cnt, *counters, *route_flag, *epoch;
   Routing *routing;
   ArgmaxPart *am_part;
@@ -164,6 +165,7 @@ struct mk_handle {
   float *dbg_hidden;
   int32_t *dbg_ids;
   float *dbg_w;
+  unsigned long long *trace;
   int inject;
   int last_error_op;
   mk_stats stats;
@@ -190,6 +192,8 @@ MK_API int mk_validate_desc(const mk_model_desc *d) {
   if (d->expert_ffn < 16 || d->expert_ffn % 16) return fail(MK_ERR_ARG, "expert_ffn must be a positive multiple of 16");
   if (d->shared_ffn < 0 || d->shared_ffn % 16) return fail(MK_ERR_ARG, "shared_ffn must be 0 or a multiple of 16");
   if (d->vocab < 1) return fail(MK_ERR_ARG, "vocab must be >= 1");
+  if (d->d_model > 6144 || d->n_q_heads * d->head_dim > 6144)
+    return fail(MK_ERR_UNSUPPORTED, "d_model and n_q_heads*head_dim must be <= 6144");
   if (d->max_rows < 1 || d->max_rows > kMaxRows)
     return fail(MK_ERR_UNSUPPORTED, "max_rows must be in [1, %d]", kMaxRows);
   if (d->max_seqs < 1 || d->max_seqs > d->max_rows) return fail(MK_ERR_ARG, "max_seqs must be in [1, max_rows]");
@@ -223,12 +227,13 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
     info->smem_bytes = (int32_t)p.smem;
     Sizes s = scratch_sizes(*desc, n_sm);
     const mk_model_desc &d = *desc;
-    size_t f = (size_t)d.max_rows * d.d_model * 2 + (size_t)d.max_rows * ceil_div(d.d_model, 8) +
+    size_t f = (size_t)d.max_rows * d.d_model * 2 + (size_t)d.max_rows * ceil_div(d.d_model, kRows) +
+               (size_t)kMaxRows * (d.top_k + 1) * d.d_model +
                (size_t)d.max_rows * (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim +
                (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml + s.attn_o1 +
                s.attn_ml1 + (size_t)ceil_div(d.d_model, kPanel) * kMaxRows * d.n_experts +
-               (size_t)kMaxRows * 2 * d.shared_ffn +
-               (size_t)std::min(d.n_experts, d.max_rows * d.top_k) * kMaxRows * 2 * d.expert_ffn +
+               (size_t)kMaxRows * d.shared_ffn +
+               (size_t)std::min(d.n_experts, d.max_rows * d.top_k) * kMaxRows * d.expert_ffn +
                (size_t)d.max_rows * d.vocab + (size_t)d.kv_capacity * d.head_dim;
     info->scratch_bytes = (int64_t)(f * 4 + s.attn_cnt * 4 + (size_t)d.n_layers * sizeof(Routing) +
                                     (size_t)p.n_warps * kMaxRows * sizeof(ArgmaxPart));
@@ -297,8 +302,8 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
   CUDA_TRY(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
   if (!coop) return fail(MK_ERR_LAUNCH, "device does not support cooperative launches");
-  const size_t smem = step_smem_bytes(n_ops_for(d.n_layers));
   for (int mm : {1, 2, 4, 8}) {
+    const size_t smem = make_plan(d, n_sm, 1, mm).smem;
     int per = max_cta_per_sm(mm, smem);
     if (per < 1) return fail(MK_ERR_LAUNCH, "kernel (M<=%d) cannot keep one CTA per SM with %zu B smem", mm, smem);
   }
@@ -323,7 +328,7 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->tmaps, sizeof(CUtensorMap) * (size_t)(L * MAPS_PER_LAYER + 1));
   HALLOC(h->norms, sizeof(void *) * 2 * L);
   HALLOC(h->h, sizeof(float) * (size_t)kMaxRows * D);
-  HALLOC(h->ss, sizeof(float) * (size_t)kMaxRows * ceil_div(D, 8));
+  HALLOC(h->ss, sizeof(float) * (size_t)kMaxRows * ceil_div(ceil_div(D, kRows), 128) * 128);
   HALLOC(h->qkv, sizeof(float) * (size_t)kMaxRows * QKVW);
   HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
   HALLOC(h->attn_o, sizeof(float) * s.attn_o);
@@ -332,10 +337,11 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->attn_ml1, sizeof(float) * s.attn_ml1);
   h->attn_cnt_bytes = sizeof(uint32_t) * s.attn_cnt;
   HALLOC(h->attn_cnt, h->attn_cnt_bytes);
-  HALLOC(h->router_part, sizeof(float) * (size_t)ceil_div(D, kPanel) * kMaxRows * d.n_experts);
+  HALLOC(h->router_part, sizeof(float) * (size_t)ceil_div(D, kTileCols) * kMaxRows * ceil_div(d.n_experts, 4) * 4);
   HALLOC(h->routing, sizeof(Routing) * (size_t)L);
-  HALLOC(h->gu_shared, sizeof(float) * (size_t)kMaxRows * 2 * std::max(d.shared_ffn, 1));
-  HALLOC(h->gu_routed, sizeof(float) * (size_t)umax * kMaxRows * 2 * d.expert_ffn);
+  HALLOC(h->act_shared, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
+  HALLOC(h->act_routed, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
+  HALLOC(h->y_part, sizeof(float) * (size_t)kMaxRows * (d.top_k + 1) * D);
   HALLOC(h->am_part, sizeof(ArgmaxPart) * (size_t)NW * kMaxRows);
   HALLOC(h->rope, sizeof(float2) * (size_t)d.kv_capacity * (d.head_dim / 2));
   h->counters_bytes = sizeof(uint32_t) * (size_t)n_ops * kCounterStride;
@@ -354,7 +360,7 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   std::vector<CUtensorMap> maps((size_t)L * MAPS_PER_LAYER + 1);
   std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
   auto enc = [&](int idx, const void *p, uint64_t rows, uint64_t cols) -> int {
-    return encode_2d(&maps[idx], p, rows, cols, kPanel, kBoxRows);
+    return encode_2d(&maps[idx], p, rows, cols, kPanel, kRows);
   };
   std::vector<const void *> norm_ptrs(2 * L);
   for (int l = 0; l < L && rc == MK_OK; ++l) {
@@ -442,7 +448,10 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.Bmax = d.max_seqs; p.cap = d.kv_capacity; p.eps = d.rms_eps;
   p.B = B; p.T = T; p.M = B * T; p.max_rows = d.max_rows;
   p.n_cta = pl.n_cta; p.n_warps = pl.n_warps; p.op_begin = 0; p.op_end = pl.n_ops; p.n_ops = pl.n_ops;
-  p.rows_per_tile = pl.rows_per_tile; p.n_hb = pl.n_hb;
+  p.n_hb = pl.n_hb;
+  p.xs_floats = pl.xs_floats;
+  p.ss_ld = ceil_div(pl.n_hb, 128) * 128;
+  p.e_ld = ceil_div(d.n_experts, 4) * 4;
   p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit; p.attn_qvp = pl.attn_qvp;
   p.attn_ppt = pl.attn_ppt; p.attn_nch_max = pl.attn_nch_max;
   p.tmaps = h->tmaps; p.norms = h->norms;
@@ -453,10 +462,13 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.h = h->h; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
   p.attn_o = h->attn_o; p.attn_ml = h->attn_ml; p.attn_o1 = h->attn_o1; p.attn_ml1 = h->attn_ml1;
   p.attn_cnt = h->attn_cnt; p.router_part = h->router_part; p.routing = h->routing;
-  p.gu_shared = h->gu_shared; p.gu_routed = h->gu_routed; p.am_part = h->am_part; p.rope = h->rope;
-  p.counters = h->counters; p.route_flag = h->route_flag; p.epoch = h->epoch; p.error = h->error;
+  p.act_shared = h->act_shared; p.act_routed = h->act_routed; p.y_part = h->y_part;
+  p.am_part = h->am_part; p.rope = h->rope;
+  p.counters = h->counters; p.route_flag = h->route_flag;
+  p.epoch = h->epoch; p.error = h->error;
   p.stats = h->stats_dev;
   p.dbg_hidden = h->dbg_hidden; p.dbg_ids = h->dbg_ids; p.dbg_w = h->dbg_w;
+  p.trace = h->trace;
   p.timeout_ns = h->timeout_ns;
   p.inject_op = -1;
   return MK_OK;
@@ -502,7 +514,7 @@ static int run_step(mk_handle *h, const int32_t *tokens, const int32_t *position
                         (uint64_t)(uintptr_t)h->dbg_hidden,
                         (uint64_t)(uintptr_t)h->dbg_ids ^ (uint64_t)(uintptr_t)h->dbg_w,
                         h->timeout_ns,
-                        0};
+                        (uint64_t)(uintptr_t)h->trace};
     cudaGraphExec_t exec = nullptr;
     for (auto &g : h->graphs)
       if (std::memcmp(g.key, key, sizeof key) == 0) exec = g.exec;
@@ -604,6 +616,12 @@ MK_API int mk_set_debug(mk_handle *h, float *hidden, int32_t *expert_ids, float 
   h->dbg_hidden = hidden;
   h->dbg_ids = expert_ids;
   h->dbg_w = expert_w;
+  return MK_OK;
+}
+
+MK_API int mk_set_trace(mk_handle *h, uint64_t *trace) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  h->trace = reinterpret_cast<unsigned long long *>(trace);
   return MK_OK;
 }
 

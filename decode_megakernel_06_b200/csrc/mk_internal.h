@@ -15,23 +15,25 @@ constexpr int kThreads = kWarpsPerCta * 32;
 constexpr int kSlots = 3;                           // ring slots per warp
 constexpr int kSlotBytes = 8192;                    // one tile: two 4 KB TMA boxes
 constexpr int kPanel = 256;                         // columns per weight box
-constexpr int kBoxRows = 8;                         // rows per weight box
-constexpr int kBoxBytes = kPanel * kBoxRows * 2;    // 4096
+constexpr int kRows = 4;                            // rows per weight box, tile and unit
+constexpr int kPanels = 4;                          // weight boxes per tile
+constexpr int kTileCols = kPanels * kPanel;         // a tile is 4 rows x 1024 columns
+constexpr int kBoxBytes = kPanel * kRows * 2;       // 2048
+constexpr int kKvBoxBytes = 4096;                   // K or V box: ppt positions x hd
 constexpr int kMaxRows = 8;                         // M = B*T cap of this build
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 16;
 constexpr int kL1Fan = 16;                          // attention merge fan-in per level
 constexpr int kMaxChunks = kL1Fan * kL1Fan;         // KV chunks per (seq, kv head, q group)
 constexpr int kCounterStride = 32;                  // uint32s between counters (128 B)
-constexpr int kRouterKChunk = 2 * kPanel;           // router split-K width (512 columns)
 
 // Ops of one step: EMBED, then per layer QKV ATTN OPROJ ROUTER SHARED_GU
-// ROUTED_GU DOWN, then LMHEAD.
+// ROUTED_GU DOWN COMBINE, then LMHEAD.
 enum OpType : int {
   OP_EMBED = 0, OP_QKV = 1, OP_ATTN = 2, OP_OPROJ = 3, OP_ROUTER = 4,
-  OP_SHARED_GU = 5, OP_ROUTED_GU = 6, OP_DOWN = 7, OP_LMHEAD = 8
+  OP_SHARED_GU = 5, OP_ROUTED_GU = 6, OP_DOWN = 7, OP_COMBINE = 8, OP_LMHEAD = 9
 };
-constexpr int kOpsPerLayer = 7;
+constexpr int kOpsPerLayer = 8;
 
 __host__ __device__ inline int n_ops_for(int L) { return kOpsPerLayer * L + 2; }
 __host__ __device__ inline int op_type_of(int op, int L) {
@@ -53,15 +55,19 @@ __host__ __device__ inline void op_deps(int op, int L, int *d0, int *d1) {
   *d1 = -1;
   switch (t) {
     case OP_EMBED: break;
-    case OP_QKV: *d0 = (l == 0) ? 0 : op_index(l - 1, OP_DOWN); break;
+    case OP_QKV: *d0 = (l == 0) ? 0 : op_index(l - 1, OP_COMBINE); break;
     case OP_ATTN: *d0 = op_index(l, OP_QKV); break;
     case OP_OPROJ: *d0 = op_index(l, OP_ATTN); break;
     case OP_ROUTER:
     case OP_SHARED_GU:
     case OP_ROUTED_GU: *d0 = op_index(l, OP_OPROJ); break;  // ROUTED_GU: + routing
     case OP_DOWN: *d0 = op_index(l, OP_SHARED_GU); *d1 = op_index(l, OP_ROUTED_GU); break;
-    case OP_LMHEAD: *d0 = op_index(L - 1, OP_DOWN); break;
+    case OP_COMBINE: *d0 = op_index(l, OP_DOWN); break;
+    case OP_LMHEAD: *d0 = op_index(L - 1, OP_COMBINE); break;
   }
+}
+__host__ __device__ inline bool op_has_tiles(int type) {
+  return type != OP_EMBED && type != OP_COMBINE;
 }
 
 // Tensor maps per layer, in this order; the lm_head map follows the last layer.
@@ -72,10 +78,12 @@ enum MapSlot : int {
 
 // Routing of one layer, written by the last warp to finish the router op.
 struct Routing {
-  int n_union;                           // distinct experts over the M rows
-  int expert[kMaxExperts];               // ascending expert ids, [n_union]
-  uint32_t rowmask[kMaxExperts];         // rows routed to expert[j]
-  float weight[kMaxExperts][kMaxRows];   // renormalised weight of row m (0 if absent)
+  int n_union;                            // distinct experts over the M rows
+  int expert[kMaxExperts];                // ascending expert ids, [n_union]
+  uint32_t rowmask[kMaxExperts];          // rows routed to expert[j]
+  int8_t kslot[kMaxExperts][kMaxRows];    // selection index of expert[j] in row m
+  int row_e[kMaxRows][kMaxTopK];          // row m's selections, in selection order
+  float row_w[kMaxRows][kMaxTopK];        // and their renormalised weights
 };
 
 struct ArgmaxPart {
@@ -92,8 +100,10 @@ struct alignas(64) Params {
   int B, T, M, max_rows;
   // grid / schedule
   int n_cta, n_warps, op_begin, op_end, n_ops;
-  int rows_per_tile;   // 16 (tall tiles) or 8 (wide tiles)
-  int n_hb;            // residual row blocks (ceil(d / rows_per_tile))
+  int n_hb;            // residual row blocks (ceil(d / kRows))
+  int xs_floats;       // shared-memory activation row (batch 1), 0 = none
+  int ss_ld;           // row stride of the sum-of-squares partials (n_hb rounded up to 128)
+  int e_ld;            // row stride of the router partials (E rounded up to 4)
   int attn_chunk, attn_qsplit, attn_qvp, attn_ppt, attn_nch_max;
   // weights
   const CUtensorMap *tmaps;              // [L][MAPS_PER_LAYER] + lm_head
@@ -110,7 +120,7 @@ struct alignas(64) Params {
   uint32_t *attn_cnt;
   float *router_part;
   Routing *routing;                      // [L]
-  float *gu_shared, *gu_routed;
+  float *act_shared, *act_routed, *y_part;   // silu(gate) * up per row; down partials
   ArgmaxPart *am_part;
   const float2 *rope;                    // [cap][hd/2] (cos, sin) of p * theta^(-2i/hd)
   uint32_t *counters, *route_flag, *epoch;
@@ -120,13 +130,15 @@ struct alignas(64) Params {
   float *dbg_hidden;
   int *dbg_ids;
   float *dbg_w;
+  unsigned long long *trace;
   unsigned long long timeout_ns;
   int inject_op;                         // op whose dependency is made unreachable, -1 none
 };
 
 // Launch entry points implemented in mk_kernel.cu.
 int launch_step(const Params &p, int mmax, bool cooperative, cudaStream_t stream);
-size_t step_smem_bytes(int n_ops);
+size_t step_smem_bytes(int n_ops, int xs_floats);
+bool kernel_stages_x(int mmax);
 int max_cta_per_sm(int mmax, size_t smem);
 
 }  // namespace mk

@@ -12,22 +12,28 @@
 // a load is issued as early as on-chip memory allows).  Only routed-expert
 // tiles wait, for the router's result.
 //
-// The step is a fixed list of ops (EMBED; per layer QKV, ATTN, OPROJ,
-// ROUTER, SHARED_GU, ROUTED_GU, DOWN; LMHEAD).  Each op's work is cut into
-// units dealt round-robin to the grid's warps.  A warp finishing its units of
-// an op arrives on that op's counter (aggregated per CTA in shared memory,
-// then one release-add per CTA); an op that needs an earlier op's output
-// spins (bounded by %globaltimer) until that counter reaches
-// epoch * n_cta.  Counters only grow, so no reset is needed between steps.
+// The step is a fixed list of ops (EMBED; per layer QKV, ATTN, OPROJ, ROUTER,
+// SHARED_GU, ROUTED_GU, DOWN, COMBINE; LMHEAD).  Each op's work is cut into
+// units of at most 64 KB of weights, dealt round-robin to the grid's warps
+// (consecutive units land on different SMs).  A warp done with an op arrives
+// on the op's counter (aggregated per CTA in shared memory, then one
+// release-add per CTA); an op that needs an earlier op's output spins (bounded
+// by %globaltimer) until that counter reaches epoch * n_cta.  Counters only
+// grow, so no reset is needed between steps.
 //
-// GEMV math: tile = 16 weight rows x 256 columns (8 rows x 512 columns when a
-// step has more than 4 rows); each lane owns 8 columns and keeps the matching
-// activations of every row in registers, so one 16-byte weight load feeds
-// 8*MJ FMAs.  Lane partial sums are combined with a butterfly
-// (transpose-reduce) of warp shuffles.  All arithmetic is fp32.
+// GEMV math: a tile is 4 weight rows x 1024 columns (four 4 x 256 TMA boxes);
+// each lane owns 8 columns of each box and keeps the matching activations of
+// every row in registers, so one 16-byte weight load feeds 8*MJ FMAs.  Lane
+// partial sums are combined with a butterfly (transpose-reduce) of warp
+// shuffles.  All arithmetic is fp32.
+//
+// Everything on the per-tile path is force-inlined so that a warp's ring and
+// cursor state stays in registers.
 #include <cstdio>
 
 #include "mk_internal.h"
+
+#define MK_INLINE __device__ __forceinline__
 
 namespace mk {
 namespace {
@@ -35,21 +41,18 @@ namespace {
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t saddr(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
+MK_INLINE uint32_t saddr(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+MK_INLINE void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(bar)), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)),
-               "r"(bytes)
+MK_INLINE void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes)
                : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+MK_INLINE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -61,18 +64,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
+MK_INLINE void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
+MK_INLINE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 2-D tiled TMA load, global -> this CTA's shared memory, completion counted
 // on `bar`.  Never multicast.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar, uint64_t policy) {
+MK_INLINE void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
+                           uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(saddr(dst)),
@@ -80,45 +79,43 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
-__device__ __forceinline__ uint64_t policy_evict_first() {
+MK_INLINE uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
-__device__ __forceinline__ uint64_t policy_evict_normal() {
+MK_INLINE uint64_t policy_evict_normal() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
-__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t *p) {
+MK_INLINE uint32_t ld_relaxed(const uint32_t *p) {
   uint32_t v;
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
-__device__ __forceinline__ void st_release(uint32_t *p, uint32_t v) {
+MK_INLINE void st_release(uint32_t *p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
+MK_INLINE uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
   uint32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
 }
 
-__device__ __forceinline__ void fence_acq_rel() {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
+MK_INLINE void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
-__device__ __forceinline__ uint64_t now_ns() {
+MK_INLINE uint64_t now_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 
-__device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
+MK_INLINE uint4 ld_shared_v4(const void *p) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
@@ -127,29 +124,27 @@ __device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
 }
 
 // bf16 pair in a 32-bit word -> two floats (exact).
-__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+MK_INLINE float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+MK_INLINE float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
-__device__ __forceinline__ void unpack8(const uint4 &w, float (&f)[8]) {
+MK_INLINE void unpack8(const uint4 &w, float (&f)[8]) {
   f[0] = bf_lo(w.x); f[1] = bf_hi(w.x); f[2] = bf_lo(w.y); f[3] = bf_hi(w.y);
   f[4] = bf_lo(w.z); f[5] = bf_hi(w.z); f[6] = bf_lo(w.w); f[7] = bf_hi(w.w);
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
-  return __ldg(reinterpret_cast<const uint4 *>(p));
-}
+MK_INLINE uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 
-__device__ __forceinline__ float silu(float u) { return u / (1.0f + expf(-u)); }
+MK_INLINE float silu(float u) { return u / (1.0f + expf(-u)); }
 
 __host__ __device__ constexpr int ilog2c(int n) { return n <= 1 ? 0 : 1 + ilog2c(n >> 1); }
 
-__device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+MK_INLINE int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 // Butterfly transpose-reduce of N partial sums over the 32 lanes.  After it,
 // for N >= 32 lane l holds the full sums of indices (N/32)*l + i in v[i];
 // for N < 32 lane l holds index l >> (5 - log2 N) in v[0].
 template <int N>
-__device__ __forceinline__ void butterfly(float (&v)[N], int lane) {
+MK_INLINE void butterfly(float (&v)[N], int lane) {
   constexpr int S = (N >= 32) ? 5 : ilog2c(N);
 #pragma unroll
   for (int s = 0; s < 5; ++s) {
@@ -159,8 +154,8 @@ __device__ __forceinline__ void butterfly(float (&v)[N], int lane) {
 #pragma unroll
       for (int i = 0; i < (N >> (s + 1)); ++i) {
         const int hh = N >> (s + 1);
-        float send = up ? v[i] : v[i + hh];
-        float recv = __shfl_xor_sync(0xffffffffu, send, o);
+        const float send = up ? v[i] : v[i + hh];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, o);
         v[i] = (up ? v[i + hh] : v[i]) + recv;
       }
     } else {
@@ -171,7 +166,7 @@ __device__ __forceinline__ void butterfly(float (&v)[N], int lane) {
 
 // Store the butterfly result so that buf[i] = full sum of index i (i < N).
 template <int N>
-__device__ __forceinline__ void butterfly_store(const float (&v)[N], float *buf, int lane) {
+MK_INLINE void butterfly_store(const float (&v)[N], float *buf, int lane) {
   if constexpr (N >= 32) {
 #pragma unroll
     for (int i = 0; i < N / 32; ++i) buf[(N / 32) * lane + i] = v[i];
@@ -181,94 +176,91 @@ __device__ __forceinline__ void butterfly_store(const float (&v)[N], float *buf,
   }
 }
 
-__device__ __forceinline__ float warp_max(float v) {
+MK_INLINE float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
+MK_INLINE float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
+// Units are dealt round-robin: warp slot s takes units u0(s) + i * n_warps,
+// with a per-op rotation so that remainders do not always land on warp 0.
+MK_INLINE int first_unit_of(int slot, int op, int nw) {
+  const int rot = static_cast<int>((static_cast<uint32_t>(op) * 2654435761u) % static_cast<uint32_t>(nw));
+  return (slot - rot + nw) % nw;
+}
+
+MK_INLINE int unit_count_of(int u0, int total, int nw) { return total > u0 ? (total - 1 - u0) / nw + 1 : 0; }
+
 // ---------------------------------------------------------------------------
-// Per-warp state
+// Per-warp state (scalars only, so that it lives in registers)
 // ---------------------------------------------------------------------------
-constexpr int kWbuf = 64;  // floats of per-warp epilogue scratch (R * MJ <= 64)
+constexpr int kWbuf = 64;  // floats of per-warp epilogue scratch (2 * 4 * MJ <= 64)
 
 struct Warp {
   const Params *P;
-  int lane, wib, slot, nw;
+  int lane, slot, nw;
   uint32_t epoch;
   uint8_t *ring;
   uint64_t *bars;
-  float *wbuf, *wacc, *wtmp;
+  float *wbuf;
   uint32_t *arrive;
-  uint32_t phase;  // bit s: parity of the next completion of slot s
+  const int *attn_prefix;  // shared: first item of each sequence, [kMaxRows + 1]
+  const int *attn_nch;     // shared: KV chunks of each sequence, [kMaxRows]
+  uint32_t phase;          // bit s: parity of the next completion of slot s
   int cslot, islot, inflight;
-  // issue cursor
-  int iop, iu, it, in_units, in_tiles;
+  // producer cursor: op, this warp's unit index in it, tile in the unit
+  int iop, iu0, in_units, iu, it, in_tiles, iunit;
+  // the current unit's tile source: maps for the first and second half of its
+  // tiles (gate / up), first row of each, first column, K, tiles per half
+  const CUtensorMap *um, *um2;
+  int urow0, urow2, ucol0, uK, uhalf;
   bool iop_init, done_issue;
-  // attention items: prefix[b] = first item of sequence b
-  int attn_prefix[kMaxRows + 1];
-  int attn_nch[kMaxRows];
   uint64_t pol_w, pol_kv;
   bool failed;
 };
 
-__device__ __forceinline__ const Params &PP(const Warp &w) { return *w.P; }
-
-__device__ void set_error(Warp &w, int code, int op) {
-  if (w.lane == 0) {
-    if (atomicCAS(&w.P->error[0], 0, code) == 0) atomicExch(&w.P->error[1], op);
+__device__ __noinline__ void report_error(const Params &P, int lane, int code, int op) {
+  if (lane == 0) {
+    if (atomicCAS(&P.error[0], 0, code) == 0) atomicExch(&P.error[1], op);
   }
+}
+
+MK_INLINE void set_error(Warp &w, int code, int op) {
+  report_error(*w.P, w.lane, code, op);
   w.failed = true;
 }
 
-__device__ __forceinline__ int rot_of(int op, int nw) {
-  return static_cast<int>((static_cast<uint32_t>(op) * 2654435761u) % static_cast<uint32_t>(nw));
-}
-
-__device__ __forceinline__ int first_unit(const Warp &w, int op) {
-  return (w.slot - rot_of(op, w.nw) + w.nw) % w.nw;
-}
-
-__device__ __forceinline__ int my_unit_count(const Warp &w, int op, int total) {
-  int u0 = first_unit(w, op);
-  return total > u0 ? (total - 1 - u0) / w.nw + 1 : 0;
-}
-
-__device__ __forceinline__ int tile_cols(const Params &P) { return P.rows_per_tile == 16 ? 256 : 512; }
-
-__device__ __forceinline__ bool routing_ready(const Warp &w, int layer) {
-  uint32_t v = 0;
-  if (w.lane == 0) v = ld_relaxed(&w.P->route_flag[layer * kCounterStride]);
-  v = __shfl_sync(0xffffffffu, v, 0);
-  bool ok = static_cast<int>(v - w.epoch) >= 0;
+// Every lane reads the flag itself, so that each lane's acquire fence follows
+// its own observation of the release.
+MK_INLINE bool routing_ready(const Warp &w, int layer) {
+  const uint32_t v = ld_relaxed(&w.P->route_flag[layer * kCounterStride]);
+  const bool ok = __all_sync(0xffffffffu, static_cast<int>(v - w.epoch) >= 0);
   if (ok) fence_acq_rel();
   return ok;
 }
 
-__device__ __forceinline__ int n_union(const Warp &w, int layer) {
-  return __ldcg(&w.P->routing[layer].n_union);
-}
+MK_INLINE int n_union(const Params &P, int layer) { return __ldcg(&P.routing[layer].n_union); }
 
 // Total units of an op over the whole grid.  ROUTED_GU / DOWN need routing.
-__device__ int op_total_units(const Warp &w, int type, int layer) {
-  const Params &P = PP(w);
-  const int R = P.rows_per_tile;
+MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
+  const Params &P = *w.P;
   switch (type) {
     case OP_EMBED: return P.n_hb;
-    case OP_QKV: return cdiv((P.Hq + 2 * P.Hkv) * P.hd, R);
+    case OP_QKV: return cdiv((P.Hq + 2 * P.Hkv) * P.hd, kRows);
     case OP_ATTN: return w.attn_prefix[P.B];
     case OP_OPROJ: return P.n_hb;
-    case OP_ROUTER: return cdiv(P.E, R) * cdiv(P.d, tile_cols(P));
-    case OP_SHARED_GU: return P.Fs > 0 ? (2 * P.Fs) / R : 0;
-    case OP_ROUTED_GU: return n_union(w, layer) * ((2 * P.F) / R);
-    case OP_DOWN: return P.n_hb;
-    case OP_LMHEAD: return cdiv(P.V, R);
+    case OP_ROUTER: return cdiv(P.E, kRows) * cdiv(P.d, kTileCols);
+    case OP_SHARED_GU: return P.Fs / kRows;
+    case OP_ROUTED_GU: return n_union(P, layer) * (P.F / kRows);
+    case OP_DOWN: return (n_union(P, layer) + (P.Fs > 0 ? 1 : 0)) * P.n_hb;
+    case OP_COMBINE: return P.n_hb;
+    case OP_LMHEAD: return cdiv(P.V, kRows);
   }
   return 0;
 }
@@ -277,161 +269,147 @@ struct AttnItem {
   int b, g, qs, c, pos0, npos, ntiles;
 };
 
-__device__ AttnItem attn_item(const Warp &w, int item) {
-  const Params &P = PP(w);
+MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs, int item) {
   AttnItem a;
   int b = 0;
-  while (b + 1 < P.B && item >= w.attn_prefix[b + 1]) ++b;
-  int rem = item - w.attn_prefix[b];
-  int nch = w.attn_nch[b];
+  while (b + 1 < P.B && item >= prefix[b + 1]) ++b;
+  const int rem = item - prefix[b];
+  const int nch = nchs[b];
   a.b = b;
   a.c = rem % nch;
   a.qs = (rem / nch) % P.attn_qsplit;
   a.g = rem / (nch * P.attn_qsplit);
-  int len = __ldg(&P.positions[b]) + P.T;
+  const int len = __ldg(&P.positions[b]) + P.T;
   a.pos0 = a.c * P.attn_chunk;
   a.npos = min(P.attn_chunk, len - a.pos0);
   a.ntiles = cdiv(a.npos, P.attn_ppt);
   return a;
 }
 
-__device__ int unit_tiles(const Warp &w, int type, int layer, int unit) {
-  const Params &P = PP(w);
-  const int TC = tile_cols(P);
+// Tiles of one unit.  Gate/up units stream their gate rows, then their up rows.
+MK_INLINE int unit_tiles(const Warp &w, int type, int layer, int unit) {
+  const Params &P = *w.P;
   switch (type) {
     case OP_QKV:
+    case OP_LMHEAD: return cdiv(P.d, kTileCols);
     case OP_SHARED_GU:
-    case OP_ROUTED_GU:
-    case OP_LMHEAD: return cdiv(P.d, TC);
-    case OP_OPROJ: return cdiv(P.Hq * P.hd, TC);
+    case OP_ROUTED_GU: return 2 * cdiv(P.d, kTileCols);
+    case OP_OPROJ: return cdiv(P.Hq * P.hd, kTileCols);
     case OP_ROUTER: return 1;
-    case OP_DOWN:
-      return n_union(w, layer) * cdiv(P.F, TC) + (P.Fs > 0 ? cdiv(P.Fs, TC) : 0);
-    case OP_ATTN: return attn_item(w, unit).ntiles;
+    case OP_DOWN: return (unit / P.n_hb) < n_union(P, layer) ? cdiv(P.F, kTileCols) : cdiv(P.Fs, kTileCols);
+    case OP_ATTN: return attn_item(P, w.attn_prefix, w.attn_nch, unit).ntiles;
     default: return 0;
   }
 }
 
 // ---------------------------------------------------------------------------
-// Producer side: issue the next tiles of this warp's stream into free slots.
+// Producer side: issue the tiles of this warp's next units into free slots.
 // ---------------------------------------------------------------------------
-__device__ void issue_tile(Warp &w, int op, int type, int layer, int unit, int t) {
-  const Params &P = PP(w);
-  const int R = P.rows_per_tile, TC = tile_cols(P);
-  const bool tall = (R == 16);
+// Where the tiles of a GEMV unit come from.
+MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
+  const Params &P = *w.P;
+  const CUtensorMap *lm = P.tmaps + layer * MAPS_PER_LAYER;
+  int row0 = unit * kRows, col0 = 0, K = P.d, half = 1 << 30, row2 = 0;
+  const CUtensorMap *m0 = nullptr, *m2 = nullptr;
+  switch (type) {
+    case OP_QKV: m0 = lm + MAP_WQKV; break;
+    case OP_OPROJ: m0 = lm + MAP_WO; K = P.Hq * P.hd; break;
+    case OP_LMHEAD: m0 = P.tmaps + P.L * MAPS_PER_LAYER; break;
+    case OP_ROUTER: {
+      const int nrb = cdiv(P.E, kRows);
+      row0 = (unit % nrb) * kRows;
+      col0 = (unit / nrb) * kTileCols;
+      m0 = lm + MAP_ROUTER;
+      break;
+    }
+    case OP_SHARED_GU:
+      m0 = lm + MAP_WSGATE;
+      m2 = lm + MAP_WSUP;
+      row2 = row0;
+      half = cdiv(P.d, kTileCols);
+      break;
+    case OP_ROUTED_GU: {
+      const int nfb = P.F / kRows;
+      const int e = __ldcg(&P.routing[layer].expert[unit / nfb]);
+      row0 = row2 = e * P.F + (unit % nfb) * kRows;
+      m0 = lm + MAP_WGATE;
+      m2 = lm + MAP_WUP;
+      half = cdiv(P.d, kTileCols);
+      break;
+    }
+    case OP_DOWN: {
+      const int seg = unit / P.n_hb, rb = unit % P.n_hb;
+      if (seg < n_union(P, layer)) {
+        const int e = __ldcg(&P.routing[layer].expert[seg]);
+        m0 = lm + MAP_WDOWN;
+        row0 = e * P.d + rb * kRows;
+        K = P.F;
+      } else {
+        m0 = lm + MAP_WSDOWN;
+        row0 = rb * kRows;
+        K = P.Fs;
+      }
+      break;
+    }
+    default: break;
+  }
+  w.um = m0;
+  w.um2 = m2;
+  w.urow0 = row0;
+  w.urow2 = row2;
+  w.ucol0 = col0;
+  w.uK = K;
+  w.uhalf = half;
+}
+
+MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
+  const Params &P = *w.P;
   uint8_t *dst = w.ring + w.islot * kSlotBytes;
   uint64_t *bar = &w.bars[w.islot];
-  const CUtensorMap *m0 = nullptr, *m1 = nullptr;
-  int x0 = 0, y0 = 0, x1 = 0, y1 = 0, K = P.d, rows = 0;
-  bool two = true;
-  uint64_t pol = w.pol_w;
-  const CUtensorMap *lm = P.tmaps + layer * MAPS_PER_LAYER;
   if (type == OP_ATTN) {
-    AttnItem a = attn_item(w, unit);
-    int pos = a.pos0 + t * P.attn_ppt;
-    int row = ((layer * P.Bmax + a.b) * P.Hkv + a.g) * P.cap + pos;
-    m0 = &P.kmap;
-    m1 = &P.vmap;
-    x0 = x1 = 0;
-    y0 = y1 = row;
-    pol = w.pol_kv;
+    const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, w.iunit);
+    const int row = ((layer * P.Bmax + a.b) * P.Hkv + a.g) * P.cap + a.pos0 + t * P.attn_ppt;
+    if (w.lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(bar, 2u * kKvBoxBytes);
+      tma_load_2d(dst, &P.kmap, 0, row, bar, w.pol_kv);
+      tma_load_2d(dst + kKvBoxBytes, &P.vmap, 0, row, bar, w.pol_kv);
+    }
   } else {
-    int row0 = 0, col0 = t * TC;
-    switch (type) {
-      case OP_QKV: m0 = lm + MAP_WQKV; row0 = unit * R; rows = (P.Hq + 2 * P.Hkv) * P.hd; break;
-      case OP_OPROJ: m0 = lm + MAP_WO; row0 = unit * R; K = P.Hq * P.hd; rows = P.d; break;
-      case OP_LMHEAD: m0 = P.tmaps + P.L * MAPS_PER_LAYER; row0 = unit * R; rows = P.V; break;
-      case OP_ROUTER: {
-        int nrb = cdiv(P.E, R);
-        row0 = (unit % nrb) * R;
-        col0 = (unit / nrb) * TC;
-        m0 = lm + MAP_ROUTER;
-        rows = P.E;
-        break;
-      }
-      case OP_SHARED_GU:
-        row0 = unit * R;
-        if (row0 < P.Fs) {
-          m0 = lm + MAP_WSGATE;
-        } else {
-          m0 = lm + MAP_WSUP;
-          row0 -= P.Fs;
-        }
-        rows = P.Fs;
-        break;
-      case OP_ROUTED_GU: {
-        int nrb = (2 * P.F) / R;
-        int j = unit / nrb;
-        int r0 = (unit % nrb) * R;
-        int e = __ldcg(&P.routing[layer].expert[j]);
-        if (r0 < P.F) {
-          m0 = lm + MAP_WGATE;
-        } else {
-          m0 = lm + MAP_WUP;
-          r0 -= P.F;
-        }
-        row0 = e * P.F + r0;
-        rows = P.E * P.F;
-        break;
-      }
-      case OP_DOWN: {
-        int U = n_union(w, layer);
-        int tpr = cdiv(P.F, TC);
-        if (t < U * tpr) {
-          int j = t / tpr;
-          int e = __ldcg(&P.routing[layer].expert[j]);
-          m0 = lm + MAP_WDOWN;
-          row0 = e * P.d + unit * R;
-          col0 = (t % tpr) * TC;
-          K = P.F;
-          rows = P.E * P.d;
-        } else {
-          m0 = lm + MAP_WSDOWN;
-          row0 = unit * R;
-          col0 = (t - U * tpr) * TC;
-          K = P.Fs;
-          rows = P.d;
-        }
-        break;
-      }
-      default: break;
+    // up to four 4 x 256 boxes side by side; boxes starting past K are skipped
+    const bool second = t >= w.uhalf;
+    const int tt = second ? t - w.uhalf : t;
+    const CUtensorMap *m = second ? w.um2 : w.um;
+    const int y = second ? w.urow2 : w.urow0;
+    const int x0 = w.ucol0 + tt * kTileCols;
+    const int nbox = min(kPanels, cdiv(w.uK - x0, kPanel));
+    if (w.lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * kBoxBytes);
+      for (int p = 0; p < nbox; ++p) tma_load_2d(dst + p * kBoxBytes, m, x0 + p * kPanel, y, bar, w.pol_w);
     }
-    m1 = m0;
-    x0 = col0;
-    y0 = row0;
-    if (tall) {
-      x1 = col0;
-      y1 = row0 + kBoxRows;
-      two = (y1 < rows);
-    } else {
-      x1 = col0 + kPanel;
-      y1 = row0;
-      two = (x1 < K);
-    }
-  }
-  if (w.lane == 0) {
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar, (two ? 2u : 1u) * kBoxBytes);
-    tma_load_2d(dst, m0, x0, y0, bar, pol);
-    if (two) tma_load_2d(dst + kBoxBytes, m1, x1, y1, bar, pol);
   }
   w.islot = (w.islot + 1 == kSlots) ? 0 : w.islot + 1;
   w.inflight++;
 }
 
-__device__ void issue_more(Warp &w) {
-  const Params &P = PP(w);
-  while (!w.done_issue && w.inflight < kSlots && !w.failed) {
+MK_INLINE void issue_more(Warp &w) {
+  const Params &P = *w.P;
+  while (!w.done_issue && !w.failed && w.inflight < kSlots) {
     if (w.iop >= P.op_end) {
       w.done_issue = true;
       break;
     }
     const int type = op_type_of(w.iop, P.L), layer = op_layer_of(w.iop, P.L);
+    if (!op_has_tiles(type)) {
+      w.iop++;
+      continue;
+    }
     if (!w.iop_init) {
       if ((type == OP_ROUTED_GU || type == OP_DOWN) && !routing_ready(w, layer)) return;
-      w.in_units = (type == OP_EMBED) ? 0 : my_unit_count(w, w.iop, op_total_units(w, type, layer));
+      w.iu0 = first_unit_of(w.slot, w.iop, w.nw);
+      w.in_units = unit_count_of(w.iu0, op_total_units(w, type, layer), w.nw);
       w.iu = 0;
-      w.it = 0;
       w.in_tiles = -1;
       w.iop_init = true;
     }
@@ -440,15 +418,18 @@ __device__ void issue_more(Warp &w) {
       w.iop_init = false;
       continue;
     }
-    const int unit = first_unit(w, w.iop) + w.iu * w.nw;
-    if (w.in_tiles < 0) w.in_tiles = unit_tiles(w, type, layer, unit);
+    if (w.in_tiles < 0) {
+      w.iunit = w.iu0 + w.iu * w.nw;
+      w.it = 0;
+      w.in_tiles = unit_tiles(w, type, layer, w.iunit);
+      if (type != OP_ATTN) unit_source(w, type, layer, w.iunit);
+    }
     if (w.it >= w.in_tiles) {
       w.iu++;
-      w.it = 0;
       w.in_tiles = -1;
       continue;
     }
-    issue_tile(w, w.iop, type, layer, unit, w.it);
+    issue_tile(w, type, layer, w.it);
     w.it++;
   }
 }
@@ -456,9 +437,18 @@ __device__ void issue_more(Warp &w) {
 // ---------------------------------------------------------------------------
 // Consumer side
 // ---------------------------------------------------------------------------
-__device__ const uint8_t *consume_begin(Warp &w, int op) {
+__device__ __noinline__ bool wait_slot_slow(uint64_t *bar, uint32_t par, unsigned long long timeout_ns) {
+  const uint64_t t0 = now_ns();
+  for (;;) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, par))) return true;
+    int bad = 0;
+    if ((threadIdx.x & 31) == 0) bad = (now_ns() - t0 > timeout_ns) ? 1 : 0;
+    if (__shfl_sync(0xffffffffu, bad, 0)) return false;
+  }
+}
+
+MK_INLINE const uint8_t *consume_begin(Warp &w, int op) {
   if (w.failed) return nullptr;
-  const Params &P = PP(w);
   if (w.inflight == 0) issue_more(w);
   if (w.inflight == 0) {  // the tile stream and the consumer loop disagree: never expected
     set_error(w, -8, op);
@@ -466,27 +456,14 @@ __device__ const uint8_t *consume_begin(Warp &w, int op) {
   }
   uint64_t *bar = &w.bars[w.cslot];
   const uint32_t par = (w.phase >> w.cslot) & 1u;
-  uint64_t t0 = 0;
-  for (int it = 0;; ++it) {
-    bool ok = mbar_try_wait(bar, par);
-    if (__all_sync(0xffffffffu, ok)) break;
-    if ((it & 63) == 63) {
-      int bad = 0;
-      if (w.lane == 0) {
-        uint64_t t = now_ns();
-        if (t0 == 0) t0 = t;
-        bad = (t - t0 > P.timeout_ns) ? 1 : 0;
-      }
-      if (__shfl_sync(0xffffffffu, bad, 0)) {
-        set_error(w, -5, op);
-        return nullptr;
-      }
-    }
+  if (!__all_sync(0xffffffffu, mbar_try_wait(bar, par)) && !wait_slot_slow(bar, par, w.P->timeout_ns)) {
+    set_error(w, -5, op);
+    return nullptr;
   }
   return w.ring + w.cslot * kSlotBytes;
 }
 
-__device__ __forceinline__ void consume_end(Warp &w) {
+MK_INLINE void consume_end(Warp &w) {
   __syncwarp();
   w.phase ^= (1u << w.cslot);
   w.cslot = (w.cslot + 1 == kSlots) ? 0 : w.cslot + 1;
@@ -495,30 +472,27 @@ __device__ __forceinline__ void consume_end(Warp &w) {
 }
 
 // Wait for `ctr` to reach `target` (bounded), filling the ring meanwhile.
-__device__ bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int op) {
-  const Params &P = PP(w);
+MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int op) {
+  const Params &P = *w.P;
   uint64_t t0 = 0;
   for (int it = 0;; ++it) {
-    uint32_t v = 0;
+    // every lane reads the counter (one broadcast transaction), so that each
+    // lane's acquire fence below follows its own observation of the release
+    const uint32_t v = ld_relaxed(ctr);
+    if (__all_sync(0xffffffffu, static_cast<int>(v - target) >= 0)) break;
     int err = 0;
-    if (w.lane == 0) {
-      v = ld_relaxed(ctr);
-      err = *reinterpret_cast<volatile const int *>(P.error);
-    }
-    v = __shfl_sync(0xffffffffu, v, 0);
-    err = __shfl_sync(0xffffffffu, err, 0);
-    if (static_cast<int>(v - target) >= 0) break;
-    if (err) {
+    if (w.lane == 0) err = *reinterpret_cast<volatile const int *>(P.error);
+    if (__shfl_sync(0xffffffffu, err, 0)) {
       w.failed = true;
       return false;
     }
     issue_more(w);
     int bad = 0;
     if (w.lane == 0) {
-      uint64_t t = now_ns();
+      const uint64_t t = now_ns();
       if (t0 == 0) t0 = t;
       bad = (t - t0 > P.timeout_ns) ? 1 : 0;
-      if (!bad && it > 8) __nanosleep(64);
+      if (!bad && it > 8) __nanosleep(32);
     }
     if (__shfl_sync(0xffffffffu, bad, 0)) {
       set_error(w, -5, op);
@@ -530,12 +504,12 @@ __device__ bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int 
   return true;
 }
 
-__device__ void drain(Warp &w) {
+MK_INLINE void drain(Warp &w) {
   // Wait (bounded) for every copy still in flight before the CTA may exit.
   while (w.inflight > 0) {
     uint64_t *bar = &w.bars[w.cslot];
     const uint32_t par = (w.phase >> w.cslot) & 1u;
-    uint64_t t0 = now_ns();
+    const uint64_t t0 = now_ns();
     while (!mbar_try_wait(bar, par)) {
       if (now_ns() - t0 > 50000000ull) break;
     }
@@ -548,21 +522,25 @@ __device__ void drain(Warp &w) {
 
 // Arrive on an op's counter once this warp's units of it are done.  Returns
 // true (on every lane) for the warp whose arrival completed the op grid-wide.
-__device__ bool arrive(Warp &w, int op) {
-  const Params &P = PP(w);
+MK_INLINE bool arrive(Warp &w, int op) {
+  const Params &P = *w.P;
   __syncwarp();
   int last = 0;
   if (w.lane == 0) {
     __threadfence();
-    uint32_t old = atomicAdd(&w.arrive[op], 1u);
+    const uint32_t old = atomicAdd(&w.arrive[op], 1u);
     if (old == kWarpsPerCta - 1) {
       __threadfence();
-      uint32_t g = atom_add_acq_rel(&P.counters[op * kCounterStride], 1u);
+      const uint32_t g = atom_add_acq_rel(&P.counters[op * kCounterStride], 1u);
       last = (g + 1 == w.epoch * static_cast<uint32_t>(P.n_cta)) ? 1 : 0;
     }
   }
   last = __shfl_sync(0xffffffffu, last, 0);
-  if (last) fence_acq_rel();
+  if (last) {
+    // every lane observes the completed count before reading others' results
+    (void)ld_relaxed(&P.counters[op * kCounterStride]);
+    fence_acq_rel();
+  }
   __syncwarp();
   return last != 0;
 }
@@ -570,15 +548,16 @@ __device__ bool arrive(Warp &w, int op) {
 // ---------------------------------------------------------------------------
 // Activation sources (one lane, 8 consecutive columns, MJ rows)
 // ---------------------------------------------------------------------------
+// RMSNorm is applied as y = inv_rms * (W (h * g)): the per-row scalar is
+// factored out of the dot product and multiplied in the epilogue.
 template <int MJ>
-struct XNorm {  // x = h * inv_rms * g
+struct XNorm {  // x = h * g
   const float *h;
   int d;
   const __nv_bfloat16 *g;
   int row[MJ];
-  float inv[MJ];
   int n;
-  __device__ __forceinline__ void load(int col, int K, float (&x)[MJ][8]) const {
+  MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
     if (col < K) {
       float gf[8];
       unpack8(ldg_nc_v4(g + col), gf);
@@ -586,11 +565,9 @@ struct XNorm {  // x = h * inv_rms * g
       for (int j = 0; j < MJ; ++j) {
         if (j < n) {
           const float4 *p = reinterpret_cast<const float4 *>(h + static_cast<size_t>(row[j]) * d + col);
-          float4 a = __ldcg(p), b = __ldcg(p + 1);
-          x[j][0] = a.x * inv[j] * gf[0]; x[j][1] = a.y * inv[j] * gf[1];
-          x[j][2] = a.z * inv[j] * gf[2]; x[j][3] = a.w * inv[j] * gf[3];
-          x[j][4] = b.x * inv[j] * gf[4]; x[j][5] = b.y * inv[j] * gf[5];
-          x[j][6] = b.z * inv[j] * gf[6]; x[j][7] = b.w * inv[j] * gf[7];
+          const float4 a = __ldca(p), b = __ldca(p + 1);
+          x[j][0] = a.x * gf[0]; x[j][1] = a.y * gf[1]; x[j][2] = a.z * gf[2]; x[j][3] = a.w * gf[3];
+          x[j][4] = b.x * gf[4]; x[j][5] = b.y * gf[5]; x[j][6] = b.z * gf[6]; x[j][7] = b.w * gf[7];
         } else {
 #pragma unroll
           for (int k = 0; k < 8; ++k) x[j][k] = 0.f;
@@ -611,12 +588,12 @@ struct XPlain {  // x = src[row][col]
   int ld;
   int row[MJ];
   int n;
-  __device__ __forceinline__ void load(int col, int K, float (&x)[MJ][8]) const {
+  MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
 #pragma unroll
     for (int j = 0; j < MJ; ++j) {
       if (col < K && j < n) {
         const float4 *p = reinterpret_cast<const float4 *>(src + static_cast<size_t>(row[j]) * ld + col);
-        float4 a = __ldcg(p), b = __ldcg(p + 1);
+        const float4 a = __ldca(p), b = __ldca(p + 1);
         x[j][0] = a.x; x[j][1] = a.y; x[j][2] = a.z; x[j][3] = a.w;
         x[j][4] = b.x; x[j][5] = b.y; x[j][6] = b.z; x[j][7] = b.w;
       } else {
@@ -627,430 +604,436 @@ struct XPlain {  // x = src[row][col]
   }
 };
 
-template <int MJ>
-struct XSwiGLU {  // x = silu(gu[row][col]) * gu[row][F + col]
-  const float *gu;
-  int ld, F;
-  int row[MJ];
-  int n;
-  __device__ __forceinline__ void load(int col, int K, float (&x)[MJ][8]) const {
+// One activation row staged in shared memory by the CTA (batch 1): x = xs[col].
+struct XSmem {
+  const float *xs;
+  MK_INLINE void load(int col, int K, float (&x)[1][8]) const {
+    if (col < K) {
+      const float4 a = *reinterpret_cast<const float4 *>(xs + col);
+      const float4 b = *reinterpret_cast<const float4 *>(xs + col + 4);
+      x[0][0] = a.x; x[0][1] = a.y; x[0][2] = a.z; x[0][3] = a.w;
+      x[0][4] = b.x; x[0][5] = b.y; x[0][6] = b.z; x[0][7] = b.w;
+    } else {
 #pragma unroll
-    for (int j = 0; j < MJ; ++j) {
-      if (col < K && j < n) {
-        const float *base = gu + static_cast<size_t>(row[j]) * ld;
-        const float4 *pg = reinterpret_cast<const float4 *>(base + col);
-        const float4 *pu = reinterpret_cast<const float4 *>(base + F + col);
-        float4 g0 = __ldcg(pg), g1 = __ldcg(pg + 1), u0 = __ldcg(pu), u1 = __ldcg(pu + 1);
-        x[j][0] = silu(g0.x) * u0.x; x[j][1] = silu(g0.y) * u0.y;
-        x[j][2] = silu(g0.z) * u0.z; x[j][3] = silu(g0.w) * u0.w;
-        x[j][4] = silu(g1.x) * u1.x; x[j][5] = silu(g1.y) * u1.y;
-        x[j][6] = silu(g1.z) * u1.z; x[j][7] = silu(g1.w) * u1.w;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[j][k] = 0.f;
-      }
+      for (int k = 0; k < 8; ++k) x[0][k] = 0.f;
     }
   }
 };
 
-// One tile: acc[r*MJ + j] += W[r][cols] . x[j][cols] over this lane's columns.
-template <int MJ, int R, int NP, class XS>
-__device__ __forceinline__ void gemv_tile(const uint8_t *slot, float (&acc)[R * MJ], int colbase,
-                                          int K, const XS &xs, int lane) {
+template <int MJ>
+MK_INLINE void gemv_panel(const uint8_t *pan, float (&acc)[kRows * MJ], const float (&x)[MJ][8]) {
 #pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    const int pc = colbase + p * kPanel;
-    if (pc >= K) break;
-    float x[MJ][8];
-    xs.load(pc + lane * 8, K, x);
-    const uint8_t *pan = slot + p * kBoxBytes + lane * 16;
+  for (int r = 0; r < kRows; ++r) {
+    float wf[8];
+    unpack8(ld_shared_v4(pan + r * (kPanel * 2)), wf);
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      float wf[8];
-      unpack8(ld_shared_v4(pan + r * (kPanel * 2)), wf);
+    for (int j = 0; j < MJ; ++j) {
+      float a = acc[r * MJ + j];
 #pragma unroll
-      for (int j = 0; j < MJ; ++j) {
-        float a = acc[r * MJ + j];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) a = fmaf(wf[k], x[j][k], a);
-        acc[r * MJ + j] = a;
-      }
+      for (int k = 0; k < 8; ++k) a = fmaf(wf[k], x[j][k], a);
+      acc[r * MJ + j] = a;
     }
   }
 }
 
-// Streams `ntiles` tiles of one segment through the ring into acc.
-template <int MJ, int R, int NP, class XS>
-__device__ bool gemv_segment(Warp &w, int op, int ntiles, int K, const XS &xs,
-                             float (&acc)[R * MJ]) {
+// One tile (4 rows x up to four boxes of 256 columns starting at colbase):
+// acc[r*MJ + j] += W[r][cols] . x[j][cols] over this lane's columns.
+template <int MJ, class XS>
+MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], int colbase, int K, const XS &xs,
+                         int lane) {
+  const uint8_t *base = slot + lane * 16;
+  if constexpr (MJ <= 2) {
+    // every panel's activations first: one memory round trip per tile
+    float x[kPanels][MJ][8];
+#pragma unroll
+    for (int p = 0; p < kPanels; ++p) xs.load(colbase + p * kPanel + lane * 8, K, x[p]);
+#pragma unroll
+    for (int p = 0; p < kPanels; ++p)
+      if (colbase + p * kPanel < K) gemv_panel<MJ>(base + p * kBoxBytes, acc, x[p]);
+  } else {
+#pragma unroll
+    for (int p = 0; p < kPanels; ++p) {
+      const int pc = colbase + p * kPanel;
+      if (pc >= K) break;
+      float x[MJ][8];
+      xs.load(pc + lane * 8, K, x);
+      gemv_panel<MJ>(base + p * kBoxBytes, acc, x);
+    }
+  }
+}
+
+// Streams `ntiles` tiles of one unit through the ring into acc (not reduced).
+template <int MJ, class XS>
+MK_INLINE bool gemv_stream(Warp &w, int op, int ntiles, int col0, int K, const XS &xs, float (&acc)[kRows * MJ]) {
+#pragma unroll
+  for (int q = 0; q < kRows * MJ; ++q) acc[q] = 0.f;
   for (int t = 0; t < ntiles; ++t) {
     const uint8_t *slot = consume_begin(w, op);
     if (!slot) return false;
-    gemv_tile<MJ, R, NP>(slot, acc, t * kPanel * NP, K, xs, w.lane);
+    gemv_tile<MJ>(slot, acc, col0 + t * kTileCols, K, xs, w.lane);
     consume_end(w);
   }
   return true;
 }
 
-// inv_rms for rows 0..M-1 from the residual producers' partial sums of squares.
-__device__ void compute_inv_rms(const Warp &w, float *inv) {
-  const Params &P = PP(w);
-  for (int m = 0; m < P.M; ++m) {
-    float s = 0.f;
-    for (int i = w.lane; i < P.n_hb; i += 32) s += __ldcg(&P.ss[m * P.n_hb + i]);
-    s = warp_sum(s);
-    inv[m] = 1.0f / sqrtf(s / static_cast<float>(P.d) + P.eps);
-  }
+// gemv_stream, then the cross-lane reduction: buf[r*MJ + j] = row r . x[j].
+template <int MJ, class XS>
+MK_INLINE bool gemv_unit(Warp &w, int op, int ntiles, int col0, int K, const XS &xs, float *buf) {
+  float acc[kRows * MJ];
+  if (!gemv_stream<MJ>(w, op, ntiles, col0, K, xs, acc)) return false;
+  butterfly<kRows * MJ>(acc, w.lane);
+  butterfly_store<kRows * MJ>(acc, buf, w.lane);
+  __syncwarp();
+  return true;
 }
 
-template <int MMAX>
-struct Cfg {
-  static constexpr int R = (MMAX <= 4) ? 16 : 8;
-  static constexpr int NP = (MMAX <= 4) ? 1 : 2;
-};
+// inv_rms for rows 0..M-1 from the residual producers' partial sums of squares.
+MK_INLINE void compute_inv_rms(const Params &P, int lane, float (&inv)[kMaxRows]) {
+  const int nk = P.ss_ld / 128;  // float4 loads per lane and row (padding is zero)
+#pragma unroll
+  for (int m = 0; m < kMaxRows; ++m) {
+    inv[m] = 0.f;
+    if (m < P.M) {
+      const float4 *row = reinterpret_cast<const float4 *>(P.ss + static_cast<size_t>(m) * P.ss_ld) + lane;
+      float s = 0.f;
+      for (int k0 = 0; k0 < nk; k0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          v[k] = (k0 + k < nk) ? __ldcg(row + 32 * (k0 + k)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s += (v[k].x + v[k].y) + (v[k].z + v[k].w);
+      }
+      s = warp_sum(s);
+      inv[m] = 1.0f / sqrtf(s / static_cast<float>(P.d) + P.eps);
+    }
+  }
+}
 
 // ---------------------------------------------------------------------------
 // Ops
 // ---------------------------------------------------------------------------
-// Residual update of rows [row0, row0+R) from wacc[r*MMAX + m], plus the
-// partial sum of squares of the new values for the next RMSNorm.
-template <int MMAX>
-__device__ void residual_epilogue(Warp &w, int unit, int row0, int dbg_layer) {
-  const Params &P = PP(w);
-  constexpr int R = Cfg<MMAX>::R;
-  for (int e = w.lane; e < R * P.M; e += 32) {
-    int m = e / R, r = e % R, row = row0 + r;
-    float sq = 0.f;
-    if (row < P.d) {
-      float *hp = P.h + static_cast<size_t>(m) * P.d + row;
-      float hn = __ldcg(hp) + w.wacc[r * MMAX + m];
-      __stcg(hp, hn);
-      sq = hn * hn;
-      if (dbg_layer >= 0 && P.dbg_hidden)
-        P.dbg_hidden[(static_cast<size_t>(dbg_layer) * P.max_rows + m) * P.d + row] = hn;
-    }
-    w.wtmp[m * R + r] = sq;
+// New residual rows [row0, row0 + 4): store, the partial sum of squares for
+// the next RMSNorm, and the debug copy.  val(m, row, r) gives the new value.
+// Lane 4m + r holds row r of activation row m.
+static_assert(kRows == 4 && kMaxRows * kRows <= 32, "one lane per (row, residual row)");
+template <class F>
+MK_INLINE void residual_rows(const Params &P, int lane, int unit, int row0, int dbg_layer, F val) {
+  const int m = lane / kRows, r = lane % kRows, row = row0 + r;
+  const bool live = lane < kRows * P.M;
+  float sq = 0.f;
+  if (live && row < P.d) {
+    const float hn = val(m, row, r);
+    __stcg(P.h + static_cast<size_t>(m) * P.d + row, hn);
+    sq = hn * hn;
+    if (dbg_layer >= 0 && P.dbg_hidden)
+      P.dbg_hidden[(static_cast<size_t>(dbg_layer) * P.max_rows + m) * P.d + row] = hn;
   }
-  __syncwarp();
-  if (w.lane < P.M) {
-    float s = 0.f;
-    for (int r = 0; r < R; ++r) s += w.wtmp[w.lane * R + r];
-    __stcg(&P.ss[w.lane * P.n_hb + unit], s);
-  }
+  sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+  if (live && r == 0) __stcg(&P.ss[m * P.ss_ld + unit], sq);
   __syncwarp();
 }
 
-template <int MMAX>
-__device__ void op_embed(Warp &w, int op) {
-  const Params &P = PP(w);
-  constexpr int R = Cfg<MMAX>::R;
-  const int n = my_unit_count(w, op, P.n_hb), u0 = first_unit(w, op);
-  for (int i = 0; i < n; ++i) {
-    const int unit = u0 + i * w.nw, row0 = unit * R;
-    for (int e = w.lane; e < R * P.M; e += 32) {
-      int m = e / R, r = e % R, row = row0 + r;
-      float sq = 0.f;
-      if (row < P.d) {
-        int tok = __ldcg(&P.tokens[m]);  // may alias the argmax output
-        if (tok < 0 || tok >= P.V) tok = 0;  // rejected at kernel start
-        float v = __bfloat162float(P.embed[static_cast<size_t>(tok) * P.d + row]);
-        __stcg(&P.h[static_cast<size_t>(m) * P.d + row], v);
-        if (P.dbg_hidden) P.dbg_hidden[static_cast<size_t>(m) * P.d + row] = v;  // layer slot 0
-        sq = v * v;
-      }
-      w.wtmp[m * R + r] = sq;
-    }
-    __syncwarp();
-    if (w.lane < P.M) {
-      float s = 0.f;
-      for (int r = 0; r < R; ++r) s += w.wtmp[w.lane * R + r];
-      __stcg(&P.ss[w.lane * P.n_hb + unit], s);
-    }
-    __syncwarp();
+MK_INLINE void op_embed(Warp &w) {
+  const Params &P = *w.P;
+  for (int unit = w.slot; unit < P.n_hb; unit += w.nw) {
+    residual_rows(P, w.lane, unit, unit * kRows, 0, [&](int m, int row, int) {
+      int tok = __ldcg(&P.tokens[m]);       // may alias the argmax output
+      if (tok < 0 || tok >= P.V) tok = 0;  // rejected at kernel start
+      return __bfloat162float(P.embed[static_cast<size_t>(tok) * P.d + row]);
+    });
   }
 }
 
-// Dense GEMV ops over all M rows: QKV, OPROJ, ROUTER, SHARED_GU, LMHEAD.
-template <int MMAX>
-__device__ bool op_dense(Warp &w, int op, int type, int layer, float &am_val, int &am_idx) {
-  const Params &P = PP(w);
-  constexpr int R = Cfg<MMAX>::R, NP = Cfg<MMAX>::NP, MJ = MMAX;
-  const int total = op_total_units(w, type, layer);
-  const int n = my_unit_count(w, op, total), u0 = first_unit(w, op);
-  if (n == 0) return true;
-  float inv[kMaxRows];
-  if (type != OP_OPROJ) compute_inv_rms(w, inv);
-  const __nv_bfloat16 *g = (type == OP_QKV)      ? P.norms[2 * layer]
-                           : (type == OP_LMHEAD) ? P.final_norm
-                                                 : P.norms[2 * layer + 1];
-  XNorm<MJ> xn;
-  XPlain<MJ> xp;
-  xn.h = P.h; xn.d = P.d; xn.g = g; xn.n = P.M;
-  xp.src = P.o; xp.ld = P.Hq * P.hd; xp.n = P.M;
+// h += (sum_s w_s y_s) + shared, in the selection order of each row.
+MK_INLINE void op_combine(Warp &w, int layer) {
+  const Params &P = *w.P;
+  const int S = P.topk + 1;
+  const Routing *rt = P.routing + layer;
+  for (int unit = w.slot; unit < P.n_hb; unit += w.nw) {
+    residual_rows(P, w.lane, unit, unit * kRows, layer + 1, [&](int m, int row, int) {
+      const float *yp = P.y_part + (static_cast<size_t>(m) * S) * P.d + row;
+      float moe = 0.f;
 #pragma unroll
-  for (int j = 0; j < MJ; ++j) {
-    xn.row[j] = j < P.M ? j : 0;
-    xn.inv[j] = (j < P.M && type != OP_OPROJ) ? inv[j] : 0.f;
-    xp.row[j] = j < P.M ? j : 0;
+      for (int s = 0; s < kMaxTopK; ++s)
+        if (s < P.topk) moe += __ldcg(&rt->row_w[m][s]) * __ldcg(yp + static_cast<size_t>(s) * P.d);
+      const float sh = P.Fs > 0 ? __ldcg(yp + static_cast<size_t>(P.topk) * P.d) : 0.f;
+      return __ldcg(P.h + static_cast<size_t>(m) * P.d + row) + (moe + sh);
+    });
   }
-  const int TC = R == 16 ? 256 : 512;
-  for (int i = 0; i < n; ++i) {
-    const int unit = u0 + i * w.nw;
-    float acc[R * MJ];
-#pragma unroll
-    for (int q = 0; q < R * MJ; ++q) acc[q] = 0.f;
-    int row0 = unit * R, N = 0;
-    bool ok;
-    if (type == OP_OPROJ) {
-      ok = gemv_segment<MJ, R, NP>(w, op, cdiv(P.Hq * P.hd, TC), P.Hq * P.hd, xp, acc);
-      N = P.d;
-    } else if (type == OP_ROUTER) {
-      const int nrb = cdiv(P.E, R), kc = unit / nrb;
-      row0 = (unit % nrb) * R;
-      // one tile of columns [kc*TC, kc*TC + TC): shift the activation source
-      const uint8_t *slot = consume_begin(w, op);
-      ok = slot != nullptr;
-      if (ok) {
-        gemv_tile<MJ, R, NP>(slot, acc, kc * TC, P.d, xn, w.lane);
-        consume_end(w);
-      }
-      N = P.E;
-    } else {
-      ok = gemv_segment<MJ, R, NP>(w, op, cdiv(P.d, TC), P.d, xn, acc);
-      N = (type == OP_QKV) ? (P.Hq + 2 * P.Hkv) * P.hd
-          : (type == OP_SHARED_GU) ? 2 * P.Fs
-                                   : P.V;
-    }
-    if (!ok) return false;
-    butterfly<R * MJ>(acc, w.lane);
-    butterfly_store<R * MJ>(acc, w.wbuf, w.lane);
-    __syncwarp();
-    switch (type) {
-      case OP_QKV: {
-        const int W3 = (P.Hq + 2 * P.Hkv) * P.hd;
-        for (int e = w.lane; e < R * P.M; e += 32) {
-          int m = e / R, r = e % R;
-          if (row0 + r < N) __stcg(&P.qkv[static_cast<size_t>(m) * W3 + row0 + r], w.wbuf[r * MJ + m]);
-        }
-        break;
-      }
-      case OP_SHARED_GU:
-        for (int e = w.lane; e < R * P.M; e += 32) {
-          int m = e / R, r = e % R;
-          if (row0 + r < N)
-            __stcg(&P.gu_shared[static_cast<size_t>(m) * 2 * P.Fs + row0 + r], w.wbuf[r * MJ + m]);
-        }
-        break;
-      case OP_ROUTER: {
-        const int kc = unit / cdiv(P.E, R);
-        for (int e = w.lane; e < R * P.M; e += 32) {
-          int m = e / R, r = e % R;
-          if (row0 + r < N)
-            __stcg(&P.router_part[(static_cast<size_t>(kc) * kMaxRows + m) * P.E + row0 + r],
-                   w.wbuf[r * MJ + m]);
-        }
-        break;
-      }
-      case OP_LMHEAD: {
-        for (int e = w.lane; e < R * P.M; e += 32) {
-          int m = e / R, r = e % R;
-          if (row0 + r < N) P.logits[static_cast<size_t>(m) * P.V + row0 + r] = w.wbuf[r * MJ + m];
-        }
-        if (w.lane < P.M) {
-          for (int r = 0; r < R && row0 + r < N; ++r) {
-            float v = w.wbuf[r * MJ + w.lane];
-            if (v > am_val) {
-              am_val = v;
-              am_idx = row0 + r;
-            }
-          }
-        }
-        break;
-      }
-      case OP_OPROJ: {
-        for (int e = w.lane; e < R * MMAX; e += 32) {
-          int r = e / MMAX, m = e % MMAX;
-          w.wacc[r * MMAX + m] = w.wbuf[r * MJ + m];
-        }
-        __syncwarp();
-        residual_epilogue<MMAX>(w, unit, row0, -1);
-        break;
-      }
-      default: break;
-    }
-    __syncwarp();
-  }
-  return true;
 }
 
-// Routed gate/up rows for every expert in the union (rows of that expert only).
-template <int MMAX, int MJ>
-__device__ bool routed_gu_unit(Warp &w, int op, int layer, int unit, const float *inv) {
-  const Params &P = PP(w);
-  constexpr int R = Cfg<MMAX>::R, NP = Cfg<MMAX>::NP, TC = R == 16 ? 256 : 512;
-  const int nrb = (2 * P.F) / R, j = unit / nrb, row0 = (unit % nrb) * R;
-  const uint32_t mask = __ldcg(&P.routing[layer].rowmask[j]);
-  XNorm<MJ> xn;
-  xn.h = P.h; xn.d = P.d; xn.g = P.norms[2 * layer + 1];
+template <int MJ>
+MK_INLINE void fill_all_rows(int (&row)[MJ], int M) {
+#pragma unroll
+  for (int j = 0; j < MJ; ++j) row[j] = j < M ? j : 0;
+}
+
+// Rows of a routed expert: row[q] = q-th row in `mask`; returns the count.
+template <int MJ>
+MK_INLINE int rows_of_mask(uint32_t mask, int (&row)[MJ]) {
   int n = 0;
 #pragma unroll
-  for (int q = 0; q < MJ; ++q) { xn.row[q] = 0; xn.inv[q] = 0.f; }
-  for (int m = 0; m < P.M; ++m) {
+  for (int q = 0; q < MJ; ++q) row[q] = 0;
+#pragma unroll
+  for (int m = 0; m < kMaxRows; ++m) {
     if (mask & (1u << m)) {
 #pragma unroll
       for (int q = 0; q < MJ; ++q)
-        if (q == n) { xn.row[q] = m; xn.inv[q] = inv[m]; }
+        if (q == n) row[q] = m;
       ++n;
     }
   }
-  xn.n = n;
-  float acc[R * MJ];
-#pragma unroll
-  for (int q = 0; q < R * MJ; ++q) acc[q] = 0.f;
-  if (!gemv_segment<MJ, R, NP>(w, op, cdiv(P.d, TC), P.d, xn, acc)) return false;
-  butterfly<R * MJ>(acc, w.lane);
-  butterfly_store<R * MJ>(acc, w.wbuf, w.lane);
-  __syncwarp();
-  const size_t ld = 2 * static_cast<size_t>(P.F);
-  for (int e = w.lane; e < R * n; e += 32) {
-    int q = e / R, r = e % R;
-    int m = 0;
-#pragma unroll
-    for (int qq = 0; qq < MJ; ++qq)
-      if (qq == q) m = xn.row[qq];
-    __stcg(&P.gu_routed[(static_cast<size_t>(j) * kMaxRows + m) * ld + row0 + r], w.wbuf[r * MJ + q]);
-  }
-  __syncwarp();
-  return true;
+  return n;
 }
 
-template <int MMAX>
-__device__ bool op_routed_gu(Warp &w, int op, int layer) {
-  const Params &P = PP(w);
-  const int total = op_total_units(w, OP_ROUTED_GU, layer);
-  const int n = my_unit_count(w, op, total), u0 = first_unit(w, op);
-  if (n == 0) return true;
-  float inv[kMaxRows];
-  compute_inv_rms(w, inv);
-  const int nrb = (2 * P.F) / Cfg<MMAX>::R;
-  for (int i = 0; i < n; ++i) {
-    const int unit = u0 + i * w.nw;
-    const uint32_t mask = __ldcg(&P.routing[layer].rowmask[unit / nrb]);
-    const int cnt = __popc(mask);
-    bool ok;
-    if (cnt <= 1) ok = routed_gu_unit<MMAX, 1>(w, op, layer, unit, inv);
-    else if (cnt <= 2) ok = routed_gu_unit<MMAX, (MMAX >= 2 ? 2 : 1)>(w, op, layer, unit, inv);
-    else if (cnt <= 4) ok = routed_gu_unit<MMAX, (MMAX >= 4 ? 4 : 1)>(w, op, layer, unit, inv);
-    else ok = routed_gu_unit<MMAX, (MMAX >= 8 ? 8 : 1)>(w, op, layer, unit, inv);
-    if (!ok) return false;
-  }
-  return true;
+template <int MJ>
+MK_INLINE int row_at(const int (&row)[MJ], int q) {
+  int m = 0;
+#pragma unroll
+  for (int qq = 0; qq < MJ; ++qq)
+    if (qq == q) m = row[qq];
+  return m;
 }
 
-// One down-projection segment (routed expert j, or the shared expert when
-// j < 0) for rows [row0, row0+R): wacc[r][m] += weight(m) * (Wd[row] . act[m]).
-template <int MMAX, int MJ>
-__device__ bool down_segment(Warp &w, int op, int layer, int j, int row0) {
-  const Params &P = PP(w);
-  constexpr int R = Cfg<MMAX>::R, NP = Cfg<MMAX>::NP, TC = R == 16 ? 256 : 512;
-  XSwiGLU<MJ> xs;
-  float wt[MJ];
-  int n = 0;
-#pragma unroll
-  for (int q = 0; q < MJ; ++q) { xs.row[q] = 0; wt[q] = 0.f; }
-  int K;
-  if (j >= 0) {
-    const uint32_t mask = __ldcg(&P.routing[layer].rowmask[j]);
-    xs.gu = P.gu_routed + static_cast<size_t>(j) * kMaxRows * 2 * P.F;
-    xs.ld = 2 * P.F;
-    xs.F = P.F;
-    K = P.F;
-    for (int m = 0; m < P.M; ++m) {
-      if (mask & (1u << m)) {
-        float wm = __ldcg(&P.routing[layer].weight[j][m]);
-#pragma unroll
-        for (int q = 0; q < MJ; ++q)
-          if (q == n) { xs.row[q] = m; wt[q] = wm; }
-        ++n;
-      }
-    }
+// Dense activations of an op: from the CTA's shared-memory copy (batch 1) or
+// from global memory through L1 (more rows).
+template <int MJ, bool XS, class Body>
+MK_INLINE bool with_dense_x(Warp &w, int type, int layer, const float *xs, Body body) {
+  const Params &P = *w.P;
+  if constexpr (XS) {
+    XSmem x;
+    x.xs = xs;
+    return body(x);
+  } else if (type == OP_OPROJ) {
+    XPlain<MJ> xp;
+    xp.src = P.o;
+    xp.ld = P.Hq * P.hd;
+    xp.n = P.M;
+    fill_all_rows<MJ>(xp.row, P.M);
+    return body(xp);
   } else {
-    xs.gu = P.gu_shared;
-    xs.ld = 2 * P.Fs;
-    xs.F = P.Fs;
-    K = P.Fs;
-    for (int m = 0; m < P.M; ++m) {
-#pragma unroll
-      for (int q = 0; q < MJ; ++q)
-        if (q == m) { xs.row[q] = m; wt[q] = 1.f; }
+    XNorm<MJ> xn;
+    xn.h = P.h;
+    xn.d = P.d;
+    xn.n = P.M;
+    xn.g = (type == OP_QKV) ? P.norms[2 * layer] : (type == OP_LMHEAD) ? P.final_norm : P.norms[2 * layer + 1];
+    fill_all_rows<MJ>(xn.row, P.M);
+    return body(xn);
+  }
+}
+
+// One unit of a dense GEMV op over all M rows (QKV, OPROJ, ROUTER, LMHEAD).
+template <int MMAX, bool XS>
+MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const float (&inv)[kMaxRows],
+                          const float *xs, float &am_val, int &am_idx) {
+  const Params &P = *w.P;
+  constexpr int MJ = MMAX;
+  float *wb = w.wbuf;
+  int row0 = unit * kRows, N = 0, col0 = 0, ntiles = 0, K = P.d;
+  switch (type) {
+    case OP_OPROJ: K = P.Hq * P.hd; ntiles = cdiv(K, kTileCols); N = P.d; break;
+    case OP_ROUTER: {
+      const int nrb = cdiv(P.E, kRows);
+      row0 = (unit % nrb) * kRows;
+      col0 = (unit / nrb) * kTileCols;
+      ntiles = 1;
+      N = P.E;
+      break;
     }
-    n = P.M;
+    case OP_QKV: ntiles = cdiv(P.d, kTileCols); N = (P.Hq + 2 * P.Hkv) * P.hd; break;
+    default: ntiles = cdiv(P.d, kTileCols); N = P.V; break;
   }
-  xs.n = n;
-  float acc[R * MJ];
+  const bool ok = with_dense_x<MJ, XS>(w, type, layer, xs, [&](const auto &x) {
+    return gemv_unit<MJ>(w, op, ntiles, col0, K, x, wb);
+  });
+  if (!ok) return false;
+  // lane 4m + r owns output (row0 + r, m); normed ops scale by inv_rms here
+  const int m = w.lane / kRows, r = w.lane % kRows;
+  const bool live = w.lane < kRows * P.M && row0 + r < N;
+  float im = 1.f;
 #pragma unroll
-  for (int q = 0; q < R * MJ; ++q) acc[q] = 0.f;
-  if (!gemv_segment<MJ, R, NP>(w, op, cdiv(K, TC), K, xs, acc)) return false;
-  butterfly<R * MJ>(acc, w.lane);
-  butterfly_store<R * MJ>(acc, w.wbuf, w.lane);
-  __syncwarp();
-  for (int e = w.lane; e < R * n; e += 32) {
-    int q = e / R, r = e % R;
-    int m = 0;
-    float wm = 0.f;
+  for (int mm = 0; mm < kMaxRows; ++mm)
+    if (mm == m) im = inv[mm];
+  switch (type) {
+    case OP_QKV:
+      if (live)
+        __stcg(&P.qkv[static_cast<size_t>(m) * (P.Hq + 2 * P.Hkv) * P.hd + row0 + r], im * wb[r * MJ + m]);
+      break;
+    case OP_ROUTER:
+      if (live)
+        __stcg(&P.router_part[(static_cast<size_t>(unit / cdiv(P.E, kRows)) * kMaxRows + m) * P.e_ld + row0 + r],
+               im * wb[r * MJ + m]);
+      break;
+    case OP_LMHEAD: {
+      const float v = im * wb[r * MJ + m];
+      if (live) P.logits[static_cast<size_t>(m) * P.V + row0 + r] = v;
+      // running argmax of row m over this warp's rows; lanes 4m..4m+3 hold
+      // consecutive rows, so reduce them in row order before lane 4m keeps it
+      float bv = live ? v : -INFINITY;
+      int bi = live ? row0 + r : 0x7fffffff;
 #pragma unroll
-    for (int qq = 0; qq < MJ; ++qq)
-      if (qq == q) { m = xs.row[qq]; wm = wt[qq]; }
-    w.wacc[r * MMAX + m] += wm * w.wbuf[r * MJ + q];
+      for (int o = 1; o < kRows; o <<= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (r == 0 && (bv > am_val || (bv == am_val && bi < am_idx))) {
+        am_val = bv;
+        am_idx = bi;
+      }
+      break;
+    }
+    case OP_OPROJ:
+      residual_rows(P, w.lane, unit, row0, -1, [&](int mm, int row, int rr) {
+        return __ldca(P.h + static_cast<size_t>(mm) * P.d + row) + wb[rr * MJ + mm];
+      });
+      break;
+    default: break;
   }
   __syncwarp();
-  (void)row0;
   return true;
 }
 
-template <int MMAX>
-__device__ bool op_down(Warp &w, int op, int layer) {
-  const Params &P = PP(w);
-  constexpr int R = Cfg<MMAX>::R;
-  const int n = my_unit_count(w, op, P.n_hb), u0 = first_unit(w, op);
-  if (n == 0) return true;
-  const int U = n_union(w, layer);
-  for (int i = 0; i < n; ++i) {
-    const int unit = u0 + i * w.nw, row0 = unit * R;
-    for (int e = w.lane; e < R * MMAX; e += 32) w.wacc[e] = 0.f;
-    __syncwarp();
-    for (int j = 0; j < U; ++j) {
-      const int cnt = __popc(__ldcg(&P.routing[layer].rowmask[j]));
-      bool ok;
-      if (cnt <= 1) ok = down_segment<MMAX, 1>(w, op, layer, j, row0);
-      else if (cnt <= 2) ok = down_segment<MMAX, (MMAX >= 2 ? 2 : 1)>(w, op, layer, j, row0);
-      else if (cnt <= 4) ok = down_segment<MMAX, (MMAX >= 4 ? 4 : 1)>(w, op, layer, j, row0);
-      else ok = down_segment<MMAX, (MMAX >= 8 ? 8 : 1)>(w, op, layer, j, row0);
-      if (!ok) return false;
-    }
-    if (P.Fs > 0) {
-      if (!down_segment<MMAX, MMAX>(w, op, layer, -1, row0)) return false;
-    }
-    residual_epilogue<MMAX>(w, unit, row0, layer + 1);
+// Gate/up unit: 4 rows of the expert's gate and up projections for the rows
+// routed to it (shared expert: all rows); writes act = silu(gate) * up.
+template <int MJ, bool XS>
+MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const float (&inv)[kMaxRows],
+                       const float *xs) {
+  const Params &P = *w.P;
+  XNorm<MJ> xn;
+  xn.h = P.h;
+  xn.d = P.d;
+  xn.g = P.norms[2 * layer + 1];
+  float *dst;
+  int ld, f0;
+  if (type == OP_ROUTED_GU) {
+    const int nfb = P.F / kRows, j = unit / nfb;
+    f0 = (unit % nfb) * kRows;
+    xn.n = rows_of_mask<MJ>(__ldcg(&P.routing[layer].rowmask[j]), xn.row);
+    dst = P.act_routed + static_cast<size_t>(j) * kMaxRows * P.F;
+    ld = P.F;
+  } else {
+    f0 = unit * kRows;
+    xn.n = P.M;
+    fill_all_rows<MJ>(xn.row, P.M);
+    dst = P.act_shared;
+    ld = P.Fs;
   }
+  const int half = cdiv(P.d, kTileCols);
+  float *wb = w.wbuf;
+  if constexpr (XS) {
+    XSmem x;
+    x.xs = xs;
+    if (!gemv_unit<MJ>(w, op, half, 0, P.d, x, wb)) return false;
+    if (!gemv_unit<MJ>(w, op, half, 0, P.d, x, wb + kRows * MJ)) return false;
+  } else {
+    if (!gemv_unit<MJ>(w, op, half, 0, P.d, xn, wb)) return false;
+    if (!gemv_unit<MJ>(w, op, half, 0, P.d, xn, wb + kRows * MJ)) return false;
+  }
+  const int q = w.lane / kRows, r = w.lane % kRows;
+  if (w.lane < kRows * xn.n) {
+    const int m = row_at<MJ>(xn.row, q);
+    float im = 0.f;
+#pragma unroll
+    for (int mm = 0; mm < kMaxRows; ++mm)
+      if (mm == m) im = inv[mm];
+    const float g = im * wb[r * MJ + q], u = im * wb[kRows * MJ + r * MJ + q];
+    __stcg(dst + static_cast<size_t>(m) * ld + f0 + r, silu(g) * u);
+  }
+  __syncwarp();
   return true;
+}
+
+// One down-projection unit: segment (routed expert j, or the shared expert
+// when j == n_union) x 4 output rows; writes the partial of every row m it
+// serves to y_part[m][slot][row] (slot = selection index, or top_k).
+template <int MJ>
+MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit) {
+  const Params &P = *w.P;
+  const int seg = unit / P.n_hb, row0 = (unit % P.n_hb) * kRows;
+  const int U = n_union(P, layer);
+  const Routing *rt = P.routing + layer;
+  XPlain<MJ> xs;
+  int K;
+  if (seg < U) {
+    xs.src = P.act_routed + static_cast<size_t>(seg) * kMaxRows * P.F;
+    xs.ld = P.F;
+    xs.n = rows_of_mask<MJ>(__ldcg(&rt->rowmask[seg]), xs.row);
+    K = P.F;
+  } else {
+    xs.src = P.act_shared;
+    xs.ld = P.Fs;
+    xs.n = P.M;
+    fill_all_rows<MJ>(xs.row, P.M);
+    K = P.Fs;
+  }
+  float *wb = w.wbuf;
+  if (!gemv_unit<MJ>(w, op, cdiv(K, kTileCols), 0, K, xs, wb)) return false;
+  const int q = w.lane / kRows, r = w.lane % kRows;
+  if (w.lane < kRows * xs.n && row0 + r < P.d) {
+    const int m = row_at<MJ>(xs.row, q);
+    const int s = (seg < U) ? static_cast<int>(__ldcg(&rt->kslot[seg][m])) : P.topk;
+    __stcg(&P.y_part[(static_cast<size_t>(m) * (P.topk + 1) + s) * P.d + row0 + r], wb[r * MJ + q]);
+  }
+  __syncwarp();
+  return true;
+}
+
+template <int MMAX, bool XS>
+MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, const float (&inv)[kMaxRows],
+                               const float *xs) {
+  const Params &P = *w.P;
+  int cnt;
+  if (type == OP_ROUTED_GU) {
+    cnt = __popc(__ldcg(&P.routing[layer].rowmask[unit / (P.F / kRows)]));
+  } else if (type == OP_DOWN) {
+    const int seg = unit / P.n_hb;
+    cnt = seg < n_union(P, layer) ? __popc(__ldcg(&P.routing[layer].rowmask[seg])) : P.M;
+  } else {
+    cnt = P.M;  // shared gate/up
+  }
+#define MK_DISPATCH(MJ_)                                      \
+  return (type == OP_DOWN) ? down_unit<MJ_>(w, op, layer, unit) \
+                           : gu_unit<MJ_, XS>(w, op, type, layer, unit, inv, xs)
+  if (cnt <= 1) {
+    MK_DISPATCH(1);
+  }
+  if constexpr (MMAX >= 2) {
+    if (cnt <= 2) {
+      MK_DISPATCH(2);
+    }
+  }
+  if constexpr (MMAX >= 4) {
+    if (cnt <= 4) {
+      MK_DISPATCH(4);
+    }
+  }
+  if constexpr (MMAX >= 8) {
+    MK_DISPATCH(8);
+  }
+#undef MK_DISPATCH
+  return false;
 }
 
 // --- attention ---------------------------------------------------------------
 template <int QVP, int DPL>
-__device__ bool attn_item_run(Warp &w, int op, int layer, int item) {
-  const Params &P = PP(w);
+MK_INLINE bool attn_item_run(Warp &w, int op, int layer, const AttnItem &a) {
+  const Params &P = *w.P;
   constexpr int PG = 32 / QVP;  // positions per butterfly group
   constexpr int hd = 32 * DPL, half = hd / 2;
   const int G = P.Hq / P.Hkv;
-  const AttnItem a = attn_item(w, item);
   const int pos_b = __ldg(&P.positions[a.b]);
   const int W3 = (P.Hq + 2 * P.Hkv) * hd;
   const float scale = 1.0f / sqrtf(static_cast<float>(hd));
+  const int lane = w.lane, ppos = lane & 15;
   // query vectors of this item: qv = qs*QVP + v  ->  (t = qv / G, head = g*G + qv % G)
   float q[QVP][DPL];
   int lim[QVP];
-  const int lane = w.lane, ppos = lane & 15;
 #pragma unroll
   for (int v = 0; v < QVP; ++v) {
     const int qv = a.qs * QVP + v;
@@ -1063,15 +1046,12 @@ __device__ bool attn_item_run(Warp &w, int op, int layer, int item) {
       const float *src = P.qkv + static_cast<size_t>(m) * W3 + head * hd + lane * DPL;
 #pragma unroll
       for (int dd = 0; dd < DPL; ++dd) {
-        float own = __ldcg(src + dd);
-        float other = __shfl_xor_sync(0xffffffffu, own, 16);
-        float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
-        float r = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
-        q[v][dd] = r * scale;
+        const float own = __ldcg(src + dd);
+        const float other = __shfl_xor_sync(0xffffffffu, own, 16);
+        const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
+        const float rr = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
+        q[v][dd] = rr * scale;
       }
-    } else {
-#pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) (void)__shfl_xor_sync(0xffffffffu, 0.f, 16);
     }
   }
   float m_run = -INFINITY, l_run = 0.f;
@@ -1081,6 +1061,10 @@ __device__ bool attn_item_run(Warp &w, int op, int layer, int item) {
 #pragma unroll
     for (int dd = 0; dd < DPL; ++dd) o[v][dd] = 0.f;
   const int my_qv = lane % QVP;
+  int my_lim = -1;
+#pragma unroll
+  for (int v = 0; v < QVP; ++v)
+    if (v == my_qv) my_lim = lim[v];
   const size_t cache_row_base =
       (static_cast<size_t>(layer) * P.Bmax + a.b) * P.Hkv * P.cap + static_cast<size_t>(a.g) * P.cap;
   for (int tt = 0; tt < a.ntiles; ++tt) {
@@ -1088,23 +1072,22 @@ __device__ bool attn_item_run(Warp &w, int op, int layer, int item) {
     if (!slot) return false;
     const int pos0 = a.pos0 + tt * P.attn_ppt;
     __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(slot);
-    __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(slot + kBoxBytes);
+    __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(slot + kKvBoxBytes);
     // New positions of this step inside the tile: rotate k, round k and v to
     // bf16, patch the tile and (once per chunk) append them to the cache.
     const int lo = max(pos0, pos_b), hi = min(pos0 + P.attn_ppt, pos_b + P.T);
-    bool patched = false;
     for (int p = lo; p < hi; ++p) {
       const int t = p - pos_b, m = a.b * P.T + t;
       const float *kq = P.qkv + static_cast<size_t>(m) * W3 + (P.Hq + a.g) * hd + lane * DPL;
       const float *vq = P.qkv + static_cast<size_t>(m) * W3 + (P.Hq + P.Hkv + a.g) * hd + lane * DPL;
 #pragma unroll
       for (int dd = 0; dd < DPL; ++dd) {
-        float own = __ldcg(kq + dd);
-        float other = __shfl_xor_sync(0xffffffffu, own, 16);
-        float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
-        float kr = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
-        __nv_bfloat16 kb = __float2bfloat16_rn(kr);
-        __nv_bfloat16 vb = __float2bfloat16_rn(__ldcg(vq + dd));
+        const float own = __ldcg(kq + dd);
+        const float other = __shfl_xor_sync(0xffffffffu, own, 16);
+        const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
+        const float kr = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
+        const __nv_bfloat16 kb = __float2bfloat16_rn(kr);
+        const __nv_bfloat16 vb = __float2bfloat16_rn(__ldcg(vq + dd));
         ks[(p - pos0) * hd + lane * DPL + dd] = kb;
         vs[(p - pos0) * hd + lane * DPL + dd] = vb;
         if (a.qs == 0) {
@@ -1112,9 +1095,8 @@ __device__ bool attn_item_run(Warp &w, int op, int layer, int item) {
           P.vc[(cache_row_base + p) * hd + lane * DPL + dd] = vb;
         }
       }
-      patched = true;
     }
-    if (patched) fence_proxy_async_smem();
+    if (lo < hi) fence_proxy_async_smem();
     __syncwarp();
     for (int jg = 0; jg < P.attn_ppt; jg += PG) {
       float part[32];
@@ -1135,12 +1117,8 @@ __device__ bool attn_item_run(Warp &w, int op, int layer, int item) {
       butterfly<32>(part, lane);
       // lane holds the score of position jg + lane / QVP for query lane % QVP
       const int pos = pos0 + jg + lane / QVP;
-      int my_lim = -1;
-#pragma unroll
-      for (int v = 0; v < QVP; ++v)
-        if (v == my_qv) my_lim = lim[v];
       const bool valid = (pos <= my_lim) && (pos < a.pos0 + a.npos);
-      float s = valid ? part[0] : -INFINITY;
+      const float s = valid ? part[0] : -INFINITY;
       float mx = s;
 #pragma unroll
       for (int o2 = QVP; o2 < 32; o2 <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
@@ -1180,146 +1158,180 @@ __device__ bool attn_item_run(Warp &w, int op, int layer, int item) {
 #pragma unroll
   for (int v = 0; v < QVP; ++v)
 #pragma unroll
-    for (int dd = 0; dd < DPL; ++dd)
-      __stcg(&P.attn_o[(pidx * QVP + v) * hd + lane * DPL + dd], o[v][dd]);
+    for (int dd = 0; dd < DPL; ++dd) __stcg(&P.attn_o[(pidx * QVP + v) * hd + lane * DPL + dd], o[v][dd]);
   if (lane < QVP) {
-    __stcg(&P.attn_ml[(static_cast<size_t>(grp) * QVP + lane) * 2 * P.attn_nch_max + a.c], m_run);
-    __stcg(&P.attn_ml[(static_cast<size_t>(grp) * QVP + lane) * 2 * P.attn_nch_max + P.attn_nch_max + a.c],
-           l_run);
+    float *ml = P.attn_ml + (static_cast<size_t>(grp) * QVP + lane) * 2 * P.attn_nch_max;
+    __stcg(ml + a.c, m_run);
+    __stcg(ml + P.attn_nch_max + a.c, l_run);
   }
   return true;
 }
 
-// Merge n partials (m_i, l_i, o_i) of each query vector: level 1 keeps the
-// unnormalised (max, sum, weighted o); level 2 writes o / l.
+// Merge n (<= 16) partials (m_i, l_i, o_i) of each query vector: level 1
+// keeps the unnormalised (max, sum, weighted o); level 2 writes o / l.
 template <int QVP, int DPL>
-__device__ void attn_merge(Warp &w, int grp, int first, int n, int nstride, const float *src_o,
-                           const float *src_ml, float *dst_o, float *dst_ml, int dst_index,
-                           int dst_stride, bool final_level, int b, int g) {
-  const Params &P = PP(w);
+__device__ __noinline__ void attn_merge(const Params &P, int lane, int grp, int first, int n, int nstride,
+                                        const float *src_o, const float *src_ml, float *dst_o, float *dst_ml,
+                                        int dst_index, int dst_stride, bool final_level, int b, int g) {
   constexpr int hd = 32 * DPL;
-  const int lane = w.lane, G = P.Hq / P.Hkv;
+  const int G = P.Hq / P.Hkv;
+  float mi[QVP], li[QVP];
+#pragma unroll
   for (int v = 0; v < QVP; ++v) {
     const float *mrow = src_ml + (static_cast<size_t>(grp) * QVP + v) * 2 * nstride;
-    float mi = -INFINITY, li = 0.f;
-    if (lane < n) {
-      mi = __ldcg(mrow + first + lane);
-      li = __ldcg(mrow + nstride + first + lane);
-    }
-    const float M = warp_max(mi);
-    const float wi = (lane < n && mi != -INFINITY) ? expf(mi - M) : 0.f;
-    const float L = warp_sum(wi * li);
-    float acc[DPL];
+    mi[v] = lane < n ? __ldcg(mrow + first + lane) : -INFINITY;
+    li[v] = lane < n ? __ldcg(mrow + nstride + first + lane) : 0.f;
+  }
+#pragma unroll 1
+  for (int v2 = 0; v2 < QVP; v2 += 2) {
+    // two query vectors per pass: all their partial loads are in flight together
+    float val[2][kL1Fan][DPL];
 #pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const float wv = __shfl_sync(0xffffffffu, wi, i);
-      const float *op = src_o + ((static_cast<size_t>(grp) * nstride + first + i) * QVP + v) * hd + lane * DPL;
+    for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(wv, __ldcg(op + dd), acc[dd]);
-    }
-    if (!final_level) {
-      float *dop = dst_o + ((static_cast<size_t>(grp) * dst_stride + dst_index) * QVP + v) * hd + lane * DPL;
+      for (int i = 0; i < kL1Fan; ++i) {
+        const float *op = src_o + ((static_cast<size_t>(grp) * nstride + first + i) * QVP + v2 + h2) * hd + lane * DPL;
 #pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) __stcg(dop + dd, acc[dd]);
-      if (lane == 0) {
-        float *dml = dst_ml + (static_cast<size_t>(grp) * QVP + v) * 2 * dst_stride;
-        __stcg(dml + dst_index, M);
-        __stcg(dml + dst_stride + dst_index, L);
+        for (int dd = 0; dd < DPL; ++dd) val[h2][i][dd] = (i < n) ? __ldcg(op + dd) : 0.f;
       }
-    } else {
-      const int qv = (grp % P.attn_qsplit) * QVP + v;
-      if (qv < G * P.T) {
-        const int t = qv / G, head = g * G + qv % G, m = b * P.T + t;
-        const float invl = 1.0f / L;
-        float *dst = P.o + static_cast<size_t>(m) * P.Hq * hd + head * hd + lane * DPL;
 #pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) __stcg(dst + dd, acc[dd] * invl);
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int v = v2 + h2;
+      float mv = -INFINITY, lv = 0.f;
+#pragma unroll
+      for (int vv = 0; vv < QVP; ++vv)
+        if (vv == v) {
+          mv = mi[vv];
+          lv = li[vv];
+        }
+      const float M = warp_max(mv);
+      const float wi = (lane < n && mv != -INFINITY) ? expf(mv - M) : 0.f;
+      const float L = warp_sum(wi * lv);
+      float acc[DPL];
+#pragma unroll
+      for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kL1Fan; ++i) {
+        const float wv = __shfl_sync(0xffffffffu, wi, i);
+#pragma unroll
+        for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(wv, val[h2][i][dd], acc[dd]);
+      }
+      if (!final_level) {
+        float *dop = dst_o + ((static_cast<size_t>(grp) * dst_stride + dst_index) * QVP + v) * hd + lane * DPL;
+#pragma unroll
+        for (int dd = 0; dd < DPL; ++dd) __stcg(dop + dd, acc[dd]);
+        if (lane == 0) {
+          float *dml = dst_ml + (static_cast<size_t>(grp) * QVP + v) * 2 * dst_stride;
+          __stcg(dml + dst_index, M);
+          __stcg(dml + dst_stride + dst_index, L);
+        }
+      } else {
+        const int qv = (grp % P.attn_qsplit) * QVP + v;
+        if (qv < G * P.T) {
+          const int t = qv / G, head = g * G + qv % G, m = b * P.T + t;
+          const float invl = 1.0f / L;
+          float *dst = P.o + static_cast<size_t>(m) * P.Hq * hd + head * hd + lane * DPL;
+#pragma unroll
+          for (int dd = 0; dd < DPL; ++dd) __stcg(dst + dd, acc[dd] * invl);
+        }
       }
     }
   }
 }
 
 // Arrival on a merge counter; true for the last of `n` arrivals (resets it).
-__device__ bool merge_arrive(Warp &w, uint32_t *ctr, int n) {
+MK_INLINE bool merge_arrive(int lane, uint32_t *ctr, int n) {
   __syncwarp();
   int last = 0;
-  if (w.lane == 0) {
+  if (lane == 0) {
     __threadfence();
-    uint32_t old = atom_add_acq_rel(ctr, 1u);
-    if (old + 1 == static_cast<uint32_t>(n)) {
-      last = 1;
-      *ctr = 0;
-    }
+    const uint32_t old = atom_add_acq_rel(ctr, 1u);
+    if (old + 1 == static_cast<uint32_t>(n)) last = 1;
   }
   last = __shfl_sync(0xffffffffu, last, 0);
-  if (last) fence_acq_rel();
+  if (last) {
+    // every lane observes the final count, then lane 0 rewinds the counter
+    (void)ld_relaxed(ctr);
+    fence_acq_rel();
+    __syncwarp();
+    if (lane == 0) *ctr = 0;
+  }
   __syncwarp();
   return last != 0;
 }
 
 template <int QVP, int DPL>
-__device__ bool op_attn(Warp &w, int op, int layer) {
-  const Params &P = PP(w);
-  const int total = w.attn_prefix[P.B];
-  const int n = my_unit_count(w, op, total), u0 = first_unit(w, op);
-  for (int i = 0; i < n; ++i) {
-    const int item = u0 + i * w.nw;
-    if (!attn_item_run<QVP, DPL>(w, op, layer, item)) return false;
-    const AttnItem a = attn_item(w, item);
-    const int grp = (a.b * P.Hkv + a.g) * P.attn_qsplit + a.qs;
-    const int nch = w.attn_nch[a.b];
-    const int k1 = a.c / kL1Fan, n1 = min(kL1Fan, nch - k1 * kL1Fan), ngrp1 = cdiv(nch, kL1Fan);
-    uint32_t *c1 = P.attn_cnt + static_cast<size_t>(grp) * (kL1Fan + 1) + k1;
-    if (merge_arrive(w, c1, n1)) {
-      attn_merge<QVP, DPL>(w, grp, k1 * kL1Fan, n1, P.attn_nch_max, P.attn_o, P.attn_ml, P.attn_o1,
-                      P.attn_ml1, k1, kL1Fan, false, a.b, a.g);
-      uint32_t *c2 = P.attn_cnt + static_cast<size_t>(grp) * (kL1Fan + 1) + kL1Fan;
-      if (merge_arrive(w, c2, ngrp1)) {
-        attn_merge<QVP, DPL>(w, grp, 0, ngrp1, kL1Fan, P.attn_o1, P.attn_ml1, nullptr, nullptr, 0, 0,
-                        true, a.b, a.g);
-      }
+MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item) {
+  const Params &P = *w.P;
+  const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, item);
+  if (!attn_item_run<QVP, DPL>(w, op, layer, a)) return false;
+  const int grp = (a.b * P.Hkv + a.g) * P.attn_qsplit + a.qs;
+  const int nch = w.attn_nch[a.b];
+  const int k1 = a.c / kL1Fan, n1 = min(kL1Fan, nch - k1 * kL1Fan), ngrp1 = cdiv(nch, kL1Fan);
+  uint32_t *c1 = P.attn_cnt + static_cast<size_t>(grp) * (kL1Fan + 1) + k1;
+  if (merge_arrive(w.lane, c1, n1)) {
+    attn_merge<QVP, DPL>(P, w.lane, grp, k1 * kL1Fan, n1, P.attn_nch_max, P.attn_o, P.attn_ml, P.attn_o1,
+                         P.attn_ml1, k1, kL1Fan, false, a.b, a.g);
+    uint32_t *c2 = P.attn_cnt + static_cast<size_t>(grp) * (kL1Fan + 1) + kL1Fan;
+    if (merge_arrive(w.lane, c2, ngrp1)) {
+      attn_merge<QVP, DPL>(P, w.lane, grp, 0, ngrp1, kL1Fan, P.attn_o1, P.attn_ml1, nullptr, nullptr, 0, 0, true,
+                           a.b, a.g);
     }
   }
   return true;
 }
 
 // --- router top-k and the final argmax (run by the op's last arriving warp) --
-__device__ void router_topk(Warp &w, int layer) {
-  const Params &P = PP(w);
-  const int lane = w.lane, E = P.E, K = P.topk;
-  const int nkc = cdiv(P.d, tile_cols(P));
-  constexpr int EPL = kMaxExperts / 32;
+// Lane l owns experts 4l..4l+3 (slots 0-3) and 128+4l..128+4l+3 (slots 4-7).
+MK_INLINE int expert_of(int lane, int i) { return (i < 4) ? 4 * lane + i : 128 + 4 * lane + (i - 4); }
+
+__device__ __noinline__ void router_topk(const Params &P, int lane, uint32_t epoch, int layer) {
+  const int E = P.E, K = P.topk;
+  const int nkc = cdiv(P.d, kTileCols);
+  constexpr int EPL = 8;
   uint32_t rmask[EPL];
-  float wsel[EPL][kMaxRows];
+  int8_t kslot[EPL][kMaxRows];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     rmask[i] = 0;
 #pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) wsel[i][m] = 0.f;
+    for (int m = 0; m < kMaxRows; ++m) kslot[i][m] = -1;
   }
+  Routing *rt = P.routing + layer;
   for (int m = 0; m < P.M; ++m) {
+    // logits = sum of the K-chunk partials in a fixed order; loads issued together
     float z[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) z[i] = 0.f;
+    for (int k0 = 0; k0 < nkc; k0 += 8) {
+      float4 va[8], vb[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float *row = P.router_part + (static_cast<size_t>(k0 + k) * kMaxRows + m) * P.e_ld;
+        const bool kin = k0 + k < nkc;
+        va[k] = (kin && 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row) + lane)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        vb[k] = (kin && 128 + 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row + 128) + lane)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        z[0] += va[k].x; z[1] += va[k].y; z[2] += va[k].z; z[3] += va[k].w;
+        z[4] += vb[k].x; z[5] += vb[k].y; z[6] += vb[k].z; z[7] += vb[k].w;
+      }
+    }
     bool taken[EPL];
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      z[i] = -INFINITY;
-      taken[i] = true;
-      if (e < E) {
-        float s = 0.f;
-        for (int kc = 0; kc < nkc; ++kc) s += __ldcg(&P.router_part[(static_cast<size_t>(kc) * kMaxRows + m) * E + e]);
-        z[i] = s;
-        taken[i] = false;
-        mx = fmaxf(mx, s);
-      }
+      taken[i] = expert_of(lane, i) >= E;
+      if (!taken[i]) mx = fmaxf(mx, z[i]);
     }
     mx = warp_max(mx);
     float pi[EPL], sum = 0.f;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-      pi[i] = (lane + 32 * i < E) ? expf(z[i] - mx) : 0.f;
+      pi[i] = taken[i] ? 0.f : expf(z[i] - mx);
       sum += pi[i];
     }
     sum = warp_sum(sum);
@@ -1333,7 +1345,7 @@ __device__ void router_topk(Warp &w, int layer) {
       int bi = 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
+        const int e = expert_of(lane, i);
         if (!taken[i] && (pi[i] > bv || (pi[i] == bv && e < bi))) {
           bv = pi[i];
           bi = e;
@@ -1341,8 +1353,8 @@ __device__ void router_topk(Warp &w, int layer) {
       }
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
         if (ov > bv || (ov == bv && oi < bi)) {
           bv = ov;
           bi = oi;
@@ -1350,43 +1362,54 @@ __device__ void router_topk(Warp &w, int layer) {
       }
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
-        if (lane + 32 * i == bi) taken[i] = true;
+        if (expert_of(lane, i) == bi) {
+          taken[i] = true;
+          rmask[i] |= (1u << m);
+#pragma unroll
+          for (int mm = 0; mm < kMaxRows; ++mm)
+            if (mm == m) kslot[i][mm] = static_cast<int8_t>(j);
+        }
       ids[j] = bi;
       ws[j] = bv;
       sel += bv;
     }
-    for (int j = 0; j < K; ++j) {
-      const float wn = ws[j] / sel;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        if (lane + 32 * i == ids[j]) {
-          rmask[i] |= (1u << m);
-#pragma unroll
-          for (int mm = 0; mm < kMaxRows; ++mm)
-            if (mm == m) wsel[i][mm] = wn;
-        }
-      }
-      if (lane == 0) {
+    if (lane == 0) {
+      for (int j = 0; j < K; ++j) {
+        const float wn = ws[j] / sel;
+        rt->row_e[m][j] = ids[j];
+        rt->row_w[m][j] = wn;
         if (P.dbg_ids) P.dbg_ids[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = ids[j];
         if (P.dbg_w) P.dbg_w[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = wn;
       }
     }
   }
-  // publish the union in ascending expert order
-  Routing *rt = P.routing + layer;
+  // publish the union in ascending expert order (block 0, then block 1;
+  // inside a block lane-major, slot-minor)
   int base = 0;
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const bool has = rmask[i] != 0;
-    const uint32_t bits = __ballot_sync(0xffffffffu, has);
-    if (has) {
-      const int pos = base + __popc(bits & ((1u << lane) - 1u));
-      rt->expert[pos] = lane + 32 * i;
-      rt->rowmask[pos] = rmask[i];
+  for (int blk = 0; blk < 2; ++blk) {
+    int cnt = 0;
 #pragma unroll
-      for (int m = 0; m < kMaxRows; ++m) rt->weight[pos][m] = wsel[i][m];
+    for (int qq = 0; qq < 4; ++qq) cnt += rmask[blk * 4 + qq] != 0 ? 1 : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
     }
-    base += __popc(bits);
+    int pos = base + incl - cnt;
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      const int i = blk * 4 + qq;
+      if (rmask[i] != 0) {
+        rt->expert[pos] = expert_of(lane, i);
+        rt->rowmask[pos] = rmask[i];
+#pragma unroll
+        for (int m = 0; m < kMaxRows; ++m) rt->kslot[pos][m] = kslot[i][m];
+        ++pos;
+      }
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
   if (lane == 0) {
     rt->n_union = base;
@@ -1395,17 +1418,16 @@ __device__ void router_topk(Warp &w, int layer) {
   __syncwarp();
   if (lane == 0) {
     __threadfence();
-    st_release(&P.route_flag[layer * kCounterStride], w.epoch);
+    st_release(&P.route_flag[layer * kCounterStride], epoch);
   }
   __syncwarp();
 }
 
-__device__ void final_argmax(Warp &w) {
-  const Params &P = PP(w);
+__device__ __noinline__ void final_argmax(const Params &P, int lane, uint32_t epoch) {
   for (int m = 0; m < P.M; ++m) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
-    for (int s = w.lane; s < P.n_warps; s += 32) {
+    for (int s = lane; s < P.n_warps; s += 32) {
       const ArgmaxPart *pp = P.am_part + static_cast<size_t>(s) * kMaxRows + m;
       const float v = __ldcg(&pp->value);
       const int ix = __ldcg(&pp->index);
@@ -1416,19 +1438,19 @@ __device__ void final_argmax(Warp &w) {
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ov > bv || (ov == bv && oi < bi)) {
         bv = ov;
         bi = oi;
       }
     }
-    if (w.lane == 0) P.argmax[m] = (bi == 0x7fffffff) ? 0 : bi;
+    if (lane == 0) P.argmax[m] = (bi == 0x7fffffff) ? 0 : bi;
   }
   __syncwarp();
-  if (w.lane == 0) {
+  if (lane == 0) {
     __threadfence();
-    st_release(P.epoch, w.epoch);
+    st_release(P.epoch, epoch);
   }
   __syncwarp();
 }
@@ -1436,23 +1458,113 @@ __device__ void final_argmax(Warp &w) {
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <int MMAX>
+// Bounded CTA-wide rendezvous on a shared-memory counter.  Not bar.sync: a
+// warp that leaves on an error must not strand the others, and this wait ends
+// on the timeout or on the error word.
+MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op) {
+  __syncwarp();
+  if (w.lane == 0) {
+    __threadfence_block();
+    atomicAdd(cnt, 1u);
+  }
+  uint64_t t0 = 0;
+  for (int it = 0;; ++it) {
+    const uint32_t v = *reinterpret_cast<volatile uint32_t *>(cnt);
+    if (__all_sync(0xffffffffu, v >= target)) break;
+    if ((it & 31) == 31) {
+      int bad = 0;
+      if (w.lane == 0) {
+        const uint64_t t = now_ns();
+        if (t0 == 0) t0 = t;
+        bad = (t - t0 > w.P->timeout_ns || *reinterpret_cast<volatile const int *>(w.P->error) != 0) ? 1 : 0;
+      }
+      if (__shfl_sync(0xffffffffu, bad, 0)) {
+        set_error(w, -5, op);
+        return false;
+      }
+    }
+  }
+  __threadfence_block();
+  __syncwarp();
+  return true;
+}
+
+// Batch 1: the CTA stages the op's activation row in shared memory once
+// (x = h * g for normed ops, x = o for the o-projection); every warp then
+// reads its columns from there.  All warps take part, with or without units.
+MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, uint32_t &seq, int op) {
+  const Params &P = *w.P;
+  const bool oproj = type == OP_OPROJ;
+  const int K = oproj ? P.Hq * P.hd : P.d;
+  const float4 *src = reinterpret_cast<const float4 *>(oproj ? P.o : P.h);
+  const __nv_bfloat16 *g = oproj ? nullptr
+                           : (type == OP_QKV)    ? P.norms[2 * layer]
+                           : (type == OP_LMHEAD) ? P.final_norm
+                                                 : P.norms[2 * layer + 1];
+  for (int c4 = threadIdx.x; c4 < K / 4; c4 += kThreads) {
+    float4 v = __ldcg(src + c4);
+    if (g) {
+      const uint2 gb = __ldg(reinterpret_cast<const uint2 *>(g + 4 * c4));
+      v.x *= bf_lo(gb.x);
+      v.y *= bf_hi(gb.x);
+      v.z *= bf_lo(gb.y);
+      v.w *= bf_hi(gb.y);
+    }
+    reinterpret_cast<float4 *>(xs)[c4] = v;
+  }
+  seq += kWarpsPerCta;
+  return cta_rendezvous(w, cnt, seq, op);
+}
+
+template <int MMAX, bool XS>
+MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, float &am_val, int &am_idx) {
+  const Params &P = *w.P;
+  const int u0 = first_unit_of(w.slot, op, w.nw);
+  const int n = unit_count_of(u0, op_total_units(w, type, layer), w.nw);
+  if (n == 0) return true;
+  float inv[kMaxRows];
+#pragma unroll
+  for (int m = 0; m < kMaxRows; ++m) inv[m] = 0.f;
+  if (type != OP_OPROJ && type != OP_DOWN && type != OP_ATTN) compute_inv_rms(P, w.lane, inv);
+  for (int i = 0; i < n; ++i) {
+    const int u = u0 + i * w.nw;
+    bool ok;
+    if (type == OP_ATTN) {
+      if (P.hd == 64)
+        ok = (P.attn_qvp == 8) ? attn_unit<8, 2>(w, op, layer, u) : attn_unit<4, 2>(w, op, layer, u);
+      else
+        ok = (P.attn_qvp == 8) ? attn_unit<8, 4>(w, op, layer, u) : attn_unit<4, 4>(w, op, layer, u);
+    } else if (type == OP_ROUTED_GU || type == OP_DOWN || type == OP_SHARED_GU) {
+      ok = routed_dispatch<MMAX, XS>(w, op, type, layer, u, inv, xs);
+    } else {
+      ok = dense_unit<MMAX, XS>(w, op, type, layer, u, inv, xs, am_val, am_idx);
+    }
+    if (!ok || w.failed) return false;
+  }
+  return true;
+}
+
+template <int MMAX, bool XS>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ int s_attn_prefix[kMaxRows + 1];
+  __shared__ int s_attn_nch[kMaxRows];
+  __shared__ uint32_t s_stage;
+  const int wib = threadIdx.x >> 5;
   Warp w;
   w.P = &P;
   w.lane = threadIdx.x & 31;
-  w.wib = threadIdx.x >> 5;
   w.nw = P.n_warps;
-  w.slot = w.wib * P.n_cta + blockIdx.x;
-  w.ring = smem + w.wib * kSlots * kSlotBytes;
-  uint8_t *after_ring = smem + kWarpsPerCta * kSlots * kSlotBytes;
-  w.bars = reinterpret_cast<uint64_t *>(after_ring) + w.wib * kSlots;
-  float *fbase = reinterpret_cast<float *>(after_ring + kWarpsPerCta * kSlots * sizeof(uint64_t));
-  w.wbuf = fbase + w.wib * 3 * kWbuf;
-  w.wacc = w.wbuf + kWbuf;
-  w.wtmp = w.wacc + kWbuf;
-  w.arrive = reinterpret_cast<uint32_t *>(fbase + kWarpsPerCta * 3 * kWbuf);
+  w.slot = wib * P.n_cta + blockIdx.x;
+  w.ring = smem + wib * kSlots * kSlotBytes;
+  float *xs = reinterpret_cast<float *>(smem + kWarpsPerCta * kSlots * kSlotBytes);
+  uint8_t *after_xs = reinterpret_cast<uint8_t *>(xs + P.xs_floats);
+  w.bars = reinterpret_cast<uint64_t *>(after_xs) + wib * kSlots;
+  float *fbase = reinterpret_cast<float *>(after_xs + kWarpsPerCta * kSlots * sizeof(uint64_t));
+  w.wbuf = fbase + wib * kWbuf;
+  w.arrive = reinterpret_cast<uint32_t *>(fbase + kWarpsPerCta * kWbuf);
+  w.attn_prefix = s_attn_prefix;
+  w.attn_nch = s_attn_nch;
   w.phase = 0;
   w.cslot = w.islot = w.inflight = 0;
   w.failed = false;
@@ -1463,7 +1575,18 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < P.n_ops; i += kThreads) w.arrive[i] = 0;
+  if (threadIdx.x == 0) {
+    s_stage = 0;
+    // attention work items per sequence
+    s_attn_prefix[0] = 0;
+    for (int b = 0; b < kMaxRows; ++b) {
+      const int nch = b < P.B ? cdiv(__ldg(&P.positions[b]) + P.T, P.attn_chunk) : 0;
+      s_attn_nch[b] = nch;
+      s_attn_prefix[b + 1] = s_attn_prefix[b] + P.Hkv * P.attn_qsplit * nch;
+    }
+  }
   __syncthreads();
+  uint32_t stage_seq = 0;
 
   w.epoch = *reinterpret_cast<volatile const uint32_t *>(P.epoch) + 1u;
 
@@ -1471,32 +1594,26 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   // Every warp evaluates the same condition, so all exit together.
   bool bad = false;
   for (int b = 0; b < P.B; ++b) {
-    int p = __ldg(&P.positions[b]);
+    const int p = __ldg(&P.positions[b]);
     if (p < 0 || p + P.T > P.cap) bad = true;
   }
   for (int m = w.lane; m < P.M; m += 32) {
-    int t = __ldcg(&P.tokens[m]);
+    const int t = __ldcg(&P.tokens[m]);
     if (t < 0 || t >= P.V) bad = true;
   }
-  bad = __any_sync(0xffffffffu, bad);
-  if (bad) {
+  if (__any_sync(0xffffffffu, bad)) {
     set_error(w, -6, P.op_begin);
     return;
-  }
-  // attention work items per sequence
-  w.attn_prefix[0] = 0;
-  for (int b = 0; b < kMaxRows; ++b) {
-    int nch = 0;
-    if (b < P.B) nch = cdiv(__ldg(&P.positions[b]) + P.T, P.attn_chunk);
-    if (b < kMaxRows) w.attn_nch[b] = nch;
-    w.attn_prefix[b + 1] = w.attn_prefix[b] + (b < P.B ? P.Hkv * P.attn_qsplit * nch : 0);
   }
 
   w.iop = P.op_begin;
   w.iop_init = false;
   w.done_issue = false;
-  w.in_units = w.iu = w.it = 0;
+  w.iu0 = w.in_units = w.iu = w.it = w.iunit = 0;
   w.in_tiles = -1;
+  w.um = w.um2 = nullptr;
+  w.urow0 = w.urow2 = w.ucol0 = w.uK = 0;
+  w.uhalf = 1 << 30;
   issue_more(w);
 
   float am_val = -INFINITY;
@@ -1509,60 +1626,76 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     const uint32_t extra = (op == P.inject_op) ? 1u : 0u;
     if (d0 >= 0 && !wait_counter(w, &P.counters[d0 * kCounterStride], target + extra, op)) break;
     if (d1 >= 0 && !wait_counter(w, &P.counters[d1 * kCounterStride], target, op)) break;
-    if (type == OP_ROUTED_GU || type == OP_DOWN) {
+    if (type == OP_ROUTED_GU || type == OP_DOWN || type == OP_COMBINE) {
       if (!wait_counter(w, &P.route_flag[layer * kCounterStride], w.epoch, op)) break;
     }
+    if constexpr (XS) {
+      // ROUTER stages the normed row that SHARED_GU and ROUTED_GU reuse; a
+      // launch that starts at one of those stages it itself
+      const bool stage = type == OP_QKV || type == OP_OPROJ || type == OP_ROUTER || type == OP_LMHEAD ||
+                         ((type == OP_SHARED_GU || type == OP_ROUTED_GU) && op == P.op_begin);
+      if (stage && !stage_x(w, type, layer, xs, &s_stage, stage_seq, op)) break;
+    }
+    if (P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * 2] = now_ns();
     bool ok = true;
-    switch (type) {
-      case OP_EMBED: op_embed<MMAX>(w, op); break;
-      case OP_ATTN:
-        if (P.hd == 64)
-          ok = (P.attn_qvp == 8) ? op_attn<8, 2>(w, op, layer) : op_attn<4, 2>(w, op, layer);
-        else
-          ok = (P.attn_qvp == 8) ? op_attn<8, 4>(w, op, layer) : op_attn<4, 4>(w, op, layer);
-        break;
-      case OP_ROUTED_GU: ok = op_routed_gu<MMAX>(w, op, layer); break;
-      case OP_DOWN: ok = op_down<MMAX>(w, op, layer); break;
-      default: ok = op_dense<MMAX>(w, op, type, layer, am_val, am_idx); break;
+    if (type == OP_EMBED) {
+      op_embed(w);
+    } else if (type == OP_COMBINE) {
+      op_combine(w, layer);
+    } else {
+      ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, am_val, am_idx);
     }
     if (!ok || w.failed) break;
-    if (type == OP_LMHEAD && w.lane < P.M) {
-      P.am_part[static_cast<size_t>(w.slot) * kMaxRows + w.lane] = ArgmaxPart{am_val, am_idx};
+    if (type == OP_LMHEAD && (w.lane % kRows) == 0 && w.lane / kRows < P.M) {
+      // lane 4m holds this warp's best (value, index) of row m
+      P.am_part[static_cast<size_t>(w.slot) * kMaxRows + w.lane / kRows] = ArgmaxPart{am_val, am_idx};
     }
     const bool last = arrive(w, op);
-    if (last && type == OP_ROUTER) router_topk(w, layer);
-    if (last && type == OP_LMHEAD) final_argmax(w);
+    if (P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * 2 + 1] = now_ns();
+    if (last && type == OP_ROUTER) router_topk(P, w.lane, w.epoch, layer);
+    if (last && type == OP_LMHEAD) final_argmax(P, w.lane, w.epoch);
   }
   drain(w);
 }
 
 }  // namespace
 
-size_t step_smem_bytes(int n_ops) {
-  return static_cast<size_t>(kWarpsPerCta) * kSlots * kSlotBytes +
-         kWarpsPerCta * kSlots * sizeof(uint64_t) + kWarpsPerCta * 3 * kWbuf * sizeof(float) +
+size_t step_smem_bytes(int n_ops, int xs_floats) {
+  return static_cast<size_t>(kWarpsPerCta) * kSlots * kSlotBytes + static_cast<size_t>(xs_floats) * sizeof(float) +
+         kWarpsPerCta * kSlots * sizeof(uint64_t) + kWarpsPerCta * kWbuf * sizeof(float) +
          static_cast<size_t>(n_ops) * sizeof(uint32_t);
 }
 
-template <int MMAX>
+template <int MMAX, bool XS>
 static const void *kernel_ptr() {
-  return reinterpret_cast<const void *>(&mk_step_kernel<MMAX>);
+  return reinterpret_cast<const void *>(&mk_step_kernel<MMAX, XS>);
 }
 
+// Batch 1 stages its activation row in shared memory; more rows read it via L1.
 static const void *kernel_for(int mmax) {
   switch (mmax) {
-    case 1: return kernel_ptr<1>();
-    case 2: return kernel_ptr<2>();
-    case 4: return kernel_ptr<4>();
-    default: return kernel_ptr<8>();
+    case 1: return kernel_ptr<1, true>();
+    case 2: return kernel_ptr<2, false>();
+    case 4: return kernel_ptr<4, false>();
+    default: return kernel_ptr<8, false>();
   }
 }
 
+bool kernel_stages_x(int mmax) { return mmax == 1; }
+
 int max_cta_per_sm(int mmax, size_t smem) {
   const void *k = kernel_for(mmax);
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return -1;
+  // Ask for the smallest shared-memory carve-out that fits, leaving the rest of
+  // the SM's unified memory to L1 (activations are re-read through it by every warp).
+  int max_sm = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  if (max_sm > 0) {
+    const int pct = static_cast<int>((smem * 100 + max_sm - 1) / max_sm);
+    cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, pct > 100 ? 100 : pct);
+  }
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) != cudaSuccess) return -1;
   return n;
@@ -1570,7 +1703,7 @@ int max_cta_per_sm(int mmax, size_t smem) {
 
 int launch_step(const Params &p, int mmax, bool cooperative, cudaStream_t stream) {
   const void *k = kernel_for(mmax);
-  const size_t smem = step_smem_bytes(p.n_ops);
+  const size_t smem = step_smem_bytes(p.n_ops, p.xs_floats);
   void *args[] = {const_cast<Params *>(&p)};
   cudaError_t e;
   if (cooperative) {

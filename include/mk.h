@@ -67,7 +67,7 @@ extern "C" {
 #define MK_FAULT_UNREACHABLE_WAIT 1 /* next step: one dependency waits for a count
                                        that is never reached (bounded wait test) */
 
-/* Model description.  Supported: head_dim in {32, 64, 128, 256};
+/* Model description.  Supported: head_dim in {64, 128};
  * n_q_heads % n_kv_heads == 0; d_model, n_q_heads*head_dim multiples of 8;
  * expert_ffn and shared_ffn multiples of 16 (shared_ffn may be 0 = no shared
  * expert); n_experts <= 256; top_k <= min(16, n_experts);
@@ -126,7 +126,7 @@ typedef struct mk_plan_info {
   int32_t n_ops;           /* ops in one step's schedule                     */
   int32_t n_cta;           /* CTAs of the persistent grid (= SM count)       */
   int32_t warps_per_cta;   /* consumer/producer warps per CTA                */
-  int32_t rows_per_tile;   /* weight rows per ring tile (16, or 8 at M > 4)  */
+  int32_t rows_per_tile;   /* weight rows per ring tile (8: tiles are 8 x 512) */
   int32_t mmax;            /* row capacity of the kernel instance (1,2,4,8)  */
   int32_t attn_chunk;      /* KV positions per attention work item          */
   int32_t attn_qsplit;     /* query-vector groups per (sequence, KV head)    */
@@ -134,15 +134,18 @@ typedef struct mk_plan_info {
   int64_t scratch_bytes;   /* device scratch owned by a handle of this shape */
 } mk_plan_info;
 
+/* Ops of one step's schedule: EMBED, then per layer QKV ATTN OPROJ ROUTER
+ * SHARED_GU ROUTED_GU DOWN COMBINE, then LMHEAD. */
 #define MK_OP_EMBED 0
-#define MK_OP_QKV 1
-#define MK_OP_ATTN 2
-#define MK_OP_OPROJ 3
-#define MK_OP_ROUTER 4
-#define MK_OP_SHARED_GU 5
-#define MK_OP_ROUTED_GU 6
-#define MK_OP_DOWN 7
-#define MK_OP_LMHEAD 8
+#define MK_OP_QKV 1        /* RMSNorm + QKV projection                          */
+#define MK_OP_ATTN 2       /* rotary, KV append, split-K attention, LSE merge   */
+#define MK_OP_OPROJ 3      /* o-projection + residual                           */
+#define MK_OP_ROUTER 4     /* RMSNorm + router logits; last warp: softmax top-k */
+#define MK_OP_SHARED_GU 5  /* shared expert gate/up rows                        */
+#define MK_OP_ROUTED_GU 6  /* routed experts' gate/up rows (union of the batch) */
+#define MK_OP_DOWN 7       /* down projections, one partial per (row, expert)   */
+#define MK_OP_COMBINE 8    /* weighted sum of the partials + residual           */
+#define MK_OP_LMHEAD 9     /* final RMSNorm + lm_head; last warp: argmax        */
 
 /* Create a handle: validates the descriptor, plans the schedule, encodes the
  * weight tensor maps, allocates scratch on the current device.  No kernel
@@ -207,6 +210,12 @@ MK_API int mk_set_debug(mk_handle *h, float *hidden, int32_t *expert_ids, float 
 
 /* Arm a fault for the next step (MK_FAULT_*). */
 MK_API int mk_debug_inject(mk_handle *h, int32_t fault);
+
+/* Per-op timeline of every following step (NULL disables): device uint64
+ * [n_ops][n_cta * warps_per_cta][2] = %globaltimer (ns) when the warp finished
+ * waiting for the op's inputs and when it arrived at the op's completion
+ * counter.  n_ops and the grid come from mk_plan_describe. */
+MK_API int mk_set_trace(mk_handle *h, uint64_t *trace);
 
 /* Copies the handle's counters; reset != 0 zeroes them afterwards.  Waits for
  * the device (reads a device counter). */

@@ -80,11 +80,15 @@ TINY = ModelConfig("tiny", 2, 256, 4, 2, 64, 8, 2, 512, 0, 1024)
 SMALL = ModelConfig("small", 8, 2048, 16, 4, 128, 64, 4, 1024, 1024, 32000)
 LARGE = ModelConfig("large", 16, 4096, 32, 8, 128, 128, 8, 1536, 1536, 64000, sigma=0.015)
 
-MODELS = {m.name: m for m in (TINY, SMALL, LARGE)}
+# The large model's dimensions with 2 layers and 16 experts (about 2.5 GB of
+# weights): the same per-op shapes, small enough for a full profiler capture.
+PROFILE = ModelConfig("profile", 2, 4096, 32, 8, 128, 16, 8, 1536, 1536, 64000, sigma=0.015)
+
+MODELS = {m.name: m for m in (TINY, SMALL, LARGE, PROFILE)}
 
 
 def workload(kind: str, batch: int = 1) -> Workload:
-    """The named workloads: tiny / small / small_batch / verify / large."""
+    """The named workloads: tiny / small / small_batch / verify / large / profile."""
     if kind == "tiny":
         return Workload("tiny_bs1", TINY, 1, 1, 127, steps=16, seed=0)
     if kind == "small":
@@ -95,6 +99,8 @@ def workload(kind: str, batch: int = 1) -> Workload:
         return Workload(f"verify_b{batch}_t7", SMALL, batch, 7, 2048, steps=64, seed=3)
     if kind == "large":
         return Workload(f"large_bs{batch}", LARGE, batch, 1, 4095, steps=32, seed=4)
+    if kind == "profile":
+        return Workload(f"profile_bs{batch}", PROFILE, batch, 1, 4095, steps=8, seed=5)
     raise ValueError(f"unknown workload {kind!r}")
 
 

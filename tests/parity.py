@@ -133,17 +133,23 @@ def compare_step(s: Session, ref, got, rep: Report, alive: np.ndarray, positions
                 assert int(am[m]) == int(ref.argmax[m]), f"argmax row {m}: {am[m]} vs {ref.argmax[m]}"
             else:
                 rep.argmax_near_ties += 1
-    # appended cache entries agree to within one bf16 ulp on live sequences
-    kd = s.k.view(torch.int16)
-    for b in range(s.B):
-        if dead[b]:
-            continue
-        p0 = positions[b]
-        got_k = kd[:, b, :, p0:p0 + T].cpu().numpy().view(np.uint16)
-        ref_k = s.k_host[:, b, :, p0:p0 + T]
-        ulps = np.abs(got_k.astype(np.int32) - ref_k.astype(np.int32)).max()
-        rep.kv_max_ulps = max(rep.kv_max_ulps, float(ulps))
-        assert ulps <= 1, f"appended keys differ by {ulps} bf16 ulps"
+    # appended cache entries: same bar as the per-layer states (max|d|/max|ref|);
+    # the largest bf16 ulp difference is reported (near-zero entries can differ
+    # by several ulps from fp32 summation order alone)
+    for cache, host in ((s.k, s.k_host), (s.v, s.v_host)):
+        cd = cache.view(torch.int16)
+        for b in range(s.B):
+            if dead[b]:
+                continue
+            p0 = positions[b]
+            got_k = cd[:, b, :, p0:p0 + T].cpu().numpy().view(np.uint16)
+            ref_k = host[:, b, :, p0:p0 + T]
+            ulps = np.abs(got_k.astype(np.int32) - ref_k.astype(np.int32)).max()
+            rep.kv_max_ulps = max(rep.kv_max_ulps, float(ulps))
+            import oracle
+
+            e = relerr(oracle.bf16_to_f32(got_k), oracle.bf16_to_f32(ref_k))
+            assert e <= HIDDEN_TOL, f"appended cache entries rel err {e}"
     alive &= ~dead
     rep.flagged_rows = int((~alive).sum())
 

@@ -85,21 +85,25 @@ def test_schedule_is_a_dag_with_the_data_dependencies(L):
     rc, info, ops = mk.mk_plan_describe(d, 148, 1, 1)
     assert rc == mk.MK_OK, mk.mk_last_error()
     Lyr = SMALL.n_layers
-    assert info.n_ops == len(ops) == 7 * Lyr + 2
+    assert info.n_ops == len(ops) == 8 * Lyr + 2
     names = [mk.OP_NAMES[t] for t, *_ in ops]
     assert names[0] == "EMBED" and names[-1] == "LMHEAD"
-    assert names[1:8] == ["QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN"]
+    assert names[1:9] == ["QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE"]
+    idx = {(mk.OP_NAMES[t], l): i for i, (t, l, _, _) in enumerate(ops)}
     reach = []
     for i, (t, layer, d0, d1) in enumerate(ops):
         assert d0 < i and d1 < i
+        deps = [d0, d1]
+        if mk.OP_NAMES[t] == "ROUTED_GU":  # also waits for the routing ROUTER publishes
+            deps.append(idx[("ROUTER", layer)])
         r = set()
-        for dep in (d0, d1):
+        for dep in deps:
             if dep >= 0:
+                assert dep < i
                 r |= {dep} | reach[dep]
         reach.append(r)
-    idx = {(mk.OP_NAMES[t], l): i for i, (t, l, _, _) in enumerate(ops)}
     for l in range(Lyr):
-        prev_h = idx[("EMBED", -1)] if l == 0 else idx[("DOWN", l - 1)]
+        prev_h = idx[("EMBED", -1)] if l == 0 else idx[("COMBINE", l - 1)]
         need = {
             "QKV": [prev_h],
             "ATTN": [idx[("QKV", l)]],
@@ -108,13 +112,16 @@ def test_schedule_is_a_dag_with_the_data_dependencies(L):
             "SHARED_GU": [idx[("OPROJ", l)]],
             "ROUTED_GU": [idx[("OPROJ", l)]],
             "DOWN": [idx[("SHARED_GU", l)], idx[("ROUTED_GU", l)], idx[("OPROJ", l)]],
+            "COMBINE": [idx[("DOWN", l)], idx[("ROUTER", l)]],
         }
         for name, deps in need.items():
             for dep in deps:
                 assert dep in reach[idx[(name, l)]], (name, l, dep)
-        # writers of h (OPROJ, DOWN) come after every reader of the previous h
+        # writers of h (OPROJ, COMBINE) come after every reader of the previous h
         assert idx[("QKV", l)] in reach[idx[("OPROJ", l)]]
-    assert idx[("DOWN", Lyr - 1)] in reach[idx[("LMHEAD", -1)]]
+        for reader in ("ROUTER", "SHARED_GU", "ROUTED_GU"):
+            assert idx[(reader, l)] in reach[idx[("COMBINE", l)]] or reader == "ROUTER"
+    assert idx[("COMBINE", Lyr - 1)] in reach[idx[("LMHEAD", -1)]]
 
 
 @pytest.mark.parametrize("model,B,T,cap", [(TINY, 1, 1, 256), (SMALL, 1, 1, 2112),
@@ -126,7 +133,7 @@ def test_plan_shapes(L, model, B, T, cap):
     assert rc == mk.MK_OK, mk.mk_last_error()
     M = B * T
     assert info.mmax >= M and info.mmax in (1, 2, 4, 8)
-    assert info.rows_per_tile == (16 if M <= 4 else 8)
+    assert info.rows_per_tile == 4
     ppt = 2048 // model.head_dim
     assert info.attn_chunk % ppt == 0 and info.attn_chunk >= ppt
     assert -(-cap // info.attn_chunk) <= 256          # two-level merge bound
