@@ -79,7 +79,7 @@ int encode_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, 
 // ---- planning ---------------------------------------------------------------------
 struct Plan {
   int M, mmax, rows_per_tile, n_hb;
-  int attn_qvp, attn_qsplit, attn_ppt, attn_chunk, attn_nch_max;
+  int attn_qsplit, attn_ppt, attn_chunk, attn_nch_max;
   int n_ops, n_cta, n_warps, xs_floats;
   size_t smem;
 };
@@ -91,28 +91,32 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.rows_per_tile = kRows;
   p.n_hb = ceil_div(d.d_model, kRows);
   const int G = d.n_q_heads / d.n_kv_heads;
-  p.attn_qvp = (G * T <= 4) ? 4 : 8;
-  p.attn_qsplit = ceil_div(G * T, p.attn_qvp);
+  p.attn_qsplit = ceil_div(G * T, kQvp);
   p.attn_ppt = 2048 / d.head_dim;
   p.n_cta = n_sm;
   p.n_warps = n_sm * kWarpsPerCta;
-  // KV chunk: about one work item per warp, a multiple of the tile height, and
-  // few enough chunks per (sequence, kv head, query group) for a two-level merge.
+  // Attention items are CTA-wide: each of the 8 warps takes attn_chunk KV
+  // positions of an item.  About one item per CTA, warp chunks a multiple of
+  // the tile height, and at most kMaxChunks items per (sequence, kv head,
+  // query group) so that one merge level combines them.
   long long total = (long long)B * d.n_kv_heads * p.attn_qsplit * d.kv_capacity;
   int c = (int)((total + p.n_warps - 1) / p.n_warps);
-  c = std::max(c, ceil_div(d.kv_capacity, kMaxChunks));
+  c = std::max(c, ceil_div(d.kv_capacity, kMaxChunks * kWarpsPerCta));
   c = std::max(c, p.attn_ppt);
   c = ceil_div(c, p.attn_ppt) * p.attn_ppt;
   p.attn_chunk = c;
-  p.attn_nch_max = ceil_div(d.kv_capacity, c);
+  p.attn_nch_max = ceil_div(d.kv_capacity, c * kWarpsPerCta);
   p.n_ops = n_ops_for(d.n_layers);
-  p.xs_floats = kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), 4) * 4 : 0;
+  // shared-memory row: the staged activations (batch 1) or the attention
+  // warps' partials, whichever is larger
+  p.xs_floats = std::max(kWarpsPerCta * kQvp * d.head_dim,
+                         kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), 4) * 4 : 0);
   p.smem = step_smem_bytes(p.n_ops, p.xs_floats);
   return p;
 }
 
 struct Sizes {
-  size_t attn_o, attn_ml, attn_o1, attn_ml1, attn_cnt;
+  size_t attn_o, attn_ml, attn_cnt;
 };
 
 Sizes scratch_sizes(const mk_model_desc &d, int n_sm) {
@@ -121,11 +125,9 @@ Sizes scratch_sizes(const mk_model_desc &d, int n_sm) {
     for (int T = 1; B * T <= d.max_rows; ++T) {
       Plan p = make_plan(d, n_sm, B, T);
       size_t ngrp = (size_t)d.max_seqs * d.n_kv_heads * p.attn_qsplit;
-      s.attn_o = std::max(s.attn_o, ngrp * p.attn_nch_max * p.attn_qvp * d.head_dim);
-      s.attn_ml = std::max(s.attn_ml, ngrp * p.attn_qvp * 2 * p.attn_nch_max);
-      s.attn_o1 = std::max(s.attn_o1, ngrp * kL1Fan * p.attn_qvp * d.head_dim);
-      s.attn_ml1 = std::max(s.attn_ml1, ngrp * p.attn_qvp * 2 * kL1Fan);
-      s.attn_cnt = std::max(s.attn_cnt, ngrp * (kL1Fan + 1));
+      s.attn_o = std::max(s.attn_o, ngrp * p.attn_nch_max * kQvp * d.head_dim);
+      s.attn_ml = std::max(s.attn_ml, ngrp * kQvp * 2 * p.attn_nch_max);
+      s.attn_cnt = std::max(s.attn_cnt, ngrp);
     }
   return s;
 }
@@ -146,7 +148,7 @@ struct mk_handle {
   std::vector<void *> allocs;
   CUtensorMap *tmaps;
   const __nv_bfloat16 **norms;
-  float *h, *ss, *qkv, *o, *attn_o, *attn_ml, *attn_o1, *attn_ml1, *router_part, *act_shared,
+  float *h, *ss, *qkv, *o, *attn_o, *attn_ml, *router_part, *act_shared,
       *act_routed, *y_part, *logits;
   uint32_t *attn_cnt, *counters, *route_flag, *epoch;
   Routing *routing;
@@ -230,8 +232,8 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
     size_t f = (size_t)d.max_rows * d.d_model * 2 + (size_t)d.max_rows * ceil_div(d.d_model, kRows) +
                (size_t)kMaxRows * (d.top_k + 1) * d.d_model +
                (size_t)d.max_rows * (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim +
-               (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml + s.attn_o1 +
-               s.attn_ml1 + (size_t)ceil_div(d.d_model, kPanel) * kMaxRows * d.n_experts +
+               (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml +
+               (size_t)ceil_div(d.d_model, kPanel) * kMaxRows * d.n_experts +
                (size_t)kMaxRows * d.shared_ffn +
                (size_t)std::min(d.n_experts, d.max_rows * d.top_k) * kMaxRows * d.expert_ffn +
                (size_t)d.max_rows * d.vocab + (size_t)d.kv_capacity * d.head_dim;
@@ -333,8 +335,6 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
   HALLOC(h->attn_o, sizeof(float) * s.attn_o);
   HALLOC(h->attn_ml, sizeof(float) * s.attn_ml);
-  HALLOC(h->attn_o1, sizeof(float) * s.attn_o1);
-  HALLOC(h->attn_ml1, sizeof(float) * s.attn_ml1);
   h->attn_cnt_bytes = sizeof(uint32_t) * s.attn_cnt;
   HALLOC(h->attn_cnt, h->attn_cnt_bytes);
   HALLOC(h->router_part, sizeof(float) * (size_t)ceil_div(D, kTileCols) * kMaxRows * ceil_div(d.n_experts, 4) * 4);
@@ -452,7 +452,7 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.xs_floats = pl.xs_floats;
   p.ss_ld = ceil_div(pl.n_hb, 128) * 128;
   p.e_ld = ceil_div(d.n_experts, 4) * 4;
-  p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit; p.attn_qvp = pl.attn_qvp;
+  p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit;
   p.attn_ppt = pl.attn_ppt; p.attn_nch_max = pl.attn_nch_max;
   p.tmaps = h->tmaps; p.norms = h->norms;
   p.embed = static_cast<const __nv_bfloat16 *>(h->embed);
@@ -460,7 +460,7 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.kc = static_cast<__nv_bfloat16 *>(kv.k); p.vc = static_cast<__nv_bfloat16 *>(kv.v);
   p.tokens = tokens; p.positions = positions; p.logits = logits ? logits : h->logits; p.argmax = argmax;
   p.h = h->h; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
-  p.attn_o = h->attn_o; p.attn_ml = h->attn_ml; p.attn_o1 = h->attn_o1; p.attn_ml1 = h->attn_ml1;
+  p.attn_o = h->attn_o; p.attn_ml = h->attn_ml;
   p.attn_cnt = h->attn_cnt; p.router_part = h->router_part; p.routing = h->routing;
   p.act_shared = h->act_shared; p.act_routed = h->act_routed; p.y_part = h->y_part;
   p.am_part = h->am_part; p.rope = h->rope;

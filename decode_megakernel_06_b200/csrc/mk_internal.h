@@ -23,8 +23,8 @@ constexpr int kKvBoxBytes = 4096;                   // K or V box: ppt positions
 constexpr int kMaxRows = 8;                         // M = B*T cap of this build
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 16;
-constexpr int kL1Fan = 16;                          // attention merge fan-in per level
-constexpr int kMaxChunks = kL1Fan * kL1Fan;         // KV chunks per (seq, kv head, q group)
+constexpr int kQvp = 4;                             // query vectors per attention item
+constexpr int kMaxChunks = 32;                      // CTA KV chunks per (seq, kv head, q group)
 constexpr int kCounterStride = 32;                  // uint32s between counters (128 B)
 
 // Ops of one step: EMBED, then per layer QKV ATTN OPROJ ROUTER SHARED_GU
@@ -76,12 +76,11 @@ enum MapSlot : int {
   MAP_WSGATE, MAP_WSUP, MAP_WSDOWN, MAPS_PER_LAYER
 };
 
-// Routing of one layer, written by the last warp to finish the router op.
+// Routing of one layer, written by the last warp to finish the router op:
+// each row's selections in selection order.  CTAs derive the expert union,
+// row masks and slots from these into a shared-memory cache.
 struct Routing {
   int n_union;                            // distinct experts over the M rows
-  int expert[kMaxExperts];                // ascending expert ids, [n_union]
-  uint32_t rowmask[kMaxExperts];          // rows routed to expert[j]
-  int8_t kslot[kMaxExperts][kMaxRows];    // selection index of expert[j] in row m
   int row_e[kMaxRows][kMaxTopK];          // row m's selections, in selection order
   float row_w[kMaxRows][kMaxTopK];        // and their renormalised weights
 };
@@ -104,7 +103,8 @@ struct alignas(64) Params {
   int xs_floats;       // shared-memory activation row (batch 1), 0 = none
   int ss_ld;           // row stride of the sum-of-squares partials (n_hb rounded up to 128)
   int e_ld;            // row stride of the router partials (E rounded up to 4)
-  int attn_chunk, attn_qsplit, attn_qvp, attn_ppt, attn_nch_max;
+  int attn_chunk;      // KV positions per warp; a CTA item covers 8 * attn_chunk
+  int attn_qsplit, attn_ppt, attn_nch_max;
   // weights
   const CUtensorMap *tmaps;              // [L][MAPS_PER_LAYER] + lm_head
   const __nv_bfloat16 *const *norms;     // [L][2]: attn_norm, ffn_norm
@@ -116,7 +116,7 @@ struct alignas(64) Params {
   int *argmax;
   // scratch
   float *h, *ss, *qkv, *o;
-  float *attn_o, *attn_ml, *attn_o1, *attn_ml1;
+  float *attn_o, *attn_ml;   // per-CTA-chunk partials (unnormalised o; max, sum)
   uint32_t *attn_cnt;
   float *router_part;
   Routing *routing;                      // [L]

@@ -202,9 +202,21 @@ MK_INLINE int unit_count_of(int u0, int total, int nw) { return total > u0 ? (to
 // ---------------------------------------------------------------------------
 constexpr int kWbuf = 64;  // floats of per-warp epilogue scratch (2 * 4 * MJ <= 64)
 
+// Per-CTA cache of one layer's routing, derived from the top-k's per-row
+// selections: the ascending expert union, rows served by each, their slots.
+struct RouteCache {
+  int ready_key, fill_key;   // layer + 1 once filled / being filled
+  int n_union;
+  int expert[kMaxExperts];
+  uint32_t rowmask[kMaxExperts];
+  int8_t kslot[kMaxExperts][kMaxRows];
+  float row_w[kMaxRows][kMaxTopK];
+};
+
 struct Warp {
   const Params *P;
-  int lane, slot, nw;
+  RouteCache *rc;
+  int lane, wib, cta, slot, nw;
   uint32_t epoch;
   uint8_t *ring;
   uint64_t *bars;
@@ -245,7 +257,90 @@ MK_INLINE bool routing_ready(const Warp &w, int layer) {
   return ok;
 }
 
-MK_INLINE int n_union(const Params &P, int layer) { return __ldcg(&P.routing[layer].n_union); }
+// Fill the CTA's routing cache for `layer` (one elected warp; the others wait,
+// bounded).  The caller has observed the layer's routing flag.
+__device__ __noinline__ void route_cache_fill(const Params &P, RouteCache *rc, int lane, int layer) {
+  const Routing *rt = P.routing + layer;
+  const int K = P.topk, MK = P.M * K;
+  // lane l gathers experts 8l..8l+7: row mask and per-row selection slot
+  uint32_t mask[8];
+  uint64_t slots[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    mask[i] = 0;
+    slots[i] = ~0ull;
+  }
+  for (int base = 0; base < MK; base += 32) {
+    const int idx = base + lane;
+    const int e_mine = idx < MK ? __ldcg(&rt->row_e[idx / K][idx % K]) : -1;
+    const int cnt = min(32, MK - base);
+    for (int q = 0; q < cnt; ++q) {
+      const int e = __shfl_sync(0xffffffffu, e_mine, q);
+      const int m = (base + q) / K, j = (base + q) % K;
+      if ((e >> 3) == lane) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if ((e & 7) == i) {
+            mask[i] |= 1u << m;
+            slots[i] = (slots[i] & ~(0xffull << (8 * m))) | (static_cast<uint64_t>(j) << (8 * m));
+          }
+      }
+    }
+  }
+  int cnt = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) cnt += mask[i] ? 1 : 0;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  int pos = incl - cnt;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (mask[i]) {
+      rc->expert[pos] = 8 * lane + i;
+      rc->rowmask[pos] = mask[i];
+#pragma unroll
+      for (int m = 0; m < kMaxRows; ++m) rc->kslot[pos][m] = static_cast<int8_t>(slots[i] >> (8 * m));
+      ++pos;
+    }
+  if (lane == 31) rc->n_union = incl;
+  for (int idx = lane; idx < MK; idx += 32) rc->row_w[idx / K][idx % K] = __ldcg(&rt->row_w[idx / K][idx % K]);
+  __threadfence_block();
+  __syncwarp();
+  if (lane == 0) *reinterpret_cast<volatile int *>(&rc->ready_key) = layer + 1;
+  __syncwarp();
+}
+
+MK_INLINE bool route_cache(Warp &w, int layer) {
+  RouteCache *rc = w.rc;
+  if (*reinterpret_cast<volatile int *>(&rc->ready_key) == layer + 1) {
+    __threadfence_block();
+    return true;
+  }
+  int filler = 0;
+  if (w.lane == 0) filler = atomicMax(&rc->fill_key, layer + 1) < layer + 1 ? 1 : 0;
+  filler = __shfl_sync(0xffffffffu, filler, 0);
+  if (filler) {
+    route_cache_fill(*w.P, rc, w.lane, layer);
+  } else {
+    const uint64_t t0 = now_ns();
+    while (*reinterpret_cast<volatile int *>(&rc->ready_key) != layer + 1) {
+      if (now_ns() - t0 > w.P->timeout_ns) {
+        report_error(*w.P, w.lane, -5, -1);
+        w.failed = true;
+        return false;
+      }
+    }
+  }
+  __threadfence_block();
+  __syncwarp();
+  return true;
+}
+
+MK_INLINE int n_union(const Warp &w) { return w.rc->n_union; }
 
 // Total units of an op over the whole grid.  ROUTED_GU / DOWN need routing.
 MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
@@ -257,31 +352,35 @@ MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
     case OP_OPROJ: return P.n_hb;
     case OP_ROUTER: return cdiv(P.E, kRows) * cdiv(P.d, kTileCols);
     case OP_SHARED_GU: return P.Fs / kRows;
-    case OP_ROUTED_GU: return n_union(P, layer) * (P.F / kRows);
-    case OP_DOWN: return (n_union(P, layer) + (P.Fs > 0 ? 1 : 0)) * P.n_hb;
+    case OP_ROUTED_GU: return n_union(w) * (P.F / kRows);
+    case OP_DOWN: return (n_union(w) + (P.Fs > 0 ? 1 : 0)) * P.n_hb;
     case OP_COMBINE: return P.n_hb;
     case OP_LMHEAD: return cdiv(P.V, kRows);
   }
   return 0;
 }
 
+// An attention item covers 8 * attn_chunk KV positions of one (sequence,
+// kv head, query group); warp `wib` of the CTA takes attn_chunk of them.
 struct AttnItem {
-  int b, g, qs, c, pos0, npos, ntiles;
+  int b, g, qs, c, nch;  // sequence, kv head, query group, CTA chunk, chunks of this sequence
+  int pos0, npos, ntiles;  // this warp's positions: [pos0, pos0 + npos), in tiles
 };
 
-MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs, int item) {
+MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs, int item, int wib) {
   AttnItem a;
   int b = 0;
   while (b + 1 < P.B && item >= prefix[b + 1]) ++b;
   const int rem = item - prefix[b];
   const int nch = nchs[b];
   a.b = b;
+  a.nch = nch;
   a.c = rem % nch;
   a.qs = (rem / nch) % P.attn_qsplit;
   a.g = rem / (nch * P.attn_qsplit);
   const int len = __ldg(&P.positions[b]) + P.T;
-  a.pos0 = a.c * P.attn_chunk;
-  a.npos = min(P.attn_chunk, len - a.pos0);
+  a.pos0 = a.c * P.attn_chunk * kWarpsPerCta + wib * P.attn_chunk;
+  a.npos = max(0, min(P.attn_chunk, len - a.pos0));
   a.ntiles = cdiv(a.npos, P.attn_ppt);
   return a;
 }
@@ -296,8 +395,8 @@ MK_INLINE int unit_tiles(const Warp &w, int type, int layer, int unit) {
     case OP_ROUTED_GU: return 2 * cdiv(P.d, kTileCols);
     case OP_OPROJ: return cdiv(P.Hq * P.hd, kTileCols);
     case OP_ROUTER: return 1;
-    case OP_DOWN: return (unit / P.n_hb) < n_union(P, layer) ? cdiv(P.F, kTileCols) : cdiv(P.Fs, kTileCols);
-    case OP_ATTN: return attn_item(P, w.attn_prefix, w.attn_nch, unit).ntiles;
+    case OP_DOWN: return (unit / P.n_hb) < n_union(w) ? cdiv(P.F, kTileCols) : cdiv(P.Fs, kTileCols);
+    case OP_ATTN: return attn_item(P, w.attn_prefix, w.attn_nch, unit, w.wib).ntiles;
     default: return 0;
   }
 }
@@ -330,7 +429,7 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
       break;
     case OP_ROUTED_GU: {
       const int nfb = P.F / kRows;
-      const int e = __ldcg(&P.routing[layer].expert[unit / nfb]);
+      const int e = w.rc->expert[unit / nfb];
       row0 = row2 = e * P.F + (unit % nfb) * kRows;
       m0 = lm + MAP_WGATE;
       m2 = lm + MAP_WUP;
@@ -339,8 +438,8 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
     }
     case OP_DOWN: {
       const int seg = unit / P.n_hb, rb = unit % P.n_hb;
-      if (seg < n_union(P, layer)) {
-        const int e = __ldcg(&P.routing[layer].expert[seg]);
+      if (seg < n_union(w)) {
+        const int e = w.rc->expert[seg];
         m0 = lm + MAP_WDOWN;
         row0 = e * P.d + rb * kRows;
         K = P.F;
@@ -367,7 +466,7 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
   uint8_t *dst = w.ring + w.islot * kSlotBytes;
   uint64_t *bar = &w.bars[w.islot];
   if (type == OP_ATTN) {
-    const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, w.iunit);
+    const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, w.iunit, w.wib);
     const int row = ((layer * P.Bmax + a.b) * P.Hkv + a.g) * P.cap + a.pos0 + t * P.attn_ppt;
     if (w.lane == 0) {
       fence_proxy_async_smem();
@@ -406,9 +505,15 @@ MK_INLINE void issue_more(Warp &w) {
       continue;
     }
     if (!w.iop_init) {
-      if ((type == OP_ROUTED_GU || type == OP_DOWN) && !routing_ready(w, layer)) return;
-      w.iu0 = first_unit_of(w.slot, w.iop, w.nw);
-      w.in_units = unit_count_of(w.iu0, op_total_units(w, type, layer), w.nw);
+      if (type == OP_ROUTED_GU || type == OP_DOWN) {
+        if (!routing_ready(w, layer)) return;
+        if (!route_cache(w, layer)) return;
+      }
+      // attention items are CTA-wide (every warp of the CTA takes a share)
+      const bool cta_items = type == OP_ATTN;
+      const int stride = cta_items ? P.n_cta : w.nw;
+      w.iu0 = cta_items ? w.cta : first_unit_of(w.slot, w.iop, w.nw);
+      w.in_units = unit_count_of(w.iu0, op_total_units(w, type, layer), stride);
       w.iu = 0;
       w.in_tiles = -1;
       w.iop_init = true;
@@ -419,7 +524,7 @@ MK_INLINE void issue_more(Warp &w) {
       continue;
     }
     if (w.in_tiles < 0) {
-      w.iunit = w.iu0 + w.iu * w.nw;
+      w.iunit = w.iu0 + w.iu * (type == OP_ATTN ? P.n_cta : w.nw);
       w.it = 0;
       w.in_tiles = unit_tiles(w, type, layer, w.iunit);
       if (type != OP_ATTN) unit_source(w, type, layer, w.iunit);
@@ -750,14 +855,14 @@ MK_INLINE void op_embed(Warp &w) {
 MK_INLINE void op_combine(Warp &w, int layer) {
   const Params &P = *w.P;
   const int S = P.topk + 1;
-  const Routing *rt = P.routing + layer;
+  const RouteCache *rt = w.rc;
   for (int unit = w.slot; unit < P.n_hb; unit += w.nw) {
     residual_rows(P, w.lane, unit, unit * kRows, layer + 1, [&](int m, int row, int) {
       const float *yp = P.y_part + (static_cast<size_t>(m) * S) * P.d + row;
       float moe = 0.f;
 #pragma unroll
       for (int s = 0; s < kMaxTopK; ++s)
-        if (s < P.topk) moe += __ldcg(&rt->row_w[m][s]) * __ldcg(yp + static_cast<size_t>(s) * P.d);
+        if (s < P.topk) moe += rt->row_w[m][s] * __ldcg(yp + static_cast<size_t>(s) * P.d);
       const float sh = P.Fs > 0 ? __ldcg(yp + static_cast<size_t>(P.topk) * P.d) : 0.f;
       return __ldcg(P.h + static_cast<size_t>(m) * P.d + row) + (moe + sh);
     });
@@ -914,7 +1019,7 @@ MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const flo
   if (type == OP_ROUTED_GU) {
     const int nfb = P.F / kRows, j = unit / nfb;
     f0 = (unit % nfb) * kRows;
-    xn.n = rows_of_mask<MJ>(__ldcg(&P.routing[layer].rowmask[j]), xn.row);
+    xn.n = rows_of_mask<MJ>(w.rc->rowmask[j], xn.row);
     dst = P.act_routed + static_cast<size_t>(j) * kMaxRows * P.F;
     ld = P.F;
   } else {
@@ -956,14 +1061,14 @@ template <int MJ>
 MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit) {
   const Params &P = *w.P;
   const int seg = unit / P.n_hb, row0 = (unit % P.n_hb) * kRows;
-  const int U = n_union(P, layer);
-  const Routing *rt = P.routing + layer;
+  const int U = n_union(w);
+  const RouteCache *rt = w.rc;
   XPlain<MJ> xs;
   int K;
   if (seg < U) {
     xs.src = P.act_routed + static_cast<size_t>(seg) * kMaxRows * P.F;
     xs.ld = P.F;
-    xs.n = rows_of_mask<MJ>(__ldcg(&rt->rowmask[seg]), xs.row);
+    xs.n = rows_of_mask<MJ>(rt->rowmask[seg], xs.row);
     K = P.F;
   } else {
     xs.src = P.act_shared;
@@ -977,7 +1082,7 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit) {
   const int q = w.lane / kRows, r = w.lane % kRows;
   if (w.lane < kRows * xs.n && row0 + r < P.d) {
     const int m = row_at<MJ>(xs.row, q);
-    const int s = (seg < U) ? static_cast<int>(__ldcg(&rt->kslot[seg][m])) : P.topk;
+    const int s = (seg < U) ? static_cast<int>(rt->kslot[seg][m]) : P.topk;
     __stcg(&P.y_part[(static_cast<size_t>(m) * (P.topk + 1) + s) * P.d + row0 + r], wb[r * MJ + q]);
   }
   __syncwarp();
@@ -990,10 +1095,10 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
   const Params &P = *w.P;
   int cnt;
   if (type == OP_ROUTED_GU) {
-    cnt = __popc(__ldcg(&P.routing[layer].rowmask[unit / (P.F / kRows)]));
+    cnt = __popc(w.rc->rowmask[unit / (P.F / kRows)]);
   } else if (type == OP_DOWN) {
     const int seg = unit / P.n_hb;
-    cnt = seg < n_union(P, layer) ? __popc(__ldcg(&P.routing[layer].rowmask[seg])) : P.M;
+    cnt = seg < n_union(w) ? __popc(w.rc->rowmask[seg]) : P.M;
   } else {
     cnt = P.M;  // shared gate/up
   }
@@ -1021,16 +1126,27 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
 }
 
 // --- attention ---------------------------------------------------------------
-template <int QVP, int DPL>
-MK_INLINE bool attn_item_run(Warp &w, int op, int layer, const AttnItem &a) {
+// One warp's share of an item: online softmax over its positions for the kQvp
+// query vectors of the item's group, left in registers (lane l keeps the
+// running (max, sum) of query l % kQvp, and o for all of them over its dims).
+template <int DPL>
+MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, float &m_run, float &l_run,
+                         float (&o)[kQvp][DPL]) {
   const Params &P = *w.P;
-  constexpr int PG = 32 / QVP;  // positions per butterfly group
+  constexpr int QVP = kQvp, PG = 32 / QVP;  // positions per butterfly group
   constexpr int hd = 32 * DPL, half = hd / 2;
   const int G = P.Hq / P.Hkv;
   const int pos_b = __ldg(&P.positions[a.b]);
   const int W3 = (P.Hq + 2 * P.Hkv) * hd;
   const float scale = 1.0f / sqrtf(static_cast<float>(hd));
   const int lane = w.lane, ppos = lane & 15;
+  m_run = -INFINITY;
+  l_run = 0.f;
+#pragma unroll
+  for (int v = 0; v < QVP; ++v)
+#pragma unroll
+    for (int dd = 0; dd < DPL; ++dd) o[v][dd] = 0.f;
+  if (a.ntiles == 0) return true;
   // query vectors of this item: qv = qs*QVP + v  ->  (t = qv / G, head = g*G + qv % G)
   float q[QVP][DPL];
   int lim[QVP];
@@ -1054,12 +1170,6 @@ MK_INLINE bool attn_item_run(Warp &w, int op, int layer, const AttnItem &a) {
       }
     }
   }
-  float m_run = -INFINITY, l_run = 0.f;
-  float o[QVP][DPL];
-#pragma unroll
-  for (int v = 0; v < QVP; ++v)
-#pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) o[v][dd] = 0.f;
   const int my_qv = lane % QVP;
   int my_lim = -1;
 #pragma unroll
@@ -1074,7 +1184,7 @@ MK_INLINE bool attn_item_run(Warp &w, int op, int layer, const AttnItem &a) {
     __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(slot);
     __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(slot + kKvBoxBytes);
     // New positions of this step inside the tile: rotate k, round k and v to
-    // bf16, patch the tile and (once per chunk) append them to the cache.
+    // bf16, patch the tile and (once per group) append them to the cache.
     const int lo = max(pos0, pos_b), hi = min(pos0 + P.attn_ppt, pos_b + P.T);
     for (int p = lo; p < hi; ++p) {
       const int t = p - pos_b, m = a.b * P.T + t;
@@ -1108,22 +1218,22 @@ MK_INLINE bool attn_item_run(Warp &w, int op, int layer, const AttnItem &a) {
         for (int dd = 0; dd < DPL; ++dd) kf[dd] = __bfloat162float(kr[dd]);
 #pragma unroll
         for (int v = 0; v < QVP; ++v) {
-          float s = 0.f;
+          float sc = 0.f;
 #pragma unroll
-          for (int dd = 0; dd < DPL; ++dd) s = fmaf(q[v][dd], kf[dd], s);
-          part[j * QVP + v] = s;
+          for (int dd = 0; dd < DPL; ++dd) sc = fmaf(q[v][dd], kf[dd], sc);
+          part[j * QVP + v] = sc;
         }
       }
       butterfly<32>(part, lane);
       // lane holds the score of position jg + lane / QVP for query lane % QVP
       const int pos = pos0 + jg + lane / QVP;
       const bool valid = (pos <= my_lim) && (pos < a.pos0 + a.npos);
-      const float s = valid ? part[0] : -INFINITY;
-      float mx = s;
+      const float sc = valid ? part[0] : -INFINITY;
+      float mx = sc;
 #pragma unroll
       for (int o2 = QVP; o2 < 32; o2 <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
       const float m_new = fmaxf(m_run, mx);
-      const float pr = valid ? expf(s - m_new) : 0.f;
+      const float pr = valid ? expf(sc - m_new) : 0.f;
       const float alpha = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
       float ps = pr;
 #pragma unroll
@@ -1152,131 +1262,126 @@ MK_INLINE bool attn_item_run(Warp &w, int op, int layer, const AttnItem &a) {
     }
     consume_end(w);
   }
-  // partial of this chunk
-  const int grp = (a.b * P.Hkv + a.g) * P.attn_qsplit + a.qs;
-  const size_t pidx = static_cast<size_t>(grp) * P.attn_nch_max + a.c;
-#pragma unroll
-  for (int v = 0; v < QVP; ++v)
-#pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) __stcg(&P.attn_o[(pidx * QVP + v) * hd + lane * DPL + dd], o[v][dd]);
-  if (lane < QVP) {
-    float *ml = P.attn_ml + (static_cast<size_t>(grp) * QVP + lane) * 2 * P.attn_nch_max;
-    __stcg(ml + a.c, m_run);
-    __stcg(ml + P.attn_nch_max + a.c, l_run);
-  }
   return true;
 }
 
-// Merge n (<= 16) partials (m_i, l_i, o_i) of each query vector: level 1
-// keeps the unnormalised (max, sum, weighted o); level 2 writes o / l.
-template <int QVP, int DPL>
-__device__ __noinline__ void attn_merge(const Params &P, int lane, int grp, int first, int n, int nstride,
-                                        const float *src_o, const float *src_ml, float *dst_o, float *dst_ml,
-                                        int dst_index, int dst_stride, bool final_level, int b, int g) {
+MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op);
+
+// Shared-memory scratch of the attention items of one CTA.
+struct AttnShared {
+  float *o;           // [8 warps][kQvp][hd] warp partials (the staging row's space)
+  float *ml;          // [8 warps][kQvp][2]
+  int *last;          // this CTA completed its group
+  uint32_t *rdv;      // rendezvous counter
+  uint32_t *seq;      // this warp's rendezvous count
+};
+
+// Final merge of one query vector over the nch CTA partials of its group:
+// o = sum_i e^(m_i - M) o_i / sum_i e^(m_i - M) l_i  (one lane per partial for
+// (m, l); the o partials are read 8 at a time, all in flight together).
+template <int DPL>
+MK_INLINE void attn_final_merge(const Params &P, int lane, int grp, int v, int nch, int b, int g) {
   constexpr int hd = 32 * DPL;
   const int G = P.Hq / P.Hkv;
-  float mi[QVP], li[QVP];
+  const int qv = (grp % P.attn_qsplit) * kQvp + v;
+  if (qv >= G * P.T) return;
+  const float *mrow = P.attn_ml + (static_cast<size_t>(grp) * kQvp + v) * 2 * P.attn_nch_max;
+  const float mi = lane < nch ? __ldcg(mrow + lane) : -INFINITY;
+  const float li = lane < nch ? __ldcg(mrow + P.attn_nch_max + lane) : 0.f;
+  const float M = warp_max(mi);
+  const float wi = (lane < nch && mi != -INFINITY) ? expf(mi - M) : 0.f;
+  const float L = warp_sum(wi * li);
+  float acc[DPL];
 #pragma unroll
-  for (int v = 0; v < QVP; ++v) {
-    const float *mrow = src_ml + (static_cast<size_t>(grp) * QVP + v) * 2 * nstride;
-    mi[v] = lane < n ? __ldcg(mrow + first + lane) : -INFINITY;
-    li[v] = lane < n ? __ldcg(mrow + nstride + first + lane) : 0.f;
-  }
-#pragma unroll 1
-  for (int v2 = 0; v2 < QVP; v2 += 2) {
-    // two query vectors per pass: all their partial loads are in flight together
-    float val[2][kL1Fan][DPL];
+  for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
+  for (int i0 = 0; i0 < nch; i0 += 8) {
+    float val[8][DPL];
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2)
+    for (int k = 0; k < 8; ++k) {
+      const float *op = P.attn_o + ((static_cast<size_t>(grp) * P.attn_nch_max + i0 + k) * kQvp + v) * hd + lane * DPL;
 #pragma unroll
-      for (int i = 0; i < kL1Fan; ++i) {
-        const float *op = src_o + ((static_cast<size_t>(grp) * nstride + first + i) * QVP + v2 + h2) * hd + lane * DPL;
+      for (int dd = 0; dd < DPL; ++dd) val[k][dd] = (i0 + k < nch) ? __ldcg(op + dd) : 0.f;
+    }
 #pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) val[h2][i][dd] = (i < n) ? __ldcg(op + dd) : 0.f;
-      }
+    for (int k = 0; k < 8; ++k) {
+      const float wv = __shfl_sync(0xffffffffu, wi, (i0 + k) & 31);
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      const int v = v2 + h2;
-      float mv = -INFINITY, lv = 0.f;
-#pragma unroll
-      for (int vv = 0; vv < QVP; ++vv)
-        if (vv == v) {
-          mv = mi[vv];
-          lv = li[vv];
-        }
-      const float M = warp_max(mv);
-      const float wi = (lane < n && mv != -INFINITY) ? expf(mv - M) : 0.f;
-      const float L = warp_sum(wi * lv);
-      float acc[DPL];
-#pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
-#pragma unroll
-      for (int i = 0; i < kL1Fan; ++i) {
-        const float wv = __shfl_sync(0xffffffffu, wi, i);
-#pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(wv, val[h2][i][dd], acc[dd]);
-      }
-      if (!final_level) {
-        float *dop = dst_o + ((static_cast<size_t>(grp) * dst_stride + dst_index) * QVP + v) * hd + lane * DPL;
-#pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) __stcg(dop + dd, acc[dd]);
-        if (lane == 0) {
-          float *dml = dst_ml + (static_cast<size_t>(grp) * QVP + v) * 2 * dst_stride;
-          __stcg(dml + dst_index, M);
-          __stcg(dml + dst_stride + dst_index, L);
-        }
-      } else {
-        const int qv = (grp % P.attn_qsplit) * QVP + v;
-        if (qv < G * P.T) {
-          const int t = qv / G, head = g * G + qv % G, m = b * P.T + t;
-          const float invl = 1.0f / L;
-          float *dst = P.o + static_cast<size_t>(m) * P.Hq * hd + head * hd + lane * DPL;
-#pragma unroll
-          for (int dd = 0; dd < DPL; ++dd) __stcg(dst + dd, acc[dd] * invl);
-        }
-      }
+      for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(wv, val[k][dd], acc[dd]);
     }
   }
+  const int t = qv / G, head = g * G + qv % G, m = b * P.T + t;
+  const float invl = 1.0f / L;
+  float *dst = P.o + static_cast<size_t>(m) * P.Hq * hd + head * hd + lane * DPL;
+#pragma unroll
+  for (int dd = 0; dd < DPL; ++dd) __stcg(dst + dd, acc[dd] * invl);
 }
 
-// Arrival on a merge counter; true for the last of `n` arrivals (resets it).
-MK_INLINE bool merge_arrive(int lane, uint32_t *ctr, int n) {
-  __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    __threadfence();
-    const uint32_t old = atom_add_acq_rel(ctr, 1u);
-    if (old + 1 == static_cast<uint32_t>(n)) last = 1;
-  }
-  last = __shfl_sync(0xffffffffu, last, 0);
-  if (last) {
-    // every lane observes the final count, then lane 0 rewinds the counter
-    (void)ld_relaxed(ctr);
-    fence_acq_rel();
-    __syncwarp();
-    if (lane == 0) *ctr = 0;
-  }
-  __syncwarp();
-  return last != 0;
-}
-
-template <int QVP, int DPL>
-MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item) {
+// One CTA-wide attention item: every warp computes its share, warps 0..3 merge
+// the 8 shares of one query vector each into the CTA's partial, and the CTA
+// that completes the group merges all CTA partials into o.
+template <int DPL>
+MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
   const Params &P = *w.P;
-  const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, item);
-  if (!attn_item_run<QVP, DPL>(w, op, layer, a)) return false;
+  constexpr int hd = 32 * DPL;
+  const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, item, w.wib);
+  float m_run, l_run, o[kQvp][DPL];
+  if (!attn_warp<DPL>(w, op, layer, a, m_run, l_run, o)) return false;
+#pragma unroll
+  for (int v = 0; v < kQvp; ++v)
+#pragma unroll
+    for (int dd = 0; dd < DPL; ++dd) sh.o[(w.wib * kQvp + v) * hd + w.lane * DPL + dd] = o[v][dd];
+  if (w.lane < kQvp) {
+    sh.ml[(w.wib * kQvp + w.lane) * 2] = m_run;
+    sh.ml[(w.wib * kQvp + w.lane) * 2 + 1] = l_run;
+  }
+  *sh.seq += kWarpsPerCta;
+  if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   const int grp = (a.b * P.Hkv + a.g) * P.attn_qsplit + a.qs;
-  const int nch = w.attn_nch[a.b];
-  const int k1 = a.c / kL1Fan, n1 = min(kL1Fan, nch - k1 * kL1Fan), ngrp1 = cdiv(nch, kL1Fan);
-  uint32_t *c1 = P.attn_cnt + static_cast<size_t>(grp) * (kL1Fan + 1) + k1;
-  if (merge_arrive(w.lane, c1, n1)) {
-    attn_merge<QVP, DPL>(P, w.lane, grp, k1 * kL1Fan, n1, P.attn_nch_max, P.attn_o, P.attn_ml, P.attn_o1,
-                         P.attn_ml1, k1, kL1Fan, false, a.b, a.g);
-    uint32_t *c2 = P.attn_cnt + static_cast<size_t>(grp) * (kL1Fan + 1) + kL1Fan;
-    if (merge_arrive(w.lane, c2, ngrp1)) {
-      attn_merge<QVP, DPL>(P, w.lane, grp, 0, ngrp1, kL1Fan, P.attn_o1, P.attn_ml1, nullptr, nullptr, 0, 0, true,
-                           a.b, a.g);
+  if (w.wib < kQvp) {
+    const int v = w.wib;
+    float mw[kWarpsPerCta], M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kWarpsPerCta; ++k) {
+      mw[k] = sh.ml[(k * kQvp + v) * 2];
+      M = fmaxf(M, mw[k]);
     }
+    float L = 0.f, acc[DPL];
+#pragma unroll
+    for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
+#pragma unroll
+    for (int k = 0; k < kWarpsPerCta; ++k) {
+      const float e = (mw[k] == -INFINITY) ? 0.f : expf(mw[k] - M);
+      L += e * sh.ml[(k * kQvp + v) * 2 + 1];
+#pragma unroll
+      for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(e, sh.o[(k * kQvp + v) * hd + w.lane * DPL + dd], acc[dd]);
+    }
+    float *dop = P.attn_o + ((static_cast<size_t>(grp) * P.attn_nch_max + a.c) * kQvp + v) * hd + w.lane * DPL;
+#pragma unroll
+    for (int dd = 0; dd < DPL; ++dd) __stcg(dop + dd, acc[dd]);
+    if (w.lane == 0) {
+      float *ml = P.attn_ml + (static_cast<size_t>(grp) * kQvp + v) * 2 * P.attn_nch_max;
+      __stcg(ml + a.c, M);
+      __stcg(ml + P.attn_nch_max + a.c, L);
+    }
+  }
+  *sh.seq += kWarpsPerCta;
+  if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
+  uint32_t *cnt = P.attn_cnt + grp;
+  if (w.wib == 0 && w.lane == 0) {
+    __threadfence();
+    *reinterpret_cast<volatile int *>(sh.last) = (atom_add_acq_rel(cnt, 1u) + 1 == static_cast<uint32_t>(a.nch)) ? 1 : 0;
+  }
+  *sh.seq += kWarpsPerCta;
+  if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
+  if (*reinterpret_cast<volatile int *>(sh.last)) {
+    if (w.wib < kQvp) {
+      (void)ld_relaxed(cnt);  // every lane observes the completed count
+      fence_acq_rel();
+      attn_final_merge<DPL>(P, w.lane, grp, w.wib, a.nch, a.b, a.g);
+    }
+    *sh.seq += kWarpsPerCta;
+    if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
+    if (w.wib == 0 && w.lane == 0) *cnt = 0;  // rewind for the next layer
   }
   return true;
 }
@@ -1289,15 +1394,10 @@ __device__ __noinline__ void router_topk(const Params &P, int lane, uint32_t epo
   const int E = P.E, K = P.topk;
   const int nkc = cdiv(P.d, kTileCols);
   constexpr int EPL = 8;
-  uint32_t rmask[EPL];
-  int8_t kslot[EPL][kMaxRows];
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    rmask[i] = 0;
-#pragma unroll
-    for (int m = 0; m < kMaxRows; ++m) kslot[i][m] = -1;
-  }
   Routing *rt = P.routing + layer;
+  uint32_t chosen[EPL];  // rows that selected each of this lane's experts
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) chosen[i] = 0;
   for (int m = 0; m < P.M; ++m) {
     // logits = sum of the K-chunk partials in a fixed order; loads issued together
     float z[EPL];
@@ -1337,9 +1437,9 @@ __device__ __noinline__ void router_topk(const Params &P, int lane, uint32_t epo
     sum = warp_sum(sum);
 #pragma unroll
     for (int i = 0; i < EPL; ++i) pi[i] = pi[i] / sum;
-    float sel = 0.f;
-    int ids[kMaxTopK];
-    float ws[kMaxTopK];
+    // k rounds of argmax (ties to the lower expert id); lane j keeps selection j
+    float sel = 0.f, my_w = 0.f;
+    int my_e = 0;
     for (int j = 0; j < K; ++j) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
@@ -1364,56 +1464,29 @@ __device__ __noinline__ void router_topk(const Params &P, int lane, uint32_t epo
       for (int i = 0; i < EPL; ++i)
         if (expert_of(lane, i) == bi) {
           taken[i] = true;
-          rmask[i] |= (1u << m);
-#pragma unroll
-          for (int mm = 0; mm < kMaxRows; ++mm)
-            if (mm == m) kslot[i][mm] = static_cast<int8_t>(j);
+          chosen[i] |= 1u << m;
         }
-      ids[j] = bi;
-      ws[j] = bv;
+      if (lane == j) {
+        my_e = bi;
+        my_w = bv;
+      }
       sel += bv;
     }
-    if (lane == 0) {
-      for (int j = 0; j < K; ++j) {
-        const float wn = ws[j] / sel;
-        rt->row_e[m][j] = ids[j];
-        rt->row_w[m][j] = wn;
-        if (P.dbg_ids) P.dbg_ids[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = ids[j];
-        if (P.dbg_w) P.dbg_w[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = wn;
-      }
+    if (lane < K) {
+      const float wn = my_w / sel;
+      rt->row_e[m][lane] = my_e;
+      rt->row_w[m][lane] = wn;
+      if (P.dbg_ids) P.dbg_ids[(static_cast<size_t>(layer) * P.max_rows + m) * K + lane] = my_e;
+      if (P.dbg_w) P.dbg_w[(static_cast<size_t>(layer) * P.max_rows + m) * K + lane] = wn;
     }
   }
-  // publish the union in ascending expert order (block 0, then block 1;
-  // inside a block lane-major, slot-minor)
-  int base = 0;
+  int nu = 0;
 #pragma unroll
-  for (int blk = 0; blk < 2; ++blk) {
-    int cnt = 0;
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq) cnt += rmask[blk * 4 + qq] != 0 ? 1 : 0;
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    int pos = base + incl - cnt;
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq) {
-      const int i = blk * 4 + qq;
-      if (rmask[i] != 0) {
-        rt->expert[pos] = expert_of(lane, i);
-        rt->rowmask[pos] = rmask[i];
-#pragma unroll
-        for (int m = 0; m < kMaxRows; ++m) rt->kslot[pos][m] = kslot[i][m];
-        ++pos;
-      }
-    }
-    base += __shfl_sync(0xffffffffu, incl, 31);
-  }
+  for (int i = 0; i < EPL; ++i) nu += chosen[i] ? 1 : 0;
+  nu = static_cast<int>(warp_sum(static_cast<float>(nu)));
   if (lane == 0) {
-    rt->n_union = base;
-    atomicAdd(&P.stats[0], static_cast<unsigned long long>(base));
+    rt->n_union = nu;
+    atomicAdd(&P.stats[0], static_cast<unsigned long long>(nu));
   }
   __syncwarp();
   if (lane == 0) {
@@ -1517,23 +1590,25 @@ MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, u
 }
 
 template <int MMAX, bool XS>
-MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, float &am_val, int &am_idx) {
+MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, AttnShared &ash, float &am_val,
+                           int &am_idx) {
   const Params &P = *w.P;
-  const int u0 = first_unit_of(w.slot, op, w.nw);
-  const int n = unit_count_of(u0, op_total_units(w, type, layer), w.nw);
+  if ((type == OP_ROUTED_GU || type == OP_DOWN) && !route_cache(w, layer)) return false;
+  // attention items are CTA-wide: all warps of a CTA work on the same items
+  const bool cta_items = type == OP_ATTN;
+  const int stride = cta_items ? P.n_cta : w.nw;
+  const int u0 = cta_items ? w.cta : first_unit_of(w.slot, op, w.nw);
+  const int n = unit_count_of(u0, op_total_units(w, type, layer), stride);
   if (n == 0) return true;
   float inv[kMaxRows];
 #pragma unroll
   for (int m = 0; m < kMaxRows; ++m) inv[m] = 0.f;
   if (type != OP_OPROJ && type != OP_DOWN && type != OP_ATTN) compute_inv_rms(P, w.lane, inv);
   for (int i = 0; i < n; ++i) {
-    const int u = u0 + i * w.nw;
+    const int u = u0 + i * stride;
     bool ok;
     if (type == OP_ATTN) {
-      if (P.hd == 64)
-        ok = (P.attn_qvp == 8) ? attn_unit<8, 2>(w, op, layer, u) : attn_unit<4, 2>(w, op, layer, u);
-      else
-        ok = (P.attn_qvp == 8) ? attn_unit<8, 4>(w, op, layer, u) : attn_unit<4, 4>(w, op, layer, u);
+      ok = (P.hd == 64) ? attn_unit<2>(w, op, layer, u, ash) : attn_unit<4>(w, op, layer, u, ash);
     } else if (type == OP_ROUTED_GU || type == OP_DOWN || type == OP_SHARED_GU) {
       ok = routed_dispatch<MMAX, XS>(w, op, type, layer, u, inv, xs);
     } else {
@@ -1550,9 +1625,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   __shared__ int s_attn_prefix[kMaxRows + 1];
   __shared__ int s_attn_nch[kMaxRows];
   __shared__ uint32_t s_stage;
+  __shared__ RouteCache s_route;
+  __shared__ float s_attn_ml[kWarpsPerCta * kQvp * 2];
+  __shared__ int s_attn_last;
   const int wib = threadIdx.x >> 5;
   Warp w;
   w.P = &P;
+  w.rc = &s_route;
+  w.wib = wib;
+  w.cta = blockIdx.x;
   w.lane = threadIdx.x & 31;
   w.nw = P.n_warps;
   w.slot = wib * P.n_cta + blockIdx.x;
@@ -1577,16 +1658,19 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   for (int i = threadIdx.x; i < P.n_ops; i += kThreads) w.arrive[i] = 0;
   if (threadIdx.x == 0) {
     s_stage = 0;
+    s_route.ready_key = s_route.fill_key = 0;
+    s_attn_last = 0;
     // attention work items per sequence
     s_attn_prefix[0] = 0;
     for (int b = 0; b < kMaxRows; ++b) {
-      const int nch = b < P.B ? cdiv(__ldg(&P.positions[b]) + P.T, P.attn_chunk) : 0;
+      const int nch = b < P.B ? cdiv(__ldg(&P.positions[b]) + P.T, P.attn_chunk * kWarpsPerCta) : 0;
       s_attn_nch[b] = nch;
       s_attn_prefix[b + 1] = s_attn_prefix[b] + P.Hkv * P.attn_qsplit * nch;
     }
   }
   __syncthreads();
   uint32_t stage_seq = 0;
+  AttnShared ash{xs, s_attn_ml, &s_attn_last, &s_stage, &stage_seq};
 
   w.epoch = *reinterpret_cast<volatile const uint32_t *>(P.epoch) + 1u;
 
@@ -1641,9 +1725,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     if (type == OP_EMBED) {
       op_embed(w);
     } else if (type == OP_COMBINE) {
-      op_combine(w, layer);
+      ok = route_cache(w, layer);
+      if (ok) op_combine(w, layer);
     } else {
-      ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, am_val, am_idx);
+      ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, ash, am_val, am_idx);
     }
     if (!ok || w.failed) break;
     if (type == OP_LMHEAD && (w.lane % kRows) == 0 && w.lane / kRows < P.M) {
