@@ -86,16 +86,66 @@ def barrier(device):
 
 
 # ---- clocks -----------------------------------------------------------------------
+# Throttle-reason bits of NVML's clocks-event mask (read only; nothing is set).
+_REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+
 class ClockSampler:
+    """Samples the SM clock and the throttle reasons every 10 ms during the
+    timed region (NVML from a thread; nvidia-smi at its 200 ms floor if NVML is
+    unavailable).  Only reads the GPU's state."""
+
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.01):
         self.gpu = gpu_index
+        self.period = period_s
         self.proc = None
+        self.thread = None
+        self.samples = []
+        self.max_mhz = None
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        import threading
+
+        try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            self._start_smi()
+            return
+        self.stop_flag = threading.Event()
+
+        def run():
+            while not self.stop_flag.is_set():
+                try:
+                    self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                         int(reasons_fn(h))))
+                except Exception:
+                    pass
+                self.stop_flag.wait(self.period)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def _start_smi(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
@@ -105,6 +155,16 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            reasons = sorted({name for _, mask in self.samples for bit, name in _REASON_BITS.items()
+                              if mask & bit})
+            return {"sm_mhz": statistics.median(s for s, _ in self.samples),
+                    "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "samples": len(self.samples), "source": "nvml, 10 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -126,7 +186,7 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(rows)}
+                "reasons": sorted(reasons), "samples": len(rows), "source": "nvidia-smi, 200 ms"}
 
 
 # ---- bytes per step ---------------------------------------------------------------
@@ -246,10 +306,12 @@ def time_e2e(dec, m, k, v, B, T, ctx, steps, warmup):
     return dt, (th.numel() + ph.numel()) * 4, out.numel() * 4
 
 
-def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1):
+def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1, min_compute_s=0.0):
     """The CPU oracle as it stands on the same workload: whole decode steps
     (all layers), weights copied from the device on demand; the copy time is
-    excluded from the compute time and reported beside it."""
+    excluded from the compute time and reported beside it.  Runs ``n_steps``
+    steps, or more until the compute time reaches ``min_compute_s`` (at most
+    40 steps)."""
     import numpy as np
 
     import oracle
@@ -277,15 +339,17 @@ def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1):
 
     timed.fetch = 0.0
     src._get = timed
-    for _ in range(n_steps):
+    done = 0
+    while done < n_steps or (t_total - timed.fetch < min_compute_s and done < 40):
         t0 = _t.perf_counter()
         r = ostep.decode_step(m, src, kh, vh, toks, pos, B, T)
         t_total += _t.perf_counter() - t0
         toks = [int(x) for x in r.argmax]
         pos = [p + T for p in pos]
+        done += 1
     compute = t_total - timed.fetch
-    return {"compute_s": compute, "fetch_s": timed.fetch, "steps": n_steps, "threads": threads,
-            "tokens": n_steps * B * T}
+    return {"compute_s": compute, "fetch_s": timed.fetch, "steps": done, "threads": threads,
+            "tokens": done * B * T}
 
 
 def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr):
@@ -393,10 +457,11 @@ def run_mine(args):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        o = oracle_sample(m, w, k, v, B, T, ctx, 1)
+        o = oracle_sample(m, w, k, v, B, T, ctx, 1, min_compute_s=10.0)
         cpu = {"value": round(o["tokens"] / o["compute_s"], 4), "unit": "tokens/s",
                "cores": o["threads"], "kind": "oracle",
-               "sample": (f"{o['steps']} full decode step(s) of the same workload on the host "
+               "sample": (f"{o['steps']} consecutive greedy decode steps of the same workload "
+                          f"(all layers, from the same cache) on the host "
                           f"(compute {o['compute_s']:.2f} s; weight copy from the device "
                           f"{o['fetch_s']:.2f} s excluded)")}
 
