@@ -34,6 +34,7 @@ VARIANTS = {"megakernel": MK_MEGAKERNEL, "multikernel": MK_MULTIKERNEL,
 
 MK_FAULT_NONE = 0
 MK_FAULT_UNREACHABLE_WAIT = 1
+MK_STATIC_SCRATCH_BYTES = 32 << 20  # the fixed working array of mk_decode_step_static
 
 OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE",
             "LMHEAD"]
@@ -97,6 +98,7 @@ def lib():
         "mk_create": (i32, [ctypes.POINTER(mk_model_desc), ctypes.POINTER(mk_weights), ctypes.POINTER(vp)]),
         "mk_decode_step": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
         "mk_decode_step_host": (i32, [vp, _I32P, _I32P, i32, i32, mk_kv_cache, vp, _I32P, vp]),
+        "mk_decode_step_static": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
         "mk_get_device_status": (i32, [vp, vp]),
         "mk_last_device_error_op": (i32, [vp]),
         "mk_last_error": (ctypes.c_char_p, []),
@@ -161,6 +163,12 @@ def mk_decode_step_host(h, tokens_host, positions_host, B: int, T: int, kv: mk_k
                         out_logits: int, out_argmax_host, stream: int) -> int:
     return lib().mk_decode_step_host(h, tokens_host, positions_host, B, T, kv, out_logits,
                                      out_argmax_host, stream)
+
+
+def mk_decode_step_static(h, tokens: int, positions: int, B: int, T: int, kv: mk_kv_cache,
+                          out_logits: int, out_argmax: int, stream: int) -> int:
+    return lib().mk_decode_step_static(h, tokens, positions, B, T, kv, out_logits, out_argmax,
+                                       stream)
 
 
 def mk_get_device_status(h, stream: int) -> int:
@@ -272,6 +280,15 @@ class Decoder:
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_step(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
                               _ptr(logits), argmax.data_ptr(), s.cuda_stream)
+
+    def step_static(self, tokens, positions, B: int, T: int, k_cache, v_cache, logits, argmax,
+                    stream=None) -> int:
+        """Like ``step``, but the step's working memory is the library's fixed
+        device array (no allocation; overlapping calls on one device race)."""
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
+        return mk_decode_step_static(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
+                                     _ptr(logits), argmax.data_ptr(), s.cuda_stream)
 
     def step_host(self, tokens_host, positions_host, B: int, T: int, k_cache, v_cache,
                   argmax_host, logits=None, stream=None) -> int:

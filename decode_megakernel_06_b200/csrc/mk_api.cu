@@ -647,3 +647,102 @@ MK_API int mk_get_stats(mk_handle *h, mk_stats *out, int32_t reset) {
 }
 
 }  // extern "C"
+
+// ---- step without allocation ----------------------------------------------------
+// Per-step working memory of mk_decode_step_static.  The array belongs to this
+// module, so it exists on a device as soon as the module is loaded there and no
+// call has to allocate it.  Every call on a device uses the same array.
+static __device__ __align__(256) unsigned char g_static_scratch[MK_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxStaticDevices = 64;
+std::mutex g_static_mu;
+void *g_static_base[kMaxStaticDevices];  // the array's address on each device, once resolved
+
+// Address of the array on `dev` (the current device); resolved on the first
+// call for that device.
+int static_scratch_base(int dev, unsigned char **out) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (dev < 0 || dev >= kMaxStaticDevices)
+    return fail(MK_ERR_UNSUPPORTED, "device %d: the static scratch serves devices 0..%d", dev, kMaxStaticDevices - 1);
+  if (!g_static_base[dev]) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(MK_ERR_CUDA, "cudaGetSymbolAddress(static scratch) on device %d failed: %s", dev,
+                  cudaGetErrorString(e));
+    g_static_base[dev] = p;
+  }
+  *out = static_cast<unsigned char *>(g_static_base[dev]);
+  return MK_OK;
+}
+
+// Bump layout of the per-step buffers inside the array (256-byte aligned).
+struct StaticCarve {
+  size_t used = 0;
+  template <typename T>
+  void take(T *&ptr, unsigned char *base, size_t bytes) {
+    ptr = reinterpret_cast<T *>(base + used);
+    used += (bytes + 255) / 256 * 256;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                                 int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
+                                 int32_t *out_argmax, void *stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  int dev = -1;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != h->device) return fail(MK_ERR_ARG, "device %d is current, the handle lives on device %d", dev, h->device);
+  Params p;
+  Plan pl;
+  int rc = fill_params(h, tokens, positions, B, T, kv, out_logits, out_argmax, p, pl);
+  if (rc) return rc;
+  unsigned char *base = nullptr;
+  rc = static_scratch_base(dev, &base);
+  if (rc) return rc;
+
+  const mk_model_desc &d = h->desc;
+  const int L = d.n_layers, D = d.d_model, QKVW = (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim;
+  const size_t ngrp = (size_t)B * d.n_kv_heads * pl.attn_qsplit;
+  const int umax = std::min(d.n_experts, d.max_rows * d.top_k);
+  StaticCarve c;
+  // words that must read zero when the step starts, first, so one memset clears them
+  c.take(p.counters, base, sizeof(uint32_t) * (size_t)pl.n_ops * kCounterStride);
+  c.take(p.route_flag, base, sizeof(uint32_t) * (size_t)L * kCounterStride);
+  c.take(p.epoch, base, sizeof(uint32_t) * kCounterStride);
+  c.take(p.attn_cnt, base, sizeof(uint32_t) * ngrp);
+  const size_t zero_bytes = c.used;
+  // buffers every step writes before it reads them
+  c.take(p.h, base, sizeof(float) * (size_t)kMaxRows * D);
+  c.take(p.ss, base, sizeof(float) * (size_t)kMaxRows * p.ss_ld);
+  c.take(p.qkv, base, sizeof(float) * (size_t)kMaxRows * QKVW);
+  c.take(p.o, base, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
+  c.take(p.attn_o, base, sizeof(float) * ngrp * pl.attn_nch_max * kQvp * d.head_dim);
+  c.take(p.attn_ml, base, sizeof(float) * ngrp * kQvp * 2 * pl.attn_nch_max);
+  c.take(p.router_part, base, sizeof(float) * (size_t)ceil_div(D, kTileCols) * kMaxRows * p.e_ld);
+  c.take(p.routing, base, sizeof(Routing) * (size_t)L);
+  c.take(p.act_shared, base, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
+  c.take(p.act_routed, base, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
+  c.take(p.y_part, base, sizeof(float) * (size_t)kMaxRows * (d.top_k + 1) * D);
+  c.take(p.am_part, base, sizeof(ArgmaxPart) * (size_t)pl.n_warps * kMaxRows);
+  if (!out_logits) c.take(p.logits, base, sizeof(float) * (size_t)B * T * d.vocab);
+  if (c.used > (size_t)MK_STATIC_SCRATCH_BYTES)
+    return fail(MK_ERR_CAPACITY, "this step needs %zu bytes of working memory; the static scratch holds %u",
+                c.used, (unsigned)MK_STATIC_SCRATCH_BYTES);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUDA_TRY(cudaMemsetAsync(base, 0, zero_bytes, s));
+  int e = launch_step(p, pl.mmax, true, s);
+  if (e) return fail(MK_ERR_LAUNCH, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
+  h->stats.kernel_launches += 1;
+  h->stats.steps += 1;
+  return MK_OK;
+}
+
+}  // extern "C"

@@ -177,6 +177,42 @@ MK_API int mk_decode_step_host(mk_handle *h, const int32_t *tokens_host,
                                mk_kv_cache kv, float *out_logits, int32_t *out_argmax_host,
                                void *stream);
 
+/* Size of the fixed device array that mk_decode_step_static works in. */
+#define MK_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* The decode step of mk_decode_step, run as the megakernel (one persistent
+ * launch, whatever variant the handle is set to), without allocating.
+ * The megakernel pages have no counterpart for this call; it exists for
+ * callers that must not allocate device memory when they step, for example a
+ * serving process that hands every free byte of the device to its own
+ * KV-cache pool once its models are loaded, where a later cudaMalloc fails.
+ *
+ * Arguments, their layout and ownership are those of mk_decode_step.  The
+ * step's working memory (hidden rows, projections, attention partials,
+ * routing, expert activations, the synchronisation counters, and the logits
+ * when out_logits is NULL) comes from one array of MK_STATIC_SCRATCH_BYTES in
+ * the library's device module instead of from the handle; the tensor maps,
+ * norm pointers, rotary table, device status word and statistics stay in the
+ * handle.  No call allocates or frees memory.
+ *
+ * The first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  The handle's device must be current.  Each call
+ * clears the counters that must start at zero (an asynchronous memset on
+ * `stream`), then launches the step.
+ *
+ * Every handle and stream on a device shares the one array: calls whose work
+ * overlaps on the GPU race and corrupt each other's results.  Order them on
+ * one stream, or finish one before the next starts.
+ *
+ * Errors: the host-side checks of mk_decode_step; MK_ERR_CAPACITY when the
+ * step (for this B, T and model) needs more than MK_STATIC_SCRATCH_BYTES, with
+ * the size it needs in mk_last_error(); MK_ERR_ARG when another device is
+ * current.  Device-side errors are read with mk_get_device_status. */
+MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                                 int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
+                                 int32_t *out_argmax, void *stream);
+
 /* Synchronises `stream`, then returns MK_OK or the first device-side error of
  * the steps since the last call (MK_ERR_TIMEOUT, MK_ERR_DEVICE_CHECK).  An
  * error clears the handle's synchronisation state so the next step starts
