@@ -354,7 +354,7 @@ def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1, min_compute_s=0.0):
             "tokens": done * B * T}
 
 
-def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr):
+def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr, save=None):
     """One traced step: per op, when the first / last warp started it and when
     the last warp finished it (microseconds from the step's first op start)."""
     import torch
@@ -364,7 +364,7 @@ def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr):
     n_sm = torch.cuda.get_device_properties(device).multi_processor_count
     rc, info, ops = mk.mk_plan_describe(dec.desc, n_sm, B, T)
     nw = info.n_cta * info.warps_per_cta
-    buf = torch.zeros((info.n_ops, nw, 2), dtype=torch.int64, device=device)
+    buf = torch.zeros((info.n_ops, nw, mk.MK_TRACE_WORDS), dtype=torch.int64, device=device)
     pos = torch.tensor([c for c in ctx], dtype=torch.int32, device=device)
     tok = torch.zeros(B * T, dtype=torch.int32, device=device)
     am = torch.empty(B * T, dtype=torch.int32, device=device)
@@ -372,7 +372,11 @@ def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr):
     assert dec.step(tok, pos, B, T, k, v, None, am) == 0
     assert dec.status() == 0
     dec.set_trace(None)
-    t = buf.cpu().numpy().astype("float64")
+    t = buf.cpu().numpy()[:, :, [0, 3]].astype("float64")  # (inputs ready, arrived) per warp
+    if save:
+        import numpy as np
+
+        np.save(save, buf.cpu().numpy())
     t0 = t[:, :, 0][t[:, :, 0] > 0].min()
     rows = []
     for i, (typ, layer, d0, d1) in enumerate(ops):
@@ -411,7 +415,7 @@ def run_mine(args):
     if args.trace:
         # warm, then one traced step (not part of the timed region)
         time_steps(dec, m, k, v, B, T, ctx, 1, 3, device)
-        trace_step(dec, m, k, v, B, T, ctx, device)
+        trace_step(dec, m, k, v, B, T, ctx, device, save=args.trace_out)
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -555,6 +559,8 @@ def main():
                     choices=["megakernel", "multikernel", "multikernel_graph"])
     ap.add_argument("--sweep", action=argparse.BooleanOptionalAction, default=True)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--trace-out", default=None,
+                    help="with --trace: save the raw per-op, per-warp [start, end] stamps (.npy)")
     ap.add_argument("--trace", action="store_true",
                     help="print a per-op timeline of one extra step to stderr")
     args = ap.parse_args()

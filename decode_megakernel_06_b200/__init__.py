@@ -34,6 +34,7 @@ VARIANTS = {"megakernel": MK_MEGAKERNEL, "multikernel": MK_MULTIKERNEL,
 
 MK_FAULT_NONE = 0
 MK_FAULT_UNREACHABLE_WAIT = 1
+MK_TRACE_WORDS = 8  # uint64 words per (op, warp) record of mk_set_trace
 MK_STATIC_SCRATCH_BYTES = 32 << 20  # the fixed working array of mk_decode_step_static
 
 OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE",

@@ -80,7 +80,7 @@ int encode_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, 
 struct Plan {
   int M, mmax, rows_per_tile, n_hb;
   int attn_qsplit, attn_ppt, attn_chunk, attn_nch_max;
-  int n_ops, n_cta, n_warps, xs_floats;
+  int n_ops, n_cta, n_warps, xs_floats, qkv_split, down_groups, down_staged;
   size_t smem;
 };
 
@@ -90,6 +90,18 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.mmax = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
   p.rows_per_tile = kRows;
   p.n_hb = ceil_div(d.d_model, kRows);
+  // QKV has few row blocks per warp (1536 for 1184 warps at the large model);
+  // halving K per unit evens out the warps' shares.
+  p.qkv_split = ceil_div(d.d_model, kTileCols) >= 2 ? 2 : 1;
+  // Down projection: two 4-row groups per unit when the F (or Fs) columns leave
+  // the 1024-column tiles partly empty, as long as the units still outnumber
+  // the warps two to one; the tiles then come out full.
+  {
+    const int nbx = ceil_div(d.expert_ffn, kPanel), nbs = d.shared_ffn > 0 ? ceil_div(d.shared_ffn, kPanel) : 0;
+    const bool partial = (nbx % kPanels) != 0 || (nbs % kPanels) != 0;
+    const long long units2 = (long long)(d.d_model / (2 * kRows)) * (d.top_k + (d.shared_ffn > 0 ? 1 : 0));
+    p.down_groups = (partial && units2 >= 2LL * n_sm * kWarpsPerCta) ? 2 : 1;
+  }
   const int G = d.n_q_heads / d.n_kv_heads;
   p.attn_qsplit = ceil_div(G * T, kQvp);
   p.attn_ppt = 2048 / d.head_dim;
@@ -111,6 +123,18 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   // warps' partials, whichever is larger
   p.xs_floats = std::max(kWarpsPerCta * kQvp * d.head_dim,
                          kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), 4) * 4 : 0);
+  // Batch 1 down projection: a CTA's contiguous range of units spans at most
+  // 1 + ceil(range / row blocks) experts; their activations must fit the
+  // shared-memory row.
+  p.down_staged = 0;
+  if (kernel_stages_x(p.mmax)) {
+    const int n_db = p.n_hb / p.down_groups;
+    const int segs = std::min(d.n_experts, d.top_k) + (d.shared_ffn > 0 ? 1 : 0);
+    const int per_cta = ceil_div(segs * n_db, p.n_cta);
+    const int span = 1 + ceil_div(per_cta, n_db);
+    const int fmax = std::max(d.expert_ffn, d.shared_ffn);
+    p.down_staged = (std::min(span, segs) * ceil_div(fmax, 4) * 4 <= p.xs_floats) ? 1 : 0;
+  }
   p.smem = step_smem_bytes(p.n_ops, p.xs_floats);
   return p;
 }
@@ -150,14 +174,13 @@ struct mk_handle {
   const __nv_bfloat16 **norms;
   float *h, *ss, *qkv, *o, *attn_o, *attn_ml, *router_part, *act_shared,
       *act_routed, *y_part, *logits;
-  uint32_t *attn_cnt, *counters, *route_flag, *epoch;
-  Routing *routing;
+  uint32_t *attn_cnt, *counters, *epoch;
   ArgmaxPart *am_part;
   float2 *rope;
   int *error;
   unsigned long long *stats_dev;
   int32_t *io_tokens, *io_positions, *io_argmax;
-  size_t counters_bytes, route_bytes, attn_cnt_bytes;
+  size_t counters_bytes, attn_cnt_bytes;
   // kv maps, re-encoded when the cache pointers change
   void *kv_k, *kv_v;
   CUtensorMap kmap, vmap;
@@ -231,13 +254,13 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
     const mk_model_desc &d = *desc;
     size_t f = (size_t)d.max_rows * d.d_model * 2 + (size_t)d.max_rows * ceil_div(d.d_model, kRows) +
                (size_t)kMaxRows * (d.top_k + 1) * d.d_model +
-               (size_t)d.max_rows * (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim +
+               2 * (size_t)d.max_rows * (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim +
                (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml +
                (size_t)ceil_div(d.d_model, kPanel) * kMaxRows * d.n_experts +
                (size_t)kMaxRows * d.shared_ffn +
                (size_t)std::min(d.n_experts, d.max_rows * d.top_k) * kMaxRows * d.expert_ffn +
                (size_t)d.max_rows * d.vocab + (size_t)d.kv_capacity * d.head_dim;
-    info->scratch_bytes = (int64_t)(f * 4 + s.attn_cnt * 4 + (size_t)d.n_layers * sizeof(Routing) +
+    info->scratch_bytes = (int64_t)(f * 4 + s.attn_cnt * 4 +
                                     (size_t)p.n_warps * kMaxRows * sizeof(ArgmaxPart));
   }
   for (int i = 0; i < p.n_ops && i < cap; ++i) {
@@ -331,14 +354,13 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->norms, sizeof(void *) * 2 * L);
   HALLOC(h->h, sizeof(float) * (size_t)kMaxRows * D);
   HALLOC(h->ss, sizeof(float) * (size_t)kMaxRows * ceil_div(ceil_div(D, kRows), 128) * 128);
-  HALLOC(h->qkv, sizeof(float) * (size_t)kMaxRows * QKVW);
+  HALLOC(h->qkv, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);  // [K half][row][QKVW]
   HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
   HALLOC(h->attn_o, sizeof(float) * s.attn_o);
   HALLOC(h->attn_ml, sizeof(float) * s.attn_ml);
   h->attn_cnt_bytes = sizeof(uint32_t) * s.attn_cnt;
   HALLOC(h->attn_cnt, h->attn_cnt_bytes);
   HALLOC(h->router_part, sizeof(float) * (size_t)ceil_div(D, kTileCols) * kMaxRows * ceil_div(d.n_experts, 4) * 4);
-  HALLOC(h->routing, sizeof(Routing) * (size_t)L);
   HALLOC(h->act_shared, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
   HALLOC(h->act_routed, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
   HALLOC(h->y_part, sizeof(float) * (size_t)kMaxRows * (d.top_k + 1) * D);
@@ -346,8 +368,6 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->rope, sizeof(float2) * (size_t)d.kv_capacity * (d.head_dim / 2));
   h->counters_bytes = sizeof(uint32_t) * (size_t)n_ops * kCounterStride;
   HALLOC(h->counters, h->counters_bytes);
-  h->route_bytes = sizeof(uint32_t) * (size_t)L * kCounterStride;
-  HALLOC(h->route_flag, h->route_bytes);
   HALLOC(h->epoch, sizeof(uint32_t) * kCounterStride);
   HALLOC(h->error, sizeof(int) * kCounterStride);
   HALLOC(h->stats_dev, sizeof(unsigned long long) * 4);
@@ -409,7 +429,6 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
 
 static int reset_sync_state(mk_handle *h, cudaStream_t s) {
   CUDA_TRY(cudaMemsetAsync(h->counters, 0, h->counters_bytes, s));
-  CUDA_TRY(cudaMemsetAsync(h->route_flag, 0, h->route_bytes, s));
   CUDA_TRY(cudaMemsetAsync(h->epoch, 0, sizeof(uint32_t) * kCounterStride, s));
   CUDA_TRY(cudaMemsetAsync(h->attn_cnt, 0, h->attn_cnt_bytes, s));
   CUDA_TRY(cudaMemsetAsync(h->error, 0, sizeof(int) * kCounterStride, s));
@@ -450,6 +469,10 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.n_cta = pl.n_cta; p.n_warps = pl.n_warps; p.op_begin = 0; p.op_end = pl.n_ops; p.n_ops = pl.n_ops;
   p.n_hb = pl.n_hb;
   p.xs_floats = pl.xs_floats;
+  p.qkv_split = pl.qkv_split;
+  p.down_groups = pl.down_groups;
+  p.n_db = pl.n_hb / pl.down_groups;
+  p.down_staged = pl.down_staged;
   p.ss_ld = ceil_div(pl.n_hb, 128) * 128;
   p.e_ld = ceil_div(d.n_experts, 4) * 4;
   p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit;
@@ -461,10 +484,10 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.tokens = tokens; p.positions = positions; p.logits = logits ? logits : h->logits; p.argmax = argmax;
   p.h = h->h; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
   p.attn_o = h->attn_o; p.attn_ml = h->attn_ml;
-  p.attn_cnt = h->attn_cnt; p.router_part = h->router_part; p.routing = h->routing;
+  p.attn_cnt = h->attn_cnt; p.router_part = h->router_part;
   p.act_shared = h->act_shared; p.act_routed = h->act_routed; p.y_part = h->y_part;
   p.am_part = h->am_part; p.rope = h->rope;
-  p.counters = h->counters; p.route_flag = h->route_flag;
+  p.counters = h->counters;
   p.epoch = h->epoch; p.error = h->error;
   p.stats = h->stats_dev;
   p.dbg_hidden = h->dbg_hidden; p.dbg_ids = h->dbg_ids; p.dbg_w = h->dbg_w;
@@ -714,19 +737,17 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
   StaticCarve c;
   // words that must read zero when the step starts, first, so one memset clears them
   c.take(p.counters, base, sizeof(uint32_t) * (size_t)pl.n_ops * kCounterStride);
-  c.take(p.route_flag, base, sizeof(uint32_t) * (size_t)L * kCounterStride);
   c.take(p.epoch, base, sizeof(uint32_t) * kCounterStride);
   c.take(p.attn_cnt, base, sizeof(uint32_t) * ngrp);
   const size_t zero_bytes = c.used;
   // buffers every step writes before it reads them
   c.take(p.h, base, sizeof(float) * (size_t)kMaxRows * D);
   c.take(p.ss, base, sizeof(float) * (size_t)kMaxRows * p.ss_ld);
-  c.take(p.qkv, base, sizeof(float) * (size_t)kMaxRows * QKVW);
+  c.take(p.qkv, base, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);
   c.take(p.o, base, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
   c.take(p.attn_o, base, sizeof(float) * ngrp * pl.attn_nch_max * kQvp * d.head_dim);
   c.take(p.attn_ml, base, sizeof(float) * ngrp * kQvp * 2 * pl.attn_nch_max);
   c.take(p.router_part, base, sizeof(float) * (size_t)ceil_div(D, kTileCols) * kMaxRows * p.e_ld);
-  c.take(p.routing, base, sizeof(Routing) * (size_t)L);
   c.take(p.act_shared, base, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
   c.take(p.act_routed, base, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
   c.take(p.y_part, base, sizeof(float) * (size_t)kMaxRows * (d.top_k + 1) * D);

@@ -33,6 +33,7 @@ enum OpType : int {
   OP_EMBED = 0, OP_QKV = 1, OP_ATTN = 2, OP_OPROJ = 3, OP_ROUTER = 4,
   OP_SHARED_GU = 5, OP_ROUTED_GU = 6, OP_DOWN = 7, OP_COMBINE = 8, OP_LMHEAD = 9
 };
+constexpr int kTraceWords = 8;  // per (op, warp) trace record, as MK_TRACE_WORDS
 constexpr int kOpsPerLayer = 8;
 
 __host__ __device__ inline int n_ops_for(int L) { return kOpsPerLayer * L + 2; }
@@ -59,8 +60,8 @@ __host__ __device__ inline void op_deps(int op, int L, int *d0, int *d1) {
     case OP_ATTN: *d0 = op_index(l, OP_QKV); break;
     case OP_OPROJ: *d0 = op_index(l, OP_ATTN); break;
     case OP_ROUTER:
-    case OP_SHARED_GU:
-    case OP_ROUTED_GU: *d0 = op_index(l, OP_OPROJ); break;  // ROUTED_GU: + routing
+    case OP_SHARED_GU: *d0 = op_index(l, OP_OPROJ); break;
+    case OP_ROUTED_GU: *d0 = op_index(l, OP_OPROJ); *d1 = op_index(l, OP_ROUTER); break;
     case OP_DOWN: *d0 = op_index(l, OP_SHARED_GU); *d1 = op_index(l, OP_ROUTED_GU); break;
     case OP_COMBINE: *d0 = op_index(l, OP_DOWN); break;
     case OP_LMHEAD: *d0 = op_index(L - 1, OP_COMBINE); break;
@@ -74,15 +75,6 @@ __host__ __device__ inline bool op_has_tiles(int type) {
 enum MapSlot : int {
   MAP_WQKV = 0, MAP_WO, MAP_ROUTER, MAP_WGATE, MAP_WUP, MAP_WDOWN,
   MAP_WSGATE, MAP_WSUP, MAP_WSDOWN, MAPS_PER_LAYER
-};
-
-// Routing of one layer, written by the last warp to finish the router op:
-// each row's selections in selection order.  CTAs derive the expert union,
-// row masks and slots from these into a shared-memory cache.
-struct Routing {
-  int n_union;                            // distinct experts over the M rows
-  int row_e[kMaxRows][kMaxTopK];          // row m's selections, in selection order
-  float row_w[kMaxRows][kMaxTopK];        // and their renormalised weights
 };
 
 struct ArgmaxPart {
@@ -101,6 +93,11 @@ struct alignas(64) Params {
   int n_cta, n_warps, op_begin, op_end, n_ops;
   int n_hb;            // residual row blocks (ceil(d / kRows))
   int xs_floats;       // shared-memory activation row (batch 1), 0 = none
+  int qkv_split;       // QKV units cover 1 or 2 halves of K; the halves are summed by their reader
+  int down_groups;     // 4-row groups per down-projection unit (1 or 2)
+  int n_db;            // down-projection row blocks (n_hb / down_groups)
+  int down_staged;     // batch 1: each CTA takes a contiguous range of down units and
+                       // stages their experts' activations in shared memory
   int ss_ld;           // row stride of the sum-of-squares partials (n_hb rounded up to 128)
   int e_ld;            // row stride of the router partials (E rounded up to 4)
   int attn_chunk;      // KV positions per warp; a CTA item covers 8 * attn_chunk
@@ -119,11 +116,10 @@ struct alignas(64) Params {
   float *attn_o, *attn_ml;   // per-CTA-chunk partials (unnormalised o; max, sum)
   uint32_t *attn_cnt;
   float *router_part;
-  Routing *routing;                      // [L]
   float *act_shared, *act_routed, *y_part;   // silu(gate) * up per row; down partials
   ArgmaxPart *am_part;
   const float2 *rope;                    // [cap][hd/2] (cos, sin) of p * theta^(-2i/hd)
-  uint32_t *counters, *route_flag, *epoch;
+  uint32_t *counters, *epoch;
   int *error;                            // [0] code, [1] op
   unsigned long long *stats;             // [0] expert union total
   // debug

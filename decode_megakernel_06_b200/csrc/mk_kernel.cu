@@ -97,6 +97,21 @@ MK_INLINE uint32_t ld_relaxed(const uint32_t *p) {
   return v;
 }
 
+// Acquire load: later loads of this thread see what was released before the
+// value it reads (and everything that release observed).
+MK_INLINE uint32_t ld_acquire(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// CTA-scope acq_rel add on a shared-memory counter (generic address).
+MK_INLINE uint32_t atom_add_acq_rel_cta(uint32_t *p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 MK_INLINE void st_release(uint32_t *p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -107,7 +122,6 @@ MK_INLINE uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
   return old;
 }
 
-MK_INLINE void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 MK_INLINE uint64_t now_ns() {
   uint64_t t;
@@ -133,6 +147,9 @@ MK_INLINE void unpack8(const uint4 &w, float (&f)[8]) {
 }
 
 MK_INLINE uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
+
+// Bring the line holding p into this SM's L1 (no register result).
+MK_INLINE void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
 MK_INLINE float silu(float u) { return u / (1.0f + expf(-u)); }
 
@@ -190,8 +207,17 @@ MK_INLINE float warp_sum(float v) {
 
 // Units are dealt round-robin: warp slot s takes units u0(s) + i * n_warps,
 // with a per-op rotation so that remainders do not always land on warp 0.
-MK_INLINE int first_unit_of(int slot, int op, int nw) {
-  const int rot = static_cast<int>((static_cast<uint32_t>(op) * 2654435761u) % static_cast<uint32_t>(nw));
+MK_INLINE int op_rotation(int op, int nw) {
+  return static_cast<int>((static_cast<uint32_t>(op) * 2654435761u) % static_cast<uint32_t>(nw));
+}
+
+// The first unit of `op` for warp slot `slot`: units go round-robin over the
+// slots from a per-op rotation.  Routed gate/up units continue the dealing of
+// the shared expert's (the op before), so the warps that took a shared unit
+// take fewer routed ones.
+MK_INLINE int first_unit_of(int slot, int op, int nw, int type, int shared_units) {
+  int rot = op_rotation(op, nw);
+  if (type == OP_ROUTED_GU) rot = (op_rotation(op - 1, nw) + shared_units) % nw;
   return (slot - rot + nw) % nw;
 }
 
@@ -202,15 +228,18 @@ MK_INLINE int unit_count_of(int u0, int total, int nw) { return total > u0 ? (to
 // ---------------------------------------------------------------------------
 constexpr int kWbuf = 64;  // floats of per-warp epilogue scratch (2 * 4 * MJ <= 64)
 
-// Per-CTA cache of one layer's routing, derived from the top-k's per-row
-// selections: the ascending expert union, rows served by each, their slots.
+// One layer's routing, computed by every CTA for itself from the router's
+// split-K partial logits: per row its selections (expert id and renormalised
+// weight, in selection order), and the ascending union of the selected
+// experts with the rows that chose each and in which selection slot.
 struct RouteCache {
-  int ready_key, fill_key;   // layer + 1 once filled / being filled
+  int ready_key, fill_key;   // layer + 1 once computed / being computed
   int n_union;
   int expert[kMaxExperts];
   uint32_t rowmask[kMaxExperts];
   int8_t kslot[kMaxExperts][kMaxRows];
   float row_w[kMaxRows][kMaxTopK];
+  uint8_t row_e[kMaxRows][kMaxTopK];
 };
 
 struct Warp {
@@ -228,6 +257,8 @@ struct Warp {
   int cslot, islot, inflight;
   // producer cursor: op, this warp's unit index in it, tile in the unit
   int iop, iu0, in_units, iu, it, in_tiles, iunit;
+  int itype, ilayer;  // type and layer of op iop, once its current unit is set up
+  int istride;        // unit stride of op iop for this warp
   // the current unit's tile source: maps for the first and second half of its
   // tiles (gate / up), first row of each, first column, K, tiles per half
   const CUtensorMap *um, *um2;
@@ -235,6 +266,10 @@ struct Warp {
   bool iop_init, done_issue;
   uint64_t pol_w, pol_kv;
   bool failed;
+  // per-op timeline (only with a trace buffer): first tile ready, last tile
+  // consumed, ns blocked on tiles, tiles consumed
+  uint64_t tr_first, tr_last, tr_wait;
+  int tr_n;
 };
 
 __device__ __noinline__ void report_error(const Params &P, int lane, int code, int op) {
@@ -248,83 +283,171 @@ MK_INLINE void set_error(Warp &w, int code, int op) {
   w.failed = true;
 }
 
-// Every lane reads the flag itself, so that each lane's acquire fence follows
-// its own observation of the release.
+// The layer's router partials are complete once the ROUTER op's counter
+// reaches its target; every lane then re-reads it with acquire semantics.
 MK_INLINE bool routing_ready(const Warp &w, int layer) {
-  const uint32_t v = ld_relaxed(&w.P->route_flag[layer * kCounterStride]);
-  const bool ok = __all_sync(0xffffffffu, static_cast<int>(v - w.epoch) >= 0);
-  if (ok) fence_acq_rel();
+  const uint32_t *ctr = &w.P->counters[op_index(layer, OP_ROUTER) * kCounterStride];
+  const uint32_t target = w.epoch * static_cast<uint32_t>(w.P->n_cta);
+  const uint32_t v = ld_relaxed(ctr);
+  const bool ok = __all_sync(0xffffffffu, static_cast<int>(v - target) >= 0);
+  if (ok) (void)ld_acquire(ctr);
   return ok;
 }
 
-// Fill the CTA's routing cache for `layer` (one elected warp; the others wait,
-// bounded).  The caller has observed the layer's routing flag.
-__device__ __noinline__ void route_cache_fill(const Params &P, RouteCache *rc, int lane, int layer) {
-  const Routing *rt = P.routing + layer;
-  const int K = P.topk, MK = P.M * K;
-  // lane l gathers experts 8l..8l+7: row mask and per-row selection slot
-  uint32_t mask[8];
-  uint64_t slots[8];
+// Lane l owns experts 4l..4l+3 and 128+4l..128+4l+3.
+MK_INLINE int expert_of(int lane, int i) { return (i < 4) ? 4 * lane + i : 128 + 4 * lane + (i - 4); }
+
+// The CTA's routing for `layer` (one warp; the caller has seen the router's
+// partials complete).  Per row: logits = the split-K partials summed in a
+// fixed order; softmax over the E experts; k rounds of argmax (ties to the
+// lower expert id); weights renormalised by their sum.  Every CTA runs this
+// on the same partials and gets the same result.
+__device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int lane, int layer) {
+  const int E = P.E, K = P.topk;
+  const int nkc = cdiv(P.d, kTileCols);
+  constexpr int EPL = 8;
+  uint32_t chosen[EPL];  // rows that selected each of this lane's experts
+  uint64_t slots[EPL];   // byte m: the selection slot row m gave it
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    mask[i] = 0;
-    slots[i] = ~0ull;
+  for (int i = 0; i < EPL; ++i) {
+    chosen[i] = 0;
+    slots[i] = 0;
   }
-  for (int base = 0; base < MK; base += 32) {
-    const int idx = base + lane;
-    const int e_mine = idx < MK ? __ldcg(&rt->row_e[idx / K][idx % K]) : -1;
-    const int cnt = min(32, MK - base);
-    for (int q = 0; q < cnt; ++q) {
-      const int e = __shfl_sync(0xffffffffu, e_mine, q);
-      const int m = (base + q) / K, j = (base + q) % K;
-      if ((e >> 3) == lane) {
+  for (int m = 0; m < P.M; ++m) {
+    float z[EPL];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if ((e & 7) == i) {
-            mask[i] |= 1u << m;
-            slots[i] = (slots[i] & ~(0xffull << (8 * m))) | (static_cast<uint64_t>(j) << (8 * m));
-          }
+    for (int i = 0; i < EPL; ++i) z[i] = 0.f;
+    for (int k0 = 0; k0 < nkc; k0 += 8) {
+      float4 va[8], vb[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float *row = P.router_part + (static_cast<size_t>(k0 + k) * kMaxRows + m) * P.e_ld;
+        const bool kin = k0 + k < nkc;
+        va[k] = (kin && 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row) + lane)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        vb[k] = (kin && 128 + 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row + 128) + lane)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        z[0] += va[k].x; z[1] += va[k].y; z[2] += va[k].z; z[3] += va[k].w;
+        z[4] += vb[k].x; z[5] += vb[k].y; z[6] += vb[k].z; z[7] += vb[k].w;
       }
     }
-  }
-  int cnt = 0;
+    bool taken[EPL];
+    float mx = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) cnt += mask[i] ? 1 : 0;
-  int incl = cnt;
+    for (int i = 0; i < EPL; ++i) {
+      taken[i] = expert_of(lane, i) >= E;
+      if (!taken[i]) mx = fmaxf(mx, z[i]);
+    }
+    mx = warp_max(mx);
+    float pi[EPL], sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      pi[i] = taken[i] ? 0.f : expf(z[i] - mx);
+      sum += pi[i];
+    }
+    sum = warp_sum(sum);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) pi[i] = pi[i] / sum;
+    // k rounds of argmax; lane j keeps selection j
+    float sel = 0.f, my_w = 0.f;
+    int my_e = 0;
+    for (int j = 0; j < K; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = expert_of(lane, i);
+        if (!taken[i] && (pi[i] > bv || (pi[i] == bv && e < bi))) {
+          bv = pi[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (expert_of(lane, i) == bi) {
+          taken[i] = true;
+          chosen[i] |= 1u << m;
+          slots[i] |= static_cast<uint64_t>(j) << (8 * m);
+        }
+      if (lane == j) {
+        my_e = bi;
+        my_w = bv;
+      }
+      sel += bv;
+    }
+    if (lane < K) {
+      rc->row_w[m][lane] = my_w / sel;
+      rc->row_e[m][lane] = static_cast<uint8_t>(my_e);
+    }
+  }
+  // ascending union: every id below 128 (slots i < 4) precedes every id above
+  int lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) (i < 4 ? lo : hi) += chosen[i] ? 1 : 0;
+  int lo_incl = lo, hi_incl = hi;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  int pos = incl - cnt;
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (mask[i]) {
-      rc->expert[pos] = 8 * lane + i;
-      rc->rowmask[pos] = mask[i];
-#pragma unroll
-      for (int m = 0; m < kMaxRows; ++m) rc->kslot[pos][m] = static_cast<int8_t>(slots[i] >> (8 * m));
-      ++pos;
+    const int a = __shfl_up_sync(0xffffffffu, lo_incl, o), b = __shfl_up_sync(0xffffffffu, hi_incl, o);
+    if (lane >= o) {
+      lo_incl += a;
+      hi_incl += b;
     }
-  if (lane == 31) rc->n_union = incl;
-  for (int idx = lane; idx < MK; idx += 32) rc->row_w[idx / K][idx % K] = __ldcg(&rt->row_w[idx / K][idx % K]);
+  }
+  const int lo_total = __shfl_sync(0xffffffffu, lo_incl, 31), hi_total = __shfl_sync(0xffffffffu, hi_incl, 31);
+  int pos_lo = lo_incl - lo, pos_hi = lo_total + hi_incl - hi;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i)
+    if (chosen[i]) {
+      const int pos = (i < 4) ? pos_lo++ : pos_hi++;
+      rc->expert[pos] = expert_of(lane, i);
+      rc->rowmask[pos] = chosen[i];
+#pragma unroll
+      for (int m = 0; m < kMaxRows; ++m) rc->kslot[pos][m] = static_cast<int8_t>((slots[i] >> (8 * m)) & 0xff);
+    }
+  if (lane == 0) rc->n_union = lo_total + hi_total;
   __threadfence_block();
   __syncwarp();
   if (lane == 0) *reinterpret_cast<volatile int *>(&rc->ready_key) = layer + 1;
   __syncwarp();
 }
 
+// Trace: when this warp first found its CTA's routing cache ready for the
+// layer, and whether it filled it (words 6 and 7 of its ROUTED_GU record).
+MK_INLINE void trace_route_cache(const Warp &w, int layer, int filler) {
+  const Params &P = *w.P;
+  if (P.trace && w.lane == 0) {
+    unsigned long long *tr = P.trace + (static_cast<size_t>(op_index(layer, OP_ROUTED_GU)) * w.nw + w.slot) * kTraceWords;
+    if (tr[6] == 0) {
+      tr[6] = now_ns();
+      tr[7] = static_cast<unsigned long long>(filler);
+    }
+  }
+}
+
 MK_INLINE bool route_cache(Warp &w, int layer) {
   RouteCache *rc = w.rc;
   if (*reinterpret_cast<volatile int *>(&rc->ready_key) == layer + 1) {
     __threadfence_block();
+    trace_route_cache(w, layer, 0);
     return true;
   }
   int filler = 0;
   if (w.lane == 0) filler = atomicMax(&rc->fill_key, layer + 1) < layer + 1 ? 1 : 0;
   filler = __shfl_sync(0xffffffffu, filler, 0);
   if (filler) {
-    route_cache_fill(*w.P, rc, w.lane, layer);
+    route_compute(*w.P, rc, w.lane, layer);
   } else {
     const uint64_t t0 = now_ns();
     while (*reinterpret_cast<volatile int *>(&rc->ready_key) != layer + 1) {
@@ -337,6 +460,7 @@ MK_INLINE bool route_cache(Warp &w, int layer) {
   }
   __threadfence_block();
   __syncwarp();
+  trace_route_cache(w, layer, filler);
   return true;
 }
 
@@ -347,17 +471,66 @@ MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
   const Params &P = *w.P;
   switch (type) {
     case OP_EMBED: return P.n_hb;
-    case OP_QKV: return cdiv((P.Hq + 2 * P.Hkv) * P.hd, kRows);
+    case OP_QKV: return cdiv((P.Hq + 2 * P.Hkv) * P.hd, kRows) * P.qkv_split;
     case OP_ATTN: return w.attn_prefix[P.B];
     case OP_OPROJ: return P.n_hb;
     case OP_ROUTER: return cdiv(P.E, kRows) * cdiv(P.d, kTileCols);
     case OP_SHARED_GU: return P.Fs / kRows;
     case OP_ROUTED_GU: return n_union(w) * (P.F / kRows);
-    case OP_DOWN: return (n_union(w) + (P.Fs > 0 ? 1 : 0)) * P.n_hb;
+    case OP_DOWN: return (n_union(w) + (P.Fs > 0 ? 1 : 0)) * P.n_db;
     case OP_COMBINE: return P.n_hb;
     case OP_LMHEAD: return cdiv(P.V, kRows);
   }
   return 0;
+}
+
+// A staged (batch 1) down projection deals CTA c the contiguous units
+// [c * total / n_cta, (c + 1) * total / n_cta), warp by warp within the CTA.
+MK_INLINE void down_cta_range(const Params &P, int cta, int total, int &c0, int &c1) {
+  c0 = static_cast<int>((static_cast<long long>(cta) * total) / P.n_cta);
+  c1 = static_cast<int>((static_cast<long long>(cta + 1) * total) / P.n_cta);
+}
+
+// This warp's units of an op: u0, u0 + stride, ... (n of them).  Attention
+// items are CTA-wide; a staged down projection takes CTA-contiguous ranges;
+// everything else goes round-robin over the warp slots.
+MK_INLINE void op_units(const Warp &w, int op, int type, int layer, int &u0, int &stride, int &n) {
+  const Params &P = *w.P;
+  const int total = op_total_units(w, type, layer);
+  if (type == OP_ATTN) {
+    u0 = w.cta;
+    stride = P.n_cta;
+  } else if (type == OP_DOWN && P.down_staged) {
+    int c0, c1;
+    down_cta_range(P, w.cta, total, c0, c1);
+    u0 = c0 + w.wib;
+    stride = kWarpsPerCta;
+    n = c1 > u0 ? (c1 - 1 - u0) / kWarpsPerCta + 1 : 0;
+    return;
+  } else {
+    u0 = first_unit_of(w.slot, op, w.nw, type, P.Fs / kRows);
+    stride = w.nw;
+  }
+  n = unit_count_of(u0, total, stride);
+}
+
+// QKV unit -> rows [row0, row0 + 4) over tiles [col0, col0 + ntiles * 1024) of
+// K: the first (rows / 4) units take the first half of K, the rest the second.
+MK_INLINE void qkv_unit(const Params &P, int unit, int &row0, int &col0, int &ntiles, int &half) {
+  const int nrb = cdiv((P.Hq + 2 * P.Hkv) * P.hd, kRows);
+  const int nt = cdiv(P.d, kTileCols);
+  const int h0 = P.qkv_split > 1 ? cdiv(nt, 2) : nt;
+  half = unit / nrb;
+  row0 = (unit - half * nrb) * kRows;
+  col0 = half ? h0 * kTileCols : 0;
+  ntiles = half ? nt - h0 : h0;
+}
+
+// One QKV output (row m's column i): the sum of its K halves.
+MK_INLINE float qkv_load(const Params &P, size_t i) {
+  float v = __ldcg(P.qkv + i);
+  if (P.qkv_split > 1) v += __ldcg(P.qkv + static_cast<size_t>(kMaxRows) * (P.Hq + 2 * P.Hkv) * P.hd + i);
+  return v;
 }
 
 // An attention item covers 8 * attn_chunk KV positions of one (sequence,
@@ -389,13 +562,20 @@ MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs
 MK_INLINE int unit_tiles(const Warp &w, int type, int layer, int unit) {
   const Params &P = *w.P;
   switch (type) {
-    case OP_QKV:
+    case OP_QKV: {
+      int row0, col0, nt, half;
+      qkv_unit(P, unit, row0, col0, nt, half);
+      return nt;
+    }
     case OP_LMHEAD: return cdiv(P.d, kTileCols);
     case OP_SHARED_GU:
     case OP_ROUTED_GU: return 2 * cdiv(P.d, kTileCols);
     case OP_OPROJ: return cdiv(P.Hq * P.hd, kTileCols);
     case OP_ROUTER: return 1;
-    case OP_DOWN: return (unit / P.n_hb) < n_union(w) ? cdiv(P.F, kTileCols) : cdiv(P.Fs, kTileCols);
+    case OP_DOWN: {
+      const int K = (unit / P.n_db) < n_union(w) ? P.F : P.Fs;
+      return cdiv(P.down_groups * cdiv(K, kPanel), kPanels);
+    }
     case OP_ATTN: return attn_item(P, w.attn_prefix, w.attn_nch, unit, w.wib).ntiles;
     default: return 0;
   }
@@ -411,7 +591,12 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
   int row0 = unit * kRows, col0 = 0, K = P.d, half = 1 << 30, row2 = 0;
   const CUtensorMap *m0 = nullptr, *m2 = nullptr;
   switch (type) {
-    case OP_QKV: m0 = lm + MAP_WQKV; break;
+    case OP_QKV: {
+      int nt, kh;
+      qkv_unit(P, unit, row0, col0, nt, kh);
+      m0 = lm + MAP_WQKV;
+      break;
+    }
     case OP_OPROJ: m0 = lm + MAP_WO; K = P.Hq * P.hd; break;
     case OP_LMHEAD: m0 = P.tmaps + P.L * MAPS_PER_LAYER; break;
     case OP_ROUTER: {
@@ -437,15 +622,15 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
       break;
     }
     case OP_DOWN: {
-      const int seg = unit / P.n_hb, rb = unit % P.n_hb;
+      const int seg = unit / P.n_db, rb = unit % P.n_db;
       if (seg < n_union(w)) {
         const int e = w.rc->expert[seg];
         m0 = lm + MAP_WDOWN;
-        row0 = e * P.d + rb * kRows;
+        row0 = e * P.d + rb * kRows * P.down_groups;
         K = P.F;
       } else {
         m0 = lm + MAP_WSDOWN;
-        row0 = rb * kRows;
+        row0 = rb * kRows * P.down_groups;
         K = P.Fs;
       }
       break;
@@ -474,6 +659,19 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
       tma_load_2d(dst, &P.kmap, 0, row, bar, w.pol_kv);
       tma_load_2d(dst + kKvBoxBytes, &P.vmap, 0, row, bar, w.pol_kv);
     }
+  } else if (type == OP_DOWN && P.down_groups > 1) {
+    // the unit's boxes run group by group (4 rows each), nbx boxes of 256
+    // columns per group; tile t takes boxes 4t .. 4t+3
+    const int nbx = cdiv(w.uK, kPanel), nb = P.down_groups * nbx, b0 = t * kPanels;
+    const int nbox = min(kPanels, nb - b0);
+    if (w.lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * kBoxBytes);
+      for (int p = 0; p < nbox; ++p) {
+        const int g = (b0 + p) / nbx, c = b0 + p - g * nbx;
+        tma_load_2d(dst + p * kBoxBytes, w.um, c * kPanel, w.urow0 + g * kRows, bar, w.pol_w);
+      }
+    }
   } else {
     // up to four 4 x 256 boxes side by side; boxes starting past K are skipped
     const bool second = t >= w.uhalf;
@@ -495,6 +693,11 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
 MK_INLINE void issue_more(Warp &w) {
   const Params &P = *w.P;
   while (!w.done_issue && !w.failed && w.inflight < kSlots) {
+    if (w.it < w.in_tiles) {  // the next tile of the current unit
+      issue_tile(w, w.itype, w.ilayer, w.it);
+      w.it++;
+      continue;
+    }
     if (w.iop >= P.op_end) {
       w.done_issue = true;
       break;
@@ -509,11 +712,9 @@ MK_INLINE void issue_more(Warp &w) {
         if (!routing_ready(w, layer)) return;
         if (!route_cache(w, layer)) return;
       }
-      // attention items are CTA-wide (every warp of the CTA takes a share)
-      const bool cta_items = type == OP_ATTN;
-      const int stride = cta_items ? P.n_cta : w.nw;
-      w.iu0 = cta_items ? w.cta : first_unit_of(w.slot, w.iop, w.nw);
-      w.in_units = unit_count_of(w.iu0, op_total_units(w, type, layer), stride);
+      int stride;
+      op_units(w, w.iop, type, layer, w.iu0, stride, w.in_units);
+      w.istride = stride;
       w.iu = 0;
       w.in_tiles = -1;
       w.iop_init = true;
@@ -524,10 +725,12 @@ MK_INLINE void issue_more(Warp &w) {
       continue;
     }
     if (w.in_tiles < 0) {
-      w.iunit = w.iu0 + w.iu * (type == OP_ATTN ? P.n_cta : w.nw);
+      w.iunit = w.iu0 + w.iu * w.istride;
       w.it = 0;
       w.in_tiles = unit_tiles(w, type, layer, w.iunit);
       if (type != OP_ATTN) unit_source(w, type, layer, w.iunit);
+      w.itype = type;
+      w.ilayer = layer;
     }
     if (w.it >= w.in_tiles) {
       w.iu++;
@@ -561,14 +764,25 @@ MK_INLINE const uint8_t *consume_begin(Warp &w, int op) {
   }
   uint64_t *bar = &w.bars[w.cslot];
   const uint32_t par = (w.phase >> w.cslot) & 1u;
+  const bool tr = w.P->trace != nullptr;
+  const uint64_t t0 = tr ? now_ns() : 0;
   if (!__all_sync(0xffffffffu, mbar_try_wait(bar, par)) && !wait_slot_slow(bar, par, w.P->timeout_ns)) {
     set_error(w, -5, op);
     return nullptr;
+  }
+  if (tr) {
+    const uint64_t t1 = now_ns();
+    w.tr_wait += t1 - t0;
+    if (w.tr_n == 0) w.tr_first = t1;
   }
   return w.ring + w.cslot * kSlotBytes;
 }
 
 MK_INLINE void consume_end(Warp &w) {
+  if (w.P->trace) {
+    w.tr_last = now_ns();
+    w.tr_n++;
+  }
   __syncwarp();
   w.phase ^= (1u << w.cslot);
   w.cslot = (w.cslot + 1 == kSlots) ? 0 : w.cslot + 1;
@@ -581,8 +795,8 @@ MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int o
   const Params &P = *w.P;
   uint64_t t0 = 0;
   for (int it = 0;; ++it) {
-    // every lane reads the counter (one broadcast transaction), so that each
-    // lane's acquire fence below follows its own observation of the release
+    // every lane reads the counter (one broadcast transaction); the final
+    // read below is an acquire on every lane
     const uint32_t v = ld_relaxed(ctr);
     if (__all_sync(0xffffffffu, static_cast<int>(v - target) >= 0)) break;
     int err = 0;
@@ -604,7 +818,8 @@ MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int o
       return false;
     }
   }
-  fence_acq_rel();
+  // the counter only grows within a step, so this read also reaches the target
+  (void)ld_acquire(ctr);
   __syncwarp();
   return true;
 }
@@ -632,10 +847,11 @@ MK_INLINE bool arrive(Warp &w, int op) {
   __syncwarp();
   int last = 0;
   if (w.lane == 0) {
-    __threadfence();
-    const uint32_t old = atomicAdd(&w.arrive[op], 1u);
+    // The warp's results (ordered before this by __syncwarp) are released to
+    // the CTA; the CTA's last warp acquires them here and releases them, with
+    // its own, grid-wide through the counter (release is cumulative).
+    const uint32_t old = atom_add_acq_rel_cta(&w.arrive[op], 1u);
     if (old == kWarpsPerCta - 1) {
-      __threadfence();
       const uint32_t g = atom_add_acq_rel(&P.counters[op * kCounterStride], 1u);
       last = (g + 1 == w.epoch * static_cast<uint32_t>(P.n_cta)) ? 1 : 0;
     }
@@ -643,8 +859,7 @@ MK_INLINE bool arrive(Warp &w, int op) {
   last = __shfl_sync(0xffffffffu, last, 0);
   if (last) {
     // every lane observes the completed count before reading others' results
-    (void)ld_relaxed(&P.counters[op * kCounterStride]);
-    fence_acq_rel();
+    (void)ld_acquire(&P.counters[op * kCounterStride]);
   }
   __syncwarp();
   return last != 0;
@@ -662,6 +877,13 @@ struct XNorm {  // x = h * g
   const __nv_bfloat16 *g;
   int row[MJ];
   int n;
+  MK_INLINE void prefetch(int col, int K) const {
+    if (col < K) {
+#pragma unroll
+      for (int j = 0; j < MJ; ++j)
+        if (j < n) prefetch_l1(h + static_cast<size_t>(row[j]) * d + col);
+    }
+  }
   MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
     if (col < K) {
       float gf[8];
@@ -693,6 +915,13 @@ struct XPlain {  // x = src[row][col]
   int ld;
   int row[MJ];
   int n;
+  MK_INLINE void prefetch(int col, int K) const {
+    if (col < K) {
+#pragma unroll
+      for (int j = 0; j < MJ; ++j)
+        if (j < n) prefetch_l1(src + static_cast<size_t>(row[j]) * ld + col);
+    }
+  }
   MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
 #pragma unroll
     for (int j = 0; j < MJ; ++j) {
@@ -712,6 +941,7 @@ struct XPlain {  // x = src[row][col]
 // One activation row staged in shared memory by the CTA (batch 1): x = xs[col].
 struct XSmem {
   const float *xs;
+  MK_INLINE void prefetch(int, int) const {}
   MK_INLINE void load(int col, int K, float (&x)[1][8]) const {
     if (col < K) {
       const float4 a = *reinterpret_cast<const float4 *>(xs + col);
@@ -725,18 +955,32 @@ struct XSmem {
   }
 };
 
+// With one or two activation rows, even and odd columns go to separate
+// accumulators (acc, acc2) so that each row has two independent FMA chains.
 template <int MJ>
-MK_INLINE void gemv_panel(const uint8_t *pan, float (&acc)[kRows * MJ], const float (&x)[MJ][8]) {
+MK_INLINE void gemv_panel(const uint8_t *pan, float (&acc)[kRows * MJ], float (&acc2)[kRows * MJ],
+                          const float (&x)[MJ][8]) {
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
     float wf[8];
     unpack8(ld_shared_v4(pan + r * (kPanel * 2)), wf);
 #pragma unroll
     for (int j = 0; j < MJ; ++j) {
-      float a = acc[r * MJ + j];
+      if constexpr (MJ <= 2) {
+        float a = acc[r * MJ + j], b = acc2[r * MJ + j];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) a = fmaf(wf[k], x[j][k], a);
-      acc[r * MJ + j] = a;
+        for (int k = 0; k < 8; k += 2) {
+          a = fmaf(wf[k], x[j][k], a);
+          b = fmaf(wf[k + 1], x[j][k + 1], b);
+        }
+        acc[r * MJ + j] = a;
+        acc2[r * MJ + j] = b;
+      } else {
+        float a = acc[r * MJ + j];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a = fmaf(wf[k], x[j][k], a);
+        acc[r * MJ + j] = a;
+      }
     }
   }
 }
@@ -744,8 +988,8 @@ MK_INLINE void gemv_panel(const uint8_t *pan, float (&acc)[kRows * MJ], const fl
 // One tile (4 rows x up to four boxes of 256 columns starting at colbase):
 // acc[r*MJ + j] += W[r][cols] . x[j][cols] over this lane's columns.
 template <int MJ, class XS>
-MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], int colbase, int K, const XS &xs,
-                         int lane) {
+MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], float (&acc2)[kRows * MJ], int colbase,
+                         int K, const XS &xs, int lane) {
   const uint8_t *base = slot + lane * 16;
   if constexpr (MJ <= 2) {
     // every panel's activations first: one memory round trip per tile
@@ -754,7 +998,7 @@ MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], int colb
     for (int p = 0; p < kPanels; ++p) xs.load(colbase + p * kPanel + lane * 8, K, x[p]);
 #pragma unroll
     for (int p = 0; p < kPanels; ++p)
-      if (colbase + p * kPanel < K) gemv_panel<MJ>(base + p * kBoxBytes, acc, x[p]);
+      if (colbase + p * kPanel < K) gemv_panel<MJ>(base + p * kBoxBytes, acc, acc2, x[p]);
   } else {
 #pragma unroll
     for (int p = 0; p < kPanels; ++p) {
@@ -762,7 +1006,7 @@ MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], int colb
       if (pc >= K) break;
       float x[MJ][8];
       xs.load(pc + lane * 8, K, x);
-      gemv_panel<MJ>(base + p * kBoxBytes, acc, x);
+      gemv_panel<MJ>(base + p * kBoxBytes, acc, acc2, x);
     }
   }
 }
@@ -770,13 +1014,18 @@ MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], int colb
 // Streams `ntiles` tiles of one unit through the ring into acc (not reduced).
 template <int MJ, class XS>
 MK_INLINE bool gemv_stream(Warp &w, int op, int ntiles, int col0, int K, const XS &xs, float (&acc)[kRows * MJ]) {
+  float acc2[kRows * MJ];  // odd columns when MJ <= 2 (dead otherwise)
 #pragma unroll
-  for (int q = 0; q < kRows * MJ; ++q) acc[q] = 0.f;
+  for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
   for (int t = 0; t < ntiles; ++t) {
     const uint8_t *slot = consume_begin(w, op);
     if (!slot) return false;
-    gemv_tile<MJ>(slot, acc, col0 + t * kTileCols, K, xs, w.lane);
+    gemv_tile<MJ>(slot, acc, acc2, col0 + t * kTileCols, K, xs, w.lane);
     consume_end(w);
+  }
+  if constexpr (MJ <= 2) {
+#pragma unroll
+    for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
   }
   return true;
 }
@@ -788,6 +1037,44 @@ MK_INLINE bool gemv_unit(Warp &w, int op, int ntiles, int col0, int K, const XS 
   if (!gemv_stream<MJ>(w, op, ntiles, col0, K, xs, acc)) return false;
   butterfly<kRows * MJ>(acc, w.lane);
   butterfly_store<kRows * MJ>(acc, buf, w.lane);
+  __syncwarp();
+  return true;
+}
+
+// A unit of `ngroups` groups of 4 rows over K columns, streamed box by box
+// (nbx boxes of 256 columns per group, four boxes per tile); when a group is
+// done its 4 x MJ sums are reduced across lanes into buf + g * 4 * MJ.
+template <int MJ, class XS>
+MK_INLINE bool gemv_groups(Warp &w, int op, int ngroups, int K, const XS &xs, float *buf) {
+  const int nbx = cdiv(K, kPanel), nb = ngroups * nbx;
+  float acc[kRows * MJ], acc2[kRows * MJ];
+#pragma unroll
+  for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
+  const uint8_t *slot = nullptr;
+  int g = 0, c = 0;
+  for (int b = 0; b < nb; ++b) {
+    const int p = b & (kPanels - 1);
+    if (p == 0) {
+      slot = consume_begin(w, op);
+      if (!slot) return false;
+    }
+    float x[MJ][8];
+    xs.load(c * kPanel + w.lane * 8, K, x);
+    gemv_panel<MJ>(slot + w.lane * 16 + p * kBoxBytes, acc, acc2, x);
+    if (p == kPanels - 1 || b == nb - 1) consume_end(w);
+    if (++c == nbx) {
+      if constexpr (MJ <= 2) {
+#pragma unroll
+        for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
+      }
+      butterfly<kRows * MJ>(acc, w.lane);
+      butterfly_store<kRows * MJ>(acc, buf + g * kRows * MJ, w.lane);
+#pragma unroll
+      for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
+      c = 0;
+      ++g;
+    }
+  }
   __syncwarp();
   return true;
 }
@@ -936,7 +1223,7 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
   const Params &P = *w.P;
   constexpr int MJ = MMAX;
   float *wb = w.wbuf;
-  int row0 = unit * kRows, N = 0, col0 = 0, ntiles = 0, K = P.d;
+  int row0 = unit * kRows, N = 0, col0 = 0, ntiles = 0, K = P.d, qkv_half = 0;
   switch (type) {
     case OP_OPROJ: K = P.Hq * P.hd; ntiles = cdiv(K, kTileCols); N = P.d; break;
     case OP_ROUTER: {
@@ -947,7 +1234,13 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
       N = P.E;
       break;
     }
-    case OP_QKV: ntiles = cdiv(P.d, kTileCols); N = (P.Hq + 2 * P.Hkv) * P.hd; break;
+    case OP_QKV: {
+      int half;
+      qkv_unit(P, unit, row0, col0, ntiles, half);
+      N = (P.Hq + 2 * P.Hkv) * P.hd;
+      qkv_half = half;
+      break;
+    }
     default: ntiles = cdiv(P.d, kTileCols); N = P.V; break;
   }
   const bool ok = with_dense_x<MJ, XS>(w, type, layer, xs, [&](const auto &x) {
@@ -964,7 +1257,8 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
   switch (type) {
     case OP_QKV:
       if (live)
-        __stcg(&P.qkv[static_cast<size_t>(m) * (P.Hq + 2 * P.Hkv) * P.hd + row0 + r], im * wb[r * MJ + m]);
+        __stcg(&P.qkv[(static_cast<size_t>(qkv_half) * kMaxRows + m) * (P.Hq + 2 * P.Hkv) * P.hd + row0 + r],
+               im * wb[r * MJ + m]);
       break;
     case OP_ROUTER:
       if (live)
@@ -1057,10 +1351,10 @@ MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const flo
 // One down-projection unit: segment (routed expert j, or the shared expert
 // when j == n_union) x 4 output rows; writes the partial of every row m it
 // serves to y_part[m][slot][row] (slot = selection index, or top_k).
-template <int MJ>
-MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit) {
+template <int MJ, bool XS>
+MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm) {
   const Params &P = *w.P;
-  const int seg = unit / P.n_hb, row0 = (unit % P.n_hb) * kRows;
+  const int seg = unit / P.n_db, row0 = (unit % P.n_db) * kRows * P.down_groups;
   const int U = n_union(w);
   const RouteCache *rt = w.rc;
   XPlain<MJ> xs;
@@ -1078,12 +1372,29 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit) {
     K = P.Fs;
   }
   float *wb = w.wbuf;
-  if (!gemv_unit<MJ>(w, op, cdiv(K, kTileCols), 0, K, xs, wb)) return false;
+  bool ok;
+  if constexpr (XS && MJ == 1) {
+    if (P.down_staged) {
+      // the CTA staged its experts' activations: slot seg - seg0 of the row
+      int c0, c1;
+      down_cta_range(P, w.cta, op_total_units(w, OP_DOWN, layer), c0, c1);
+      XSmem xst;
+      xst.xs = xsm + (seg - c0 / P.n_db) * (cdiv(max(P.F, P.Fs), 4) * 4);
+      ok = gemv_groups<MJ>(w, op, P.down_groups, K, xst, wb);
+    } else {
+      ok = gemv_groups<MJ>(w, op, P.down_groups, K, xs, wb);
+    }
+  } else {
+    ok = gemv_groups<MJ>(w, op, P.down_groups, K, xs, wb);
+  }
+  if (!ok) return false;
   const int q = w.lane / kRows, r = w.lane % kRows;
-  if (w.lane < kRows * xs.n && row0 + r < P.d) {
+  if (w.lane < kRows * xs.n) {
     const int m = row_at<MJ>(xs.row, q);
     const int s = (seg < U) ? static_cast<int>(rt->kslot[seg][m]) : P.topk;
-    __stcg(&P.y_part[(static_cast<size_t>(m) * (P.topk + 1) + s) * P.d + row0 + r], wb[r * MJ + q]);
+    float *dst = P.y_part + (static_cast<size_t>(m) * (P.topk + 1) + s) * P.d;
+    for (int g = 0; g < P.down_groups; ++g)
+      if (row0 + g * kRows + r < P.d) __stcg(dst + row0 + g * kRows + r, wb[(g * kRows + r) * MJ + q]);
   }
   __syncwarp();
   return true;
@@ -1097,13 +1408,13 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
   if (type == OP_ROUTED_GU) {
     cnt = __popc(w.rc->rowmask[unit / (P.F / kRows)]);
   } else if (type == OP_DOWN) {
-    const int seg = unit / P.n_hb;
+    const int seg = unit / P.n_db;
     cnt = seg < n_union(w) ? __popc(w.rc->rowmask[seg]) : P.M;
   } else {
     cnt = P.M;  // shared gate/up
   }
 #define MK_DISPATCH(MJ_)                                      \
-  return (type == OP_DOWN) ? down_unit<MJ_>(w, op, layer, unit) \
+  return (type == OP_DOWN) ? down_unit<MJ_, XS>(w, op, layer, unit, xs) \
                            : gu_unit<MJ_, XS>(w, op, type, layer, unit, inv, xs)
   if (cnt <= 1) {
     MK_DISPATCH(1);
@@ -1159,10 +1470,10 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, float &m
     if (qv < G * P.T) {
       const int t = qv / G, head = a.g * G + qv % G, m = a.b * P.T + t, p = pos_b + t;
       lim[v] = p;
-      const float *src = P.qkv + static_cast<size_t>(m) * W3 + head * hd + lane * DPL;
+      const size_t src = static_cast<size_t>(m) * W3 + head * hd + lane * DPL;
 #pragma unroll
       for (int dd = 0; dd < DPL; ++dd) {
-        const float own = __ldcg(src + dd);
+        const float own = qkv_load(P, src + dd);
         const float other = __shfl_xor_sync(0xffffffffu, own, 16);
         const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
         const float rr = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
@@ -1188,16 +1499,16 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, float &m
     const int lo = max(pos0, pos_b), hi = min(pos0 + P.attn_ppt, pos_b + P.T);
     for (int p = lo; p < hi; ++p) {
       const int t = p - pos_b, m = a.b * P.T + t;
-      const float *kq = P.qkv + static_cast<size_t>(m) * W3 + (P.Hq + a.g) * hd + lane * DPL;
-      const float *vq = P.qkv + static_cast<size_t>(m) * W3 + (P.Hq + P.Hkv + a.g) * hd + lane * DPL;
+      const size_t kq = static_cast<size_t>(m) * W3 + (P.Hq + a.g) * hd + lane * DPL;
+      const size_t vq = static_cast<size_t>(m) * W3 + (P.Hq + P.Hkv + a.g) * hd + lane * DPL;
 #pragma unroll
       for (int dd = 0; dd < DPL; ++dd) {
-        const float own = __ldcg(kq + dd);
+        const float own = qkv_load(P, kq + dd);
         const float other = __shfl_xor_sync(0xffffffffu, own, 16);
         const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
         const float kr = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
         const __nv_bfloat16 kb = __float2bfloat16_rn(kr);
-        const __nv_bfloat16 vb = __float2bfloat16_rn(__ldcg(vq + dd));
+        const __nv_bfloat16 vb = __float2bfloat16_rn(qkv_load(P, vq + dd));
         ks[(p - pos0) * hd + lane * DPL + dd] = kb;
         vs[(p - pos0) * hd + lane * DPL + dd] = vb;
         if (a.qs == 0) {
@@ -1375,8 +1686,7 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
   if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   if (*reinterpret_cast<volatile int *>(sh.last)) {
     if (w.wib < kQvp) {
-      (void)ld_relaxed(cnt);  // every lane observes the completed count
-      fence_acq_rel();
+      (void)ld_acquire(cnt);  // every lane observes the completed count
       attn_final_merge<DPL>(P, w.lane, grp, w.wib, a.nch, a.b, a.g);
     }
     *sh.seq += kWarpsPerCta;
@@ -1388,110 +1698,16 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
 
 // --- router top-k and the final argmax (run by the op's last arriving warp) --
 // Lane l owns experts 4l..4l+3 (slots 0-3) and 128+4l..128+4l+3 (slots 4-7).
-MK_INLINE int expert_of(int lane, int i) { return (i < 4) ? 4 * lane + i : 128 + 4 * lane + (i - 4); }
-
-__device__ __noinline__ void router_topk(const Params &P, int lane, uint32_t epoch, int layer) {
-  const int E = P.E, K = P.topk;
-  const int nkc = cdiv(P.d, kTileCols);
-  constexpr int EPL = 8;
-  Routing *rt = P.routing + layer;
-  uint32_t chosen[EPL];  // rows that selected each of this lane's experts
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) chosen[i] = 0;
-  for (int m = 0; m < P.M; ++m) {
-    // logits = sum of the K-chunk partials in a fixed order; loads issued together
-    float z[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) z[i] = 0.f;
-    for (int k0 = 0; k0 < nkc; k0 += 8) {
-      float4 va[8], vb[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float *row = P.router_part + (static_cast<size_t>(k0 + k) * kMaxRows + m) * P.e_ld;
-        const bool kin = k0 + k < nkc;
-        va[k] = (kin && 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row) + lane)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-        vb[k] = (kin && 128 + 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row + 128) + lane)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        z[0] += va[k].x; z[1] += va[k].y; z[2] += va[k].z; z[3] += va[k].w;
-        z[4] += vb[k].x; z[5] += vb[k].y; z[6] += vb[k].z; z[7] += vb[k].w;
-      }
-    }
-    bool taken[EPL];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      taken[i] = expert_of(lane, i) >= E;
-      if (!taken[i]) mx = fmaxf(mx, z[i]);
-    }
-    mx = warp_max(mx);
-    float pi[EPL], sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      pi[i] = taken[i] ? 0.f : expf(z[i] - mx);
-      sum += pi[i];
-    }
-    sum = warp_sum(sum);
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) pi[i] = pi[i] / sum;
-    // k rounds of argmax (ties to the lower expert id); lane j keeps selection j
-    float sel = 0.f, my_w = 0.f;
-    int my_e = 0;
-    for (int j = 0; j < K; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = expert_of(lane, i);
-        if (!taken[i] && (pi[i] > bv || (pi[i] == bv && e < bi))) {
-          bv = pi[i];
-          bi = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (expert_of(lane, i) == bi) {
-          taken[i] = true;
-          chosen[i] |= 1u << m;
-        }
-      if (lane == j) {
-        my_e = bi;
-        my_w = bv;
-      }
-      sel += bv;
-    }
-    if (lane < K) {
-      const float wn = my_w / sel;
-      rt->row_e[m][lane] = my_e;
-      rt->row_w[m][lane] = wn;
-      if (P.dbg_ids) P.dbg_ids[(static_cast<size_t>(layer) * P.max_rows + m) * K + lane] = my_e;
-      if (P.dbg_w) P.dbg_w[(static_cast<size_t>(layer) * P.max_rows + m) * K + lane] = wn;
-    }
-  }
-  int nu = 0;
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) nu += chosen[i] ? 1 : 0;
-  nu = static_cast<int>(warp_sum(static_cast<float>(nu)));
-  if (lane == 0) {
-    rt->n_union = nu;
-    atomicAdd(&P.stats[0], static_cast<unsigned long long>(nu));
-  }
-  __syncwarp();
-  if (lane == 0) {
-    __threadfence();
-    st_release(&P.route_flag[layer * kCounterStride], epoch);
+// The warp that completed the router op records the layer's union size in
+// the statistics and, if requested, the routing in the debug buffers (from its
+// CTA's cache; nothing waits for this).
+__device__ __noinline__ void route_publish(const Params &P, const RouteCache *rc, int lane, int layer) {
+  if (lane == 0) atomicAdd(&P.stats[0], static_cast<unsigned long long>(rc->n_union));
+  const int K = P.topk;
+  for (int idx = lane; idx < P.M * K; idx += 32) {
+    const int m = idx / K, j = idx % K;
+    if (P.dbg_ids) P.dbg_ids[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = rc->row_e[m][j];
+    if (P.dbg_w) P.dbg_w[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = rc->row_w[m][j];
   }
   __syncwarp();
 }
@@ -1589,16 +1805,36 @@ MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, u
   return cta_rendezvous(w, cnt, seq, op);
 }
 
+// Batch 1 down projection: the CTA copies the activations of the experts its
+// unit range covers (routed rows first, then the shared expert) into the
+// shared-memory row, one max(F, Fs) slot per expert from the range's first.
+MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t &seq, int op) {
+  const Params &P = *w.P;
+  if (!route_cache(w, layer)) return false;
+  const int U = n_union(w), total = op_total_units(w, OP_DOWN, layer);
+  int c0, c1;
+  down_cta_range(P, w.cta, total, c0, c1);
+  if (c1 > c0) {
+    const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, ld = cdiv(max(P.F, P.Fs), 4) * 4;
+    for (int sg = seg0; sg <= seg1; ++sg) {
+      const float4 *src = reinterpret_cast<const float4 *>(
+          sg < U ? P.act_routed + static_cast<size_t>(sg) * kMaxRows * P.F : P.act_shared);
+      const int K = sg < U ? P.F : P.Fs;
+      float4 *dst = reinterpret_cast<float4 *>(xs + (sg - seg0) * ld);
+      for (int c4 = threadIdx.x; c4 < K / 4; c4 += kThreads) dst[c4] = __ldcg(src + c4);
+    }
+  }
+  seq += kWarpsPerCta;
+  return cta_rendezvous(w, cnt, seq, op);
+}
+
 template <int MMAX, bool XS>
 MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, AttnShared &ash, float &am_val,
                            int &am_idx) {
   const Params &P = *w.P;
   if ((type == OP_ROUTED_GU || type == OP_DOWN) && !route_cache(w, layer)) return false;
-  // attention items are CTA-wide: all warps of a CTA work on the same items
-  const bool cta_items = type == OP_ATTN;
-  const int stride = cta_items ? P.n_cta : w.nw;
-  const int u0 = cta_items ? w.cta : first_unit_of(w.slot, op, w.nw);
-  const int n = unit_count_of(u0, op_total_units(w, type, layer), stride);
+  int u0, stride, n;
+  op_units(w, op, type, layer, u0, stride, n);
   if (n == 0) return true;
   float inv[kMaxRows];
 #pragma unroll
@@ -1694,6 +1930,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.iop_init = false;
   w.done_issue = false;
   w.iu0 = w.in_units = w.iu = w.it = w.iunit = 0;
+  w.itype = w.ilayer = 0;
+  w.istride = 1;
   w.in_tiles = -1;
   w.um = w.um2 = nullptr;
   w.urow0 = w.urow2 = w.ucol0 = w.uK = 0;
@@ -1710,17 +1948,17 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     const uint32_t extra = (op == P.inject_op) ? 1u : 0u;
     if (d0 >= 0 && !wait_counter(w, &P.counters[d0 * kCounterStride], target + extra, op)) break;
     if (d1 >= 0 && !wait_counter(w, &P.counters[d1 * kCounterStride], target, op)) break;
-    if (type == OP_ROUTED_GU || type == OP_DOWN || type == OP_COMBINE) {
-      if (!wait_counter(w, &P.route_flag[layer * kCounterStride], w.epoch, op)) break;
-    }
     if constexpr (XS) {
       // ROUTER stages the normed row that SHARED_GU and ROUTED_GU reuse; a
       // launch that starts at one of those stages it itself
       const bool stage = type == OP_QKV || type == OP_OPROJ || type == OP_ROUTER || type == OP_LMHEAD ||
                          ((type == OP_SHARED_GU || type == OP_ROUTED_GU) && op == P.op_begin);
       if (stage && !stage_x(w, type, layer, xs, &s_stage, stage_seq, op)) break;
+      if (type == OP_DOWN && P.down_staged && !stage_down(w, layer, xs, &s_stage, stage_seq, op)) break;
     }
-    if (P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * 2] = now_ns();
+    if (P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords] = now_ns();
+    w.tr_first = w.tr_last = w.tr_wait = 0;
+    w.tr_n = 0;
     bool ok = true;
     if (type == OP_EMBED) {
       op_embed(w);
@@ -1736,8 +1974,24 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       P.am_part[static_cast<size_t>(w.slot) * kMaxRows + w.lane / kRows] = ArgmaxPart{am_val, am_idx};
     }
     const bool last = arrive(w, op);
-    if (P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * 2 + 1] = now_ns();
-    if (last && type == OP_ROUTER) router_topk(P, w.lane, w.epoch, layer);
+    if (P.trace && w.lane == 0) {
+      unsigned long long *tr = P.trace + (static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords;
+      tr[1] = w.tr_first;
+      tr[2] = w.tr_last;
+      tr[3] = now_ns();
+      tr[4] = w.tr_wait;
+      tr[5] = static_cast<unsigned long long>(w.tr_n);
+    }
+    if (last && type == OP_ROUTER) {
+      const uint64_t t_topk = P.trace ? now_ns() : 0;
+      if (!route_cache(w, layer)) break;
+      route_publish(P, w.rc, w.lane, layer);
+      if (P.trace && w.lane == 0) {
+        unsigned long long *tr = P.trace + (static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords;
+        tr[6] = t_topk;
+        tr[7] = now_ns();
+      }
+    }
     if (last && type == OP_LMHEAD) final_argmax(P, w.lane, w.epoch);
   }
   drain(w);

@@ -126,7 +126,7 @@ typedef struct mk_plan_info {
   int32_t n_ops;           /* ops in one step's schedule                     */
   int32_t n_cta;           /* CTAs of the persistent grid (= SM count)       */
   int32_t warps_per_cta;   /* consumer/producer warps per CTA                */
-  int32_t rows_per_tile;   /* weight rows per ring tile (8: tiles are 8 x 512) */
+  int32_t rows_per_tile;   /* weight rows per ring tile (4: tiles are 4 x 1024) */
   int32_t mmax;            /* row capacity of the kernel instance (1,2,4,8)  */
   int32_t attn_chunk;      /* KV positions per attention work item          */
   int32_t attn_qsplit;     /* query-vector groups per (sequence, KV head)    */
@@ -140,9 +140,10 @@ typedef struct mk_plan_info {
 #define MK_OP_QKV 1        /* RMSNorm + QKV projection                          */
 #define MK_OP_ATTN 2       /* rotary, KV append, split-K attention, LSE merge   */
 #define MK_OP_OPROJ 3      /* o-projection + residual                           */
-#define MK_OP_ROUTER 4     /* RMSNorm + router logits; last warp: softmax top-k */
+#define MK_OP_ROUTER 4     /* RMSNorm + router logits (split-K partials)        */
 #define MK_OP_SHARED_GU 5  /* shared expert gate/up rows                        */
-#define MK_OP_ROUTED_GU 6  /* routed experts' gate/up rows (union of the batch) */
+#define MK_OP_ROUTED_GU 6  /* routed experts' gate/up rows (union of the batch);
+                              each CTA first computes the softmax top-k itself */
 #define MK_OP_DOWN 7       /* down projections, one partial per (row, expert)   */
 #define MK_OP_COMBINE 8    /* weighted sum of the partials + residual           */
 #define MK_OP_LMHEAD 9     /* final RMSNorm + lm_head; last warp: argmax        */
@@ -248,9 +249,19 @@ MK_API int mk_set_debug(mk_handle *h, float *hidden, int32_t *expert_ids, float 
 MK_API int mk_debug_inject(mk_handle *h, int32_t fault);
 
 /* Per-op timeline of every following step (NULL disables): device uint64
- * [n_ops][n_cta * warps_per_cta][2] = %globaltimer (ns) when the warp finished
- * waiting for the op's inputs and when it arrived at the op's completion
- * counter.  n_ops and the grid come from mk_plan_describe. */
+ * [n_ops][n_cta * warps_per_cta][MK_TRACE_WORDS] per warp slot:
+ *   [0] %globaltimer (ns) when the warp finished waiting for the op's inputs,
+ *   [1] when its first weight/KV tile of the op was ready (0: none),
+ *   [2] when it finished consuming its last tile of the op (0: none),
+ *   [3] when it arrived at the op's completion counter,
+ *   [4] ns it spent blocked on tiles that had not landed yet,
+ *   [5] tiles it consumed in the op,
+ *   [6], [7] ROUTER, the warp that completed it: when it began its CTA's
+ *            routing and when it had recorded the statistics; ROUTED_GU:
+ *            when this warp first found its CTA's routing ready, and 1 if it
+ *            computed it; otherwise zero.
+ * n_ops and the grid come from mk_plan_describe. */
+#define MK_TRACE_WORDS 8
 MK_API int mk_set_trace(mk_handle *h, uint64_t *trace);
 
 /* Copies the handle's counters; reset != 0 zeroes them afterwards.  Waits for
@@ -263,8 +274,7 @@ MK_API int mk_validate_desc(const mk_model_desc *desc);
 /* Host-only: plan the step for a shape on a GPU with n_sm SMs and report the
  * schedule.  If op_types/op_layers/op_dep0/op_dep1 are non-NULL they receive
  * up to `cap` entries: each op's MK_OP_* type, layer (-1 = none) and the
- * indices of the ops whose completion it waits for (-1 = none; ROUTED_GU also
- * waits for its layer's routing, published by the ROUTER op). */
+ * indices of the ops whose completion it waits for (-1 = none). */
 MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, int32_t T,
                             mk_plan_info *info, int32_t *op_types, int32_t *op_layers,
                             int32_t *op_dep0, int32_t *op_dep1, int32_t cap);
