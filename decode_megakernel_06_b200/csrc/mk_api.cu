@@ -100,28 +100,28 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
     const int nbx = ceil_div(d.expert_ffn, kPanel), nbs = d.shared_ffn > 0 ? ceil_div(d.shared_ffn, kPanel) : 0;
     const bool partial = (nbx % kPanels) != 0 || (nbs % kPanels) != 0;
     const long long units2 = (long long)(d.d_model / (2 * kRows)) * (d.top_k + (d.shared_ffn > 0 ? 1 : 0));
-    p.down_groups = (partial && units2 >= 2LL * n_sm * kWarpsPerCta) ? 2 : 1;
+    p.down_groups = (partial && units2 >= 2LL * n_sm * kConsumers) ? 2 : 1;
   }
   const int G = d.n_q_heads / d.n_kv_heads;
   p.attn_qsplit = ceil_div(G * T, kQvp);
   p.attn_ppt = 2048 / d.head_dim;
   p.n_cta = n_sm;
-  p.n_warps = n_sm * kWarpsPerCta;
-  // Attention items are CTA-wide: each of the 8 warps takes attn_chunk KV
+  p.n_warps = n_sm * kConsumers;
+  // Attention items are CTA-wide: each of the 6 compute warps takes attn_chunk KV
   // positions of an item.  About one item per CTA, warp chunks a multiple of
   // the tile height, and at most kMaxChunks items per (sequence, kv head,
   // query group) so that one merge level combines them.
   long long total = (long long)B * d.n_kv_heads * p.attn_qsplit * d.kv_capacity;
   int c = (int)((total + p.n_warps - 1) / p.n_warps);
-  c = std::max(c, ceil_div(d.kv_capacity, kMaxChunks * kWarpsPerCta));
+  c = std::max(c, ceil_div(d.kv_capacity, kMaxChunks * kConsumers));
   c = std::max(c, p.attn_ppt);
   c = ceil_div(c, p.attn_ppt) * p.attn_ppt;
   p.attn_chunk = c;
-  p.attn_nch_max = ceil_div(d.kv_capacity, c * kWarpsPerCta);
+  p.attn_nch_max = ceil_div(d.kv_capacity, c * kConsumers);
   p.n_ops = n_ops_for(d.n_layers);
   // shared-memory row: the staged activations (batch 1) or the attention
   // warps' partials, whichever is larger
-  p.xs_floats = std::max(kWarpsPerCta * kQvp * d.head_dim,
+  p.xs_floats = std::max(kConsumers * kQvp * d.head_dim,
                          kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), 4) * 4 : 0);
   // Batch 1 down projection: a CTA's contiguous range of units spans at most
   // 1 + ceil(range / row blocks) experts; their activations must fit the
@@ -244,7 +244,7 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
   if (info) {
     info->n_ops = p.n_ops;
     info->n_cta = p.n_cta;
-    info->warps_per_cta = kWarpsPerCta;
+    info->warps_per_cta = kConsumers;
     info->rows_per_tile = p.rows_per_tile;
     info->mmax = p.mmax;
     info->attn_chunk = p.attn_chunk;
@@ -347,7 +347,7 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   h->last_error_op = -1;
 
   const int L = d.n_layers, D = d.d_model, QKVW = (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim;
-  const int n_ops = n_ops_for(L), NW = n_sm * kWarpsPerCta;
+  const int n_ops = n_ops_for(L), NW = n_sm * kConsumers;
   Sizes s = scratch_sizes(d, n_sm);
   const int umax = std::min(d.n_experts, d.max_rows * d.top_k);
   HALLOC(h->tmaps, sizeof(CUtensorMap) * (size_t)(L * MAPS_PER_LAYER + 1));

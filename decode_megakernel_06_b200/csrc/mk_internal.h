@@ -10,10 +10,14 @@
 namespace mk {
 
 // ---- geometry ------------------------------------------------------------------
-constexpr int kWarpsPerCta = 8;                     // each warp: producer + consumer
+constexpr int kConsumers = 4;                       // compute warps per CTA
+constexpr int kProducers = 4;                       // TMA-issuing warps per CTA
+constexpr int kFeeds = kConsumers / kProducers;     // consumers fed by one producer
+constexpr int kWarpsPerCta = kConsumers + kProducers;
 constexpr int kThreads = kWarpsPerCta * 32;
-constexpr int kSlots = 3;                           // ring slots per warp
-constexpr int kSlotBytes = 8192;                    // one tile: two 4 KB TMA boxes
+constexpr int kConsumerThreads = kConsumers * 32;
+constexpr int kSlots = 6;                           // ring slots per consumer
+constexpr int kSlotBytes = 8192;                    // one tile: four 2 KB weight boxes
 constexpr int kPanel = 256;                         // columns per weight box
 constexpr int kRows = 4;                            // rows per weight box, tile and unit
 constexpr int kPanels = 4;                          // weight boxes per tile

@@ -64,6 +64,21 @@ MK_INLINE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking: has the phase of `parity` completed?
+MK_INLINE bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(saddr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+MK_INLINE void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(bar)) : "memory");
+}
+
 MK_INLINE void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
 MK_INLINE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -247,15 +262,22 @@ struct Warp {
   RouteCache *rc;
   int lane, wib, cta, slot, nw;
   uint32_t epoch;
-  uint8_t *ring;
-  uint64_t *bars;
+  uint8_t *ring;           // this consumer's kSlots tiles
+  uint64_t *full, *empty;  // per slot: tile landed / tile released
   float *wbuf;
   uint32_t *arrive;
   const int *attn_prefix;  // shared: first item of each sequence, [kMaxRows + 1]
   const int *attn_nch;     // shared: KV chunks of each sequence, [kMaxRows]
-  uint32_t phase;          // bit s: parity of the next completion of slot s
-  int cslot, islot, inflight;
-  // producer cursor: op, this warp's unit index in it, tile in the unit
+  // consumer side: bit s = parity of the next completion of full[s]
+  uint32_t phase;
+  int cslot;
+  // producer side (a consumer's record, kept by the warp that feeds it): bit s
+  // of ephase = parity to wait for on empty[s] before refilling it; filled =
+  // slots filled at least once
+  uint32_t ephase, filled;
+  int islot;
+  bool producer;
+  // producer cursor: op, this consumer's unit index in it, tile in the unit
   int iop, iu0, in_units, iu, it, in_tiles, iunit;
   int itype, ilayer;  // type and layer of op iop, once its current unit is set up
   int istride;        // unit stride of op iop for this warp
@@ -427,7 +449,7 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
 // layer, and whether it filled it (words 6 and 7 of its ROUTED_GU record).
 MK_INLINE void trace_route_cache(const Warp &w, int layer, int filler) {
   const Params &P = *w.P;
-  if (P.trace && w.lane == 0) {
+  if (P.trace && w.lane == 0 && !w.producer) {
     unsigned long long *tr = P.trace + (static_cast<size_t>(op_index(layer, OP_ROUTED_GU)) * w.nw + w.slot) * kTraceWords;
     if (tr[6] == 0) {
       tr[6] = now_ns();
@@ -504,8 +526,8 @@ MK_INLINE void op_units(const Warp &w, int op, int type, int layer, int &u0, int
     int c0, c1;
     down_cta_range(P, w.cta, total, c0, c1);
     u0 = c0 + w.wib;
-    stride = kWarpsPerCta;
-    n = c1 > u0 ? (c1 - 1 - u0) / kWarpsPerCta + 1 : 0;
+    stride = kConsumers;
+    n = c1 > u0 ? (c1 - 1 - u0) / kConsumers + 1 : 0;
     return;
   } else {
     u0 = first_unit_of(w.slot, op, w.nw, type, P.Fs / kRows);
@@ -552,7 +574,7 @@ MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs
   a.qs = (rem / nch) % P.attn_qsplit;
   a.g = rem / (nch * P.attn_qsplit);
   const int len = __ldg(&P.positions[b]) + P.T;
-  a.pos0 = a.c * P.attn_chunk * kWarpsPerCta + wib * P.attn_chunk;
+  a.pos0 = a.c * P.attn_chunk * kConsumers + wib * P.attn_chunk;
   a.npos = max(0, min(P.attn_chunk, len - a.pos0));
   a.ntiles = cdiv(a.npos, P.attn_ppt);
   return a;
@@ -649,7 +671,7 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
 MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
   const Params &P = *w.P;
   uint8_t *dst = w.ring + w.islot * kSlotBytes;
-  uint64_t *bar = &w.bars[w.islot];
+  uint64_t *bar = &w.full[w.islot];
   if (type == OP_ATTN) {
     const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, w.iunit, w.wib);
     const int row = ((layer * P.Bmax + a.b) * P.Hkv + a.g) * P.cap + a.pos0 + t * P.attn_ppt;
@@ -686,20 +708,36 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
       for (int p = 0; p < nbox; ++p) tma_load_2d(dst + p * kBoxBytes, m, x0 + p * kPanel, y, bar, w.pol_w);
     }
   }
+  w.ephase ^= 1u << w.islot;
+  w.filled |= 1u << w.islot;
   w.islot = (w.islot + 1 == kSlots) ? 0 : w.islot + 1;
-  w.inflight++;
 }
 
-MK_INLINE void issue_more(Warp &w) {
+// Producer: issue the fed consumer's next tiles into its released slots, in
+// the order it will take them (the same dealing and tile order as the
+// consumer's own loop).  Weights and KV do not depend on this step's
+// activations, so the stream runs ahead across ops and layers; it stops only
+// at a full ring and where the routing is not known yet.  Returns true if it
+// issued a tile or finished the stream.
+MK_INLINE bool feed_more(Warp &w) {
   const Params &P = *w.P;
-  while (!w.done_issue && !w.failed && w.inflight < kSlots) {
+  bool progress = false;
+  while (!w.done_issue && !w.failed) {
     if (w.it < w.in_tiles) {  // the next tile of the current unit
+      if (!mbar_test_wait(&w.empty[w.islot], (w.ephase >> w.islot) & 1u)) break;
       issue_tile(w, w.itype, w.ilayer, w.it);
       w.it++;
+      progress = true;
+      continue;
+    }
+    if (w.in_tiles >= 0) {  // the current unit is issued
+      w.iu++;
+      w.in_tiles = -1;
       continue;
     }
     if (w.iop >= P.op_end) {
       w.done_issue = true;
+      progress = true;
       break;
     }
     const int type = op_type_of(w.iop, P.L), layer = op_layer_of(w.iop, P.L);
@@ -709,14 +747,13 @@ MK_INLINE void issue_more(Warp &w) {
     }
     if (!w.iop_init) {
       if (type == OP_ROUTED_GU || type == OP_DOWN) {
-        if (!routing_ready(w, layer)) return;
-        if (!route_cache(w, layer)) return;
+        if (!routing_ready(w, layer)) break;
+        if (!route_cache(w, layer)) break;
       }
       int stride;
       op_units(w, w.iop, type, layer, w.iu0, stride, w.in_units);
       w.istride = stride;
       w.iu = 0;
-      w.in_tiles = -1;
       w.iop_init = true;
     }
     if (w.iu >= w.in_units) {
@@ -724,22 +761,14 @@ MK_INLINE void issue_more(Warp &w) {
       w.iop_init = false;
       continue;
     }
-    if (w.in_tiles < 0) {
-      w.iunit = w.iu0 + w.iu * w.istride;
-      w.it = 0;
-      w.in_tiles = unit_tiles(w, type, layer, w.iunit);
-      if (type != OP_ATTN) unit_source(w, type, layer, w.iunit);
-      w.itype = type;
-      w.ilayer = layer;
-    }
-    if (w.it >= w.in_tiles) {
-      w.iu++;
-      w.in_tiles = -1;
-      continue;
-    }
-    issue_tile(w, type, layer, w.it);
-    w.it++;
+    w.iunit = w.iu0 + w.iu * w.istride;
+    w.it = 0;
+    w.in_tiles = unit_tiles(w, type, layer, w.iunit);
+    if (type != OP_ATTN) unit_source(w, type, layer, w.iunit);
+    w.itype = type;
+    w.ilayer = layer;
   }
+  return progress;
 }
 
 // ---------------------------------------------------------------------------
@@ -755,14 +784,10 @@ __device__ __noinline__ bool wait_slot_slow(uint64_t *bar, uint32_t par, unsigne
   }
 }
 
+// Consumer: wait (bounded) for the next tile of this warp's stream.
 MK_INLINE const uint8_t *consume_begin(Warp &w, int op) {
   if (w.failed) return nullptr;
-  if (w.inflight == 0) issue_more(w);
-  if (w.inflight == 0) {  // the tile stream and the consumer loop disagree: never expected
-    set_error(w, -8, op);
-    return nullptr;
-  }
-  uint64_t *bar = &w.bars[w.cslot];
+  uint64_t *bar = &w.full[w.cslot];
   const uint32_t par = (w.phase >> w.cslot) & 1u;
   const bool tr = w.P->trace != nullptr;
   const uint64_t t0 = tr ? now_ns() : 0;
@@ -783,14 +808,13 @@ MK_INLINE void consume_end(Warp &w) {
     w.tr_last = now_ns();
     w.tr_n++;
   }
-  __syncwarp();
+  __syncwarp();  // every lane is done with the slot before it is released
+  if (w.lane == 0) mbar_arrive(&w.empty[w.cslot]);
   w.phase ^= (1u << w.cslot);
   w.cslot = (w.cslot + 1 == kSlots) ? 0 : w.cslot + 1;
-  w.inflight--;
-  issue_more(w);
 }
 
-// Wait for `ctr` to reach `target` (bounded), filling the ring meanwhile.
+// Wait for `ctr` to reach `target` (bounded).
 MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int op) {
   const Params &P = *w.P;
   uint64_t t0 = 0;
@@ -805,7 +829,6 @@ MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int o
       w.failed = true;
       return false;
     }
-    issue_more(w);
     int bad = 0;
     if (w.lane == 0) {
       const uint64_t t = now_ns();
@@ -824,20 +847,17 @@ MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int o
   return true;
 }
 
-MK_INLINE void drain(Warp &w) {
-  // Wait (bounded) for every copy still in flight before the CTA may exit.
-  while (w.inflight > 0) {
-    uint64_t *bar = &w.bars[w.cslot];
-    const uint32_t par = (w.phase >> w.cslot) & 1u;
+// Producer, before the CTA exits: wait (bounded) until every tile it issued
+// for a consumer has landed, consumed or not.  The last fill of slot s
+// completes the phase of parity ephase bit s.
+MK_INLINE void drain_feed(const Warp &f) {
+  for (int s = 0; s < kSlots; ++s) {
+    if (!((f.filled >> s) & 1u)) continue;
     const uint64_t t0 = now_ns();
-    while (!mbar_try_wait(bar, par)) {
+    while (!mbar_try_wait(&f.full[s], (f.ephase >> s) & 1u)) {
       if (now_ns() - t0 > 50000000ull) break;
     }
-    w.phase ^= (1u << w.cslot);
-    w.cslot = (w.cslot + 1 == kSlots) ? 0 : w.cslot + 1;
-    w.inflight--;
   }
-  __syncwarp();
 }
 
 // Arrive on an op's counter once this warp's units of it are done.  Returns
@@ -851,7 +871,7 @@ MK_INLINE bool arrive(Warp &w, int op) {
     // the CTA; the CTA's last warp acquires them here and releases them, with
     // its own, grid-wide through the counter (release is cumulative).
     const uint32_t old = atom_add_acq_rel_cta(&w.arrive[op], 1u);
-    if (old == kWarpsPerCta - 1) {
+    if (old == kConsumers - 1) {
       const uint32_t g = atom_add_acq_rel(&P.counters[op * kCounterStride], 1u);
       last = (g + 1 == w.epoch * static_cast<uint32_t>(P.n_cta)) ? 1 : 0;
     }
@@ -1580,8 +1600,8 @@ MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op);
 
 // Shared-memory scratch of the attention items of one CTA.
 struct AttnShared {
-  float *o;           // [8 warps][kQvp][hd] warp partials (the staging row's space)
-  float *ml;          // [8 warps][kQvp][2]
+  float *o;           // [compute warps][kQvp][hd] partials (the staging row's space)
+  float *ml;          // [compute warps][kQvp][2]
   int *last;          // this CTA completed its group
   uint32_t *rdv;      // rendezvous counter
   uint32_t *seq;      // this warp's rendezvous count
@@ -1645,14 +1665,14 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
     sh.ml[(w.wib * kQvp + w.lane) * 2] = m_run;
     sh.ml[(w.wib * kQvp + w.lane) * 2 + 1] = l_run;
   }
-  *sh.seq += kWarpsPerCta;
+  *sh.seq += kConsumers;
   if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   const int grp = (a.b * P.Hkv + a.g) * P.attn_qsplit + a.qs;
   if (w.wib < kQvp) {
     const int v = w.wib;
-    float mw[kWarpsPerCta], M = -INFINITY;
+    float mw[kConsumers], M = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < kWarpsPerCta; ++k) {
+    for (int k = 0; k < kConsumers; ++k) {
       mw[k] = sh.ml[(k * kQvp + v) * 2];
       M = fmaxf(M, mw[k]);
     }
@@ -1660,7 +1680,7 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
 #pragma unroll
     for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
 #pragma unroll
-    for (int k = 0; k < kWarpsPerCta; ++k) {
+    for (int k = 0; k < kConsumers; ++k) {
       const float e = (mw[k] == -INFINITY) ? 0.f : expf(mw[k] - M);
       L += e * sh.ml[(k * kQvp + v) * 2 + 1];
 #pragma unroll
@@ -1675,21 +1695,21 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
       __stcg(ml + P.attn_nch_max + a.c, L);
     }
   }
-  *sh.seq += kWarpsPerCta;
+  *sh.seq += kConsumers;
   if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   uint32_t *cnt = P.attn_cnt + grp;
   if (w.wib == 0 && w.lane == 0) {
     __threadfence();
     *reinterpret_cast<volatile int *>(sh.last) = (atom_add_acq_rel(cnt, 1u) + 1 == static_cast<uint32_t>(a.nch)) ? 1 : 0;
   }
-  *sh.seq += kWarpsPerCta;
+  *sh.seq += kConsumers;
   if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   if (*reinterpret_cast<volatile int *>(sh.last)) {
     if (w.wib < kQvp) {
       (void)ld_acquire(cnt);  // every lane observes the completed count
       attn_final_merge<DPL>(P, w.lane, grp, w.wib, a.nch, a.b, a.g);
     }
-    *sh.seq += kWarpsPerCta;
+    *sh.seq += kConsumers;
     if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
     if (w.wib == 0 && w.lane == 0) *cnt = 0;  // rewind for the next layer
   }
@@ -1790,7 +1810,7 @@ MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, u
                            : (type == OP_QKV)    ? P.norms[2 * layer]
                            : (type == OP_LMHEAD) ? P.final_norm
                                                  : P.norms[2 * layer + 1];
-  for (int c4 = threadIdx.x; c4 < K / 4; c4 += kThreads) {
+  for (int c4 = threadIdx.x; c4 < K / 4; c4 += kConsumerThreads) {
     float4 v = __ldcg(src + c4);
     if (g) {
       const uint2 gb = __ldg(reinterpret_cast<const uint2 *>(g + 4 * c4));
@@ -1801,7 +1821,7 @@ MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, u
     }
     reinterpret_cast<float4 *>(xs)[c4] = v;
   }
-  seq += kWarpsPerCta;
+  seq += kConsumers;
   return cta_rendezvous(w, cnt, seq, op);
 }
 
@@ -1821,10 +1841,10 @@ MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t
           sg < U ? P.act_routed + static_cast<size_t>(sg) * kMaxRows * P.F : P.act_shared);
       const int K = sg < U ? P.F : P.Fs;
       float4 *dst = reinterpret_cast<float4 *>(xs + (sg - seg0) * ld);
-      for (int c4 = threadIdx.x; c4 < K / 4; c4 += kThreads) dst[c4] = __ldcg(src + c4);
+      for (int c4 = threadIdx.x; c4 < K / 4; c4 += kConsumerThreads) dst[c4] = __ldcg(src + c4);
     }
   }
-  seq += kWarpsPerCta;
+  seq += kConsumers;
   return cta_rendezvous(w, cnt, seq, op);
 }
 
@@ -1855,6 +1875,62 @@ MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs
   return true;
 }
 
+// Producer warp: keep the rings of its kFeeds consumers filled until every
+// tile of the launch's ops has been issued, then wait for the last copies.
+// With one consumer per producer its stream state stays in registers;
+// otherwise each consumer's state lives in shared memory between visits.
+MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane) {
+  Warp mine = feeds[first];
+  mine.lane = lane;
+  uint64_t t_idle = 0;
+  for (int it = 0;; ++it) {
+    bool progress = false, all_done = true;
+    if constexpr (kFeeds == 1) {
+      if (!mine.done_issue && !mine.failed) progress = feed_more(mine);
+      all_done = mine.done_issue || mine.failed;
+    } else {
+      for (int k = 0; k < kFeeds; ++k) {
+        Warp f = feeds[first + k];
+        if (f.done_issue || f.failed) continue;
+        f.lane = lane;
+        progress |= feed_more(f);
+        all_done = all_done && (f.done_issue || f.failed);
+        __syncwarp();
+        if (lane == 0) feeds[first + k] = f;
+        __syncwarp();
+      }
+    }
+    if (all_done) break;
+    int stop = 0;
+    if (lane == 0) {
+      if (*reinterpret_cast<volatile const int *>(P.error) != 0) {
+        stop = 1;
+      } else if (progress) {
+        t_idle = 0;
+      } else {
+        const uint64_t t = now_ns();
+        if (t_idle == 0) t_idle = t;
+        // consumers' own waits report a stall first (with the op that
+        // stalled); this bound only guarantees the producer ends
+        if (t - t_idle > 4 * P.timeout_ns) {
+          stop = 2;
+        } else if (it > 4) {
+          __nanosleep(32);
+        }
+      }
+    }
+    stop = __shfl_sync(0xffffffffu, stop, 0);
+    if (stop == 2) report_error(P, lane, -5, -1);
+    if (stop) break;
+  }
+  if constexpr (kFeeds == 1) {
+    drain_feed(mine);
+  } else {
+    for (int k = 0; k < kFeeds; ++k) drain_feed(feeds[first + k]);
+  }
+  __syncwarp();
+}
+
 template <int MMAX, bool XS>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1862,9 +1938,19 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   __shared__ int s_attn_nch[kMaxRows];
   __shared__ uint32_t s_stage;
   __shared__ RouteCache s_route;
-  __shared__ float s_attn_ml[kWarpsPerCta * kQvp * 2];
+  __shared__ float s_attn_ml[kConsumers * kQvp * 2];
   __shared__ int s_attn_last;
+  __shared__ Warp s_feed[kConsumers];  // each consumer's tile stream, as its producer keeps it
   const int wib = threadIdx.x >> 5;
+  const bool consumer = wib < kConsumers;
+  // dynamic shared memory: rings | activation row | full and empty barriers |
+  // epilogue scratch | per-op arrival counts
+  float *xs = reinterpret_cast<float *>(smem + kConsumers * kSlots * kSlotBytes);
+  uint8_t *after_xs = reinterpret_cast<uint8_t *>(xs + P.xs_floats);
+  uint64_t *fulls = reinterpret_cast<uint64_t *>(after_xs);
+  uint64_t *empties = fulls + kConsumers * kSlots;
+  float *fbase = reinterpret_cast<float *>(empties + kConsumers * kSlots);
+  uint32_t *arrive_cnt = reinterpret_cast<uint32_t *>(fbase + kConsumers * kWbuf);
   Warp w;
   w.P = &P;
   w.rc = &s_route;
@@ -1872,26 +1958,48 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.cta = blockIdx.x;
   w.lane = threadIdx.x & 31;
   w.nw = P.n_warps;
-  w.slot = wib * P.n_cta + blockIdx.x;
-  w.ring = smem + wib * kSlots * kSlotBytes;
-  float *xs = reinterpret_cast<float *>(smem + kWarpsPerCta * kSlots * kSlotBytes);
-  uint8_t *after_xs = reinterpret_cast<uint8_t *>(xs + P.xs_floats);
-  w.bars = reinterpret_cast<uint64_t *>(after_xs) + wib * kSlots;
-  float *fbase = reinterpret_cast<float *>(after_xs + kWarpsPerCta * kSlots * sizeof(uint64_t));
-  w.wbuf = fbase + wib * kWbuf;
-  w.arrive = reinterpret_cast<uint32_t *>(fbase + kWarpsPerCta * kWbuf);
+  w.slot = consumer ? wib * P.n_cta + blockIdx.x : -1;
+  const int c = consumer ? wib : 0;  // producers reach their consumers' records through s_feed
+  w.ring = smem + c * kSlots * kSlotBytes;
+  w.full = fulls + c * kSlots;
+  w.empty = empties + c * kSlots;
+  w.wbuf = fbase + c * kWbuf;
+  w.arrive = arrive_cnt;
   w.attn_prefix = s_attn_prefix;
   w.attn_nch = s_attn_nch;
   w.phase = 0;
-  w.cslot = w.islot = w.inflight = 0;
+  w.cslot = 0;
+  w.islot = 0;
+  w.ephase = (1u << kSlots) - 1u;  // a fresh barrier's previous phase counts as complete
+  w.filled = 0;
+  w.producer = false;
   w.failed = false;
   w.pol_w = policy_evict_first();
   w.pol_kv = policy_evict_normal();
-  if (w.lane == 0) {
-    for (int s = 0; s < kSlots; ++s) mbar_init(&w.bars[s], 1);
+  w.epoch = *reinterpret_cast<volatile const uint32_t *>(P.epoch) + 1u;
+  w.iop = P.op_begin;
+  w.iop_init = false;
+  w.done_issue = false;
+  w.iu0 = w.in_units = w.iu = w.it = w.iunit = 0;
+  w.itype = w.ilayer = 0;
+  w.istride = 1;
+  w.in_tiles = -1;
+  w.um = w.um2 = nullptr;
+  w.urow0 = w.urow2 = w.ucol0 = w.uK = 0;
+  w.uhalf = 1 << 30;
+  w.tr_first = w.tr_last = w.tr_wait = 0;
+  w.tr_n = 0;
+  if (consumer && w.lane == 0) {
+    for (int sl = 0; sl < kSlots; ++sl) {
+      mbar_init(&w.full[sl], 1);
+      mbar_init(&w.empty[sl], 1);
+    }
     fence_mbar_init();
+    Warp f = w;
+    f.producer = true;
+    s_feed[wib] = f;
   }
-  for (int i = threadIdx.x; i < P.n_ops; i += kThreads) w.arrive[i] = 0;
+  for (int i = threadIdx.x; i < P.n_ops; i += kThreads) arrive_cnt[i] = 0;
   if (threadIdx.x == 0) {
     s_stage = 0;
     s_route.ready_key = s_route.fill_key = 0;
@@ -1899,16 +2007,12 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     // attention work items per sequence
     s_attn_prefix[0] = 0;
     for (int b = 0; b < kMaxRows; ++b) {
-      const int nch = b < P.B ? cdiv(__ldg(&P.positions[b]) + P.T, P.attn_chunk * kWarpsPerCta) : 0;
+      const int nch = b < P.B ? cdiv(__ldg(&P.positions[b]) + P.T, P.attn_chunk * kConsumers) : 0;
       s_attn_nch[b] = nch;
       s_attn_prefix[b + 1] = s_attn_prefix[b] + P.Hkv * P.attn_qsplit * nch;
     }
   }
   __syncthreads();
-  uint32_t stage_seq = 0;
-  AttnShared ash{xs, s_attn_ml, &s_attn_last, &s_stage, &stage_seq};
-
-  w.epoch = *reinterpret_cast<volatile const uint32_t *>(P.epoch) + 1u;
 
   // Reject bad positions / token ids before any memory is touched with them.
   // Every warp evaluates the same condition, so all exit together.
@@ -1922,22 +2026,17 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     if (t < 0 || t >= P.V) bad = true;
   }
   if (__any_sync(0xffffffffu, bad)) {
-    set_error(w, -6, P.op_begin);
+    if (wib == 0) set_error(w, -6, P.op_begin);
     return;
   }
 
-  w.iop = P.op_begin;
-  w.iop_init = false;
-  w.done_issue = false;
-  w.iu0 = w.in_units = w.iu = w.it = w.iunit = 0;
-  w.itype = w.ilayer = 0;
-  w.istride = 1;
-  w.in_tiles = -1;
-  w.um = w.um2 = nullptr;
-  w.urow0 = w.urow2 = w.ucol0 = w.uK = 0;
-  w.uhalf = 1 << 30;
-  issue_more(w);
+  if (!consumer) {
+    producer_run(P, s_feed, (wib - kConsumers) * kFeeds, w.lane);
+    return;
+  }
 
+  uint32_t stage_seq = 0;
+  AttnShared ash{xs, s_attn_ml, &s_attn_last, &s_stage, &stage_seq};
   float am_val = -INFINITY;
   int am_idx = 0x7fffffff;
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {
@@ -1994,14 +2093,13 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     }
     if (last && type == OP_LMHEAD) final_argmax(P, w.lane, w.epoch);
   }
-  drain(w);
 }
 
 }  // namespace
 
 size_t step_smem_bytes(int n_ops, int xs_floats) {
-  return static_cast<size_t>(kWarpsPerCta) * kSlots * kSlotBytes + static_cast<size_t>(xs_floats) * sizeof(float) +
-         kWarpsPerCta * kSlots * sizeof(uint64_t) + kWarpsPerCta * kWbuf * sizeof(float) +
+  return static_cast<size_t>(kConsumers) * kSlots * kSlotBytes + static_cast<size_t>(xs_floats) * sizeof(float) +
+         2 * kConsumers * kSlots * sizeof(uint64_t) + kConsumers * kWbuf * sizeof(float) +
          static_cast<size_t>(n_ops) * sizeof(uint32_t);
 }
 

@@ -125,7 +125,7 @@ typedef struct mk_stats {
 typedef struct mk_plan_info {
   int32_t n_ops;           /* ops in one step's schedule                     */
   int32_t n_cta;           /* CTAs of the persistent grid (= SM count)       */
-  int32_t warps_per_cta;   /* consumer/producer warps per CTA                */
+  int32_t warps_per_cta;   /* compute warps per CTA (as many more issue TMA) */
   int32_t rows_per_tile;   /* weight rows per ring tile (4: tiles are 4 x 1024) */
   int32_t mmax;            /* row capacity of the kernel instance (1,2,4,8)  */
   int32_t attn_chunk;      /* KV positions per attention work item          */

@@ -136,11 +136,11 @@ def test_plan_shapes(L, model, B, T, cap):
     assert info.rows_per_tile == 4
     ppt = 2048 // model.head_dim
     assert info.attn_chunk % ppt == 0 and info.attn_chunk >= ppt
-    assert -(-cap // (8 * info.attn_chunk)) <= 32    # one merge level over CTA chunks
+    assert -(-cap // (info.warps_per_cta * info.attn_chunk)) <= 32    # one merge level over CTA chunks
     G = model.n_q_heads // model.n_kv_heads
     assert info.attn_qsplit == -(-G * T // 4)
     assert info.smem_bytes <= 227 * 1024
-    assert info.n_cta == 148 and info.warps_per_cta == 8
+    assert info.n_cta == 148 and 4 <= info.warps_per_cta <= 8   # compute warps (the rest issue TMA loads)
 
 
 def test_plan_rejects_shapes_beyond_the_handle(L):
