@@ -80,7 +80,7 @@ int encode_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, 
 struct Plan {
   int M, mmax, rows_per_tile, n_hb;
   int attn_qsplit, attn_ppt, attn_chunk, attn_nch_max;
-  int n_ops, n_cta, n_warps, xs_floats, qkv_split, down_groups, down_staged;
+  int n_ops, n_cta, n_warps, xs_floats, qkv_split, down_groups, down_staged, down_cols;
   size_t smem;
 };
 
@@ -135,6 +135,9 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
     const int fmax = std::max(d.expert_ffn, d.shared_ffn);
     p.down_staged = (std::min(span, segs) * ceil_div(fmax, 4) * 4 <= p.xs_floats) ? 1 : 0;
   }
+  // with one or two rows per step the two groups of an 8-row down unit can
+  // keep separate accumulators, so its tiles go column by column
+  p.down_cols = (p.down_groups == 2 && p.mmax <= 2) ? 1 : 0;
   p.smem = step_smem_bytes(p.n_ops, p.xs_floats);
   return p;
 }
@@ -473,6 +476,7 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.down_groups = pl.down_groups;
   p.n_db = pl.n_hb / pl.down_groups;
   p.down_staged = pl.down_staged;
+  p.down_cols = pl.down_cols;
   p.ss_ld = ceil_div(pl.n_hb, 128) * 128;
   p.e_ld = ceil_div(d.n_experts, 4) * 4;
   p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit;

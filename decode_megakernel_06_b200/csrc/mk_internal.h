@@ -100,6 +100,8 @@ struct alignas(64) Params {
   int qkv_split;       // QKV units cover 1 or 2 halves of K; the halves are summed by their reader
   int down_groups;     // 4-row groups per down-projection unit (1 or 2)
   int n_db;            // down-projection row blocks (n_hb / down_groups)
+  int down_cols;       // 8-row down units: boxes ordered column by column, both groups
+                       // per column (1-2 rows per step), else group by group
   int down_staged;     // batch 1: each CTA takes a contiguous range of down units and
                        // stages their experts' activations in shared memory
   int ss_ld;           // row stride of the sum-of-squares partials (n_hb rounded up to 128)

@@ -277,6 +277,7 @@ struct Warp {
   uint32_t ephase, filled;
   int islot;
   bool producer;
+  int dseg0;  // staged down projection: the first expert segment of this CTA's range
   // producer cursor: op, this consumer's unit index in it, tile in the unit
   int iop, iu0, in_units, iu, it, in_tiles, iunit;
   int itype, ilayer;  // type and layer of op iop, once its current unit is set up
@@ -508,9 +509,11 @@ MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
 
 // A staged (batch 1) down projection deals CTA c the contiguous units
 // [c * total / n_cta, (c + 1) * total / n_cta), warp by warp within the CTA.
+// (cta + 1) * total stays far below 2^31: at most 148 CTAs x 257 segments x
+// 1536 row blocks.
 MK_INLINE void down_cta_range(const Params &P, int cta, int total, int &c0, int &c1) {
-  c0 = static_cast<int>((static_cast<long long>(cta) * total) / P.n_cta);
-  c1 = static_cast<int>((static_cast<long long>(cta + 1) * total) / P.n_cta);
+  c0 = (cta * total) / P.n_cta;
+  c1 = ((cta + 1) * total) / P.n_cta;
 }
 
 // This warp's units of an op: u0, u0 + stride, ... (n of them).  Attention
@@ -690,7 +693,10 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * kBoxBytes);
       for (int p = 0; p < nbox; ++p) {
-        const int g = (b0 + p) / nbx, c = b0 + p - g * nbx;
+        // box b: group b % 2, column b / 2 (column order) or group b / nbx,
+        // column b % nbx (group order)
+        const int b = b0 + p;
+        const int g = P.down_cols ? (b & 1) : b / nbx, c = P.down_cols ? (b >> 1) : b - g * nbx;
         tma_load_2d(dst + p * kBoxBytes, w.um, c * kPanel, w.urow0 + g * kRows, bar, w.pol_w);
       }
     }
@@ -1063,37 +1069,79 @@ MK_INLINE bool gemv_unit(Warp &w, int op, int ntiles, int col0, int K, const XS 
 
 // A unit of `ngroups` groups of 4 rows over K columns, streamed box by box
 // (nbx boxes of 256 columns per group, four boxes per tile); when a group is
-// done its 4 x MJ sums are reduced across lanes into buf + g * 4 * MJ.
+// done its 4 x MJ sums are reduced across lanes into buf + g * 4 * MJ.  A
+// tile whose four boxes lie in one group runs unrolled with its activations
+// loaded first; a tile across two groups goes box by box.
+template <int MJ>
+MK_INLINE void group_done(float (&acc)[kRows * MJ], float (&acc2)[kRows * MJ], float *buf, int lane) {
+  if constexpr (MJ <= 2) {
+#pragma unroll
+    for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
+  }
+  butterfly<kRows * MJ>(acc, lane);
+  butterfly_store<kRows * MJ>(acc, buf, lane);
+#pragma unroll
+  for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
+}
+
+// Two 4-row groups with their boxes in column order: tile t holds (group 0,
+// column 2t), (group 1, column 2t), (group 0, column 2t + 1), (group 1,
+// column 2t + 1); each column's activations serve both groups.
+template <int MJ, class XS>
+MK_INLINE bool gemv_two_groups_by_column(Warp &w, int op, int K, const XS &xs, float *buf) {
+  const int nbx = cdiv(K, kPanel);
+  float a0[kRows * MJ], a0b[kRows * MJ], a1[kRows * MJ], a1b[kRows * MJ];
+#pragma unroll
+  for (int q = 0; q < kRows * MJ; ++q) a0[q] = a0b[q] = a1[q] = a1b[q] = 0.f;
+  for (int c = 0; c < nbx; c += 2) {
+    const uint8_t *slot = consume_begin(w, op);
+    if (!slot) return false;
+    const uint8_t *base = slot + w.lane * 16;
+    float x0[MJ][8], x1[MJ][8];
+    xs.load(c * kPanel + w.lane * 8, K, x0);
+    const bool two = c + 1 < nbx;
+    if (two) xs.load((c + 1) * kPanel + w.lane * 8, K, x1);
+    gemv_panel<MJ>(base, a0, a0b, x0);
+    gemv_panel<MJ>(base + kBoxBytes, a1, a1b, x0);
+    if (two) {
+      gemv_panel<MJ>(base + 2 * kBoxBytes, a0, a0b, x1);
+      gemv_panel<MJ>(base + 3 * kBoxBytes, a1, a1b, x1);
+    }
+    consume_end(w);
+  }
+  group_done<MJ>(a0, a0b, buf, w.lane);
+  group_done<MJ>(a1, a1b, buf + kRows * MJ, w.lane);
+  __syncwarp();
+  return true;
+}
+
 template <int MJ, class XS>
 MK_INLINE bool gemv_groups(Warp &w, int op, int ngroups, int K, const XS &xs, float *buf) {
+  if constexpr (MJ <= 2) {
+    if (ngroups == 2 && w.P->down_cols) return gemv_two_groups_by_column<MJ>(w, op, K, xs, buf);
+  }
   const int nbx = cdiv(K, kPanel), nb = ngroups * nbx;
   float acc[kRows * MJ], acc2[kRows * MJ];
 #pragma unroll
   for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
-  const uint8_t *slot = nullptr;
-  int g = 0, c = 0;
-  for (int b = 0; b < nb; ++b) {
-    const int p = b & (kPanels - 1);
-    if (p == 0) {
-      slot = consume_begin(w, op);
-      if (!slot) return false;
-    }
-    float x[MJ][8];
-    xs.load(c * kPanel + w.lane * 8, K, x);
-    gemv_panel<MJ>(slot + w.lane * 16 + p * kBoxBytes, acc, acc2, x);
-    if (p == kPanels - 1 || b == nb - 1) consume_end(w);
-    if (++c == nbx) {
-      if constexpr (MJ <= 2) {
-#pragma unroll
-        for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
+  for (int b0 = 0; b0 < nb; b0 += kPanels) {
+    const uint8_t *slot = consume_begin(w, op);
+    if (!slot) return false;
+    const uint8_t *base = slot + w.lane * 16;
+    const int g0 = b0 / nbx, c0 = b0 - g0 * nbx;
+    if (b0 + kPanels <= nb && c0 + kPanels <= nbx) {
+      gemv_tile<MJ>(slot, acc, acc2, c0 * kPanel, K, xs, w.lane);
+      if (c0 + kPanels == nbx) group_done<MJ>(acc, acc2, buf + g0 * kRows * MJ, w.lane);
+    } else {
+      for (int q = 0; q < kPanels && b0 + q < nb; ++q) {
+        const int b = b0 + q, g = b / nbx, c = b - g * nbx;
+        float x[MJ][8];
+        xs.load(c * kPanel + w.lane * 8, K, x);
+        gemv_panel<MJ>(base + q * kBoxBytes, acc, acc2, x);
+        if (c == nbx - 1) group_done<MJ>(acc, acc2, buf + g * kRows * MJ, w.lane);
       }
-      butterfly<kRows * MJ>(acc, w.lane);
-      butterfly_store<kRows * MJ>(acc, buf + g * kRows * MJ, w.lane);
-#pragma unroll
-      for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
-      c = 0;
-      ++g;
     }
+    consume_end(w);
   }
   __syncwarp();
   return true;
@@ -1395,11 +1443,9 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm)
   bool ok;
   if constexpr (XS && MJ == 1) {
     if (P.down_staged) {
-      // the CTA staged its experts' activations: slot seg - seg0 of the row
-      int c0, c1;
-      down_cta_range(P, w.cta, op_total_units(w, OP_DOWN, layer), c0, c1);
+      // the CTA staged its experts' activations: slot seg - dseg0 of the row
       XSmem xst;
-      xst.xs = xsm + (seg - c0 / P.n_db) * (cdiv(max(P.F, P.Fs), 4) * 4);
+      xst.xs = xsm + (seg - w.dseg0) * (cdiv(max(P.F, P.Fs), 4) * 4);
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xst, wb);
     } else {
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xs, wb);
@@ -1801,7 +1847,9 @@ MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op) {
 // Batch 1: the CTA stages the op's activation row in shared memory once
 // (x = h * g for normed ops, x = o for the o-projection); every warp then
 // reads its columns from there.  All warps take part, with or without units.
-MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, uint32_t &seq, int op) {
+// For normed ops it also sums h^2 over the columns each warp staged into
+// ssp[warp] (a fixed assignment, so the sum below is deterministic).
+MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, float *ssp, uint32_t *cnt, uint32_t &seq, int op) {
   const Params &P = *w.P;
   const bool oproj = type == OP_OPROJ;
   const int K = oproj ? P.Hq * P.hd : P.d;
@@ -1810,9 +1858,14 @@ MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, u
                            : (type == OP_QKV)    ? P.norms[2 * layer]
                            : (type == OP_LMHEAD) ? P.final_norm
                                                  : P.norms[2 * layer + 1];
+  float sq = 0.f;
   for (int c4 = threadIdx.x; c4 < K / 4; c4 += kConsumerThreads) {
     float4 v = __ldcg(src + c4);
     if (g) {
+      sq = fmaf(v.x, v.x, sq);
+      sq = fmaf(v.y, v.y, sq);
+      sq = fmaf(v.z, v.z, sq);
+      sq = fmaf(v.w, v.w, sq);
       const uint2 gb = __ldg(reinterpret_cast<const uint2 *>(g + 4 * c4));
       v.x *= bf_lo(gb.x);
       v.y *= bf_hi(gb.x);
@@ -1821,8 +1874,20 @@ MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, uint32_t *cnt, u
     }
     reinterpret_cast<float4 *>(xs)[c4] = v;
   }
+  if (g) {
+    sq = warp_sum(sq);
+    if (w.lane == 0) ssp[w.wib] = sq;
+  }
   seq += kConsumers;
   return cta_rendezvous(w, cnt, seq, op);
+}
+
+// 1 / rms of the staged row from the warps' partial sums (batch 1).
+MK_INLINE float staged_inv_rms(const Params &P, const float *ssp) {
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < kConsumers; ++k) s += ssp[k];
+  return 1.0f / sqrtf(s / static_cast<float>(P.d) + P.eps);
 }
 
 // Batch 1 down projection: the CTA copies the activations of the experts its
@@ -1834,6 +1899,7 @@ MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t
   const int U = n_union(w), total = op_total_units(w, OP_DOWN, layer);
   int c0, c1;
   down_cta_range(P, w.cta, total, c0, c1);
+  w.dseg0 = c0 / P.n_db;
   if (c1 > c0) {
     const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, ld = cdiv(max(P.F, P.Fs), 4) * 4;
     for (int sg = seg0; sg <= seg1; ++sg) {
@@ -1849,8 +1915,8 @@ MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t
 }
 
 template <int MMAX, bool XS>
-MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, AttnShared &ash, float &am_val,
-                           int &am_idx) {
+MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, const float *ssp, AttnShared &ash,
+                           float &am_val, int &am_idx) {
   const Params &P = *w.P;
   if ((type == OP_ROUTED_GU || type == OP_DOWN) && !route_cache(w, layer)) return false;
   int u0, stride, n;
@@ -1859,7 +1925,13 @@ MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs
   float inv[kMaxRows];
 #pragma unroll
   for (int m = 0; m < kMaxRows; ++m) inv[m] = 0.f;
-  if (type != OP_OPROJ && type != OP_DOWN && type != OP_ATTN) compute_inv_rms(P, w.lane, inv);
+  if (type != OP_OPROJ && type != OP_DOWN && type != OP_ATTN) {
+    if constexpr (XS) {
+      inv[0] = staged_inv_rms(P, ssp);  // the row staged for this op (or, for gate/up, by ROUTER)
+    } else {
+      compute_inv_rms(P, w.lane, inv);
+    }
+  }
   for (int i = 0; i < n; ++i) {
     const int u = u0 + i * stride;
     bool ok;
@@ -1941,6 +2013,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   __shared__ float s_attn_ml[kConsumers * kQvp * 2];
   __shared__ int s_attn_last;
   __shared__ Warp s_feed[kConsumers];  // each consumer's tile stream, as its producer keeps it
+  __shared__ float s_ssp[kConsumers];  // batch 1: partial sums of h^2 of the staged row
   const int wib = threadIdx.x >> 5;
   const bool consumer = wib < kConsumers;
   // dynamic shared memory: rings | activation row | full and empty barriers |
@@ -1973,6 +2046,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.ephase = (1u << kSlots) - 1u;  // a fresh barrier's previous phase counts as complete
   w.filled = 0;
   w.producer = false;
+  w.dseg0 = 0;
   w.failed = false;
   w.pol_w = policy_evict_first();
   w.pol_kv = policy_evict_normal();
@@ -2052,7 +2126,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       // launch that starts at one of those stages it itself
       const bool stage = type == OP_QKV || type == OP_OPROJ || type == OP_ROUTER || type == OP_LMHEAD ||
                          ((type == OP_SHARED_GU || type == OP_ROUTED_GU) && op == P.op_begin);
-      if (stage && !stage_x(w, type, layer, xs, &s_stage, stage_seq, op)) break;
+      if (stage && !stage_x(w, type, layer, xs, s_ssp, &s_stage, stage_seq, op)) break;
       if (type == OP_DOWN && P.down_staged && !stage_down(w, layer, xs, &s_stage, stage_seq, op)) break;
     }
     if (P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords] = now_ns();
@@ -2065,7 +2139,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       ok = route_cache(w, layer);
       if (ok) op_combine(w, layer);
     } else {
-      ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, ash, am_val, am_idx);
+      ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, s_ssp, ash, am_val, am_idx);
     }
     if (!ok || w.failed) break;
     if (type == OP_LMHEAD && (w.lane % kRows) == 0 && w.lane / kRows < P.M) {
