@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["mk_kernel.cu", "mk_api.cu"]
+SOURCES = ["mk_kernel.cu", "mk_api.cu", "mk_wide.cu"]
 HEADERS = ["mk_internal.h", os.path.join("..", "..", "include", "mk.h")]
 
 NVCC = os.environ.get("NVCC", "nvcc")

@@ -148,10 +148,12 @@ struct Sizes {
 
 Sizes scratch_sizes(const mk_model_desc &d, int n_sm) {
   Sizes s{};
-  for (int B = 1; B <= d.max_seqs; ++B)
-    for (int T = 1; B * T <= d.max_rows; ++T) {
+  // the persistent kernel serves blocks of up to kMaxRows rows
+  const int mseqs = std::min(d.max_seqs, kMaxRows), mrows = std::min(d.max_rows, kMaxRows);
+  for (int B = 1; B <= mseqs; ++B)
+    for (int T = 1; B * T <= mrows; ++T) {
       Plan p = make_plan(d, n_sm, B, T);
-      size_t ngrp = (size_t)d.max_seqs * d.n_kv_heads * p.attn_qsplit;
+      size_t ngrp = (size_t)mseqs * d.n_kv_heads * p.attn_qsplit;
       s.attn_o = std::max(s.attn_o, ngrp * p.attn_nch_max * kQvp * d.head_dim);
       s.attn_ml = std::max(s.attn_ml, ngrp * kQvp * 2 * p.attn_nch_max);
       s.attn_cnt = std::max(s.attn_cnt, ngrp);
@@ -199,6 +201,13 @@ struct mk_handle {
   mk_stats stats;
   std::vector<GraphEntry> graphs;
   cudaStream_t capture_stream;
+  // wide blocks (more than kMaxRows rows): scratch of the launch sequence
+  int wide_ldx, wide_lda;
+  float *w_h, *w_qkv, *w_o, *w_rlog, *w_selw, *w_gu, *w_yd, *w_gs, *w_ys, *w_part;
+  long long w_part_floats;
+  int32_t *w_sele, *w_tok, *w_pos;
+  int *w_count, *w_off, *w_pair_row, *w_pair_slot;
+  __nv_bfloat16 *w_xhi, *w_xlo, *w_ghi, *w_glo, *w_ahi, *w_alo, *w_shi, *w_slo;
 };
 
 extern "C" {
@@ -222,8 +231,8 @@ MK_API int mk_validate_desc(const mk_model_desc *d) {
   if (d->vocab < 1) return fail(MK_ERR_ARG, "vocab must be >= 1");
   if (d->d_model > 6144 || d->n_q_heads * d->head_dim > 6144)
     return fail(MK_ERR_UNSUPPORTED, "d_model and n_q_heads*head_dim must be <= 6144");
-  if (d->max_rows < 1 || d->max_rows > kMaxRows)
-    return fail(MK_ERR_UNSUPPORTED, "max_rows must be in [1, %d]", kMaxRows);
+  if (d->max_rows < 1 || d->max_rows > kWideMaxRows)
+    return fail(MK_ERR_UNSUPPORTED, "max_rows must be in [1, %d]", kWideMaxRows);
   if (d->max_seqs < 1 || d->max_seqs > d->max_rows) return fail(MK_ERR_ARG, "max_seqs must be in [1, max_rows]");
   if (d->kv_capacity < 1) return fail(MK_ERR_ARG, "kv_capacity must be >= 1");
   if (!(d->rope_theta > 0.f) || !(d->rms_eps >= 0.f)) return fail(MK_ERR_ARG, "rope_theta > 0 and rms_eps >= 0 required");
@@ -243,6 +252,9 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
   if (n_sm < 1) return fail(MK_ERR_ARG, "n_sm must be >= 1");
   if (B < 1 || T < 1 || B > desc->max_seqs || B * T > desc->max_rows)
     return fail(MK_ERR_CAPACITY, "B=%d T=%d outside max_seqs=%d max_rows=%d", B, T, desc->max_seqs, desc->max_rows);
+  if (B * T > kMaxRows)
+    return fail(MK_ERR_UNSUPPORTED, "B*T=%d: blocks above %d rows run as a sequence of launches, not a schedule",
+                B * T, kMaxRows);
   Plan p = make_plan(*desc, n_sm, B, T);
   if (info) {
     info->n_ops = p.n_ops;
@@ -352,7 +364,7 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   const int L = d.n_layers, D = d.d_model, QKVW = (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim;
   const int n_ops = n_ops_for(L), NW = n_sm * kConsumers;
   Sizes s = scratch_sizes(d, n_sm);
-  const int umax = std::min(d.n_experts, d.max_rows * d.top_k);
+  const int umax = std::min(d.n_experts, std::min(d.max_rows, kMaxRows) * d.top_k);
   HALLOC(h->tmaps, sizeof(CUtensorMap) * (size_t)(L * MAPS_PER_LAYER + 1));
   HALLOC(h->norms, sizeof(void *) * 2 * L);
   HALLOC(h->h, sizeof(float) * (size_t)kMaxRows * D);
@@ -375,9 +387,49 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->error, sizeof(int) * kCounterStride);
   HALLOC(h->stats_dev, sizeof(unsigned long long) * 4);
   HALLOC(h->logits, sizeof(float) * (size_t)d.max_rows * d.vocab);
-  HALLOC(h->io_tokens, sizeof(int32_t) * kMaxRows);
-  HALLOC(h->io_positions, sizeof(int32_t) * kMaxRows);
-  HALLOC(h->io_argmax, sizeof(int32_t) * kMaxRows);
+  HALLOC(h->io_tokens, sizeof(int32_t) * (size_t)d.max_rows);
+  HALLOC(h->io_positions, sizeof(int32_t) * (size_t)d.max_seqs);
+  HALLOC(h->io_argmax, sizeof(int32_t) * (size_t)d.max_rows);
+  if (d.max_rows > kMaxRows) {  // buffers of the wide-block path
+    const int MR = d.max_rows, MK = MR * d.top_k, HD = d.n_q_heads * d.head_dim;
+    const int ldx = ceil_div(std::max(D, HD), 8) * 8, lda = ceil_div(std::max(d.expert_ffn, std::max(d.shared_ffn, 1)), 8) * 8;
+    const int Fs = std::max(d.shared_ffn, 1);
+    h->wide_ldx = ldx;
+    h->wide_lda = lda;
+    HALLOC(h->w_h, sizeof(float) * (size_t)MR * D);
+    HALLOC(h->w_qkv, sizeof(float) * (size_t)MR * QKVW);
+    HALLOC(h->w_o, sizeof(float) * (size_t)MR * HD);
+    HALLOC(h->w_rlog, sizeof(float) * (size_t)MR * d.n_experts);
+    HALLOC(h->w_selw, sizeof(float) * (size_t)MK);
+    HALLOC(h->w_sele, sizeof(int32_t) * (size_t)MK);
+    HALLOC(h->w_count, sizeof(int) * (size_t)d.n_experts);
+    HALLOC(h->w_off, sizeof(int) * (size_t)d.n_experts);
+    HALLOC(h->w_pair_row, sizeof(int) * (size_t)MK);
+    HALLOC(h->w_pair_slot, sizeof(int) * (size_t)MK);
+    HALLOC(h->w_tok, sizeof(int32_t) * (size_t)MR);
+    HALLOC(h->w_pos, sizeof(int32_t) * (size_t)d.max_seqs);
+    HALLOC(h->w_xhi, sizeof(__nv_bfloat16) * (size_t)MR * ldx);
+    HALLOC(h->w_xlo, sizeof(__nv_bfloat16) * (size_t)MR * ldx);
+    HALLOC(h->w_ghi, sizeof(__nv_bfloat16) * (size_t)MK * ldx);
+    HALLOC(h->w_glo, sizeof(__nv_bfloat16) * (size_t)MK * ldx);
+    HALLOC(h->w_gu, sizeof(float) * (size_t)MK * 2 * d.expert_ffn);
+    HALLOC(h->w_ahi, sizeof(__nv_bfloat16) * (size_t)MK * lda);
+    HALLOC(h->w_alo, sizeof(__nv_bfloat16) * (size_t)MK * lda);
+    HALLOC(h->w_yd, sizeof(float) * (size_t)MK * D);
+    HALLOC(h->w_gs, sizeof(float) * (size_t)MR * 2 * Fs);
+    HALLOC(h->w_shi, sizeof(__nv_bfloat16) * (size_t)MR * lda);
+    HALLOC(h->w_slo, sizeof(__nv_bfloat16) * (size_t)MR * lda);
+    HALLOC(h->w_ys, sizeof(float) * (size_t)MR * D);
+    // split-K partials of the dense products: at most 16 K shares of MR rows
+    const int ld_max = std::max(std::max(QKVW, D), std::max(2 * Fs, std::max(d.n_experts, HD)));
+    h->w_part_floats = 16LL * MR * ld_max;
+    HALLOC(h->w_part, sizeof(float) * (size_t)h->w_part_floats);
+    cudaError_t pe = wide_prepare();
+    if (pe != cudaSuccess) {
+      mk_destroy(h);
+      return fail(MK_ERR_CUDA, "wide-block setup failed: %s", cudaGetErrorString(pe));
+    }
+  }
 
   // tensor maps of every weight matrix
   std::vector<CUtensorMap> maps((size_t)L * MAPS_PER_LAYER + 1);
@@ -520,9 +572,52 @@ static int launch_variant(mk_handle *h, Params &p, const Plan &pl, cudaStream_t 
   return MK_OK;
 }
 
+// A block of more than kMaxRows rows: the launch sequence of mk_wide.cu.
+static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T, mk_kv_cache kv,
+                    float *logits, int32_t *argmax, cudaStream_t stream) {
+  const mk_model_desc &d = h->desc;
+  if (!tokens || !positions || !argmax) return fail(MK_ERR_ARG, "tokens, positions and out_argmax are required");
+  if (!kv.k || !kv.v) return fail(MK_ERR_ARG, "kv.k and kv.v are required");
+  if (B > d.max_seqs || (long long)B * T > d.max_rows)
+    return fail(MK_ERR_CAPACITY, "B=%d T=%d exceeds max_seqs=%d / max_rows=%d", B, T, d.max_seqs, d.max_rows);
+  if (T > d.kv_capacity) return fail(MK_ERR_CAPACITY, "T=%d exceeds kv_capacity=%d", T, d.kv_capacity);
+  WideStep s{};
+  s.L = d.n_layers; s.d = d.d_model; s.Hq = d.n_q_heads; s.Hkv = d.n_kv_heads; s.hd = d.head_dim;
+  s.E = d.n_experts; s.topk = d.top_k; s.F = d.expert_ffn; s.Fs = d.shared_ffn; s.V = d.vocab;
+  s.Bmax = d.max_seqs; s.cap = d.kv_capacity; s.eps = d.rms_eps;
+  s.layers = h->layers.data();
+  s.embed = static_cast<const __nv_bfloat16 *>(h->embed);
+  s.final_norm = static_cast<const __nv_bfloat16 *>(h->final_norm);
+  s.lm_head = static_cast<const __nv_bfloat16 *>(h->lm_head);
+  s.rope = h->rope;
+  s.B = B; s.T = T; s.max_rows = d.max_rows; s.n_sm = h->n_sm;
+  s.tokens = tokens; s.positions = positions;
+  s.tokens_safe = h->w_tok; s.positions_safe = h->w_pos;
+  s.kc = static_cast<__nv_bfloat16 *>(kv.k); s.vc = static_cast<__nv_bfloat16 *>(kv.v);
+  s.logits = logits ? logits : h->logits;
+  s.argmax = argmax;
+  s.error = h->error;
+  s.stats = h->stats_dev;
+  s.dbg_hidden = h->dbg_hidden; s.dbg_ids = h->dbg_ids; s.dbg_w = h->dbg_w;
+  s.ldx = h->wide_ldx; s.lda = h->wide_lda;
+  s.h = h->w_h; s.qkv = h->w_qkv; s.o = h->w_o; s.rlog = h->w_rlog; s.sel_w = h->w_selw; s.gu = h->w_gu;
+  s.yd = h->w_yd; s.gs = h->w_gs; s.ys = h->w_ys; s.part = h->w_part; s.part_floats = h->w_part_floats;
+  s.sel_e = h->w_sele; s.count = h->w_count; s.off = h->w_off; s.pair_row = h->w_pair_row;
+  s.pair_slot = h->w_pair_slot;
+  s.xhi = h->w_xhi; s.xlo = h->w_xlo; s.ghi = h->w_ghi; s.glo = h->w_glo; s.ahi = h->w_ahi; s.alo = h->w_alo;
+  s.shi = h->w_shi; s.slo = h->w_slo;
+  int launches = 0;
+  cudaError_t e = wide_step(s, stream, &launches);
+  if (e != cudaSuccess) return fail(MK_ERR_LAUNCH, "wide-block launch failed: %s", cudaGetErrorString(e));
+  h->stats.kernel_launches += launches;
+  h->stats.steps += 1;
+  return MK_OK;
+}
+
 static int run_step(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T,
                     mk_kv_cache kv, float *logits, int32_t *argmax, cudaStream_t stream) {
   if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (B >= 1 && T >= 1 && (long long)B * T > kMaxRows) return run_wide(h, tokens, positions, B, T, kv, logits, argmax, stream);
   Params p;
   Plan pl;
   int rc = fill_params(h, tokens, positions, B, T, kv, logits, argmax, p, pl);
@@ -723,6 +818,8 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
                                  int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
                                  int32_t *out_argmax, void *stream) {
   if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (B >= 1 && T >= 1 && (long long)B * T > kMaxRows)
+    return fail(MK_ERR_UNSUPPORTED, "B*T=%d: blocks above %d rows take mk_decode_step", B * T, kMaxRows);
   int dev = -1;
   CUDA_TRY(cudaGetDevice(&dev));
   if (dev != h->device) return fail(MK_ERR_ARG, "device %d is current, the handle lives on device %d", dev, h->device);
@@ -737,7 +834,7 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
   const mk_model_desc &d = h->desc;
   const int L = d.n_layers, D = d.d_model, QKVW = (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim;
   const size_t ngrp = (size_t)B * d.n_kv_heads * pl.attn_qsplit;
-  const int umax = std::min(d.n_experts, d.max_rows * d.top_k);
+  const int umax = std::min(d.n_experts, std::min(d.max_rows, kMaxRows) * d.top_k);
   StaticCarve c;
   // words that must read zero when the step starts, first, so one memset clears them
   c.take(p.counters, base, sizeof(uint32_t) * (size_t)pl.n_ops * kCounterStride);

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/mk.h"
+
 namespace mk {
 
 // ---- geometry ------------------------------------------------------------------
@@ -139,6 +141,40 @@ struct alignas(64) Params {
 
 // Launch entry points implemented in mk_kernel.cu.
 int launch_step(const Params &p, int mmax, bool cooperative, cudaStream_t stream);
+// ---- wide blocks (8 < M <= 64 rows): a sequence of launches ----------------------
+constexpr int kWideMaxRows = 64;
+
+struct WideStep {
+  // model
+  int L, d, Hq, Hkv, hd, E, topk, F, Fs, V, Bmax, cap;
+  float eps;
+  const mk_layer_weights *layers;  // host array [L]
+  const __nv_bfloat16 *embed, *final_norm, *lm_head;
+  const float2 *rope;
+  // step
+  int B, T, max_rows, n_sm;
+  const int32_t *tokens, *positions;
+  int32_t *tokens_safe, *positions_safe;
+  __nv_bfloat16 *kc, *vc;
+  float *logits;
+  int32_t *argmax;
+  int *error;
+  unsigned long long *stats;
+  float *dbg_hidden;
+  int32_t *dbg_ids;
+  float *dbg_w;
+  // scratch
+  int ldx, lda;
+  float *h, *qkv, *o, *rlog, *sel_w, *gu, *yd, *gs, *ys, *part;
+  long long part_floats;
+  int32_t *sel_e;
+  int *count, *off, *pair_row, *pair_slot;
+  __nv_bfloat16 *xhi, *xlo, *ghi, *glo, *ahi, *alo, *shi, *slo;
+};
+
+cudaError_t wide_prepare();
+cudaError_t wide_step(const WideStep &s, cudaStream_t stream, int *launches);
+
 size_t step_smem_bytes(int n_ops, int xs_floats);
 bool kernel_stages_x(int mmax);
 int max_cta_per_sm(int mmax, size_t smem);

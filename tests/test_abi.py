@@ -68,7 +68,7 @@ def test_validate_accepts_the_workload_models(L):
     ("top_k", 9, mk.MK_ERR_ARG),
     ("expert_ffn", 40, mk.MK_ERR_ARG),
     ("shared_ffn", 8, mk.MK_ERR_ARG),
-    ("max_rows", 9, mk.MK_ERR_UNSUPPORTED),
+    ("max_rows", 65, mk.MK_ERR_UNSUPPORTED),
     ("max_seqs", 0, mk.MK_ERR_ARG),
     ("variant", 3, mk.MK_ERR_ARG),
     ("rope_theta", 0.0, mk.MK_ERR_ARG),

@@ -71,6 +71,43 @@ def test_ragged_shapes(B, T):
     print(B, T, rep)
 
 
+# Blocks of more than 8 rows take the tensor-core launch sequence: the
+# speculative verify block of 8 sequences x 7 rows on the small model, and the
+# ragged model (K = 264, F = 48, Fs = 32 off every 64-column tile) at 15, 64
+# and 16 x 4 rows.
+def test_verify_block_56_rows():
+    s = Session(workload("verify", 8))
+    rep = run_verify(s, 2)
+    s.close()
+    assert rep.rows_compared >= 56
+    print(rep)
+
+
+@pytest.mark.parametrize("B,T", [(3, 5), (8, 8), (16, 4)])
+def test_ragged_wide_blocks(B, T):
+    wl = Workload(f"ragged_wide_b{B}_t{T}", RAGGED, B, T, context=None, context_range=(1, 70), steps=3, seed=11)
+    s = Session(wl, capacity=96)
+    rep = run_greedy(s, 2) if T == 1 else run_verify(s, 2)
+    s.close()
+    assert rep.rows_compared >= B * T
+    print(B, T, rep)
+
+
+def test_wide_block_rejects_bad_inputs_on_device():
+    wl = Workload("ragged_wide_bad", RAGGED, 4, 4, context=None, context_range=(1, 40), steps=1, seed=12)
+    s = Session(wl, capacity=64)
+    dev = s.dev
+    tok = torch.full((16,), 3, dtype=torch.int32, device=dev)
+    tok[5] = RAGGED.vocab
+    pos = torch.tensor([10, 10, 10, 10], dtype=torch.int32, device=dev)
+    assert s.dec.step(tok, pos, 4, 4, s.k, s.v, s.logits, s.argmax) == mk.MK_OK
+    assert s.dec.status() == mk.MK_ERR_DEVICE_CHECK
+    tok[5] = 1
+    assert s.dec.step(tok, pos, 4, 4, s.k, s.v, s.logits, s.argmax) == mk.MK_OK
+    assert s.dec.status() == mk.MK_OK
+    s.close()
+
+
 def test_empty_cache_and_full_capacity():
     """Position 0 (the token attends only itself) and a block ending exactly at
     the last cache slot."""
