@@ -389,6 +389,35 @@ def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr, save=None):
     return rows
 
 
+def measure_verify_wide(device, steps=10, warmup=3):
+    """The 56-row speculative-verify block (8 sequences x 7 rows, the small
+    model) through the wide-block tensor-core path."""
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+    from synthetic import make_kv_cache, make_weights, workload
+
+    wl = workload("verify", 8)
+    m, B, T = wl.model, wl.batch, wl.tokens_per_step
+    w = make_weights(m, wl.seed, device)
+    ctx = [wl.context] * B
+    cap = (wl.context + (steps + warmup + 2) * T + 63) // 64 * 64
+    k, v = make_kv_cache(m, B, cap, wl.seed, device)
+    dec = mk.Decoder(m, w, max_rows=B * T, max_seqs=B, kv_capacity=cap)
+    total, per, st = time_steps(dec, m, k, v, B, T, ctx, steps, warmup, device)
+    union = st.expert_union_total / steps / m.n_layers
+    lens = [c + (warmup + steps // 2) * T + T for c in ctx]
+    by = step_bytes(m, B, T, lens, st.expert_union_total / steps)
+    ms = total / steps
+    dec.close()
+    del w, k, v
+    torch.cuda.empty_cache()
+    return {"workload": f"{wl.name} ({m.name} model, {B * T} rows per step)", "ms_per_step": round(ms, 4),
+            "rows_per_s": round(B * T / (ms / 1e3), 1), "hbm_gbs": round(by / (ms / 1e3) / 1e9, 1),
+            "expert_union_per_layer": round(union, 1), "launches_per_step": st.kernel_launches // steps,
+            "path": "tensor-core launch sequence (blocks above 8 rows)"}
+
+
 def run_mine(args):
     import torch
 
@@ -461,6 +490,10 @@ def run_mine(args):
             sweep[f"bs{bb}"] = row
         dec.set_variant(args.variant)
 
+    verify56 = None
+    if args.sweep and ws == 1 and args.workload == "large":
+        verify56 = measure_verify_wide(device)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         o = oracle_sample(m, w, k, v, B, T, ctx, 1, min_compute_s=10.0)
@@ -499,6 +532,8 @@ def run_mine(args):
         }
         if sweep is not None:
             line["batch_sweep"] = sweep
+        if verify56 is not None:
+            line["verify_56"] = verify56
         print(json.dumps(line), flush=True)
     dec.close()
     import torch.distributed as dist

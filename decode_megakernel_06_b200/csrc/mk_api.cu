@@ -90,9 +90,15 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.mmax = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
   p.rows_per_tile = kRows;
   p.n_hb = ceil_div(d.d_model, kRows);
-  // QKV has few row blocks per warp (1536 for 1184 warps at the large model);
-  // halving K per unit evens out the warps' shares.
-  p.qkv_split = ceil_div(d.d_model, kTileCols) >= 2 ? 2 : 1;
+  // QKV has few row blocks per warp; halving K per unit can even out the
+  // warps' shares.  Split only if it lowers the busiest warp's tiles (each
+  // unit costs a fixed overhead besides its tiles).
+  {
+    const int nt = ceil_div(d.d_model, kTileCols), nrb = ceil_div((d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim, kRows);
+    const int nw = n_sm * kConsumers;
+    const int full = ceil_div(nrb, nw) * nt, half = ceil_div(2 * nrb, nw) * ceil_div(nt, 2);
+    p.qkv_split = (nt >= 2 && half < full) ? 2 : 1;
+  }
   // Down projection: two 4-row groups per unit when the F (or Fs) columns leave
   // the 1024-column tiles partly empty, as long as the units still outnumber
   // the warps two to one; the tiles then come out full.

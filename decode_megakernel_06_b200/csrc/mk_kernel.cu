@@ -1506,6 +1506,23 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
 // One warp's share of an item: online softmax over its positions for the kQvp
 // query vectors of the item's group, left in registers (lane l keeps the
 // running (max, sum) of query l % kQvp, and o for all of them over its dims).
+// DPL consecutive bf16 values of a K or V row (this lane's dimensions) in one load.
+template <int DPL>
+MK_INLINE void load_bf16_dims(const __nv_bfloat16 *p, float (&f)[DPL]) {
+  static_assert(DPL == 2 || DPL == 4, "head_dim 64 or 128");
+  if constexpr (DPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    f[0] = bf_lo(u.x);
+    f[1] = bf_hi(u.x);
+    f[2] = bf_lo(u.y);
+    f[3] = bf_hi(u.y);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
+    f[0] = bf_lo(u);
+    f[1] = bf_hi(u);
+  }
+}
+
 template <int DPL>
 MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, float &m_run, float &l_run,
                          float (&o)[kQvp][DPL]) {
@@ -1590,9 +1607,7 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, float &m
 #pragma unroll
       for (int j = 0; j < PG; ++j) {
         float kf[DPL];
-        const __nv_bfloat16 *kr = ks + (jg + j) * hd + lane * DPL;
-#pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) kf[dd] = __bfloat162float(kr[dd]);
+        load_bf16_dims<DPL>(ks + (jg + j) * hd + lane * DPL, kf);
 #pragma unroll
         for (int v = 0; v < QVP; ++v) {
           float sc = 0.f;
@@ -1623,18 +1638,21 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, float &m
 #pragma unroll
         for (int dd = 0; dd < DPL; ++dd) o[v][dd] *= av;
       }
+      // every lane needs all 32 probabilities: one store each, then 8 float4
+      // broadcast loads from the warp's scratch (lane 4j + v holds position j, query v)
+      __syncwarp();
+      w.wbuf[lane] = pr;
+      __syncwarp();
 #pragma unroll
       for (int j = 0; j < PG; ++j) {
         float vf[DPL];
-        const __nv_bfloat16 *vr = vs + (jg + j) * hd + lane * DPL;
+        load_bf16_dims<DPL>(vs + (jg + j) * hd + lane * DPL, vf);
+        const float4 p4 = *reinterpret_cast<const float4 *>(w.wbuf + j * QVP);
+        const float pj[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) vf[dd] = __bfloat162float(vr[dd]);
+        for (int v = 0; v < QVP; ++v)
 #pragma unroll
-        for (int v = 0; v < QVP; ++v) {
-          const float pj = __shfl_sync(0xffffffffu, pr, j * QVP + v);
-#pragma unroll
-          for (int dd = 0; dd < DPL; ++dd) o[v][dd] = fmaf(pj, vf[dd], o[v][dd]);
-        }
+          for (int dd = 0; dd < DPL; ++dd) o[v][dd] = fmaf(pj[v], vf[dd], o[v][dd]);
       }
     }
     consume_end(w);
