@@ -141,11 +141,11 @@ def mk_validate_desc(desc: mk_model_desc) -> int:
 def mk_plan_describe(desc: mk_model_desc, n_sm: int, B: int, T: int):
     """Returns (rc, mk_plan_info, [(type, layer, dep0, dep1)] per op)."""
     info = mk_plan_info()
-    n = 8 * desc.n_layers + 2
+    n = 8 * desc.n_layers + 2  # an upper bound on the schedule's length
     arrs = [(ctypes.c_int32 * n)() for _ in range(4)]
     rc = lib().mk_plan_describe(ctypes.byref(desc), n_sm, B, T, ctypes.byref(info),
                                 *[ctypes.cast(a, _I32P) for a in arrs], n)
-    ops = list(zip(*[list(a) for a in arrs])) if rc == MK_OK else []
+    ops = list(zip(*[list(a)[:info.n_ops] for a in arrs])) if rc == MK_OK else []
     return rc, info, ops
 
 
