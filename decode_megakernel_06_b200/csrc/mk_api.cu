@@ -126,8 +126,8 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.attn_nch_max = ceil_div(d.kv_capacity, c * kConsumers);
   p.n_ops = n_ops_for(d.n_layers);
   // shared-memory row: the staged activations (batch 1) or the attention
-  // warps' partials, whichever is larger
-  p.xs_floats = std::max(kConsumers * kQvp * d.head_dim,
+  // warps' partials and the item's query vectors, whichever is larger
+  p.xs_floats = std::max((kConsumers + 1) * kQvp * d.head_dim,
                          kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), 4) * 4 : 0);
   // Batch 1 down projection: a CTA's contiguous range of units spans at most
   // 1 + ceil(range / row blocks) experts; their activations must fit the

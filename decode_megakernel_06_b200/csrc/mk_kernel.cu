@@ -64,13 +64,14 @@ MK_INLINE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking: has the phase of `parity` completed?
-MK_INLINE bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+// Blocking with a time limit: the thread may be suspended (issuing nothing)
+// for up to about `ns` nanoseconds until the phase of `parity` completes.
+MK_INLINE bool mbar_wait_hint(uint64_t *bar, uint32_t parity, uint32_t ns) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
-      : "r"(saddr(bar)), "r"(parity)
+      : "r"(saddr(bar)), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }
@@ -208,6 +209,14 @@ MK_INLINE void butterfly_store(const float (&v)[N], float *buf, int lane) {
   }
 }
 
+// Order-preserving map of a float onto uint32 (a larger float has a larger
+// key), for warp-wide integer max reductions, and its inverse.
+MK_INLINE uint32_t float_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+MK_INLINE float key_float(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k); }
+
 MK_INLINE float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -322,9 +331,13 @@ MK_INLINE int expert_of(int lane, int i) { return (i < 4) ? 4 * lane + i : 128 +
 
 // The CTA's routing for `layer` (one warp; the caller has seen the router's
 // partials complete).  Per row: logits = the split-K partials summed in a
-// fixed order; softmax over the E experts; k rounds of argmax (ties to the
-// lower expert id); weights renormalised by their sum.  Every CTA runs this
-// on the same partials and gets the same result.
+// fixed order; k rounds of argmax (ties to the lower expert id); weights =
+// the softmax renormalised over the chosen experts.  Softmax is monotone, so
+// ranking the logits ranks the probabilities, and the full softmax's
+// normaliser cancels in the renormalisation: w_j = e^(z_j - z_max) /
+// sum over chosen i of e^(z_i - z_max).  Every CTA runs this on the same
+// partials and gets the same result.  The code runs once per layer per CTA
+// (cold), so it is kept short.
 __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int lane, int layer) {
   const int E = P.E, K = P.topk;
   const int nkc = cdiv(P.d, kTileCols);
@@ -340,6 +353,7 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
     float z[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) z[i] = 0.f;
+    // up to 8 K-chunks' partials in flight at once
     for (int k0 = 0; k0 < nkc; k0 += 8) {
       float4 va[8], vb[8];
 #pragma unroll
@@ -357,61 +371,43 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
         z[4] += vb[k].x; z[5] += vb[k].y; z[6] += vb[k].z; z[7] += vb[k].w;
       }
     }
-    bool taken[EPL];
-    float mx = -INFINITY;
+    // the keys of this lane's experts; 0 = not a candidate (absent or taken)
+    uint32_t key[EPL];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      taken[i] = expert_of(lane, i) >= E;
-      if (!taken[i]) mx = fmaxf(mx, z[i]);
-    }
-    mx = warp_max(mx);
-    float pi[EPL], sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      pi[i] = taken[i] ? 0.f : expf(z[i] - mx);
-      sum += pi[i];
-    }
-    sum = warp_sum(sum);
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) pi[i] = pi[i] / sum;
-    // k rounds of argmax; lane j keeps selection j
-    float sel = 0.f, my_w = 0.f;
+    for (int i = 0; i < EPL; ++i) key[i] = expert_of(lane, i) < E ? float_key(z[i]) : 0u;
+    // k rounds of argmax; lane j keeps selection j.  The lane scans its
+    // candidates in ascending expert id (strict >), and among lanes holding
+    // the maximum the lowest id wins.
+    float my_z = 0.f;
     int my_e = 0;
     for (int j = 0; j < K; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+      uint32_t bk = 0u;
+      int bl = 0;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = expert_of(lane, i);
-        if (!taken[i] && (pi[i] > bv || (pi[i] == bv && e < bi))) {
-          bv = pi[i];
-          bi = e;
+      for (int i = 0; i < EPL; ++i)
+        if (key[i] > bk) {
+          bk = key[i];
+          bl = expert_of(lane, i);
         }
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
+      const uint32_t best = __reduce_max_sync(0xffffffffu, bk);
+      const int bi = static_cast<int>(__reduce_min_sync(0xffffffffu, bk == best ? static_cast<uint32_t>(bl) : 0xffffffffu));
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
         if (expert_of(lane, i) == bi) {
-          taken[i] = true;
+          key[i] = 0u;
           chosen[i] |= 1u << m;
           slots[i] |= static_cast<uint64_t>(j) << (8 * m);
         }
       if (lane == j) {
         my_e = bi;
-        my_w = bv;
+        my_z = key_float(best);
       }
-      sel += bv;
     }
+    const float zmax = __shfl_sync(0xffffffffu, my_z, 0);
+    const float e = lane < K ? expf(my_z - zmax) : 0.f;
+    const float sel = warp_sum(e);
     if (lane < K) {
-      rc->row_w[m][lane] = my_w / sel;
+      rc->row_w[m][lane] = e / sel;
       rc->row_e[m][lane] = static_cast<uint8_t>(my_e);
     }
   }
@@ -474,6 +470,7 @@ MK_INLINE bool route_cache(Warp &w, int layer) {
   } else {
     const uint64_t t0 = now_ns();
     while (*reinterpret_cast<volatile int *>(&rc->ready_key) != layer + 1) {
+      __nanosleep(64);  // leave the issue slots to the warp computing it
       if (now_ns() - t0 > w.P->timeout_ns) {
         report_error(*w.P, w.lane, -5, -1);
         w.failed = true;
@@ -730,7 +727,9 @@ MK_INLINE bool feed_more(Warp &w) {
   bool progress = false;
   while (!w.done_issue && !w.failed) {
     if (w.it < w.in_tiles) {  // the next tile of the current unit
-      if (!mbar_test_wait(&w.empty[w.islot], (w.ephase >> w.islot) & 1u)) break;
+      // sleep on the slot's release rather than polling it: a polling warp
+      // shares its scheduler (and instruction cache) with the consumer
+      if (!mbar_wait_hint(&w.empty[w.islot], (w.ephase >> w.islot) & 1u, 2000u)) break;
       issue_tile(w, w.itype, w.ilayer, w.it);
       w.it++;
       progress = true;
@@ -1393,14 +1392,17 @@ MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const flo
   }
   const int half = cdiv(P.d, kTileCols);
   float *wb = w.wbuf;
+  // gate rows, then up rows: one rolled loop, one copy of the stream code
   if constexpr (XS) {
     XSmem x;
     x.xs = xs;
-    if (!gemv_unit<MJ>(w, op, half, 0, P.d, x, wb)) return false;
-    if (!gemv_unit<MJ>(w, op, half, 0, P.d, x, wb + kRows * MJ)) return false;
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh)
+      if (!gemv_unit<MJ>(w, op, half, 0, P.d, x, wb + hh * kRows * MJ)) return false;
   } else {
-    if (!gemv_unit<MJ>(w, op, half, 0, P.d, xn, wb)) return false;
-    if (!gemv_unit<MJ>(w, op, half, 0, P.d, xn, wb + kRows * MJ)) return false;
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh)
+      if (!gemv_unit<MJ>(w, op, half, 0, P.d, xn, wb + hh * kRows * MJ)) return false;
   }
   const int q = w.lane / kRows, r = w.lane % kRows;
   if (w.lane < kRows * xn.n) {
@@ -1503,173 +1505,234 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
 }
 
 // --- attention ---------------------------------------------------------------
-// One warp's share of an item: online softmax over its positions for the kQvp
-// query vectors of the item's group, left in registers (lane l keeps the
-// running (max, sum) of query l % kQvp, and o for all of them over its dims).
-// DPL consecutive bf16 values of a K or V row (this lane's dimensions) in one load.
-template <int DPL>
-MK_INLINE void load_bf16_dims(const __nv_bfloat16 *p, float (&f)[DPL]) {
-  static_assert(DPL == 2 || DPL == 4, "head_dim 64 or 128");
-  if constexpr (DPL == 4) {
+// Lane layout of an attention warp: lane = 8 * pg + dl.  A tile is read in
+// groups of four consecutive positions, pg picking one of them; dl owns the
+// head dimensions [c*dl, c*dl + c) and [hd/2 + c*dl, hd/2 + c*dl + c) with
+// c = hd / 16, which are exactly rotate-half RoPE pairs, so q's rotation stays
+// in the lane.  A score is reduced over the 8 dl lanes only; the kQvp = 4
+// query vectors of the item end up one per lane pair (query dl / 2).
+
+// c consecutive bf16 values (c = 8 or 4) from shared memory, as floats.
+template <int C>
+MK_INLINE void lds_bf16(const __nv_bfloat16 *p, float (&f)[C]) {
+  static_assert(C == 8 || C == 4, "head_dim 128 or 64");
+  if constexpr (C == 8) {
+    unpack8(ld_shared_v4(p), f);
+  } else {
     const uint2 u = *reinterpret_cast<const uint2 *>(p);
     f[0] = bf_lo(u.x);
     f[1] = bf_hi(u.x);
     f[2] = bf_lo(u.y);
     f[3] = bf_hi(u.y);
-  } else {
-    const uint32_t u = *reinterpret_cast<const uint32_t *>(p);
-    f[0] = bf_lo(u);
-    f[1] = bf_hi(u);
   }
 }
 
-template <int DPL>
-MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, float &m_run, float &l_run,
-                         float (&o)[kQvp][DPL]) {
-  const Params &P = *w.P;
-  constexpr int QVP = kQvp, PG = 32 / QVP;  // positions per butterfly group
-  constexpr int hd = 32 * DPL, half = hd / 2;
-  const int G = P.Hq / P.Hkv;
-  const int pos_b = __ldg(&P.positions[a.b]);
-  const int W3 = (P.Hq + 2 * P.Hkv) * hd;
-  const float scale = 1.0f / sqrtf(static_cast<float>(hd));
-  const int lane = w.lane, ppos = lane & 15;
-  m_run = -INFINITY;
-  l_run = 0.f;
-#pragma unroll
-  for (int v = 0; v < QVP; ++v)
-#pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) o[v][dd] = 0.f;
-  if (a.ntiles == 0) return true;
-  // query vectors of this item: qv = qs*QVP + v  ->  (t = qv / G, head = g*G + qv % G)
-  float q[QVP][DPL];
-  int lim[QVP];
-#pragma unroll
-  for (int v = 0; v < QVP; ++v) {
-    const int qv = a.qs * QVP + v;
-    lim[v] = -1;
-#pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) q[v][dd] = 0.f;
-    if (qv < G * P.T) {
-      const int t = qv / G, head = a.g * G + qv % G, m = a.b * P.T + t, p = pos_b + t;
-      lim[v] = p;
-      const size_t src = static_cast<size_t>(m) * W3 + head * hd + lane * DPL;
-#pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) {
-        const float own = qkv_load(P, src + dd);
-        const float other = __shfl_xor_sync(0xffffffffu, own, 16);
-        const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
-        const float rr = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
-        q[v][dd] = rr * scale;
-      }
-    }
-  }
-  const int my_qv = lane % QVP;
-  int my_lim = -1;
-#pragma unroll
-  for (int v = 0; v < QVP; ++v)
-    if (v == my_qv) my_lim = lim[v];
-  const size_t cache_row_base =
-      (static_cast<size_t>(layer) * P.Bmax + a.b) * P.Hkv * P.cap + static_cast<size_t>(a.g) * P.cap;
-  for (int tt = 0; tt < a.ntiles; ++tt) {
-    uint8_t *slot = const_cast<uint8_t *>(consume_begin(w, op));
-    if (!slot) return false;
-    const int pos0 = a.pos0 + tt * P.attn_ppt;
-    __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(slot);
-    __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(slot + kKvBoxBytes);
-    // New positions of this step inside the tile: rotate k, round k and v to
-    // bf16, patch the tile and (once per group) append them to the cache.
-    const int lo = max(pos0, pos_b), hi = min(pos0 + P.attn_ppt, pos_b + P.T);
-    for (int p = lo; p < hi; ++p) {
-      const int t = p - pos_b, m = a.b * P.T + t;
-      const size_t kq = static_cast<size_t>(m) * W3 + (P.Hq + a.g) * hd + lane * DPL;
-      const size_t vq = static_cast<size_t>(m) * W3 + (P.Hq + P.Hkv + a.g) * hd + lane * DPL;
-#pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) {
-        const float own = qkv_load(P, kq + dd);
-        const float other = __shfl_xor_sync(0xffffffffu, own, 16);
-        const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * half + ppos * DPL + dd]);
-        const float kr = (lane < 16) ? own * cs.x - other * cs.y : own * cs.x + other * cs.y;
-        const __nv_bfloat16 kb = __float2bfloat16_rn(kr);
-        const __nv_bfloat16 vb = __float2bfloat16_rn(qkv_load(P, vq + dd));
-        ks[(p - pos0) * hd + lane * DPL + dd] = kb;
-        vs[(p - pos0) * hd + lane * DPL + dd] = vb;
-        if (a.qs == 0) {
-          P.kc[(cache_row_base + p) * hd + lane * DPL + dd] = kb;
-          P.vc[(cache_row_base + p) * hd + lane * DPL + dd] = vb;
-        }
-      }
-    }
-    if (lo < hi) fence_proxy_async_smem();
-    __syncwarp();
-    for (int jg = 0; jg < P.attn_ppt; jg += PG) {
-      float part[32];
-#pragma unroll
-      for (int j = 0; j < PG; ++j) {
-        float kf[DPL];
-        load_bf16_dims<DPL>(ks + (jg + j) * hd + lane * DPL, kf);
-#pragma unroll
-        for (int v = 0; v < QVP; ++v) {
-          float sc = 0.f;
-#pragma unroll
-          for (int dd = 0; dd < DPL; ++dd) sc = fmaf(q[v][dd], kf[dd], sc);
-          part[j * QVP + v] = sc;
-        }
-      }
-      butterfly<32>(part, lane);
-      // lane holds the score of position jg + lane / QVP for query lane % QVP
-      const int pos = pos0 + jg + lane / QVP;
-      const bool valid = (pos <= my_lim) && (pos < a.pos0 + a.npos);
-      const float sc = valid ? part[0] : -INFINITY;
-      float mx = sc;
-#pragma unroll
-      for (int o2 = QVP; o2 < 32; o2 <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
-      const float m_new = fmaxf(m_run, mx);
-      const float pr = valid ? expf(sc - m_new) : 0.f;
-      const float alpha = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
-      float ps = pr;
-#pragma unroll
-      for (int o2 = QVP; o2 < 32; o2 <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o2);
-      l_run = l_run * alpha + ps;
-      m_run = m_new;
-#pragma unroll
-      for (int v = 0; v < QVP; ++v) {
-        const float av = __shfl_sync(0xffffffffu, alpha, v);
-#pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) o[v][dd] *= av;
-      }
-      // every lane needs all 32 probabilities: one store each, then 8 float4
-      // broadcast loads from the warp's scratch (lane 4j + v holds position j, query v)
-      __syncwarp();
-      w.wbuf[lane] = pr;
-      __syncwarp();
-#pragma unroll
-      for (int j = 0; j < PG; ++j) {
-        float vf[DPL];
-        load_bf16_dims<DPL>(vs + (jg + j) * hd + lane * DPL, vf);
-        const float4 p4 = *reinterpret_cast<const float4 *>(w.wbuf + j * QVP);
-        const float pj[4] = {p4.x, p4.y, p4.z, p4.w};
-#pragma unroll
-        for (int v = 0; v < QVP; ++v)
-#pragma unroll
-          for (int dd = 0; dd < DPL; ++dd) o[v][dd] = fmaf(pj[v], vf[dd], o[v][dd]);
-      }
-    }
-    consume_end(w);
-  }
-  return true;
+// Four partial scores (one per query) summed over the 8 dl lanes of a
+// position: the lane keeps query dl / 2's full score.
+MK_INLINE float reduce_scores8(const float (&p)[kQvp], int dl) {
+  const bool up4 = (dl & 4) != 0, up2 = (dl & 2) != 0;
+  float k0 = up4 ? p[2] : p[0], k1 = up4 ? p[3] : p[1];
+  const float s0 = up4 ? p[0] : p[2], s1 = up4 ? p[1] : p[3];
+  k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
+  k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
+  float k = up2 ? k1 : k0;
+  k += __shfl_xor_sync(0xffffffffu, up2 ? k0 : k1, 2);
+  k += __shfl_xor_sync(0xffffffffu, k, 1);
+  return k;
 }
-
-MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op);
 
 // Shared-memory scratch of the attention items of one CTA.
 struct AttnShared {
   float *o;           // [compute warps][kQvp][hd] partials (the staging row's space)
+  float *q;           // [kQvp][hd] the item's query vectors, rotated and scaled
   float *ml;          // [compute warps][kQvp][2]
   int *last;          // this CTA completed its group
   uint32_t *rdv;      // rendezvous counter
   uint32_t *seq;      // this warp's rendezvous count
 };
+
+// One warp's share of an item: online softmax over its positions for the
+// item's kQvp query vectors; the unnormalised o, the running max and the sum
+// go to the CTA's scratch at warp slot wib.  The item's code runs once per
+// layer, so its loops are kept rolled: fewer distinct instructions to fetch.
+template <int HD>
+MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShared &sh) {
+  const Params &P = *w.P;
+  constexpr int C = HD / 16, DL = 2 * C, HALF = HD / 2, QVP = kQvp;
+  constexpr int NS = kKvBoxBytes / (2 * HD) / 4;  // groups of four positions per tile
+  static_assert(QVP == 4, "one query vector per lane pair");
+  const int G = P.Hq / P.Hkv;
+  const int pos_b = __ldg(&P.positions[a.b]);
+  const int W3 = (P.Hq + 2 * P.Hkv) * HD;
+  const int lane = w.lane, pg = lane >> 3, dl = lane & 7, myq = dl >> 1;
+  const int d0 = C * dl, d1 = HALF + C * dl;
+  float m_run = -INFINITY, l_run = 0.f;
+  float o[QVP][DL];
+#pragma unroll
+  for (int v = 0; v < QVP; ++v)
+#pragma unroll
+    for (int k = 0; k < DL; ++k) o[v][k] = 0.f;
+  if (a.ntiles > 0) {
+    // the item's query vectors, staged by the CTA: this lane's dimensions
+    float q[QVP][DL];
+#pragma unroll
+    for (int v = 0; v < QVP; ++v) {
+#pragma unroll
+      for (int k = 0; k < C; k += 4) {
+        const float4 x1 = *reinterpret_cast<const float4 *>(sh.q + v * HD + d0 + k);
+        const float4 x2 = *reinterpret_cast<const float4 *>(sh.q + v * HD + d1 + k);
+        q[v][k] = x1.x; q[v][k + 1] = x1.y; q[v][k + 2] = x1.z; q[v][k + 3] = x1.w;
+        q[v][C + k] = x2.x; q[v][C + k + 1] = x2.y; q[v][C + k + 2] = x2.z; q[v][C + k + 3] = x2.w;
+      }
+    }
+    // last position query myq may see (-1: no such query vector)
+    const int my_qv = a.qs * QVP + myq;
+    const int lim = my_qv < G * P.T ? pos_b + my_qv / G : -1;
+    const int end = a.pos0 + a.npos;
+    const size_t cache_row_base =
+        (static_cast<size_t>(layer) * P.Bmax + a.b) * P.Hkv * P.cap + static_cast<size_t>(a.g) * P.cap;
+    for (int tt = 0; tt < a.ntiles; ++tt) {
+      uint8_t *slot = const_cast<uint8_t *>(consume_begin(w, op));
+      if (!slot) return false;
+      const int pos0 = a.pos0 + tt * P.attn_ppt;
+      __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(slot);
+      __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(slot + kKvBoxBytes);
+      // New positions of this step inside the tile: rotate k, round k and v to
+      // bf16, patch the tile and (once per group) append them to the cache.
+      const int lo = max(pos0, pos_b), hi = min(pos0 + P.attn_ppt, pos_b + P.T);
+      for (int p = lo; p < hi; ++p) {
+        const int t = p - pos_b, m = a.b * P.T + t;
+        const size_t kq = static_cast<size_t>(m) * W3 + (P.Hq + a.g) * HD;
+        const size_t vq = static_cast<size_t>(m) * W3 + (P.Hq + P.Hkv + a.g) * HD;
+        for (int i = lane; i < HALF; i += 32) {
+          const float x1 = qkv_load(P, kq + i), x2 = qkv_load(P, kq + i + HALF);
+          const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * HALF + i]);
+          const __nv_bfloat16 k1 = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
+          const __nv_bfloat16 k2 = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
+          const __nv_bfloat16 v1 = __float2bfloat16_rn(qkv_load(P, vq + i));
+          const __nv_bfloat16 v2 = __float2bfloat16_rn(qkv_load(P, vq + i + HALF));
+          const int r = (p - pos0) * HD;
+          ks[r + i] = k1;
+          ks[r + i + HALF] = k2;
+          vs[r + i] = v1;
+          vs[r + i + HALF] = v2;
+          if (a.qs == 0) {
+            const size_t c = (cache_row_base + p) * HD;
+            P.kc[c + i] = k1;
+            P.kc[c + i + HALF] = k2;
+            P.vc[c + i] = v1;
+            P.vc[c + i + HALF] = v2;
+          }
+        }
+      }
+      if (lo < hi) fence_proxy_async_smem();
+      __syncwarp();
+      // scores, two groups of four positions per iteration: lane (pg, dl)
+      // gets position pos0 + 4s + pg for query myq; results enter sc at the end
+      float sc[NS];
+#pragma unroll 1
+      for (int s = 0; s < NS; s += 2) {
+        float x[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const __nv_bfloat16 *kr = ks + (4 * (s + h) + pg) * HD;
+          float k1[C], k2[C];
+          lds_bf16<C>(kr + d0, k1);
+          lds_bf16<C>(kr + d1, k2);
+          float part[QVP];
+#pragma unroll
+          for (int v = 0; v < QVP; ++v) {
+            float a1 = 0.f, a2 = 0.f;
+#pragma unroll
+            for (int k = 0; k < C; ++k) {
+              a1 = fmaf(q[v][k], k1[k], a1);
+              a2 = fmaf(q[v][C + k], k2[k], a2);
+            }
+            part[v] = a1 + a2;
+          }
+          x[h] = reduce_scores8(part, dl);
+        }
+#pragma unroll
+        for (int r = 0; r + 2 < NS; ++r) sc[r] = sc[r + 2];
+        sc[NS - 2] = x[0];
+        sc[NS - 1] = x[1];
+      }
+      // online softmax over the tile (per query: the 4 pg lanes x NS groups)
+      float mt = -INFINITY;
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const int pos = pos0 + 4 * s + pg;
+        if (!(pos <= lim && pos < end)) sc[s] = -INFINITY;
+        mt = fmaxf(mt, sc[s]);
+      }
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+      const float m_new = fmaxf(m_run, mt);
+      const float alpha = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
+      float ps = 0.f;
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        sc[s] = (sc[s] == -INFINITY) ? 0.f : expf(sc[s] - m_new);
+        ps += sc[s];
+      }
+      ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+      l_run = l_run * alpha + ps;
+      m_run = m_new;
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int v = 0; v < QVP; ++v) {
+          const float av = __shfl_sync(0xffffffffu, alpha, 2 * v);
+#pragma unroll
+          for (int k = 0; k < DL; ++k) o[v][k] *= av;
+        }
+      }
+      // o[v] += p(position, v) * V[position]; the probabilities leave sc from
+      // the front, two groups per iteration
+#pragma unroll 1
+      for (int s = 0; s < NS; s += 2) {
+        const float pj[2] = {sc[0], sc[1]};
+#pragma unroll
+        for (int r = 0; r + 2 < NS; ++r) sc[r] = sc[r + 2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const __nv_bfloat16 *vr = vs + (4 * (s + h) + pg) * HD;
+          float v1[C], v2[C];
+          lds_bf16<C>(vr + d0, v1);
+          lds_bf16<C>(vr + d1, v2);
+#pragma unroll
+          for (int v = 0; v < QVP; ++v) {
+            const float pv = __shfl_sync(0xffffffffu, pj[h], pg * 8 + 2 * v);
+#pragma unroll
+            for (int k = 0; k < C; ++k) {
+              o[v][k] = fmaf(pv, v1[k], o[v][k]);
+              o[v][C + k] = fmaf(pv, v2[k], o[v][C + k]);
+            }
+          }
+        }
+      }
+      consume_end(w);
+    }
+  }
+  // sum o over the four pg lanes, leaving lane (pg, dl) with query pg
+  const bool u16 = (lane & 16) != 0, u8 = (lane & 8) != 0;
+  float *so = sh.o + (w.wib * QVP + pg) * HD;
+#pragma unroll
+  for (int k = 0; k < DL; ++k) {
+    const float s0 = u16 ? o[0][k] : o[2][k], s1 = u16 ? o[1][k] : o[3][k];
+    const float r0 = (u16 ? o[2][k] : o[0][k]) + __shfl_xor_sync(0xffffffffu, s0, 16);
+    const float r1 = (u16 ? o[3][k] : o[1][k]) + __shfl_xor_sync(0xffffffffu, s1, 16);
+    const float r = (u8 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, u8 ? r0 : r1, 8);
+    so[(k < C ? d0 : d1 - C) + k] = r;
+  }
+  if (pg == 0 && (dl & 1) == 0) {
+    sh.ml[(w.wib * QVP + myq) * 2] = m_run;
+    sh.ml[(w.wib * QVP + myq) * 2 + 1] = l_run;
+  }
+  return true;
+}
+
+MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op);
 
 // Final merge of one query vector over the nch CTA partials of its group:
 // o = sum_i e^(m_i - M) o_i / sum_i e^(m_i - M) l_i  (one lane per partial for
@@ -1719,16 +1782,39 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
   const Params &P = *w.P;
   constexpr int hd = 32 * DPL;
   const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, item, w.wib);
-  float m_run, l_run, o[kQvp][DPL];
-  if (!attn_warp<DPL>(w, op, layer, a, m_run, l_run, o)) return false;
+  {
+    // the item's query vectors, once per CTA: warp v rotates (rotate-half
+    // pairs (i, i + hd/2) over its lanes) and scales query vector v
+    static_assert(kConsumers == kQvp, "one query vector per compute warp");
+    constexpr int HALF = hd / 2;
+    const int v = w.wib, qv = a.qs * kQvp + v, G = P.Hq / P.Hkv;
+    float *dst = sh.q + v * hd;
+    if (qv < G * P.T) {
+      const int t = qv / G, head = a.g * G + qv % G, m = a.b * P.T + t, p = __ldg(&P.positions[a.b]) + t;
+      const size_t src = static_cast<size_t>(m) * (P.Hq + 2 * P.Hkv) * hd + head * hd;
+      const float scale = 1.0f / sqrtf(static_cast<float>(hd));
+      float x1[HALF / 32], x2[HALF / 32];
+      float2 cs[HALF / 32];
 #pragma unroll
-  for (int v = 0; v < kQvp; ++v)
+      for (int j = 0; j < HALF / 32; ++j) {
+        const int i = w.lane + 32 * j;
+        x1[j] = qkv_load(P, src + i);
+        x2[j] = qkv_load(P, src + i + HALF);
+        cs[j] = __ldg(&P.rope[static_cast<size_t>(p) * HALF + i]);
+      }
 #pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) sh.o[(w.wib * kQvp + v) * hd + w.lane * DPL + dd] = o[v][dd];
-  if (w.lane < kQvp) {
-    sh.ml[(w.wib * kQvp + w.lane) * 2] = m_run;
-    sh.ml[(w.wib * kQvp + w.lane) * 2 + 1] = l_run;
+      for (int j = 0; j < HALF / 32; ++j) {
+        const int i = w.lane + 32 * j;
+        dst[i] = (x1[j] * cs[j].x - x2[j] * cs[j].y) * scale;
+        dst[i + HALF] = (x2[j] * cs[j].x + x1[j] * cs[j].y) * scale;
+      }
+    } else {
+      for (int i = w.lane; i < hd; i += 32) dst[i] = 0.f;
+    }
+    *sh.seq += kConsumers;
+    if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   }
+  if (!attn_warp<hd>(w, op, layer, a, sh)) return false;
   *sh.seq += kConsumers;
   if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   const int grp = (a.b * P.Hkv + a.g) * P.attn_qsplit + a.qs;
@@ -2128,7 +2214,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   }
 
   uint32_t stage_seq = 0;
-  AttnShared ash{xs, s_attn_ml, &s_attn_last, &s_stage, &stage_seq};
+  AttnShared ash{xs, xs + kConsumers * kQvp * P.hd, s_attn_ml, &s_attn_last, &s_stage, &stage_seq};
   float am_val = -INFINITY;
   int am_idx = 0x7fffffff;
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {
