@@ -157,6 +157,12 @@ MK_INLINE uint4 ld_shared_v4(const void *p) {
 MK_INLINE float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 MK_INLINE float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
+// A bf16 pair (low half = even element) as floats.
+MK_INLINE float2 bf2(uint32_t u) { return make_float2(bf_lo(u), bf_hi(u)); }
+// Two fp32 FMAs / products in one instruction, each rounded as its scalar form.
+MK_INLINE float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+MK_INLINE float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
 MK_INLINE void unpack8(const uint4 &w, float (&f)[8]) {
   f[0] = bf_lo(w.x); f[1] = bf_hi(w.x); f[2] = bf_lo(w.y); f[3] = bf_hi(w.y);
   f[4] = bf_lo(w.z); f[5] = bf_hi(w.z); f[6] = bf_lo(w.w); f[7] = bf_hi(w.w);
@@ -987,20 +993,23 @@ MK_INLINE void gemv_panel(const uint8_t *pan, float (&acc)[kRows * MJ], float (&
                           const float (&x)[MJ][8]) {
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
-    float wf[8];
-    unpack8(ld_shared_v4(pan + r * (kPanel * 2)), wf);
+    if constexpr (MJ <= 2) {
+      // each (even, odd) column pair in one packed FMA
+      const uint4 u = ld_shared_v4(pan + r * (kPanel * 2));
+      const float2 wp[4] = {bf2(u.x), bf2(u.y), bf2(u.z), bf2(u.w)};
 #pragma unroll
-    for (int j = 0; j < MJ; ++j) {
-      if constexpr (MJ <= 2) {
-        float a = acc[r * MJ + j], b = acc2[r * MJ + j];
+      for (int j = 0; j < MJ; ++j) {
+        float2 ab = make_float2(acc[r * MJ + j], acc2[r * MJ + j]);
 #pragma unroll
-        for (int k = 0; k < 8; k += 2) {
-          a = fmaf(wf[k], x[j][k], a);
-          b = fmaf(wf[k + 1], x[j][k + 1], b);
-        }
-        acc[r * MJ + j] = a;
-        acc2[r * MJ + j] = b;
-      } else {
+        for (int k = 0; k < 4; ++k) ab = fma2(wp[k], make_float2(x[j][2 * k], x[j][2 * k + 1]), ab);
+        acc[r * MJ + j] = ab.x;
+        acc2[r * MJ + j] = ab.y;
+      }
+    } else {
+      float wf[8];
+      unpack8(ld_shared_v4(pan + r * (kPanel * 2)), wf);
+#pragma unroll
+      for (int j = 0; j < MJ; ++j) {
         float a = acc[r * MJ + j];
 #pragma unroll
         for (int k = 0; k < 8; ++k) a = fmaf(wf[k], x[j][k], a);
@@ -1512,18 +1521,21 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
 // in the lane.  A score is reduced over the 8 dl lanes only; the kQvp = 4
 // query vectors of the item end up one per lane pair (query dl / 2).
 
-// c consecutive bf16 values (c = 8 or 4) from shared memory, as floats.
+// c consecutive bf16 values (c = 8 or 4) from shared memory, as c / 2
+// (even, odd) float pairs.
 template <int C>
-MK_INLINE void lds_bf16(const __nv_bfloat16 *p, float (&f)[C]) {
+MK_INLINE void lds_bf16x2(const __nv_bfloat16 *p, float2 (&f)[C / 2]) {
   static_assert(C == 8 || C == 4, "head_dim 128 or 64");
   if constexpr (C == 8) {
-    unpack8(ld_shared_v4(p), f);
+    const uint4 u = ld_shared_v4(p);
+    f[0] = bf2(u.x);
+    f[1] = bf2(u.y);
+    f[2] = bf2(u.z);
+    f[3] = bf2(u.w);
   } else {
     const uint2 u = *reinterpret_cast<const uint2 *>(p);
-    f[0] = bf_lo(u.x);
-    f[1] = bf_hi(u.x);
-    f[2] = bf_lo(u.y);
-    f[3] = bf_hi(u.y);
+    f[0] = bf2(u.x);
+    f[1] = bf2(u.y);
   }
 }
 
@@ -1567,22 +1579,25 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
   const int lane = w.lane, pg = lane >> 3, dl = lane & 7, myq = dl >> 1;
   const int d0 = C * dl, d1 = HALF + C * dl;
   float m_run = -INFINITY, l_run = 0.f;
-  float o[QVP][DL];
+  constexpr int DP = DL / 2, CP = C / 2;  // float pairs per lane and per chunk
+  float2 o[QVP][DP];
 #pragma unroll
   for (int v = 0; v < QVP; ++v)
 #pragma unroll
-    for (int k = 0; k < DL; ++k) o[v][k] = 0.f;
+    for (int k = 0; k < DP; ++k) o[v][k] = make_float2(0.f, 0.f);
   if (a.ntiles > 0) {
     // the item's query vectors, staged by the CTA: this lane's dimensions
-    float q[QVP][DL];
+    float2 q[QVP][DP];
 #pragma unroll
     for (int v = 0; v < QVP; ++v) {
 #pragma unroll
-      for (int k = 0; k < C; k += 4) {
-        const float4 x1 = *reinterpret_cast<const float4 *>(sh.q + v * HD + d0 + k);
-        const float4 x2 = *reinterpret_cast<const float4 *>(sh.q + v * HD + d1 + k);
-        q[v][k] = x1.x; q[v][k + 1] = x1.y; q[v][k + 2] = x1.z; q[v][k + 3] = x1.w;
-        q[v][C + k] = x2.x; q[v][C + k + 1] = x2.y; q[v][C + k + 2] = x2.z; q[v][C + k + 3] = x2.w;
+      for (int k = 0; k < CP; k += 2) {
+        const float4 x1 = *reinterpret_cast<const float4 *>(sh.q + v * HD + d0 + 2 * k);
+        const float4 x2 = *reinterpret_cast<const float4 *>(sh.q + v * HD + d1 + 2 * k);
+        q[v][k] = make_float2(x1.x, x1.y);
+        q[v][k + 1] = make_float2(x1.z, x1.w);
+        q[v][CP + k] = make_float2(x2.x, x2.y);
+        q[v][CP + k + 1] = make_float2(x2.z, x2.w);
       }
     }
     // last position query myq may see (-1: no such query vector)
@@ -1636,19 +1651,18 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const __nv_bfloat16 *kr = ks + (4 * (s + h) + pg) * HD;
-          float k1[C], k2[C];
-          lds_bf16<C>(kr + d0, k1);
-          lds_bf16<C>(kr + d1, k2);
+          float2 k1[CP], k2[CP];
+          lds_bf16x2<C>(kr + d0, k1);
+          lds_bf16x2<C>(kr + d1, k2);
           float part[QVP];
 #pragma unroll
           for (int v = 0; v < QVP; ++v) {
-            float a1 = 0.f, a2 = 0.f;
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < C; ++k) {
-              a1 = fmaf(q[v][k], k1[k], a1);
-              a2 = fmaf(q[v][C + k], k2[k], a2);
-            }
-            part[v] = a1 + a2;
+            for (int k = 0; k < CP; ++k) acc = fma2(q[v][k], k1[k], acc);
+#pragma unroll
+            for (int k = 0; k < CP; ++k) acc = fma2(q[v][CP + k], k2[k], acc);
+            part[v] = acc.x + acc.y;
           }
           x[h] = reduce_scores8(part, dl);
         }
@@ -1684,7 +1698,7 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
         for (int v = 0; v < QVP; ++v) {
           const float av = __shfl_sync(0xffffffffu, alpha, 2 * v);
 #pragma unroll
-          for (int k = 0; k < DL; ++k) o[v][k] *= av;
+          for (int k = 0; k < DP; ++k) o[v][k] = mul2(o[v][k], make_float2(av, av));
         }
       }
       // o[v] += p(position, v) * V[position]; the probabilities leave sc from
@@ -1697,16 +1711,17 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const __nv_bfloat16 *vr = vs + (4 * (s + h) + pg) * HD;
-          float v1[C], v2[C];
-          lds_bf16<C>(vr + d0, v1);
-          lds_bf16<C>(vr + d1, v2);
+          float2 v1[CP], v2[CP];
+          lds_bf16x2<C>(vr + d0, v1);
+          lds_bf16x2<C>(vr + d1, v2);
 #pragma unroll
           for (int v = 0; v < QVP; ++v) {
             const float pv = __shfl_sync(0xffffffffu, pj[h], pg * 8 + 2 * v);
+            const float2 pp = make_float2(pv, pv);
 #pragma unroll
-            for (int k = 0; k < C; ++k) {
-              o[v][k] = fmaf(pv, v1[k], o[v][k]);
-              o[v][C + k] = fmaf(pv, v2[k], o[v][C + k]);
+            for (int k = 0; k < CP; ++k) {
+              o[v][k] = fma2(pp, v1[k], o[v][k]);
+              o[v][CP + k] = fma2(pp, v2[k], o[v][CP + k]);
             }
           }
         }
@@ -1719,9 +1734,13 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
   float *so = sh.o + (w.wib * QVP + pg) * HD;
 #pragma unroll
   for (int k = 0; k < DL; ++k) {
-    const float s0 = u16 ? o[0][k] : o[2][k], s1 = u16 ? o[1][k] : o[3][k];
-    const float r0 = (u16 ? o[2][k] : o[0][k]) + __shfl_xor_sync(0xffffffffu, s0, 16);
-    const float r1 = (u16 ? o[3][k] : o[1][k]) + __shfl_xor_sync(0xffffffffu, s1, 16);
+    const int kp = k >> 1;
+    const bool hi = k & 1;
+#define MK_OV(v) (hi ? o[v][kp].y : o[v][kp].x)
+    const float s0 = u16 ? MK_OV(0) : MK_OV(2), s1 = u16 ? MK_OV(1) : MK_OV(3);
+    const float r0 = (u16 ? MK_OV(2) : MK_OV(0)) + __shfl_xor_sync(0xffffffffu, s0, 16);
+    const float r1 = (u16 ? MK_OV(3) : MK_OV(1)) + __shfl_xor_sync(0xffffffffu, s1, 16);
+#undef MK_OV
     const float r = (u8 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, u8 ? r0 : r1, 8);
     so[(k < C ? d0 : d1 - C) + k] = r;
   }
