@@ -1203,15 +1203,39 @@ MK_INLINE void residual_rows(const Params &P, int lane, int unit, int row0, int 
   __syncwarp();
 }
 
+// New residual rows of whole units, several units per pass when the rows
+// leave lanes free: lane = 4 * (g * M + m) + r takes row r of activation row
+// m of the pass's g-th unit, so that all of a pass's loads are in flight
+// together.  Units are this warp's: slot, slot + nw, ...
+template <class F>
+MK_INLINE void residual_units(const Params &P, int lane, int slot, int nw, int dbg_layer, F val) {
+  const int lanes_per_unit = kRows * P.M, per = 32 / lanes_per_unit;
+  const int g = lane / lanes_per_unit, m = (lane / kRows) % P.M, r = lane % kRows;
+  for (int base = slot; base < P.n_hb; base += per * nw) {
+    const int unit = base + g * nw, row = unit * kRows + r;
+    const bool live = g < per && unit < P.n_hb;
+    float sq = 0.f;
+    if (live && row < P.d) {
+      const float hn = val(m, row);
+      __stcg(P.h + static_cast<size_t>(m) * P.d + row, hn);
+      sq = hn * hn;
+      if (dbg_layer >= 0 && P.dbg_hidden)
+        P.dbg_hidden[(static_cast<size_t>(dbg_layer) * P.max_rows + m) * P.d + row] = hn;
+    }
+    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+    if (live && r == 0) __stcg(&P.ss[m * P.ss_ld + unit], sq);
+  }
+  __syncwarp();
+}
+
 MK_INLINE void op_embed(Warp &w) {
   const Params &P = *w.P;
-  for (int unit = w.slot; unit < P.n_hb; unit += w.nw) {
-    residual_rows(P, w.lane, unit, unit * kRows, 0, [&](int m, int row, int) {
-      int tok = __ldcg(&P.tokens[m]);       // may alias the argmax output
-      if (tok < 0 || tok >= P.V) tok = 0;  // rejected at kernel start
-      return __bfloat162float(P.embed[static_cast<size_t>(tok) * P.d + row]);
-    });
-  }
+  residual_units(P, w.lane, w.slot, w.nw, 0, [&](int m, int row) {
+    int tok = __ldcg(&P.tokens[m]);       // may alias the argmax output
+    if (tok < 0 || tok >= P.V) tok = 0;  // rejected at kernel start
+    return __bfloat162float(P.embed[static_cast<size_t>(tok) * P.d + row]);
+  });
 }
 
 // h += (sum_s w_s y_s) + shared, in the selection order of each row.
@@ -1219,17 +1243,15 @@ MK_INLINE void op_combine(Warp &w, int layer) {
   const Params &P = *w.P;
   const int S = P.topk + 1;
   const RouteCache *rt = w.rc;
-  for (int unit = w.slot; unit < P.n_hb; unit += w.nw) {
-    residual_rows(P, w.lane, unit, unit * kRows, layer + 1, [&](int m, int row, int) {
-      const float *yp = P.y_part + (static_cast<size_t>(m) * S) * P.d + row;
-      float moe = 0.f;
+  residual_units(P, w.lane, w.slot, w.nw, layer + 1, [&](int m, int row) {
+    const float *yp = P.y_part + (static_cast<size_t>(m) * S) * P.d + row;
+    float moe = 0.f;
 #pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s)
-        if (s < P.topk) moe += rt->row_w[m][s] * __ldcg(yp + static_cast<size_t>(s) * P.d);
-      const float sh = P.Fs > 0 ? __ldcg(yp + static_cast<size_t>(P.topk) * P.d) : 0.f;
-      return __ldcg(P.h + static_cast<size_t>(m) * P.d + row) + (moe + sh);
-    });
-  }
+    for (int s = 0; s < kMaxTopK; ++s)
+      if (s < P.topk) moe += rt->row_w[m][s] * __ldcg(yp + static_cast<size_t>(s) * P.d);
+    const float sh = P.Fs > 0 ? __ldcg(yp + static_cast<size_t>(P.topk) * P.d) : 0.f;
+    return __ldcg(P.h + static_cast<size_t>(m) * P.d + row) + (moe + sh);
+  });
 }
 
 template <int MJ>
@@ -1758,29 +1780,35 @@ MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op);
 // (m, l); the o partials are read 8 at a time, all in flight together).
 template <int DPL>
 MK_INLINE void attn_final_merge(const Params &P, int lane, int grp, int v, int nch, int b, int g) {
-  constexpr int hd = 32 * DPL;
+  constexpr int hd = 32 * DPL, B = 16;  // partials loaded per batch, all in flight with (m, l)
   const int G = P.Hq / P.Hkv;
   const int qv = (grp % P.attn_qsplit) * kQvp + v;
   if (qv >= G * P.T) return;
   const float *mrow = P.attn_ml + (static_cast<size_t>(grp) * kQvp + v) * 2 * P.attn_nch_max;
+  const float *obase = P.attn_o + (static_cast<size_t>(grp) * P.attn_nch_max * kQvp + v) * hd + lane * DPL;
+  const size_t ostride = static_cast<size_t>(kQvp) * hd;  // one CTA partial to the next
   const float mi = lane < nch ? __ldcg(mrow + lane) : -INFINITY;
   const float li = lane < nch ? __ldcg(mrow + P.attn_nch_max + lane) : 0.f;
+  float val[B][DPL];
+#pragma unroll
+  for (int k = 0; k < B; ++k)
+#pragma unroll
+    for (int dd = 0; dd < DPL; ++dd) val[k][dd] = (k < nch) ? __ldcg(obase + k * ostride + dd) : 0.f;
   const float M = warp_max(mi);
   const float wi = (lane < nch && mi != -INFINITY) ? expf(mi - M) : 0.f;
   const float L = warp_sum(wi * li);
   float acc[DPL];
 #pragma unroll
   for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
-  for (int i0 = 0; i0 < nch; i0 += 8) {
-    float val[8][DPL];
+  for (int i0 = 0; i0 < nch; i0 += B) {
+    if (i0 > 0) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float *op = P.attn_o + ((static_cast<size_t>(grp) * P.attn_nch_max + i0 + k) * kQvp + v) * hd + lane * DPL;
+      for (int k = 0; k < B; ++k)
 #pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) val[k][dd] = (i0 + k < nch) ? __ldcg(op + dd) : 0.f;
+        for (int dd = 0; dd < DPL; ++dd) val[k][dd] = (i0 + k < nch) ? __ldcg(obase + (i0 + k) * ostride + dd) : 0.f;
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < B; ++k) {
       const float wv = __shfl_sync(0xffffffffu, wi, (i0 + k) & 31);
 #pragma unroll
       for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(wv, val[k][dd], acc[dd]);
