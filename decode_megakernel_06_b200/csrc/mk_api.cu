@@ -127,8 +127,9 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.n_ops = n_ops_for(d.n_layers);
   // shared-memory row: the staged activations (batch 1) or the attention
   // warps' partials and the item's query vectors, whichever is larger
+  // (whole 256-column panels: the staged layout permutes columns within one)
   p.xs_floats = std::max((kConsumers + 1) * kQvp * d.head_dim,
-                         kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), 4) * 4 : 0);
+                         kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), kPanel) * kPanel : 0);
   // Batch 1 down projection: a CTA's contiguous range of units spans at most
   // 1 + ceil(range / row blocks) experts; their activations must fit the
   // shared-memory row.
@@ -139,7 +140,7 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
     const int per_cta = ceil_div(segs * n_db, p.n_cta);
     const int span = 1 + ceil_div(per_cta, n_db);
     const int fmax = std::max(d.expert_ffn, d.shared_ffn);
-    p.down_staged = (std::min(span, segs) * ceil_div(fmax, 4) * 4 <= p.xs_floats) ? 1 : 0;
+    p.down_staged = (std::min(span, segs) * ceil_div(fmax, kPanel) * kPanel <= p.xs_floats) ? 1 : 0;
   }
   // with one or two rows per step the two groups of an 8-row down unit can
   // keep separate accumulators, so its tiles go column by column

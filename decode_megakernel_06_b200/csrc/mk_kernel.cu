@@ -969,14 +969,21 @@ struct XPlain {  // x = src[row][col]
   }
 };
 
-// One activation row staged in shared memory by the CTA (batch 1): x = xs[col].
+// One activation row staged in shared memory by the CTA (batch 1).  Within
+// each 256-column panel, columns 8g..8g+3 sit at 4g and columns 8g+4..8g+7 at
+// 128 + 4g, so that the 32 lanes' float4 reads (lane g takes columns 8g..8g+7
+// of a panel) are 16 bytes apart and free of bank conflicts.
+MK_INLINE int xs_pos4(int c4) {  // float4 slot of columns 4*c4 .. 4*c4+3
+  return (c4 & ~63) | ((c4 & 1) << 5) | ((c4 & 63) >> 1);
+}
 struct XSmem {
   const float *xs;
   MK_INLINE void prefetch(int, int) const {}
   MK_INLINE void load(int col, int K, float (&x)[1][8]) const {
     if (col < K) {
-      const float4 a = *reinterpret_cast<const float4 *>(xs + col);
-      const float4 b = *reinterpret_cast<const float4 *>(xs + col + 4);
+      const float *pb = xs + (col & ~(kPanel - 1)) + ((col & (kPanel - 1)) >> 1);
+      const float4 a = *reinterpret_cast<const float4 *>(pb);
+      const float4 b = *reinterpret_cast<const float4 *>(pb + kPanel / 2);
       x[0][0] = a.x; x[0][1] = a.y; x[0][2] = a.z; x[0][3] = a.w;
       x[0][4] = b.x; x[0][5] = b.y; x[0][6] = b.z; x[0][7] = b.w;
     } else {
@@ -1341,13 +1348,16 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
     }
     default: ntiles = cdiv(P.d, kTileCols); N = P.V; break;
   }
+  // lane 4m + r owns output (row0 + r, m); normed ops scale by inv_rms here
+  const int m = w.lane / kRows, r = w.lane % kRows;
+  const bool live = w.lane < kRows * P.M && row0 + r < N;
+  // the o-projection's residual input, loaded before the stream so that its
+  // latency hides behind the tiles
+  const float h_old = (type == OP_OPROJ && live) ? __ldcg(P.h + static_cast<size_t>(m) * P.d + row0 + r) : 0.f;
   const bool ok = with_dense_x<MJ, XS>(w, type, layer, xs, [&](const auto &x) {
     return gemv_unit<MJ>(w, op, ntiles, col0, K, x, wb);
   });
   if (!ok) return false;
-  // lane 4m + r owns output (row0 + r, m); normed ops scale by inv_rms here
-  const int m = w.lane / kRows, r = w.lane % kRows;
-  const bool live = w.lane < kRows * P.M && row0 + r < N;
   float im = 1.f;
 #pragma unroll
   for (int mm = 0; mm < kMaxRows; ++mm)
@@ -1386,9 +1396,7 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
       break;
     }
     case OP_OPROJ:
-      residual_rows(P, w.lane, unit, row0, -1, [&](int mm, int row, int rr) {
-        return __ldca(P.h + static_cast<size_t>(mm) * P.d + row) + wb[rr * MJ + mm];
-      });
+      residual_rows(P, w.lane, unit, row0, -1, [&](int mm, int, int rr) { return h_old + wb[rr * MJ + mm]; });
       break;
     default: break;
   }
@@ -1478,7 +1486,7 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm)
     if (P.down_staged) {
       // the CTA staged its experts' activations: slot seg - dseg0 of the row
       XSmem xst;
-      xst.xs = xsm + (seg - w.dseg0) * (cdiv(max(P.F, P.Fs), 4) * 4);
+      xst.xs = xsm + (seg - w.dseg0) * (cdiv(max(P.F, P.Fs), kPanel) * kPanel);
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xst, wb);
     } else {
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xs, wb);
@@ -2023,7 +2031,7 @@ MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, float *ssp, uint
       v.z *= bf_lo(gb.y);
       v.w *= bf_hi(gb.y);
     }
-    reinterpret_cast<float4 *>(xs)[c4] = v;
+    reinterpret_cast<float4 *>(xs)[xs_pos4(c4)] = v;
   }
   if (g) {
     sq = warp_sum(sq);
@@ -2043,7 +2051,8 @@ MK_INLINE float staged_inv_rms(const Params &P, const float *ssp) {
 
 // Batch 1 down projection: the CTA copies the activations of the experts its
 // unit range covers (routed rows first, then the shared expert) into the
-// shared-memory row, one max(F, Fs) slot per expert from the range's first.
+// shared-memory row, one slot of max(F, Fs) rounded up to whole panels per
+// expert from the range's first, each in the panel layout of XSmem.
 MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t &seq, int op) {
   const Params &P = *w.P;
   if (!route_cache(w, layer)) return false;
@@ -2052,13 +2061,13 @@ MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t
   down_cta_range(P, w.cta, total, c0, c1);
   w.dseg0 = c0 / P.n_db;
   if (c1 > c0) {
-    const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, ld = cdiv(max(P.F, P.Fs), 4) * 4;
+    const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, ld = cdiv(max(P.F, P.Fs), kPanel) * kPanel;
     for (int sg = seg0; sg <= seg1; ++sg) {
       const float4 *src = reinterpret_cast<const float4 *>(
           sg < U ? P.act_routed + static_cast<size_t>(sg) * kMaxRows * P.F : P.act_shared);
       const int K = sg < U ? P.F : P.Fs;
       float4 *dst = reinterpret_cast<float4 *>(xs + (sg - seg0) * ld);
-      for (int c4 = threadIdx.x; c4 < K / 4; c4 += kConsumerThreads) dst[c4] = __ldcg(src + c4);
+      for (int c4 = threadIdx.x; c4 < K / 4; c4 += kConsumerThreads) dst[xs_pos4(c4)] = __ldcg(src + c4);
     }
   }
   seq += kConsumers;
@@ -2126,7 +2135,9 @@ MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane) {
     if (all_done) break;
     int stop = 0;
     if (lane == 0) {
-      if (*reinterpret_cast<volatile const int *>(P.error) != 0) {
+      // the error word is a global round trip: look at it every 16th pass only,
+      // so that an idle producer polls its next dependency at a short interval
+      if ((it & 15) == 15 && *reinterpret_cast<volatile const int *>(P.error) != 0) {
         stop = 1;
       } else if (progress) {
         t_idle = 0;
