@@ -163,7 +163,7 @@ Sizes scratch_sizes(const mk_model_desc &d, int n_sm) {
       size_t ngrp = (size_t)mseqs * d.n_kv_heads * p.attn_qsplit;
       s.attn_o = std::max(s.attn_o, ngrp * p.attn_nch_max * kQvp * d.head_dim);
       s.attn_ml = std::max(s.attn_ml, ngrp * kQvp * 2 * p.attn_nch_max);
-      s.attn_cnt = std::max(s.attn_cnt, ngrp);
+      s.attn_cnt = std::max(s.attn_cnt, ngrp * kQvp);
     }
   return s;
 }
@@ -846,7 +846,7 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
   // words that must read zero when the step starts, first, so one memset clears them
   c.take(p.counters, base, sizeof(uint32_t) * (size_t)pl.n_ops * kCounterStride);
   c.take(p.epoch, base, sizeof(uint32_t) * kCounterStride);
-  c.take(p.attn_cnt, base, sizeof(uint32_t) * ngrp);
+  c.take(p.attn_cnt, base, sizeof(uint32_t) * ngrp * kQvp);
   const size_t zero_bytes = c.used;
   // buffers every step writes before it reads them
   c.take(p.h, base, sizeof(float) * (size_t)kMaxRows * D);

@@ -1588,7 +1588,6 @@ struct AttnShared {
   float *o;           // [compute warps][kQvp][hd] partials (the staging row's space)
   float *q;           // [kQvp][hd] the item's query vectors, rotated and scaled
   float *ml;          // [compute warps][kQvp][2]
-  int *last;          // this CTA completed its group
   uint32_t *rdv;      // rendezvous counter
   uint32_t *seq;      // this warp's rendezvous count
 };
@@ -1829,9 +1828,9 @@ MK_INLINE void attn_final_merge(const Params &P, int lane, int grp, int v, int n
   for (int dd = 0; dd < DPL; ++dd) __stcg(dst + dd, acc[dd] * invl);
 }
 
-// One CTA-wide attention item: every warp computes its share, warps 0..3 merge
-// the 8 shares of one query vector each into the CTA's partial, and the CTA
-// that completes the group merges all CTA partials into o.
+// One CTA-wide attention item: every warp computes its share, warp v (v < 4)
+// merges the warps' shares of query vector v into the CTA's partial, and the
+// warp that completes the count of (group, v) merges all CTA partials into o.
 template <int DPL>
 MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
   const Params &P = *w.P;
@@ -1899,25 +1898,25 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
       __stcg(ml + a.c, M);
       __stcg(ml + P.attn_nch_max + a.c, L);
     }
-  }
-  *sh.seq += kConsumers;
-  if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
-  uint32_t *cnt = P.attn_cnt + grp;
-  if (w.wib == 0 && w.lane == 0) {
-    __threadfence();
-    *reinterpret_cast<volatile int *>(sh.last) = (atom_add_acq_rel(cnt, 1u) + 1 == static_cast<uint32_t>(a.nch)) ? 1 : 0;
-  }
-  *sh.seq += kConsumers;
-  if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
-  if (*reinterpret_cast<volatile int *>(sh.last)) {
-    if (w.wib < kQvp) {
-      (void)ld_acquire(cnt);  // every lane observes the completed count
-      attn_final_merge<DPL>(P, w.lane, grp, w.wib, a.nch, a.b, a.g);
+    // count this CTA's partial of query v; the warp that completes the
+    // (group, v) count merges all of them into o and rewinds the counter
+    uint32_t *cnt = P.attn_cnt + static_cast<size_t>(grp) * kQvp + v;
+    __syncwarp();
+    int last = 0;
+    if (w.lane == 0) {
+      __threadfence();
+      last = (atom_add_acq_rel(cnt, 1u) + 1 == static_cast<uint32_t>(a.nch)) ? 1 : 0;
     }
-    *sh.seq += kConsumers;
-    if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
-    if (w.wib == 0 && w.lane == 0) *cnt = 0;  // rewind for the next layer
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      (void)ld_acquire(cnt);  // every lane observes the completed count
+      attn_final_merge<DPL>(P, w.lane, grp, v, a.nch, a.b, a.g);
+      __syncwarp();
+      if (w.lane == 0) *cnt = 0;
+    }
   }
+  // No CTA barrier here: a next item's query staging ends in one (before any
+  // warp overwrites the partials), and the next op waits for every CTA's arrival.
   return true;
 }
 
@@ -2173,7 +2172,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   __shared__ uint32_t s_stage;
   __shared__ RouteCache s_route;
   __shared__ float s_attn_ml[kConsumers * kQvp * 2];
-  __shared__ int s_attn_last;
   __shared__ Warp s_feed[kConsumers];  // each consumer's tile stream, as its producer keeps it
   __shared__ float s_ssp[kConsumers];  // batch 1: partial sums of h^2 of the staged row
   const int wib = threadIdx.x >> 5;
@@ -2239,7 +2237,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   if (threadIdx.x == 0) {
     s_stage = 0;
     s_route.ready_key = s_route.fill_key = 0;
-    s_attn_last = 0;
     // attention work items per sequence
     s_attn_prefix[0] = 0;
     for (int b = 0; b < kMaxRows; ++b) {
@@ -2272,7 +2269,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   }
 
   uint32_t stage_seq = 0;
-  AttnShared ash{xs, xs + kConsumers * kQvp * P.hd, s_attn_ml, &s_attn_last, &s_stage, &stage_seq};
+  AttnShared ash{xs, xs + kConsumers * kQvp * P.hd, s_attn_ml, &s_stage, &stage_seq};
   float am_val = -INFINITY;
   int am_idx = 0x7fffffff;
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {
