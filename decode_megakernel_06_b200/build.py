@@ -1,6 +1,7 @@
 """Build ``libmk.so`` (the C-ABI decode-step library) in-tree for sm_100a.
 
-Each ``.cu`` file is compiled to an object with nvcc (in parallel), then
+Each ``.cu`` file is compiled to an object with nvcc (in parallel; the step
+kernels twice, with and without the timeline trace), then
 linked into a shared library next to this file.  Only the ``MK_API``
 symbols of ``include/mk.h`` are exported.
 """
@@ -16,7 +17,11 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["mk_kernel.cu", "mk_api.cu", "mk_wide.cu"]
+# (source, object name, extra flags): the step kernels are built twice, the
+# second time with the timeline trace compiled in.
+UNITS = [("mk_kernel.cu", "mk_kernel", []), ("mk_kernel.cu", "mk_kernel_trace", ["-DMK_TRACE=1"]),
+         ("mk_api.cu", "mk_api", []), ("mk_wide.cu", "mk_wide", [])]
+SOURCES = sorted({u[0] for u in UNITS})
 HEADERS = ["mk_internal.h", os.path.join("..", "..", "include", "mk.h")]
 
 NVCC = os.environ.get("NVCC", "nvcc")
@@ -32,29 +37,30 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str) -> str:
-    obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
+def _compile(unit) -> str:
+    src, name, extra = unit
+    obj = os.path.join(BUILD, name + ".o")
     deps = [os.path.join(CSRC, src)] + [os.path.join(CSRC, h) for h in HEADERS]
     if _stale(obj, deps):
-        cmd = [NVCC, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+        cmd = [NVCC, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
-        log = os.path.join(BUILD, os.path.splitext(src)[0] + ".ptxas.txt")
+        log = os.path.join(BUILD, name + ".ptxas.txt")
         with open(log, "w") as fh:
             fh.write(r.stdout + r.stderr)
         if r.returncode != 0:
-            raise RuntimeError(f"nvcc failed for {src}:\n{r.stderr[-4000:]}")
+            raise RuntimeError(f"nvcc failed for {src} ({name}):\n{r.stderr[-4000:]}")
     return obj
 
 
 def build(force: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     if force:
-        for s in SOURCES:
-            o = os.path.join(BUILD, os.path.splitext(s)[0] + ".o")
+        for _, name, _ in UNITS:
+            o = os.path.join(BUILD, name + ".o")
             if os.path.exists(o):
                 os.remove(o)
-    with cf.ThreadPoolExecutor(len(SOURCES)) as ex:
-        objs = list(ex.map(_compile, SOURCES))
+    with cf.ThreadPoolExecutor(len(UNITS)) as ex:
+        objs = list(ex.map(_compile, UNITS))
     if _stale(LIB, objs):
         cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs,
                "-o", LIB + ".tmp", "-lcudart_static", "-ldl", "-lrt", "-lpthread"]

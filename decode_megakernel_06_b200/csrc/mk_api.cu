@@ -353,6 +353,8 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     const size_t smem = make_plan(d, n_sm, 1, mm).smem;
     int per = max_cta_per_sm(mm, smem);
     if (per < 1) return fail(MK_ERR_LAUNCH, "kernel (M<=%d) cannot keep one CTA per SM with %zu B smem", mm, smem);
+    per = max_cta_per_sm_traced(mm, smem);
+    if (per < 1) return fail(MK_ERR_LAUNCH, "traced kernel (M<=%d) cannot keep one CTA per SM with %zu B smem", mm, smem);
   }
 
   mk_handle *h = new mk_handle();
@@ -562,7 +564,7 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
 
 static int launch_variant(mk_handle *h, Params &p, const Plan &pl, cudaStream_t stream, int variant) {
   if (variant == MK_MEGAKERNEL) {
-    int e = launch_step(p, pl.mmax, true, stream);
+    int e = launch_step_any(p, pl.mmax, true, stream);
     if (e) return fail(MK_ERR_LAUNCH, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
     h->stats.kernel_launches += 1;
     return MK_OK;
@@ -570,7 +572,7 @@ static int launch_variant(mk_handle *h, Params &p, const Plan &pl, cudaStream_t 
   for (int op = 0; op < pl.n_ops; ++op) {
     p.op_begin = op;
     p.op_end = op + 1;
-    int e = launch_step(p, pl.mmax, false, stream);
+    int e = launch_step_any(p, pl.mmax, false, stream);
     if (e) return fail(MK_ERR_LAUNCH, "launch of op %d failed: %s", op, cudaGetErrorString((cudaError_t)e));
   }
   p.op_begin = 0;
@@ -867,7 +869,7 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUDA_TRY(cudaMemsetAsync(base, 0, zero_bytes, s));
-  int e = launch_step(p, pl.mmax, true, s);
+  int e = launch_step_any(p, pl.mmax, true, s);
   if (e) return fail(MK_ERR_LAUNCH, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
   h->stats.kernel_launches += 1;
   h->stats.steps += 1;

@@ -139,8 +139,14 @@ struct alignas(64) Params {
   int inject_op;                         // op whose dependency is made unreachable, -1 none
 };
 
-// Launch entry points implemented in mk_kernel.cu.
+// Launch entry points implemented in mk_kernel.cu.  The *_traced forms are the
+// same kernels built with the timeline trace compiled in (Params::trace set).
 int launch_step(const Params &p, int mmax, bool cooperative, cudaStream_t stream);
+int launch_step_traced(const Params &p, int mmax, bool cooperative, cudaStream_t stream);
+int max_cta_per_sm_traced(int mmax, size_t smem);
+inline int launch_step_any(const Params &p, int mmax, bool cooperative, cudaStream_t stream) {
+  return p.trace ? launch_step_traced(p, mmax, cooperative, stream) : launch_step(p, mmax, cooperative, stream);
+}
 // ---- wide blocks (8 < M <= 64 rows): a sequence of launches ----------------------
 constexpr int kWideMaxRows = 64;
 

@@ -35,8 +35,22 @@
 
 #define MK_INLINE __device__ __forceinline__
 
+#ifndef MK_TRACE
+#define MK_TRACE 0
+#endif
+#if MK_TRACE
+#define MK_ENTRY(name) name##_traced
+#else
+#define MK_ENTRY(name) name
+#endif
+
 namespace mk {
 namespace {
+
+// This file is compiled twice: MK_TRACE=0 gives the step kernels, MK_TRACE=1
+// the same kernels with the per-op / per-tile timeline compiled in (launched
+// only when a trace buffer is set), so that the timed kernels carry no trace code.
+constexpr bool kTrace = MK_TRACE != 0;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -452,7 +466,7 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
 // layer, and whether it filled it (words 6 and 7 of its ROUTED_GU record).
 MK_INLINE void trace_route_cache(const Warp &w, int layer, int filler) {
   const Params &P = *w.P;
-  if (P.trace && w.lane == 0 && !w.producer) {
+  if (kTrace && P.trace && w.lane == 0 && !w.producer) {
     unsigned long long *tr = P.trace + (static_cast<size_t>(op_index(layer, OP_ROUTED_GU)) * w.nw + w.slot) * kTraceWords;
     if (tr[6] == 0) {
       tr[6] = now_ns();
@@ -800,7 +814,7 @@ MK_INLINE const uint8_t *consume_begin(Warp &w, int op) {
   if (w.failed) return nullptr;
   uint64_t *bar = &w.full[w.cslot];
   const uint32_t par = (w.phase >> w.cslot) & 1u;
-  const bool tr = w.P->trace != nullptr;
+  constexpr bool tr = kTrace;
   const uint64_t t0 = tr ? now_ns() : 0;
   if (!__all_sync(0xffffffffu, mbar_try_wait(bar, par)) && !wait_slot_slow(bar, par, w.P->timeout_ns)) {
     set_error(w, -5, op);
@@ -815,7 +829,7 @@ MK_INLINE const uint8_t *consume_begin(Warp &w, int op) {
 }
 
 MK_INLINE void consume_end(Warp &w) {
-  if (w.P->trace) {
+  if constexpr (kTrace) {
     w.tr_last = now_ns();
     w.tr_n++;
   }
@@ -2288,7 +2302,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       if (stage && !stage_x(w, type, layer, xs, s_ssp, &s_stage, stage_seq, op)) break;
       if (type == OP_DOWN && P.down_staged && !stage_down(w, layer, xs, &s_stage, stage_seq, op)) break;
     }
-    if (P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords] = now_ns();
+    if (kTrace && P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords] = now_ns();
     w.tr_first = w.tr_last = w.tr_wait = 0;
     w.tr_n = 0;
     bool ok = true;
@@ -2306,7 +2320,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       P.am_part[static_cast<size_t>(w.slot) * kMaxRows + w.lane / kRows] = ArgmaxPart{am_val, am_idx};
     }
     const bool last = arrive(w, op);
-    if (P.trace && w.lane == 0) {
+    if (kTrace && P.trace && w.lane == 0) {
       unsigned long long *tr = P.trace + (static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords;
       tr[1] = w.tr_first;
       tr[2] = w.tr_last;
@@ -2315,10 +2329,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       tr[5] = static_cast<unsigned long long>(w.tr_n);
     }
     if (last && type == OP_ROUTER) {
-      const uint64_t t_topk = P.trace ? now_ns() : 0;
+      const uint64_t t_topk = (kTrace && P.trace) ? now_ns() : 0;
       if (!route_cache(w, layer)) break;
       route_publish(P, w.rc, w.lane, layer);
-      if (P.trace && w.lane == 0) {
+      if (kTrace && P.trace && w.lane == 0) {
         unsigned long long *tr = P.trace + (static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords;
         tr[6] = t_topk;
         tr[7] = now_ns();
@@ -2330,11 +2344,15 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
 
 }  // namespace
 
+#if !MK_TRACE
 size_t step_smem_bytes(int n_ops, int xs_floats) {
   return static_cast<size_t>(kConsumers) * kSlots * kSlotBytes + static_cast<size_t>(xs_floats) * sizeof(float) +
          2 * kConsumers * kSlots * sizeof(uint64_t) + kConsumers * kWbuf * sizeof(float) +
          static_cast<size_t>(n_ops) * sizeof(uint32_t);
 }
+
+bool kernel_stages_x(int mmax) { return mmax == 1; }
+#endif
 
 template <int MMAX, bool XS>
 static const void *kernel_ptr() {
@@ -2351,9 +2369,7 @@ static const void *kernel_for(int mmax) {
   }
 }
 
-bool kernel_stages_x(int mmax) { return mmax == 1; }
-
-int max_cta_per_sm(int mmax, size_t smem) {
+int MK_ENTRY(max_cta_per_sm)(int mmax, size_t smem) {
   const void *k = kernel_for(mmax);
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return -1;
@@ -2371,7 +2387,7 @@ int max_cta_per_sm(int mmax, size_t smem) {
   return n;
 }
 
-int launch_step(const Params &p, int mmax, bool cooperative, cudaStream_t stream) {
+int MK_ENTRY(launch_step)(const Params &p, int mmax, bool cooperative, cudaStream_t stream) {
   const void *k = kernel_for(mmax);
   const size_t smem = step_smem_bytes(p.n_ops, p.xs_floats);
   void *args[] = {const_cast<Params *>(&p)};
