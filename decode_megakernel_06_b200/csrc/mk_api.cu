@@ -277,7 +277,7 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
     size_t f = (size_t)d.max_rows * d.d_model * 2 + (size_t)d.max_rows * ceil_div(d.d_model, kRows) +
                (size_t)kMaxRows * (d.top_k + 1) * d.d_model +
                2 * (size_t)d.max_rows * (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim +
-               (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml +
+               (size_t)d.max_rows * d.d_model + (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml +
                (size_t)ceil_div(d.d_model, kPanel) * kMaxRows * d.n_experts +
                (size_t)kMaxRows * d.shared_ffn +
                (size_t)std::min(d.n_experts, d.max_rows * d.top_k) * kMaxRows * d.expert_ffn +
@@ -376,7 +376,7 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   const int umax = std::min(d.n_experts, std::min(d.max_rows, kMaxRows) * d.top_k);
   HALLOC(h->tmaps, sizeof(CUtensorMap) * (size_t)(L * MAPS_PER_LAYER + 1));
   HALLOC(h->norms, sizeof(void *) * 2 * L);
-  HALLOC(h->h, sizeof(float) * (size_t)kMaxRows * D);
+  HALLOC(h->h, sizeof(float) * 2 * (size_t)kMaxRows * D);  // h, then h * gain (xg)
   HALLOC(h->ss, sizeof(float) * (size_t)kMaxRows * ceil_div(ceil_div(D, kRows), 128) * 128);
   HALLOC(h->qkv, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);  // [K half][row][QKVW]
   HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
@@ -548,6 +548,7 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.kc = static_cast<__nv_bfloat16 *>(kv.k); p.vc = static_cast<__nv_bfloat16 *>(kv.v);
   p.tokens = tokens; p.positions = positions; p.logits = logits ? logits : h->logits; p.argmax = argmax;
   p.h = h->h; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
+  p.xg = h->h + (size_t)kMaxRows * d.d_model;
   p.attn_o = h->attn_o; p.attn_ml = h->attn_ml;
   p.attn_cnt = h->attn_cnt; p.router_part = h->router_part;
   p.act_shared = h->act_shared; p.act_routed = h->act_routed; p.y_part = h->y_part;
@@ -851,7 +852,8 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
   c.take(p.attn_cnt, base, sizeof(uint32_t) * ngrp * kQvp);
   const size_t zero_bytes = c.used;
   // buffers every step writes before it reads them
-  c.take(p.h, base, sizeof(float) * (size_t)kMaxRows * D);
+  c.take(p.h, base, sizeof(float) * 2 * (size_t)kMaxRows * D);
+  p.xg = p.h + (size_t)kMaxRows * D;
   c.take(p.ss, base, sizeof(float) * (size_t)kMaxRows * p.ss_ld);
   c.take(p.qkv, base, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);
   c.take(p.o, base, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);

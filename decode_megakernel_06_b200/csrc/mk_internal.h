@@ -121,6 +121,7 @@ struct alignas(64) Params {
   int *argmax;
   // scratch
   float *h, *ss, *qkv, *o;
+  float *xg;                             // M > 1: h * (the next norm's gain), written with h
   float *attn_o, *attn_ml;   // per-CTA-chunk partials (unnormalised o; max, sum)
   uint32_t *attn_cnt;
   float *router_part;

@@ -914,46 +914,8 @@ MK_INLINE bool arrive(Warp &w, int op) {
 // Activation sources (one lane, 8 consecutive columns, MJ rows)
 // ---------------------------------------------------------------------------
 // RMSNorm is applied as y = inv_rms * (W (h * g)): the per-row scalar is
-// factored out of the dot product and multiplied in the epilogue.
-template <int MJ>
-struct XNorm {  // x = h * g
-  const float *h;
-  int d;
-  const __nv_bfloat16 *g;
-  int row[MJ];
-  int n;
-  MK_INLINE void prefetch(int col, int K) const {
-    if (col < K) {
-#pragma unroll
-      for (int j = 0; j < MJ; ++j)
-        if (j < n) prefetch_l1(h + static_cast<size_t>(row[j]) * d + col);
-    }
-  }
-  MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
-    if (col < K) {
-      float gf[8];
-      unpack8(ldg_nc_v4(g + col), gf);
-#pragma unroll
-      for (int j = 0; j < MJ; ++j) {
-        if (j < n) {
-          const float4 *p = reinterpret_cast<const float4 *>(h + static_cast<size_t>(row[j]) * d + col);
-          const float4 a = __ldca(p), b = __ldca(p + 1);
-          x[j][0] = a.x * gf[0]; x[j][1] = a.y * gf[1]; x[j][2] = a.z * gf[2]; x[j][3] = a.w * gf[3];
-          x[j][4] = b.x * gf[4]; x[j][5] = b.y * gf[5]; x[j][6] = b.z * gf[6]; x[j][7] = b.w * gf[7];
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) x[j][k] = 0.f;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < MJ; ++j)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[j][k] = 0.f;
-    }
-  }
-};
-
+// factored out of the dot product and multiplied in the epilogue.  At M > 1
+// the gained rows h * g are written next to h by the op that produces h.
 template <int MJ>
 struct XPlain {  // x = src[row][col]
   const float *src;
@@ -1007,35 +969,24 @@ struct XSmem {
   }
 };
 
-// With one or two activation rows, even and odd columns go to separate
-// accumulators (acc, acc2) so that each row has two independent FMA chains.
+// Even and odd columns go to separate accumulators (acc, acc2): one packed FMA
+// serves both, and each row has two independent FMA chains.
 template <int MJ>
 MK_INLINE void gemv_panel(const uint8_t *pan, float (&acc)[kRows * MJ], float (&acc2)[kRows * MJ],
                           const float (&x)[MJ][8]) {
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
-    if constexpr (MJ <= 2) {
-      // each (even, odd) column pair in one packed FMA
-      const uint4 u = ld_shared_v4(pan + r * (kPanel * 2));
-      const float2 wp[4] = {bf2(u.x), bf2(u.y), bf2(u.z), bf2(u.w)};
+    // each (even, odd) column pair in one packed FMA: acc holds the even
+    // columns' partial sums, acc2 the odd ones'
+    const uint4 u = ld_shared_v4(pan + r * (kPanel * 2));
+    const float2 wp[4] = {bf2(u.x), bf2(u.y), bf2(u.z), bf2(u.w)};
 #pragma unroll
-      for (int j = 0; j < MJ; ++j) {
-        float2 ab = make_float2(acc[r * MJ + j], acc2[r * MJ + j]);
+    for (int j = 0; j < MJ; ++j) {
+      float2 ab = make_float2(acc[r * MJ + j], acc2[r * MJ + j]);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) ab = fma2(wp[k], make_float2(x[j][2 * k], x[j][2 * k + 1]), ab);
-        acc[r * MJ + j] = ab.x;
-        acc2[r * MJ + j] = ab.y;
-      }
-    } else {
-      float wf[8];
-      unpack8(ld_shared_v4(pan + r * (kPanel * 2)), wf);
-#pragma unroll
-      for (int j = 0; j < MJ; ++j) {
-        float a = acc[r * MJ + j];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) a = fmaf(wf[k], x[j][k], a);
-        acc[r * MJ + j] = a;
-      }
+      for (int k = 0; k < 4; ++k) ab = fma2(wp[k], make_float2(x[j][2 * k], x[j][2 * k + 1]), ab);
+      acc[r * MJ + j] = ab.x;
+      acc2[r * MJ + j] = ab.y;
     }
   }
 }
@@ -1069,7 +1020,7 @@ MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], float (&
 // Streams `ntiles` tiles of one unit through the ring into acc (not reduced).
 template <int MJ, class XS>
 MK_INLINE bool gemv_stream(Warp &w, int op, int ntiles, int col0, int K, const XS &xs, float (&acc)[kRows * MJ]) {
-  float acc2[kRows * MJ];  // odd columns when MJ <= 2 (dead otherwise)
+  float acc2[kRows * MJ];  // the odd columns' partial sums
 #pragma unroll
   for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
   for (int t = 0; t < ntiles; ++t) {
@@ -1078,10 +1029,8 @@ MK_INLINE bool gemv_stream(Warp &w, int op, int ntiles, int col0, int K, const X
     gemv_tile<MJ>(slot, acc, acc2, col0 + t * kTileCols, K, xs, w.lane);
     consume_end(w);
   }
-  if constexpr (MJ <= 2) {
 #pragma unroll
-    for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
-  }
+  for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
   return true;
 }
 
@@ -1103,10 +1052,8 @@ MK_INLINE bool gemv_unit(Warp &w, int op, int ntiles, int col0, int K, const XS 
 // loaded first; a tile across two groups goes box by box.
 template <int MJ>
 MK_INLINE void group_done(float (&acc)[kRows * MJ], float (&acc2)[kRows * MJ], float *buf, int lane) {
-  if constexpr (MJ <= 2) {
 #pragma unroll
-    for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
-  }
+  for (int q = 0; q < kRows * MJ; ++q) acc[q] += acc2[q];
   butterfly<kRows * MJ>(acc, lane);
   butterfly_store<kRows * MJ>(acc, buf, lane);
 #pragma unroll
@@ -1203,17 +1150,21 @@ MK_INLINE void compute_inv_rms(const Params &P, int lane, float (&inv)[kMaxRows]
 // Ops
 // ---------------------------------------------------------------------------
 // New residual rows [row0, row0 + 4): store, the partial sum of squares for
-// the next RMSNorm, and the debug copy.  val(m, row, r) gives the new value.
+// the next RMSNorm, the debug copy and, with gx (the next norm's gain, M > 1
+// only), the gained row xg = h * g that the next op's dot products read.
+// val(m, row, r) gives the new value.
 // Lane 4m + r holds row r of activation row m.
 static_assert(kRows == 4 && kMaxRows * kRows <= 32, "one lane per (row, residual row)");
 template <class F>
-MK_INLINE void residual_rows(const Params &P, int lane, int unit, int row0, int dbg_layer, F val) {
+MK_INLINE void residual_rows(const Params &P, int lane, int unit, int row0, int dbg_layer, const __nv_bfloat16 *gx,
+                             F val) {
   const int m = lane / kRows, r = lane % kRows, row = row0 + r;
   const bool live = lane < kRows * P.M;
   float sq = 0.f;
   if (live && row < P.d) {
     const float hn = val(m, row, r);
     __stcg(P.h + static_cast<size_t>(m) * P.d + row, hn);
+    if (gx) __stcg(P.xg + static_cast<size_t>(m) * P.d + row, hn * __bfloat162float(gx[row]));
     sq = hn * hn;
     if (dbg_layer >= 0 && P.dbg_hidden)
       P.dbg_hidden[(static_cast<size_t>(dbg_layer) * P.max_rows + m) * P.d + row] = hn;
@@ -1229,7 +1180,8 @@ MK_INLINE void residual_rows(const Params &P, int lane, int unit, int row0, int 
 // m of the pass's g-th unit, so that all of a pass's loads are in flight
 // together.  Units are this warp's: slot, slot + nw, ...
 template <class F>
-MK_INLINE void residual_units(const Params &P, int lane, int slot, int nw, int dbg_layer, F val) {
+MK_INLINE void residual_units(const Params &P, int lane, int slot, int nw, int dbg_layer, const __nv_bfloat16 *gx,
+                              F val) {
   const int lanes_per_unit = kRows * P.M, per = 32 / lanes_per_unit;
   const int g = lane / lanes_per_unit, m = (lane / kRows) % P.M, r = lane % kRows;
   for (int base = slot; base < P.n_hb; base += per * nw) {
@@ -1239,6 +1191,7 @@ MK_INLINE void residual_units(const Params &P, int lane, int slot, int nw, int d
     if (live && row < P.d) {
       const float hn = val(m, row);
       __stcg(P.h + static_cast<size_t>(m) * P.d + row, hn);
+      if (gx) __stcg(P.xg + static_cast<size_t>(m) * P.d + row, hn * __bfloat162float(gx[row]));
       sq = hn * hn;
       if (dbg_layer >= 0 && P.dbg_hidden)
         P.dbg_hidden[(static_cast<size_t>(dbg_layer) * P.max_rows + m) * P.d + row] = hn;
@@ -1250,9 +1203,9 @@ MK_INLINE void residual_units(const Params &P, int lane, int slot, int nw, int d
   __syncwarp();
 }
 
-MK_INLINE void op_embed(Warp &w) {
+MK_INLINE void op_embed(Warp &w, bool gained) {
   const Params &P = *w.P;
-  residual_units(P, w.lane, w.slot, w.nw, 0, [&](int m, int row) {
+  residual_units(P, w.lane, w.slot, w.nw, 0, gained ? P.norms[0] : nullptr, [&](int m, int row) {
     int tok = __ldcg(&P.tokens[m]);       // may alias the argmax output
     if (tok < 0 || tok >= P.V) tok = 0;  // rejected at kernel start
     return __bfloat162float(P.embed[static_cast<size_t>(tok) * P.d + row]);
@@ -1260,11 +1213,12 @@ MK_INLINE void op_embed(Warp &w) {
 }
 
 // h += (sum_s w_s y_s) + shared, in the selection order of each row.
-MK_INLINE void op_combine(Warp &w, int layer) {
+MK_INLINE void op_combine(Warp &w, int layer, bool gained) {
   const Params &P = *w.P;
   const int S = P.topk + 1;
   const RouteCache *rt = w.rc;
-  residual_units(P, w.lane, w.slot, w.nw, layer + 1, [&](int m, int row) {
+  const __nv_bfloat16 *gx = !gained ? nullptr : (layer + 1 < P.L) ? P.norms[2 * (layer + 1)] : P.final_norm;
+  residual_units(P, w.lane, w.slot, w.nw, layer + 1, gx, [&](int m, int row) {
     const float *yp = P.y_part + (static_cast<size_t>(m) * S) * P.d + row;
     float moe = 0.f;
 #pragma unroll
@@ -1325,11 +1279,11 @@ MK_INLINE bool with_dense_x(Warp &w, int type, int layer, const float *xs, Body 
     fill_all_rows<MJ>(xp.row, P.M);
     return body(xp);
   } else {
-    XNorm<MJ> xn;
-    xn.h = P.h;
-    xn.d = P.d;
+    // x = h * g, written with h by the op that produced it
+    XPlain<MJ> xn;
+    xn.src = P.xg;
+    xn.ld = P.d;
     xn.n = P.M;
-    xn.g = (type == OP_QKV) ? P.norms[2 * layer] : (type == OP_LMHEAD) ? P.final_norm : P.norms[2 * layer + 1];
     fill_all_rows<MJ>(xn.row, P.M);
     return body(xn);
   }
@@ -1410,7 +1364,8 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
       break;
     }
     case OP_OPROJ:
-      residual_rows(P, w.lane, unit, row0, -1, [&](int mm, int, int rr) { return h_old + wb[rr * MJ + mm]; });
+      residual_rows(P, w.lane, unit, row0, -1, XS ? nullptr : P.norms[2 * layer + 1],
+                    [&](int mm, int, int rr) { return h_old + wb[rr * MJ + mm]; });
       break;
     default: break;
   }
@@ -1424,10 +1379,9 @@ template <int MJ, bool XS>
 MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const float (&inv)[kMaxRows],
                        const float *xs) {
   const Params &P = *w.P;
-  XNorm<MJ> xn;
-  xn.h = P.h;
-  xn.d = P.d;
-  xn.g = P.norms[2 * layer + 1];
+  XPlain<MJ> xn;  // x = h * g (M > 1), written with h by the o-projection
+  xn.src = P.xg;
+  xn.ld = P.d;
   float *dst;
   int ld, f0;
   if (type == OP_ROUTED_GU) {
@@ -2307,10 +2261,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     w.tr_n = 0;
     bool ok = true;
     if (type == OP_EMBED) {
-      op_embed(w);
+      op_embed(w, !XS);
     } else if (type == OP_COMBINE) {
       ok = route_cache(w, layer);
-      if (ok) op_combine(w, layer);
+      if (ok) op_combine(w, layer, !XS);
     } else {
       ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, s_ssp, ash, am_val, am_idx);
     }
