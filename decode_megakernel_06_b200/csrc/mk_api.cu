@@ -145,7 +145,7 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   // with one or two rows per step the two groups of an 8-row down unit can
   // keep separate accumulators, so its tiles go column by column
   p.down_cols = (p.down_groups == 2 && p.mmax <= 2) ? 1 : 0;
-  p.smem = step_smem_bytes(p.n_ops, p.xs_floats);
+  p.smem = step_smem_bytes(p.n_ops, p.xs_floats, p.mmax);
   return p;
 }
 

@@ -18,7 +18,11 @@ constexpr int kFeeds = kConsumers / kProducers;     // consumers fed by one prod
 constexpr int kWarpsPerCta = kConsumers + kProducers;
 constexpr int kThreads = kWarpsPerCta * 32;
 constexpr int kConsumerThreads = kConsumers * 32;
-constexpr int kSlots = 6;                           // ring slots per consumer
+constexpr int kMaxSlots = 6;                        // ring slots per consumer, at most
+// Ring slots per consumer for a kernel of up to `mmax` rows: six at batch 1;
+// four above, where the smaller shared-memory carve-out leaves L1 room for
+// the activation rows that every warp re-reads.
+__host__ __device__ constexpr int ring_slots(int mmax) { return mmax == 1 ? 6 : 4; }
 constexpr int kSlotBytes = 8192;                    // one tile: four 2 KB weight boxes
 constexpr int kPanel = 256;                         // columns per weight box
 constexpr int kRows = 4;                            // rows per weight box, tile and unit
@@ -182,7 +186,7 @@ struct WideStep {
 cudaError_t wide_prepare();
 cudaError_t wide_step(const WideStep &s, cudaStream_t stream, int *launches);
 
-size_t step_smem_bytes(int n_ops, int xs_floats);
+size_t step_smem_bytes(int n_ops, int xs_floats, int mmax);
 bool kernel_stages_x(int mmax);
 int max_cta_per_sm(int mmax, size_t smem);
 

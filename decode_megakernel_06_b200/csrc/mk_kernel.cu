@@ -291,7 +291,8 @@ struct Warp {
   RouteCache *rc;
   int lane, wib, cta, slot, nw;
   uint32_t epoch;
-  uint8_t *ring;           // this consumer's kSlots tiles
+  uint8_t *ring;           // this consumer's nslots tiles
+  int nslots;
   uint64_t *full, *empty;  // per slot: tile landed / tile released
   float *wbuf;
   uint32_t *arrive;
@@ -733,7 +734,7 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
   }
   w.ephase ^= 1u << w.islot;
   w.filled |= 1u << w.islot;
-  w.islot = (w.islot + 1 == kSlots) ? 0 : w.islot + 1;
+  w.islot = (w.islot + 1 == w.nslots) ? 0 : w.islot + 1;
 }
 
 // Producer: issue the fed consumer's next tiles into its released slots, in
@@ -836,7 +837,7 @@ MK_INLINE void consume_end(Warp &w) {
   __syncwarp();  // every lane is done with the slot before it is released
   if (w.lane == 0) mbar_arrive(&w.empty[w.cslot]);
   w.phase ^= (1u << w.cslot);
-  w.cslot = (w.cslot + 1 == kSlots) ? 0 : w.cslot + 1;
+  w.cslot = (w.cslot + 1 == w.nslots) ? 0 : w.cslot + 1;
 }
 
 // Wait for `ctr` to reach `target` (bounded).
@@ -876,7 +877,7 @@ MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int o
 // for a consumer has landed, consumed or not.  The last fill of slot s
 // completes the phase of parity ephase bit s.
 MK_INLINE void drain_feed(const Warp &f) {
-  for (int s = 0; s < kSlots; ++s) {
+  for (int s = 0; s < f.nslots; ++s) {
     if (!((f.filled >> s) & 1u)) continue;
     const uint64_t t0 = now_ns();
     while (!mbar_try_wait(&f.full[s], (f.ephase >> s) & 1u)) {
@@ -2146,11 +2147,12 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   const bool consumer = wib < kConsumers;
   // dynamic shared memory: rings | activation row | full and empty barriers |
   // epilogue scratch | per-op arrival counts
-  float *xs = reinterpret_cast<float *>(smem + kConsumers * kSlots * kSlotBytes);
+  constexpr int S = ring_slots(MMAX);
+  float *xs = reinterpret_cast<float *>(smem + kConsumers * S * kSlotBytes);
   uint8_t *after_xs = reinterpret_cast<uint8_t *>(xs + P.xs_floats);
   uint64_t *fulls = reinterpret_cast<uint64_t *>(after_xs);
-  uint64_t *empties = fulls + kConsumers * kSlots;
-  float *fbase = reinterpret_cast<float *>(empties + kConsumers * kSlots);
+  uint64_t *empties = fulls + kConsumers * S;
+  float *fbase = reinterpret_cast<float *>(empties + kConsumers * S);
   uint32_t *arrive_cnt = reinterpret_cast<uint32_t *>(fbase + kConsumers * kWbuf);
   Warp w;
   w.P = &P;
@@ -2161,9 +2163,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.nw = P.n_warps;
   w.slot = consumer ? wib * P.n_cta + blockIdx.x : -1;
   const int c = consumer ? wib : 0;  // producers reach their consumers' records through s_feed
-  w.ring = smem + c * kSlots * kSlotBytes;
-  w.full = fulls + c * kSlots;
-  w.empty = empties + c * kSlots;
+  w.ring = smem + c * S * kSlotBytes;
+  w.nslots = S;
+  w.full = fulls + c * S;
+  w.empty = empties + c * S;
   w.wbuf = fbase + c * kWbuf;
   w.arrive = arrive_cnt;
   w.attn_prefix = s_attn_prefix;
@@ -2171,7 +2174,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.phase = 0;
   w.cslot = 0;
   w.islot = 0;
-  w.ephase = (1u << kSlots) - 1u;  // a fresh barrier's previous phase counts as complete
+  w.ephase = (1u << S) - 1u;  // a fresh barrier's previous phase counts as complete
   w.filled = 0;
   w.producer = false;
   w.dseg0 = 0;
@@ -2192,7 +2195,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.tr_first = w.tr_last = w.tr_wait = 0;
   w.tr_n = 0;
   if (consumer && w.lane == 0) {
-    for (int sl = 0; sl < kSlots; ++sl) {
+    for (int sl = 0; sl < S; ++sl) {
       mbar_init(&w.full[sl], 1);
       mbar_init(&w.empty[sl], 1);
     }
@@ -2299,9 +2302,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
 }  // namespace
 
 #if !MK_TRACE
-size_t step_smem_bytes(int n_ops, int xs_floats) {
-  return static_cast<size_t>(kConsumers) * kSlots * kSlotBytes + static_cast<size_t>(xs_floats) * sizeof(float) +
-         2 * kConsumers * kSlots * sizeof(uint64_t) + kConsumers * kWbuf * sizeof(float) +
+size_t step_smem_bytes(int n_ops, int xs_floats, int mmax) {
+  const int S = ring_slots(mmax);
+  return static_cast<size_t>(kConsumers) * S * kSlotBytes + static_cast<size_t>(xs_floats) * sizeof(float) +
+         2 * kConsumers * S * sizeof(uint64_t) + kConsumers * kWbuf * sizeof(float) +
          static_cast<size_t>(n_ops) * sizeof(uint32_t);
 }
 
@@ -2343,7 +2347,7 @@ int MK_ENTRY(max_cta_per_sm)(int mmax, size_t smem) {
 
 int MK_ENTRY(launch_step)(const Params &p, int mmax, bool cooperative, cudaStream_t stream) {
   const void *k = kernel_for(mmax);
-  const size_t smem = step_smem_bytes(p.n_ops, p.xs_floats);
+  const size_t smem = step_smem_bytes(p.n_ops, p.xs_floats, mmax);
   void *args[] = {const_cast<Params *>(&p)};
   cudaError_t e;
   if (cooperative) {
