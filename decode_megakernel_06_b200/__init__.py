@@ -98,6 +98,7 @@ def lib():
     sig = {
         "mk_create": (i32, [ctypes.POINTER(mk_model_desc), ctypes.POINTER(mk_weights), ctypes.POINTER(vp)]),
         "mk_decode_step": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
+        "mk_decode_steps": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
         "mk_decode_step_host": (i32, [vp, _I32P, _I32P, i32, i32, mk_kv_cache, vp, _I32P, vp]),
         "mk_decode_step_static": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
         "mk_get_device_status": (i32, [vp, vp]),
@@ -153,6 +154,12 @@ def mk_create(desc: mk_model_desc, weights: mk_weights) -> ctypes.c_void_p:
     h = ctypes.c_void_p()
     _check(lib().mk_create(ctypes.byref(desc), ctypes.byref(weights), ctypes.byref(h)))
     return h
+
+
+def mk_decode_steps(h, tokens: int, positions: int, B: int, n_steps: int, kv: mk_kv_cache,
+                    out_logits: int, out_tokens: int, stream: int) -> int:
+    """n_steps greedy steps in one launch (see include/mk.h)."""
+    return lib().mk_decode_steps(h, tokens, positions, B, n_steps, kv, out_logits, out_tokens, stream)
 
 
 def mk_decode_step(h, tokens: int, positions: int, B: int, T: int, kv: mk_kv_cache,
@@ -281,6 +288,15 @@ class Decoder:
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_step(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
                               _ptr(logits), argmax.data_ptr(), s.cuda_stream)
+
+    def steps(self, tokens, positions, B: int, n_steps: int, k_cache, v_cache, logits, out_tokens,
+              stream=None) -> int:
+        """Enqueue n_steps greedy steps as one launch; out_tokens is int32
+        [n_steps, B] on the device.  Returns the launch status code."""
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
+        return mk_decode_steps(self.h, tokens.data_ptr(), positions.data_ptr(), B, n_steps, kv,
+                               _ptr(logits), out_tokens.data_ptr(), s.cuda_stream)
 
     def step_static(self, tokens, positions, B: int, T: int, k_cache, v_cache, logits, argmax,
                     stream=None) -> int:

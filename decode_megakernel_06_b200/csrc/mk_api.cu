@@ -530,6 +530,7 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.E = d.n_experts; p.topk = d.top_k; p.F = d.expert_ffn; p.Fs = d.shared_ffn; p.V = d.vocab;
   p.Bmax = d.max_seqs; p.cap = d.kv_capacity; p.eps = d.rms_eps;
   p.B = B; p.T = T; p.M = B * T; p.max_rows = d.max_rows;
+  p.n_steps = 1;
   p.n_cta = pl.n_cta; p.n_warps = pl.n_warps; p.op_begin = 0; p.op_end = pl.n_ops; p.n_ops = pl.n_ops;
   p.n_hb = pl.n_hb;
   p.xs_floats = pl.xs_floats;
@@ -689,6 +690,26 @@ MK_API int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *po
                           int32_t T, mk_kv_cache kv, float *out_logits, int32_t *out_argmax,
                           void *stream) {
   return run_step(h, tokens, positions, B, T, kv, out_logits, out_argmax, static_cast<cudaStream_t>(stream));
+}
+
+MK_API int mk_decode_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
+                           int32_t n_steps, mk_kv_cache kv, float *out_logits, int32_t *out_tokens,
+                           void *stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (n_steps < 1) return fail(MK_ERR_ARG, "n_steps must be >= 1");
+  if (B > kMaxRows) return fail(MK_ERR_UNSUPPORTED, "a multi-step launch serves at most %d sequences", kMaxRows);
+  if (n_steps > h->desc.kv_capacity) return fail(MK_ERR_CAPACITY, "n_steps=%d exceeds kv_capacity", n_steps);
+  Params p;
+  Plan pl;
+  int rc = fill_params(h, tokens, positions, B, 1, kv, out_logits, out_tokens, p, pl);
+  if (rc) return rc;
+  p.n_steps = n_steps;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int e = launch_step_any(p, pl.mmax, true, s);
+  if (e) return fail(MK_ERR_LAUNCH, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
+  h->stats.kernel_launches += 1;
+  h->stats.steps += n_steps;
+  return MK_OK;
 }
 
 MK_API int mk_get_device_status(mk_handle *h, void *stream) {

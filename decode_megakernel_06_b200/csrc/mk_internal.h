@@ -99,6 +99,9 @@ struct alignas(64) Params {
   int L, d, Hq, Hkv, hd, E, topk, F, Fs, V, Bmax, cap;
   float eps;
   int B, T, M, max_rows;
+  int n_steps;         // greedy steps in this launch (T = 1 when > 1); step s embeds
+                       // tokens (s = 0) or argmax[s-1], appends at positions[b] + s and
+                       // writes its argmax to argmax[s * M ..]
   // grid / schedule
   int n_cta, n_warps, op_begin, op_end, n_ops;
   int n_hb;            // residual row blocks (ceil(d / kRows))

@@ -177,15 +177,9 @@ MK_INLINE float2 bf2(uint32_t u) { return make_float2(bf_lo(u), bf_hi(u)); }
 MK_INLINE float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 MK_INLINE float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
-MK_INLINE void unpack8(const uint4 &w, float (&f)[8]) {
-  f[0] = bf_lo(w.x); f[1] = bf_hi(w.x); f[2] = bf_lo(w.y); f[3] = bf_hi(w.y);
-  f[4] = bf_lo(w.z); f[5] = bf_hi(w.z); f[6] = bf_lo(w.w); f[7] = bf_hi(w.w);
-}
 
-MK_INLINE uint4 ldg_nc_v4(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
 
 // Bring the line holding p into this SM's L1 (no register result).
-MK_INLINE void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
 MK_INLINE float silu(float u) { return u / (1.0f + expf(-u)); }
 
@@ -277,7 +271,7 @@ constexpr int kWbuf = 64;  // floats of per-warp epilogue scratch (2 * 4 * MJ <=
 // weight, in selection order), and the ascending union of the selected
 // experts with the rows that chose each and in which selection slot.
 struct RouteCache {
-  int ready_key, fill_key;   // layer + 1 once computed / being computed
+  int ready_key, fill_key;   // route_key of the layer once computed / being computed
   int n_union;
   int expert[kMaxExperts];
   uint32_t rowmask[kMaxExperts];
@@ -296,8 +290,9 @@ struct Warp {
   uint64_t *full, *empty;  // per slot: tile landed / tile released
   float *wbuf;
   uint32_t *arrive;
-  const int *attn_prefix;  // shared: first item of each sequence, [kMaxRows + 1]
-  const int *attn_nch;     // shared: KV chunks of each sequence, [kMaxRows]
+  int *attn_prefix;        // this warp's: first item of each sequence, [kMaxRows + 1]
+  int *attn_nch;           // this warp's: KV chunks of each sequence, [kMaxRows]
+  int step;                // the step (of a multi-step launch) this warp is in
   // consumer side: bit s = parity of the next completion of full[s]
   uint32_t phase;
   int cslot;
@@ -359,7 +354,7 @@ MK_INLINE int expert_of(int lane, int i) { return (i < 4) ? 4 * lane + i : 128 +
 // sum over chosen i of e^(z_i - z_max).  Every CTA runs this on the same
 // partials and gets the same result.  The code runs once per layer per CTA
 // (cold), so it is kept short.
-__device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int lane, int layer) {
+__device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int lane, int key) {
   const int E = P.E, K = P.topk;
   const int nkc = cdiv(P.d, kTileCols);
   constexpr int EPL = 8;
@@ -459,7 +454,7 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
   if (lane == 0) rc->n_union = lo_total + hi_total;
   __threadfence_block();
   __syncwarp();
-  if (lane == 0) *reinterpret_cast<volatile int *>(&rc->ready_key) = layer + 1;
+  if (lane == 0) *reinterpret_cast<volatile int *>(&rc->ready_key) = key;
   __syncwarp();
 }
 
@@ -476,21 +471,25 @@ MK_INLINE void trace_route_cache(const Warp &w, int layer, int filler) {
   }
 }
 
+// The routing of (step, layer) is identified by step * L + layer + 1.
+MK_INLINE int route_key(const Warp &w, int layer) { return w.step * w.P->L + layer + 1; }
+
 MK_INLINE bool route_cache(Warp &w, int layer) {
   RouteCache *rc = w.rc;
-  if (*reinterpret_cast<volatile int *>(&rc->ready_key) == layer + 1) {
+  const int key = route_key(w, layer);
+  if (*reinterpret_cast<volatile int *>(&rc->ready_key) == key) {
     __threadfence_block();
     trace_route_cache(w, layer, 0);
     return true;
   }
   int filler = 0;
-  if (w.lane == 0) filler = atomicMax(&rc->fill_key, layer + 1) < layer + 1 ? 1 : 0;
+  if (w.lane == 0) filler = atomicMax(&rc->fill_key, key) < key ? 1 : 0;
   filler = __shfl_sync(0xffffffffu, filler, 0);
   if (filler) {
-    route_compute(*w.P, rc, w.lane, layer);
+    route_compute(*w.P, rc, w.lane, key);
   } else {
     const uint64_t t0 = now_ns();
-    while (*reinterpret_cast<volatile int *>(&rc->ready_key) != layer + 1) {
+    while (*reinterpret_cast<volatile int *>(&rc->ready_key) != key) {
       __nanosleep(64);  // leave the issue slots to the warp computing it
       if (now_ns() - t0 > w.P->timeout_ns) {
         report_error(*w.P, w.lane, -5, -1);
@@ -583,7 +582,24 @@ struct AttnItem {
   int pos0, npos, ntiles;  // this warp's positions: [pos0, pos0 + npos), in tiles
 };
 
-MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs, int item, int wib) {
+// Cache index of sequence b's first new row in step `step` of the launch.
+MK_INLINE int seq_pos(const Params &P, int b, int step) { return __ldg(&P.positions[b]) + step * P.T; }
+
+// Attention items of one step: per sequence its KV chunks and first item
+// (lane 0 computes, the warp reads).
+MK_INLINE void attn_layout(const Params &P, int step, int *prefix, int *nch, int lane) {
+  if (lane == 0) {
+    prefix[0] = 0;
+    for (int b = 0; b < kMaxRows; ++b) {
+      const int n = b < P.B ? cdiv(seq_pos(P, b, step) + P.T, P.attn_chunk * kConsumers) : 0;
+      nch[b] = n;
+      prefix[b + 1] = prefix[b] + P.Hkv * P.attn_qsplit * n;
+    }
+  }
+  __syncwarp();
+}
+
+MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs, int item, int wib, int step) {
   AttnItem a;
   int b = 0;
   while (b + 1 < P.B && item >= prefix[b + 1]) ++b;
@@ -594,7 +610,7 @@ MK_INLINE AttnItem attn_item(const Params &P, const int *prefix, const int *nchs
   a.c = rem % nch;
   a.qs = (rem / nch) % P.attn_qsplit;
   a.g = rem / (nch * P.attn_qsplit);
-  const int len = __ldg(&P.positions[b]) + P.T;
+  const int len = seq_pos(P, b, step) + P.T;
   a.pos0 = a.c * P.attn_chunk * kConsumers + wib * P.attn_chunk;
   a.npos = max(0, min(P.attn_chunk, len - a.pos0));
   a.ntiles = cdiv(a.npos, P.attn_ppt);
@@ -619,7 +635,7 @@ MK_INLINE int unit_tiles(const Warp &w, int type, int layer, int unit) {
       const int K = (unit / P.n_db) < n_union(w) ? P.F : P.Fs;
       return cdiv(P.down_groups * cdiv(K, kPanel), kPanels);
     }
-    case OP_ATTN: return attn_item(P, w.attn_prefix, w.attn_nch, unit, w.wib).ntiles;
+    case OP_ATTN: return attn_item(P, w.attn_prefix, w.attn_nch, unit, w.wib, w.step).ntiles;
     default: return 0;
   }
 }
@@ -694,7 +710,7 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
   uint8_t *dst = w.ring + w.islot * kSlotBytes;
   uint64_t *bar = &w.full[w.islot];
   if (type == OP_ATTN) {
-    const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, w.iunit, w.wib);
+    const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, w.iunit, w.wib, w.step);
     const int row = ((layer * P.Bmax + a.b) * P.Hkv + a.g) * P.cap + a.pos0 + t * P.attn_ppt;
     if (w.lane == 0) {
       fence_proxy_async_smem();
@@ -762,6 +778,14 @@ MK_INLINE bool feed_more(Warp &w) {
       continue;
     }
     if (w.iop >= P.op_end) {
+      if (w.step + 1 < P.n_steps) {  // the next step of the launch
+        w.step++;
+        w.epoch++;
+        w.iop = P.op_begin;
+        w.iop_init = false;
+        attn_layout(P, w.step, w.attn_prefix, w.attn_nch, w.lane);
+        continue;
+      }
       w.done_issue = true;
       progress = true;
       break;
@@ -896,8 +920,8 @@ MK_INLINE bool arrive(Warp &w, int op) {
     // The warp's results (ordered before this by __syncwarp) are released to
     // the CTA; the CTA's last warp acquires them here and releases them, with
     // its own, grid-wide through the counter (release is cumulative).
-    const uint32_t old = atom_add_acq_rel_cta(&w.arrive[op], 1u);
-    if (old == kConsumers - 1) {
+    const uint32_t old = atom_add_acq_rel_cta(&w.arrive[op], 1u);  // counts on over the launch's steps
+    if (old % kConsumers == kConsumers - 1) {
       const uint32_t g = atom_add_acq_rel(&P.counters[op * kCounterStride], 1u);
       last = (g + 1 == w.epoch * static_cast<uint32_t>(P.n_cta)) ? 1 : 0;
     }
@@ -923,13 +947,6 @@ struct XPlain {  // x = src[row][col]
   int ld;
   int row[MJ];
   int n;
-  MK_INLINE void prefetch(int col, int K) const {
-    if (col < K) {
-#pragma unroll
-      for (int j = 0; j < MJ; ++j)
-        if (j < n) prefetch_l1(src + static_cast<size_t>(row[j]) * ld + col);
-    }
-  }
   MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
 #pragma unroll
     for (int j = 0; j < MJ; ++j) {
@@ -955,7 +972,6 @@ MK_INLINE int xs_pos4(int c4) {  // float4 slot of columns 4*c4 .. 4*c4+3
 }
 struct XSmem {
   const float *xs;
-  MK_INLINE void prefetch(int, int) const {}
   MK_INLINE void load(int col, int K, float (&x)[1][8]) const {
     if (col < K) {
       const float *pb = xs + (col & ~(kPanel - 1)) + ((col & (kPanel - 1)) >> 1);
@@ -1207,7 +1223,9 @@ MK_INLINE void residual_units(const Params &P, int lane, int slot, int nw, int d
 MK_INLINE void op_embed(Warp &w, bool gained) {
   const Params &P = *w.P;
   residual_units(P, w.lane, w.slot, w.nw, 0, gained ? P.norms[0] : nullptr, [&](int m, int row) {
-    int tok = __ldcg(&P.tokens[m]);       // may alias the argmax output
+    // step 0: the given tokens (may alias the argmax output); later steps:
+    // the previous step's argmax
+    int tok = w.step ? __ldcg(&P.argmax[(w.step - 1) * P.M + m]) : __ldcg(&P.tokens[m]);
     if (tok < 0 || tok >= P.V) tok = 0;  // rejected at kernel start
     return __bfloat162float(P.embed[static_cast<size_t>(tok) * P.d + row]);
   });
@@ -1572,7 +1590,7 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
   constexpr int NS = kKvBoxBytes / (2 * HD) / 4;  // groups of four positions per tile
   static_assert(QVP == 4, "one query vector per lane pair");
   const int G = P.Hq / P.Hkv;
-  const int pos_b = __ldg(&P.positions[a.b]);
+  const int pos_b = seq_pos(P, a.b, w.step);
   const int W3 = (P.Hq + 2 * P.Hkv) * HD;
   const int lane = w.lane, pg = lane >> 3, dl = lane & 7, myq = dl >> 1;
   const int d0 = C * dl, d1 = HALF + C * dl;
@@ -1804,7 +1822,7 @@ template <int DPL>
 MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
   const Params &P = *w.P;
   constexpr int hd = 32 * DPL;
-  const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, item, w.wib);
+  const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, item, w.wib, w.step);
   {
     // the item's query vectors, once per CTA: warp v rotates (rotate-half
     // pairs (i, i + hd/2) over its lanes) and scales query vector v
@@ -1813,7 +1831,7 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
     const int v = w.wib, qv = a.qs * kQvp + v, G = P.Hq / P.Hkv;
     float *dst = sh.q + v * hd;
     if (qv < G * P.T) {
-      const int t = qv / G, head = a.g * G + qv % G, m = a.b * P.T + t, p = __ldg(&P.positions[a.b]) + t;
+      const int t = qv / G, head = a.g * G + qv % G, m = a.b * P.T + t, p = seq_pos(P, a.b, w.step) + t;
       const size_t src = static_cast<size_t>(m) * (P.Hq + 2 * P.Hkv) * hd + head * hd;
       const float scale = 1.0f / sqrtf(static_cast<float>(hd));
       float x1[HALF / 32], x2[HALF / 32];
@@ -1905,7 +1923,7 @@ __device__ __noinline__ void route_publish(const Params &P, const RouteCache *rc
   __syncwarp();
 }
 
-__device__ __noinline__ void final_argmax(const Params &P, int lane, uint32_t epoch) {
+__device__ __noinline__ void final_argmax(const Params &P, int lane, uint32_t epoch, int step) {
   for (int m = 0; m < P.M; ++m) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
@@ -1927,7 +1945,7 @@ __device__ __noinline__ void final_argmax(const Params &P, int lane, uint32_t ep
         bi = oi;
       }
     }
-    if (lane == 0) P.argmax[m] = (bi == 0x7fffffff) ? 0 : bi;
+    if (lane == 0) P.argmax[step * P.M + m] = (bi == 0x7fffffff) ? 0 : bi;
   }
   __syncwarp();
   if (lane == 0) {
@@ -2075,31 +2093,22 @@ MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs
   return true;
 }
 
-// Producer warp: keep the rings of its kFeeds consumers filled until every
-// tile of the launch's ops has been issued, then wait for the last copies.
-// With one consumer per producer its stream state stays in registers;
-// otherwise each consumer's state lives in shared memory between visits.
-MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane) {
+// Producer warp: keep its consumer's ring filled until every tile of the
+// launch's ops (all its steps) has been issued, then wait for the last copies.
+// The consumer's stream state stays in registers; the producer keeps its own
+// per-step attention layout (it may be a step ahead of its consumer).
+MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane, int *prefix, int *nch) {
+  static_assert(kFeeds == 1, "one consumer per producer");
   Warp mine = feeds[first];
   mine.lane = lane;
+  mine.attn_prefix = prefix;
+  mine.attn_nch = nch;
+  attn_layout(P, 0, prefix, nch, lane);
   uint64_t t_idle = 0;
   for (int it = 0;; ++it) {
     bool progress = false, all_done = true;
-    if constexpr (kFeeds == 1) {
-      if (!mine.done_issue && !mine.failed) progress = feed_more(mine);
-      all_done = mine.done_issue || mine.failed;
-    } else {
-      for (int k = 0; k < kFeeds; ++k) {
-        Warp f = feeds[first + k];
-        if (f.done_issue || f.failed) continue;
-        f.lane = lane;
-        progress |= feed_more(f);
-        all_done = all_done && (f.done_issue || f.failed);
-        __syncwarp();
-        if (lane == 0) feeds[first + k] = f;
-        __syncwarp();
-      }
-    }
+    if (!mine.done_issue && !mine.failed) progress = feed_more(mine);
+    all_done = mine.done_issue || mine.failed;
     if (all_done) break;
     int stop = 0;
     if (lane == 0) {
@@ -2125,19 +2134,15 @@ MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane) {
     if (stop == 2) report_error(P, lane, -5, -1);
     if (stop) break;
   }
-  if constexpr (kFeeds == 1) {
-    drain_feed(mine);
-  } else {
-    for (int k = 0; k < kFeeds; ++k) drain_feed(feeds[first + k]);
-  }
+  drain_feed(mine);
   __syncwarp();
 }
 
 template <int MMAX, bool XS>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ int s_attn_prefix[kMaxRows + 1];
-  __shared__ int s_attn_nch[kMaxRows];
+  __shared__ int s_attn_prefix[kWarpsPerCta][kMaxRows + 1];  // each warp's, for its step
+  __shared__ int s_attn_nch[kWarpsPerCta][kMaxRows];
   __shared__ uint32_t s_stage;
   __shared__ RouteCache s_route;
   __shared__ float s_attn_ml[kConsumers * kQvp * 2];
@@ -2169,8 +2174,9 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.empty = empties + c * S;
   w.wbuf = fbase + c * kWbuf;
   w.arrive = arrive_cnt;
-  w.attn_prefix = s_attn_prefix;
-  w.attn_nch = s_attn_nch;
+  w.attn_prefix = s_attn_prefix[wib];
+  w.attn_nch = s_attn_nch[wib];
+  w.step = 0;
   w.phase = 0;
   w.cslot = 0;
   w.islot = 0;
@@ -2208,13 +2214,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   if (threadIdx.x == 0) {
     s_stage = 0;
     s_route.ready_key = s_route.fill_key = 0;
-    // attention work items per sequence
-    s_attn_prefix[0] = 0;
-    for (int b = 0; b < kMaxRows; ++b) {
-      const int nch = b < P.B ? cdiv(__ldg(&P.positions[b]) + P.T, P.attn_chunk * kConsumers) : 0;
-      s_attn_nch[b] = nch;
-      s_attn_prefix[b + 1] = s_attn_prefix[b] + P.Hkv * P.attn_qsplit * nch;
-    }
   }
   __syncthreads();
 
@@ -2223,7 +2222,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   bool bad = false;
   for (int b = 0; b < P.B; ++b) {
     const int p = __ldg(&P.positions[b]);
-    if (p < 0 || p + P.T > P.cap) bad = true;
+    if (p < 0 || p + P.T * P.n_steps > P.cap) bad = true;
   }
   for (int m = w.lane; m < P.M; m += 32) {
     const int t = __ldcg(&P.tokens[m]);
@@ -2235,12 +2234,16 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   }
 
   if (!consumer) {
-    producer_run(P, s_feed, (wib - kConsumers) * kFeeds, w.lane);
+    producer_run(P, s_feed, (wib - kConsumers) * kFeeds, w.lane, s_attn_prefix[wib], s_attn_nch[wib]);
     return;
   }
 
   uint32_t stage_seq = 0;
   AttnShared ash{xs, xs + kConsumers * kQvp * P.hd, s_attn_ml, &s_stage, &stage_seq};
+  for (; w.step < P.n_steps && !w.failed; ++w.step, ++w.epoch) {
+  attn_layout(P, w.step, w.attn_prefix, w.attn_nch, w.lane);
+  // a later step embeds the previous step's argmax: wait for its publication
+  if (w.step > 0 && !wait_counter(w, P.epoch, w.epoch - 1u, P.op_begin)) break;
   float am_val = -INFINITY;
   int am_idx = 0x7fffffff;
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {
@@ -2295,8 +2298,9 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
         tr[7] = now_ns();
       }
     }
-    if (last && type == OP_LMHEAD) final_argmax(P, w.lane, w.epoch);
+    if (last && type == OP_LMHEAD) final_argmax(P, w.lane, w.epoch, w.step);
   }
+  }  // steps
 }
 
 }  // namespace

@@ -169,6 +169,28 @@ MK_API int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *po
                           int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
                           int32_t *out_argmax, void *stream);
 
+/* n_steps greedy decode steps of B sequences (one new token each, T = 1) in
+ * ONE persistent launch, with no host round trip between steps: step s
+ * embeds `tokens` (s = 0) or step s-1's argmax, appends K/V at
+ * positions[b] + s, and writes its argmax to out_tokens[s*B + b].  The
+ * megakernel pages' single program extended over steps; the schedule of each
+ * step is that of mk_decode_step (same arithmetic, same results).
+ *   tokens     : device int32 [B], ids in [0, vocab)
+ *   positions  : device int32 [B]; 0 <= positions[b], positions[b] + n_steps <= kv_capacity
+ *   B          : 1 <= B <= min(max_seqs, max_rows, 8)
+ *   n_steps    : >= 1
+ *   kv         : the cache, appended in place
+ *   out_logits : device fp32 [B][vocab]: the LAST step's logits, or NULL
+ *   out_tokens : device int32 [n_steps][B] (row 0 may alias tokens)
+ *   stream     : cudaStream_t (NULL = legacy default stream)
+ * Always runs as the megakernel, whatever variant the handle is set to.
+ * Asynchronous; device-side errors (bad ids or positions, timeouts) stop the
+ * launch and are read with mk_get_device_status.  Errors: MK_ERR_ARG,
+ * MK_ERR_CAPACITY and MK_ERR_UNSUPPORTED (B > 8) from the host checks. */
+MK_API int mk_decode_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                           int32_t B, int32_t n_steps, mk_kv_cache kv, float *out_logits,
+                           int32_t *out_tokens, void *stream);
+
 /* The same step driven from HOST buffers: copies tokens [B*T] and positions
  * [B] to the device, runs the step, copies argmax [B*T] back to
  * out_argmax_host, and waits for the stream.  Logits stay on the device
