@@ -389,6 +389,34 @@ def trace_step(dec, m, k, v, B, T, ctx, device, out=sys.stderr, save=None):
     return rows
 
 
+def measure_multi_step(dec, m, k, v, B, ctx, n_steps, device):
+    """n_steps greedy steps in ONE persistent launch (mk_decode_steps), each
+    step feeding its argmax to the next on the device; CUDA events around one
+    launch after two warm-up launches.  The launch streams n_steps x the
+    step's bytes, far more than L2."""
+    import torch
+
+    from synthetic import make_tokens
+
+    tok = torch.tensor(make_tokens(m.vocab, B, 77), dtype=torch.int32, device=device)
+    pos = torch.tensor(ctx[:B], dtype=torch.int32, device=device)
+    out = torch.empty((n_steps, B), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        assert dec.steps(tok, pos, B, n_steps, k, v, None, out) == 0
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    assert dec.steps(tok, pos, B, n_steps, k, v, None, out) == 0
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    ms = e0.elapsed_time(e1)
+    return {"steps_per_launch": n_steps, "batch": B, "ms_per_step": round(ms / n_steps, 4),
+            "tok_s": round(n_steps * B / (ms / 1e3), 1), "launches": 1,
+            "path": "mk_decode_steps: one persistent launch, argmax fed back on the device"}
+
+
 def measure_verify_wide(device, steps=10, warmup=3):
     """The 56-row speculative-verify block (8 sequences x 7 rows, the small
     model) through the wide-block tensor-core path."""
@@ -490,6 +518,10 @@ def run_mine(args):
             sweep[f"bs{bb}"] = row
         dec.set_variant(args.variant)
 
+    multi = None
+    if args.sweep and T == 1:
+        multi = measure_multi_step(dec, m, k, v, B, ctx, 32, device)
+
     verify56 = None
     if args.sweep and ws == 1 and args.workload == "large":
         verify56 = measure_verify_wide(device)
@@ -532,6 +564,8 @@ def run_mine(args):
         }
         if sweep is not None:
             line["batch_sweep"] = sweep
+        if multi is not None:
+            line["multi_step"] = multi
         if verify56 is not None:
             line["verify_56"] = verify56
         print(json.dumps(line), flush=True)

@@ -759,6 +759,7 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
 // activations, so the stream runs ahead across ops and layers; it stops only
 // at a full ring and where the routing is not known yet.  Returns true if it
 // issued a tile or finished the stream.
+template <bool MULTI>
 MK_INLINE bool feed_more(Warp &w) {
   const Params &P = *w.P;
   bool progress = false;
@@ -778,7 +779,7 @@ MK_INLINE bool feed_more(Warp &w) {
       continue;
     }
     if (w.iop >= P.op_end) {
-      if (w.step + 1 < P.n_steps) {  // the next step of the launch
+      if (MULTI && w.step + 1 < P.n_steps) {  // the next step of the launch
         w.step++;
         w.epoch++;
         w.iop = P.op_begin;
@@ -2097,6 +2098,7 @@ MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs
 // launch's ops (all its steps) has been issued, then wait for the last copies.
 // The consumer's stream state stays in registers; the producer keeps its own
 // per-step attention layout (it may be a step ahead of its consumer).
+template <bool MULTI>
 MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane, int *prefix, int *nch) {
   static_assert(kFeeds == 1, "one consumer per producer");
   Warp mine = feeds[first];
@@ -2107,7 +2109,7 @@ MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane, i
   uint64_t t_idle = 0;
   for (int it = 0;; ++it) {
     bool progress = false, all_done = true;
-    if (!mine.done_issue && !mine.failed) progress = feed_more(mine);
+    if (!mine.done_issue && !mine.failed) progress = feed_more<MULTI>(mine);
     all_done = mine.done_issue || mine.failed;
     if (all_done) break;
     int stop = 0;
@@ -2138,7 +2140,9 @@ MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane, i
   __syncwarp();
 }
 
-template <int MMAX, bool XS>
+// MULTI: several steps per launch (P.n_steps); the single-step instance keeps
+// the step index a compile-time zero.
+template <int MMAX, bool XS, bool MULTI>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ int s_attn_prefix[kWarpsPerCta][kMaxRows + 1];  // each warp's, for its step
@@ -2234,16 +2238,22 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   }
 
   if (!consumer) {
-    producer_run(P, s_feed, (wib - kConsumers) * kFeeds, w.lane, s_attn_prefix[wib], s_attn_nch[wib]);
+    producer_run<MULTI>(P, s_feed, (wib - kConsumers) * kFeeds, w.lane, s_attn_prefix[wib], s_attn_nch[wib]);
     return;
   }
 
   uint32_t stage_seq = 0;
   AttnShared ash{xs, xs + kConsumers * kQvp * P.hd, s_attn_ml, &s_stage, &stage_seq};
-  for (; w.step < P.n_steps && !w.failed; ++w.step, ++w.epoch) {
+  const uint32_t epoch0 = w.epoch;
+  const int n_steps = MULTI ? P.n_steps : 1;
+  for (int step = 0; step < n_steps && !w.failed; ++step) {
+  if constexpr (MULTI) {
+    w.step = step;
+    w.epoch = epoch0 + static_cast<uint32_t>(step);
+  }
   attn_layout(P, w.step, w.attn_prefix, w.attn_nch, w.lane);
   // a later step embeds the previous step's argmax: wait for its publication
-  if (w.step > 0 && !wait_counter(w, P.epoch, w.epoch - 1u, P.op_begin)) break;
+  if (MULTI && step > 0 && !wait_counter(w, P.epoch, w.epoch - 1u, P.op_begin)) break;
   float am_val = -INFINITY;
   int am_idx = 0x7fffffff;
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {
@@ -2316,41 +2326,53 @@ size_t step_smem_bytes(int n_ops, int xs_floats, int mmax) {
 bool kernel_stages_x(int mmax) { return mmax == 1; }
 #endif
 
-template <int MMAX, bool XS>
+template <int MMAX, bool XS, bool MULTI>
 static const void *kernel_ptr() {
-  return reinterpret_cast<const void *>(&mk_step_kernel<MMAX, XS>);
+  return reinterpret_cast<const void *>(&mk_step_kernel<MMAX, XS, MULTI>);
 }
 
 // Batch 1 stages its activation row in shared memory; more rows read it via L1.
-static const void *kernel_for(int mmax) {
+static const void *kernel_for(int mmax, bool multi) {
+  if (multi) {
+    switch (mmax) {
+      case 1: return kernel_ptr<1, true, true>();
+      case 2: return kernel_ptr<2, false, true>();
+      case 4: return kernel_ptr<4, false, true>();
+      default: return kernel_ptr<8, false, true>();
+    }
+  }
   switch (mmax) {
-    case 1: return kernel_ptr<1, true>();
-    case 2: return kernel_ptr<2, false>();
-    case 4: return kernel_ptr<4, false>();
-    default: return kernel_ptr<8, false>();
+    case 1: return kernel_ptr<1, true, false>();
+    case 2: return kernel_ptr<2, false, false>();
+    case 4: return kernel_ptr<4, false, false>();
+    default: return kernel_ptr<8, false, false>();
   }
 }
 
 int MK_ENTRY(max_cta_per_sm)(int mmax, size_t smem) {
-  const void *k = kernel_for(mmax);
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-    return -1;
-  // Ask for the smallest shared-memory carve-out that fits, leaving the rest of
-  // the SM's unified memory to L1 (activations are re-read through it by every warp).
-  int max_sm = 0, dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&max_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-  if (max_sm > 0) {
-    const int pct = static_cast<int>((smem * 100 + max_sm - 1) / max_sm);
-    cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, pct > 100 ? 100 : pct);
+  int n_min = 1 << 30;
+  for (int multi = 0; multi < 2; ++multi) {  // both forms, single- and multi-step
+    const void *k = kernel_for(mmax, multi != 0);
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+      return -1;
+    // Ask for the smallest shared-memory carve-out that fits, leaving the rest of
+    // the SM's unified memory to L1 (activations are re-read through it by every warp).
+    int max_sm = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&max_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (max_sm > 0) {
+      const int pct = static_cast<int>((smem * 100 + max_sm - 1) / max_sm);
+      cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, pct > 100 ? 100 : pct);
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) != cudaSuccess) return -1;
+    n_min = n < n_min ? n : n_min;
   }
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) != cudaSuccess) return -1;
-  return n;
+  return n_min;
 }
 
 int MK_ENTRY(launch_step)(const Params &p, int mmax, bool cooperative, cudaStream_t stream) {
-  const void *k = kernel_for(mmax);
+  const void *k = kernel_for(mmax, p.n_steps > 1);
   const size_t smem = step_smem_bytes(p.n_ops, p.xs_floats, mmax);
   void *args[] = {const_cast<Params *>(&p)};
   cudaError_t e;
