@@ -236,7 +236,7 @@ def build_workload(kind, B, device):
     if kind == "small":
         wl = workload("small") if B == 1 else workload("small_batch", B)
     else:
-        wl = workload(kind, B) if kind in ("large", "profile") else workload(kind)
+        wl = workload(kind, B) if kind in ("large", "profile", "dense") else workload(kind)
     m = wl.model
     t0 = time.perf_counter()
     w = make_weights(m, wl.seed, device)
@@ -417,6 +417,34 @@ def measure_multi_step(dec, m, k, v, B, ctx, n_steps, device):
             "path": "mk_decode_steps: one persistent launch, argmax fed back on the device"}
 
 
+def measure_dense(device, steps=20, warmup=3):
+    """The dense-decoder variant at batch 1 (no router; a 14336-wide SwiGLU FFN
+    per layer on the large model's attention): tokens/s and HBM bandwidth."""
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+    from synthetic import make_kv_cache, make_weights, workload
+
+    wl = workload("dense", 1)
+    m, B, T = wl.model, wl.batch, wl.tokens_per_step
+    w = make_weights(m, wl.seed, device)
+    ctx = [wl.context] * B
+    cap = (wl.context + (steps + warmup + 2) * T + 63) // 64 * 64
+    k, v = make_kv_cache(m, B, cap, wl.seed, device)
+    dec = mk.Decoder(m, w, max_rows=B * T, max_seqs=B, kv_capacity=cap)
+    total, per, st = time_steps(dec, m, k, v, B, T, ctx, steps, warmup, device)
+    lens = [c + (warmup + steps // 2) * T + T for c in ctx]
+    by = step_bytes(m, B, T, lens, 0)
+    ms = total / steps
+    dec.close()
+    del w, k, v
+    torch.cuda.empty_cache()
+    return {"workload": f"{wl.name} ({m.name} model: {m.n_layers} layers, d {m.d_model}, FFN {m.shared_ffn}, "
+                        f"no router)", "ms_per_step": round(ms, 4), "tok_s": round(B * T / (ms / 1e3), 1),
+            "hbm_gbs": round(by / (ms / 1e3) / 1e9, 1), "bytes_per_step": int(by),
+            "launches_per_step": st.kernel_launches // steps}
+
+
 def measure_verify_wide(device, steps=10, warmup=3):
     """The 56-row speculative-verify block (8 sequences x 7 rows, the small
     model) through the wide-block tensor-core path."""
@@ -522,9 +550,10 @@ def run_mine(args):
     if args.sweep and T == 1:
         multi = measure_multi_step(dec, m, k, v, B, ctx, 32, device)
 
-    verify56 = None
+    verify56 = dense = None
     if args.sweep and ws == 1 and args.workload == "large":
         verify56 = measure_verify_wide(device)
+        dense = measure_dense(device)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -568,6 +597,8 @@ def run_mine(args):
             line["multi_step"] = multi
         if verify56 is not None:
             line["verify_56"] = verify56
+        if dense is not None:
+            line["dense"] = dense
         print(json.dumps(line), flush=True)
     dec.close()
     import torch.distributed as dist
@@ -622,7 +653,8 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
-    ap.add_argument("--workload", default="large", choices=["large", "small", "tiny", "profile"])
+    ap.add_argument("--workload", default="large",
+                    choices=["large", "small", "tiny", "profile", "dense", "tiny_dense"])
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--variant", default="megakernel",
                     choices=["megakernel", "multikernel", "multikernel_graph"])

@@ -229,10 +229,19 @@ MK_API int mk_validate_desc(const mk_model_desc *d) {
     return fail(MK_ERR_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
   if (d->head_dim != 64 && d->head_dim != 128)
     return fail(MK_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", d->head_dim);
-  if (d->n_experts < 1 || d->n_experts > kMaxExperts)
-    return fail(MK_ERR_UNSUPPORTED, "n_experts must be in [1, %d]", kMaxExperts);
-  if (d->top_k < 1 || d->top_k > d->n_experts || d->top_k > kMaxTopK)
-    return fail(MK_ERR_ARG, "top_k must be in [1, min(%d, n_experts)]", kMaxTopK);
+  if (d->n_experts == 0) {
+    // a dense decoder: one SwiGLU FFN per layer, given as the shared expert;
+    // no router, no routed experts
+    if (d->top_k != 0 || d->shared_ffn < 16)
+      return fail(MK_ERR_ARG, "a dense model (n_experts = 0) needs top_k = 0 and shared_ffn > 0");
+    if (d->max_rows > kMaxRows)
+      return fail(MK_ERR_UNSUPPORTED, "a dense model serves at most %d rows per step", kMaxRows);
+  } else {
+    if (d->n_experts < 1 || d->n_experts > kMaxExperts)
+      return fail(MK_ERR_UNSUPPORTED, "n_experts must be in [0, %d]", kMaxExperts);
+    if (d->top_k < 1 || d->top_k > d->n_experts || d->top_k > kMaxTopK)
+      return fail(MK_ERR_ARG, "top_k must be in [1, min(%d, n_experts)]", kMaxTopK);
+  }
   if (d->expert_ffn < 16 || d->expert_ffn % 16) return fail(MK_ERR_ARG, "expert_ffn must be a positive multiple of 16");
   if (d->shared_ffn < 0 || d->shared_ffn % 16) return fail(MK_ERR_ARG, "shared_ffn must be 0 or a multiple of 16");
   if (d->vocab < 1) return fail(MK_ERR_ARG, "vocab must be >= 1");
@@ -337,8 +346,8 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   const mk_model_desc &d = *desc;
   for (int l = 0; l < d.n_layers; ++l) {
     const mk_layer_weights &lw = w->layers[l];
-    if (!lw.attn_norm || !lw.wqkv || !lw.wo || !lw.ffn_norm || !lw.router || !lw.w_gate || !lw.w_up ||
-        !lw.w_down)
+    if (!lw.attn_norm || !lw.wqkv || !lw.wo || !lw.ffn_norm ||
+        (d.n_experts > 0 && (!lw.router || !lw.w_gate || !lw.w_up || !lw.w_down)))
       return fail(MK_ERR_ARG, "layer %d: a required weight pointer is NULL", l);
     if (d.shared_ffn > 0 && (!lw.ws_gate || !lw.ws_up || !lw.ws_down))
       return fail(MK_ERR_ARG, "layer %d: shared expert weights are NULL but shared_ffn > 0", l);
@@ -453,10 +462,12 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     const uint64_t E = d.n_experts, F = d.expert_ffn, Fs = d.shared_ffn;
     rc = enc(b + MAP_WQKV, lw.wqkv, QKVW, D);
     if (!rc) rc = enc(b + MAP_WO, lw.wo, D, (uint64_t)d.n_q_heads * d.head_dim);
-    if (!rc) rc = enc(b + MAP_ROUTER, lw.router, E, D);
-    if (!rc) rc = enc(b + MAP_WGATE, lw.w_gate, E * F, D);
-    if (!rc) rc = enc(b + MAP_WUP, lw.w_up, E * F, D);
-    if (!rc) rc = enc(b + MAP_WDOWN, lw.w_down, E * D, F);
+    if (E > 0) {  // a dense model has no router and no routed experts
+      if (!rc) rc = enc(b + MAP_ROUTER, lw.router, E, D);
+      if (!rc) rc = enc(b + MAP_WGATE, lw.w_gate, E * F, D);
+      if (!rc) rc = enc(b + MAP_WUP, lw.w_up, E * F, D);
+      if (!rc) rc = enc(b + MAP_WDOWN, lw.w_down, E * D, F);
+    }
     if (!rc && Fs > 0) rc = enc(b + MAP_WSGATE, lw.ws_gate, Fs, D);
     if (!rc && Fs > 0) rc = enc(b + MAP_WSUP, lw.ws_up, Fs, D);
     if (!rc && Fs > 0) rc = enc(b + MAP_WSDOWN, lw.ws_down, D, Fs);

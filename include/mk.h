@@ -71,7 +71,11 @@ extern "C" {
  * n_q_heads % n_kv_heads == 0; d_model, n_q_heads*head_dim multiples of 8;
  * expert_ffn and shared_ffn multiples of 16 (shared_ffn may be 0 = no shared
  * expert); n_experts <= 256; top_k <= min(16, n_experts);
- * 1 <= max_rows <= 8; 1 <= max_seqs <= max_rows. */
+ * 1 <= max_rows <= 64; 1 <= max_seqs <= max_rows.
+ * A dense decoder (one SwiGLU FFN per layer, no router) is n_experts = 0 and
+ * top_k = 0 with the FFN given as the shared expert (shared_ffn > 0, weights
+ * ws_gate/ws_up/ws_down; router and w_gate/w_up/w_down may be NULL and
+ * expert_ffn is ignored beyond its check); it serves max_rows <= 8. */
 typedef struct mk_model_desc {
   int32_t n_layers, d_model, n_q_heads, n_kv_heads, head_dim;
   int32_t n_experts, top_k, expert_ffn, shared_ffn, vocab;

@@ -84,11 +84,19 @@ LARGE = ModelConfig("large", 16, 4096, 32, 8, 128, 128, 8, 1536, 1536, 64000, si
 # weights): the same per-op shapes, small enough for a full profiler capture.
 PROFILE = ModelConfig("profile", 2, 4096, 32, 8, 128, 16, 8, 1536, 1536, 64000, sigma=0.015)
 
-MODELS = {m.name: m for m in (TINY, SMALL, LARGE, PROFILE)}
+# Dense decoders (no router; one SwiGLU FFN per layer, held as the shared
+# expert): the tiny model's shapes, and the large model's attention, vocab and
+# a Llama-3-8B-sized FFN (about 7.5 GB read per step, like the large MoE's
+# active bytes).
+TINY_DENSE = ModelConfig("tiny_dense", 2, 256, 4, 2, 64, 0, 0, 16, 512, 1024)
+DENSE = ModelConfig("dense", 16, 4096, 32, 8, 128, 0, 0, 16, 14336, 64000, sigma=0.015)
+
+MODELS = {m.name: m for m in (TINY, SMALL, LARGE, PROFILE, TINY_DENSE, DENSE)}
 
 
 def workload(kind: str, batch: int = 1) -> Workload:
-    """The named workloads: tiny / small / small_batch / verify / large / profile."""
+    """The named workloads: tiny / small / small_batch / verify / large / profile,
+    and the dense decoders tiny_dense / dense."""
     if kind == "tiny":
         return Workload("tiny_bs1", TINY, 1, 1, 127, steps=16, seed=0)
     if kind == "small":
@@ -101,6 +109,10 @@ def workload(kind: str, batch: int = 1) -> Workload:
         return Workload(f"large_bs{batch}", LARGE, batch, 1, 4095, steps=32, seed=4)
     if kind == "profile":
         return Workload(f"profile_bs{batch}", PROFILE, batch, 1, 4095, steps=8, seed=5)
+    if kind == "tiny_dense":
+        return Workload("tiny_dense_bs1", TINY_DENSE, 1, 1, 127, steps=16, seed=6)
+    if kind == "dense":
+        return Workload(f"dense_bs{batch}", DENSE, batch, 1, 4095, steps=32, seed=7)
     raise ValueError(f"unknown workload {kind!r}")
 
 
