@@ -471,7 +471,7 @@ def measure_verify_wide(device, steps=10, warmup=3):
     return {"workload": f"{wl.name} ({m.name} model, {B * T} rows per step)", "ms_per_step": round(ms, 4),
             "rows_per_s": round(B * T / (ms / 1e3), 1), "hbm_gbs": round(by / (ms / 1e3) / 1e9, 1),
             "expert_union_per_layer": round(union, 1), "launches_per_step": st.kernel_launches // steps,
-            "path": "tensor-core launch sequence (blocks above 8 rows)"}
+            "path": "tensor-core launch sequence (blocks above 8 rows), replayed as a CUDA graph"}
 
 
 def run_mine(args):

@@ -173,6 +173,7 @@ Sizes scratch_sizes(const mk_model_desc &d, int n_sm) {
 struct GraphEntry {
   uint64_t key[12];
   cudaGraphExec_t exec;
+  int launches;  // kernels per replay
 };
 
 struct mk_handle {
@@ -628,9 +629,52 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
   s.pair_slot = h->w_pair_slot;
   s.xhi = h->w_xhi; s.xlo = h->w_xlo; s.ghi = h->w_ghi; s.glo = h->w_glo; s.ahi = h->w_ahi; s.alo = h->w_alo;
   s.shi = h->w_shi; s.slo = h->w_slo;
+  // The launch sequence is recorded once per (shape, buffers) into a CUDA graph
+  // and replayed: a graph launch issues the ~300 kernels without a host call
+  // each.  Graphs live in the handle's cache next to the multi-kernel ones.
+  const uint64_t key[12] = {(uint64_t)B | (0x57ull << 56),  // wide-block entries
+                            (uint64_t)T,
+                            (uint64_t)(uintptr_t)tokens,
+                            (uint64_t)(uintptr_t)positions,
+                            (uint64_t)(uintptr_t)s.logits,
+                            (uint64_t)(uintptr_t)argmax,
+                            (uint64_t)(uintptr_t)kv.k,
+                            (uint64_t)(uintptr_t)kv.v,
+                            (uint64_t)(uintptr_t)h->dbg_hidden,
+                            (uint64_t)(uintptr_t)h->dbg_ids ^ (uint64_t)(uintptr_t)h->dbg_w,
+                            0,
+                            0};
+  for (auto &g : h->graphs)
+    if (std::memcmp(g.key, key, sizeof key) == 0) {
+      CUDA_TRY(cudaGraphLaunch(g.exec, stream));
+      h->stats.kernel_launches += g.launches;
+      h->stats.steps += 1;
+      return MK_OK;
+    }
   int launches = 0;
-  cudaError_t e = wide_step(s, stream, &launches);
-  if (e != cudaSuccess) return fail(MK_ERR_LAUNCH, "wide-block launch failed: %s", cudaGetErrorString(e));
+  CUDA_TRY(cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal));
+  cudaError_t e = wide_step(s, h->capture_stream, &launches);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(h->capture_stream, &graph);
+  if (e != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    return fail(MK_ERR_LAUNCH, "wide-block launch failed: %s", cudaGetErrorString(e));
+  }
+  if (ce != cudaSuccess) return fail(MK_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(ce));
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) return fail(MK_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(e));
+  if (h->graphs.size() >= 8) {
+    cudaGraphExecDestroy(h->graphs.front().exec);
+    h->graphs.erase(h->graphs.begin());
+  }
+  GraphEntry ge;
+  std::memcpy(ge.key, key, sizeof key);
+  ge.exec = exec;
+  ge.launches = launches;
+  h->graphs.push_back(ge);
+  CUDA_TRY(cudaGraphLaunch(exec, stream));
   h->stats.kernel_launches += launches;
   h->stats.steps += 1;
   return MK_OK;
@@ -682,6 +726,7 @@ static int run_step(mk_handle *h, const int32_t *tokens, const int32_t *position
       GraphEntry ge;
       std::memcpy(ge.key, key, sizeof key);
       ge.exec = exec;
+      ge.launches = pl.n_ops;
       h->graphs.push_back(ge);
       h->stats.kernel_launches -= pl.n_ops;  // counted again below on replay
     }
