@@ -445,15 +445,16 @@ def measure_dense(device, steps=20, warmup=3):
             "launches_per_step": st.kernel_launches // steps}
 
 
-def measure_verify_wide(device, steps=10, warmup=3):
-    """The 56-row speculative-verify block (8 sequences x 7 rows, the small
-    model) through the wide-block tensor-core path."""
+def measure_verify_wide(device, steps=10, warmup=3, batch=8):
+    """A speculative-verify block of 7 rows per sequence on the small model:
+    8 sequences (56 rows, the wide-block tensor-core path) or 1 (7 rows, the
+    megakernel)."""
     import torch
 
     import decode_megakernel_06_b200 as mk
     from synthetic import make_kv_cache, make_weights, workload
 
-    wl = workload("verify", 8)
+    wl = workload("verify", batch)
     m, B, T = wl.model, wl.batch, wl.tokens_per_step
     w = make_weights(m, wl.seed, device)
     ctx = [wl.context] * B
@@ -471,7 +472,8 @@ def measure_verify_wide(device, steps=10, warmup=3):
     return {"workload": f"{wl.name} ({m.name} model, {B * T} rows per step)", "ms_per_step": round(ms, 4),
             "rows_per_s": round(B * T / (ms / 1e3), 1), "hbm_gbs": round(by / (ms / 1e3) / 1e9, 1),
             "expert_union_per_layer": round(union, 1), "launches_per_step": st.kernel_launches // steps,
-            "path": "tensor-core launch sequence (blocks above 8 rows), replayed as a CUDA graph"}
+            "path": ("tensor-core launch sequence (blocks above 8 rows), replayed as a CUDA graph"
+                     if B * T > 8 else "megakernel")}
 
 
 def run_mine(args):
@@ -550,9 +552,10 @@ def run_mine(args):
     if args.sweep and T == 1:
         multi = measure_multi_step(dec, m, k, v, B, ctx, 32, device)
 
-    verify56 = dense = None
+    verify56 = verify7 = dense = None
     if args.sweep and ws == 1 and args.workload == "large":
         verify56 = measure_verify_wide(device)
+        verify7 = measure_verify_wide(device, batch=1)
         dense = measure_dense(device)
 
     cpu = None
@@ -597,6 +600,8 @@ def run_mine(args):
             line["multi_step"] = multi
         if verify56 is not None:
             line["verify_56"] = verify56
+        if verify7 is not None:
+            line["verify_7"] = verify7
         if dense is not None:
             line["dense"] = dense
         print(json.dumps(line), flush=True)

@@ -557,23 +557,19 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.attn_norm), d, s.eps, s.xhi,
                                        s.xlo, ldx);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wqkv), 0, W3, d, s.xhi, s.xlo, ldx, nullptr, nullptr, 1, M,
                   s.qkv, W3, 0, st));
     wide_kv_append<<<dim3(M, s.Hkv), 128, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, s.rope, s.kc,
                                                    s.vc, s.Bmax, s.cap, l);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     wide_attention<<<dim3(M, s.Hq), kAttnWarps * 32, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd,
                                                               s.rope, s.kc, s.vc, s.Bmax, s.cap, l, s.o);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     wide_split<<<M, 256, 0, st>>>(s.o, HD, HD, s.xhi, s.xlo, ldx);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), 0, d, HD, s.xhi, s.xlo, ldx, nullptr, nullptr, 1, M,
                   s.h, d, 1, st));
@@ -581,7 +577,6 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.ffn_norm), d, s.eps, s.xhi, s.xlo,
                                        ldx);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), 0, E, d, s.xhi, s.xlo, ldx, nullptr, nullptr, 1, M,
                   s.rlog, E, 0, st));
@@ -589,16 +584,13 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     float *dbg_w = s.dbg_w ? s.dbg_w + static_cast<long long>(l) * s.max_rows * K : nullptr;
     wide_topk<<<M, 32, 0, st>>>(s.rlog, E, K, s.sel_e, s.sel_w, dbg_ids, dbg_w);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     wide_expert_lists<<<1, 256, 0, st>>>(s.sel_e, M, K, E, s.count, s.off, s.pair_row, s.pair_slot, s.stats);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     // routed experts: gate and up over each expert's rows, SwiGLU, down
     wide_gather<<<M * K, 256, 0, st>>>(s.xhi, s.xlo, ldx, s.pair_row, d, s.ghi, s.glo);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), static_cast<long long>(F) * d, F, d, s.ghi, s.glo,
                   ldx, s.off, s.count, E, M * K, s.gu, 2 * F, 0, st));
@@ -606,7 +598,6 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
                   ldx, s.off, s.count, E, M * K, s.gu + F, 2 * F, 0, st));
     wide_swiglu<<<M * K, 256, 0, st>>>(s.gu, F, s.ahi, s.alo, s.lda);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), static_cast<long long>(d) * F, d, F, s.ahi, s.alo,
                   s.lda, s.off, s.count, E, M * K, s.yd, d, 0, st));
@@ -618,15 +609,13 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
                     M, s.gs + Fs, 2 * Fs, 0, st));
       wide_swiglu<<<M, 256, 0, st>>>(s.gs, Fs, s.shi, s.slo, s.lda);
       WIDE_TRY(cudaGetLastError());
-  ++n;
-    ++n;
+      ++n;
       WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), 0, d, Fs, s.shi, s.slo, s.lda, nullptr, nullptr,
                     1, M, s.ys, d, 0, st));
     }
     float *dbg = s.dbg_hidden ? s.dbg_hidden + static_cast<long long>(l + 1) * s.max_rows * d : nullptr;
     wide_combine<<<M, 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr, dbg);
     WIDE_TRY(cudaGetLastError());
-  ++n;
     ++n;
   }
   // final norm, lm_head, argmax
