@@ -99,6 +99,7 @@ def lib():
         "mk_create": (i32, [ctypes.POINTER(mk_model_desc), ctypes.POINTER(mk_weights), ctypes.POINTER(vp)]),
         "mk_decode_step": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
         "mk_decode_steps": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
+        "mk_verify_steps": (i32, [vp, vp, vp, i32, i32, i32, vp, i32, mk_kv_cache, vp, vp, vp, vp]),
         "mk_decode_step_host": (i32, [vp, _I32P, _I32P, i32, i32, mk_kv_cache, vp, _I32P, vp]),
         "mk_decode_step_static": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
         "mk_get_device_status": (i32, [vp, vp]),
@@ -160,6 +161,14 @@ def mk_decode_steps(h, tokens: int, positions: int, B: int, n_steps: int, kv: mk
                     out_logits: int, out_tokens: int, stream: int) -> int:
     """n_steps greedy steps in one launch (see include/mk.h)."""
     return lib().mk_decode_steps(h, tokens, positions, B, n_steps, kv, out_logits, out_tokens, stream)
+
+
+def mk_verify_steps(h, tokens: int, positions: int, B: int, T: int, n_steps: int, drafts: int,
+                    draft_len: int, kv: mk_kv_cache, out_logits: int, out_tokens: int,
+                    out_accepted: int, stream: int) -> int:
+    """n_steps speculative-verify steps in one launch (see include/mk.h)."""
+    return lib().mk_verify_steps(h, tokens, positions, B, T, n_steps, drafts, draft_len, kv, out_logits,
+                                 out_tokens, out_accepted, stream)
 
 
 def mk_decode_step(h, tokens: int, positions: int, B: int, T: int, kv: mk_kv_cache,
@@ -297,6 +306,17 @@ class Decoder:
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_steps(self.h, tokens.data_ptr(), positions.data_ptr(), B, n_steps, kv,
                                _ptr(logits), out_tokens.data_ptr(), s.cuda_stream)
+
+    def verify_steps(self, tokens, positions, B: int, T: int, n_steps: int, drafts, k_cache, v_cache,
+                     logits, out_tokens, out_accepted, stream=None) -> int:
+        """Enqueue n_steps verify blocks of T rows as one launch; drafts is int32
+        [B, draft_len] on the device, out_tokens [n_steps, B*T], out_accepted
+        [n_steps, B].  Returns the launch status code."""
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
+        return mk_verify_steps(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, n_steps,
+                               drafts.data_ptr(), drafts.shape[-1], kv, _ptr(logits),
+                               out_tokens.data_ptr(), out_accepted.data_ptr(), s.cuda_stream)
 
     def step_static(self, tokens, positions, B: int, T: int, k_cache, v_cache, logits, argmax,
                     stream=None) -> int:

@@ -208,6 +208,8 @@ struct mk_handle {
   int last_error_op;
   mk_stats stats;
   std::vector<GraphEntry> graphs;
+  int *vbuf = nullptr;   // verify launches: block positions, block tokens, argmax per step
+  size_t vbuf_ints = 0;
   cudaStream_t capture_stream;
   // wide blocks (more than kMaxRows rows): scratch of the launch sequence
   int wide_ldx, wide_lda;
@@ -746,6 +748,48 @@ MK_API int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *po
                           int32_t T, mk_kv_cache kv, float *out_logits, int32_t *out_argmax,
                           void *stream) {
   return run_step(h, tokens, positions, B, T, kv, out_logits, out_argmax, static_cast<cudaStream_t>(stream));
+}
+
+MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
+                           int32_t T, int32_t n_steps, const int32_t *drafts, int32_t draft_len,
+                           mk_kv_cache kv, float *out_logits, int32_t *out_tokens, int32_t *out_accepted,
+                           void *stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (n_steps < 1) return fail(MK_ERR_ARG, "n_steps must be >= 1");
+  if (T < 2) return fail(MK_ERR_ARG, "a verify block has T >= 2 rows");
+  if ((long long)B * T > kMaxRows)
+    return fail(MK_ERR_UNSUPPORTED, "a verify launch serves at most %d rows per step", kMaxRows);
+  if (!drafts || !out_tokens || !out_accepted) return fail(MK_ERR_ARG, "drafts, out_tokens and out_accepted are required");
+  if ((long long)draft_len < (long long)n_steps * T)
+    return fail(MK_ERR_ARG, "draft_len=%d is shorter than n_steps * T = %lld", draft_len, (long long)n_steps * T);
+  if ((long long)n_steps * T > h->desc.kv_capacity) return fail(MK_ERR_CAPACITY, "n_steps * T exceeds kv_capacity");
+  const size_t need = (size_t)(n_steps + 1) * B + (size_t)(n_steps + 1) * B * T + (size_t)n_steps * B * T;
+  if (need > h->vbuf_ints) {
+    void *nb = nullptr;
+    int rc = halloc(h, &nb, need * sizeof(int32_t));
+    if (rc) return rc;
+    h->vbuf = static_cast<int *>(nb);
+    h->vbuf_ints = need;
+  }
+  int *vpos = h->vbuf, *vtok = vpos + (size_t)(n_steps + 1) * B, *am = vtok + (size_t)(n_steps + 1) * B * T;
+  Params p;
+  Plan pl;
+  int rc = fill_params(h, tokens, positions, B, T, kv, out_logits, am, p, pl);
+  if (rc) return rc;
+  p.n_steps = n_steps;
+  p.vpos = vpos;
+  p.vtok = vtok;
+  p.drafts = drafts;
+  p.draft_len = draft_len;
+  p.out_tokens = out_tokens;
+  p.out_accepted = out_accepted;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUDA_TRY(cudaMemcpyAsync(vpos, positions, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, s));
+  int e = launch_step_any(p, pl.mmax, true, s);
+  if (e) return fail(MK_ERR_LAUNCH, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
+  h->stats.kernel_launches += 1;
+  h->stats.steps += n_steps;
+  return MK_OK;
 }
 
 MK_API int mk_decode_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,

@@ -99,9 +99,19 @@ struct alignas(64) Params {
   int L, d, Hq, Hkv, hd, E, topk, F, Fs, V, Bmax, cap;
   float eps;
   int B, T, M, max_rows;
-  int n_steps;         // greedy steps in this launch (T = 1 when > 1); step s embeds
-                       // tokens (s = 0) or argmax[s-1], appends at positions[b] + s and
-                       // writes its argmax to argmax[s * M ..]
+  int n_steps;         // steps in this launch; step s writes its argmax to argmax[s * M ..].
+                       // Greedy (T = 1, vpos null): step s embeds tokens (s = 0) or
+                       // argmax[s-1] and appends at positions[b] + s.
+  // Speculative verify over the steps (vpos set): step s scores the block whose
+  // start positions are vpos[s][b] and whose tokens are tokens (s = 0) or
+  // vtok[s]; its final-argmax warp accepts the longest prefix of drafts its
+  // argmax confirms plus one token, and writes the next block from it.
+  int *vpos;                             // [n_steps + 1][B]; row 0 set by the host
+  int *vtok;                             // [n_steps + 1][M]
+  const int *drafts;                     // [B][draft_len]: token proposed for position positions[b] + j
+  int draft_len;
+  int *out_tokens;                       // [n_steps][M]: accepted tokens, -1 past the count
+  int *out_accepted;                     // [n_steps][B]
   // grid / schedule
   int n_cta, n_warps, op_begin, op_end, n_ops;
   int n_hb;            // residual row blocks (ceil(d / kRows))

@@ -293,6 +293,7 @@ struct Warp {
   int *attn_prefix;        // this warp's: first item of each sequence, [kMaxRows + 1]
   int *attn_nch;           // this warp's: KV chunks of each sequence, [kMaxRows]
   int step;                // the step (of a multi-step launch) this warp is in
+  int lstep;               // the step its attention layout was computed for
   // consumer side: bit s = parity of the next completion of full[s]
   uint32_t phase;
   int cslot;
@@ -582,8 +583,11 @@ struct AttnItem {
   int pos0, npos, ntiles;  // this warp's positions: [pos0, pos0 + npos), in tiles
 };
 
-// Cache index of sequence b's first new row in step `step` of the launch.
-MK_INLINE int seq_pos(const Params &P, int b, int step) { return __ldg(&P.positions[b]) + step * P.T; }
+// Cache index of sequence b's first new row in step `step` of the launch:
+// fixed strides for greedy steps, the accepted length so far for verify steps.
+MK_INLINE int seq_pos(const Params &P, int b, int step) {
+  return P.vpos ? __ldcg(&P.vpos[step * P.B + b]) : __ldg(&P.positions[b]) + step * P.T;
+}
 
 // Attention items of one step: per sequence its KV chunks and first item
 // (lane 0 computes, the warp reads).
@@ -784,7 +788,6 @@ MK_INLINE bool feed_more(Warp &w) {
         w.epoch++;
         w.iop = P.op_begin;
         w.iop_init = false;
-        attn_layout(P, w.step, w.attn_prefix, w.attn_nch, w.lane);
         continue;
       }
       w.done_issue = true;
@@ -797,6 +800,17 @@ MK_INLINE bool feed_more(Warp &w) {
       continue;
     }
     if (!w.iop_init) {
+      if (type == OP_ATTN && w.lstep != w.step) {
+        // a verify step's positions come from the previous step's acceptance:
+        // wait (by polling, like the routing) until that step has published
+        if (P.vpos && w.step > 0) {
+          const uint32_t v = ld_relaxed(P.epoch);
+          if (!__all_sync(0xffffffffu, static_cast<int>(v - (w.epoch - 1u)) >= 0)) break;
+          (void)ld_acquire(P.epoch);
+        }
+        attn_layout(P, w.step, w.attn_prefix, w.attn_nch, w.lane);
+        w.lstep = w.step;
+      }
       if (type == OP_ROUTED_GU || type == OP_DOWN) {
         if (!routing_ready(w, layer)) break;
         if (!route_cache(w, layer)) break;
@@ -1226,7 +1240,8 @@ MK_INLINE void op_embed(Warp &w, bool gained) {
   residual_units(P, w.lane, w.slot, w.nw, 0, gained ? P.norms[0] : nullptr, [&](int m, int row) {
     // step 0: the given tokens (may alias the argmax output); later steps:
     // the previous step's argmax
-    int tok = w.step ? __ldcg(&P.argmax[(w.step - 1) * P.M + m]) : __ldcg(&P.tokens[m]);
+    int tok = w.step == 0 ? __ldcg(&P.tokens[m])
+              : P.vpos ? __ldcg(&P.vtok[w.step * P.M + m]) : __ldcg(&P.argmax[(w.step - 1) * P.M + m]);
     if (tok < 0 || tok >= P.V) tok = 0;  // rejected at kernel start
     return __bfloat162float(P.embed[static_cast<size_t>(tok) * P.d + row]);
   });
@@ -1949,6 +1964,31 @@ __device__ __noinline__ void final_argmax(const Params &P, int lane, uint32_t ep
     if (lane == 0) P.argmax[step * P.M + m] = (bi == 0x7fffffff) ? 0 : bi;
   }
   __syncwarp();
+  if (P.vpos) {
+    // Verify step: sequence b (one lane each) accepts its block's drafts while
+    // each equals the argmax of the row before it, plus one token; the next
+    // block starts after the accepted tokens with the last of them, then the
+    // drafts proposed for the positions that follow.
+    const int T = P.T;
+    const int *am = P.argmax + step * P.M;
+    for (int b = lane; b < P.B; b += 32) {
+      const int base = b * T;
+      const int *blk = step == 0 ? P.tokens + base : P.vtok + step * P.M + base;
+      int a = 1;
+      while (a < T && __ldcg(&blk[a]) == __ldcg(&am[base + a - 1])) ++a;
+      P.out_accepted[step * P.B + b] = a;
+      for (int t = 0; t < T; ++t) P.out_tokens[step * P.M + base + t] = t < a ? __ldcg(&am[base + t]) : -1;
+      const int p_next = __ldcg(&P.vpos[step * P.B + b]) + a, p0 = __ldg(&P.positions[b]);
+      P.vpos[(step + 1) * P.B + b] = p_next;
+      int *nb = P.vtok + (step + 1) * P.M + base;
+      nb[0] = __ldcg(&am[base + a - 1]);
+      for (int t = 1; t < T; ++t) {
+        const int j = p_next - p0 + t;  // < draft_len: n_steps * T <= draft_len is checked by the host
+        nb[t] = j < P.draft_len ? __ldg(&P.drafts[static_cast<size_t>(b) * P.draft_len + j]) : 0;
+      }
+    }
+    __syncwarp();
+  }
   if (lane == 0) {
     __threadfence();
     st_release(P.epoch, epoch);
@@ -2106,6 +2146,7 @@ MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane, i
   mine.attn_prefix = prefix;
   mine.attn_nch = nch;
   attn_layout(P, 0, prefix, nch, lane);
+  mine.lstep = 0;
   uint64_t t_idle = 0;
   for (int it = 0;; ++it) {
     bool progress = false, all_done = true;
@@ -2181,6 +2222,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.attn_prefix = s_attn_prefix[wib];
   w.attn_nch = s_attn_nch[wib];
   w.step = 0;
+  w.lstep = -1;
   w.phase = 0;
   w.cslot = 0;
   w.islot = 0;
@@ -2251,9 +2293,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     w.step = step;
     w.epoch = epoch0 + static_cast<uint32_t>(step);
   }
-  attn_layout(P, w.step, w.attn_prefix, w.attn_nch, w.lane);
-  // a later step embeds the previous step's argmax: wait for its publication
+  // a later step embeds the previous step's argmax (and, verifying, starts
+  // where its acceptance left the sequence): wait for its publication
   if (MULTI && step > 0 && !wait_counter(w, P.epoch, w.epoch - 1u, P.op_begin)) break;
+  attn_layout(P, w.step, w.attn_prefix, w.attn_nch, w.lane);
   float am_val = -INFINITY;
   int am_idx = 0x7fffffff;
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {

@@ -195,6 +195,31 @@ MK_API int mk_decode_steps(mk_handle *h, const int32_t *tokens, const int32_t *p
                            int32_t B, int32_t n_steps, mk_kv_cache kv, float *out_logits,
                            int32_t *out_tokens, void *stream);
 
+/* n_steps speculative-verify steps of B sequences in ONE persistent launch,
+ * with greedy acceptance and rollback on the device.  Step s scores, for each
+ * sequence, a block of T rows at positions p_s .. p_s + T - 1 (p_0 =
+ * positions[b]): row 0 is the last accepted token, rows 1..T-1 the drafts
+ * proposed for the next positions.  Its argmax accepts the longest prefix of
+ * drafts that each equal the argmax of the row before them, plus one token
+ * (a = 1..T tokens: the argmax of rows 0..a-1).  The next block starts at
+ * p_{s+1} = p_s + a with the last accepted token; K/V rows written past the
+ * accepted ones are overwritten by the next block before anything reads them.
+ *   tokens      : device int32 [B*T], the first block (row b*T + t)
+ *   positions   : device int32 [B]; positions[b] + n_steps*T <= kv_capacity
+ *   B, T        : T >= 2, B*T <= min(max_rows, 8)
+ *   drafts      : device int32 [B][draft_len]: drafts[b][j] is the token proposed
+ *                 for cache position positions[b] + j; draft_len >= n_steps*T
+ *   out_logits  : device fp32 [B*T][vocab] of the LAST step, or NULL
+ *   out_tokens  : device int32 [n_steps][B*T]: accepted tokens, -1 after the count
+ *   out_accepted: device int32 [n_steps][B]: tokens accepted per step (1..T)
+ * Always the megakernel.  Asynchronous; device-side errors are read with
+ * mk_get_device_status.  Errors: MK_ERR_ARG, MK_ERR_CAPACITY, MK_ERR_UNSUPPORTED
+ * (more than 8 rows) from the host checks. */
+MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                           int32_t B, int32_t T, int32_t n_steps, const int32_t *drafts,
+                           int32_t draft_len, mk_kv_cache kv, float *out_logits,
+                           int32_t *out_tokens, int32_t *out_accepted, void *stream);
+
 /* The same step driven from HOST buffers: copies tokens [B*T] and positions
  * [B] to the device, runs the step, copies argmax [B*T] back to
  * out_argmax_host, and waits for the stream.  Logits stay on the device
