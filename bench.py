@@ -445,6 +445,64 @@ def measure_dense(device, steps=20, warmup=3):
             "launches_per_step": st.kernel_launches // steps}
 
 
+def measure_verify_loop(device, n_steps=16):
+    """Speculative verify on the device (mk_verify_steps) on the small model:
+    one sequence, blocks of 7 rows (the last accepted token + 6 drafts), n_steps
+    blocks in one launch.  The synthetic drafter proposes the model's own
+    greedy continuation (taken from a greedy multi-step launch first) with
+    every 6th draft replaced, so that each block accepts 5 drafts plus one
+    token: acceptance length 6.  Reports accepted tokens per second."""
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+    from synthetic import make_kv_cache, make_tokens, make_weights, workload
+
+    wl = workload("verify", 1)
+    m, T = wl.model, wl.tokens_per_step
+    acc_len = T - 1
+    w = make_weights(m, wl.seed, device)
+    p0 = wl.context
+    cap = (p0 + (n_steps + 2) * T + 64 + 63) // 64 * 64
+    k, v = make_kv_cache(m, 1, cap, wl.seed, device)
+    dec = mk.Decoder(m, w, max_rows=T, max_seqs=1, kv_capacity=cap)
+    first = make_tokens(m.vocab, 1, 55)[0]
+    ng = n_steps * acc_len + T
+    greedy = torch.empty((ng, 1), dtype=torch.int32, device=device)
+    assert dec.steps(torch.tensor([first], dtype=torch.int32, device=device),
+                     torch.tensor([p0], dtype=torch.int32, device=device), 1, ng, k, v, None, greedy) == 0
+    drafts = torch.empty((1, n_steps * T + T), dtype=torch.int32, device=device)
+    drafts[0, 0] = first
+    drafts[0, 1:ng + 1] = greedy[:, 0]
+    drafts[0, ng + 1:] = 0
+    for s in range(1, n_steps + 2):
+        j = s * acc_len
+        if j < drafts.shape[1]:
+            drafts[0, j] = (drafts[0, j] + 1) % m.vocab
+    blk = drafts[0, :T].clone()
+    pos = torch.tensor([p0], dtype=torch.int32, device=device)
+    out = torch.empty((n_steps, T), dtype=torch.int32, device=device)
+    acc = torch.empty((n_steps, 1), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        assert dec.verify_steps(blk, pos, 1, T, n_steps, drafts, k, v, None, out, acc) == 0
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    assert dec.verify_steps(blk, pos, 1, T, n_steps, drafts, k, v, None, out, acc) == 0
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    ms = e0.elapsed_time(e1)
+    accepted = int(acc.sum().item())
+    dec.close()
+    del w, k, v
+    torch.cuda.empty_cache()
+    return {"workload": f"verify_b1_t{T} ({m.name} model), {n_steps} blocks in one launch",
+            "accepted_tok_s": round(accepted / (ms / 1e3), 1), "mean_acceptance": round(accepted / n_steps, 2),
+            "ms_per_block": round(ms / n_steps, 4), "launches": 1,
+            "drafter": "the model's greedy continuation with every 6th draft replaced"}
+
+
 def measure_verify_wide(device, steps=10, warmup=3, batch=8):
     """A speculative-verify block of 7 rows per sequence on the small model:
     8 sequences (56 rows, the wide-block tensor-core path) or 1 (7 rows, the
@@ -552,10 +610,11 @@ def run_mine(args):
     if args.sweep and T == 1:
         multi = measure_multi_step(dec, m, k, v, B, ctx, 32, device)
 
-    verify56 = verify7 = dense = None
+    verify56 = verify7 = vloop = dense = None
     if args.sweep and ws == 1 and args.workload == "large":
         verify56 = measure_verify_wide(device)
         verify7 = measure_verify_wide(device, batch=1)
+        vloop = measure_verify_loop(device)
         dense = measure_dense(device)
 
     cpu = None
@@ -602,6 +661,8 @@ def run_mine(args):
             line["verify_56"] = verify56
         if verify7 is not None:
             line["verify_7"] = verify7
+        if vloop is not None:
+            line["speculative"] = vloop
         if dense is not None:
             line["dense"] = dense
         print(json.dumps(line), flush=True)
