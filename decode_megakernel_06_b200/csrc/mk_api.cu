@@ -113,7 +113,7 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.attn_ppt = 2048 / d.head_dim;
   p.n_cta = n_sm;
   p.n_warps = n_sm * kConsumers;
-  // Attention items are CTA-wide: each of the 6 compute warps takes attn_chunk KV
+  // Attention items are CTA-wide: each of the compute warps takes attn_chunk KV
   // positions of an item.  About one item per CTA, warp chunks a multiple of
   // the tile height, and at most kMaxChunks items per (sequence, kv head,
   // query group) so that one merge level combines them.
