@@ -225,3 +225,19 @@ def make_tokens(vocab: int, count: int, seed: int, name: str = "tokens") -> List
 def bf16_bits(t: torch.Tensor):
     """Raw uint16 bit pattern of a bf16 tensor as a numpy array (on the host)."""
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")
+
+
+def make_logits(rows: int, vocab: int, sigma: float, seed: int) -> torch.Tensor:
+    """fp32 ``[rows][vocab]`` logits, N(0, sigma), on the host: the sampler's
+    stand-alone input (a decode step's own logits are the other)."""
+    gen = torch.Generator()
+    gen.manual_seed(tensor_seed(seed, "logits", vocab))
+    return torch.randn((rows, vocab), generator=gen, dtype=torch.float32).mul_(sigma)
+
+
+def make_uniforms(count: int, seed: int, name: str = "uniforms") -> List[float]:
+    """``count`` fp64 uniforms in [0, 1): the random numbers a sampler draws,
+    passed to it as inputs."""
+    gen = torch.Generator()
+    gen.manual_seed(tensor_seed(seed, name))
+    return [float(v) for v in torch.rand((count,), generator=gen, dtype=torch.float64)]
