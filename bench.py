@@ -417,6 +417,55 @@ def measure_multi_step(dec, m, k, v, B, ctx, n_steps, device):
             "path": "mk_decode_steps: one persistent launch, argmax fed back on the device"}
 
 
+def measure_sampled(dec, m, k, v, B, ctx, device, steps=20, warmup=3, temperature=1.0, top_p=0.9):
+    """Sampled decode (mk_decode_step_sample: the step, then temperature / top-p
+    sampling of its logits) with each step's token fed to the next on the
+    device, and the sampler alone (mk_sample_top_p) on 1, 8 and 64 rows of
+    this vocabulary.  CUDA events on the launching stream."""
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+    from synthetic import make_logits, make_tokens, make_uniforms
+
+    n = warmup + steps
+    pos = torch.tensor([[ctx[b] + s for b in range(B)] for s in range(n)], dtype=torch.int32, device=device)
+    u = torch.tensor(make_uniforms(n * B, 55), dtype=torch.float64, device=device).view(n, B)
+    bufs = [torch.tensor(make_tokens(m.vocab, B, 56), dtype=torch.int32, device=device),
+            torch.empty(B, dtype=torch.int32, device=device)]
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for s in range(n):
+        if s == warmup:
+            torch.cuda.synchronize()
+            ev[0].record(stream)
+        rc = dec.step_sample(bufs[s % 2], pos[s], B, 1, k, v, None, temperature, top_p, u[s], bufs[(s + 1) % 2])
+        assert rc == 0, mk.mk_last_error()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    ms = ev[0].elapsed_time(ev[1]) / steps
+    alone = {}
+    for rows in (1, 8, 64):
+        lg = make_logits(rows, m.vocab, 1.0, 57).to(device)
+        uu = torch.tensor(make_uniforms(rows, 58), dtype=torch.float64, device=device)
+        out = torch.empty(rows, dtype=torch.int32, device=device)
+        for _ in range(3):
+            assert mk.sample_top_p(lg, temperature, top_p, uu, out) == 0
+        torch.cuda.synchronize()
+        reps = 50
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            mk.sample_top_p(lg, temperature, top_p, uu, out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        alone[f"rows{rows}_us"] = round(e0.elapsed_time(e1) / reps * 1e3, 2)
+    return {"batch": B, "temperature": temperature, "top_p": top_p, "ms_per_step": round(ms, 4),
+            "tok_s": round(B / (ms / 1e3), 1), "launches_per_step": 2,
+            "sampler_alone": alone, "vocab": m.vocab,
+            "path": "mk_decode_step_sample: the megakernel step, then the cluster top-p sampler on its logits"}
+
+
 def measure_dense(device, steps=20, warmup=3):
     """The dense-decoder variant at batch 1 (no router; a 14336-wide SwiGLU FFN
     per layer on the large model's attention): tokens/s and HBM bandwidth."""
@@ -610,6 +659,10 @@ def run_mine(args):
     if args.sweep and T == 1:
         multi = measure_multi_step(dec, m, k, v, B, ctx, 32, device)
 
+    sampled = None
+    if args.sweep and T == 1:
+        sampled = measure_sampled(dec, m, k, v, B, ctx, device)
+
     verify56 = verify7 = vloop = dense = None
     if args.sweep and ws == 1 and args.workload == "large":
         verify56 = measure_verify_wide(device)
@@ -657,6 +710,8 @@ def run_mine(args):
             line["batch_sweep"] = sweep
         if multi is not None:
             line["multi_step"] = multi
+        if sampled is not None:
+            line["sampled"] = sampled
         if verify56 is not None:
             line["verify_56"] = verify56
         if verify7 is not None:

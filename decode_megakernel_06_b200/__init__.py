@@ -102,6 +102,9 @@ def lib():
         "mk_verify_steps": (i32, [vp, vp, vp, i32, i32, i32, vp, i32, mk_kv_cache, vp, vp, vp, vp]),
         "mk_decode_step_host": (i32, [vp, _I32P, _I32P, i32, i32, mk_kv_cache, vp, _I32P, vp]),
         "mk_decode_step_static": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
+        "mk_sample_top_p": (i32, [vp, i32, i32, ctypes.c_float, ctypes.c_float, vp, vp, vp]),
+        "mk_decode_step_sample": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, ctypes.c_float,
+                                        ctypes.c_float, vp, vp, vp]),
         "mk_get_device_status": (i32, [vp, vp]),
         "mk_last_device_error_op": (i32, [vp]),
         "mk_last_error": (ctypes.c_char_p, []),
@@ -186,6 +189,30 @@ def mk_decode_step_static(h, tokens: int, positions: int, B: int, T: int, kv: mk
                           out_logits: int, out_argmax: int, stream: int) -> int:
     return lib().mk_decode_step_static(h, tokens, positions, B, T, kv, out_logits, out_argmax,
                                        stream)
+
+
+def mk_sample_top_p(logits: int, rows: int, vocab: int, temperature: float, top_p: float,
+                    uniforms: int, out_tokens: int, stream: int) -> int:
+    return lib().mk_sample_top_p(logits, rows, vocab, temperature, top_p, uniforms, out_tokens, stream)
+
+
+def mk_decode_step_sample(h, tokens: int, positions: int, B: int, T: int, kv: mk_kv_cache,
+                          out_logits: int, temperature: float, top_p: float, uniforms: int,
+                          out_tokens: int, stream: int) -> int:
+    return lib().mk_decode_step_sample(h, tokens, positions, B, T, kv, out_logits, temperature, top_p,
+                                       uniforms, out_tokens, stream)
+
+
+def sample_top_p(logits, temperature: float, top_p: float, uniforms, out_tokens, stream=None) -> int:
+    """Torch-tensor form of mk_sample_top_p: logits fp32 [rows, vocab], uniforms
+    fp64 [rows] (or None when temperature <= 0), out_tokens int32 [rows], all on
+    the device.  Returns the launch status code."""
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    rows, vocab = logits.shape
+    return mk_sample_top_p(logits.data_ptr(), rows, vocab, temperature, top_p, _ptr(uniforms),
+                           out_tokens.data_ptr(), s.cuda_stream)
 
 
 def mk_get_device_status(h, stream: int) -> int:
@@ -297,6 +324,16 @@ class Decoder:
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_step(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
                               _ptr(logits), argmax.data_ptr(), s.cuda_stream)
+
+    def step_sample(self, tokens, positions, B: int, T: int, k_cache, v_cache, logits, temperature: float,
+                    top_p: float, uniforms, out_tokens, stream=None) -> int:
+        """One step whose next tokens are sampled (temperature / top-p) from its
+        logits with the given fp64 uniforms [B*T].  Returns the launch status code."""
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
+        return mk_decode_step_sample(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
+                                     _ptr(logits), temperature, top_p, _ptr(uniforms),
+                                     out_tokens.data_ptr(), s.cuda_stream)
 
     def steps(self, tokens, positions, B: int, n_steps: int, k_cache, v_cache, logits, out_tokens,
               stream=None) -> int:

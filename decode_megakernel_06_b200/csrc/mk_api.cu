@@ -750,6 +750,42 @@ MK_API int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *po
   return run_step(h, tokens, positions, B, T, kv, out_logits, out_argmax, static_cast<cudaStream_t>(stream));
 }
 
+static int check_sample_args(const void *logits, int32_t rows, int32_t vocab, float temperature,
+                             float top_p, const double *uniforms, const int32_t *out) {
+  if (!logits || !out) return fail(MK_ERR_ARG, "logits and out_tokens must not be NULL");
+  if (rows < 1 || vocab < 1) return fail(MK_ERR_ARG, "rows and vocab must be >= 1 (got %d, %d)", rows, vocab);
+  if (vocab > kSampleMaxVocab)
+    return fail(MK_ERR_UNSUPPORTED, "the sampler takes vocab <= %d (got %d)", kSampleMaxVocab, vocab);
+  if (std::isnan(temperature) || std::isnan(top_p)) return fail(MK_ERR_ARG, "temperature and top_p must not be NaN");
+  if (temperature > 0.0f && !uniforms) return fail(MK_ERR_ARG, "sampling with temperature > 0 needs uniforms");
+  return MK_OK;
+}
+
+MK_API int mk_sample_top_p(const float *logits, int32_t rows, int32_t vocab, float temperature, float top_p,
+                           const double *uniforms, int32_t *out_tokens, void *stream) {
+  int rc = check_sample_args(logits, rows, vocab, temperature, top_p, uniforms, out_tokens);
+  if (rc) return rc;
+  CUDA_TRY(launch_top_p(logits, rows, vocab, temperature, top_p, uniforms, out_tokens,
+                        static_cast<cudaStream_t>(stream)));
+  return MK_OK;
+}
+
+MK_API int mk_decode_step_sample(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
+                                 int32_t T, mk_kv_cache kv, float *out_logits, float temperature, float top_p,
+                                 const double *uniforms, int32_t *out_tokens, void *stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  int rc = check_sample_args(h, B * T, h->desc.vocab, temperature, top_p, uniforms, out_tokens);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *logits = out_logits ? out_logits : h->logits;
+  // the step writes its argmax to out_tokens; the sampler then overwrites it
+  rc = run_step(h, tokens, positions, B, T, kv, logits, out_tokens, s);
+  if (rc) return rc;
+  CUDA_TRY(launch_top_p(logits, B * T, h->desc.vocab, temperature, top_p, uniforms, out_tokens, s));
+  h->stats.kernel_launches += 1;
+  return MK_OK;
+}
+
 MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
                            int32_t T, int32_t n_steps, const int32_t *drafts, int32_t draft_len,
                            mk_kv_cache kv, float *out_logits, int32_t *out_tokens, int32_t *out_accepted,

@@ -203,4 +203,13 @@ size_t step_smem_bytes(int n_ops, int xs_floats, int mmax);
 bool kernel_stages_x(int mmax);
 int max_cta_per_sm(int mmax, size_t smem);
 
+// Temperature / top-p sampler: one cluster of kSampleCluster CTAs per row,
+// each holding a slice of ceil(V / kSampleCluster) logits in shared memory.
+constexpr int kSampleCluster = 8;
+constexpr int kSampleThreads = 512;
+constexpr int kSampleMaxVocab = 131072;  // 64-bit mass sums and shared memory both cover this
+size_t sample_smem_bytes(int slice);
+cudaError_t launch_top_p(const float *logits, int rows, int vocab, float temperature, float top_p,
+                         const double *uniforms, int32_t *out, cudaStream_t stream);
+
 }  // namespace mk

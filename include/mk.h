@@ -220,6 +220,42 @@ MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *p
                            int32_t draft_len, mk_kv_cache kv, float *out_logits,
                            int32_t *out_tokens, int32_t *out_accepted, void *stream);
 
+/* Temperature / top-p (nucleus) sampling of one token per logits row, the
+ * sampler that stands in place of the argmax (tpu-megakernels README, serving
+ * demos: greedy or temperature / top-p generation; the nucleus is Holtzman et
+ * al. 2020, section 3.1).  Per row of V logits l and its uniform u:
+ *   p_i = exp((l_i - max l) / T) in fp64, held as the fixed-point mass
+ *   q_i = round_half_even(p_i * 2^46) (all sums exact integers);
+ *   need = max(1, min(Q, ceil(top_p * Q))), Q = sum q, computed in fp64;
+ *   nucleus = the smallest prefix of the tokens sorted by logit, descending,
+ *   ties by lower id, whose mass reaches need;
+ *   token = the first nucleus id, in id order, whose cumulative mass exceeds
+ *   y = min(S - 1, floor(u * S)), S the nucleus mass.
+ * temperature <= 0 is greedy (the argmax, lowest id on ties; uniforms unread).
+ * top_p <= 0 keeps the most probable token, top_p >= 1 every token.
+ *   logits     : device fp32 [rows][vocab], finite (non-finite rows give an
+ *                unspecified token or none, never an out-of-bounds access)
+ *   rows       : >= 1;  vocab: 1 .. 131072
+ *   uniforms   : device fp64 [rows], each in [0, 1) (values outside are clamped);
+ *                the random numbers are the caller's, so a draw is reproducible
+ *   out_tokens : device int32 [rows]
+ *   stream     : cudaStream_t (NULL = legacy default stream)
+ * One launch: a cluster of 8 CTAs per row.  Asynchronous.  Errors: MK_ERR_ARG
+ * (NULL pointer, rows or vocab < 1, NaN temperature or top_p, uniforms NULL
+ * with temperature > 0), MK_ERR_UNSUPPORTED (vocab > 131072), MK_ERR_CUDA. */
+MK_API int mk_sample_top_p(const float *logits, int32_t rows, int32_t vocab, float temperature,
+                           float top_p, const double *uniforms, int32_t *out_tokens, void *stream);
+
+/* mk_decode_step followed by mk_sample_top_p on its logits: one decode step of
+ * B*T rows whose next tokens are sampled instead of taken greedily.  Arguments
+ * as mk_decode_step (out_logits may be NULL: the handle's scratch holds them)
+ * and mk_sample_top_p (uniforms [B*T]); out_tokens [B*T] receives the sampled
+ * ids (the step's argmax passes through it first).  Errors: those of both. */
+MK_API int mk_decode_step_sample(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                                 int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
+                                 float temperature, float top_p, const double *uniforms,
+                                 int32_t *out_tokens, void *stream);
+
 /* The same step driven from HOST buffers: copies tokens [B*T] and positions
  * [B] to the device, runs the step, copies argmax [B*T] back to
  * out_argmax_host, and waits for the stream.  Logits stay on the device

@@ -48,7 +48,8 @@ class Sample:
     total_mass: int      # Q, fixed point
     need: int            # mass the nucleus had to reach
     y: int               # the draw's point in [0, S)
-    margin: int          # distance (fixed point) from the nearest decision boundary
+    margin: int          # distance (fixed point) from the nearest decision boundary that
+                         # rounding of the masses could move
 
 
 def probabilities(logits: np.ndarray, temperature: float) -> np.ndarray:
@@ -111,8 +112,9 @@ def sample_top_p(logits: np.ndarray, temperature: float, top_p: float, u: float)
     token = int(ids[j])
     before = int(acum[j - 1]) if j > 0 else 0
     margin = min(y - before, int(acum[j]) - 1 - y)
-    below = int(cum[k - 2]) if k > 1 else 0
-    margin = min(margin, int(cum[k - 1]) - need, need - 1 - below)
+    if 1 < need < total:  # need = 1 or need = Q fixes the nucleus whatever the masses' rounding
+        below = int(cum[k - 2]) if k > 1 else 0
+        margin = min(margin, int(cum[k - 1]) - need, need - 1 - below)
     return Sample(token, k, s, total, need, y, margin)
 
 

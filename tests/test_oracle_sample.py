@@ -164,3 +164,14 @@ def test_rejects_bad_inputs():
                 lambda: osample.sample_top_p(np.zeros(0, np.float32), 1.0, 0.5, 0.1)):
         with pytest.raises(ValueError):
             bad()
+
+
+def test_margin_ignores_forced_nucleus_boundaries():
+    """top_p 0 keeps one token and top_p 1 all of them whatever the masses'
+    rounding: only the draw's own boundary bounds the margin there."""
+    l = _rows(1, 400, 1.0, 16)[0]
+    for top_p in (0.0, 1.0):
+        s = osample.sample_top_p(l, 1.0, top_p, 0.37)
+        assert s.margin > 0
+    s = osample.sample_top_p(l, 1.0, 0.8, 0.37)
+    assert 1 < s.need < s.total_mass and s.margin > 0
