@@ -48,8 +48,28 @@ class Sample:
     total_mass: int      # Q, fixed point
     need: int            # mass the nucleus had to reach
     y: int               # the draw's point in [0, S)
-    margin: int          # distance (fixed point) from the nearest decision boundary that
-                         # rounding of the masses could move
+    draw_margin: int     # distance of y from the ends of the drawn token's interval
+    nucleus_margin: int  # distance of the prefix sums from need at the nucleus boundary
+                         # (unbounded where no rounding can move the boundary)
+    boundary_mass: int   # largest mass that could enter or leave at that boundary
+
+    def robust(self, slack: int) -> bool:
+        """True when no change of the masses' sums by at most ``slack`` units can
+        change the token: the draw is clear of its interval's ends, and the
+        nucleus boundary either cannot move or, if it does, shifts the draw's
+        point and interval ends by less than the draw's distance to them."""
+        if self.total_mass == 0:
+            return True  # greedy
+        if self.draw_margin <= slack:
+            return False
+        return self.nucleus_margin > slack or self.draw_margin > self.boundary_mass + 2 * slack
+
+    @property
+    def margin(self) -> int:
+        return min(self.draw_margin, self.nucleus_margin)
+
+
+UNBOUNDED = 1 << 80
 
 
 def probabilities(logits: np.ndarray, temperature: float) -> np.ndarray:
@@ -93,7 +113,7 @@ def sample_top_p(logits: np.ndarray, temperature: float, top_p: float, u: float)
         raise ValueError("u must lie in [0, 1)")
     if float(np.float32(temperature)) <= 0.0:
         t = greedy(l)
-        return Sample(t, 1, 0, 0, 0, 0, 0)
+        return Sample(t, 1, 0, 0, 0, 0, UNBOUNDED, UNBOUNDED, 0)
     q = masses(l, temperature)
     total = int(q.sum(dtype=np.uint64))
     need = nucleus_need(total, top_p)
@@ -111,11 +131,18 @@ def sample_top_p(logits: np.ndarray, temperature: float, top_p: float, u: float)
     j = int(np.searchsorted(acum, np.uint64(y), side="right"))  # first acum > y
     token = int(ids[j])
     before = int(acum[j - 1]) if j > 0 else 0
-    margin = min(y - before, int(acum[j]) - 1 - y)
-    if 1 < need < total:  # need = 1 or need = Q fixes the nucleus whatever the masses' rounding
+    draw_margin = min(y - before, int(acum[j]) - 1 - y)
+    # the nucleus boundary: need = 1 keeps the top token whatever the rounding;
+    # the nucleus cannot grow once it holds every token with mass
+    nucleus_margin, boundary = UNBOUNDED, 0
+    if need > 1:
         below = int(cum[k - 2]) if k > 1 else 0
-        margin = min(margin, int(cum[k - 1]) - need, need - 1 - below)
-    return Sample(token, k, s, total, need, y, margin)
+        nucleus_margin = need - 1 - below
+        boundary = int(q[order[k - 1]])
+        if k < int(np.count_nonzero(q)):
+            nucleus_margin = min(nucleus_margin, int(cum[k - 1]) - need)
+            boundary = max(boundary, int(q[order[k]]))
+    return Sample(token, k, s, total, need, y, draw_margin, nucleus_margin, boundary)
 
 
 def sample_rows(logits: np.ndarray, temperature: float, top_p: float, u) -> list:

@@ -51,7 +51,7 @@ def _compare(logits, T, top_p, u):
     checked = 0
     for r in range(logits.shape[0]):
         ref = osample.sample_top_p(logits[r], T, top_p, 0.0 if u is None else float(u[r]))
-        if T > 0 and ref.margin <= FIXED_POINT_SLACK:
+        if not ref.robust(FIXED_POINT_SLACK):
             continue
         assert int(got[r]) == ref.token, (r, T, top_p, int(got[r]), ref)
         checked += 1
@@ -169,7 +169,7 @@ def test_decode_step_sample_against_oracle():
                 o = osample.sample_top_p(ref.logits[r], T, top_p, float(uh[r]))
                 total += 1
                 bound = 0 if T <= 0 else 2 * o.total_mass * math.expm1(2 * delta / T) + FIXED_POINT_SLACK
-                if T > 0 and o.margin <= bound:
+                if T > 0 and not o.robust(int(bound)):
                     continue
                 if T <= 0 and np.sort(ref.logits[r])[-1] - np.sort(ref.logits[r])[-2] <= 2 * delta:
                     continue
