@@ -421,7 +421,9 @@ def measure_sampled(dec, m, k, v, B, ctx, device, steps=20, warmup=3, temperatur
     """Sampled decode (mk_decode_step_sample: the step, then temperature / top-p
     sampling of its logits) with each step's token fed to the next on the
     device, and the sampler alone (mk_sample_top_p) on 1, 8 and 64 rows of
-    this vocabulary.  CUDA events on the launching stream."""
+    this vocabulary: 50 launches queued behind a device-side sleep, so that the
+    events time the device and not the host's launch rate.  CUDA events on the
+    launching stream."""
     import torch
 
     import decode_megakernel_06_b200 as mk
@@ -454,6 +456,7 @@ def measure_sampled(dec, m, k, v, B, ctx, device, steps=20, warmup=3, temperatur
         torch.cuda.synchronize()
         reps = 50
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(100_000_000)  # the host queues every launch before the device reaches them
         e0.record(stream)
         for _ in range(reps):
             mk.sample_top_p(lg, temperature, top_p, uu, out)

@@ -29,6 +29,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "mk_internal.h"
 
 namespace cg = cooperative_groups;
@@ -40,6 +43,7 @@ constexpr int kSThreads = kSampleThreads;
 constexpr int kSWarps = kSThreads / 32;
 constexpr int kHistCopies = 8;  // warp w adds into copy w % 8
 constexpr double kMassScale = 70368744177664.0;  // 2^46
+constexpr int kSampleMaxDevices = 64;
 
 // Order-preserving key: larger logit <-> larger key; -0 and +0 share one key.
 __device__ __forceinline__ uint32_t logit_key(float x) {
@@ -73,10 +77,29 @@ __device__ __forceinline__ uint64_t warp_incl_scan_u64(uint64_t v, int lane) {
   return v;
 }
 
+// Adds mass q to bucket b of hist for every lane with `valid`; lanes that hit
+// the same bucket are summed first and their lowest lane adds once, so a warp
+// issues one atomic per distinct bucket instead of one per lane.  All 32 lanes
+// must call it together; stage is this warp's 32-word scratch.
+__device__ __forceinline__ void hist_add(uint64_t *hist, uint32_t b, uint64_t qv, bool valid,
+                                         uint64_t *stage, int lane) {
+  if (!__any_sync(0xffffffffu, valid)) return;
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? b : 0xffffffffu);
+  stage[lane] = qv;
+  __syncwarp();
+  if (valid && lane == __ffs(peers) - 1) {
+    uint64_t sum = 0;
+    for (unsigned mm = peers; mm; mm &= mm - 1) sum += stage[__ffs(mm) - 1];
+    atomicAdd(reinterpret_cast<unsigned long long *>(&hist[b]), (unsigned long long)sum);
+  }
+  __syncwarp();
+}
+
 struct SampleShared {
   uint64_t chist[2][256];   // this CTA's merged histogram, read by the cluster
   uint64_t tot[256];        // cluster totals of the current pass
   uint64_t seg[2];          // this CTA's (mass above tau, tokens at tau), read by the cluster
+  uint64_t stage[kSWarps][32];  // per-warp scratch of hist_add
   uint64_t wmass[kSWarps];   // per-warp segment totals
   uint32_t wtie[kSWarps];
   uint32_t wkey[kSWarps];
@@ -91,7 +114,7 @@ struct SampleShared {
 
 __global__ void __launch_bounds__(kSThreads, 1)
 top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_t, float top_p,
-             int greedy, const double *__restrict__ uniforms, int32_t *__restrict__ out) {
+             int greedy, int vec4, const double *__restrict__ uniforms, int32_t *__restrict__ out) {
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ SampleShared sh;
@@ -108,10 +131,22 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
   for (int i = tid; i < kHistCopies * 256; i += kSThreads) whist[i] = 0;
   // ---- load the slice; this CTA's largest key --------------------------------
   uint32_t kmax = 0;
-  for (int i = tid; i < n; i += kSThreads) {
-    float x = src[i];
-    l[i] = x;
-    kmax = max(kmax, logit_key(x));
+  if (vec4) {  // rows and slices start on 16-byte boundaries and n % 4 == 0
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    float4 *l4 = reinterpret_cast<float4 *>(l);
+#pragma unroll 4
+    for (int i = tid; i < n / 4; i += kSThreads) {
+      float4 x = s4[i];
+      l4[i] = x;
+      kmax = max(max(kmax, max(logit_key(x.x), logit_key(x.y))), max(logit_key(x.z), logit_key(x.w)));
+    }
+  } else {
+#pragma unroll 8
+    for (int i = tid; i < n; i += kSThreads) {
+      float x = src[i];
+      l[i] = x;
+      kmax = max(kmax, logit_key(x));
+    }
   }
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   if (lane == 0) sh.wkey[warp] = kmax;
@@ -156,12 +191,18 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
   // ---- masses and the histogram of the top key byte ------------------------------
   const float m = key_logit(gkey);
   uint64_t *myhist = whist + (warp % kHistCopies) * 256;
-  for (int i = tid; i < n; i += kSThreads) {
-    float x = l[i];
-    uint64_t qi = mass_of(x, m, inv_t);
-    q[i] = qi;
-    if (qi) atomicAdd(reinterpret_cast<unsigned long long *>(&myhist[logit_key(x) >> 24]),
-                      (unsigned long long)qi);
+  uint64_t *stage = sh.stage[warp];
+  for (int i0 = tid - lane; i0 < n; i0 += kSThreads) {  // warp-uniform trip count
+    const int i = i0 + lane;
+    uint64_t qi = 0;
+    uint32_t k = 0;
+    if (i < n) {
+      float x = l[i];
+      qi = mass_of(x, m, inv_t);
+      q[i] = qi;
+      k = logit_key(x);
+    }
+    hist_add(myhist, k >> 24, qi, qi != 0, stage, lane);
   }
   if (tid == 0) {
     sh.prefix = 0;
@@ -184,6 +225,7 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
     cluster.sync();  // 2..5: every CTA's histogram of this pass is visible
     if (tid < 256) {
       uint64_t s = 0;
+#pragma unroll
       for (unsigned r = 0; r < kSampleCluster; ++r) s += cluster.map_shared_rank(&sh.chist[buf][0], r)[tid];
       sh.tot[tid] = s;
     }
@@ -233,12 +275,15 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
     if (d < 3) {
       const uint32_t pre = sh.prefix;
       const int shift = 24 - 8 * d;  // bits above the next digit
-      for (int i = tid; i < n; i += kSThreads) {
-        uint32_t k = logit_key(l[i]);
-        uint64_t qi = q[i];
-        if ((k >> shift) == pre && qi)
-          atomicAdd(reinterpret_cast<unsigned long long *>(&myhist[(k >> (shift - 8)) & 255u]),
-                    (unsigned long long)qi);
+      for (int i0 = tid - lane; i0 < n; i0 += kSThreads) {  // warp-uniform trip count
+        const int i = i0 + lane;
+        uint32_t k = 0;
+        uint64_t qi = 0;
+        if (i < n) {
+          k = logit_key(l[i]);
+          qi = q[i];
+        }
+        hist_add(myhist, (k >> (shift - 8)) & 255u, qi, i < n && qi != 0 && (k >> shift) == pre, stage, lane);
       }
     }
   }
@@ -332,8 +377,22 @@ cudaError_t launch_top_p(const float *logits, int rows, int vocab, float tempera
                          const double *uniforms, int32_t *out, cudaStream_t stream) {
   const int slice = (vocab + kSampleCluster - 1) / kSampleCluster;
   const size_t smem = sample_smem_bytes(slice);
-  cudaError_t e = cudaFuncSetAttribute(top_p_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the largest dynamic size set so far, per device: the attribute is set only
+  // when a launch needs more than that (never on the steady-state path)
+  static std::atomic<size_t> configured[kSampleMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kSampleMaxDevices) return cudaErrorInvalidDevice;
+  if (smem > configured[dev].load(std::memory_order_acquire)) {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (smem > configured[dev].load(std::memory_order_relaxed)) {
+      e = cudaFuncSetAttribute(top_p_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      configured[dev].store(smem, std::memory_order_release);
+    }
+  }
   const int greedy = !(temperature > 0.0f);
   const double inv_t = greedy ? 0.0 : 1.0 / (double)temperature;
   cudaLaunchConfig_t cfg = {};
@@ -348,7 +407,8 @@ cudaError_t launch_top_p(const float *logits, int rows, int vocab, float tempera
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, top_p_kernel, logits, vocab, slice, inv_t, top_p, greedy, uniforms, out);
+  const int vec4 = (vocab % 4 == 0) && (slice % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15) == 0);
+  return cudaLaunchKernelEx(&cfg, top_p_kernel, logits, vocab, slice, inv_t, top_p, greedy, vec4, uniforms, out);
 }
 
 }  // namespace mk
