@@ -173,3 +173,21 @@ def test_null_arguments_are_rejected(L):
     kv = mk.mk_kv_cache(None, None)
     assert L.mk_decode_step(None, None, None, 1, 1, kv, None, None, None) == mk.MK_ERR_ARG
     L.mk_destroy(None)  # safe on NULL
+
+
+def test_sampler_checks_its_arguments_on_the_host(L):
+    """mk_sample_top_p rejects bad arguments before any CUDA call (the pointers
+    below are never dereferenced)."""
+    lg, u, out = 256, 512, 768  # stand-in addresses: every call here fails its host checks
+    nan = float("nan")
+    assert L.mk_sample_top_p(None, 1, 10, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p(lg, 1, 10, 1.0, 0.9, u, None, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p(lg, 0, 10, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p(lg, 1, 0, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p(lg, 1, 10, nan, 0.9, u, out, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p(lg, 1, 10, 1.0, nan, u, out, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p(lg, 1, 10, 0.7, 0.9, None, out, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p(lg, 1, 131073, 1.0, 0.9, u, out, None) == mk.MK_ERR_UNSUPPORTED
+    assert "131072" in mk.mk_last_error()
+    kv = mk.mk_kv_cache(None, None)
+    assert L.mk_decode_step_sample(None, None, None, 1, 1, kv, None, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
