@@ -143,9 +143,3 @@ def sample_top_p(logits: np.ndarray, temperature: float, top_p: float, u: float)
             nucleus_margin = min(nucleus_margin, int(cum[k - 1]) - need)
             boundary = max(boundary, int(q[order[k]]))
     return Sample(token, k, s, total, need, y, draw_margin, nucleus_margin, boundary)
-
-
-def sample_rows(logits: np.ndarray, temperature: float, top_p: float, u) -> list:
-    """sample_top_p over each row of a [rows][V] array, with u[row]."""
-    logits = np.asarray(logits, dtype=np.float32)
-    return [sample_top_p(logits[r], temperature, top_p, float(u[r])) for r in range(logits.shape[0])]
