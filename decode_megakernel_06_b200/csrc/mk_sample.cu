@@ -6,8 +6,8 @@
 // What is computed, per row of V fp32 logits l, with one uniform u in [0, 1):
 //   p_i = exp((l_i - max l) / T) in fp64; q_i = round_half_even(p_i * 2^46),
 //   an exact fixed-point mass (every later sum is an integer sum, so no
-//   decision depends on a summation order); need = max(1, ceil(top_p * Q)),
-//   Q = sum q; the nucleus is the smallest prefix of the tokens sorted by
+//   decision depends on a summation order); need = max(1, min(Q, ceil(top_p *
+//   Q))), Q = sum q, the product in fp64; the nucleus is the smallest prefix of the tokens sorted by
 //   logit, descending, ties by lower id, whose mass reaches need; the token is
 //   the first nucleus id, in id order, whose cumulative mass exceeds
 //   y = min(S - 1, floor(u * S)), S the nucleus mass.  T <= 0 is greedy: the
@@ -24,7 +24,8 @@
 // number r of tokens tied at tau that enter the nucleus are known.  The draw is
 // an inverse CDF in id order: per-warp segment totals are summed across the
 // cluster, and only the warp whose segment holds the point y scans its
-// segment element by element.  Seven cluster barriers in all; no spin-waits.
+// segment, 32 tokens at a time.  Seven cluster barriers when sampling, three
+// when greedy; no spin-waits.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
