@@ -175,3 +175,16 @@ def test_margin_ignores_forced_nucleus_boundaries():
         assert s.margin > 0
     s = osample.sample_top_p(l, 1.0, 0.8, 0.37)
     assert 1 < s.need < s.total_mass and s.margin > 0
+
+
+def test_largest_row_sums_without_overflow():
+    """At the largest vocabulary, equal logits give Q = 2^17 * 2^46 = 2^63 exactly:
+    the 64-bit sums hold the worst case, and every token is equally likely."""
+    l = np.zeros(osample.MAX_VOCAB, np.float32)
+    s = osample.sample_top_p(l, 1.0, 1.0, 0.5)
+    assert s.total_mass == 1 << 63 and s.nucleus == osample.MAX_VOCAB
+    assert s.token == osample.MAX_VOCAB // 2
+    s = osample.sample_top_p(l, 1.0, 0.25, 0.5)
+    assert s.nucleus == osample.MAX_VOCAB // 4 and s.token == osample.MAX_VOCAB // 8
+    with pytest.raises(ValueError):
+        osample.sample_top_p(np.zeros(osample.MAX_VOCAB + 1, np.float32), 1.0, 0.5, 0.5)
