@@ -308,7 +308,7 @@ def time_e2e(dec, m, k, v, B, T, ctx, steps, warmup):
     return dt, (th.numel() + ph.numel()) * 4, out.numel() * 4
 
 
-def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1, min_compute_s=0.0):
+def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1, min_compute_s=0.0, threads=0):
     """The CPU oracle as it stands on the same workload: whole decode steps
     (all layers), weights copied from the device on demand; the copy time is
     excluded from the compute time and reported beside it.  Runs ``n_steps``
@@ -320,7 +320,7 @@ def oracle_sample(m, w, k_dev, v_dev, B, T, ctx, n_steps=1, min_compute_s=0.0):
     from oracle import step as ostep
     from synthetic import bf16_bits, make_tokens
 
-    threads = oracle.set_threads(0)
+    threads = oracle.set_threads(threads)
     src = ostep.WeightSource(w, cache=False)
     # only the sequences' live layers of the cache are needed; copy it once
     kh = bf16_bits(k_dev[:, :B]).copy()
@@ -497,25 +497,29 @@ def measure_dense(device, steps=20, warmup=3):
             "launches_per_step": st.kernel_launches // steps}
 
 
-def measure_verify_loop(device, n_steps=16):
-    """Speculative verify on the device (mk_verify_steps) on the small model:
-    one sequence, blocks of 7 rows (the last accepted token + 6 drafts), n_steps
-    blocks in one launch.  The synthetic drafter proposes the model's own
-    greedy continuation (taken from a greedy multi-step launch first) with
-    every 6th draft replaced, so that each block accepts 5 drafts plus one
-    token: acceptance length 6.  Reports accepted tokens per second."""
+def measure_verify_loop(device, n_steps=16, model=None, weights=None, seed=None, context=None):
+    """Speculative verify on the device (mk_verify_steps): one sequence, blocks
+    of 7 rows (the last accepted token + 6 drafts), n_steps blocks in one
+    launch, on the small model (default) or on the given model and weights.
+    The synthetic drafter proposes the model's own greedy continuation (taken
+    from a greedy multi-step launch first) with every 6th draft replaced, so
+    that each block accepts 5 drafts plus one token: acceptance length 6.
+    Reports accepted tokens per second."""
     import torch
 
     import decode_megakernel_06_b200 as mk
     from synthetic import make_kv_cache, make_tokens, make_weights, workload
 
     wl = workload("verify", 1)
-    m, T = wl.model, wl.tokens_per_step
+    T = wl.tokens_per_step
+    if model is None:
+        m, seed, p0 = wl.model, wl.seed, wl.context
+        w = make_weights(m, seed, device)
+    else:
+        m, w, p0 = model, weights, context
     acc_len = T - 1
-    w = make_weights(m, wl.seed, device)
-    p0 = wl.context
     cap = (p0 + (n_steps + 2) * T + 64 + 63) // 64 * 64
-    k, v = make_kv_cache(m, 1, cap, wl.seed, device)
+    k, v = make_kv_cache(m, 1, cap, seed, device)
     dec = mk.Decoder(m, w, max_rows=T, max_seqs=1, kv_capacity=cap)
     first = make_tokens(m.vocab, 1, 55)[0]
     ng = n_steps * acc_len + T
@@ -547,9 +551,11 @@ def measure_verify_loop(device, n_steps=16):
     ms = e0.elapsed_time(e1)
     accepted = int(acc.sum().item())
     dec.close()
-    del w, k, v
+    del k, v
+    if model is None:
+        del w
     torch.cuda.empty_cache()
-    return {"workload": f"verify_b1_t{T} ({m.name} model), {n_steps} blocks in one launch",
+    return {"workload": f"verify_b1_t{T} ({m.name} model, context {p0}), {n_steps} blocks in one launch",
             "accepted_tok_s": round(accepted / (ms / 1e3), 1), "mean_acceptance": round(accepted / n_steps, 2),
             "ms_per_block": round(ms / n_steps, 4), "launches": 1,
             "drafter": "the model's greedy continuation with every 6th draft replaced"}
@@ -584,6 +590,75 @@ def measure_verify_wide(device, steps=10, warmup=3, batch=8):
             "expert_union_per_layer": round(union, 1), "launches_per_step": st.kernel_launches // steps,
             "path": ("tensor-core launch sequence (blocks above 8 rows), replayed as a CUDA graph"
                      if B * T > 8 else "megakernel")}
+
+
+def measure_read_probe(device, gib=4):
+    """The read-only HBM ceiling on this device (mk_hbm_read_probe over a
+    buffer far larger than L2): the better of the vector-load and bulk-copy
+    forms, 3 calls of 5 timed passes each."""
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+
+    buf = torch.empty(gib << 30, dtype=torch.uint8, device=device)
+    buf.fill_(1)
+    forms = {}
+    for form, name in ((0, "vector_loads"), (1, "bulk_copies")):
+        forms[name] = round(max(mk.hbm_read_probe(buf, form, 5) for _ in range(3)), 1)
+    del buf
+    torch.cuda.empty_cache()
+    return {"gbs": max(forms.values()), "forms": forms, "bytes": gib << 30,
+            "how": "mk_hbm_read_probe: each byte read once per pass, nothing written; best of 3 x 5 passes"}
+
+
+# The synthetic workloads besides the large model (each also on both
+# multi-kernel forms): latency of the tiny model, the small model at batch 1,
+# the small model at batches 2/4/8 with per-sequence random contexts, and the
+# 7-row speculative-verify block.
+CONFIG_LINES = [("tiny_bs1", "tiny", 1), ("small_bs1", "small", 1), ("small_bs2", "small_batch", 2),
+                ("small_bs4", "small_batch", 4), ("small_bs8", "small_batch", 8), ("verify_b1_t7", "verify", 1)]
+
+
+def measure_config_lines(device, peak, probe_gbs, steps=20, warmup=3):
+    import torch
+
+    import decode_megakernel_06_b200 as mk
+    from synthetic import make_context_lengths, make_kv_cache, make_weights, workload
+
+    out = {}
+    for key, kind, B in CONFIG_LINES:
+        wl = workload(kind, B)
+        m, T = wl.model, wl.tokens_per_step
+        w = make_weights(m, wl.seed, device)
+        ctx = make_context_lengths(wl)
+        cap = (max(ctx) + (steps + warmup + 2) * T + 63) // 64 * 64
+        k, v = make_kv_cache(m, B, cap, wl.seed, device)
+        dec = mk.Decoder(m, w, max_rows=B * T, max_seqs=B, kv_capacity=cap)
+        row = {"workload": f"{wl.name}: {m.name} model ({m.n_layers} layers, d {m.d_model}, "
+                           f"{m.n_experts} experts top-{m.top_k}), B {B}, T {T}, context "
+                           + (str(wl.context) if wl.context else f"U{list(wl.context_range)} per sequence")}
+        for var in ("megakernel", "multikernel", "multikernel_graph"):
+            dec.set_variant(var)
+            tot, per, st = time_steps(dec, m, k, v, B, T, ctx, steps, warmup, device)
+            ms = tot / steps
+            r = {"ms_per_step": round(ms, 4), "ms_per_step_p50": round(statistics.median(per), 4),
+                 "tok_s": round(B * T / (ms / 1e3), 1), "launches_per_step": st.kernel_launches // steps}
+            if kind != "tiny":  # the tiny model stays in L2: latency only
+                lens = [c + (warmup + steps // 2) * T + T for c in ctx]
+                by = step_bytes(m, B, T, lens, st.expert_union_total / steps)
+                gbs = by / (ms / 1e3) / 1e9
+                r.update({"hbm_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                          "frac_of_read_probe": round(gbs / probe_gbs, 4) if probe_gbs else None,
+                          "bytes_per_step": int(by)})
+            row[var] = r
+        mkv = row["megakernel"]["tok_s"]
+        row["megakernel_vs_multikernel"] = round(mkv / row["multikernel"]["tok_s"], 3)
+        row["megakernel_vs_multikernel_graph"] = round(mkv / row["multikernel_graph"]["tok_s"], 3)
+        out[key] = row
+        dec.close()
+        del w, k, v
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_mine(args):
@@ -666,22 +741,31 @@ def run_mine(args):
     if args.sweep and T == 1:
         sampled = measure_sampled(dec, m, k, v, B, ctx, device)
 
-    verify56 = verify7 = vloop = dense = None
+    probe = measure_read_probe(device) if not args.no_probe else None
+    probe_gbs = probe["gbs"] if probe else None
+
+    verify56 = vloop = vloop_large = dense = configs = None
     if args.sweep and ws == 1 and args.workload == "large":
         verify56 = measure_verify_wide(device)
-        verify7 = measure_verify_wide(device, batch=1)
         vloop = measure_verify_loop(device)
+        vloop_large = measure_verify_loop(device, model=m, weights=w, seed=wl.seed, context=wl.context)
         dense = measure_dense(device)
+        configs = measure_config_lines(device, peak, probe_gbs)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        # all host cores (the reported value), then one thread on a shorter sample
         o = oracle_sample(m, w, k, v, B, T, ctx, 1, min_compute_s=10.0)
+        o1 = oracle_sample(m, w, k, v, B, T, ctx, 1, threads=1)
         cpu = {"value": round(o["tokens"] / o["compute_s"], 4), "unit": "tokens/s",
                "cores": o["threads"], "kind": "oracle",
                "sample": (f"{o['steps']} consecutive greedy decode steps of the same workload "
                           f"(all layers, from the same cache) on the host "
                           f"(compute {o['compute_s']:.2f} s; weight copy from the device "
-                          f"{o['fetch_s']:.2f} s excluded)")}
+                          f"{o['fetch_s']:.2f} s excluded)"),
+               "one_thread": {"value": round(o1["tokens"] / o1["compute_s"], 4), "unit": "tokens/s",
+                              "cores": 1, "sample": (f"{o1['steps']} decode step(s), compute "
+                                                     f"{o1['compute_s']:.2f} s on one thread")}}
 
     traffic = profile_traffic(f"large_bs{B}_{args.variant}") if args.workload == "large" else None
     if rank == 0:
@@ -701,7 +785,14 @@ def run_mine(args):
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peaks_kind} copy bandwidth",
                          "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                         "traffic": traffic, "algorithmic_bytes_per_step": int(alg_bytes),
+                         "traffic": traffic,
+                         "traffic_kind": ("ncu dram bytes of the profile model's launch (2 layers, same per-op "
+                                          "shapes), scaled to this launch by its algorithmic bytes; null once the "
+                                          "kernel source differs from the captured one") if args.workload == "large"
+                                         else None,
+                         "peak_read_probe": probe_gbs,
+                         "frac_of_read_probe": round(achieved / probe_gbs, 4) if probe_gbs else None,
+                         "algorithmic_bytes_per_step": int(alg_bytes),
                          "expert_union_per_step": round(union_per_step, 2)},
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -717,10 +808,14 @@ def run_mine(args):
             line["sampled"] = sampled
         if verify56 is not None:
             line["verify_56"] = verify56
-        if verify7 is not None:
-            line["verify_7"] = verify7
+        if probe is not None:
+            line["read_probe"] = probe
+        if configs is not None:
+            line["configs"] = configs
         if vloop is not None:
             line["speculative"] = vloop
+        if vloop_large is not None:
+            line["speculative_large"] = vloop_large
         if dense is not None:
             line["dense"] = dense
         print(json.dumps(line), flush=True)
@@ -784,6 +879,7 @@ def main():
                     choices=["megakernel", "multikernel", "multikernel_graph"])
     ap.add_argument("--sweep", action=argparse.BooleanOptionalAction, default=True)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-probe", action="store_true", help="skip the read-only HBM probe")
     ap.add_argument("--trace-out", default=None,
                     help="with --trace: save the raw per-op, per-warp [start, end] stamps (.npy)")
     ap.add_argument("--trace", action="store_true",

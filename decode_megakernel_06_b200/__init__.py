@@ -34,11 +34,10 @@ VARIANTS = {"megakernel": MK_MEGAKERNEL, "multikernel": MK_MULTIKERNEL,
 
 MK_FAULT_NONE = 0
 MK_FAULT_UNREACHABLE_WAIT = 1
-MK_TRACE_WORDS = 8  # uint64 words per (op, warp) record of mk_set_trace
+MK_TRACE_WORDS = 12  # uint64 words per (op, warp) record of mk_set_trace
 MK_STATIC_SCRATCH_BYTES = 32 << 20  # the fixed working array of mk_decode_step_static
 
-OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE",
-            "LMHEAD"]
+OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE", "LMHEAD"]
 
 
 class mk_model_desc(ctypes.Structure):
@@ -115,6 +114,7 @@ def lib():
         "mk_debug_inject": (i32, [vp, i32]),
         "mk_set_trace": (i32, [vp, vp]),
         "mk_get_stats": (i32, [vp, ctypes.POINTER(mk_stats), i32]),
+        "mk_hbm_read_probe": (i32, [vp, u64, i32, i32, ctypes.POINTER(ctypes.c_double), vp]),
         "mk_validate_desc": (i32, [ctypes.POINTER(mk_model_desc)]),
         "mk_plan_describe": (i32, [ctypes.POINTER(mk_model_desc), i32, i32, i32,
                                    ctypes.POINTER(mk_plan_info), _I32P, _I32P, _I32P, _I32P, i32]),
@@ -203,16 +203,52 @@ def mk_decode_step_sample(h, tokens: int, positions: int, B: int, T: int, kv: mk
                                        uniforms, out_tokens, stream)
 
 
+def _need(t, dtype, min_numel: int, name: str, device=None, dims: Optional[int] = None):
+    """Check a tensor handed to a kernel by its data pointer: dtype, a
+    contiguous layout with at least ``min_numel`` elements, optionally the
+    number of dimensions, then that it lives on ``device`` (a CUDA device).
+    A wrong tensor would otherwise make the kernel read or write past it."""
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name}: {t.dim()}-D, expected {dims}-D")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, at least {min_numel} needed")
+    if t.device.type != "cuda" or (device is not None and t.device != device):
+        raise ValueError(f"{name}: on {t.device}, expected " + (str(device) if device is not None else "a CUDA device"))
+
+
 def sample_top_p(logits, temperature: float, top_p: float, uniforms, out_tokens, stream=None) -> int:
     """Torch-tensor form of mk_sample_top_p: logits fp32 [rows, vocab], uniforms
-    fp64 [rows] (or None when temperature <= 0), out_tokens int32 [rows], all on
-    the device.  Returns the launch status code."""
+    fp64 [rows] (or None when temperature <= 0), out_tokens int32 [rows], all
+    contiguous on one CUDA device (checked: ValueError otherwise).  Returns the
+    launch status code."""
     import torch
 
-    s = stream if stream is not None else torch.cuda.current_stream()
+    _need(logits, torch.float32, 1, "logits", dims=2)
     rows, vocab = logits.shape
+    if uniforms is not None:
+        _need(uniforms, torch.float64, rows, "uniforms", logits.device)
+    _need(out_tokens, torch.int32, rows, "out_tokens", logits.device)
+    s = stream if stream is not None else torch.cuda.current_stream()
     return mk_sample_top_p(logits.data_ptr(), rows, vocab, temperature, top_p, _ptr(uniforms),
                            out_tokens.data_ptr(), s.cuda_stream)
+
+
+def hbm_read_probe(buf, form: int = 0, reps: int = 5, stream=None) -> float:
+    """Read-only HBM bandwidth in GB/s over the CUDA tensor ``buf`` (16-byte
+    aligned, >= 64 MiB; see mk_hbm_read_probe).  Raises on failure."""
+    import torch
+
+    if buf.device.type != "cuda" or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous CUDA tensor")
+    s = stream if stream is not None else torch.cuda.current_stream()
+    out = ctypes.c_double(0.0)
+    _check(lib().mk_hbm_read_probe(buf.data_ptr(), buf.numel() * buf.element_size(), form, reps,
+                                   ctypes.byref(out), s.cuda_stream))
+    return out.value
 
 
 def mk_get_device_status(h, stream: int) -> int:
@@ -317,9 +353,25 @@ class Decoder:
     def inject(self, fault: int):
         _check(mk_debug_inject(self.h, fault))
 
+    def _io(self, tokens, positions, B: int, rows: int, k_cache, v_cache, logits=None):
+        """The checks every device-tensor call shares (ValueError on a mismatch)."""
+        t = self._torch
+        _need(tokens, t.int32, rows, "tokens")
+        dev = tokens.device
+        _need(positions, t.int32, B, "positions", dev)
+        kv_numel = (self.model.n_layers * self.max_seqs * self.model.n_kv_heads * self.kv_capacity
+                    * self.model.head_dim)
+        _need(k_cache, t.bfloat16, kv_numel, "k_cache", dev)
+        _need(v_cache, t.bfloat16, kv_numel, "v_cache", dev)
+        if logits is not None:
+            _need(logits, t.float32, rows * self.model.vocab, "logits", dev)
+        return dev
+
     def step(self, tokens, positions, B: int, T: int, k_cache, v_cache, logits, argmax,
              stream=None) -> int:
         """Enqueue one step (device tensors); returns the launch status code."""
+        dev = self._io(tokens, positions, B, B * T, k_cache, v_cache, logits)
+        _need(argmax, self._torch.int32, B * T, "argmax", dev)
         s = stream if stream is not None else self._torch.cuda.current_stream()
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_step(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
@@ -329,6 +381,10 @@ class Decoder:
                     top_p: float, uniforms, out_tokens, stream=None) -> int:
         """One step whose next tokens are sampled (temperature / top-p) from its
         logits with the given fp64 uniforms [B*T].  Returns the launch status code."""
+        dev = self._io(tokens, positions, B, B * T, k_cache, v_cache, logits)
+        if uniforms is not None:
+            _need(uniforms, self._torch.float64, B * T, "uniforms", dev)
+        _need(out_tokens, self._torch.int32, B * T, "out_tokens", dev)
         s = stream if stream is not None else self._torch.cuda.current_stream()
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_step_sample(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
@@ -339,6 +395,8 @@ class Decoder:
               stream=None) -> int:
         """Enqueue n_steps greedy steps as one launch; out_tokens is int32
         [n_steps, B] on the device.  Returns the launch status code."""
+        dev = self._io(tokens, positions, B, B, k_cache, v_cache, logits)
+        _need(out_tokens, self._torch.int32, n_steps * B, "out_tokens", dev)
         s = stream if stream is not None else self._torch.cuda.current_stream()
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_steps(self.h, tokens.data_ptr(), positions.data_ptr(), B, n_steps, kv,
@@ -349,6 +407,10 @@ class Decoder:
         """Enqueue n_steps verify blocks of T rows as one launch; drafts is int32
         [B, draft_len] on the device, out_tokens [n_steps, B*T], out_accepted
         [n_steps, B].  Returns the launch status code."""
+        dev = self._io(tokens, positions, B, B * T, k_cache, v_cache, logits)
+        _need(drafts, self._torch.int32, B * drafts.shape[-1], "drafts", dev, dims=2)
+        _need(out_tokens, self._torch.int32, n_steps * B * T, "out_tokens", dev)
+        _need(out_accepted, self._torch.int32, n_steps * B, "out_accepted", dev)
         s = stream if stream is not None else self._torch.cuda.current_stream()
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_verify_steps(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, n_steps,
@@ -359,6 +421,8 @@ class Decoder:
                     stream=None) -> int:
         """Like ``step``, but the step's working memory is the library's fixed
         device array (no allocation; overlapping calls on one device race)."""
+        dev = self._io(tokens, positions, B, B * T, k_cache, v_cache, logits)
+        _need(argmax, self._torch.int32, B * T, "argmax", dev)
         s = stream if stream is not None else self._torch.cuda.current_stream()
         kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
         return mk_decode_step_static(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,

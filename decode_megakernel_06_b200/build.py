@@ -20,7 +20,8 @@ LIB = os.path.join(HERE, "libmk.so")
 # (source, object name, extra flags): the step kernels are built twice, the
 # second time with the timeline trace compiled in.
 UNITS = [("mk_kernel.cu", "mk_kernel", []), ("mk_kernel.cu", "mk_kernel_trace", ["-DMK_TRACE=1"]),
-         ("mk_api.cu", "mk_api", []), ("mk_wide.cu", "mk_wide", []), ("mk_sample.cu", "mk_sample", [])]
+         ("mk_api.cu", "mk_api", []), ("mk_wide.cu", "mk_wide", []), ("mk_sample.cu", "mk_sample", []),
+         ("mk_probe.cu", "mk_probe", [])]
 SOURCES = sorted({u[0] for u in UNITS})
 HEADERS = ["mk_internal.h", os.path.join("..", "..", "include", "mk.h")]
 

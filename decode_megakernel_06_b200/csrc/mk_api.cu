@@ -128,7 +128,7 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   // shared-memory row: the staged activations (batch 1) or the attention
   // warps' partials and the item's query vectors, whichever is larger
   // (whole 256-column panels: the staged layout permutes columns within one)
-  p.xs_floats = std::max((kConsumers + 1) * kQvp * d.head_dim,
+  p.xs_floats = std::max((kConsumers + 1) * kQvp * d.head_dim + kMaxRows * d.head_dim,  // + new bf16 K/V rows
                          kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), kPanel) * kPanel : 0);
   // Batch 1 down projection: a CTA's contiguous range of units spans at most
   // 1 + ceil(range / row blocks) experts; their activations must fit the
@@ -185,8 +185,9 @@ struct mk_handle {
   std::vector<void *> allocs;
   CUtensorMap *tmaps;
   const __nv_bfloat16 **norms;
-  float *h, *ss, *qkv, *o, *attn_o, *attn_ml, *router_part, *act_shared,
-      *act_routed, *y_part, *logits;
+  float *h, *hm, *ss, *qkv, *o, *attn_o, *attn_ml, *act_shared, *act_routed, *logits;
+  long long *hacc, *racc;
+  size_t hacc_bytes, racc_bytes;
   uint32_t *attn_cnt, *counters, *epoch;
   ArgmaxPart *am_part;
   float2 *rope;
@@ -287,10 +288,10 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
     Sizes s = scratch_sizes(*desc, n_sm);
     const mk_model_desc &d = *desc;
     size_t f = (size_t)d.max_rows * d.d_model * 2 + (size_t)d.max_rows * ceil_div(d.d_model, kRows) +
-               (size_t)kMaxRows * (d.top_k + 1) * d.d_model +
+               (size_t)kMaxRows * d.d_model * 3 +  // h_mid, and the int64 expert-output sums
                2 * (size_t)d.max_rows * (d.n_q_heads + 2 * d.n_kv_heads) * d.head_dim +
                (size_t)d.max_rows * d.d_model + (size_t)d.max_rows * d.n_q_heads * d.head_dim + s.attn_o + s.attn_ml +
-               (size_t)ceil_div(d.d_model, kPanel) * kMaxRows * d.n_experts +
+               (size_t)d.n_layers * kMaxRows * (ceil_div(std::max(d.n_experts, 1), 4) * 4) * 2 +  // int64 router sums
                (size_t)kMaxRows * d.shared_ffn +
                (size_t)std::min(d.n_experts, d.max_rows * d.top_k) * kMaxRows * d.expert_ffn +
                (size_t)d.max_rows * d.vocab + (size_t)d.kv_capacity * d.head_dim;
@@ -299,7 +300,7 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
   }
   for (int i = 0; i < p.n_ops && i < cap; ++i) {
     int d0, d1;
-    op_deps(i, desc->n_layers, &d0, &d1);
+    op_deps(i, desc->n_layers, p.mmax == 1, &d0, &d1);
     if (op_types) op_types[i] = op_type_of(i, desc->n_layers);
     if (op_layers) op_layers[i] = op_layer_of(i, desc->n_layers);
     if (op_dep0) op_dep0[i] = d0;
@@ -389,6 +390,11 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->tmaps, sizeof(CUtensorMap) * (size_t)(L * MAPS_PER_LAYER + 1));
   HALLOC(h->norms, sizeof(void *) * 2 * L);
   HALLOC(h->h, sizeof(float) * 2 * (size_t)kMaxRows * D);  // h, then h * gain (xg)
+  HALLOC(h->hm, sizeof(float) * (size_t)kMaxRows * D);
+  h->hacc_bytes = sizeof(long long) * (size_t)kMaxRows * D;
+  HALLOC(h->hacc, h->hacc_bytes);
+  h->racc_bytes = sizeof(long long) * (size_t)L * kMaxRows * (ceil_div(std::max(d.n_experts, 1), 4) * 4);
+  HALLOC(h->racc, h->racc_bytes);
   HALLOC(h->ss, sizeof(float) * (size_t)kMaxRows * ceil_div(ceil_div(D, kRows), 128) * 128);
   HALLOC(h->qkv, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);  // [K half][row][QKVW]
   HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
@@ -396,10 +402,8 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->attn_ml, sizeof(float) * s.attn_ml);
   h->attn_cnt_bytes = sizeof(uint32_t) * s.attn_cnt;
   HALLOC(h->attn_cnt, h->attn_cnt_bytes);
-  HALLOC(h->router_part, sizeof(float) * (size_t)ceil_div(D, kTileCols) * kMaxRows * ceil_div(d.n_experts, 4) * 4);
   HALLOC(h->act_shared, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
   HALLOC(h->act_routed, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
-  HALLOC(h->y_part, sizeof(float) * (size_t)kMaxRows * (d.top_k + 1) * D);
   HALLOC(h->am_part, sizeof(ArgmaxPart) * (size_t)NW * kMaxRows);
   HALLOC(h->rope, sizeof(float2) * (size_t)d.kv_capacity * (d.head_dim / 2));
   h->counters_bytes = sizeof(uint32_t) * (size_t)n_ops * kCounterStride;
@@ -411,6 +415,13 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   HALLOC(h->io_tokens, sizeof(int32_t) * (size_t)d.max_rows);
   HALLOC(h->io_positions, sizeof(int32_t) * (size_t)d.max_seqs);
   HALLOC(h->io_argmax, sizeof(int32_t) * (size_t)d.max_rows);
+  // speculative-verify launches: per step the block starts, the block tokens
+  // and the argmax; n_steps * T <= kv_capacity and B * T <= 8 bound them
+  {
+    const size_t mr = std::min(d.max_rows, kMaxRows), cap = (size_t)d.kv_capacity;
+    h->vbuf_ints = (cap / 2 + 1) * mr + (cap / 2 + 1) * mr + cap * mr;
+    HALLOC(h->vbuf, sizeof(int32_t) * h->vbuf_ints);
+  }
   if (d.max_rows > kMaxRows) {  // buffers of the wide-block path
     const int MR = d.max_rows, MK = MR * d.top_k, HD = d.n_q_heads * d.head_dim;
     const int ldx = ceil_div(std::max(D, HD), 8) * 8, lda = ceil_div(std::max(d.expert_ffn, std::max(d.shared_ffn, 1)), 8) * 8;
@@ -466,7 +477,9 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     rc = enc(b + MAP_WQKV, lw.wqkv, QKVW, D);
     if (!rc) rc = enc(b + MAP_WO, lw.wo, D, (uint64_t)d.n_q_heads * d.head_dim);
     if (E > 0) {  // a dense model has no router and no routed experts
-      if (!rc) rc = enc(b + MAP_ROUTER, lw.router, E, D);
+      // the router is read 8 columns x all E rows at a time, next to the
+      // o-projection rows it multiplies
+      if (!rc) rc = encode_2d(&maps[b + MAP_ROUTER], lw.router, E, D, 8, (uint32_t)E);
       if (!rc) rc = enc(b + MAP_WGATE, lw.w_gate, E * F, D);
       if (!rc) rc = enc(b + MAP_WUP, lw.w_up, E * F, D);
       if (!rc) rc = enc(b + MAP_WDOWN, lw.w_down, E * D, F);
@@ -510,6 +523,9 @@ static int reset_sync_state(mk_handle *h, cudaStream_t s) {
   CUDA_TRY(cudaMemsetAsync(h->epoch, 0, sizeof(uint32_t) * kCounterStride, s));
   CUDA_TRY(cudaMemsetAsync(h->attn_cnt, 0, h->attn_cnt_bytes, s));
   CUDA_TRY(cudaMemsetAsync(h->error, 0, sizeof(int) * kCounterStride, s));
+  // a failed step may leave partial fixed-point sums behind
+  CUDA_TRY(cudaMemsetAsync(h->hacc, 0, h->hacc_bytes, s));
+  CUDA_TRY(cudaMemsetAsync(h->racc, 0, h->racc_bytes, s));
   CUDA_TRY(cudaStreamSynchronize(s));
   return MK_OK;
 }
@@ -554,7 +570,8 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.down_staged = pl.down_staged;
   p.down_cols = pl.down_cols;
   p.ss_ld = ceil_div(pl.n_hb, 128) * 128;
-  p.e_ld = ceil_div(d.n_experts, 4) * 4;
+  p.e_ld = ceil_div(std::max(d.n_experts, 1), 4) * 4;
+  p.fused = pl.mmax == 1 ? 1 : 0;
   p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit;
   p.attn_ppt = pl.attn_ppt; p.attn_nch_max = pl.attn_nch_max;
   p.tmaps = h->tmaps; p.norms = h->norms;
@@ -562,11 +579,12 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.final_norm = static_cast<const __nv_bfloat16 *>(h->final_norm);
   p.kc = static_cast<__nv_bfloat16 *>(kv.k); p.vc = static_cast<__nv_bfloat16 *>(kv.v);
   p.tokens = tokens; p.positions = positions; p.logits = logits ? logits : h->logits; p.argmax = argmax;
-  p.h = h->h; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
+  p.h = h->h; p.hm = h->hm; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
+  p.hacc = h->hacc; p.racc = h->racc;
   p.xg = h->h + (size_t)kMaxRows * d.d_model;
   p.attn_o = h->attn_o; p.attn_ml = h->attn_ml;
-  p.attn_cnt = h->attn_cnt; p.router_part = h->router_part;
-  p.act_shared = h->act_shared; p.act_routed = h->act_routed; p.y_part = h->y_part;
+  p.attn_cnt = h->attn_cnt;
+  p.act_shared = h->act_shared; p.act_routed = h->act_routed;
   p.am_part = h->am_part; p.rope = h->rope;
   p.counters = h->counters;
   p.epoch = h->epoch; p.error = h->error;
@@ -800,13 +818,8 @@ MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *p
     return fail(MK_ERR_ARG, "draft_len=%d is shorter than n_steps * T = %lld", draft_len, (long long)n_steps * T);
   if ((long long)n_steps * T > h->desc.kv_capacity) return fail(MK_ERR_CAPACITY, "n_steps * T exceeds kv_capacity");
   const size_t need = (size_t)(n_steps + 1) * B + (size_t)(n_steps + 1) * B * T + (size_t)n_steps * B * T;
-  if (need > h->vbuf_ints) {
-    void *nb = nullptr;
-    int rc = halloc(h, &nb, need * sizeof(int32_t));
-    if (rc) return rc;
-    h->vbuf = static_cast<int *>(nb);
-    h->vbuf_ints = need;
-  }
+  if (need > h->vbuf_ints)  // sized at mk_create for every launch the checks above admit
+    return fail(MK_ERR_CAPACITY, "verify buffers: %zu ints needed, %zu held", need, h->vbuf_ints);
   int *vpos = h->vbuf, *vtok = vpos + (size_t)(n_steps + 1) * B, *am = vtok + (size_t)(n_steps + 1) * B * T;
   Params p;
   Plan pl;
@@ -921,6 +934,45 @@ MK_API int mk_debug_inject(mk_handle *h, int32_t fault) {
   return MK_OK;
 }
 
+MK_API int mk_hbm_read_probe(const void *buf, uint64_t bytes, int32_t form, int32_t reps, double *out_gbs,
+                             void *stream) {
+  if (!buf || !out_gbs) return fail(MK_ERR_ARG, "buf and out_gbs are required");
+  if (reinterpret_cast<uintptr_t>(buf) % 16) return fail(MK_ERR_ARG, "buf must be 16-byte aligned");
+  if (form != 0 && form != 1) return fail(MK_ERR_ARG, "form must be 0 (vector loads) or 1 (bulk copies)");
+  if (reps < 1) return fail(MK_ERR_ARG, "reps must be >= 1");
+  const uint64_t unit = form == 0 ? 16 : 32768;
+  const uint64_t used = bytes / unit * unit;
+  if (used < (64ull << 20)) return fail(MK_ERR_ARG, "the probe needs at least 64 MiB (got %llu bytes)",
+                                        (unsigned long long)bytes);
+  int dev = 0, n_sm = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t words = probe_sink_words(n_sm);
+  uint32_t *sink = nullptr;
+  CUDA_TRY(cudaMalloc(&sink, words * sizeof(uint32_t)));
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  cudaError_t e = cudaMemsetAsync(sink, 0, words * sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = launch_read_probe(buf, used, form, n_sm, sink, s);  // warm-up pass
+  if (e == cudaSuccess) e = cudaEventCreate(&e0);
+  if (e == cudaSuccess) e = cudaEventCreate(&e1);
+  if (e == cudaSuccess) e = cudaEventRecord(e0, s);
+  for (int r = 0; r < reps && e == cudaSuccess; ++r) e = launch_read_probe(buf, used, form, n_sm, sink, s);
+  if (e == cudaSuccess) e = cudaEventRecord(e1, s);
+  if (e == cudaSuccess) e = cudaEventSynchronize(e1);
+  float ms = 0.f;
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, e0, e1);
+  uint32_t flag = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&flag, sink + words - 1, sizeof flag, cudaMemcpyDeviceToHost);
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  cudaFree(sink);
+  if (e != cudaSuccess) return fail(MK_ERR_CUDA, "read probe failed: %s", cudaGetErrorString(e));
+  if (flag) return fail(MK_ERR_TIMEOUT, "a bounded wait of the bulk read probe ran out");
+  *out_gbs = (double)used * reps / (ms * 1e-3) / 1e9;
+  return MK_OK;
+}
+
 MK_API int mk_get_stats(mk_handle *h, mk_stats *out, int32_t reset) {
   if (!h || !out) return fail(MK_ERR_ARG, "handle and out are required");
   unsigned long long dev[4] = {0, 0, 0, 0};
@@ -945,25 +997,17 @@ static __device__ __align__(256) unsigned char g_static_scratch[MK_STATIC_SCRATC
 
 namespace {
 
-constexpr int kMaxStaticDevices = 64;
-std::mutex g_static_mu;
-void *g_static_base[kMaxStaticDevices];  // the array's address on each device, once resolved
-
-// Address of the array on `dev` (the current device); resolved on the first
-// call for that device.
+// Address of the array on the current device.  Resolved on every call (a
+// host-side query that allocates nothing), so that a device reset, which
+// reloads the module, can never leave a stale address behind.  The first
+// call on a device may load the module there.
 int static_scratch_base(int dev, unsigned char **out) {
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (dev < 0 || dev >= kMaxStaticDevices)
-    return fail(MK_ERR_UNSUPPORTED, "device %d: the static scratch serves devices 0..%d", dev, kMaxStaticDevices - 1);
-  if (!g_static_base[dev]) {
-    void *p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(MK_ERR_CUDA, "cudaGetSymbolAddress(static scratch) on device %d failed: %s", dev,
-                  cudaGetErrorString(e));
-    g_static_base[dev] = p;
-  }
-  *out = static_cast<unsigned char *>(g_static_base[dev]);
+  void *p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(MK_ERR_CUDA, "cudaGetSymbolAddress(static scratch) on device %d failed: %s", dev,
+                cudaGetErrorString(e));
+  *out = static_cast<unsigned char *>(p);
   return MK_OK;
 }
 
@@ -1007,19 +1051,22 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
   c.take(p.counters, base, sizeof(uint32_t) * (size_t)pl.n_ops * kCounterStride);
   c.take(p.epoch, base, sizeof(uint32_t) * kCounterStride);
   c.take(p.attn_cnt, base, sizeof(uint32_t) * ngrp * kQvp);
+  // fixed-point sums: the kernel clears them after use, but the array may hold
+  // another handle's (or a failed step's) leftovers
+  c.take(p.hacc, base, sizeof(long long) * (size_t)kMaxRows * D);
+  c.take(p.racc, base, sizeof(long long) * (size_t)L * kMaxRows * p.e_ld);
   const size_t zero_bytes = c.used;
   // buffers every step writes before it reads them
   c.take(p.h, base, sizeof(float) * 2 * (size_t)kMaxRows * D);
   p.xg = p.h + (size_t)kMaxRows * D;
+  c.take(p.hm, base, sizeof(float) * (size_t)kMaxRows * D);
   c.take(p.ss, base, sizeof(float) * (size_t)kMaxRows * p.ss_ld);
   c.take(p.qkv, base, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);
   c.take(p.o, base, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
   c.take(p.attn_o, base, sizeof(float) * ngrp * pl.attn_nch_max * kQvp * d.head_dim);
   c.take(p.attn_ml, base, sizeof(float) * ngrp * kQvp * 2 * pl.attn_nch_max);
-  c.take(p.router_part, base, sizeof(float) * (size_t)ceil_div(D, kTileCols) * kMaxRows * p.e_ld);
   c.take(p.act_shared, base, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
   c.take(p.act_routed, base, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
-  c.take(p.y_part, base, sizeof(float) * (size_t)kMaxRows * (d.top_k + 1) * D);
   c.take(p.am_part, base, sizeof(ArgmaxPart) * (size_t)pl.n_warps * kMaxRows);
   if (!out_logits) c.take(p.logits, base, sizeof(float) * (size_t)B * T * d.vocab);
   if (c.used > (size_t)MK_STATIC_SCRATCH_BYTES)

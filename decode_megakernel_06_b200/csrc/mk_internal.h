@@ -37,14 +37,19 @@ constexpr int kQvp = 4;                             // query vectors per attenti
 constexpr int kMaxChunks = 32;                      // CTA KV chunks per (seq, kv head, q group)
 constexpr int kCounterStride = 32;                  // uint32s between counters (128 B)
 
-// Ops of one step: EMBED, then per layer QKV ATTN OPROJ ROUTER SHARED_GU
-// ROUTED_GU DOWN COMBINE, then LMHEAD.
+// Ops of one step: EMBED, then per layer QKV ATTN OPROJ SHARED_GU ROUTED_GU
+// DOWN COMBINE, then LMHEAD.  OPROJ also forms the layer's router logits; the
+// routing itself is computed by every CTA before its routed gate/up units.
 enum OpType : int {
-  OP_EMBED = 0, OP_QKV = 1, OP_ATTN = 2, OP_OPROJ = 3, OP_ROUTER = 4,
-  OP_SHARED_GU = 5, OP_ROUTED_GU = 6, OP_DOWN = 7, OP_COMBINE = 8, OP_LMHEAD = 9
+  OP_EMBED = 0, OP_QKV = 1, OP_ATTN = 2, OP_OPROJ = 3, OP_SHARED_GU = 4,
+  OP_ROUTED_GU = 5, OP_DOWN = 6, OP_COMBINE = 7, OP_LMHEAD = 8
 };
-constexpr int kTraceWords = 8;  // per (op, warp) trace record, as MK_TRACE_WORDS
-constexpr int kOpsPerLayer = 8;
+constexpr int kTraceWords = 12;  // per (op, warp) trace record, as MK_TRACE_WORDS
+constexpr int kOpsPerLayer = 7;
+// Fixed-point scale of the integer accumulators (router logits, expert
+// outputs): a value v is held as round(v * 2^32) in an int64, so that sums
+// are exact integer additions whose result does not depend on their order.
+constexpr int kFixShift = 32;
 
 __host__ __device__ inline int n_ops_for(int L) { return kOpsPerLayer * L + 2; }
 __host__ __device__ inline int op_type_of(int op, int L) {
@@ -59,22 +64,25 @@ __host__ __device__ inline int op_layer_of(int op, int L) {
 __host__ __device__ inline int op_index(int layer, int type) {
   return 1 + kOpsPerLayer * layer + (type - 1);
 }
-// Ops whose completion `op` waits for (-1 = none).
-__host__ __device__ inline void op_deps(int op, int L, int *d0, int *d1) {
+// Ops whose completion `op` waits for (-1 = none).  With `fused` (batch 1),
+// the layer's residual sum is formed by the next op's staging pass from the
+// down projection's accumulator, so the next QKV / LMHEAD waits for DOWN and
+// COMBINE has no work.
+__host__ __device__ inline void op_deps(int op, int L, bool fused, int *d0, int *d1) {
   int t = op_type_of(op, L), l = op_layer_of(op, L);
   *d0 = -1;
   *d1 = -1;
+  const int last = fused ? OP_DOWN : OP_COMBINE;
   switch (t) {
     case OP_EMBED: break;
-    case OP_QKV: *d0 = (l == 0) ? 0 : op_index(l - 1, OP_COMBINE); break;
+    case OP_QKV: *d0 = (l == 0) ? 0 : op_index(l - 1, last); break;
     case OP_ATTN: *d0 = op_index(l, OP_QKV); break;
     case OP_OPROJ: *d0 = op_index(l, OP_ATTN); break;
-    case OP_ROUTER:
-    case OP_SHARED_GU: *d0 = op_index(l, OP_OPROJ); break;
-    case OP_ROUTED_GU: *d0 = op_index(l, OP_OPROJ); *d1 = op_index(l, OP_ROUTER); break;
+    case OP_SHARED_GU:
+    case OP_ROUTED_GU: *d0 = op_index(l, OP_OPROJ); break;
     case OP_DOWN: *d0 = op_index(l, OP_SHARED_GU); *d1 = op_index(l, OP_ROUTED_GU); break;
     case OP_COMBINE: *d0 = op_index(l, OP_DOWN); break;
-    case OP_LMHEAD: *d0 = op_index(L - 1, OP_COMBINE); break;
+    case OP_LMHEAD: *d0 = op_index(L - 1, last); break;
   }
 }
 __host__ __device__ inline bool op_has_tiles(int type) {
@@ -124,7 +132,8 @@ struct alignas(64) Params {
   int down_staged;     // batch 1: each CTA takes a contiguous range of down units and
                        // stages their experts' activations in shared memory
   int ss_ld;           // row stride of the sum-of-squares partials (n_hb rounded up to 128)
-  int e_ld;            // row stride of the router partials (E rounded up to 4)
+  int e_ld;            // row stride of the router logits (E rounded up to 4)
+  int fused;           // batch 1: the residual sum is formed by the next op's staging
   int attn_chunk;      // KV positions per warp; a CTA item covers 8 * attn_chunk
   int attn_qsplit, attn_ppt, attn_nch_max;
   // weights
@@ -137,12 +146,15 @@ struct alignas(64) Params {
   float *logits;
   int *argmax;
   // scratch
-  float *h, *ss, *qkv, *o;
+  float *h;                              // residual entering the layer [8][d]
+  float *hm;                             // residual after the o-projection [8][d]
+  float *ss, *qkv, *o;
   float *xg;                             // M > 1: h * (the next norm's gain), written with h
+  long long *hacc;                       // [8][d] fixed-point sum of the expert outputs
+  long long *racc;                       // [L][8][e_ld] fixed-point router logits (before 1/rms)
   float *attn_o, *attn_ml;   // per-CTA-chunk partials (unnormalised o; max, sum)
   uint32_t *attn_cnt;
-  float *router_part;
-  float *act_shared, *act_routed, *y_part;   // silu(gate) * up per row; down partials
+  float *act_shared, *act_routed;        // silu(gate) * up per row
   ArgmaxPart *am_part;
   const float2 *rope;                    // [cap][hd/2] (cos, sin) of p * theta^(-2i/hd)
   uint32_t *counters, *epoch;
@@ -211,5 +223,11 @@ constexpr int kSampleMaxVocab = 131072;  // 64-bit mass sums and shared memory b
 size_t sample_smem_bytes(int slice);
 cudaError_t launch_top_p(const float *logits, int rows, int vocab, float temperature, float top_p,
                          const double *uniforms, int32_t *out, cudaStream_t stream);
+
+// Read-only HBM probe (mk_probe.cu).  form 0: 16-byte vector loads; form 1:
+// bulk asynchronous copies into shared memory.  sink: probe_sink_words(n_sm)
+// zeroed words; its last word is set if a bounded wait of form 1 ran out.
+size_t probe_sink_words(int n_sm);
+cudaError_t launch_read_probe(const void *buf, size_t bytes, int form, int n_sm, uint32_t *sink, cudaStream_t s);
 
 }  // namespace mk

@@ -152,6 +152,22 @@ MK_INLINE uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
   return old;
 }
 
+// Release-add with no result: the arriving warp does not wait for the reply.
+MK_INLINE void red_add_release(uint32_t *p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Fixed-point accumulation (kFixShift fraction bits in an int64): integer
+// additions are exact and associative, so a sum of many contributions is the
+// same whatever order the warps add them in.
+MK_INLINE long long to_fix(float v) { return __float2ll_rn(v * 4294967296.0f); }
+MK_INLINE float from_fix(long long a) { return static_cast<float>(static_cast<double>(a) * 0x1p-32); }
+static_assert(kFixShift == 32, "to_fix / from_fix scale by 2^32");
+
+MK_INLINE void red_add_fix(long long *p, long long v) {
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 
 MK_INLINE uint64_t now_ns() {
   uint64_t t;
@@ -290,6 +306,9 @@ struct Warp {
   uint64_t *full, *empty;  // per slot: tile landed / tile released
   float *wbuf;
   uint32_t *arrive;
+  float *rpart;                // this warp's router-logit partials of the current layer, [MMAX][kMaxExperts]
+  float *rpart_cta;            // all compute warps' rows, [kConsumers][MMAX][kMaxExperts]
+  int rpart_ld;                // MMAX * kMaxExperts: one warp's rows to the next
   int *attn_prefix;        // this warp's: first item of each sequence, [kMaxRows + 1]
   int *attn_nch;           // this warp's: KV chunks of each sequence, [kMaxRows]
   int step;                // the step (of a multi-step launch) this warp is in
@@ -332,10 +351,11 @@ MK_INLINE void set_error(Warp &w, int code, int op) {
   w.failed = true;
 }
 
-// The layer's router partials are complete once the ROUTER op's counter
-// reaches its target; every lane then re-reads it with acquire semantics.
+// The layer's router logits are complete once the o-projection's counter
+// reaches its target (its units add them up); every lane then re-reads it
+// with acquire semantics.
 MK_INLINE bool routing_ready(const Warp &w, int layer) {
-  const uint32_t *ctr = &w.P->counters[op_index(layer, OP_ROUTER) * kCounterStride];
+  const uint32_t *ctr = &w.P->counters[op_index(layer, OP_OPROJ) * kCounterStride];
   const uint32_t target = w.epoch * static_cast<uint32_t>(w.P->n_cta);
   const uint32_t v = ld_relaxed(ctr);
   const bool ok = __all_sync(0xffffffffu, static_cast<int>(v - target) >= 0);
@@ -343,21 +363,43 @@ MK_INLINE bool routing_ready(const Warp &w, int layer) {
   return ok;
 }
 
+// inv_rms for rows 0..M-1 from the residual producers' partial sums of squares.
+MK_INLINE void compute_inv_rms(const Params &P, int lane, float (&inv)[kMaxRows]) {
+  const int nk = P.ss_ld / 128;  // float4 loads per lane and row (padding is zero)
+#pragma unroll
+  for (int m = 0; m < kMaxRows; ++m) {
+    inv[m] = 0.f;
+    if (m < P.M) {
+      const float4 *row = reinterpret_cast<const float4 *>(P.ss + static_cast<size_t>(m) * P.ss_ld) + lane;
+      float s = 0.f;
+      for (int k0 = 0; k0 < nk; k0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          v[k] = (k0 + k < nk) ? __ldcg(row + 32 * (k0 + k)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s += (v[k].x + v[k].y) + (v[k].z + v[k].w);
+      }
+      s = warp_sum(s);
+      inv[m] = 1.0f / sqrtf(s / static_cast<float>(P.d) + P.eps);
+    }
+  }
+}
+
 // Lane l owns experts 4l..4l+3 and 128+4l..128+4l+3.
 MK_INLINE int expert_of(int lane, int i) { return (i < 4) ? 4 * lane + i : 128 + 4 * lane + (i - 4); }
 
-// The CTA's routing for `layer` (one warp; the caller has seen the router's
-// partials complete).  Per row: logits = the split-K partials summed in a
-// fixed order; k rounds of argmax (ties to the lower expert id); weights =
-// the softmax renormalised over the chosen experts.  Softmax is monotone, so
-// ranking the logits ranks the probabilities, and the full softmax's
-// normaliser cancels in the renormalisation: w_j = e^(z_j - z_max) /
-// sum over chosen i of e^(z_i - z_max).  Every CTA runs this on the same
-// partials and gets the same result.  The code runs once per layer per CTA
-// (cold), so it is kept short.
-__device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int lane, int key) {
+// The CTA's routing for `layer` (one warp; the caller has seen the
+// o-projection complete).  Per row: the router logits z = u / rms(h), u the
+// fixed-point sums of W_r (h * g_ffn) that the o-projection units added up;
+// k rounds of argmax (ties to the lower expert id); weights = the softmax
+// renormalised over the chosen experts.  Softmax is monotone, so ranking the
+// logits ranks the probabilities, and the full softmax's normaliser cancels
+// in the renormalisation: w_j = e^(z_j - z_max) / sum over chosen i of
+// e^(z_i - z_max).  Every CTA runs this on the same sums and gets the same
+// result.  The code runs once per layer per CTA (cold), so it is kept short.
+__device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int lane, int key, int layer) {
   const int E = P.E, K = P.topk;
-  const int nkc = cdiv(P.d, kTileCols);
   constexpr int EPL = 8;
   uint32_t chosen[EPL];  // rows that selected each of this lane's experts
   uint64_t slots[EPL];   // byte m: the selection slot row m gave it
@@ -366,28 +408,25 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
     chosen[i] = 0;
     slots[i] = 0;
   }
+  float inv[kMaxRows];
+  compute_inv_rms(P, lane, inv);
   for (int m = 0; m < P.M; ++m) {
-    float z[EPL];
+    const long long *row = P.racc + (static_cast<size_t>(layer) * kMaxRows + m) * P.e_ld;
+    longlong2 ua[2], ub[2];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) z[i] = 0.f;
-    // up to 8 K-chunks' partials in flight at once
-    for (int k0 = 0; k0 < nkc; k0 += 8) {
-      float4 va[8], vb[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float *row = P.router_part + (static_cast<size_t>(k0 + k) * kMaxRows + m) * P.e_ld;
-        const bool kin = k0 + k < nkc;
-        va[k] = (kin && 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row) + lane)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-        vb[k] = (kin && 128 + 4 * lane < E) ? __ldcg(reinterpret_cast<const float4 *>(row + 128) + lane)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        z[0] += va[k].x; z[1] += va[k].y; z[2] += va[k].z; z[3] += va[k].w;
-        z[4] += vb[k].x; z[5] += vb[k].y; z[6] += vb[k].z; z[7] += vb[k].w;
-      }
+    for (int h = 0; h < 2; ++h) {
+      ua[h] = 4 * lane < E ? __ldcg(reinterpret_cast<const longlong2 *>(row + 4 * lane) + h) : make_longlong2(0, 0);
+      ub[h] = 128 + 4 * lane < E ? __ldcg(reinterpret_cast<const longlong2 *>(row + 128 + 4 * lane) + h)
+                                 : make_longlong2(0, 0);
     }
+    float z[EPL];
+    const long long u[EPL] = {ua[0].x, ua[0].y, ua[1].x, ua[1].y, ub[0].x, ub[0].y, ub[1].x, ub[1].y};
+    float im = 0.f;
+#pragma unroll
+    for (int mm = 0; mm < kMaxRows; ++mm)
+      if (mm == m) im = inv[mm];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) z[i] = im * from_fix(u[i]);
     // the keys of this lane's experts; 0 = not a candidate (absent or taken)
     uint32_t key[EPL];
 #pragma unroll
@@ -459,6 +498,21 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
   __syncwarp();
 }
 
+// The layer's routing statistics and debug copy, written once per (step,
+// layer) by the warp that computed CTA 0's routing (nothing waits for this):
+// the union size into the statistics and, if requested, each row's experts
+// and weights in selection order.
+__device__ __noinline__ void route_publish(const Params &P, const RouteCache *rc, int lane, int layer) {
+  if (lane == 0) atomicAdd(&P.stats[0], static_cast<unsigned long long>(rc->n_union));
+  const int K = P.topk;
+  for (int idx = lane; idx < P.M * K; idx += 32) {
+    const int m = idx / K, j = idx % K;
+    if (P.dbg_ids) P.dbg_ids[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = rc->row_e[m][j];
+    if (P.dbg_w) P.dbg_w[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = rc->row_w[m][j];
+  }
+  __syncwarp();
+}
+
 // Trace: when this warp first found its CTA's routing cache ready for the
 // layer, and whether it filled it (words 6 and 7 of its ROUTED_GU record).
 MK_INLINE void trace_route_cache(const Warp &w, int layer, int filler) {
@@ -487,7 +541,11 @@ MK_INLINE bool route_cache(Warp &w, int layer) {
   if (w.lane == 0) filler = atomicMax(&rc->fill_key, key) < key ? 1 : 0;
   filler = __shfl_sync(0xffffffffu, filler, 0);
   if (filler) {
-    route_compute(*w.P, rc, w.lane, key);
+    route_compute(*w.P, rc, w.lane, key, layer);
+    // once per (step, layer): CTA 0 of the launch that holds the routed gate/up
+    // op (a one-op-per-launch variant recomputes the routing in later launches)
+    const int rgu = op_index(layer, OP_ROUTED_GU);
+    if (w.cta == 0 && w.P->op_begin <= rgu && rgu < w.P->op_end) route_publish(*w.P, rc, w.lane, layer);
   } else {
     const uint64_t t0 = now_ns();
     while (*reinterpret_cast<volatile int *>(&rc->ready_key) != key) {
@@ -515,7 +573,6 @@ MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
     case OP_QKV: return cdiv((P.Hq + 2 * P.Hkv) * P.hd, kRows) * P.qkv_split;
     case OP_ATTN: return w.attn_prefix[P.B];
     case OP_OPROJ: return P.n_hb;
-    case OP_ROUTER: return cdiv(P.E, kRows) * cdiv(P.d, kTileCols);
     case OP_SHARED_GU: return P.Fs / kRows;
     case OP_ROUTED_GU: return n_union(w) * (P.F / kRows);
     case OP_DOWN: return (n_union(w) + (P.Fs > 0 ? 1 : 0)) * P.n_db;
@@ -525,6 +582,9 @@ MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
   return 0;
 }
 
+// This warp's units of an op: u0, u0 + stride, ... (n of them).  Attention
+// items are CTA-wide; a staged down projection takes CTA-contiguous ranges;
+// everything else goes round-robin over the warp slots.
 // A staged (batch 1) down projection deals CTA c the contiguous units
 // [c * total / n_cta, (c + 1) * total / n_cta), warp by warp within the CTA.
 // (cta + 1) * total stays far below 2^31: at most 148 CTAs x 257 segments x
@@ -534,9 +594,6 @@ MK_INLINE void down_cta_range(const Params &P, int cta, int total, int &c0, int 
   c1 = ((cta + 1) * total) / P.n_cta;
 }
 
-// This warp's units of an op: u0, u0 + stride, ... (n of them).  Attention
-// items are CTA-wide; a staged down projection takes CTA-contiguous ranges;
-// everything else goes round-robin over the warp slots.
 MK_INLINE void op_units(const Warp &w, int op, int type, int layer, int &u0, int &stride, int &n) {
   const Params &P = *w.P;
   const int total = op_total_units(w, type, layer);
@@ -555,6 +612,14 @@ MK_INLINE void op_units(const Warp &w, int op, int type, int layer, int &u0, int
     stride = w.nw;
   }
   n = unit_count_of(u0, total, stride);
+}
+
+// Down-projection unit -> segment (routed expert j of the union, 0 .. U-1, or
+// the shared expert, U) and row block.
+MK_INLINE void down_unit_seg(const Warp &w, int unit, int &seg, int &rb) {
+  const Params &P = *w.P;
+  seg = unit / P.n_db;
+  rb = unit - seg * P.n_db;
 }
 
 // QKV unit -> rows [row0, row0 + 4) over tiles [col0, col0 + ntiles * 1024) of
@@ -633,10 +698,13 @@ MK_INLINE int unit_tiles(const Warp &w, int type, int layer, int unit) {
     case OP_LMHEAD: return cdiv(P.d, kTileCols);
     case OP_SHARED_GU:
     case OP_ROUTED_GU: return 2 * cdiv(P.d, kTileCols);
-    case OP_OPROJ: return cdiv(P.Hq * P.hd, kTileCols);
-    case OP_ROUTER: return 1;
+    // the o-projection's tiles, then (with a router) one box of the router's
+    // columns of the unit's rows
+    case OP_OPROJ: return cdiv(P.Hq * P.hd, kTileCols) + (P.E > 0 ? 1 : 0);
     case OP_DOWN: {
-      const int K = (unit / P.n_db) < n_union(w) ? P.F : P.Fs;
+      int seg, rb;
+      down_unit_seg(w, unit, seg, rb);
+      const int K = seg < n_union(w) ? P.F : P.Fs;
       return cdiv(P.down_groups * cdiv(K, kPanel), kPanels);
     }
     case OP_ATTN: return attn_item(P, w.attn_prefix, w.attn_nch, unit, w.wib, w.step).ntiles;
@@ -660,15 +728,13 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
       m0 = lm + MAP_WQKV;
       break;
     }
-    case OP_OPROJ: m0 = lm + MAP_WO; K = P.Hq * P.hd; break;
-    case OP_LMHEAD: m0 = P.tmaps + P.L * MAPS_PER_LAYER; break;
-    case OP_ROUTER: {
-      const int nrb = cdiv(P.E, kRows);
-      row0 = (unit % nrb) * kRows;
-      col0 = (unit / nrb) * kTileCols;
-      m0 = lm + MAP_ROUTER;
+    case OP_OPROJ:
+      m0 = lm + MAP_WO;
+      m2 = lm + MAP_ROUTER;
+      K = P.Hq * P.hd;
+      half = cdiv(K, kTileCols);  // the tile after the o-projection's is the router box
       break;
-    }
+    case OP_LMHEAD: m0 = P.tmaps + P.L * MAPS_PER_LAYER; break;
     case OP_SHARED_GU:
       m0 = lm + MAP_WSGATE;
       m2 = lm + MAP_WSUP;
@@ -685,7 +751,8 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
       break;
     }
     case OP_DOWN: {
-      const int seg = unit / P.n_db, rb = unit % P.n_db;
+      int seg, rb;
+      down_unit_seg(w, unit, seg, rb);
       if (seg < n_union(w)) {
         const int e = w.rc->expert[seg];
         m0 = lm + MAP_WDOWN;
@@ -709,18 +776,30 @@ MK_INLINE void unit_source(Warp &w, int type, int layer, int unit) {
   w.uhalf = half;
 }
 
+// Issue tile t of the warp's current unit into the next ring slot: its boxes
+// as TMA loads completing on the slot's full barrier.
 MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
   const Params &P = *w.P;
   uint8_t *dst = w.ring + w.islot * kSlotBytes;
   uint64_t *bar = &w.full[w.islot];
+  auto expect = [&](uint32_t bytes) {
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(bar, bytes);
+  };
   if (type == OP_ATTN) {
     const AttnItem a = attn_item(P, w.attn_prefix, w.attn_nch, w.iunit, w.wib, w.step);
     const int row = ((layer * P.Bmax + a.b) * P.Hkv + a.g) * P.cap + a.pos0 + t * P.attn_ppt;
     if (w.lane == 0) {
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bar, 2u * kKvBoxBytes);
+      expect(2u * kKvBoxBytes);
       tma_load_2d(dst, &P.kmap, 0, row, bar, w.pol_kv);
       tma_load_2d(dst + kKvBoxBytes, &P.vmap, 0, row, bar, w.pol_kv);
+    }
+  } else if (type == OP_OPROJ && t >= w.uhalf) {
+    // the router's columns [x, x + 8) of all E rows, x the unit's first row
+    // rounded down to 8 (a box of 8 columns x E rows, 16 bytes per row)
+    if (w.lane == 0) {
+      expect(static_cast<uint32_t>(P.E) * 16u);
+      tma_load_2d(dst, w.um2, w.urow0 & ~7, 0, bar, w.pol_w);
     }
   } else if (type == OP_DOWN && P.down_groups > 1) {
     // the unit's boxes run group by group (4 rows each), nbx boxes of 256
@@ -728,8 +807,7 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
     const int nbx = cdiv(w.uK, kPanel), nb = P.down_groups * nbx, b0 = t * kPanels;
     const int nbox = min(kPanels, nb - b0);
     if (w.lane == 0) {
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * kBoxBytes);
+      expect(static_cast<uint32_t>(nbox) * kBoxBytes);
       for (int p = 0; p < nbox; ++p) {
         // box b: group b % 2, column b / 2 (column order) or group b / nbx,
         // column b % nbx (group order)
@@ -747,8 +825,7 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
     const int x0 = w.ucol0 + tt * kTileCols;
     const int nbox = min(kPanels, cdiv(w.uK - x0, kPanel));
     if (w.lane == 0) {
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * kBoxBytes);
+      expect(static_cast<uint32_t>(nbox) * kBoxBytes);
       for (int p = 0; p < nbox; ++p) tma_load_2d(dst + p * kBoxBytes, m, x0 + p * kPanel, y, bar, w.pol_w);
     }
   }
@@ -763,16 +840,30 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
 // activations, so the stream runs ahead across ops and layers; it stops only
 // at a full ring and where the routing is not known yet.  Returns true if it
 // issued a tile or finished the stream.
+// Why feed_more stopped without issuing: a full ring, or an input that the
+// next tile's address or release depends on.
+enum FeedStop : int { FEED_PROGRESS = 0, FEED_RING_FULL = 1, FEED_DEPENDENCY = 2 };
+
 template <bool MULTI>
-MK_INLINE bool feed_more(Warp &w) {
+MK_INLINE int feed_more(Warp &w) {
   const Params &P = *w.P;
   bool progress = false;
+  int stop = FEED_DEPENDENCY;
   while (!w.done_issue && !w.failed) {
     if (w.it < w.in_tiles) {  // the next tile of the current unit
       // sleep on the slot's release rather than polling it: a polling warp
       // shares its scheduler (and instruction cache) with the consumer
-      if (!mbar_wait_hint(&w.empty[w.islot], (w.ephase >> w.islot) & 1u, 2000u)) break;
+      if (!mbar_wait_hint(&w.empty[w.islot], (w.ephase >> w.islot) & 1u, 2000u)) {
+        stop = FEED_RING_FULL;
+        break;
+      }
       issue_tile(w, w.itype, w.ilayer, w.it);
+      if (kTrace && w.P->trace && w.lane == 0) {
+        unsigned long long *tr = w.P->trace + (static_cast<size_t>(w.iop) * w.nw + w.slot) * kTraceWords;
+        const unsigned long long t = now_ns();
+        if (tr[8] == 0) tr[8] = t;
+        tr[9] = t;
+      }
       w.it++;
       progress = true;
       continue;
@@ -833,7 +924,7 @@ MK_INLINE bool feed_more(Warp &w) {
     w.itype = type;
     w.ilayer = layer;
   }
-  return progress;
+  return progress || w.done_issue ? FEED_PROGRESS : stop;
 }
 
 // ---------------------------------------------------------------------------
@@ -879,37 +970,44 @@ MK_INLINE void consume_end(Warp &w) {
   w.cslot = (w.cslot + 1 == w.nslots) ? 0 : w.cslot + 1;
 }
 
-// Wait for `ctr` to reach `target` (bounded).
+// Wait for `ctr` to reach `target` (bounded).  Lane 0 polls with acquire
+// loads, so the read that sees the target is itself the acquire (no second
+// round trip); the __syncwarp after it orders the other lanes' later loads
+// behind it.  The error word and the clock are looked at every 8th poll.
 MK_INLINE bool wait_counter(Warp &w, const uint32_t *ctr, uint32_t target, int op) {
   const Params &P = *w.P;
-  uint64_t t0 = 0;
-  for (int it = 0;; ++it) {
-    // every lane reads the counter (one broadcast transaction); the final
-    // read below is an acquire on every lane
-    const uint32_t v = ld_relaxed(ctr);
-    if (__all_sync(0xffffffffu, static_cast<int>(v - target) >= 0)) break;
-    int err = 0;
-    if (w.lane == 0) err = *reinterpret_cast<volatile const int *>(P.error);
-    if (__shfl_sync(0xffffffffu, err, 0)) {
-      w.failed = true;
-      return false;
-    }
-    int bad = 0;
-    if (w.lane == 0) {
-      const uint64_t t = now_ns();
-      if (t0 == 0) t0 = t;
-      bad = (t - t0 > P.timeout_ns) ? 1 : 0;
-      if (!bad && it > 8) __nanosleep(32);
-    }
-    if (__shfl_sync(0xffffffffu, bad, 0)) {
-      set_error(w, -5, op);
-      return false;
+  int state = 0;  // 1: reached, 2: another warp reported an error, 3: timed out
+  if (w.lane == 0) {
+    uint64_t t0 = 0;
+    for (int it = 0;; ++it) {
+      if (static_cast<int>(ld_acquire(ctr) - target) >= 0) {
+        state = 1;
+        break;
+      }
+      if ((it & 7) == 7) {
+        if (*reinterpret_cast<volatile const int *>(P.error)) {
+          state = 2;
+          break;
+        }
+        const uint64_t t = now_ns();
+        if (t0 == 0) {
+          t0 = t;
+        } else if (t - t0 > P.timeout_ns) {
+          state = 3;
+          break;
+        }
+      }
     }
   }
-  // the counter only grows within a step, so this read also reaches the target
-  (void)ld_acquire(ctr);
+  state = __shfl_sync(0xffffffffu, state, 0);
   __syncwarp();
-  return true;
+  if (state == 1) return true;
+  if (state == 2) {
+    w.failed = true;
+    return false;
+  }
+  set_error(w, -5, op);
+  return false;
 }
 
 // Producer, before the CTA exits: wait (bounded) until every tile it issued
@@ -925,20 +1023,45 @@ MK_INLINE void drain_feed(const Warp &f) {
   }
 }
 
-// Arrive on an op's counter once this warp's units of it are done.  Returns
-// true (on every lane) for the warp whose arrival completed the op grid-wide.
-MK_INLINE bool arrive(Warp &w, int op) {
+// Arrive on an op's counter once this warp's units of it are done.  The
+// CTA's last warp to arrive publishes for the CTA: after the o-projection it
+// first adds the CTA's router-logit sums into the layer's global fixed-point
+// sums (and clears them for the next layer).  Returns true (on every lane) for
+// the warp whose arrival completed the LMHEAD op grid-wide; other ops' counters
+// are bumped without waiting for the reply.
+MK_INLINE bool arrive(Warp &w, int op, int type, int layer) {
   const Params &P = *w.P;
   __syncwarp();
-  int last = 0;
+  int cta_last = 0;
   if (w.lane == 0) {
     // The warp's results (ordered before this by __syncwarp) are released to
     // the CTA; the CTA's last warp acquires them here and releases them, with
     // its own, grid-wide through the counter (release is cumulative).
     const uint32_t old = atom_add_acq_rel_cta(&w.arrive[op], 1u);  // counts on over the launch's steps
-    if (old % kConsumers == kConsumers - 1) {
-      const uint32_t g = atom_add_acq_rel(&P.counters[op * kCounterStride], 1u);
-      last = (g + 1 == w.epoch * static_cast<uint32_t>(P.n_cta)) ? 1 : 0;
+    cta_last = (old % kConsumers == kConsumers - 1) ? 1 : 0;
+  }
+  cta_last = __shfl_sync(0xffffffffu, cta_last, 0);
+  if (!cta_last) return false;
+  if (type == OP_OPROJ && P.E > 0) {
+    // the CTA's router-logit partials: the compute warps' rows summed in a
+    // fixed order, then added into the layer's global fixed-point sums
+    long long *dst = P.racc + static_cast<size_t>(layer) * kMaxRows * P.e_ld;
+    for (int i = w.lane; i < P.M * P.E; i += 32) {
+      const int m = i / P.E, e = i - m * P.E;
+      float sum = 0.f;
+#pragma unroll
+      for (int k = 0; k < kConsumers; ++k) sum += w.rpart_cta[k * w.rpart_ld + m * kMaxExperts + e];
+      if (sum != 0.f) red_add_fix(dst + m * P.e_ld + e, to_fix(sum));
+    }
+    __syncwarp();
+  }
+  int last = 0;
+  if (w.lane == 0) {
+    uint32_t *ctr = &P.counters[op * kCounterStride];
+    if (type == OP_LMHEAD) {
+      last = (atom_add_acq_rel(ctr, 1u) + 1 == w.epoch * static_cast<uint32_t>(P.n_cta)) ? 1 : 0;
+    } else {
+      red_add_release(ctr, 1u);
     }
   }
   last = __shfl_sync(0xffffffffu, last, 0);
@@ -948,6 +1071,16 @@ MK_INLINE bool arrive(Warp &w, int op) {
   }
   __syncwarp();
   return last != 0;
+}
+
+// Clear this warp's share of a layer's global router-logit sums once every CTA
+// has read them (called after the dependency wait of a later op).
+MK_INLINE void clear_router_sums(const Warp &w, int layer) {
+  const Params &P = *w.P;
+  if (P.E == 0) return;
+  long long *buf = P.racc + static_cast<size_t>(layer) * kMaxRows * P.e_ld;
+  const int n = P.M * P.e_ld;
+  for (int i = w.slot * 32 + w.lane; i < n; i += w.nw * 32) buf[i] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -1155,57 +1288,11 @@ MK_INLINE bool gemv_groups(Warp &w, int op, int ngroups, int K, const XS &xs, fl
   return true;
 }
 
-// inv_rms for rows 0..M-1 from the residual producers' partial sums of squares.
-MK_INLINE void compute_inv_rms(const Params &P, int lane, float (&inv)[kMaxRows]) {
-  const int nk = P.ss_ld / 128;  // float4 loads per lane and row (padding is zero)
-#pragma unroll
-  for (int m = 0; m < kMaxRows; ++m) {
-    inv[m] = 0.f;
-    if (m < P.M) {
-      const float4 *row = reinterpret_cast<const float4 *>(P.ss + static_cast<size_t>(m) * P.ss_ld) + lane;
-      float s = 0.f;
-      for (int k0 = 0; k0 < nk; k0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          v[k] = (k0 + k < nk) ? __ldcg(row + 32 * (k0 + k)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) s += (v[k].x + v[k].y) + (v[k].z + v[k].w);
-      }
-      s = warp_sum(s);
-      inv[m] = 1.0f / sqrtf(s / static_cast<float>(P.d) + P.eps);
-    }
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Ops
 // ---------------------------------------------------------------------------
-// New residual rows [row0, row0 + 4): store, the partial sum of squares for
-// the next RMSNorm, the debug copy and, with gx (the next norm's gain, M > 1
-// only), the gained row xg = h * g that the next op's dot products read.
-// val(m, row, r) gives the new value.
-// Lane 4m + r holds row r of activation row m.
+// Lane 4m + r of a GEMV unit's epilogue holds output row r of activation row m.
 static_assert(kRows == 4 && kMaxRows * kRows <= 32, "one lane per (row, residual row)");
-template <class F>
-MK_INLINE void residual_rows(const Params &P, int lane, int unit, int row0, int dbg_layer, const __nv_bfloat16 *gx,
-                             F val) {
-  const int m = lane / kRows, r = lane % kRows, row = row0 + r;
-  const bool live = lane < kRows * P.M;
-  float sq = 0.f;
-  if (live && row < P.d) {
-    const float hn = val(m, row, r);
-    __stcg(P.h + static_cast<size_t>(m) * P.d + row, hn);
-    if (gx) __stcg(P.xg + static_cast<size_t>(m) * P.d + row, hn * __bfloat162float(gx[row]));
-    sq = hn * hn;
-    if (dbg_layer >= 0 && P.dbg_hidden)
-      P.dbg_hidden[(static_cast<size_t>(dbg_layer) * P.max_rows + m) * P.d + row] = hn;
-  }
-  sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-  sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-  if (live && r == 0) __stcg(&P.ss[m * P.ss_ld + unit], sq);
-  __syncwarp();
-}
 
 // New residual rows of whole units, several units per pass when the rows
 // leave lanes free: lane = 4 * (g * M + m) + r takes row r of activation row
@@ -1247,20 +1334,15 @@ MK_INLINE void op_embed(Warp &w, bool gained) {
   });
 }
 
-// h += (sum_s w_s y_s) + shared, in the selection order of each row.
-MK_INLINE void op_combine(Warp &w, int layer, bool gained) {
+// Above batch 1: the residual entering the next layer, h = h_mid + the expert
+// outputs' fixed-point sum (the routing weights are applied by the down
+// units), with x = h * g of the next norm and the sum-of-squares partials.
+MK_INLINE void op_combine(Warp &w, int layer) {
   const Params &P = *w.P;
-  const int S = P.topk + 1;
-  const RouteCache *rt = w.rc;
-  const __nv_bfloat16 *gx = !gained ? nullptr : (layer + 1 < P.L) ? P.norms[2 * (layer + 1)] : P.final_norm;
+  const __nv_bfloat16 *gx = (layer + 1 < P.L) ? P.norms[2 * (layer + 1)] : P.final_norm;
   residual_units(P, w.lane, w.slot, w.nw, layer + 1, gx, [&](int m, int row) {
-    const float *yp = P.y_part + (static_cast<size_t>(m) * S) * P.d + row;
-    float moe = 0.f;
-#pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s)
-      if (s < P.topk) moe += rt->row_w[m][s] * __ldcg(yp + static_cast<size_t>(s) * P.d);
-    const float sh = P.Fs > 0 ? __ldcg(yp + static_cast<size_t>(P.topk) * P.d) : 0.f;
-    return __ldcg(P.h + static_cast<size_t>(m) * P.d + row) + (moe + sh);
+    const size_t i = static_cast<size_t>(m) * P.d + row;
+    return __ldcg(P.hm + i) + from_fix(__ldcg(P.hacc + i));
   });
 }
 
@@ -1324,7 +1406,62 @@ MK_INLINE bool with_dense_x(Warp &w, int type, int layer, const float *xs, Body 
   }
 }
 
-// One unit of a dense GEMV op over all M rows (QKV, OPROJ, ROUTER, LMHEAD).
+// The o-projection unit's epilogue.  Lane 4m + r holds row row0 + r of the new
+// residual of activation row m (h_mid = h + Wo o): it stores it (with, above
+// batch 1, x = h_mid * g_ffn for the expert GEMVs), its square into the
+// sum-of-squares partials, and clears the expert-output accumulator's entry
+// for the layer that follows.  With a router, the unit's last ring slot holds
+// the router's 8 columns around these rows (all E rows): the unit adds its
+// share of the router logits, u[m][e] += sum_r Wr[e][row0 + r] g[row0 + r]
+// h_mid[m][row0 + r], into this warp's partial row in shared memory (lane l
+// owns experts l, l + 32, ..., so the adds need no atomics and follow the
+// warp's unit order).
+template <int MJ>
+MK_INLINE bool oproj_epilogue(Warp &w, int op, int layer, int unit, int row0, float h_old, const float *wb) {
+  const Params &P = *w.P;
+  const int m = w.lane / kRows, r = w.lane % kRows, row = row0 + r;
+  const bool live = w.lane < kRows * P.M && row < P.d;
+  const __nv_bfloat16 *g = P.norms[2 * layer + 1];
+  float hn = 0.f, gx = 0.f, sq = 0.f;
+  if (live) {
+    hn = h_old + wb[r * MJ + m];
+    gx = hn * __bfloat162float(g[row]);
+    const size_t i = static_cast<size_t>(m) * P.d + row;
+    __stcg(P.hm + i, hn);
+    if (!P.fused) __stcg(P.xg + i, gx);
+    __stcg(reinterpret_cast<unsigned long long *>(P.hacc) + i, 0ull);
+    sq = hn * hn;
+  }
+  sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+  if (live && r == 0) __stcg(&P.ss[m * P.ss_ld + unit], sq);
+  if (P.E == 0) return true;
+  const uint8_t *slot = consume_begin(w, op);
+  if (!slot) return false;
+  // lane l takes experts l, l + 32, ...: rows of 16 bytes, the unit's four
+  // columns at byte (row0 & 4) * 2 of each
+  const int ne = cdiv(P.E, 32);
+#pragma unroll 1
+  for (int i = 0; i < ne; ++i) {
+    const int e = w.lane + 32 * i;
+    const uint2 wr = (e < P.E) ? *reinterpret_cast<const uint2 *>(slot + e * 16 + (row0 & 4) * 2) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int mm = 0; mm < MJ; ++mm) {
+      if (mm >= P.M) break;
+      const float x0 = __shfl_sync(0xffffffffu, gx, kRows * mm), x1 = __shfl_sync(0xffffffffu, gx, kRows * mm + 1);
+      const float x2 = __shfl_sync(0xffffffffu, gx, kRows * mm + 2), x3 = __shfl_sync(0xffffffffu, gx, kRows * mm + 3);
+      float u = bf_lo(wr.x) * x0;
+      u = fmaf(bf_hi(wr.x), x1, u);
+      u = fmaf(bf_lo(wr.y), x2, u);
+      u = fmaf(bf_hi(wr.y), x3, u);
+      if (e < P.E) w.rpart[mm * kMaxExperts + e] += u;
+    }
+  }
+  consume_end(w);
+  return true;
+}
+
+// One unit of a dense GEMV op over all M rows (QKV, OPROJ, LMHEAD).
 template <int MMAX, bool XS>
 MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const float (&inv)[kMaxRows],
                           const float *xs, float &am_val, int &am_idx) {
@@ -1334,14 +1471,6 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
   int row0 = unit * kRows, N = 0, col0 = 0, ntiles = 0, K = P.d, qkv_half = 0;
   switch (type) {
     case OP_OPROJ: K = P.Hq * P.hd; ntiles = cdiv(K, kTileCols); N = P.d; break;
-    case OP_ROUTER: {
-      const int nrb = cdiv(P.E, kRows);
-      row0 = (unit % nrb) * kRows;
-      col0 = (unit / nrb) * kTileCols;
-      ntiles = 1;
-      N = P.E;
-      break;
-    }
     case OP_QKV: {
       int half;
       qkv_unit(P, unit, row0, col0, ntiles, half);
@@ -1371,11 +1500,6 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
         __stcg(&P.qkv[(static_cast<size_t>(qkv_half) * kMaxRows + m) * (P.Hq + 2 * P.Hkv) * P.hd + row0 + r],
                im * wb[r * MJ + m]);
       break;
-    case OP_ROUTER:
-      if (live)
-        __stcg(&P.router_part[(static_cast<size_t>(unit / cdiv(P.E, kRows)) * kMaxRows + m) * P.e_ld + row0 + r],
-               im * wb[r * MJ + m]);
-      break;
     case OP_LMHEAD: {
       const float v = im * wb[r * MJ + m];
       if (live) P.logits[static_cast<size_t>(m) * P.V + row0 + r] = v;
@@ -1399,8 +1523,7 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
       break;
     }
     case OP_OPROJ:
-      residual_rows(P, w.lane, unit, row0, -1, XS ? nullptr : P.norms[2 * layer + 1],
-                    [&](int mm, int, int rr) { return h_old + wb[rr * MJ + mm]; });
+      if (!oproj_epilogue<MJ>(w, op, layer, unit, row0, h_old, wb)) return false;
       break;
     default: break;
   }
@@ -1461,12 +1584,13 @@ MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const flo
 }
 
 // One down-projection unit: segment (routed expert j, or the shared expert
-// when j == n_union) x 4 output rows; writes the partial of every row m it
-// serves to y_part[m][slot][row] (slot = selection index, or top_k).
+// when j == n_union) x 4 or 8 output rows, for every row m the segment serves.
 template <int MJ, bool XS>
 MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm) {
   const Params &P = *w.P;
-  const int seg = unit / P.n_db, row0 = (unit % P.n_db) * kRows * P.down_groups;
+  int seg, rb;
+  down_unit_seg(w, unit, seg, rb);
+  const int row0 = rb * kRows * P.down_groups;
   const int U = n_union(w);
   const RouteCache *rt = w.rc;
   XPlain<MJ> xs;
@@ -1498,13 +1622,15 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm)
     ok = gemv_groups<MJ>(w, op, P.down_groups, K, xs, wb);
   }
   if (!ok) return false;
+  // add w * y (w the row's routing weight, 1 for the shared expert) into the
+  // fixed-point sum of the expert outputs of row m
   const int q = w.lane / kRows, r = w.lane % kRows;
   if (w.lane < kRows * xs.n) {
     const int m = row_at<MJ>(xs.row, q);
-    const int s = (seg < U) ? static_cast<int>(rt->kslot[seg][m]) : P.topk;
-    float *dst = P.y_part + (static_cast<size_t>(m) * (P.topk + 1) + s) * P.d;
+    const float wgt = (seg < U) ? rt->row_w[m][rt->kslot[seg][m]] : 1.f;
+    long long *dst = P.hacc + static_cast<size_t>(m) * P.d + row0 + r;
     for (int g = 0; g < P.down_groups; ++g)
-      if (row0 + g * kRows + r < P.d) __stcg(dst + row0 + g * kRows + r, wb[(g * kRows + r) * MJ + q]);
+      if (row0 + g * kRows + r < P.d) red_add_fix(dst + g * kRows, to_fix(wgt * wb[(g * kRows + r) * MJ + q]));
   }
   __syncwarp();
   return true;
@@ -1518,7 +1644,8 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
   if (type == OP_ROUTED_GU) {
     cnt = __popc(w.rc->rowmask[unit / (P.F / kRows)]);
   } else if (type == OP_DOWN) {
-    const int seg = unit / P.n_db;
+    int seg, rb;
+    down_unit_seg(w, unit, seg, rb);
     cnt = seg < n_union(w) ? __popc(w.rc->rowmask[seg]) : P.M;
   } else {
     cnt = P.M;  // shared gate/up
@@ -1590,6 +1717,8 @@ MK_INLINE float reduce_scores8(const float (&p)[kQvp], int dl) {
 struct AttnShared {
   float *o;           // [compute warps][kQvp][hd] partials (the staging row's space)
   float *q;           // [kQvp][hd] the item's query vectors, rotated and scaled
+  __nv_bfloat16 *kn;  // [kMaxRows][hd] this step's new keys (rotated, bf16) inside the item's chunk
+  __nv_bfloat16 *vn;  // [kMaxRows][hd] and values (bf16)
   float *ml;          // [compute warps][kQvp][2]
   uint32_t *rdv;      // rendezvous counter
   uint32_t *seq;      // this warp's rendezvous count
@@ -1607,7 +1736,6 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
   static_assert(QVP == 4, "one query vector per lane pair");
   const int G = P.Hq / P.Hkv;
   const int pos_b = seq_pos(P, a.b, w.step);
-  const int W3 = (P.Hq + 2 * P.Hkv) * HD;
   const int lane = w.lane, pg = lane >> 3, dl = lane & 7, myq = dl >> 1;
   const int d0 = C * dl, d1 = HALF + C * dl;
   float m_run = -INFINITY, l_run = 0.f;
@@ -1636,40 +1764,22 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
     const int my_qv = a.qs * QVP + myq;
     const int lim = my_qv < G * P.T ? pos_b + my_qv / G : -1;
     const int end = a.pos0 + a.npos;
-    const size_t cache_row_base =
-        (static_cast<size_t>(layer) * P.Bmax + a.b) * P.Hkv * P.cap + static_cast<size_t>(a.g) * P.cap;
     for (int tt = 0; tt < a.ntiles; ++tt) {
       uint8_t *slot = const_cast<uint8_t *>(consume_begin(w, op));
       if (!slot) return false;
       const int pos0 = a.pos0 + tt * P.attn_ppt;
       __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(slot);
       __nv_bfloat16 *vs = reinterpret_cast<__nv_bfloat16 *>(slot + kKvBoxBytes);
-      // New positions of this step inside the tile: rotate k, round k and v to
-      // bf16, patch the tile and (once per group) append them to the cache.
+      // New positions of this step inside the tile: patch the tile with the
+      // rotated, bf16-rounded rows the item staged (16 lanes per row each)
       const int lo = max(pos0, pos_b), hi = min(pos0 + P.attn_ppt, pos_b + P.T);
       for (int p = lo; p < hi; ++p) {
-        const int t = p - pos_b, m = a.b * P.T + t;
-        const size_t kq = static_cast<size_t>(m) * W3 + (P.Hq + a.g) * HD;
-        const size_t vq = static_cast<size_t>(m) * W3 + (P.Hq + P.Hkv + a.g) * HD;
-        for (int i = lane; i < HALF; i += 32) {
-          const float x1 = qkv_load(P, kq + i), x2 = qkv_load(P, kq + i + HALF);
-          const float2 cs = __ldg(&P.rope[static_cast<size_t>(p) * HALF + i]);
-          const __nv_bfloat16 k1 = __float2bfloat16_rn(x1 * cs.x - x2 * cs.y);
-          const __nv_bfloat16 k2 = __float2bfloat16_rn(x2 * cs.x + x1 * cs.y);
-          const __nv_bfloat16 v1 = __float2bfloat16_rn(qkv_load(P, vq + i));
-          const __nv_bfloat16 v2 = __float2bfloat16_rn(qkv_load(P, vq + i + HALF));
-          const int r = (p - pos0) * HD;
-          ks[r + i] = k1;
-          ks[r + i + HALF] = k2;
-          vs[r + i] = v1;
-          vs[r + i + HALF] = v2;
-          if (a.qs == 0) {
-            const size_t c = (cache_row_base + p) * HD;
-            P.kc[c + i] = k1;
-            P.kc[c + i + HALF] = k2;
-            P.vc[c + i] = v1;
-            P.vc[c + i + HALF] = v2;
-          }
+        const int t = p - pos_b, r = (p - pos0) * HD;
+        constexpr int V16 = HD / 8;  // 16-byte pieces per row
+        if (lane < 2 * V16) {
+          const int j = lane % V16;
+          const uint4 *srow = reinterpret_cast<const uint4 *>((lane < V16 ? sh.kn : sh.vn) + t * HD);
+          reinterpret_cast<uint4 *>((lane < V16 ? ks : vs) + r)[j] = srow[j];
         }
       }
       if (lo < hi) fence_proxy_async_smem();
@@ -1868,6 +1978,47 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
     } else {
       for (int i = w.lane; i < hd; i += 32) dst[i] = 0.f;
     }
+    // This step's new rows that fall in the item's chunk: rotate k, round k
+    // and v to bf16, keep them for the tile patches and (one query group)
+    // append them to the cache.  Warp v takes new rows v, v + 4, ...
+    const int pos_b = seq_pos(P, a.b, w.step);
+    const int c0 = a.c * P.attn_chunk * kConsumers;
+    const int lo = max(c0, pos_b), hi = min(c0 + P.attn_chunk * kConsumers, pos_b + P.T);
+    const int W3 = (P.Hq + 2 * P.Hkv) * hd;
+    for (int p = lo + w.wib; p < hi; p += kConsumers) {
+      const int t = p - pos_b, m = a.b * P.T + t;
+      const size_t kq = static_cast<size_t>(m) * W3 + (P.Hq + a.g) * hd;
+      const size_t vq = static_cast<size_t>(m) * W3 + (P.Hq + P.Hkv + a.g) * hd;
+      float x1[HALF / 32], x2[HALF / 32], y1[HALF / 32], y2[HALF / 32];
+      float2 cs[HALF / 32];
+#pragma unroll
+      for (int j = 0; j < HALF / 32; ++j) {  // every load of the row in flight at once
+        const int i = w.lane + 32 * j;
+        x1[j] = qkv_load(P, kq + i);
+        x2[j] = qkv_load(P, kq + i + HALF);
+        y1[j] = qkv_load(P, vq + i);
+        y2[j] = qkv_load(P, vq + i + HALF);
+        cs[j] = __ldg(&P.rope[static_cast<size_t>(p) * HALF + i]);
+      }
+      const size_t crow = (((static_cast<size_t>(layer) * P.Bmax + a.b) * P.Hkv + a.g) * P.cap + p) * hd;
+#pragma unroll
+      for (int j = 0; j < HALF / 32; ++j) {
+        const int i = w.lane + 32 * j;
+        const __nv_bfloat16 k1 = __float2bfloat16_rn(x1[j] * cs[j].x - x2[j] * cs[j].y);
+        const __nv_bfloat16 k2 = __float2bfloat16_rn(x2[j] * cs[j].x + x1[j] * cs[j].y);
+        const __nv_bfloat16 v1 = __float2bfloat16_rn(y1[j]), v2 = __float2bfloat16_rn(y2[j]);
+        sh.kn[t * hd + i] = k1;
+        sh.kn[t * hd + i + HALF] = k2;
+        sh.vn[t * hd + i] = v1;
+        sh.vn[t * hd + i + HALF] = v2;
+        if (a.qs == 0) {
+          P.kc[crow + i] = k1;
+          P.kc[crow + i + HALF] = k2;
+          P.vc[crow + i] = v1;
+          P.vc[crow + i + HALF] = v2;
+        }
+      }
+    }
     *sh.seq += kConsumers;
     if (!cta_rendezvous(w, sh.rdv, *sh.seq, op)) return false;
   }
@@ -1902,17 +2053,17 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
       __stcg(ml + P.attn_nch_max + a.c, L);
     }
     // count this CTA's partial of query v; the warp that completes the
-    // (group, v) count merges all of them into o and rewinds the counter
+    // (group, v) count merges all of them into o and rewinds the counter.
+    // Lane 0's acq_rel add releases the warp's partial (ordered before it by
+    // __syncwarp) and, for the last arrival, acquires every other CTA's; the
+    // second __syncwarp orders the other lanes' loads behind it.
     uint32_t *cnt = P.attn_cnt + static_cast<size_t>(grp) * kQvp + v;
     __syncwarp();
     int last = 0;
-    if (w.lane == 0) {
-      __threadfence();
-      last = (atom_add_acq_rel(cnt, 1u) + 1 == static_cast<uint32_t>(a.nch)) ? 1 : 0;
-    }
+    if (w.lane == 0) last = (atom_add_acq_rel(cnt, 1u) + 1 == static_cast<uint32_t>(a.nch)) ? 1 : 0;
     last = __shfl_sync(0xffffffffu, last, 0);
+    __syncwarp();
     if (last) {
-      (void)ld_acquire(cnt);  // every lane observes the completed count
       attn_final_merge<DPL>(P, w.lane, grp, v, a.nch, a.b, a.g);
       __syncwarp();
       if (w.lane == 0) *cnt = 0;
@@ -1923,22 +2074,7 @@ MK_INLINE bool attn_unit(Warp &w, int op, int layer, int item, AttnShared &sh) {
   return true;
 }
 
-// --- router top-k and the final argmax (run by the op's last arriving warp) --
-// Lane l owns experts 4l..4l+3 (slots 0-3) and 128+4l..128+4l+3 (slots 4-7).
-// The warp that completed the router op records the layer's union size in
-// the statistics and, if requested, the routing in the debug buffers (from its
-// CTA's cache; nothing waits for this).
-__device__ __noinline__ void route_publish(const Params &P, const RouteCache *rc, int lane, int layer) {
-  if (lane == 0) atomicAdd(&P.stats[0], static_cast<unsigned long long>(rc->n_union));
-  const int K = P.topk;
-  for (int idx = lane; idx < P.M * K; idx += 32) {
-    const int m = idx / K, j = idx % K;
-    if (P.dbg_ids) P.dbg_ids[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = rc->row_e[m][j];
-    if (P.dbg_w) P.dbg_w[(static_cast<size_t>(layer) * P.max_rows + m) * K + j] = rc->row_w[m][j];
-  }
-  __syncwarp();
-}
-
+// --- the final argmax (run by the LMHEAD op's last arriving warp) -----------
 __device__ __noinline__ void final_argmax(const Params &P, int lane, uint32_t epoch, int step) {
   for (int m = 0; m < P.M; ++m) {
     float bv = -INFINITY;
@@ -2033,32 +2169,71 @@ MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op) {
 // Batch 1: the CTA stages the op's activation row in shared memory once
 // (x = h * g for normed ops, x = o for the o-projection); every warp then
 // reads its columns from there.  All warps take part, with or without units.
-// For normed ops it also sums h^2 over the columns each warp staged into
-// ssp[warp] (a fixed assignment, so the sum below is deterministic).
+// The normed ops' h: the embedding (layer 0's QKV), h_mid (the expert
+// GEMVs), or, for the next layer's QKV and for LMHEAD, the layer's end
+// h_mid + the expert outputs' fixed-point sum; each CTA then also writes its
+// share of that sum (float4 c4 with c4 % n_cta == cta) as the next residual
+// and to the debug copy.  Normed ops also sum h^2 over the columns each warp
+// staged into ssp[warp] (a fixed assignment, so the sum is deterministic).
 MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, float *ssp, uint32_t *cnt, uint32_t &seq, int op) {
   const Params &P = *w.P;
   const bool oproj = type == OP_OPROJ;
+  const bool sum = P.fused && ((type == OP_QKV && layer > 0) || type == OP_LMHEAD);
   const int K = oproj ? P.Hq * P.hd : P.d;
-  const float4 *src = reinterpret_cast<const float4 *>(oproj ? P.o : P.h);
+  const float4 *src = reinterpret_cast<const float4 *>(oproj                                      ? P.o
+                                                       : (type == OP_QKV || type == OP_LMHEAD) && !sum ? P.h
+                                                                                                   : P.hm);
   const __nv_bfloat16 *g = oproj ? nullptr
                            : (type == OP_QKV)    ? P.norms[2 * layer]
                            : (type == OP_LMHEAD) ? P.final_norm
                                                  : P.norms[2 * layer + 1];
+  float *dbg = (sum && P.dbg_hidden) ? P.dbg_hidden + static_cast<size_t>(type == OP_QKV ? layer : P.L) * P.max_rows * P.d
+                                     : nullptr;
+  // four float4 columns per thread in flight at once: the row was just written
+  // by other SMs, so every load is an L2 round trip
+  constexpr int U = 4;
+  const int n4 = K / 4;
   float sq = 0.f;
-  for (int c4 = threadIdx.x; c4 < K / 4; c4 += kConsumerThreads) {
-    float4 v = __ldcg(src + c4);
-    if (g) {
-      sq = fmaf(v.x, v.x, sq);
-      sq = fmaf(v.y, v.y, sq);
-      sq = fmaf(v.z, v.z, sq);
-      sq = fmaf(v.w, v.w, sq);
-      const uint2 gb = __ldg(reinterpret_cast<const uint2 *>(g + 4 * c4));
-      v.x *= bf_lo(gb.x);
-      v.y *= bf_hi(gb.x);
-      v.z *= bf_lo(gb.y);
-      v.w *= bf_hi(gb.y);
+  for (int c0 = threadIdx.x; c0 < n4; c0 += U * kConsumerThreads) {
+    float4 v[U];
+    longlong2 a[U], b[U];
+    uint2 gb[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int c4 = c0 + j * kConsumerThreads;
+      const bool in = c4 < n4;
+      v[j] = in ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      a[j] = (in && sum) ? __ldcg(reinterpret_cast<const longlong2 *>(P.hacc) + 2 * c4) : make_longlong2(0, 0);
+      b[j] = (in && sum) ? __ldcg(reinterpret_cast<const longlong2 *>(P.hacc) + 2 * c4 + 1) : make_longlong2(0, 0);
+      gb[j] = (in && g) ? __ldg(reinterpret_cast<const uint2 *>(g + 4 * c4)) : make_uint2(0u, 0u);
     }
-    reinterpret_cast<float4 *>(xs)[xs_pos4(c4)] = v;
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int c4 = c0 + j * kConsumerThreads;
+      if (c4 >= n4) break;
+      float4 x = v[j];
+      if (sum) {
+        x.x += from_fix(a[j].x);
+        x.y += from_fix(a[j].y);
+        x.z += from_fix(b[j].x);
+        x.w += from_fix(b[j].y);
+        if (c4 % P.n_cta == w.cta) {
+          if (type == OP_QKV) __stcg(reinterpret_cast<float4 *>(P.h) + c4, x);
+          if (dbg) reinterpret_cast<float4 *>(dbg)[c4] = x;
+        }
+      }
+      if (g) {
+        sq = fmaf(x.x, x.x, sq);
+        sq = fmaf(x.y, x.y, sq);
+        sq = fmaf(x.z, x.z, sq);
+        sq = fmaf(x.w, x.w, sq);
+        x.x *= bf_lo(gb[j].x);
+        x.y *= bf_hi(gb[j].x);
+        x.z *= bf_lo(gb[j].y);
+        x.w *= bf_hi(gb[j].y);
+      }
+      reinterpret_cast<float4 *>(xs)[xs_pos4(c4)] = x;
+    }
   }
   if (g) {
     sq = warp_sum(sq);
@@ -2094,7 +2269,17 @@ MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t
           sg < U ? P.act_routed + static_cast<size_t>(sg) * kMaxRows * P.F : P.act_shared);
       const int K = sg < U ? P.F : P.Fs;
       float4 *dst = reinterpret_cast<float4 *>(xs + (sg - seg0) * ld);
-      for (int c4 = threadIdx.x; c4 < K / 4; c4 += kConsumerThreads) dst[xs_pos4(c4)] = __ldcg(src + c4);
+      for (int c0 = threadIdx.x; c0 < K / 4; c0 += 4 * kConsumerThreads) {
+        float4 v[4];  // four loads in flight per thread
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c4 = c0 + j * kConsumerThreads;
+          v[j] = c4 < K / 4 ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (c0 + j * kConsumerThreads < K / 4) dst[xs_pos4(c0 + j * kConsumerThreads)] = v[j];
+      }
     }
   }
   seq += kConsumers;
@@ -2114,7 +2299,7 @@ MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs
   for (int m = 0; m < kMaxRows; ++m) inv[m] = 0.f;
   if (type != OP_OPROJ && type != OP_DOWN && type != OP_ATTN) {
     if constexpr (XS) {
-      inv[0] = staged_inv_rms(P, ssp);  // the row staged for this op (or, for gate/up, by ROUTER)
+      inv[0] = staged_inv_rms(P, ssp);  // the row staged for this op (or, for routed gate/up, by SHARED_GU)
     } else {
       compute_inv_rms(P, w.lane, inv);
     }
@@ -2150,7 +2335,16 @@ MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane, i
   uint64_t t_idle = 0;
   for (int it = 0;; ++it) {
     bool progress = false, all_done = true;
-    if (!mine.done_issue && !mine.failed) progress = feed_more<MULTI>(mine);
+    const uint64_t t_it = (kTrace && P.trace) ? now_ns() : 0;
+    const int iop = mine.iop;
+    int why = FEED_PROGRESS;
+    if (!mine.done_issue && !mine.failed) why = feed_more<MULTI>(mine);
+    progress = why == FEED_PROGRESS;
+    if (kTrace && P.trace && lane == 0 && !progress && iop < P.op_end) {
+      // the producer's idle time on this op, by reason (in the consumer's record)
+      unsigned long long *tr = P.trace + (static_cast<size_t>(iop) * mine.nw + mine.slot) * kTraceWords;
+      tr[why == FEED_RING_FULL ? 11 : 10] += now_ns() - t_it;
+    }
     all_done = mine.done_issue || mine.failed;
     if (all_done) break;
     int stop = 0;
@@ -2193,6 +2387,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   __shared__ float s_attn_ml[kConsumers * kQvp * 2];
   __shared__ Warp s_feed[kConsumers];  // each consumer's tile stream, as its producer keeps it
   __shared__ float s_ssp[kConsumers];  // batch 1: partial sums of h^2 of the staged row
+  __shared__ float s_rpart[kConsumers * MMAX * kMaxExperts];  // the compute warps' router-logit partials
   const int wib = threadIdx.x >> 5;
   const bool consumer = wib < kConsumers;
   // dynamic shared memory: rings | activation row | full and empty barriers |
@@ -2219,6 +2414,9 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.empty = empties + c * S;
   w.wbuf = fbase + c * kWbuf;
   w.arrive = arrive_cnt;
+  w.rpart_cta = s_rpart;
+  w.rpart = s_rpart + (consumer ? wib : 0) * MMAX * kMaxExperts;
+  w.rpart_ld = MMAX * kMaxExperts;
   w.attn_prefix = s_attn_prefix[wib];
   w.attn_nch = s_attn_nch[wib];
   w.step = 0;
@@ -2285,7 +2483,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   }
 
   uint32_t stage_seq = 0;
-  AttnShared ash{xs, xs + kConsumers * kQvp * P.hd, s_attn_ml, &s_stage, &stage_seq};
+  __nv_bfloat16 *knew = reinterpret_cast<__nv_bfloat16 *>(xs + (kConsumers + 1) * kQvp * P.hd);
+  AttnShared ash{xs, xs + kConsumers * kQvp * P.hd, knew, knew + kMaxRows * P.hd, s_attn_ml, &s_stage, &stage_seq};
   const uint32_t epoch0 = w.epoch;
   const int n_steps = MULTI ? P.n_steps : 1;
   for (int step = 0; step < n_steps && !w.failed; ++step) {
@@ -2302,19 +2501,33 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {
     const int type = op_type_of(op, P.L), layer = op_layer_of(op, P.L);
     int d0, d1;
-    op_deps(op, P.L, &d0, &d1);
+    op_deps(op, P.L, P.fused != 0, &d0, &d1);
     const uint32_t target = w.epoch * static_cast<uint32_t>(P.n_cta);
     const uint32_t extra = (op == P.inject_op) ? 1u : 0u;
     if (d0 >= 0 && !wait_counter(w, &P.counters[d0 * kCounterStride], target + extra, op)) break;
     if (d1 >= 0 && !wait_counter(w, &P.counters[d1 * kCounterStride], target, op)) break;
+    if (kTrace && P.trace && w.lane == 0 && type != OP_ROUTED_GU)
+      P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords + 6] = now_ns();
+    // the previous layer's router sums have been read by every CTA (its down
+    // projection is complete): clear them for the next step
+    if (type == OP_OPROJ && layer > 0) clear_router_sums(w, layer - 1);
+    if (type == OP_OPROJ && P.E > 0) {
+      // this warp's router-logit partials start the layer at zero (the CTA's
+      // last warp read the previous layer's before the CTA arrived there)
+      for (int i = w.lane; i < P.M * kMaxExperts; i += 32) w.rpart[i] = 0.f;
+      __syncwarp();
+    }
+    if (type == OP_LMHEAD) clear_router_sums(w, P.L - 1);
     if constexpr (XS) {
-      // ROUTER stages the normed row that SHARED_GU and ROUTED_GU reuse; a
-      // launch that starts at one of those stages it itself
-      const bool stage = type == OP_QKV || type == OP_OPROJ || type == OP_ROUTER || type == OP_LMHEAD ||
-                         ((type == OP_SHARED_GU || type == OP_ROUTED_GU) && op == P.op_begin);
+      // SHARED_GU stages the normed row that ROUTED_GU reuses; a launch that
+      // starts at ROUTED_GU stages it itself
+      const bool stage = type == OP_QKV || type == OP_OPROJ || type == OP_SHARED_GU || type == OP_LMHEAD ||
+                         (type == OP_ROUTED_GU && op == P.op_begin);
       if (stage && !stage_x(w, type, layer, xs, s_ssp, &s_stage, stage_seq, op)) break;
       if (type == OP_DOWN && P.down_staged && !stage_down(w, layer, xs, &s_stage, stage_seq, op)) break;
     }
+    if (kTrace && P.trace && w.lane == 0 && type != OP_ROUTED_GU)
+      P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords + 7] = now_ns();
     if (kTrace && P.trace && w.lane == 0) P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords] = now_ns();
     w.tr_first = w.tr_last = w.tr_wait = 0;
     w.tr_n = 0;
@@ -2322,8 +2535,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     if (type == OP_EMBED) {
       op_embed(w, !XS);
     } else if (type == OP_COMBINE) {
-      ok = route_cache(w, layer);
-      if (ok) op_combine(w, layer, !XS);
+      if (!P.fused) op_combine(w, layer);  // at batch 1 the next op's staging forms the sum
     } else {
       ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, s_ssp, ash, am_val, am_idx);
     }
@@ -2332,7 +2544,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       // lane 4m holds this warp's best (value, index) of row m
       P.am_part[static_cast<size_t>(w.slot) * kMaxRows + w.lane / kRows] = ArgmaxPart{am_val, am_idx};
     }
-    const bool last = arrive(w, op);
+    const bool last = arrive(w, op, type, layer);
     if (kTrace && P.trace && w.lane == 0) {
       unsigned long long *tr = P.trace + (static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords;
       tr[1] = w.tr_first;
@@ -2340,16 +2552,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
       tr[3] = now_ns();
       tr[4] = w.tr_wait;
       tr[5] = static_cast<unsigned long long>(w.tr_n);
-    }
-    if (last && type == OP_ROUTER) {
-      const uint64_t t_topk = (kTrace && P.trace) ? now_ns() : 0;
-      if (!route_cache(w, layer)) break;
-      route_publish(P, w.rc, w.lane, layer);
-      if (kTrace && P.trace && w.lane == 0) {
-        unsigned long long *tr = P.trace + (static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords;
-        tr[6] = t_topk;
-        tr[7] = now_ns();
-      }
     }
     if (last && type == OP_LMHEAD) final_argmax(P, w.lane, w.epoch, w.step);
   }

@@ -138,26 +138,36 @@ typedef struct mk_plan_info {
   int64_t scratch_bytes;   /* device scratch owned by a handle of this shape */
 } mk_plan_info;
 
-/* Ops of one step's schedule: EMBED, then per layer QKV ATTN OPROJ ROUTER
- * SHARED_GU ROUTED_GU DOWN COMBINE, then LMHEAD. */
+/* Ops of one step's schedule: EMBED, then per layer QKV ATTN OPROJ SHARED_GU
+ * ROUTED_GU DOWN COMBINE, then LMHEAD. */
 #define MK_OP_EMBED 0
 #define MK_OP_QKV 1        /* RMSNorm + QKV projection                          */
 #define MK_OP_ATTN 2       /* rotary, KV append, split-K attention, LSE merge   */
-#define MK_OP_OPROJ 3      /* o-projection + residual                           */
-#define MK_OP_ROUTER 4     /* RMSNorm + router logits (split-K partials)        */
-#define MK_OP_SHARED_GU 5  /* shared expert gate/up rows                        */
-#define MK_OP_ROUTED_GU 6  /* routed experts' gate/up rows (union of the batch);
+#define MK_OP_OPROJ 3      /* o-projection + residual; each unit also adds its
+                              rows' share of the router logits (fixed point)   */
+#define MK_OP_SHARED_GU 4  /* shared expert gate/up rows                        */
+#define MK_OP_ROUTED_GU 5  /* routed experts' gate/up rows (union of the batch);
                               each CTA first computes the softmax top-k itself */
-#define MK_OP_DOWN 7       /* down projections, one partial per (row, expert)   */
-#define MK_OP_COMBINE 8    /* weighted sum of the partials + residual           */
-#define MK_OP_LMHEAD 9     /* final RMSNorm + lm_head; last warp: argmax        */
+#define MK_OP_DOWN 6       /* down projections, added into the residual's
+                              fixed-point sum with the routing weights          */
+#define MK_OP_COMBINE 7    /* above one row per step: residual + that sum; at one
+                              row the next op's staging forms it (no work here) */
+#define MK_OP_LMHEAD 8     /* final RMSNorm + lm_head; last warp: argmax        */
 
 /* Create a handle: validates the descriptor, plans the schedule, encodes the
  * weight tensor maps, allocates scratch on the current device.  No kernel
- * runs.  `out` receives the handle (NULL on failure). */
+ * runs.  `out` receives the handle (NULL on failure).
+ * Passage: one of the two calls of the decode-step specification this library
+ * implements, mk_create(model_desc, weight_ptrs); the plan it builds is the
+ * pages' whole-model program with decoupled weight loads (video "700 tok/s on
+ * a 2.8 Trillion Model", key technical takeaways). */
 MK_API int mk_create(const mk_model_desc *desc, const mk_weights *weights, mk_handle **out);
 
 /* One decode step of M = B*T rows (row m = b*T + t).
+ * Passage: the specification's mk_decode_step(tokens, positions, kv_cache,
+ * out_logits, out_argmax, stream), with the handle, B and T added; the step
+ * is the pages' fused decoder (tpu-megakernels README, FAQ on what the
+ * megakernel fuses: attention, MoE, normalisation, residual).
  *   tokens     : device int32 [B*T], ids in [0, vocab)
  *   positions  : device int32 [B], cache index of sequence b's first new token;
  *                0 <= positions[b] and positions[b] + T <= kv_capacity
@@ -283,11 +293,12 @@ MK_API int mk_decode_step_host(mk_handle *h, const int32_t *tokens_host,
  * norm pointers, rotary table, device status word and statistics stay in the
  * handle.  No call allocates or frees memory.
  *
- * The first call on each device resolves the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  The handle's device must be current.  Each call
- * clears the counters that must start at zero (an asynchronous memset on
- * `stream`), then launches the step.
+ * Every call resolves the array's device address (cudaGetSymbolAddress, a
+ * host-side query that allocates nothing) with the handle's device current;
+ * the first call on a device may load the library's device module there, so
+ * make that first call before any stream capture.  Each call clears the
+ * counters and fixed-point sums that must start at zero (an asynchronous
+ * memset on `stream`), then launches the step.
  *
  * Every handle and stream on a device shares the one array: calls whose work
  * overlaps on the GPU race and corrupt each other's results.  Order them on
@@ -301,7 +312,9 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
                                  int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
                                  int32_t *out_argmax, void *stream);
 
-/* Synchronises `stream`, then returns MK_OK or the first device-side error of
+/* Passage: none in the pages (they define no error interface); this call
+ * completes the boundary with the device-side status of bounded waits.
+ * Synchronises `stream`, then returns MK_OK or the first device-side error of
  * the steps since the last call (MK_ERR_TIMEOUT, MK_ERR_DEVICE_CHECK).  An
  * error clears the handle's synchronisation state so the next step starts
  * clean; the failed step's outputs and cache writes are undefined. */
@@ -311,11 +324,12 @@ MK_API int mk_get_device_status(mk_handle *h, void *stream);
  * the op index that failed (or -1). */
 MK_API int mk_last_device_error_op(mk_handle *h);
 
-/* Thread-local message for the last failing call (never NULL). */
+/* Thread-local message for the last failing call (never NULL).  Passage: none
+ * in the pages; part of the boundary's error reporting. */
 MK_API const char *mk_last_error(void);
 
 /* Frees everything the handle owns.  Safe on NULL.  Call after the last step
- * has finished. */
+ * has finished.  Passage: none in the pages; the handle's end of life. */
 MK_API void mk_destroy(mk_handle *h);
 
 /* Switch the execution variant (MK_MEGAKERNEL, MK_MULTIKERNEL,
@@ -325,31 +339,58 @@ MK_API int mk_set_variant(mk_handle *h, int32_t variant);
 /* Bound for every device-side wait, in nanoseconds (default 1e9). */
 MK_API int mk_set_timeout(mk_handle *h, uint64_t timeout_ns);
 
-/* Test/debug outputs, written by every following step (NULL disables):
+/* Passage: none in the pages; the per-layer states these buffers receive are
+ * what the parity tests compare with the oracle's.
+ * Test/debug outputs, written by every following step (NULL disables):
  *   hidden     : device fp32 [n_layers + 1][max_rows][d]: the residual stream
  *                after the embedding and after each layer
  *   expert_ids : device int32 [n_layers][max_rows][top_k], selection order
  *   expert_w   : device fp32  [n_layers][max_rows][top_k], renormalised */
 MK_API int mk_set_debug(mk_handle *h, float *hidden, int32_t *expert_ids, float *expert_w);
 
-/* Arm a fault for the next step (MK_FAULT_*). */
+/* Arm a fault for the next step (MK_FAULT_*).  Passage: none in the pages;
+ * it makes one bounded wait run out so that the error path can be tested
+ * without faulting the GPU. */
 MK_API int mk_debug_inject(mk_handle *h, int32_t fault);
 
 /* Per-op timeline of every following step (NULL disables): device uint64
  * [n_ops][n_cta * warps_per_cta][MK_TRACE_WORDS] per warp slot:
- *   [0] %globaltimer (ns) when the warp finished waiting for the op's inputs,
+ *   [0] %globaltimer (ns) when the warp began the op's units (inputs ready),
  *   [1] when its first weight/KV tile of the op was ready (0: none),
  *   [2] when it finished consuming its last tile of the op (0: none),
  *   [3] when it arrived at the op's completion counter,
  *   [4] ns it spent blocked on tiles that had not landed yet,
  *   [5] tiles it consumed in the op,
- *   [6], [7] ROUTER, the warp that completed it: when it began its CTA's
- *            routing and when it had recorded the statistics; ROUTED_GU:
- *            when this warp first found its CTA's routing ready, and 1 if it
- *            computed it; otherwise zero.
+ *   [6], [7] ROUTED_GU: when this warp first found its CTA's routing
+ *            ready, and 1 if it computed it; other ops: when the warp's wait
+ *            for the op's inputs ended, and when its CTA had staged them
+ *            (the staged activation row of a batch-1 step; else = [6]);
+ *   [8], [9] the warp's TMA-issuing warp: when it issued its first and its
+ *            last tile of the op (0: none),
+ *   [10] ns that issuing warp spent, while on this op, waiting for an input
+ *        its tile addresses or their release depend on (the routing, an
+ *        expert's gate/up units),
+ *   [11] ns it spent, while on this op, waiting for a free ring slot.
  * n_ops and the grid come from mk_plan_describe. */
-#define MK_TRACE_WORDS 8
+#define MK_TRACE_WORDS 12
 MK_API int mk_set_trace(mk_handle *h, uint64_t *trace);
+
+/* Read-only HBM bandwidth probe: the ceiling that the decode step, which only
+ * reads its weights and cache, is measured against beside the copy peak.
+ * Reads the first bytes of `buf` (rounded down to 16 B for form 0, to 32 KiB
+ * for form 1) once per pass and writes nothing but a few words of its own:
+ *   form 0: 16-byte vector loads that bypass L1, 8 in flight per thread, a
+ *           grid of whole waves of resident blocks;
+ *   form 1: bulk asynchronous copies (cp.async.bulk, 32 KiB each, 4 in flight
+ *           per SM) into shared memory, the engine of the step's weight ring.
+ * One untimed pass, then `reps` passes timed with CUDA events on `stream`;
+ * *out_gbs = bytes read / time in GB/s (1e9).  buf: device, 16-byte aligned,
+ * at least 64 MiB (use a buffer well above the 126 MB L2); caller-owned and
+ * unchanged.  Allocates and frees a small result buffer; synchronises the
+ * stream.  Errors: MK_ERR_ARG, MK_ERR_CUDA, MK_ERR_TIMEOUT (a bounded wait of
+ * form 1 ran out). */
+MK_API int mk_hbm_read_probe(const void *buf, uint64_t bytes, int32_t form, int32_t reps, double *out_gbs,
+                             void *stream);
 
 /* Copies the handle's counters; reset != 0 zeroes them afterwards.  Waits for
  * the device (reads a device counter). */

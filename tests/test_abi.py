@@ -78,50 +78,51 @@ def test_validate_rejects(L, field, value, code):
     assert mk.mk_last_error() != "ok"
 
 
-def test_schedule_is_a_dag_with_the_data_dependencies(L):
+@pytest.mark.parametrize("B", [1, 2])
+def test_schedule_is_a_dag_with_the_data_dependencies(L, B):
     """Every op waits only for earlier ops, and for each op the ops producing
-    its inputs are reachable through its waits."""
-    d = _desc(SMALL, kv_capacity=2112)
-    rc, info, ops = mk.mk_plan_describe(d, 148, 1, 1)
+    its inputs are reachable through its waits.  At one row per step (B = 1)
+    the next layer's staging forms the residual sum from the down projection's
+    accumulator, so its QKV waits for DOWN; above, for COMBINE."""
+    d = _desc(SMALL, kv_capacity=2112, max_seqs=B, max_rows=B)
+    rc, info, ops = mk.mk_plan_describe(d, 148, B, 1)
     assert rc == mk.MK_OK, mk.mk_last_error()
     Lyr = SMALL.n_layers
-    assert info.n_ops == len(ops) == 8 * Lyr + 2
+    assert info.n_ops == len(ops) == 7 * Lyr + 2
     names = [mk.OP_NAMES[t] for t, *_ in ops]
     assert names[0] == "EMBED" and names[-1] == "LMHEAD"
-    assert names[1:9] == ["QKV", "ATTN", "OPROJ", "ROUTER", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE"]
+    assert names[1:8] == ["QKV", "ATTN", "OPROJ", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE"]
     idx = {(mk.OP_NAMES[t], l): i for i, (t, l, _, _) in enumerate(ops)}
     reach = []
     for i, (t, layer, d0, d1) in enumerate(ops):
         assert d0 < i and d1 < i
-        deps = [d0, d1]
-        if mk.OP_NAMES[t] == "ROUTED_GU":  # also waits for the routing ROUTER publishes
-            deps.append(idx[("ROUTER", layer)])
         r = set()
-        for dep in deps:
+        for dep in (d0, d1):
             if dep >= 0:
-                assert dep < i
                 r |= {dep} | reach[dep]
         reach.append(r)
+    end = "DOWN" if B == 1 else "COMBINE"
     for l in range(Lyr):
-        prev_h = idx[("EMBED", -1)] if l == 0 else idx[("COMBINE", l - 1)]
+        # the residual entering layer l: the embedding, or the previous layer's end
+        prev_h = [idx[("EMBED", -1)]] if l == 0 else [idx[(end, l - 1)], idx[("OPROJ", l - 1)]]
         need = {
-            "QKV": [prev_h],
+            "QKV": prev_h,
             "ATTN": [idx[("QKV", l)]],
-            "OPROJ": [idx[("ATTN", l)]],
-            "ROUTER": [idx[("OPROJ", l)]],
+            "OPROJ": [idx[("ATTN", l)], idx[("QKV", l)]],
             "SHARED_GU": [idx[("OPROJ", l)]],
-            "ROUTED_GU": [idx[("OPROJ", l)]],
+            "ROUTED_GU": [idx[("OPROJ", l)]],  # router sums complete with the o-projection
             "DOWN": [idx[("SHARED_GU", l)], idx[("ROUTED_GU", l)], idx[("OPROJ", l)]],
-            "COMBINE": [idx[("DOWN", l)], idx[("ROUTER", l)]],
+            "COMBINE": [idx[("DOWN", l)]],
         }
         for name, deps in need.items():
             for dep in deps:
                 assert dep in reach[idx[(name, l)]], (name, l, dep)
-        # writers of h (OPROJ, COMBINE) come after every reader of the previous h
+        # OPROJ rewrites h_mid and clears the expert-output sums: every reader of
+        # the previous layer's (the staging of this QKV, or COMBINE) comes first
         assert idx[("QKV", l)] in reach[idx[("OPROJ", l)]]
-        for reader in ("ROUTER", "SHARED_GU", "ROUTED_GU"):
-            assert idx[(reader, l)] in reach[idx[("COMBINE", l)]] or reader == "ROUTER"
-    assert idx[("COMBINE", Lyr - 1)] in reach[idx[("LMHEAD", -1)]]
+        if l > 0:
+            assert idx[(end, l - 1)] in reach[idx[("OPROJ", l)]]
+    assert idx[(end, Lyr - 1)] in reach[idx[("LMHEAD", -1)]]
 
 
 @pytest.mark.parametrize("model,B,T,cap", [(TINY, 1, 1, 256), (SMALL, 1, 1, 2112),
@@ -191,3 +192,28 @@ def test_sampler_checks_its_arguments_on_the_host(L):
     assert "131072" in mk.mk_last_error()
     kv = mk.mk_kv_cache(None, None)
     assert L.mk_decode_step_sample(None, None, None, 1, 1, kv, None, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
+
+
+def test_torch_wrappers_check_tensors_before_any_launch():
+    """The torch-tensor wrappers hand raw data pointers to the kernels, so they
+    check dtype, layout, size and device first: a float32 or short uniforms
+    vector, or a strided logits view, would otherwise be read past its end."""
+    import torch
+
+    lg = torch.zeros((4, 100), dtype=torch.float32)
+    u = torch.zeros(4, dtype=torch.float64)
+    out = torch.zeros(4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="dtype"):
+        mk.sample_top_p(lg.double(), 1.0, 0.9, u, out)
+    with pytest.raises(ValueError, match="2-D"):
+        mk.sample_top_p(lg.view(-1), 1.0, 0.9, u, out)
+    with pytest.raises(ValueError, match="contiguous"):
+        mk.sample_top_p(lg.t(), 1.0, 0.9, u, out)
+    with pytest.raises(ValueError, match="CUDA|cuda"):
+        mk.sample_top_p(lg, 1.0, 0.9, u, out)  # CPU tensors never reach the library
+    with pytest.raises(ValueError, match="dtype"):
+        mk._need(u.float(), torch.float64, 4, "uniforms")
+    with pytest.raises(ValueError, match="at least 4"):
+        mk._need(u[:3], torch.float64, 4, "uniforms")
+    with pytest.raises(ValueError, match="dtype"):
+        mk._need(out.long(), torch.int32, 4, "out_tokens")

@@ -54,3 +54,14 @@ def test_mid_dense(B):
     s.close()
     assert rep.argmax_checked >= 2
     print(B, rep)
+
+
+def test_dense_full_size():
+    """The benchmark's dense workload at full size (16 layers, d 4096, a
+    14336-wide FFN, vocab 64000; about 8 GB of weights), two whole steps; the
+    oracle fetches each layer's weights from the device."""
+    s = Session(workload("dense", 1), cache_host_weights=False)
+    rep = run_greedy(s, 2)
+    s.close()
+    assert rep.argmax_checked >= 1
+    print(rep)

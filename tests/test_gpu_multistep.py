@@ -12,6 +12,7 @@ import pytest
 import torch
 
 import decode_megakernel_06_b200 as mk
+from oracle import step as ostep
 from synthetic import ModelConfig, Workload, make_context_lengths, make_tokens, workload
 
 from parity import MARGIN, Session
@@ -111,6 +112,32 @@ def test_tiny_launch_follows_the_oracle():
         pos = [p + 1 for p in pos]
     s.close()
     assert checked >= 12, checked
+
+
+def test_small_launch_follows_the_oracle():
+    """The same on the small model (8 layers, d 2048, 64 experts top-4): one
+    launch of 8 greedy steps against the oracle's greedy decode."""
+    wl = workload("small")
+    n = 8
+    s = Session(wl, capacity=wl.kv_capacity() + n)
+    s.dec.set_debug(None, None, None)
+    positions = make_context_lengths(wl)
+    tokens = make_tokens(s.m.vocab, s.B, wl.seed)
+    got_tok, _ = _one_launch(s, tokens, positions, n)
+    checked = 0
+    tok, pos = list(tokens), list(positions)
+    for i in range(n):
+        ref = s.oracle_step(tok, pos)
+        top2 = np.sort(ref.logits[0])[-2:]
+        # stop at the first near tie of the argmax or of any layer's routing
+        if top2[1] - top2[0] <= MARGIN or ostep.router_margins(ref.router_logits, s.m.top_k).min() <= MARGIN:
+            break
+        assert int(got_tok[i, 0]) == int(ref.argmax[0]), f"step {i}: {got_tok[i, 0]} vs {ref.argmax[0]}"
+        checked += 1
+        tok = [int(ref.argmax[0])]
+        pos = [p + 1 for p in pos]
+    s.close()
+    assert checked >= 2, checked
 
 
 def test_launch_rejects_bad_arguments():

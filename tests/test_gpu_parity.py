@@ -155,8 +155,15 @@ def test_invalid_inputs_are_rejected_on_device():
     bad_pos = torch.tensor([s.cap], dtype=torch.int32, device=dev)
     assert s.dec.step(ok_tok, bad_pos, 1, 1, s.k, s.v, s.logits, s.argmax) == mk.MK_OK
     assert s.dec.status() == mk.MK_ERR_DEVICE_CHECK
-    # host-side capacity checks
-    assert s.dec.step(ok_tok, pos, 2, 1, s.k, s.v, s.logits, s.argmax) == mk.MK_ERR_CAPACITY
+    # host-side capacity checks of the library itself (the torch wrapper would
+    # already refuse the one-token buffer for B = 2)
+    kv = mk.mk_kv_cache(s.k.data_ptr(), s.v.data_ptr())
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = mk.mk_decode_step(s.dec.h, ok_tok.data_ptr(), pos.data_ptr(), 2, 1, kv, s.logits.data_ptr(),
+                           s.argmax.data_ptr(), stream)
+    assert rc == mk.MK_ERR_CAPACITY
+    with pytest.raises(ValueError):
+        s.dec.step(ok_tok, pos, 2, 1, s.k, s.v, s.logits, s.argmax)
     # and the handle still works
     rep = run_greedy(s, 2)
     s.close()

@@ -188,3 +188,57 @@ def test_largest_row_sums_without_overflow():
     assert s.nucleus == osample.MAX_VOCAB // 4 and s.token == osample.MAX_VOCAB // 8
     with pytest.raises(ValueError):
         osample.sample_top_p(np.zeros(osample.MAX_VOCAB + 1, np.float32), 1.0, 0.5, 0.5)
+
+
+def test_fixed_point_nucleus_is_the_real_valued_one():
+    """The fixed-point decisions (masses rounded to 2^-46, integer sums) give
+    the nucleus and the token that exact real arithmetic on the same fp64
+    probabilities gives, wherever the real boundary is not within the
+    quantisation's reach: each mass moves by at most half a unit, so a sum of
+    V masses by at most V/2 units (V * 2^-47 in units of the largest p), and
+    the fp64 products top_p * Q and u * S add a relative 2^-53 each."""
+    from fractions import Fraction
+
+    rng = np.random.default_rng(2024)
+    checked = skipped = 0
+    for it in range(120):
+        V = int(rng.choice([7, 31, 200, 1000]))
+        sigma = float(rng.choice([0.3, 1.0, 3.0]))
+        T = float(rng.choice([0.5, 1.0, 2.0]))
+        top_p = float(rng.choice([0.1, 0.5, 0.9, 0.99]))
+        u = float(rng.random())
+        l = (rng.standard_normal(V) * sigma).astype(np.float32)
+        got = osample.sample_top_p(l, T, top_p, u)
+        # exact rationals of the fp64 probabilities (the largest is exactly 1)
+        l64 = l.astype(np.float64)
+        p = np.exp((l64 - l64.max()) * (1.0 / float(np.float32(T))))
+        F = [Fraction(float(x)) for x in p]
+        total = sum(F)
+        order = np.argsort(-l64, kind="stable")
+        need = Fraction(float(np.float32(top_p))) * total
+        cum, k = Fraction(0), None
+        cums = []
+        for j, t in enumerate(order):
+            cum += F[t]
+            cums.append(cum)
+            if k is None and cum >= need:
+                k = j + 1
+        eps = Fraction(V, 2 ** 47) + total * Fraction(1, 2 ** 52)
+        near = abs(cums[k - 1] - need) <= eps or (k >= 2 and abs(cums[k - 2] - need) <= eps)
+        if near:
+            skipped += 1
+            continue
+        assert got.nucleus == k, (it, got.nucleus, k)
+        S = cums[k - 1]
+        y = Fraction(u) * S
+        acc, tok, gap = Fraction(0), None, None
+        for t in sorted(int(x) for x in order[:k]):
+            lo, acc = acc, acc + F[t]
+            if tok is None and acc > y:
+                tok, gap = t, min(y - lo, acc - y)
+        if gap <= eps + S * Fraction(1, 2 ** 52):
+            skipped += 1
+            continue
+        assert got.token == tok, (it, got.token, tok)
+        checked += 1
+    assert checked >= 100 and skipped <= 20, (checked, skipped)
