@@ -114,38 +114,56 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   p.n_cta = n_sm;
   p.n_warps = n_sm * kConsumers;
   // Attention items are CTA-wide: each of the compute warps takes attn_chunk KV
-  // positions of an item.  About one item per CTA, warp chunks a multiple of
-  // the tile height, and at most kMaxChunks items per (sequence, kv head,
-  // query group) so that one merge level combines them.
-  long long total = (long long)B * d.n_kv_heads * p.attn_qsplit * d.kv_capacity;
-  int c = (int)((total + p.n_warps - 1) / p.n_warps);
-  c = std::max(c, ceil_div(d.kv_capacity, kMaxChunks * kConsumers));
-  c = std::max(c, p.attn_ppt);
-  c = ceil_div(c, p.attn_ppt) * p.attn_ppt;
-  p.attn_chunk = c;
+  // positions of an item, a multiple of the tile height, with at most
+  // kMaxChunks items per (sequence, kv head, query group) so that one merge
+  // level combines them.  The chunk minimises the busiest CTA's time, taking
+  // every sequence at the cache's capacity: rounds of items over the CTAs x
+  // (tiles per warp + kItemCost, the fixed cost of an item -- query staging
+  // and the merges -- in tile times).  A chunk just under an even split can
+  // leave a second round of items for a few CTAs, which costs more than a
+  // somewhat larger chunk.
+  {
+    constexpr long long kItemCost = 3;
+    const long long seqs = (long long)B * d.n_kv_heads * p.attn_qsplit;
+    const int c_min = std::max(p.attn_ppt, ceil_div(d.kv_capacity, kMaxChunks * kConsumers));
+    int best_c = 0;
+    long long best_cost = 0;
+    for (int c = ceil_div(c_min, p.attn_ppt) * p.attn_ppt; c <= std::max(c_min, d.kv_capacity) + p.attn_ppt;
+         c += p.attn_ppt) {
+      const long long items = seqs * ceil_div(d.kv_capacity, c * kConsumers);
+      const long long cost = ((items + n_sm - 1) / n_sm) * (c / p.attn_ppt + kItemCost);
+      if (best_c == 0 || cost < best_cost) {
+        best_c = c;
+        best_cost = cost;
+      }
+    }
+    p.attn_chunk = best_c;
+  }
+  const int c = p.attn_chunk;
   p.attn_nch_max = ceil_div(d.kv_capacity, c * kConsumers);
   p.n_ops = n_ops_for(d.n_layers);
   // shared-memory row: the staged activations (batch 1) or the attention
   // warps' partials and the item's query vectors, whichever is larger
   // (whole 256-column panels: the staged layout permutes columns within one)
   p.xs_floats = std::max((kConsumers + 1) * kQvp * d.head_dim + kMaxRows * d.head_dim,  // + new bf16 K/V rows
-                         kernel_stages_x(p.mmax) ? ceil_div(std::max(d.d_model, d.n_q_heads * d.head_dim), kPanel) * kPanel : 0);
+                         kernel_stages_x(p.mmax) ? p.mmax * panel_ld(std::max(d.d_model, d.n_q_heads * d.head_dim)) : 0);
   // Batch 1 down projection: a CTA's contiguous range of units spans at most
   // 1 + ceil(range / row blocks) experts; their activations must fit the
   // shared-memory row.
   p.down_staged = 0;
-  if (kernel_stages_x(p.mmax)) {
+  if (p.mmax == 1) {
     const int n_db = p.n_hb / p.down_groups;
     const int segs = std::min(d.n_experts, d.top_k) + (d.shared_ffn > 0 ? 1 : 0);
     const int per_cta = ceil_div(segs * n_db, p.n_cta);
     const int span = 1 + ceil_div(per_cta, n_db);
     const int fmax = std::max(d.expert_ffn, d.shared_ffn);
-    p.down_staged = (std::min(span, segs) * ceil_div(fmax, kPanel) * kPanel <= p.xs_floats) ? 1 : 0;
+    p.down_staged = (std::min(span, segs) <= kMaxStageSegs && std::min(span, segs) * panel_ld(fmax) <= p.xs_floats) ? 1 : 0;
   }
-  // with one or two rows per step the two groups of an 8-row down unit can
-  // keep separate accumulators, so its tiles go column by column
-  p.down_cols = (p.down_groups == 2 && p.mmax <= 2) ? 1 : 0;
-  p.smem = step_smem_bytes(p.n_ops, p.xs_floats, p.mmax);
+  // an 8-row down unit of one or two activation rows keeps both groups' sums
+  // at once, so its tiles go column by column (each column's activations
+  // serve both groups); units of more rows go group by group
+  p.down_cols = (p.down_groups == 2) ? 1 : 0;
+  p.smem = step_smem_bytes(p.n_ops, p.xs_floats, p.mmax, ceil_div(std::max(d.n_experts, 1), 4) * 4);
   return p;
 }
 
@@ -185,8 +203,8 @@ struct mk_handle {
   std::vector<void *> allocs;
   CUtensorMap *tmaps;
   const __nv_bfloat16 **norms;
-  float *h, *hm, *ss, *qkv, *o, *attn_o, *attn_ml, *act_shared, *act_routed, *logits;
-  long long *hacc, *racc;
+  float *h, *hm, *qkv, *o, *attn_o, *attn_ml, *act_shared, *act_routed, *logits;
+  long long *hacc, *racc, *ssq;
   size_t hacc_bytes, racc_bytes;
   uint32_t *attn_cnt, *counters, *epoch;
   ArgmaxPart *am_part;
@@ -300,7 +318,7 @@ MK_API int mk_plan_describe(const mk_model_desc *desc, int32_t n_sm, int32_t B, 
   }
   for (int i = 0; i < p.n_ops && i < cap; ++i) {
     int d0, d1;
-    op_deps(i, desc->n_layers, p.mmax == 1, &d0, &d1);
+    op_deps(i, desc->n_layers, &d0, &d1);
     if (op_types) op_types[i] = op_type_of(i, desc->n_layers);
     if (op_layers) op_layers[i] = op_layer_of(i, desc->n_layers);
     if (op_dep0) op_dep0[i] = d0;
@@ -389,21 +407,21 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   const int umax = std::min(d.n_experts, std::min(d.max_rows, kMaxRows) * d.top_k);
   HALLOC(h->tmaps, sizeof(CUtensorMap) * (size_t)(L * MAPS_PER_LAYER + 1));
   HALLOC(h->norms, sizeof(void *) * 2 * L);
-  HALLOC(h->h, sizeof(float) * 2 * (size_t)kMaxRows * D);  // h, then h * gain (xg)
+  HALLOC(h->h, sizeof(float) * (size_t)kMaxRows * (D + panel_ld(D)));  // h, then h * gain (xg)
   HALLOC(h->hm, sizeof(float) * (size_t)kMaxRows * D);
   h->hacc_bytes = sizeof(long long) * (size_t)kMaxRows * D;
   HALLOC(h->hacc, h->hacc_bytes);
   h->racc_bytes = sizeof(long long) * (size_t)L * kMaxRows * (ceil_div(std::max(d.n_experts, 1), 4) * 4);
   HALLOC(h->racc, h->racc_bytes);
-  HALLOC(h->ss, sizeof(float) * (size_t)kMaxRows * ceil_div(ceil_div(D, kRows), 128) * 128);
+  HALLOC(h->ssq, sizeof(long long) * 2 * kMaxRows);
   HALLOC(h->qkv, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);  // [K half][row][QKVW]
-  HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
+  HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * panel_ld(d.n_q_heads * d.head_dim));
   HALLOC(h->attn_o, sizeof(float) * s.attn_o);
   HALLOC(h->attn_ml, sizeof(float) * s.attn_ml);
   h->attn_cnt_bytes = sizeof(uint32_t) * s.attn_cnt;
   HALLOC(h->attn_cnt, h->attn_cnt_bytes);
-  HALLOC(h->act_shared, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
-  HALLOC(h->act_routed, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
+  HALLOC(h->act_shared, sizeof(float) * (size_t)kMaxRows * panel_ld(std::max(d.shared_ffn, 1)));
+  HALLOC(h->act_routed, sizeof(float) * (size_t)umax * kMaxRows * panel_ld(std::max(d.expert_ffn, 1)));
   HALLOC(h->am_part, sizeof(ArgmaxPart) * (size_t)NW * kMaxRows);
   HALLOC(h->rope, sizeof(float2) * (size_t)d.kv_capacity * (d.head_dim / 2));
   h->counters_bytes = sizeof(uint32_t) * (size_t)n_ops * kCounterStride;
@@ -526,6 +544,7 @@ static int reset_sync_state(mk_handle *h, cudaStream_t s) {
   // a failed step may leave partial fixed-point sums behind
   CUDA_TRY(cudaMemsetAsync(h->hacc, 0, h->hacc_bytes, s));
   CUDA_TRY(cudaMemsetAsync(h->racc, 0, h->racc_bytes, s));
+  CUDA_TRY(cudaMemsetAsync(h->ssq, 0, sizeof(long long) * 2 * kMaxRows, s));
   CUDA_TRY(cudaStreamSynchronize(s));
   return MK_OK;
 }
@@ -569,9 +588,9 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.n_db = pl.n_hb / pl.down_groups;
   p.down_staged = pl.down_staged;
   p.down_cols = pl.down_cols;
-  p.ss_ld = ceil_div(pl.n_hb, 128) * 128;
   p.e_ld = ceil_div(std::max(d.n_experts, 1), 4) * 4;
-  p.fused = pl.mmax == 1 ? 1 : 0;
+  p.ldx = panel_ld(d.d_model); p.ldo = panel_ld(d.n_q_heads * d.head_dim);
+  p.ldf = panel_ld(std::max(d.expert_ffn, 1)); p.ldfs = panel_ld(std::max(d.shared_ffn, 1));
   p.attn_chunk = pl.attn_chunk; p.attn_qsplit = pl.attn_qsplit;
   p.attn_ppt = pl.attn_ppt; p.attn_nch_max = pl.attn_nch_max;
   p.tmaps = h->tmaps; p.norms = h->norms;
@@ -579,7 +598,7 @@ static int fill_params(mk_handle *h, const int32_t *tokens, const int32_t *posit
   p.final_norm = static_cast<const __nv_bfloat16 *>(h->final_norm);
   p.kc = static_cast<__nv_bfloat16 *>(kv.k); p.vc = static_cast<__nv_bfloat16 *>(kv.v);
   p.tokens = tokens; p.positions = positions; p.logits = logits ? logits : h->logits; p.argmax = argmax;
-  p.h = h->h; p.hm = h->hm; p.ss = h->ss; p.qkv = h->qkv; p.o = h->o;
+  p.h = h->h; p.hm = h->hm; p.ssq = h->ssq; p.qkv = h->qkv; p.o = h->o;
   p.hacc = h->hacc; p.racc = h->racc;
   p.xg = h->h + (size_t)kMaxRows * d.d_model;
   p.attn_o = h->attn_o; p.attn_ml = h->attn_ml;
@@ -1055,18 +1074,18 @@ MK_API int mk_decode_step_static(mk_handle *h, const int32_t *tokens, const int3
   // another handle's (or a failed step's) leftovers
   c.take(p.hacc, base, sizeof(long long) * (size_t)kMaxRows * D);
   c.take(p.racc, base, sizeof(long long) * (size_t)L * kMaxRows * p.e_ld);
+  c.take(p.ssq, base, sizeof(long long) * 2 * kMaxRows);
   const size_t zero_bytes = c.used;
   // buffers every step writes before it reads them
-  c.take(p.h, base, sizeof(float) * 2 * (size_t)kMaxRows * D);
+  c.take(p.h, base, sizeof(float) * (size_t)kMaxRows * (D + panel_ld(D)));
   p.xg = p.h + (size_t)kMaxRows * D;
   c.take(p.hm, base, sizeof(float) * (size_t)kMaxRows * D);
-  c.take(p.ss, base, sizeof(float) * (size_t)kMaxRows * p.ss_ld);
   c.take(p.qkv, base, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);
-  c.take(p.o, base, sizeof(float) * (size_t)kMaxRows * d.n_q_heads * d.head_dim);
+  c.take(p.o, base, sizeof(float) * (size_t)kMaxRows * panel_ld(d.n_q_heads * d.head_dim));
   c.take(p.attn_o, base, sizeof(float) * ngrp * pl.attn_nch_max * kQvp * d.head_dim);
   c.take(p.attn_ml, base, sizeof(float) * ngrp * kQvp * 2 * pl.attn_nch_max);
-  c.take(p.act_shared, base, sizeof(float) * (size_t)kMaxRows * std::max(d.shared_ffn, 1));
-  c.take(p.act_routed, base, sizeof(float) * (size_t)umax * kMaxRows * d.expert_ffn);
+  c.take(p.act_shared, base, sizeof(float) * (size_t)kMaxRows * panel_ld(std::max(d.shared_ffn, 1)));
+  c.take(p.act_routed, base, sizeof(float) * (size_t)umax * kMaxRows * panel_ld(std::max(d.expert_ffn, 1)));
   c.take(p.am_part, base, sizeof(ArgmaxPart) * (size_t)pl.n_warps * kMaxRows);
   if (!out_logits) c.take(p.logits, base, sizeof(float) * (size_t)B * T * d.vocab);
   if (c.used > (size_t)MK_STATIC_SCRATCH_BYTES)

@@ -19,10 +19,10 @@ constexpr int kWarpsPerCta = kConsumers + kProducers;
 constexpr int kThreads = kWarpsPerCta * 32;
 constexpr int kConsumerThreads = kConsumers * 32;
 constexpr int kMaxSlots = 6;                        // ring slots per consumer, at most
-// Ring slots per consumer for a kernel of up to `mmax` rows: six at batch 1;
-// four above, where the smaller shared-memory carve-out leaves L1 room for
-// the activation rows that every warp re-reads.
-__host__ __device__ constexpr int ring_slots(int mmax) { return mmax == 1 ? 6 : 4; }
+// Ring slots per consumer for a kernel of up to `mmax` rows: what shared
+// memory leaves beside the staged activation rows (mmax rows of up to 4096
+// floats): six at one row, four at two and four rows, two at eight.
+__host__ __device__ constexpr int ring_slots(int mmax) { return mmax == 1 ? 6 : mmax <= 4 ? 4 : 2; }
 constexpr int kSlotBytes = 8192;                    // one tile: four 2 KB weight boxes
 constexpr int kPanel = 256;                         // columns per weight box
 constexpr int kRows = 4;                            // rows per weight box, tile and unit
@@ -36,6 +36,10 @@ constexpr int kMaxTopK = 16;
 constexpr int kQvp = 4;                             // query vectors per attention item
 constexpr int kMaxChunks = 32;                      // CTA KV chunks per (seq, kv head, q group)
 constexpr int kCounterStride = 32;                  // uint32s between counters (128 B)
+constexpr int kMaxStageSegs = 4;                    // experts a CTA's staged down range may span
+// Row stride of an activation row of k columns: whole 256-column panels (the
+// rows are stored panel-permuted, see xs_pos4 in mk_kernel.cu).
+__host__ __device__ constexpr int panel_ld(int k) { return (k + kPanel - 1) / kPanel * kPanel; }
 
 // Ops of one step: EMBED, then per layer QKV ATTN OPROJ SHARED_GU ROUTED_GU
 // DOWN COMBINE, then LMHEAD.  OPROJ also forms the layer's router logits; the
@@ -64,15 +68,12 @@ __host__ __device__ inline int op_layer_of(int op, int L) {
 __host__ __device__ inline int op_index(int layer, int type) {
   return 1 + kOpsPerLayer * layer + (type - 1);
 }
-// Ops whose completion `op` waits for (-1 = none).  With `fused` (batch 1),
-// the layer's residual sum is formed by the next op's staging pass from the
-// down projection's accumulator, so the next QKV / LMHEAD waits for DOWN and
-// COMBINE has no work.
-__host__ __device__ inline void op_deps(int op, int L, bool fused, int *d0, int *d1) {
+// Ops whose completion `op` waits for (-1 = none).
+__host__ __device__ inline void op_deps(int op, int L, int *d0, int *d1) {
   int t = op_type_of(op, L), l = op_layer_of(op, L);
   *d0 = -1;
   *d1 = -1;
-  const int last = fused ? OP_DOWN : OP_COMBINE;
+  const int last = OP_COMBINE;
   switch (t) {
     case OP_EMBED: break;
     case OP_QKV: *d0 = (l == 0) ? 0 : op_index(l - 1, last); break;
@@ -127,13 +128,12 @@ struct alignas(64) Params {
   int qkv_split;       // QKV units cover 1 or 2 halves of K; the halves are summed by their reader
   int down_groups;     // 4-row groups per down-projection unit (1 or 2)
   int n_db;            // down-projection row blocks (n_hb / down_groups)
-  int down_cols;       // 8-row down units: boxes ordered column by column, both groups
-                       // per column (1-2 rows per step), else group by group
+  int down_cols;       // 8-row down units of 1-2 activation rows: boxes ordered column
+                       // by column, both groups per column (others group by group)
   int down_staged;     // batch 1: each CTA takes a contiguous range of down units and
                        // stages their experts' activations in shared memory
-  int ss_ld;           // row stride of the sum-of-squares partials (n_hb rounded up to 128)
   int e_ld;            // row stride of the router logits (E rounded up to 4)
-  int fused;           // batch 1: the residual sum is formed by the next op's staging
+  int ldx, ldo, ldf, ldfs;  // activation row strides (panel_ld of d, Hq*hd, F, Fs)
   int attn_chunk;      // KV positions per warp; a CTA item covers 8 * attn_chunk
   int attn_qsplit, attn_ppt, attn_nch_max;
   // weights
@@ -148,13 +148,18 @@ struct alignas(64) Params {
   // scratch
   float *h;                              // residual entering the layer [8][d]
   float *hm;                             // residual after the o-projection [8][d]
-  float *ss, *qkv, *o;
-  float *xg;                             // M > 1: h * (the next norm's gain), written with h
+  float *qkv;
+  float *o;                              // attention output, panel-permuted rows [8][ldo]
+  long long *ssq;                        // [2][8] fixed-point sums of h^2: the residual entering
+                                         // the layer, then the residual after the o-projection
+  float *xg;                             // h * (the next norm's gain), written with h,
+                                         // panel-permuted rows [8][ldx]
   long long *hacc;                       // [8][d] fixed-point sum of the expert outputs
   long long *racc;                       // [L][8][e_ld] fixed-point router logits (before 1/rms)
   float *attn_o, *attn_ml;   // per-CTA-chunk partials (unnormalised o; max, sum)
   uint32_t *attn_cnt;
-  float *act_shared, *act_routed;        // silu(gate) * up per row
+  float *act_shared, *act_routed;        // silu(gate) * up per row, panel-permuted rows:
+                                         // [8][ldfs] and [union][8][ldf]
   ArgmaxPart *am_part;
   const float2 *rope;                    // [cap][hd/2] (cos, sin) of p * theta^(-2i/hd)
   uint32_t *counters, *epoch;
@@ -211,7 +216,7 @@ struct WideStep {
 cudaError_t wide_prepare();
 cudaError_t wide_step(const WideStep &s, cudaStream_t stream, int *launches);
 
-size_t step_smem_bytes(int n_ops, int xs_floats, int mmax);
+size_t step_smem_bytes(int n_ops, int xs_floats, int mmax, int e_ld);
 bool kernel_stages_x(int mmax);
 int max_cta_per_sm(int mmax, size_t smem);
 

@@ -109,6 +109,9 @@ MK_INLINE void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint
       : "memory");
 }
 
+// Bring the 128-byte line at p into L2 (no register result, no completion).
+MK_INLINE void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 MK_INLINE uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -306,9 +309,8 @@ struct Warp {
   uint64_t *full, *empty;  // per slot: tile landed / tile released
   float *wbuf;
   uint32_t *arrive;
-  float *rpart;                // this warp's router-logit partials of the current layer, [MMAX][kMaxExperts]
-  float *rpart_cta;            // all compute warps' rows, [kConsumers][MMAX][kMaxExperts]
-  int rpart_ld;                // MMAX * kMaxExperts: one warp's rows to the next
+  long long *rsum;             // the CTA's router-logit sums of the current layer, [MMAX][e_ld],
+                               // 2^-32 fixed point (shared memory)
   int *attn_prefix;        // this warp's: first item of each sequence, [kMaxRows + 1]
   int *attn_nch;           // this warp's: KV chunks of each sequence, [kMaxRows]
   int step;                // the step (of a multi-step launch) this warp is in
@@ -323,6 +325,7 @@ struct Warp {
   int islot;
   bool producer;
   int dseg0;  // staged down projection: the first expert segment of this CTA's range
+  uint32_t xphase;  // batch 1: stagings of the activation row so far
   // producer cursor: op, this consumer's unit index in it, tile in the unit
   int iop, iu0, in_units, iu, it, in_tiles, iunit;
   int itype, ilayer;  // type and layer of op iop, once its current unit is set up
@@ -363,29 +366,6 @@ MK_INLINE bool routing_ready(const Warp &w, int layer) {
   return ok;
 }
 
-// inv_rms for rows 0..M-1 from the residual producers' partial sums of squares.
-MK_INLINE void compute_inv_rms(const Params &P, int lane, float (&inv)[kMaxRows]) {
-  const int nk = P.ss_ld / 128;  // float4 loads per lane and row (padding is zero)
-#pragma unroll
-  for (int m = 0; m < kMaxRows; ++m) {
-    inv[m] = 0.f;
-    if (m < P.M) {
-      const float4 *row = reinterpret_cast<const float4 *>(P.ss + static_cast<size_t>(m) * P.ss_ld) + lane;
-      float s = 0.f;
-      for (int k0 = 0; k0 < nk; k0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          v[k] = (k0 + k < nk) ? __ldcg(row + 32 * (k0 + k)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) s += (v[k].x + v[k].y) + (v[k].z + v[k].w);
-      }
-      s = warp_sum(s);
-      inv[m] = 1.0f / sqrtf(s / static_cast<float>(P.d) + P.eps);
-    }
-  }
-}
-
 // Lane l owns experts 4l..4l+3 and 128+4l..128+4l+3.
 MK_INLINE int expert_of(int lane, int i) { return (i < 4) ? 4 * lane + i : 128 + 4 * lane + (i - 4); }
 
@@ -408,8 +388,9 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
     chosen[i] = 0;
     slots[i] = 0;
   }
-  float inv[kMaxRows];
-  compute_inv_rms(P, lane, inv);
+  // the rows' sums of squares are loaded with the first row's logits (one
+  // round trip at batch 1)
+  const long long sqv = lane < P.M ? __ldcg(P.ssq + kMaxRows + lane) : 0ll;
   for (int m = 0; m < P.M; ++m) {
     const long long *row = P.racc + (static_cast<size_t>(layer) * kMaxRows + m) * P.e_ld;
     longlong2 ua[2], ub[2];
@@ -421,10 +402,8 @@ __device__ __noinline__ void route_compute(const Params &P, RouteCache *rc, int 
     }
     float z[EPL];
     const long long u[EPL] = {ua[0].x, ua[0].y, ua[1].x, ua[1].y, ub[0].x, ub[0].y, ub[1].x, ub[1].y};
-    float im = 0.f;
-#pragma unroll
-    for (int mm = 0; mm < kMaxRows; ++mm)
-      if (mm == m) im = inv[mm];
+    const long long sqm = __shfl_sync(0xffffffffu, sqv, m);
+    const float im = 1.0f / sqrtf(static_cast<float>(static_cast<double>(sqm) * 0x1p-32) / static_cast<float>(P.d) + P.eps);
 #pragma unroll
     for (int i = 0; i < EPL; ++i) z[i] = im * from_fix(u[i]);
     // the keys of this lane's experts; 0 = not a candidate (absent or taken)
@@ -806,13 +785,18 @@ MK_INLINE void issue_tile(Warp &w, int type, int layer, int t) {
     // columns per group; tile t takes boxes 4t .. 4t+3
     const int nbx = cdiv(w.uK, kPanel), nb = P.down_groups * nbx, b0 = t * kPanels;
     const int nbox = min(kPanels, nb - b0);
+    // column order for a unit of at most two rows (its consumer keeps both
+    // groups' sums at once), group order above
+    int seg, rb;
+    down_unit_seg(w, w.iunit, seg, rb);
+    const bool cols = P.down_cols && (seg < n_union(w) ? __popc(w.rc->rowmask[seg]) : P.M) <= 2;
     if (w.lane == 0) {
       expect(static_cast<uint32_t>(nbox) * kBoxBytes);
       for (int p = 0; p < nbox; ++p) {
         // box b: group b % 2, column b / 2 (column order) or group b / nbx,
         // column b % nbx (group order)
         const int b = b0 + p;
-        const int g = P.down_cols ? (b & 1) : b / nbx, c = P.down_cols ? (b >> 1) : b - g * nbx;
+        const int g = cols ? (b & 1) : b / nbx, c = cols ? (b >> 1) : b - g * nbx;
         tma_load_2d(dst + p * kBoxBytes, w.um, c * kPanel, w.urow0 + g * kRows, bar, w.pol_w);
       }
     }
@@ -858,11 +842,9 @@ MK_INLINE int feed_more(Warp &w) {
         break;
       }
       issue_tile(w, w.itype, w.ilayer, w.it);
-      if (kTrace && w.P->trace && w.lane == 0) {
-        unsigned long long *tr = w.P->trace + (static_cast<size_t>(w.iop) * w.nw + w.slot) * kTraceWords;
-        const unsigned long long t = now_ns();
-        if (tr[8] == 0) tr[8] = t;
-        tr[9] = t;
+      if (kTrace && w.P->trace && w.lane == 0 && w.it == 0 && w.iu == 0) {
+        // the op's first tile (one clock read per op: the trace must stay light)
+        w.P->trace[(static_cast<size_t>(w.iop) * w.nw + w.slot) * kTraceWords + 8] = now_ns();
       }
       w.it++;
       progress = true;
@@ -913,6 +895,8 @@ MK_INLINE int feed_more(Warp &w) {
       w.iop_init = true;
     }
     if (w.iu >= w.in_units) {
+      if (kTrace && P.trace && w.lane == 0 && w.in_units > 0)  // the op's last tile is out
+        P.trace[(static_cast<size_t>(w.iop) * w.nw + w.slot) * kTraceWords + 9] = now_ns();
       w.iop++;
       w.iop_init = false;
       continue;
@@ -1043,15 +1027,14 @@ MK_INLINE bool arrive(Warp &w, int op, int type, int layer) {
   cta_last = __shfl_sync(0xffffffffu, cta_last, 0);
   if (!cta_last) return false;
   if (type == OP_OPROJ && P.E > 0) {
-    // the CTA's router-logit partials: the compute warps' rows summed in a
-    // fixed order, then added into the layer's global fixed-point sums
+    // the CTA's router-logit sums, added into the layer's global ones and
+    // cleared for the next layer's o-projection
     long long *dst = P.racc + static_cast<size_t>(layer) * kMaxRows * P.e_ld;
     for (int i = w.lane; i < P.M * P.E; i += 32) {
       const int m = i / P.E, e = i - m * P.E;
-      float sum = 0.f;
-#pragma unroll
-      for (int k = 0; k < kConsumers; ++k) sum += w.rpart_cta[k * w.rpart_ld + m * kMaxExperts + e];
-      if (sum != 0.f) red_add_fix(dst + m * P.e_ld + e, to_fix(sum));
+      const long long sum = w.rsum[m * P.e_ld + e];
+      if (sum != 0) red_add_fix(dst + m * P.e_ld + e, sum);
+      w.rsum[m * P.e_ld + e] = 0;
     }
     __syncwarp();
   }
@@ -1089,8 +1072,22 @@ MK_INLINE void clear_router_sums(const Warp &w, int layer) {
 // RMSNorm is applied as y = inv_rms * (W (h * g)): the per-row scalar is
 // factored out of the dot product and multiplied in the epilogue.  At M > 1
 // the gained rows h * g are written next to h by the op that produces h.
-template <int MJ>
-struct XPlain {  // x = src[row][col]
+// Activation rows are stored panel-permuted: within each 256-column panel,
+// columns 8g..8g+3 sit at 4g and columns 8g+4..8g+7 at 128 + 4g, so that the
+// 32 lanes' float4 reads (lane g takes columns 8g..8g+7 of a panel) are 16
+// bytes apart, free of shared-memory bank conflicts.  Every producer of an
+// activation row writes it in this layout, so that a row is staged into shared
+// memory by a plain bulk copy.
+MK_INLINE int xs_pos4(int c4) {  // float4 slot of columns 4*c4 .. 4*c4+3
+  return (c4 & ~63) | ((c4 & 1) << 5) | ((c4 & 63) >> 1);
+}
+MK_INLINE int xperm(int col) { return 4 * xs_pos4(col >> 2) + (col & 3); }
+
+// MJ activation rows (row[j] of src, stride ld), read 8 consecutive columns
+// per lane: from global memory through L1 (SH false) or from the CTA's staged
+// copy in shared memory (SH true).
+template <int MJ, bool SH>
+struct XRows {
   const float *src;
   int ld;
   int row[MJ];
@@ -1099,8 +1096,15 @@ struct XPlain {  // x = src[row][col]
 #pragma unroll
     for (int j = 0; j < MJ; ++j) {
       if (col < K && j < n) {
-        const float4 *p = reinterpret_cast<const float4 *>(src + static_cast<size_t>(row[j]) * ld + col);
-        const float4 a = __ldca(p), b = __ldca(p + 1);
+        const float *pb = src + static_cast<size_t>(row[j]) * ld + (col & ~(kPanel - 1)) + ((col & (kPanel - 1)) >> 1);
+        float4 a, b;
+        if constexpr (SH) {
+          a = *reinterpret_cast<const float4 *>(pb);
+          b = *reinterpret_cast<const float4 *>(pb + kPanel / 2);
+        } else {
+          a = __ldca(reinterpret_cast<const float4 *>(pb));
+          b = __ldca(reinterpret_cast<const float4 *>(pb + kPanel / 2));
+        }
         x[j][0] = a.x; x[j][1] = a.y; x[j][2] = a.z; x[j][3] = a.w;
         x[j][4] = b.x; x[j][5] = b.y; x[j][6] = b.z; x[j][7] = b.w;
       } else {
@@ -1110,29 +1114,20 @@ struct XPlain {  // x = src[row][col]
     }
   }
 };
+template <int MJ>
+using XPlain = XRows<MJ, false>;
+template <int MJ>
+using XSmem = XRows<MJ, true>;
 
-// One activation row staged in shared memory by the CTA (batch 1).  Within
-// each 256-column panel, columns 8g..8g+3 sit at 4g and columns 8g+4..8g+7 at
-// 128 + 4g, so that the 32 lanes' float4 reads (lane g takes columns 8g..8g+7
-// of a panel) are 16 bytes apart and free of bank conflicts.
-MK_INLINE int xs_pos4(int c4) {  // float4 slot of columns 4*c4 .. 4*c4+3
-  return (c4 & ~63) | ((c4 & 1) << 5) | ((c4 & 63) >> 1);
+// The CTA's staged row at batch 1 (one row) as an XSmem source.
+MK_INLINE XSmem<1> staged_row(const float *xs) {
+  XSmem<1> x;
+  x.src = xs;
+  x.ld = 0;
+  x.row[0] = 0;
+  x.n = 1;
+  return x;
 }
-struct XSmem {
-  const float *xs;
-  MK_INLINE void load(int col, int K, float (&x)[1][8]) const {
-    if (col < K) {
-      const float *pb = xs + (col & ~(kPanel - 1)) + ((col & (kPanel - 1)) >> 1);
-      const float4 a = *reinterpret_cast<const float4 *>(pb);
-      const float4 b = *reinterpret_cast<const float4 *>(pb + kPanel / 2);
-      x[0][0] = a.x; x[0][1] = a.y; x[0][2] = a.z; x[0][3] = a.w;
-      x[0][4] = b.x; x[0][5] = b.y; x[0][6] = b.z; x[0][7] = b.w;
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) x[0][k] = 0.f;
-    }
-  }
-};
 
 // Even and odd columns go to separate accumulators (acc, acc2): one packed FMA
 // serves both, and each row has two independent FMA chains.
@@ -1310,21 +1305,21 @@ MK_INLINE void residual_units(const Params &P, int lane, int slot, int nw, int d
     if (live && row < P.d) {
       const float hn = val(m, row);
       __stcg(P.h + static_cast<size_t>(m) * P.d + row, hn);
-      if (gx) __stcg(P.xg + static_cast<size_t>(m) * P.d + row, hn * __bfloat162float(gx[row]));
+      __stcg(P.xg + static_cast<size_t>(m) * P.ldx + xperm(row), hn * __bfloat162float(gx[row]));
       sq = hn * hn;
       if (dbg_layer >= 0 && P.dbg_hidden)
         P.dbg_hidden[(static_cast<size_t>(dbg_layer) * P.max_rows + m) * P.d + row] = hn;
     }
     sq += __shfl_xor_sync(0xffffffffu, sq, 1);
     sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-    if (live && r == 0) __stcg(&P.ss[m * P.ss_ld + unit], sq);
+    if (live && r == 0) red_add_fix(P.ssq + m, to_fix(sq));
   }
   __syncwarp();
 }
 
-MK_INLINE void op_embed(Warp &w, bool gained) {
+MK_INLINE void op_embed(Warp &w) {
   const Params &P = *w.P;
-  residual_units(P, w.lane, w.slot, w.nw, 0, gained ? P.norms[0] : nullptr, [&](int m, int row) {
+  residual_units(P, w.lane, w.slot, w.nw, 0, P.norms[0], [&](int m, int row) {
     // step 0: the given tokens (may alias the argmax output); later steps:
     // the previous step's argmax
     int tok = w.step == 0 ? __ldcg(&P.tokens[m])
@@ -1334,9 +1329,9 @@ MK_INLINE void op_embed(Warp &w, bool gained) {
   });
 }
 
-// Above batch 1: the residual entering the next layer, h = h_mid + the expert
-// outputs' fixed-point sum (the routing weights are applied by the down
-// units), with x = h * g of the next norm and the sum-of-squares partials.
+// The residual entering the next layer, h = h_mid + the expert outputs'
+// fixed-point sum (the routing weights are applied by the down units), its
+// sum of squares and x = h * g of the next norm.
 MK_INLINE void op_combine(Warp &w, int layer) {
   const Params &P = *w.P;
   const __nv_bfloat16 *gx = (layer + 1 < P.L) ? P.norms[2 * (layer + 1)] : P.final_norm;
@@ -1384,31 +1379,30 @@ MK_INLINE int row_at(const int (&row)[MJ], int q) {
 template <int MJ, bool XS, class Body>
 MK_INLINE bool with_dense_x(Warp &w, int type, int layer, const float *xs, Body body) {
   const Params &P = *w.P;
-  if constexpr (XS) {
-    XSmem x;
-    x.xs = xs;
+  if constexpr (XS && MJ == 1) {
+    return body(staged_row(xs));
+  } else if constexpr (XS) {
+    // the op's M rows, staged by the CTA with their global row strides
+    XSmem<MJ> x;
+    x.src = xs;
+    x.ld = type == OP_OPROJ ? P.ldo : P.ldx;
+    x.n = P.M;
+    fill_all_rows<MJ>(x.row, P.M);
     return body(x);
-  } else if (type == OP_OPROJ) {
+  } else {
+    // x = o, or h * g written with h by the op that produced it
     XPlain<MJ> xp;
-    xp.src = P.o;
-    xp.ld = P.Hq * P.hd;
+    xp.src = type == OP_OPROJ ? P.o : P.xg;
+    xp.ld = type == OP_OPROJ ? P.ldo : P.ldx;
     xp.n = P.M;
     fill_all_rows<MJ>(xp.row, P.M);
     return body(xp);
-  } else {
-    // x = h * g, written with h by the op that produced it
-    XPlain<MJ> xn;
-    xn.src = P.xg;
-    xn.ld = P.d;
-    xn.n = P.M;
-    fill_all_rows<MJ>(xn.row, P.M);
-    return body(xn);
   }
 }
 
 // The o-projection unit's epilogue.  Lane 4m + r holds row row0 + r of the new
-// residual of activation row m (h_mid = h + Wo o): it stores it (with, above
-// batch 1, x = h_mid * g_ffn for the expert GEMVs), its square into the
+// residual of activation row m (h_mid = h + Wo o): it stores it (with x =
+// h_mid * g_ffn, panel-permuted, for the expert GEMVs), its square into the
 // sum-of-squares partials, and clears the expert-output accumulator's entry
 // for the layer that follows.  With a router, the unit's last ring slot holds
 // the router's 8 columns around these rows (all E rows): the unit adds its
@@ -1417,24 +1411,24 @@ MK_INLINE bool with_dense_x(Warp &w, int type, int layer, const float *xs, Body 
 // owns experts l, l + 32, ..., so the adds need no atomics and follow the
 // warp's unit order).
 template <int MJ>
-MK_INLINE bool oproj_epilogue(Warp &w, int op, int layer, int unit, int row0, float h_old, const float *wb) {
+MK_INLINE bool oproj_epilogue(Warp &w, int op, int layer, int unit, int row0, float h_old, float g_row,
+                              const float *wb) {
   const Params &P = *w.P;
   const int m = w.lane / kRows, r = w.lane % kRows, row = row0 + r;
   const bool live = w.lane < kRows * P.M && row < P.d;
-  const __nv_bfloat16 *g = P.norms[2 * layer + 1];
   float hn = 0.f, gx = 0.f, sq = 0.f;
   if (live) {
     hn = h_old + wb[r * MJ + m];
-    gx = hn * __bfloat162float(g[row]);
+    gx = hn * g_row;
     const size_t i = static_cast<size_t>(m) * P.d + row;
     __stcg(P.hm + i, hn);
-    if (!P.fused) __stcg(P.xg + i, gx);
+    __stcg(P.xg + static_cast<size_t>(m) * P.ldx + xperm(row), gx);
     __stcg(reinterpret_cast<unsigned long long *>(P.hacc) + i, 0ull);
     sq = hn * hn;
   }
   sq += __shfl_xor_sync(0xffffffffu, sq, 1);
   sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-  if (live && r == 0) __stcg(&P.ss[m * P.ss_ld + unit], sq);
+  if (live && r == 0) red_add_fix(P.ssq + kMaxRows + m, to_fix(sq));
   if (P.E == 0) return true;
   const uint8_t *slot = consume_begin(w, op);
   if (!slot) return false;
@@ -1454,7 +1448,9 @@ MK_INLINE bool oproj_epilogue(Warp &w, int op, int layer, int unit, int row0, fl
       u = fmaf(bf_hi(wr.x), x1, u);
       u = fmaf(bf_lo(wr.y), x2, u);
       u = fmaf(bf_hi(wr.y), x3, u);
-      if (e < P.E) w.rpart[mm * kMaxExperts + e] += u;
+      // integer adds: the CTA's sum does not depend on the warps' order
+      if (e < P.E) atomicAdd(reinterpret_cast<unsigned long long *>(&w.rsum[mm * P.e_ld + e]),
+                             static_cast<unsigned long long>(to_fix(u)));
     }
   }
   consume_end(w);
@@ -1486,6 +1482,7 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
   // the o-projection's residual input, loaded before the stream so that its
   // latency hides behind the tiles
   const float h_old = (type == OP_OPROJ && live) ? __ldcg(P.h + static_cast<size_t>(m) * P.d + row0 + r) : 0.f;
+  const float g_row = (type == OP_OPROJ && live) ? __bfloat162float(P.norms[2 * layer + 1][row0 + r]) : 0.f;
   const bool ok = with_dense_x<MJ, XS>(w, type, layer, xs, [&](const auto &x) {
     return gemv_unit<MJ>(w, op, ntiles, col0, K, x, wb);
   });
@@ -1523,7 +1520,7 @@ MK_INLINE bool dense_unit(Warp &w, int op, int type, int layer, int unit, const 
       break;
     }
     case OP_OPROJ:
-      if (!oproj_epilogue<MJ>(w, op, layer, unit, row0, h_old, wb)) return false;
+      if (!oproj_epilogue<MJ>(w, op, layer, unit, row0, h_old, g_row, wb)) return false;
       break;
     default: break;
   }
@@ -1537,30 +1534,35 @@ template <int MJ, bool XS>
 MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const float (&inv)[kMaxRows],
                        const float *xs) {
   const Params &P = *w.P;
-  XPlain<MJ> xn;  // x = h * g (M > 1), written with h by the o-projection
+  XPlain<MJ> xn;  // x = h * g, written with h by the o-projection
   xn.src = P.xg;
-  xn.ld = P.d;
+  xn.ld = P.ldx;
   float *dst;
   int ld, f0;
   if (type == OP_ROUTED_GU) {
     const int nfb = P.F / kRows, j = unit / nfb;
     f0 = (unit % nfb) * kRows;
     xn.n = rows_of_mask<MJ>(w.rc->rowmask[j], xn.row);
-    dst = P.act_routed + static_cast<size_t>(j) * kMaxRows * P.F;
-    ld = P.F;
+    dst = P.act_routed + static_cast<size_t>(j) * kMaxRows * P.ldf;
+    ld = P.ldf;
   } else {
     f0 = unit * kRows;
     xn.n = P.M;
     fill_all_rows<MJ>(xn.row, P.M);
     dst = P.act_shared;
-    ld = P.Fs;
+    ld = P.ldfs;
   }
   const int half = cdiv(P.d, kTileCols);
   float *wb = w.wbuf;
   // gate rows, then up rows: one rolled loop, one copy of the stream code
   if constexpr (XS) {
-    XSmem x;
-    x.xs = xs;
+    // the rows staged by SHARED_GU (all M rows, stride ldx)
+    XSmem<MJ> x;
+    x.src = xs;
+    x.ld = P.ldx;
+    x.n = xn.n;
+#pragma unroll
+    for (int j = 0; j < MJ; ++j) x.row[j] = xn.row[j];
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh)
       if (!gemv_unit<MJ>(w, op, half, 0, P.d, x, wb + hh * kRows * MJ)) return false;
@@ -1577,7 +1579,7 @@ MK_INLINE bool gu_unit(Warp &w, int op, int type, int layer, int unit, const flo
     for (int mm = 0; mm < kMaxRows; ++mm)
       if (mm == m) im = inv[mm];
     const float g = im * wb[r * MJ + q], u = im * wb[kRows * MJ + r * MJ + q];
-    __stcg(dst + static_cast<size_t>(m) * ld + f0 + r, silu(g) * u);
+    __stcg(dst + static_cast<size_t>(m) * ld + xperm(f0 + r), silu(g) * u);
   }
   __syncwarp();
   return true;
@@ -1596,13 +1598,13 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm)
   XPlain<MJ> xs;
   int K;
   if (seg < U) {
-    xs.src = P.act_routed + static_cast<size_t>(seg) * kMaxRows * P.F;
-    xs.ld = P.F;
+    xs.src = P.act_routed + static_cast<size_t>(seg) * kMaxRows * P.ldf;
+    xs.ld = P.ldf;
     xs.n = rows_of_mask<MJ>(rt->rowmask[seg], xs.row);
     K = P.F;
   } else {
     xs.src = P.act_shared;
-    xs.ld = P.Fs;
+    xs.ld = P.ldfs;
     xs.n = P.M;
     fill_all_rows<MJ>(xs.row, P.M);
     K = P.Fs;
@@ -1612,8 +1614,7 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm)
   if constexpr (XS && MJ == 1) {
     if (P.down_staged) {
       // the CTA staged its experts' activations: slot seg - dseg0 of the row
-      XSmem xst;
-      xst.xs = xsm + (seg - w.dseg0) * (cdiv(max(P.F, P.Fs), kPanel) * kPanel);
+      const XSmem<1> xst = staged_row(xsm + (seg - w.dseg0) * panel_ld(max(P.F, P.Fs)));
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xst, wb);
     } else {
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xs, wb);
@@ -1936,9 +1937,16 @@ MK_INLINE void attn_final_merge(const Params &P, int lane, int grp, int v, int n
   }
   const int t = qv / G, head = g * G + qv % G, m = b * P.T + t;
   const float invl = 1.0f / L;
-  float *dst = P.o + static_cast<size_t>(m) * P.Hq * hd + head * hd + lane * DPL;
+  // o is stored panel-permuted: this lane's DPL columns (2 or 4, aligned to
+  // their count) stay together within one float4 slot
+  const int col = head * hd + lane * DPL;
+  float *dst = P.o + static_cast<size_t>(m) * P.ldo + xperm(col);
+  if constexpr (DPL == 4) {
+    __stcg(reinterpret_cast<float4 *>(dst), make_float4(acc[0] * invl, acc[1] * invl, acc[2] * invl, acc[3] * invl));
+  } else {
 #pragma unroll
-  for (int dd = 0; dd < DPL; ++dd) __stcg(dst + dd, acc[dd] * invl);
+    for (int dd = 0; dd < DPL; ++dd) __stcg(dst + dd, acc[dd] * invl);
+  }
 }
 
 // One CTA-wide attention item: every warp computes its share, warp v (v < 4)
@@ -2125,6 +2133,8 @@ __device__ __noinline__ void final_argmax(const Params &P, int lane, uint32_t ep
     }
     __syncwarp();
   }
+  if (lane < P.M) P.ssq[lane] = 0;  // the entering residual's sums, read by LMHEAD
+  __syncwarp();
   if (lane == 0) {
     __threadfence();
     st_release(P.epoch, epoch);
@@ -2166,128 +2176,117 @@ MK_INLINE bool cta_rendezvous(Warp &w, uint32_t *cnt, uint32_t target, int op) {
   return true;
 }
 
-// Batch 1: the CTA stages the op's activation row in shared memory once
-// (x = h * g for normed ops, x = o for the o-projection); every warp then
-// reads its columns from there.  All warps take part, with or without units.
-// The normed ops' h: the embedding (layer 0's QKV), h_mid (the expert
-// GEMVs), or, for the next layer's QKV and for LMHEAD, the layer's end
-// h_mid + the expert outputs' fixed-point sum; each CTA then also writes its
-// share of that sum (float4 c4 with c4 % n_cta == cta) as the next residual
-// and to the debug copy.  Normed ops also sum h^2 over the columns each warp
-// staged into ssp[warp] (a fixed assignment, so the sum is deterministic).
-MK_INLINE bool stage_x(Warp &w, int type, int layer, float *xs, float *ssp, uint32_t *cnt, uint32_t &seq, int op) {
-  const Params &P = *w.P;
-  const bool oproj = type == OP_OPROJ;
-  const bool sum = P.fused && ((type == OP_QKV && layer > 0) || type == OP_LMHEAD);
-  const int K = oproj ? P.Hq * P.hd : P.d;
-  const float4 *src = reinterpret_cast<const float4 *>(oproj                                      ? P.o
-                                                       : (type == OP_QKV || type == OP_LMHEAD) && !sum ? P.h
-                                                                                                   : P.hm);
-  const __nv_bfloat16 *g = oproj ? nullptr
-                           : (type == OP_QKV)    ? P.norms[2 * layer]
-                           : (type == OP_LMHEAD) ? P.final_norm
-                                                 : P.norms[2 * layer + 1];
-  float *dbg = (sum && P.dbg_hidden) ? P.dbg_hidden + static_cast<size_t>(type == OP_QKV ? layer : P.L) * P.max_rows * P.d
-                                     : nullptr;
-  // four float4 columns per thread in flight at once: the row was just written
-  // by other SMs, so every load is an L2 round trip
-  constexpr int U = 4;
-  const int n4 = K / 4;
-  float sq = 0.f;
-  for (int c0 = threadIdx.x; c0 < n4; c0 += U * kConsumerThreads) {
-    float4 v[U];
-    longlong2 a[U], b[U];
-    uint2 gb[U];
-#pragma unroll
-    for (int j = 0; j < U; ++j) {
-      const int c4 = c0 + j * kConsumerThreads;
-      const bool in = c4 < n4;
-      v[j] = in ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-      a[j] = (in && sum) ? __ldcg(reinterpret_cast<const longlong2 *>(P.hacc) + 2 * c4) : make_longlong2(0, 0);
-      b[j] = (in && sum) ? __ldcg(reinterpret_cast<const longlong2 *>(P.hacc) + 2 * c4 + 1) : make_longlong2(0, 0);
-      gb[j] = (in && g) ? __ldg(reinterpret_cast<const uint2 *>(g + 4 * c4)) : make_uint2(0u, 0u);
-    }
-#pragma unroll
-    for (int j = 0; j < U; ++j) {
-      const int c4 = c0 + j * kConsumerThreads;
-      if (c4 >= n4) break;
-      float4 x = v[j];
-      if (sum) {
-        x.x += from_fix(a[j].x);
-        x.y += from_fix(a[j].y);
-        x.z += from_fix(b[j].x);
-        x.w += from_fix(b[j].y);
-        if (c4 % P.n_cta == w.cta) {
-          if (type == OP_QKV) __stcg(reinterpret_cast<float4 *>(P.h) + c4, x);
-          if (dbg) reinterpret_cast<float4 *>(dbg)[c4] = x;
-        }
-      }
-      if (g) {
-        sq = fmaf(x.x, x.x, sq);
-        sq = fmaf(x.y, x.y, sq);
-        sq = fmaf(x.z, x.z, sq);
-        sq = fmaf(x.w, x.w, sq);
-        x.x *= bf_lo(gb[j].x);
-        x.y *= bf_hi(gb[j].x);
-        x.z *= bf_lo(gb[j].y);
-        x.w *= bf_hi(gb[j].y);
-      }
-      reinterpret_cast<float4 *>(xs)[xs_pos4(c4)] = x;
-    }
-  }
-  if (g) {
-    sq = warp_sum(sq);
-    if (w.lane == 0) ssp[w.wib] = sq;
-  }
-  seq += kConsumers;
-  return cta_rendezvous(w, cnt, seq, op);
+// ---- batch 1: the op's activation row staged in shared memory --------------
+// The rows live in global memory in the panel-permuted layout XSmem reads, so
+// a CTA stages one with a plain bulk copy.  The first compute warp of the CTA
+// past the op's dependency wait issues the copies (one mbarrier, expecting
+// their bytes); every compute warp then waits for that barrier's phase.  The
+// copies may overwrite shared memory that the previous staged op read: every
+// op that stages waits (directly or through its dependencies) for the
+// completion of the op that last used the row, so no warp of the CTA still
+// reads it.
+struct StageCtl {
+  uint64_t bar;    // completes once per staging, when the copies have landed
+  uint32_t elect;  // staging arrivals; the first of each kConsumers issues
+};
+
+MK_INLINE void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   saddr(dst)),
+               "l"(src), "r"(bytes), "r"(saddr(bar))
+               : "memory");
 }
 
-// 1 / rms of the staged row from the warps' partial sums (batch 1).
-MK_INLINE float staged_inv_rms(const Params &P, const float *ssp) {
-  float s = 0.f;
-#pragma unroll
-  for (int k = 0; k < kConsumers; ++k) s += ssp[k];
-  return 1.0f / sqrtf(s / static_cast<float>(P.d) + P.eps);
+// Stage `n` rows: row i (bytes[i] bytes, a multiple of 16) from src[i] to
+// xs + off[i] floats.  All four compute warps call it in the same order;
+// w.xphase counts the stagings.
+MK_INLINE bool stage_rows(Warp &w, StageCtl *sc, float *xs, const float *const *src, const uint32_t *bytes,
+                          const int *off, int n, int op) {
+  int issuer = 0;
+  if (w.lane == 0) issuer = (atomicAdd(&sc->elect, 1u) % kConsumers) == 0 ? 1 : 0;
+  issuer = __shfl_sync(0xffffffffu, issuer, 0);
+  if (issuer && w.lane == 0) {
+    // the rows were published by other SMs and acquired by this thread's
+    // dependency wait (generic proxy); the bulk copies read them, and write
+    // shared memory last read by generic loads, through the async proxy
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    fence_proxy_async_smem();
+    uint32_t total = 0;
+    for (int i = 0; i < n; ++i) total += bytes[i];
+    mbar_arrive_expect_tx(&sc->bar, total);
+    for (int i = 0; i < n; ++i) bulk_g2s(xs + off[i], src[i], bytes[i], &sc->bar);
+  }
+  const uint32_t par = w.xphase & 1u;
+  w.xphase++;
+  if (!__all_sync(0xffffffffu, mbar_try_wait(&sc->bar, par)) && !wait_slot_slow(&sc->bar, par, w.P->timeout_ns)) {
+    set_error(w, -5, op);
+    return false;
+  }
+  return true;
+}
+
+// The op's input row: x = h * g (QKV, LMHEAD: the residual entering the
+// layer, or the final one, with the norm's gain; SHARED_GU, ROUTED_GU: the
+// residual after the o-projection with the FFN norm's gain) or x = o
+// (OPROJ).  Every producer of these rows writes them gained and permuted.
+MK_INLINE bool stage_x(Warp &w, StageCtl *sc, int type, float *xs, int op) {
+  const Params &P = *w.P;
+  const bool oproj = type == OP_OPROJ;
+  const float *src = oproj ? P.o : P.xg;
+  // rows 0..M-1 are contiguous: one copy
+  const uint32_t bytes = static_cast<uint32_t>(P.M * (oproj ? P.ldo : P.ldx) * sizeof(float));
+  const int off = 0;
+  return stage_rows(w, sc, xs, &src, &bytes, &off, 1, op);
 }
 
 // Batch 1 down projection: the CTA copies the activations of the experts its
 // unit range covers (routed rows first, then the shared expert) into the
-// shared-memory row, one slot of max(F, Fs) rounded up to whole panels per
-// expert from the range's first, each in the panel layout of XSmem.
-MK_INLINE bool stage_down(Warp &w, int layer, float *xs, uint32_t *cnt, uint32_t &seq, int op) {
+// shared-memory row, one slot of panel_ld(max(F, Fs)) floats per expert from
+// the range's first.
+MK_INLINE bool stage_down(Warp &w, StageCtl *sc, int layer, float *xs, int op) {
   const Params &P = *w.P;
   if (!route_cache(w, layer)) return false;
   const int U = n_union(w), total = op_total_units(w, OP_DOWN, layer);
   int c0, c1;
   down_cta_range(P, w.cta, total, c0, c1);
   w.dseg0 = c0 / P.n_db;
+  const float *src[kMaxStageSegs];
+  uint32_t bytes[kMaxStageSegs];
+  int off[kMaxStageSegs];
+  int n = 0;
   if (c1 > c0) {
-    const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, ld = cdiv(max(P.F, P.Fs), kPanel) * kPanel;
-    for (int sg = seg0; sg <= seg1; ++sg) {
-      const float4 *src = reinterpret_cast<const float4 *>(
-          sg < U ? P.act_routed + static_cast<size_t>(sg) * kMaxRows * P.F : P.act_shared);
-      const int K = sg < U ? P.F : P.Fs;
-      float4 *dst = reinterpret_cast<float4 *>(xs + (sg - seg0) * ld);
-      for (int c0 = threadIdx.x; c0 < K / 4; c0 += 4 * kConsumerThreads) {
-        float4 v[4];  // four loads in flight per thread
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c4 = c0 + j * kConsumerThreads;
-          v[j] = c4 < K / 4 ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (c0 + j * kConsumerThreads < K / 4) dst[xs_pos4(c0 + j * kConsumerThreads)] = v[j];
-      }
+    const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, ld = panel_ld(max(P.F, P.Fs));
+    for (int sg = seg0; sg <= seg1 && n < kMaxStageSegs; ++sg, ++n) {
+      src[n] = sg < U ? P.act_routed + static_cast<size_t>(sg) * kMaxRows * P.ldf : P.act_shared;
+      bytes[n] = static_cast<uint32_t>((sg < U ? P.ldf : P.ldfs) * sizeof(float));
+      off[n] = (sg - seg0) * ld;
     }
   }
-  seq += kConsumers;
-  return cta_rendezvous(w, cnt, seq, op);
+  return stage_rows(w, sc, xs, src, bytes, off, n, op);
+}
+
+// inv_rms of rows 0..M-1 from v, lane m's copy of the fixed-point sum of
+// squares of row m (loaded by the caller ahead of time).
+MK_INLINE float inv_rms_of(long long sum, const Params &P) {
+  return 1.0f / sqrtf(static_cast<float>(static_cast<double>(sum) * 0x1p-32) / static_cast<float>(P.d) + P.eps);
+}
+template <int MMAX>
+MK_INLINE void inv_from_ssq(const Params &P, long long v, float (&inv)[kMaxRows]) {
+#pragma unroll
+  for (int m = 0; m < MMAX; ++m) {
+    const long long vm = __shfl_sync(0xffffffffu, v, m);
+    inv[m] = m < P.M ? inv_rms_of(vm, P) : 0.f;  // rows past M: no work
+  }
+}
+
+// Ops whose units scale by an inv_rms, and which residual's sums they use
+// (0: entering the layer, 1: after the o-projection), else -1.
+MK_INLINE int normed_ssq(int type) {
+  return (type == OP_QKV || type == OP_LMHEAD) ? 0 : (type == OP_SHARED_GU || type == OP_ROUTED_GU) ? 1 : -1;
 }
 
 template <int MMAX, bool XS>
-MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, const float *ssp, AttnShared &ash,
+MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs, long long sqv, AttnShared &ash,
                            float &am_val, int &am_idx) {
   const Params &P = *w.P;
   if ((type == OP_ROUTED_GU || type == OP_DOWN) && !route_cache(w, layer)) return false;
@@ -2297,13 +2296,7 @@ MK_INLINE bool run_tile_op(Warp &w, int op, int type, int layer, const float *xs
   float inv[kMaxRows];
 #pragma unroll
   for (int m = 0; m < kMaxRows; ++m) inv[m] = 0.f;
-  if (type != OP_OPROJ && type != OP_DOWN && type != OP_ATTN) {
-    if constexpr (XS) {
-      inv[0] = staged_inv_rms(P, ssp);  // the row staged for this op (or, for routed gate/up, by SHARED_GU)
-    } else {
-      compute_inv_rms(P, w.lane, inv);
-    }
-  }
+  if (normed_ssq(type) >= 0) inv_from_ssq<MMAX>(P, sqv, inv);
   for (int i = 0; i < n; ++i) {
     const int u = u0 + i * stride;
     bool ok;
@@ -2333,17 +2326,25 @@ MK_INLINE void producer_run(const Params &P, Warp *feeds, int first, int lane, i
   attn_layout(P, 0, prefix, nch, lane);
   mine.lstep = 0;
   uint64_t t_idle = 0;
+  int idle_reason = 0, idle_op = 0;  // trace only
+  uint64_t idle_t0 = 0;
   for (int it = 0;; ++it) {
     bool progress = false, all_done = true;
-    const uint64_t t_it = (kTrace && P.trace) ? now_ns() : 0;
-    const int iop = mine.iop;
     int why = FEED_PROGRESS;
     if (!mine.done_issue && !mine.failed) why = feed_more<MULTI>(mine);
     progress = why == FEED_PROGRESS;
-    if (kTrace && P.trace && lane == 0 && !progress && iop < P.op_end) {
-      // the producer's idle time on this op, by reason (in the consumer's record)
-      unsigned long long *tr = P.trace + (static_cast<size_t>(iop) * mine.nw + mine.slot) * kTraceWords;
-      tr[why == FEED_RING_FULL ? 11 : 10] += now_ns() - t_it;
+    if (kTrace && P.trace && lane == 0) {
+      // the producer's idle episodes on its current op, by reason: a clock read
+      // when one starts and when it ends, added to the consumer's record
+      const int reason = progress ? 0 : (why == FEED_RING_FULL ? 11 : 10);
+      if (reason != idle_reason) {
+        const uint64_t t = now_ns();
+        if (idle_reason && idle_op < P.op_end)
+          P.trace[(static_cast<size_t>(idle_op) * mine.nw + mine.slot) * kTraceWords + idle_reason] += t - idle_t0;
+        idle_reason = reason;
+        idle_t0 = t;
+        idle_op = mine.iop;
+      }
     }
     all_done = mine.done_issue || mine.failed;
     if (all_done) break;
@@ -2386,18 +2387,18 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   __shared__ RouteCache s_route;
   __shared__ float s_attn_ml[kConsumers * kQvp * 2];
   __shared__ Warp s_feed[kConsumers];  // each consumer's tile stream, as its producer keeps it
-  __shared__ float s_ssp[kConsumers];  // batch 1: partial sums of h^2 of the staged row
-  __shared__ float s_rpart[kConsumers * MMAX * kMaxExperts];  // the compute warps' router-logit partials
+  __shared__ StageCtl s_xstage;        // batch 1: the staged activation row's copies
   const int wib = threadIdx.x >> 5;
   const bool consumer = wib < kConsumers;
   // dynamic shared memory: rings | activation row | full and empty barriers |
-  // epilogue scratch | per-op arrival counts
+  // router-logit sums | epilogue scratch | per-op arrival counts
   constexpr int S = ring_slots(MMAX);
   float *xs = reinterpret_cast<float *>(smem + kConsumers * S * kSlotBytes);
   uint8_t *after_xs = reinterpret_cast<uint8_t *>(xs + P.xs_floats);
   uint64_t *fulls = reinterpret_cast<uint64_t *>(after_xs);
   uint64_t *empties = fulls + kConsumers * S;
-  float *fbase = reinterpret_cast<float *>(empties + kConsumers * S);
+  long long *rsum = reinterpret_cast<long long *>(empties + kConsumers * S);
+  float *fbase = reinterpret_cast<float *>(rsum + MMAX * P.e_ld);
   uint32_t *arrive_cnt = reinterpret_cast<uint32_t *>(fbase + kConsumers * kWbuf);
   Warp w;
   w.P = &P;
@@ -2414,9 +2415,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.empty = empties + c * S;
   w.wbuf = fbase + c * kWbuf;
   w.arrive = arrive_cnt;
-  w.rpart_cta = s_rpart;
-  w.rpart = s_rpart + (consumer ? wib : 0) * MMAX * kMaxExperts;
-  w.rpart_ld = MMAX * kMaxExperts;
+  w.rsum = rsum;
   w.attn_prefix = s_attn_prefix[wib];
   w.attn_nch = s_attn_nch[wib];
   w.step = 0;
@@ -2428,6 +2427,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   w.filled = 0;
   w.producer = false;
   w.dseg0 = 0;
+  w.xphase = 0;
   w.failed = false;
   w.pol_w = policy_evict_first();
   w.pol_kv = policy_evict_normal();
@@ -2455,9 +2455,13 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     s_feed[wib] = f;
   }
   for (int i = threadIdx.x; i < P.n_ops; i += kThreads) arrive_cnt[i] = 0;
+  for (int i = threadIdx.x; i < MMAX * P.e_ld; i += kThreads) rsum[i] = 0;
   if (threadIdx.x == 0) {
     s_stage = 0;
     s_route.ready_key = s_route.fill_key = 0;
+    s_xstage.elect = 0;
+    mbar_init(&s_xstage.bar, 1);
+    fence_mbar_init();
   }
   __syncthreads();
 
@@ -2501,30 +2505,48 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   for (int op = P.op_begin; op < P.op_end && !w.failed; ++op) {
     const int type = op_type_of(op, P.L), layer = op_layer_of(op, P.L);
     int d0, d1;
-    op_deps(op, P.L, P.fused != 0, &d0, &d1);
+    op_deps(op, P.L, &d0, &d1);
+    // batch 1: SHARED_GU stages the normed row that ROUTED_GU reuses; a launch
+    // that starts at ROUTED_GU stages it itself
+    const bool stage = XS && (type == OP_QKV || type == OP_OPROJ || type == OP_SHARED_GU || type == OP_LMHEAD ||
+                              (type == OP_ROUTED_GU && op == P.op_begin));
+    if (type == OP_ATTN) {
+      // the rotary rows of this step's new positions (read by the attention
+      // items' staging), pulled into L2 while the QKV op finishes: lane 4r + i
+      // takes 128-byte line i of new row r (row r = b * T + t)
+      const int r = w.lane >> 2;
+      if (r < P.M) {
+        const int pos = seq_pos(P, r / P.T, w.step) + r % P.T;
+        if (pos < P.cap && 128 * (w.lane & 3) < P.hd * 4)  // a row is hd/2 float2 = hd * 4 bytes
+          prefetch_l2(reinterpret_cast<const char *>(P.rope + static_cast<size_t>(pos) * (P.hd / 2)) +
+                      128 * (w.lane & 3));
+      }
+    }
     const uint32_t target = w.epoch * static_cast<uint32_t>(P.n_cta);
     const uint32_t extra = (op == P.inject_op) ? 1u : 0u;
     if (d0 >= 0 && !wait_counter(w, &P.counters[d0 * kCounterStride], target + extra, op)) break;
     if (d1 >= 0 && !wait_counter(w, &P.counters[d1 * kCounterStride], target, op)) break;
     if (kTrace && P.trace && w.lane == 0 && type != OP_ROUTED_GU)
       P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords + 6] = now_ns();
+    // a normed op's rows' sums of squares, loaded now so that the load overlaps
+    // the staging (lane m holds row m's)
+    const int which = normed_ssq(type);
+    const long long sqv = (which >= 0 && w.lane < P.M) ? __ldcg(P.ssq + which * kMaxRows + w.lane) : 0ll;
+    // The sums of squares are cleared once their readers are done: the
+    // o-projection's (read by the routing and the expert GEMVs) at the next
+    // QKV, the entering residual's (read by QKV) at the o-projection, and, for
+    // the next step's embedding, by the final argmax.
+    if (w.slot == 0 && w.lane < P.M) {
+      if (type == OP_QKV) P.ssq[kMaxRows + w.lane] = 0;
+      if (type == OP_OPROJ) P.ssq[w.lane] = 0;
+    }
     // the previous layer's router sums have been read by every CTA (its down
     // projection is complete): clear them for the next step
     if (type == OP_OPROJ && layer > 0) clear_router_sums(w, layer - 1);
-    if (type == OP_OPROJ && P.E > 0) {
-      // this warp's router-logit partials start the layer at zero (the CTA's
-      // last warp read the previous layer's before the CTA arrived there)
-      for (int i = w.lane; i < P.M * kMaxExperts; i += 32) w.rpart[i] = 0.f;
-      __syncwarp();
-    }
     if (type == OP_LMHEAD) clear_router_sums(w, P.L - 1);
     if constexpr (XS) {
-      // SHARED_GU stages the normed row that ROUTED_GU reuses; a launch that
-      // starts at ROUTED_GU stages it itself
-      const bool stage = type == OP_QKV || type == OP_OPROJ || type == OP_SHARED_GU || type == OP_LMHEAD ||
-                         (type == OP_ROUTED_GU && op == P.op_begin);
-      if (stage && !stage_x(w, type, layer, xs, s_ssp, &s_stage, stage_seq, op)) break;
-      if (type == OP_DOWN && P.down_staged && !stage_down(w, layer, xs, &s_stage, stage_seq, op)) break;
+      if (stage && !stage_x(w, &s_xstage, type, xs, op)) break;
+      if (type == OP_DOWN && P.down_staged && !stage_down(w, &s_xstage, layer, xs, op)) break;
     }
     if (kTrace && P.trace && w.lane == 0 && type != OP_ROUTED_GU)
       P.trace[(static_cast<size_t>(op) * w.nw + w.slot) * kTraceWords + 7] = now_ns();
@@ -2533,11 +2555,11 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     w.tr_n = 0;
     bool ok = true;
     if (type == OP_EMBED) {
-      op_embed(w, !XS);
+      op_embed(w);
     } else if (type == OP_COMBINE) {
-      if (!P.fused) op_combine(w, layer);  // at batch 1 the next op's staging forms the sum
+      op_combine(w, layer);
     } else {
-      ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, s_ssp, ash, am_val, am_idx);
+      ok = run_tile_op<MMAX, XS>(w, op, type, layer, xs, sqv, ash, am_val, am_idx);
     }
     if (!ok || w.failed) break;
     if (type == OP_LMHEAD && (w.lane % kRows) == 0 && w.lane / kRows < P.M) {
@@ -2561,14 +2583,14 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
 }  // namespace
 
 #if !MK_TRACE
-size_t step_smem_bytes(int n_ops, int xs_floats, int mmax) {
+size_t step_smem_bytes(int n_ops, int xs_floats, int mmax, int e_ld) {
   const int S = ring_slots(mmax);
   return static_cast<size_t>(kConsumers) * S * kSlotBytes + static_cast<size_t>(xs_floats) * sizeof(float) +
-         2 * kConsumers * S * sizeof(uint64_t) + kConsumers * kWbuf * sizeof(float) +
-         static_cast<size_t>(n_ops) * sizeof(uint32_t);
+         2 * kConsumers * S * sizeof(uint64_t) + static_cast<size_t>(mmax) * e_ld * sizeof(long long) +
+         kConsumers * kWbuf * sizeof(float) + static_cast<size_t>(n_ops) * sizeof(uint32_t);
 }
 
-bool kernel_stages_x(int mmax) { return mmax == 1; }
+bool kernel_stages_x(int mmax) { return mmax <= 8; }
 #endif
 
 template <int MMAX, bool XS, bool MULTI>
@@ -2581,16 +2603,16 @@ static const void *kernel_for(int mmax, bool multi) {
   if (multi) {
     switch (mmax) {
       case 1: return kernel_ptr<1, true, true>();
-      case 2: return kernel_ptr<2, false, true>();
-      case 4: return kernel_ptr<4, false, true>();
-      default: return kernel_ptr<8, false, true>();
+      case 2: return kernel_ptr<2, true, true>();
+      case 4: return kernel_ptr<4, true, true>();
+      default: return kernel_ptr<8, true, true>();
     }
   }
   switch (mmax) {
     case 1: return kernel_ptr<1, true, false>();
-    case 2: return kernel_ptr<2, false, false>();
-    case 4: return kernel_ptr<4, false, false>();
-    default: return kernel_ptr<8, false, false>();
+    case 2: return kernel_ptr<2, true, false>();
+    case 4: return kernel_ptr<4, true, false>();
+    default: return kernel_ptr<8, true, false>();
   }
 }
 
@@ -2618,7 +2640,7 @@ int MK_ENTRY(max_cta_per_sm)(int mmax, size_t smem) {
 
 int MK_ENTRY(launch_step)(const Params &p, int mmax, bool cooperative, cudaStream_t stream) {
   const void *k = kernel_for(mmax, p.n_steps > 1);
-  const size_t smem = step_smem_bytes(p.n_ops, p.xs_floats, mmax);
+  const size_t smem = step_smem_bytes(p.n_ops, p.xs_floats, mmax, p.e_ld);
   void *args[] = {const_cast<Params *>(&p)};
   cudaError_t e;
   if (cooperative) {

@@ -81,9 +81,7 @@ def test_validate_rejects(L, field, value, code):
 @pytest.mark.parametrize("B", [1, 2])
 def test_schedule_is_a_dag_with_the_data_dependencies(L, B):
     """Every op waits only for earlier ops, and for each op the ops producing
-    its inputs are reachable through its waits.  At one row per step (B = 1)
-    the next layer's staging forms the residual sum from the down projection's
-    accumulator, so its QKV waits for DOWN; above, for COMBINE."""
+    its inputs are reachable through its waits."""
     d = _desc(SMALL, kv_capacity=2112, max_seqs=B, max_rows=B)
     rc, info, ops = mk.mk_plan_describe(d, 148, B, 1)
     assert rc == mk.MK_OK, mk.mk_last_error()
@@ -101,7 +99,7 @@ def test_schedule_is_a_dag_with_the_data_dependencies(L, B):
             if dep >= 0:
                 r |= {dep} | reach[dep]
         reach.append(r)
-    end = "DOWN" if B == 1 else "COMBINE"
+    end = "COMBINE"
     for l in range(Lyr):
         # the residual entering layer l: the embedding, or the previous layer's end
         prev_h = [idx[("EMBED", -1)]] if l == 0 else [idx[(end, l - 1)], idx[("OPROJ", l - 1)]]
