@@ -56,6 +56,28 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// 2-D bf16 map over [rows][cols] with row stride ld elements, box 64 columns
+// x box_rows rows, 128-byte swizzle (the tensor-core operand layout of the
+// wide-block products).  Rows or columns past the matrix read as zeros.
+int encode_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t ld,
+                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MK_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0 || (ld * 2) % 16 != 0)
+    return fail(MK_ERR_ARG, "tensor base %p or row stride %llu is not 16-byte aligned", base, (unsigned long long)ld);
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MK_ERR_CUDA, "cuTensorMapEncodeTiled(rows=%llu, cols=%llu, 128B swizzle) failed: %d",
+                (unsigned long long)rows, (unsigned long long)cols, (int)r);
+  return MK_OK;
+}
+
 // 2-D bf16 map over a row-major [rows][cols] matrix, box [box_cols][box_rows].
 int encode_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
               uint32_t box_rows) {
@@ -147,17 +169,22 @@ Plan make_plan(const mk_model_desc &d, int n_sm, int B, int T) {
   // (whole 256-column panels: the staged layout permutes columns within one)
   p.xs_floats = std::max((kConsumers + 1) * kQvp * d.head_dim + kMaxRows * d.head_dim,  // + new bf16 K/V rows
                          kernel_stages_x(p.mmax) ? p.mmax * panel_ld(std::max(d.d_model, d.n_q_heads * d.head_dim)) : 0);
-  // Batch 1 down projection: a CTA's contiguous range of units spans at most
-  // 1 + ceil(range / row blocks) experts; their activations must fit the
-  // shared-memory row.
+  // Staged down projection (one row per step): a CTA's contiguous range of
+  // units spans at most 1 + ceil(range / row blocks) experts (largest with the
+  // largest union), whose rows must fit the shared-memory rows.  Above one row
+  // the shared expert's units (all rows each) cost several routed ones, and
+  // contiguous ranges leave the CTAs that hold them far behind (measured at 4
+  // and 8 rows: the down projection's last CTA finished 80 and 300 us after
+  // the median), so there units go round-robin and read their rows via L1.
   p.down_staged = 0;
   if (p.mmax == 1) {
     const int n_db = p.n_hb / p.down_groups;
-    const int segs = std::min(d.n_experts, d.top_k) + (d.shared_ffn > 0 ? 1 : 0);
+    const int segs = std::min(d.n_experts, p.mmax * d.top_k) + (d.shared_ffn > 0 ? 1 : 0);
     const int per_cta = ceil_div(segs * n_db, p.n_cta);
-    const int span = 1 + ceil_div(per_cta, n_db);
+    const int span = std::min(1 + ceil_div(per_cta, n_db), segs);
     const int fmax = std::max(d.expert_ffn, d.shared_ffn);
-    p.down_staged = (std::min(span, segs) <= kMaxStageSegs && std::min(span, segs) * panel_ld(fmax) <= p.xs_floats) ? 1 : 0;
+    p.down_staged = (kernel_stages_x(p.mmax) && span <= kMaxStageSegs &&
+                     (long long)span * p.mmax * panel_ld(fmax) <= p.xs_floats) ? 1 : 0;
   }
   // an 8-row down unit of one or two activation rows keeps both groups' sums
   // at once, so its tiles go column by column (each column's activations
@@ -187,6 +214,11 @@ Sizes scratch_sizes(const mk_model_desc &d, int n_sm) {
 }
 
 }  // namespace
+
+int mk::encode_2d_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t ld,
+                        uint32_t box_rows) {
+  return encode_sw128(map, base, rows, cols, ld, box_rows);
+}
 
 struct GraphEntry {
   uint64_t key[12];

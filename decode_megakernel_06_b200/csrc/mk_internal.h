@@ -130,8 +130,8 @@ struct alignas(64) Params {
   int n_db;            // down-projection row blocks (n_hb / down_groups)
   int down_cols;       // 8-row down units of 1-2 activation rows: boxes ordered column
                        // by column, both groups per column (others group by group)
-  int down_staged;     // batch 1: each CTA takes a contiguous range of down units and
-                       // stages their experts' activations in shared memory
+  int down_staged;     // each CTA takes a contiguous range of down units and stages
+                       // their experts' activation rows in shared memory
   int e_ld;            // row stride of the router logits (E rounded up to 4)
   int ldx, ldo, ldf, ldfs;  // activation row strides (panel_ld of d, Hq*hd, F, Fs)
   int attn_chunk;      // KV positions per warp; a CTA item covers 8 * attn_chunk
@@ -214,6 +214,8 @@ struct WideStep {
 };
 
 cudaError_t wide_prepare();
+// A 128B-swizzled bf16 tensor map, box 64 columns x box_rows rows (mk_api.cu).
+int encode_2d_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
 cudaError_t wide_step(const WideStep &s, cudaStream_t stream, int *launches);
 
 size_t step_smem_bytes(int n_ops, int xs_floats, int mmax, int e_ld);

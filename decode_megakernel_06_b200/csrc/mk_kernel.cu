@@ -564,7 +564,7 @@ MK_INLINE int op_total_units(const Warp &w, int type, int layer) {
 // This warp's units of an op: u0, u0 + stride, ... (n of them).  Attention
 // items are CTA-wide; a staged down projection takes CTA-contiguous ranges;
 // everything else goes round-robin over the warp slots.
-// A staged (batch 1) down projection deals CTA c the contiguous units
+// A staged down projection deals CTA c the contiguous units
 // [c * total / n_cta, (c + 1) * total / n_cta), warp by warp within the CTA.
 // (cta + 1) * total stays far below 2^31: at most 148 CTAs x 257 segments x
 // 1536 row blocks.
@@ -1611,10 +1611,16 @@ MK_INLINE bool down_unit(Warp &w, int op, int layer, int unit, const float *xsm)
   }
   float *wb = w.wbuf;
   bool ok;
-  if constexpr (XS && MJ == 1) {
+  if constexpr (XS) {
     if (P.down_staged) {
-      // the CTA staged its experts' activations: slot seg - dseg0 of the row
-      const XSmem<1> xst = staged_row(xsm + (seg - w.dseg0) * panel_ld(max(P.F, P.Fs)));
+      // the CTA staged its experts' activation rows: slot seg - dseg0 of the
+      // staged block holds rows 0..M-1 of the segment at their global stride
+      XSmem<MJ> xst;
+      xst.src = xsm + (seg - w.dseg0) * P.M * panel_ld(max(P.F, P.Fs));
+      xst.ld = xs.ld;
+      xst.n = xs.n;
+#pragma unroll
+      for (int j = 0; j < MJ; ++j) xst.row[j] = xs.row[j];
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xst, wb);
     } else {
       ok = gemv_groups<MJ>(w, op, P.down_groups, K, xs, wb);
@@ -2239,10 +2245,10 @@ MK_INLINE bool stage_x(Warp &w, StageCtl *sc, int type, float *xs, int op) {
   return stage_rows(w, sc, xs, &src, &bytes, &off, 1, op);
 }
 
-// Batch 1 down projection: the CTA copies the activations of the experts its
-// unit range covers (routed rows first, then the shared expert) into the
-// shared-memory row, one slot of panel_ld(max(F, Fs)) floats per expert from
-// the range's first.
+// Staged down projection: the CTA copies the activation rows (rows 0..M-1) of
+// the experts its unit range covers (routed experts first, then the shared
+// one) into shared memory, one slot of M * panel_ld(max(F, Fs)) floats per
+// expert from the range's first, each a single bulk copy.
 MK_INLINE bool stage_down(Warp &w, StageCtl *sc, int layer, float *xs, int op) {
   const Params &P = *w.P;
   if (!route_cache(w, layer)) return false;
@@ -2255,11 +2261,11 @@ MK_INLINE bool stage_down(Warp &w, StageCtl *sc, int layer, float *xs, int op) {
   int off[kMaxStageSegs];
   int n = 0;
   if (c1 > c0) {
-    const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, ld = panel_ld(max(P.F, P.Fs));
+    const int seg0 = c0 / P.n_db, seg1 = (c1 - 1) / P.n_db, slot = P.M * panel_ld(max(P.F, P.Fs));
     for (int sg = seg0; sg <= seg1 && n < kMaxStageSegs; ++sg, ++n) {
       src[n] = sg < U ? P.act_routed + static_cast<size_t>(sg) * kMaxRows * P.ldf : P.act_shared;
-      bytes[n] = static_cast<uint32_t>((sg < U ? P.ldf : P.ldfs) * sizeof(float));
-      off[n] = (sg - seg0) * ld;
+      bytes[n] = static_cast<uint32_t>(P.M * (sg < U ? P.ldf : P.ldfs) * sizeof(float));
+      off[n] = (sg - seg0) * slot;
     }
   }
   return stage_rows(w, sc, xs, src, bytes, off, n, op);

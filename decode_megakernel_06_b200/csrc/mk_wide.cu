@@ -1,8 +1,9 @@
 // mk_wide.cu -- the decode step for wide blocks (8 < M <= 64 rows, e.g. a
 // speculative verify block of 7 rows for 8 sequences), as a short sequence of
 // launches.  With this many rows the dense projections are real contractions,
-// so every matrix product runs on the tensor cores (mma.sync m16n8k16, bf16 in,
-// fp32 accumulate).  Activations enter the tensor cores as a bf16 pair
+// so every matrix product runs on the 5th-generation tensor cores (tcgen05.mma
+// from TMA-fed shared memory into a tensor-memory accumulator, bf16 in, fp32
+// accumulate).  Activations enter the tensor cores as a bf16 pair
 // (x = hi + lo, hi = bf16(x), lo = bf16(x - hi)), so each product keeps close
 // to fp32 accuracy; weights are bf16 already.  The remaining steps (norms,
 // rotary + cache append, attention, top-k, expert lists, SwiGLU, combine,
@@ -11,54 +12,49 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "mk_internal.h"
 
 namespace mk {
 namespace {
 
-constexpr int kGemmN = 64;    // weight rows per block (MMA M, 4 warps x 16)
-constexpr int kGemmR = 64;    // activation rows per block (MMA N, 8 x 8)
-constexpr int kGemmK = 64;    // K columns per stage
-constexpr int kLd = kGemmK + 8;  // padded smem row (bf16): ldmatrix without bank conflicts
-constexpr int kGemmThreads = 128;
-
 __device__ __forceinline__ uint32_t sptr(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
-// 16-byte async copy; src_bytes < 16 fills the rest with zeros.
-__device__ __forceinline__ void cp16(void *dst, const void *src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sptr(dst)), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_wait_all_but_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(sptr(p)));
-}
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // ---------------------------------------------------------------------------
-// Y[r][n] (+)= sum_k W[n][k] * (xhi[r][k] + xlo[r][k]) for the rows of one
-// problem.  grid = (ceil(N / 64), ksplit, problems).  Problem p uses weights
-// W + p * wstride, activation rows [row_off[p], row_off[p] + row_cnt[p]) (or
-// [0, R) when row_off is NULL) and writes the same rows of Y.  With ksplit > 1
-// the block writes its K share into part[ks][row][n] for wide_gemm_finish.
+// Y[r][n] (+)= sum_k W[n][k] * (xhi[r][k] + xlo[r][k]) on the 5th-generation
+// tensor cores.  A CTA owns 128 weight rows (the MMA's M) of one problem and
+// all of its activation rows (the MMA's N: 16 to 64), over its share of K:
+//  - warp 0 (one thread) streams K in stages of 64 columns by TMA: a 128 x 64
+//    weight box and the activation rows in 16-row boxes, hi and lo, all
+//    128B-swizzled, completing on the stage's full mbarrier;
+//  - warp 1 (one thread) issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
+//    K = 16 each, hi then lo into one accumulator in tensor memory, and
+//    releases the stage with tcgen05.commit on its empty mbarrier;
+//  - then every warp reads its 32 accumulator lanes (weight rows) with
+//    tcgen05.ld and writes them out.
+// grid = (ceil(N / 128), ksplit, problems).  Problem p's weights are rows
+// [p * N, (p + 1) * N) of the weight map, its activation rows [row_off[p],
+// row_off[p] + row_cnt[p]) (or [0, R) when row_off is NULL); it writes the
+// same rows of Y.  With ksplit > 1 the CTA writes its K share into
+// part[ks][row][n] for wide_gemm_finish.
 // ---------------------------------------------------------------------------
+constexpr int kTcM = 128;                              // weight rows per CTA (MMA M)
+constexpr int kTcK = 64;                               // K columns per stage: one 128-byte swizzled row
+constexpr int kTcStages = 6;
+constexpr int kTcRowBox = 16;                          // activation rows per TMA box
+constexpr int kTcBoxBytes = kTcRowBox * kTcK * 2;      // 2 KB
+constexpr int kTcA = kTcM * kTcK * 2;                  // 16 KB of weights per stage
+constexpr int kTcB = kWideMaxRows * kTcK * 2;          // 8 KB per activation half (hi or lo)
+constexpr int kTcStage = kTcA + 2 * kTcB;
+constexpr int kTcThreads = 128;
+constexpr int kTcTmemCols = 64;                        // fp32 accumulator columns: one per activation row
+static_assert(kWideMaxRows <= kTcTmemCols, "one accumulator column per activation row");
+
 struct GemmArgs {
-  const __nv_bfloat16 *W;
-  long long wstride;
+  CUtensorMap mw;          // weights: [problems * N rows][K], box 64 x 128
+  CUtensorMap mxh, mxl;    // activations hi / lo: [rows][K], box 64 x 16
   int N, K;
-  const __nv_bfloat16 *xhi, *xlo;
-  int ldx;
   const int *row_off, *row_cnt;
   int R;
   float *Y;
@@ -66,103 +62,157 @@ struct GemmArgs {
   int accumulate;  // 1: Y += result (ksplit == 1 only)
   float *part;     // [ksplit][rows][ldy] when ksplit > 1
   int rows_total;  // rows of Y (for part's stride)
+  int *error;      // [0] code, [1] op: a bounded wait that ran out
 };
 
-__global__ void __launch_bounds__(kGemmThreads) wide_gemm(GemmArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__device__ __forceinline__ uint64_t tc_now() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool tc_try_wait(uint64_t *bar, uint32_t par) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(r)
+      : "r"(sptr(bar)), "r"(par)
+      : "memory");
+  return r != 0;
+}
+// Bounded wait (1 s); on timeout the error word is set and false returned.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t par, int *error) {
+  const uint64_t t0 = tc_now();
+  while (!tc_try_wait(bar, par)) {
+    if (tc_now() - t0 > 1000000000ull) {
+      if (atomicCAS(&error[0], 0, -5) == 0) atomicExch(&error[1], -2);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tc_tma(void *dst, const CUtensorMap *m, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          sptr(dst)),
+      "l"(m), "r"(x), "r"(y), "r"(sptr(bar))
+      : "memory");
+}
+// Shared-memory operand descriptor: K-major rows of 128 bytes, 128-byte
+// swizzle, 8-row groups 1024 bytes apart (descriptor version 1).
+__device__ __forceinline__ uint64_t tc_desc(const void *p) {
+  return static_cast<uint64_t>((sptr(p) >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(sptr(bar))
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  // stages start on 1024-byte boundaries (the 128-byte swizzle repeats every 8 rows)
+  uint8_t *smem = smem_raw + ((1024u - (sptr(smem_raw) & 1023u)) & 1023u);
+  __shared__ __align__(8) uint64_t full[kTcStages], empty[kTcStages], done;
+  __shared__ uint32_t tmem_base;
   const int prob = blockIdx.z;
   const int r0 = a.row_off ? a.row_off[prob] : 0;
   const int R = a.row_off ? a.row_cnt[prob] : a.R;
-  if (R <= 0) return;
-  const int n0 = blockIdx.x * kGemmN;
+  if (R <= 0) return;  // the whole CTA, before anything is allocated
+  const int n0 = blockIdx.x * kTcM;
   const int ksplit = gridDim.y, ks = blockIdx.y;
-  const int nkc = (a.K + kGemmK - 1) / kGemmK;
-  const int kc0 = (nkc * ks) / ksplit, kc1 = (nkc * (ks + 1)) / ksplit;
-  const __nv_bfloat16 *W = a.W + static_cast<long long>(prob) * a.wstride;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  __nv_bfloat16 *sW = reinterpret_cast<__nv_bfloat16 *>(smem);           // [2][64][kLd]
-  __nv_bfloat16 *sH = sW + 2 * kGemmN * kLd;                               // [2][64][kLd]
-  __nv_bfloat16 *sL = sH + 2 * kGemmR * kLd;                               // [2][64][kLd]
-
-  auto load_stage = [&](int st, int kc) {
-    const int k0 = kc * kGemmK;
-    // weights: 64 rows x 8 chunks of 8 bf16
-    for (int i = tid; i < kGemmN * 8; i += kGemmThreads) {
-      const int row = i >> 3, ch = i & 7, k = k0 + ch * 8, n = n0 + row;
-      const bool ok = n < a.N && k < a.K;
-      const __nv_bfloat16 *src = ok ? W + static_cast<long long>(n) * a.K + k : W;
-      cp16(sW + (st * kGemmN + row) * kLd + ch * 8, src, ok ? 16 : 0);
-    }
-    for (int i = tid; i < kGemmR * 8; i += kGemmThreads) {
-      const int row = i >> 3, ch = i & 7, k = k0 + ch * 8;
-      const bool ok = row < R && k < a.K;
-      const long long off = ok ? static_cast<long long>(r0 + row) * a.ldx + k : 0;
-      cp16(sH + (st * kGemmR + row) * kLd + ch * 8, a.xhi + off, ok ? 16 : 0);
-      cp16(sL + (st * kGemmR + row) * kLd + ch * 8, a.xlo + off, ok ? 16 : 0);
-    }
-    cp_commit();
-  };
-
-  float acc[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
-  const int nrt = (R + 7) / 8;  // 8-row activation tiles that hold rows
-
-  if (kc0 < kc1) load_stage(0, kc0);
-  for (int kc = kc0; kc < kc1; ++kc) {
-    const int st = (kc - kc0) & 1;
-    if (kc + 1 < kc1) {
-      load_stage(st ^ 1, kc + 1);
-      cp_wait_all_but_one();
-    } else {
-      cp_wait_all();
-    }
-    __syncthreads();
-    const __nv_bfloat16 *w_s = sW + st * kGemmN * kLd;
-    const __nv_bfloat16 *h_s = sH + st * kGemmR * kLd;
-    const __nv_bfloat16 *l_s = sL + st * kGemmR * kLd;
-#pragma unroll
-    for (int kk = 0; kk < kGemmK; kk += 16) {
-      uint32_t af[4];
-      {
-        const int mi = lane >> 3, ri = lane & 7;
-        ldsm_x4(af, w_s + (warp * 16 + (mi & 1) * 8 + ri) * kLd + kk + (mi >> 1) * 8);
-      }
-#pragma unroll
-      for (int jp = 0; jp < 4; ++jp) {  // two 8-row activation tiles per ldmatrix
-        if (2 * jp >= nrt) break;
-        const int mi = lane >> 3, ri = lane & 7;
-        const int row = jp * 16 + (mi >> 1) * 8 + ri, col = kk + (mi & 1) * 8;
-        uint32_t bh[4], bl[4];
-        ldsm_x4(bh, h_s + row * kLd + col);
-        ldsm_x4(bl, l_s + row * kLd + col);
-        mma_bf16(acc[2 * jp], af, bh[0], bh[1]);
-        mma_bf16(acc[2 * jp], af, bl[0], bl[1]);
-        mma_bf16(acc[2 * jp + 1], af, bh[2], bh[3]);
-        mma_bf16(acc[2 * jp + 1], af, bl[2], bl[3]);
-      }
-    }
-    __syncthreads();
+  const int nkc = (a.K + kTcK - 1) / kTcK;
+  const int kc0 = (nkc * ks) / ksplit, kc1 = (nkc * (ks + 1)) / ksplit, nk = kc1 - kc0;
+  const int G = (R + kTcRowBox - 1) / kTcRowBox, NM = kTcRowBox * G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sptr(&tmem_base)),
+                 "r"(kTcTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // D fragment: acc[j] = (weight row g, act rows 2t, 2t+1), (weight row g + 8, same)
-  const int g = lane >> 2, t = lane & 3;
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kTcStages; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&full[s])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&empty[s])) : "memory");
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&done)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = tmem_base;
+  // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
+  // K-major, N = NM, M = 128
+  const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(NM >> 3) << 17) |
+                         (static_cast<uint32_t>(kTcM >> 4) << 24);
+  if (warp == 0 && lane == 0) {  // TMA producer
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % kTcStages;
+      if (i >= kTcStages && !tc_wait(&empty[s], ((i / kTcStages) & 1) ^ 1, a.error)) break;
+      uint8_t *st = smem + s * kTcStage;
+      const int x = (kc0 + i) * kTcK;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&full[s])),
+                   "r"(kTcA + 2 * G * kTcBoxBytes)
+                   : "memory");
+      tc_tma(st, &a.mw, x, prob * a.N + n0, &full[s]);
+      for (int g = 0; g < G; ++g) {
+        tc_tma(st + kTcA + g * kTcBoxBytes, &a.mxh, x, r0 + kTcRowBox * g, &full[s]);
+        tc_tma(st + kTcA + kTcB + g * kTcBoxBytes, &a.mxl, x, r0 + kTcRowBox * g, &full[s]);
+      }
+    }
+  }
+  if (warp == 1 && lane == 0) {  // MMA issuer
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % kTcStages;
+      if (!tc_wait(&full[s], (i / kTcStages) & 1, a.error)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint8_t *st = smem + s * kTcStage;
+      const uint64_t da = tc_desc(st), dh = tc_desc(st + kTcA), dl = tc_desc(st + kTcA + kTcB);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+      for (int kk = 0; kk < kTcK / 16; ++kk) {  // 16 columns = 32 bytes = 2 descriptor units
+        tc_mma(tmem, da + 2 * kk, dh + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        tc_mma(tmem, da + 2 * kk, dl + 2 * kk, idesc, 1u);
+      }
+      tc_commit(&empty[s]);  // the stage is free once these products have read it
+    }
+    tc_commit(&done);
+  }
+  __syncwarp();
+  const bool ok = tc_wait(&done, 0, a.error) && nk > 0;
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  // warp w holds accumulator lanes 32w .. 32w + 31 = weight rows n0 + 32w + lane
+  const int n = n0 + 32 * warp + lane;
+  for (int c0 = 0; c0 < NM; c0 += 16) {
+    uint32_t v[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(tmem + (static_cast<uint32_t>(32 * warp) << 16) + static_cast<uint32_t>(c0)));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int n = n0 + warp * 16 + g + (q >> 1) * 8;
-      const int r = j * 8 + 2 * t + (q & 1);
-      if (n >= a.N || r >= R) continue;
+    for (int j = 0; j < 16; ++j) {
+      const int r = c0 + j;
+      if (r >= R || n >= a.N) continue;
+      const float val = ok ? __uint_as_float(v[j]) : 0.f;
       if (ksplit > 1) {
-        a.part[(static_cast<long long>(ks) * a.rows_total + r0 + r) * a.ldy + n] = acc[j][q];
+        a.part[(static_cast<long long>(ks) * a.rows_total + r0 + r) * a.ldy + n] = val;
       } else {
         float *y = a.Y + static_cast<long long>(r0 + r) * a.ldy + n;
-        *y = a.accumulate ? *y + acc[j][q] : acc[j][q];
+        *y = a.accumulate ? *y + val : val;
       }
     }
   }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols) : "memory");
 }
 
 // Y[r][n] (+)= sum over ks of part[ks][r][n], in order.
@@ -484,7 +534,7 @@ __global__ void wide_check(const int32_t *tokens, const int32_t *positions, int 
   if (bad && atomicCAS(&error[0], 0, -6) == 0) atomicExch(&error[1], 0);
 }
 
-int gemm_smem_bytes() { return 2 * (kGemmN + 2 * kGemmR) * kLd * static_cast<int>(sizeof(__nv_bfloat16)); }
+int gemm_smem_bytes() { return kTcStages * kTcStage + 1024; }  // + room to align the stages to 1024 bytes
 
 }  // namespace
 
@@ -497,18 +547,20 @@ int gemm_smem_bytes() { return 2 * (kGemmN + 2 * kGemmR) * kLd * static_cast<int
     if (e__ != cudaSuccess) return e__; \
   } while (0)
 
-static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, long long wstride, int N, int K,
-                        const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, const int *row_off,
-                        const int *row_cnt, int problems, int R, float *Y, int ldy, int accumulate,
-                        cudaStream_t st) {
+// One product (or one grouped launch of per-expert products) on the tensor
+// cores: weight rows [p * N, (p + 1) * N) x K for problem p, activation rows
+// of the xrows-row buffers xhi / xlo (row stride ldx).  A single dense problem
+// whose 128-row tiles do not fill the GPU splits K.
+static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, int problems, int N, int K,
+                        const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, int xrows, const int *row_off,
+                        const int *row_cnt, int R, float *Y, int ldy, int accumulate, cudaStream_t st) {
   GemmArgs a{};
-  a.W = W;
-  a.wstride = wstride;
+  if (encode_2d_sw128(&a.mw, W, static_cast<uint64_t>(problems) * N, K, K, kTcM) != MK_OK ||
+      encode_2d_sw128(&a.mxh, xhi, xrows, K, ldx, kTcRowBox) != MK_OK ||
+      encode_2d_sw128(&a.mxl, xlo, xrows, K, ldx, kTcRowBox) != MK_OK)
+    return cudaErrorInvalidValue;
   a.N = N;
   a.K = K;
-  a.xhi = xhi;
-  a.xlo = xlo;
-  a.ldx = ldx;
   a.row_off = row_off;
   a.row_cnt = row_cnt;
   a.R = R;
@@ -516,15 +568,16 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, long 
   a.ldy = ldy;
   a.accumulate = accumulate;
   a.rows_total = R;
-  const int nb = (N + kGemmN - 1) / kGemmN;
+  a.error = s.error;
+  const int nb = (N + kTcM - 1) / kTcM;
   int ksplit = 1;
-  if (!row_off) {  // one dense problem: split K until the grid covers the GPU twice
-    const int nkc = (K + kGemmK - 1) / kGemmK;
-    while (nb * ksplit < 2 * s.n_sm && ksplit * 2 <= nkc && ksplit < 16) ksplit *= 2;
+  if (!row_off) {  // one dense problem: about one CTA per SM, at least two K stages each
+    const int nkc = (K + kTcK - 1) / kTcK;
+    ksplit = std::max(1, std::min(std::min(s.n_sm / nb, nkc / 2), 16));
     if (static_cast<long long>(ksplit) * R * ldy > s.part_floats) ksplit = 1;
   }
   a.part = ksplit > 1 ? s.part : nullptr;
-  wide_gemm<<<dim3(nb, ksplit, problems), kGemmThreads, gemm_smem_bytes(), st>>>(a);
+  wide_gemm<<<dim3(nb, ksplit, problems), kTcThreads, gemm_smem_bytes(), st>>>(a);
   WIDE_TRY(cudaGetLastError());
   ++n;
   if (ksplit > 1) {
@@ -558,7 +611,7 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
                                        s.xlo, ldx);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wqkv), 0, W3, d, s.xhi, s.xlo, ldx, nullptr, nullptr, 1, M,
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wqkv), 1, W3, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M,
                   s.qkv, W3, 0, st));
     wide_kv_append<<<dim3(M, s.Hkv), 128, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, s.rope, s.kc,
                                                    s.vc, s.Bmax, s.cap, l);
@@ -571,14 +624,14 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     wide_split<<<M, 256, 0, st>>>(s.o, HD, HD, s.xhi, s.xlo, ldx);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), 0, d, HD, s.xhi, s.xlo, ldx, nullptr, nullptr, 1, M,
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), 1, d, HD, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M,
                   s.h, d, 1, st));
     // MoE block: router on the normed row, top-k, expert lists
     wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.ffn_norm), d, s.eps, s.xhi, s.xlo,
                                        ldx);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), 0, E, d, s.xhi, s.xlo, ldx, nullptr, nullptr, 1, M,
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), 1, E, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M,
                   s.rlog, E, 0, st));
     int32_t *dbg_ids = s.dbg_ids ? s.dbg_ids + static_cast<long long>(l) * s.max_rows * K : nullptr;
     float *dbg_w = s.dbg_w ? s.dbg_w + static_cast<long long>(l) * s.max_rows * K : nullptr;
@@ -592,26 +645,26 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     wide_gather<<<M * K, 256, 0, st>>>(s.xhi, s.xlo, ldx, s.pair_row, d, s.ghi, s.glo);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), static_cast<long long>(F) * d, F, d, s.ghi, s.glo,
-                  ldx, s.off, s.count, E, M * K, s.gu, 2 * F, 0, st));
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_up), static_cast<long long>(F) * d, F, d, s.ghi, s.glo,
-                  ldx, s.off, s.count, E, M * K, s.gu + F, 2 * F, 0, st));
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), E, F, d, s.ghi, s.glo, ldx, M * K, s.off, s.count,
+                  M * K, s.gu, 2 * F, 0, st));
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_up), E, F, d, s.ghi, s.glo, ldx, M * K, s.off, s.count,
+                  M * K, s.gu + F, 2 * F, 0, st));
     wide_swiglu<<<M * K, 256, 0, st>>>(s.gu, F, s.ahi, s.alo, s.lda);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), static_cast<long long>(d) * F, d, F, s.ahi, s.alo,
-                  s.lda, s.off, s.count, E, M * K, s.yd, d, 0, st));
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), E, d, F, s.ahi, s.alo, s.lda, M * K, s.off,
+                  s.count, M * K, s.yd, d, 0, st));
     // shared expert on every row
     if (Fs > 0) {
-      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_gate), 0, Fs, d, s.xhi, s.xlo, ldx, nullptr, nullptr,
-                    1, M, s.gs, 2 * Fs, 0, st));
-      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_up), 0, Fs, d, s.xhi, s.xlo, ldx, nullptr, nullptr, 1,
+      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_gate), 1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr,
+                    nullptr, M, s.gs, 2 * Fs, 0, st));
+      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_up), 1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr,
                     M, s.gs + Fs, 2 * Fs, 0, st));
       wide_swiglu<<<M, 256, 0, st>>>(s.gs, Fs, s.shi, s.slo, s.lda);
       WIDE_TRY(cudaGetLastError());
       ++n;
-      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), 0, d, Fs, s.shi, s.slo, s.lda, nullptr, nullptr,
-                    1, M, s.ys, d, 0, st));
+      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), 1, d, Fs, s.shi, s.slo, s.lda, M, nullptr,
+                    nullptr, M, s.ys, d, 0, st));
     }
     float *dbg = s.dbg_hidden ? s.dbg_hidden + static_cast<long long>(l + 1) * s.max_rows * d : nullptr;
     wide_combine<<<M, 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr, dbg);
@@ -622,7 +675,7 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
   wide_norm_split<<<M, 256, 0, st>>>(s.h, s.final_norm, d, s.eps, s.xhi, s.xlo, ldx);
   WIDE_TRY(cudaGetLastError());
   ++n;
-  WIDE_TRY(gemm(n, s, s.lm_head, 0, s.V, d, s.xhi, s.xlo, ldx, nullptr, nullptr, 1, M, s.logits, s.V, 0, st));
+  WIDE_TRY(gemm(n, s, s.lm_head, 1, s.V, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.logits, s.V, 0, st));
   wide_argmax<<<M, 256, 0, st>>>(s.logits, s.V, s.argmax);
   WIDE_TRY(cudaGetLastError());
   if (launches) *launches = n + 1;
