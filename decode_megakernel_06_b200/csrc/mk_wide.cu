@@ -25,9 +25,9 @@ __device__ __forceinline__ uint32_t sptr(const void *p) { return static_cast<uin
 // Y[r][n] (+)= sum_k W[n][k] * (xhi[r][k] + xlo[r][k]) on the 5th-generation
 // tensor cores.  A CTA owns 128 weight rows (the MMA's M) of one problem and
 // all of its activation rows (the MMA's N: 16 to 64), over its share of K:
-//  - warp 0 (one thread) streams K in stages of 64 columns by TMA: a 128 x 64
-//    weight box and the activation rows in 16-row boxes, hi and lo, all
-//    128B-swizzled, completing on the stage's full mbarrier;
+//  - warp 0 (one thread) streams K in stages of 128 columns by TMA: per 64
+//    columns a 128 x 64 weight box and the activation rows in 16-row boxes,
+//    hi and lo, all 128B-swizzled, completing on the stage's full mbarrier;
 //  - warp 1 (one thread) issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
 //    K = 16 each, hi then lo into one accumulator in tensor memory, and
 //    releases the stage with tcgen05.commit on its empty mbarrier;
@@ -40,12 +40,15 @@ __device__ __forceinline__ uint32_t sptr(const void *p) { return static_cast<uin
 // part[ks][row][n] for wide_gemm_finish.
 // ---------------------------------------------------------------------------
 constexpr int kTcM = 128;                              // weight rows per CTA (MMA M)
-constexpr int kTcK = 64;                               // K columns per stage: one 128-byte swizzled row
-constexpr int kTcStages = 6;
+constexpr int kTcK = 64;                               // K columns per box: one 128-byte swizzled row
+constexpr int kTcBoxes = 2;                            // K boxes per stage (a stage spans 128 columns)
+constexpr int kTcStages = 3;                           // measured against 1 box x 6 stages: 4.7 / 4.0 TB/s
 constexpr int kTcRowBox = 16;                          // activation rows per TMA box
 constexpr int kTcBoxBytes = kTcRowBox * kTcK * 2;      // 2 KB
-constexpr int kTcA = kTcM * kTcK * 2;                  // 16 KB of weights per stage
-constexpr int kTcB = kWideMaxRows * kTcK * 2;          // 8 KB per activation half (hi or lo)
+constexpr int kTcWBox = kTcM * kTcK * 2;               // 16 KB weight box
+constexpr int kTcXBox = kWideMaxRows * kTcK * 2;       // 8 KB: up to 64 activation rows of one box
+constexpr int kTcA = kTcBoxes * kTcWBox;               // weights per stage
+constexpr int kTcB = kTcBoxes * kTcXBox;               // one activation half (hi or lo) per stage
 constexpr int kTcStage = kTcA + 2 * kTcB;
 constexpr int kTcThreads = 128;
 constexpr int kTcTmemCols = 64;                        // fp32 accumulator columns: one per activation row
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
   if (R <= 0) return;  // the whole CTA, before anything is allocated
   const int n0 = blockIdx.x * kTcM;
   const int ksplit = gridDim.y, ks = blockIdx.y;
-  const int nkc = (a.K + kTcK - 1) / kTcK;
+  const int nkc = (a.K + kTcBoxes * kTcK - 1) / (kTcBoxes * kTcK);
   const int kc0 = (nkc * ks) / ksplit, kc1 = (nkc * (ks + 1)) / ksplit, nk = kc1 - kc0;
   const int G = (R + kTcRowBox - 1) / kTcRowBox, NM = kTcRowBox * G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -156,14 +159,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       const int s = i % kTcStages;
       if (i >= kTcStages && !tc_wait(&empty[s], ((i / kTcStages) & 1) ^ 1, a.error)) break;
       uint8_t *st = smem + s * kTcStage;
-      const int x = (kc0 + i) * kTcK;
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&full[s])),
-                   "r"(kTcA + 2 * G * kTcBoxBytes)
+                   "r"(kTcBoxes * (kTcWBox + 2 * G * kTcBoxBytes))
                    : "memory");
-      tc_tma(st, &a.mw, x, prob * a.N + n0, &full[s]);
-      for (int g = 0; g < G; ++g) {
-        tc_tma(st + kTcA + g * kTcBoxBytes, &a.mxh, x, r0 + kTcRowBox * g, &full[s]);
-        tc_tma(st + kTcA + kTcB + g * kTcBoxBytes, &a.mxl, x, r0 + kTcRowBox * g, &full[s]);
+      for (int b = 0; b < kTcBoxes; ++b) {  // columns past K read as zeros
+        const int x = ((kc0 + i) * kTcBoxes + b) * kTcK;
+        tc_tma(st + b * kTcWBox, &a.mw, x, prob * a.N + n0, &full[s]);
+        for (int g = 0; g < G; ++g) {
+          tc_tma(st + kTcA + b * kTcXBox + g * kTcBoxBytes, &a.mxh, x, r0 + kTcRowBox * g, &full[s]);
+          tc_tma(st + kTcA + kTcB + b * kTcXBox + g * kTcBoxBytes, &a.mxl, x, r0 + kTcRowBox * g, &full[s]);
+        }
       }
     }
   }
@@ -173,11 +178,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       if (!tc_wait(&full[s], (i / kTcStages) & 1, a.error)) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint8_t *st = smem + s * kTcStage;
-      const uint64_t da = tc_desc(st), dh = tc_desc(st + kTcA), dl = tc_desc(st + kTcA + kTcB);
 #pragma unroll
-      for (int kk = 0; kk < kTcK / 16; ++kk) {  // 16 columns = 32 bytes = 2 descriptor units
-        tc_mma(tmem, da + 2 * kk, dh + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-        tc_mma(tmem, da + 2 * kk, dl + 2 * kk, idesc, 1u);
+      for (int b = 0; b < kTcBoxes; ++b) {
+        const uint64_t da = tc_desc(st + b * kTcWBox), dh = tc_desc(st + kTcA + b * kTcXBox),
+                       dl = tc_desc(st + kTcA + kTcB + b * kTcXBox);
+#pragma unroll
+        for (int kk = 0; kk < kTcK / 16; ++kk) {  // 16 columns = 32 bytes = 2 descriptor units
+          tc_mma(tmem, da + 2 * kk, dh + 2 * kk, idesc, (i > 0 || b > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem, da + 2 * kk, dl + 2 * kk, idesc, 1u);
+        }
       }
       tc_commit(&empty[s]);  // the stage is free once these products have read it
     }
@@ -302,64 +311,136 @@ __global__ void wide_kv_append(const float *qkv, int W3, const int32_t *position
   }
 }
 
-// Softmax attention of one (row, query head) over cache positions 0..p,
-// including the rows this step appended.  grid = (M, Hq), 128 threads: each
-// warp keeps an online softmax over every 4th position, lanes across the
-// head dimension; the warps merge at the end.
-constexpr int kAttnWarps = 4;
-__global__ void __launch_bounds__(kAttnWarps * 32) wide_attention(
-    const float *qkv, int W3, const int32_t *positions, int T, int Hq, int Hkv, int hd, const float2 *rope,
-    const __nv_bfloat16 *kc, const __nv_bfloat16 *vc, int Bmax, int cap, int layer, float *o) {
-  __shared__ float sq[128];
-  __shared__ float sm[kAttnWarps], sl[kAttnWarps];
-  __shared__ float so[kAttnWarps][128];
-  const int m = blockIdx.x, h = blockIdx.y, b = m / T, t = m % T;
-  const int p = positions[b] + t, half = hd / 2, G = Hq / Hkv, g = h / G;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float scale = 1.0f / sqrtf(static_cast<float>(hd));
-  const float *q = qkv + static_cast<long long>(m) * W3 + h * hd;
-  for (int i = threadIdx.x; i < hd; i += blockDim.x) {
-    const int j = i < half ? i : i - half;
-    const float2 cs = rope[static_cast<long long>(p) * half + j];
-    const float qr = i < half ? q[i] * cs.x - q[i + half] * cs.y : q[i] * cs.x + q[i - half] * cs.y;
-    sq[i] = qr * scale;
-  }
-  __syncthreads();
-  const int dpl = hd / 32;  // 2 or 4 dims per lane
-  float qv[4], acc[4];
-  for (int i = 0; i < 4; ++i) {
-    qv[i] = i < dpl ? sq[lane * dpl + i] : 0.f;
-    acc[i] = 0.f;
-  }
+// Attention of a wide block, split over the KV positions: one block per
+// (sequence, KV head, chunk of kWaChunk positions) stages the chunk's K and V
+// rows in shared memory once and scores every query vector of the group
+// against them (T rows x Hq/Hkv heads, each seeing positions up to its own),
+// writing per query an unnormalised partial output with its running max and
+// sum; wide_attn_merge combines a query's chunks with the log-sum-exp rule.
+// Lane j of a warp scores positions j and j + 32 of the chunk (rows padded
+// by 8 bf16 so that the lanes' row reads fall in different banks); for P.V
+// lane l owns dims [DPL l, DPL l + DPL).
+constexpr int kWaChunk = 64;
+constexpr int kWaWarps = 8;
+constexpr int kWaPad = 8;
+template <int DPL>
+__global__ void __launch_bounds__(kWaWarps * 32) wide_attn_chunk(
+    const float *qkv, int W3, const int32_t *positions, int T, int Hq, int Hkv, const float2 *rope,
+    const __nv_bfloat16 *kc, const __nv_bfloat16 *vc, int Bmax, int cap, int layer, int nch_max, float *opart,
+    float *mlpart) {
+  constexpr int HD = 32 * DPL, HALF = HD / 2, LD = HD + kWaPad;
+  __shared__ __align__(16) __nv_bfloat16 sk[kWaChunk * LD], sv[kWaChunk * LD];
+  __shared__ __align__(16) float sq[kWaWarps][HD];
+  const int c = blockIdx.x, bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
+  const int pos0 = positions[b], last = pos0 + T - 1;  // the block's last query sees up to `last`
+  const int j0 = c * kWaChunk;
+  if (j0 > last) return;
+  const int nj = min(kWaChunk, last + 1 - j0);
   const long long base = ((static_cast<long long>(layer) * Bmax + b) * Hkv + g) * cap;
-  float mrun = -INFINITY, lrun = 0.f;
-  for (int j = warp; j <= p; j += kAttnWarps) {
-    const __nv_bfloat16 *kr = kc + (base + j) * hd + lane * dpl;
-    float s = 0.f;
-    for (int i = 0; i < dpl; ++i) s = fmaf(qv[i], __bfloat162float(kr[i]), s);
-    for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    const float mn = fmaxf(mrun, s);
-    const float a = (mrun == -INFINITY) ? 0.f : expf(mrun - mn);
-    const float e = expf(s - mn);
-    lrun = lrun * a + e;
-    const __nv_bfloat16 *vr = vc + (base + j) * hd + lane * dpl;
-    for (int i = 0; i < dpl; ++i) acc[i] = acc[i] * a + e * __bfloat162float(vr[i]);
-    mrun = mn;
+  // stage the chunk's rows: 16-byte pieces, HD / 8 per row
+  for (int i = threadIdx.x; i < nj * (HD / 8); i += blockDim.x) {
+    const int j = i / (HD / 8), piece = i % (HD / 8);
+    const uint4 kv4 = *reinterpret_cast<const uint4 *>(kc + (base + j0 + j) * HD + piece * 8);
+    const uint4 vv4 = *reinterpret_cast<const uint4 *>(vc + (base + j0 + j) * HD + piece * 8);
+    *reinterpret_cast<uint4 *>(sk + j * LD + piece * 8) = kv4;
+    *reinterpret_cast<uint4 *>(sv + j * LD + piece * 8) = vv4;
   }
-  if (lane == 0) {
-    sm[warp] = mrun;
-    sl[warp] = lrun;
-  }
-  for (int i = 0; i < dpl; ++i) so[warp][lane * dpl + i] = acc[i];
   __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float scale = 1.0f / sqrtf(static_cast<float>(HD));
+  const int Q = T * G;
+  for (int qi = warp; qi < Q; qi += kWaWarps) {
+    const int t = qi / G, h = g * G + qi % G, m = b * T + t, lim = pos0 + t;
+    // the query vector, rotated (rotate-half pairs) and scaled, in this warp's buffer
+    const float *q = qkv + static_cast<long long>(m) * W3 + h * HD;
+    for (int i = lane; i < HALF; i += 32) {
+      const float2 cs = rope[static_cast<long long>(lim) * HALF + i];
+      const float x1 = q[i], x2 = q[i + HALF];
+      sq[warp][i] = (x1 * cs.x - x2 * cs.y) * scale;
+      sq[warp][i + HALF] = (x2 * cs.x + x1 * cs.y) * scale;
+    }
+    __syncwarp();
+    float s[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = lane + 32 * u;
+      float acc = 0.f;
+      if (j < nj && j0 + j <= lim) {
+        const __nv_bfloat16 *kr = sk + j * LD;
+#pragma unroll 8
+        for (int d = 0; d < HD; d += 8) {
+          const uint4 kk = *reinterpret_cast<const uint4 *>(kr + d);
+          const float4 qa = *reinterpret_cast<const float4 *>(&sq[warp][d]);
+          const float4 qb = *reinterpret_cast<const float4 *>(&sq[warp][d + 4]);
+          acc = fmaf(qa.x, __uint_as_float(kk.x << 16), acc);
+          acc = fmaf(qa.y, __uint_as_float(kk.x & 0xffff0000u), acc);
+          acc = fmaf(qa.z, __uint_as_float(kk.y << 16), acc);
+          acc = fmaf(qa.w, __uint_as_float(kk.y & 0xffff0000u), acc);
+          acc = fmaf(qb.x, __uint_as_float(kk.z << 16), acc);
+          acc = fmaf(qb.y, __uint_as_float(kk.z & 0xffff0000u), acc);
+          acc = fmaf(qb.z, __uint_as_float(kk.w << 16), acc);
+          acc = fmaf(qb.w, __uint_as_float(kk.w & 0xffff0000u), acc);
+        }
+        s[u] = acc;
+      } else {
+        s[u] = -INFINITY;
+      }
+    }
+    float mx = fmaxf(s[0], s[1]);
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float p[2], l = 0.f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      p[u] = (s[u] == -INFINITY) ? 0.f : expf(s[u] - mx);
+      l += p[u];
+    }
+    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    float acc[DPL];
+#pragma unroll
+    for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
+    if (mx != -INFINITY) {
+      for (int j = 0; j < nj; ++j) {
+        const float pj = __shfl_sync(0xffffffffu, p[j >> 5], j & 31);
+        const __nv_bfloat16 *vr = sv + j * LD + lane * DPL;
+#pragma unroll
+        for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(pj, __bfloat162float(vr[dd]), acc[dd]);
+      }
+    }
+    const long long slot = (static_cast<long long>(bg) * nch_max + c) * (static_cast<long long>(T) * G) + qi;
+    float *dst = opart + slot * HD + lane * DPL;
+#pragma unroll
+    for (int dd = 0; dd < DPL; ++dd) dst[dd] = acc[dd];
+    if (lane == 0) {
+      mlpart[2 * slot] = mx;
+      mlpart[2 * slot + 1] = l;
+    }
+    __syncwarp();  // the buffer of q is rewritten by the warp's next query
+  }
+}
+
+// o[m][h] = the log-sum-exp combination of query (m, h)'s chunk partials.
+// One block of HD threads per (row, head); thread i owns dim i.
+__global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv, int hd, int nch_max,
+                                const float *opart, const float *mlpart, float *o) {
+  const int m = blockIdx.x, h = blockIdx.y, b = m / T, t = m % T, G = Hq / Hkv, g = h / G;
+  const int qi = t * G + h % G, bg = b * Hkv + g;
+  const int nch = (positions[b] + t) / kWaChunk + 1;  // chunks holding positions this query sees
   float M = -INFINITY;
-  for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, sm[w]);
-  float L = 0.f;
-  for (int w = 0; w < kAttnWarps; ++w) L += (sm[w] == -INFINITY) ? 0.f : expf(sm[w] - M) * sl[w];
+  for (int c = 0; c < nch; ++c) {
+    const long long slot = (static_cast<long long>(bg) * nch_max + c) * (static_cast<long long>(T) * G) + qi;
+    M = fmaxf(M, mlpart[2 * slot]);
+  }
   for (int i = threadIdx.x; i < hd; i += blockDim.x) {
-    float s = 0.f;
-    for (int w = 0; w < kAttnWarps; ++w) s += (sm[w] == -INFINITY) ? 0.f : expf(sm[w] - M) * so[w][i];
-    o[static_cast<long long>(m) * Hq * hd + h * hd + i] = s / L;
+    float num = 0.f, den = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const long long slot = (static_cast<long long>(bg) * nch_max + c) * (static_cast<long long>(T) * G) + qi;
+      const float mc = mlpart[2 * slot];
+      if (mc == -INFINITY) continue;
+      const float w = expf(mc - M);
+      num = fmaf(w, opart[slot * hd + i], num);
+      den = fmaf(w, mlpart[2 * slot + 1], den);
+    }
+    o[static_cast<long long>(m) * Hq * hd + h * hd + i] = num / den;
   }
 }
 
@@ -572,7 +653,7 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, int p
   const int nb = (N + kTcM - 1) / kTcM;
   int ksplit = 1;
   if (!row_off) {  // one dense problem: about one CTA per SM, at least two K stages each
-    const int nkc = (K + kTcK - 1) / kTcK;
+    const int nkc = (K + kTcBoxes * kTcK - 1) / (kTcBoxes * kTcK);
     ksplit = std::max(1, std::min(std::min(s.n_sm / nb, nkc / 2), 16));
     if (static_cast<long long>(ksplit) * R * ldy > s.part_floats) ksplit = 1;
   }
@@ -617,10 +698,22 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
                                                    s.vc, s.Bmax, s.cap, l);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    wide_attention<<<dim3(M, s.Hq), kAttnWarps * 32, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd,
-                                                              s.rope, s.kc, s.vc, s.Bmax, s.cap, l, s.o);
-    WIDE_TRY(cudaGetLastError());
-    ++n;
+    {
+      const int nch = (s.cap + kWaChunk - 1) / kWaChunk;
+      const dim3 grid(nch, s.B * s.Hkv);
+      if (s.hd == 64)
+        wide_attn_chunk<2><<<grid, kWaWarps * 32, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.rope, s.kc,
+                                                            s.vc, s.Bmax, s.cap, l, nch, s.attn_o, s.attn_ml);
+      else
+        wide_attn_chunk<4><<<grid, kWaWarps * 32, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.rope, s.kc,
+                                                            s.vc, s.Bmax, s.cap, l, nch, s.attn_o, s.attn_ml);
+      WIDE_TRY(cudaGetLastError());
+      ++n;
+      wide_attn_merge<<<dim3(M, s.Hq), s.hd, 0, st>>>(s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
+                                                      s.attn_ml, s.o);
+      WIDE_TRY(cudaGetLastError());
+      ++n;
+    }
     wide_split<<<M, 256, 0, st>>>(s.o, HD, HD, s.xhi, s.xlo, ldx);
     WIDE_TRY(cudaGetLastError());
     ++n;
