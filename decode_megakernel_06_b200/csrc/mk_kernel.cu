@@ -1083,35 +1083,64 @@ MK_INLINE int xs_pos4(int c4) {  // float4 slot of columns 4*c4 .. 4*c4+3
 }
 MK_INLINE int xperm(int col) { return 4 * xs_pos4(col >> 2) + (col & 3); }
 
-// MJ activation rows (row[j] of src, stride ld), read 8 consecutive columns
-// per lane: from global memory through L1 (SH false) or from the CTA's staged
-// copy in shared memory (SH true).
+// The rows' addresses, resolved once per unit: rows past the unit's count
+// repeat its first row (their sums are never stored), so every load is
+// unconditional and the loads of all rows issue together.  Shared memory rows
+// are held as 32-bit shared addresses, global ones as 32-bit offsets from one
+// base, to keep the unit's loop light on registers.
+MK_INLINE float4 lds_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+template <int MJ, bool SH>
+struct XPtrs {
+  const float *base;  // global rows
+  uint32_t ra[MJ];    // shared: byte address of row j; global: float offset of row j from base
+  MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
+    if (col < K) {
+      const int off = (col & ~(kPanel - 1)) + ((col & (kPanel - 1)) >> 1);
+#pragma unroll
+      for (int j = 0; j < MJ; ++j) {
+        float4 a, b;
+        if constexpr (SH) {
+          a = lds_f4(ra[j] + 4u * off);
+          b = lds_f4(ra[j] + 4u * (off + kPanel / 2));
+        } else {
+          const float *pb = base + ra[j] + off;
+          a = __ldca(reinterpret_cast<const float4 *>(pb));
+          b = __ldca(reinterpret_cast<const float4 *>(pb + kPanel / 2));
+        }
+        x[j][0] = a.x; x[j][1] = a.y; x[j][2] = a.z; x[j][3] = a.w;
+        x[j][4] = b.x; x[j][5] = b.y; x[j][6] = b.z; x[j][7] = b.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < MJ; ++j)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[j][k] = 0.f;
+    }
+  }
+};
+
+// MJ activation rows (row[j] of src, stride ld, n of them), read 8
+// consecutive columns per lane: from global memory through L1 (SH false) or
+// from the CTA's staged copy in shared memory (SH true).
 template <int MJ, bool SH>
 struct XRows {
   const float *src;
   int ld;
   int row[MJ];
   int n;
-  MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
+  MK_INLINE XPtrs<MJ, SH> ptrs() const {
+    XPtrs<MJ, SH> p;
+    p.base = src;
 #pragma unroll
     for (int j = 0; j < MJ; ++j) {
-      if (col < K && j < n) {
-        const float *pb = src + static_cast<size_t>(row[j]) * ld + (col & ~(kPanel - 1)) + ((col & (kPanel - 1)) >> 1);
-        float4 a, b;
-        if constexpr (SH) {
-          a = *reinterpret_cast<const float4 *>(pb);
-          b = *reinterpret_cast<const float4 *>(pb + kPanel / 2);
-        } else {
-          a = __ldca(reinterpret_cast<const float4 *>(pb));
-          b = __ldca(reinterpret_cast<const float4 *>(pb + kPanel / 2));
-        }
-        x[j][0] = a.x; x[j][1] = a.y; x[j][2] = a.z; x[j][3] = a.w;
-        x[j][4] = b.x; x[j][5] = b.y; x[j][6] = b.z; x[j][7] = b.w;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) x[j][k] = 0.f;
-      }
+      const uint32_t r = static_cast<uint32_t>(j < n ? row[j] : row[0]) * static_cast<uint32_t>(ld);
+      p.ra[j] = SH ? saddr(src) + 4u * r : r;
     }
+    return p;
   }
 };
 template <int MJ>
@@ -1155,7 +1184,7 @@ MK_INLINE void gemv_panel(const uint8_t *pan, float (&acc)[kRows * MJ], float (&
 // acc[r*MJ + j] += W[r][cols] . x[j][cols] over this lane's columns.
 template <int MJ, class XS>
 MK_INLINE void gemv_tile(const uint8_t *slot, float (&acc)[kRows * MJ], float (&acc2)[kRows * MJ], int colbase,
-                         int K, const XS &xs, int lane) {
+                         int K, const XS &xs, int lane) {  // xs: an XPtrs
   const uint8_t *base = slot + lane * 16;
   if constexpr (MJ <= 2) {
     // every panel's activations first: one memory round trip per tile
@@ -1183,10 +1212,11 @@ MK_INLINE bool gemv_stream(Warp &w, int op, int ntiles, int col0, int K, const X
   float acc2[kRows * MJ];  // the odd columns' partial sums
 #pragma unroll
   for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
+  const auto xp = xs.ptrs();
   for (int t = 0; t < ntiles; ++t) {
     const uint8_t *slot = consume_begin(w, op);
     if (!slot) return false;
-    gemv_tile<MJ>(slot, acc, acc2, col0 + t * kTileCols, K, xs, w.lane);
+    gemv_tile<MJ>(slot, acc, acc2, col0 + t * kTileCols, K, xp, w.lane);
     consume_end(w);
   }
 #pragma unroll
@@ -1229,14 +1259,15 @@ MK_INLINE bool gemv_two_groups_by_column(Warp &w, int op, int K, const XS &xs, f
   float a0[kRows * MJ], a0b[kRows * MJ], a1[kRows * MJ], a1b[kRows * MJ];
 #pragma unroll
   for (int q = 0; q < kRows * MJ; ++q) a0[q] = a0b[q] = a1[q] = a1b[q] = 0.f;
+  const auto xp = xs.ptrs();
   for (int c = 0; c < nbx; c += 2) {
     const uint8_t *slot = consume_begin(w, op);
     if (!slot) return false;
     const uint8_t *base = slot + w.lane * 16;
     float x0[MJ][8], x1[MJ][8];
-    xs.load(c * kPanel + w.lane * 8, K, x0);
+    xp.load(c * kPanel + w.lane * 8, K, x0);
     const bool two = c + 1 < nbx;
-    if (two) xs.load((c + 1) * kPanel + w.lane * 8, K, x1);
+    if (two) xp.load((c + 1) * kPanel + w.lane * 8, K, x1);
     gemv_panel<MJ>(base, a0, a0b, x0);
     gemv_panel<MJ>(base + kBoxBytes, a1, a1b, x0);
     if (two) {
@@ -1260,19 +1291,20 @@ MK_INLINE bool gemv_groups(Warp &w, int op, int ngroups, int K, const XS &xs, fl
   float acc[kRows * MJ], acc2[kRows * MJ];
 #pragma unroll
   for (int q = 0; q < kRows * MJ; ++q) acc[q] = acc2[q] = 0.f;
+  const auto xp = xs.ptrs();
   for (int b0 = 0; b0 < nb; b0 += kPanels) {
     const uint8_t *slot = consume_begin(w, op);
     if (!slot) return false;
     const uint8_t *base = slot + w.lane * 16;
     const int g0 = b0 / nbx, c0 = b0 - g0 * nbx;
     if (b0 + kPanels <= nb && c0 + kPanels <= nbx) {
-      gemv_tile<MJ>(slot, acc, acc2, c0 * kPanel, K, xs, w.lane);
+      gemv_tile<MJ>(slot, acc, acc2, c0 * kPanel, K, xp, w.lane);
       if (c0 + kPanels == nbx) group_done<MJ>(acc, acc2, buf + g0 * kRows * MJ, w.lane);
     } else {
       for (int q = 0; q < kPanels && b0 + q < nb; ++q) {
         const int b = b0 + q, g = b / nbx, c = b - g * nbx;
         float x[MJ][8];
-        xs.load(c * kPanel + w.lane * 8, K, x);
+        xp.load(c * kPanel + w.lane * 8, K, x);
         gemv_panel<MJ>(base + q * kBoxBytes, acc, acc2, x);
         if (c == nbx - 1) group_done<MJ>(acc, acc2, buf + g * kRows * MJ, w.lane);
       }
