@@ -1097,17 +1097,19 @@ template <int MJ, bool SH>
 struct XPtrs {
   const float *base;  // global rows
   uint32_t ra[MJ];    // shared: byte address of row j; global: float offset of row j from base
-  MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const {
+  // rows J0 .. J0 + JN - 1
+  template <int J0, int JN>
+  MK_INLINE void load_part(int col, int K, float (&x)[JN][8]) const {
     if (col < K) {
       const int off = (col & ~(kPanel - 1)) + ((col & (kPanel - 1)) >> 1);
 #pragma unroll
-      for (int j = 0; j < MJ; ++j) {
+      for (int j = 0; j < JN; ++j) {
         float4 a, b;
         if constexpr (SH) {
-          a = lds_f4(ra[j] + 4u * off);
-          b = lds_f4(ra[j] + 4u * (off + kPanel / 2));
+          a = lds_f4(ra[J0 + j] + 4u * off);
+          b = lds_f4(ra[J0 + j] + 4u * (off + kPanel / 2));
         } else {
-          const float *pb = base + ra[j] + off;
+          const float *pb = base + ra[J0 + j] + off;
           a = __ldca(reinterpret_cast<const float4 *>(pb));
           b = __ldca(reinterpret_cast<const float4 *>(pb + kPanel / 2));
         }
@@ -1116,11 +1118,12 @@ struct XPtrs {
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < MJ; ++j)
+      for (int j = 0; j < JN; ++j)
 #pragma unroll
         for (int k = 0; k < 8; ++k) x[j][k] = 0.f;
     }
   }
+  MK_INLINE void load(int col, int K, float (&x)[MJ][8]) const { load_part<0, MJ>(col, K, x); }
 };
 
 // MJ activation rows (row[j] of src, stride ld, n of them), read 8
@@ -1720,12 +1723,22 @@ MK_INLINE bool routed_dispatch(Warp &w, int op, int type, int layer, int unit, c
 // in the lane.  A score is reduced over the 8 dl lanes only; the kQvp = 4
 // query vectors of the item end up one per lane pair (query dl / 2).
 
-// c consecutive bf16 values (c = 8 or 4) from shared memory, as c / 2
+// c consecutive bf16 values (c = 16, 8 or 4) from shared memory, as c / 2
 // (even, odd) float pairs.
 template <int C>
 MK_INLINE void lds_bf16x2(const __nv_bfloat16 *p, float2 (&f)[C / 2]) {
-  static_assert(C == 8 || C == 4, "head_dim 128 or 64");
-  if constexpr (C == 8) {
+  static_assert(C == 16 || C == 8 || C == 4, "8 or 16 values of a 64- or 128-wide head");
+  if constexpr (C == 16) {
+    const uint4 u = ld_shared_v4(p), u2 = ld_shared_v4(p + 8);
+    f[0] = bf2(u.x);
+    f[1] = bf2(u.y);
+    f[2] = bf2(u.z);
+    f[3] = bf2(u.w);
+    f[4] = bf2(u2.x);
+    f[5] = bf2(u2.y);
+    f[6] = bf2(u2.z);
+    f[7] = bf2(u2.w);
+  } else if constexpr (C == 8) {
     const uint4 u = ld_shared_v4(p);
     f[0] = bf2(u.x);
     f[1] = bf2(u.y);
@@ -1779,11 +1792,12 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
   const int d0 = C * dl, d1 = HALF + C * dl;
   float m_run = -INFINITY, l_run = 0.f;
   constexpr int DP = DL / 2, CP = C / 2;  // float pairs per lane and per chunk
-  float2 o[QVP][DP];
+  // P.V runs on another lane layout: lane (vq, dc) = (lane >> 3, lane & 7)
+  // accumulates query vq's output on dims [DL dc, DL dc + DL)
+  const int vq = lane >> 3, dc = lane & 7;
+  float2 ov[DP];
 #pragma unroll
-  for (int v = 0; v < QVP; ++v)
-#pragma unroll
-    for (int k = 0; k < DP; ++k) o[v][k] = make_float2(0.f, 0.f);
+  for (int k = 0; k < DP; ++k) ov[k] = make_float2(0.f, 0.f);
   if (a.ntiles > 0) {
     // the item's query vectors, staged by the CTA: this lane's dimensions
     float2 q[QVP][DP];
@@ -1874,56 +1888,36 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
       ps += __shfl_xor_sync(0xffffffffu, ps, 16);
       l_run = l_run * alpha + ps;
       m_run = m_new;
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      // rescale query vq's output (alpha is the same on every lane of a query)
+      const float av = __shfl_sync(0xffffffffu, alpha, 2 * vq);
+      if (__any_sync(0xffffffffu, av != 1.f)) {
 #pragma unroll
-        for (int v = 0; v < QVP; ++v) {
-          const float av = __shfl_sync(0xffffffffu, alpha, 2 * v);
-#pragma unroll
-          for (int k = 0; k < DP; ++k) o[v][k] = mul2(o[v][k], make_float2(av, av));
-        }
+        for (int k = 0; k < DP; ++k) ov[k] = mul2(ov[k], make_float2(av, av));
       }
-      // o[v] += p(position, v) * V[position]; the probabilities leave sc from
-      // the front, two groups per iteration
-#pragma unroll 1
-      for (int s = 0; s < NS; s += 2) {
-        const float pj[2] = {sc[0], sc[1]};
+      // o[vq] += p(position, vq) * V[position]: position 4s + g's probability
+      // for query vq sits on lane (g, 2 vq) in sc[s]
 #pragma unroll
-        for (int r = 0; r + 2 < NS; ++r) sc[r] = sc[r + 2];
+      for (int s2 = 0; s2 < NS; ++s2) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const __nv_bfloat16 *vr = vs + (4 * (s + h) + pg) * HD;
-          float2 v1[CP], v2[CP];
-          lds_bf16x2<C>(vr + d0, v1);
-          lds_bf16x2<C>(vr + d1, v2);
+        for (int g4 = 0; g4 < 4; ++g4) {
+          const float pv = __shfl_sync(0xffffffffu, sc[s2], g4 * 8 + 2 * vq);
+          const __nv_bfloat16 *vr = vs + (4 * s2 + g4) * HD + DL * dc;
+          float2 vv[DP];
+          lds_bf16x2<DL>(vr, vv);
+          const float2 pp = make_float2(pv, pv);
 #pragma unroll
-          for (int v = 0; v < QVP; ++v) {
-            const float pv = __shfl_sync(0xffffffffu, pj[h], pg * 8 + 2 * v);
-            const float2 pp = make_float2(pv, pv);
-#pragma unroll
-            for (int k = 0; k < CP; ++k) {
-              o[v][k] = fma2(pp, v1[k], o[v][k]);
-              o[v][CP + k] = fma2(pp, v2[k], o[v][CP + k]);
-            }
-          }
+          for (int k = 0; k < DP; ++k) ov[k] = fma2(pp, vv[k], ov[k]);
         }
       }
       consume_end(w);
     }
   }
-  // sum o over the four pg lanes, leaving lane (pg, dl) with query pg
-  const bool u16 = (lane & 16) != 0, u8 = (lane & 8) != 0;
-  float *so = sh.o + (w.wib * QVP + pg) * HD;
+  // this warp's share of query vq's output: dims [DL dc, DL dc + DL)
+  float *so = sh.o + (w.wib * QVP + vq) * HD + DL * dc;
 #pragma unroll
-  for (int k = 0; k < DL; ++k) {
-    const int kp = k >> 1;
-    const bool hi = k & 1;
-#define MK_OV(v) (hi ? o[v][kp].y : o[v][kp].x)
-    const float s0 = u16 ? MK_OV(0) : MK_OV(2), s1 = u16 ? MK_OV(1) : MK_OV(3);
-    const float r0 = (u16 ? MK_OV(2) : MK_OV(0)) + __shfl_xor_sync(0xffffffffu, s0, 16);
-    const float r1 = (u16 ? MK_OV(3) : MK_OV(1)) + __shfl_xor_sync(0xffffffffu, s1, 16);
-#undef MK_OV
-    const float r = (u8 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, u8 ? r0 : r1, 8);
-    so[(k < C ? d0 : d1 - C) + k] = r;
+  for (int k = 0; k < DP; ++k) {
+    so[2 * k] = ov[k].x;
+    so[2 * k + 1] = ov[k].y;
   }
   if (pg == 0 && (dl & 1) == 0) {
     sh.ml[(w.wib * QVP + myq) * 2] = m_run;
