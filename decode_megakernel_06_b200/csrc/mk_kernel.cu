@@ -1840,7 +1840,7 @@ MK_INLINE bool attn_warp(Warp &w, int op, int layer, const AttnItem &a, AttnShar
       // scores, two groups of four positions per iteration: lane (pg, dl)
       // gets position pos0 + 4s + pg for query myq; results enter sc at the end
       float sc[NS];
-#pragma unroll 1
+#pragma unroll
       for (int s = 0; s < NS; s += 2) {
         float x[2];
 #pragma unroll
