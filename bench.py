@@ -463,9 +463,29 @@ def measure_sampled(dec, m, k, v, B, ctx, device, steps=20, warmup=3, temperatur
         e1.record(stream)
         torch.cuda.synchronize()
         alone[f"rows{rows}_us"] = round(e0.elapsed_time(e1) / reps * 1e3, 2)
+    # where one row's sampler time goes: the device clock at each phase
+    # boundary of row 0's first CTA (mk_sample_top_p_phases), median of 21 calls
+    lg = make_logits(1, m.vocab, 1.0, 57).to(device)
+    uu = torch.tensor(make_uniforms(1, 58), dtype=torch.float64, device=device)
+    out = torch.empty(1, dtype=torch.int32, device=device)
+    stamps = torch.zeros(mk.MK_SAMPLE_PHASES, dtype=torch.int64, device=device)
+    names = ["load slice, largest key", "barrier 1 (share largest key)", "masses, first histogram",
+             "radix pass 0", "radix pass 1", "radix pass 2", "radix pass 3", "nucleus, segment totals",
+             "barrier 6 (share totals)", "draw", "barrier 7 (exit)"]
+    deltas = []
+    for _ in range(21):
+        assert mk.sample_top_p_phases(lg, temperature, top_p, uu, out, stamps) == 0
+        torch.cuda.synchronize()
+        t = stamps.cpu().tolist()
+        deltas.append([(t[i + 1] - t[i]) / 1e3 for i in range(len(names))])
+    med = [sorted(col)[len(col) // 2] for col in zip(*deltas)]
+    phases = {nm: round(v, 2) for nm, v in zip(names, med)}
+    phases["total (first stamp to last)"] = round(sum(med), 2)
+    phases["how"] = ("%globaltimer at each phase boundary of row 0's first CTA, median of 21 calls; the "
+                     "device clock advances in steps of a few hundred ns")
     return {"batch": B, "temperature": temperature, "top_p": top_p, "ms_per_step": round(ms, 4),
             "tok_s": round(B / (ms / 1e3), 1), "launches_per_step": 2,
-            "sampler_alone": alone, "vocab": m.vocab,
+            "sampler_alone": alone, "sampler_phases_rows1_us": phases, "vocab": m.vocab,
             "path": "mk_decode_step_sample: the megakernel step, then the cluster top-p sampler on its logits"}
 
 

@@ -35,6 +35,7 @@ VARIANTS = {"megakernel": MK_MEGAKERNEL, "multikernel": MK_MULTIKERNEL,
 MK_FAULT_NONE = 0
 MK_FAULT_UNREACHABLE_WAIT = 1
 MK_TRACE_WORDS = 12  # uint64 words per (op, warp) record of mk_set_trace
+MK_SAMPLE_PHASES = 12  # phase stamps of mk_sample_top_p_phases
 MK_STATIC_SCRATCH_BYTES = 32 << 20  # the fixed working array of mk_decode_step_static
 
 OP_NAMES = ["EMBED", "QKV", "ATTN", "OPROJ", "SHARED_GU", "ROUTED_GU", "DOWN", "COMBINE", "LMHEAD"]
@@ -102,6 +103,7 @@ def lib():
         "mk_decode_step_host": (i32, [vp, _I32P, _I32P, i32, i32, mk_kv_cache, vp, _I32P, vp]),
         "mk_decode_step_static": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, vp, vp]),
         "mk_sample_top_p": (i32, [vp, i32, i32, ctypes.c_float, ctypes.c_float, vp, vp, vp]),
+        "mk_sample_top_p_phases": (i32, [vp, i32, i32, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]),
         "mk_decode_step_sample": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, ctypes.c_float,
                                         ctypes.c_float, vp, vp, vp]),
         "mk_get_device_status": (i32, [vp, vp]),
@@ -196,6 +198,12 @@ def mk_sample_top_p(logits: int, rows: int, vocab: int, temperature: float, top_
     return lib().mk_sample_top_p(logits, rows, vocab, temperature, top_p, uniforms, out_tokens, stream)
 
 
+def mk_sample_top_p_phases(logits: int, rows: int, vocab: int, temperature: float, top_p: float,
+                           uniforms: int, out_tokens: int, stamps: int, stream: int = 0) -> int:
+    return lib().mk_sample_top_p_phases(logits, rows, vocab, temperature, top_p, uniforms, out_tokens, stamps,
+                                        stream)
+
+
 def mk_decode_step_sample(h, tokens: int, positions: int, B: int, T: int, kv: mk_kv_cache,
                           out_logits: int, temperature: float, top_p: float, uniforms: int,
                           out_tokens: int, stream: int) -> int:
@@ -235,6 +243,24 @@ def sample_top_p(logits, temperature: float, top_p: float, uniforms, out_tokens,
     s = stream if stream is not None else torch.cuda.current_stream()
     return mk_sample_top_p(logits.data_ptr(), rows, vocab, temperature, top_p, _ptr(uniforms),
                            out_tokens.data_ptr(), s.cuda_stream)
+
+
+def sample_top_p_phases(logits, temperature: float, top_p: float, uniforms, out_tokens, stamps, stream=None) -> int:
+    """sample_top_p, also writing the device clock (ns) at each of the
+    MK_SAMPLE_PHASES phase boundaries of row 0 into ``stamps`` (int64 CUDA
+    tensor of at least MK_SAMPLE_PHASES elements; see mk_sample_top_p_phases).
+    The same checks as sample_top_p; returns the launch status code."""
+    import torch
+
+    _need(logits, torch.float32, 1, "logits", dims=2)
+    rows, vocab = logits.shape
+    if uniforms is not None:
+        _need(uniforms, torch.float64, rows, "uniforms", logits.device)
+    _need(out_tokens, torch.int32, rows, "out_tokens", logits.device)
+    _need(stamps, torch.int64, MK_SAMPLE_PHASES, "stamps", logits.device)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return mk_sample_top_p_phases(logits.data_ptr(), rows, vocab, temperature, top_p, _ptr(uniforms),
+                                  out_tokens.data_ptr(), stamps.data_ptr(), s.cuda_stream)
 
 
 def hbm_read_probe(buf, form: int = 0, reps: int = 5, stream=None) -> float:

@@ -845,6 +845,18 @@ MK_API int mk_sample_top_p(const float *logits, int32_t rows, int32_t vocab, flo
   return MK_OK;
 }
 
+MK_API int mk_sample_top_p_phases(const float *logits, int32_t rows, int32_t vocab, float temperature,
+                                  float top_p, const double *uniforms, int32_t *out_tokens,
+                                  unsigned long long *stamps, void *stream) {
+  static_assert(MK_SAMPLE_PHASES == kSamplePhases, "phase count of the header and the kernel");
+  if (!stamps) return fail(MK_ERR_ARG, "stamps is NULL");
+  int rc = check_sample_args(logits, rows, vocab, temperature, top_p, uniforms, out_tokens);
+  if (rc) return rc;
+  CUDA_TRY(launch_top_p(logits, rows, vocab, temperature, top_p, uniforms, out_tokens,
+                        static_cast<cudaStream_t>(stream), stamps));
+  return MK_OK;
+}
+
 MK_API int mk_decode_step_sample(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
                                  int32_t T, mk_kv_cache kv, float *out_logits, float temperature, float top_p,
                                  const double *uniforms, int32_t *out_tokens, void *stream) {

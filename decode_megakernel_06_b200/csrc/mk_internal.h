@@ -229,8 +229,10 @@ constexpr int kSampleCluster = 8;
 constexpr int kSampleThreads = 512;
 constexpr int kSampleMaxVocab = 131072;  // 64-bit mass sums and shared memory both cover this
 size_t sample_smem_bytes(int slice);
+constexpr int kSamplePhases = 12;  // phase stamps of a traced sampler launch
 cudaError_t launch_top_p(const float *logits, int rows, int vocab, float temperature, float top_p,
-                         const double *uniforms, int32_t *out, cudaStream_t stream);
+                         const double *uniforms, int32_t *out, cudaStream_t stream,
+                         unsigned long long *stamps = nullptr);
 
 // Read-only HBM probe (mk_probe.cu).  form 0: 16-byte vector loads; form 1:
 // bulk asynchronous copies into shared memory.  sink: probe_sink_words(n_sm)

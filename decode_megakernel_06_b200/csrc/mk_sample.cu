@@ -113,9 +113,20 @@ struct SampleShared {
   uint64_t need;
 };
 
+// Phase clock (stamps != nullptr): thread 0 of the first CTA of row 0 records
+// %globaltimer at each phase boundary, stamps[0 .. kSamplePhases).
+__device__ __forceinline__ void phase_stamp(unsigned long long *stamps, int i, bool me) {
+  if (stamps && me) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    stamps[i] = t;
+  }
+}
+
 __global__ void __launch_bounds__(kSThreads, 1)
 top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_t, float top_p,
-             int greedy, int vec4, const double *__restrict__ uniforms, int32_t *__restrict__ out) {
+             int greedy, int vec4, const double *__restrict__ uniforms, int32_t *__restrict__ out,
+             unsigned long long *stamps) {
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) unsigned char dyn[];
   __shared__ SampleShared sh;
@@ -128,6 +139,8 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
   float *l = reinterpret_cast<float *>(dyn + sizeof(uint64_t) * (size_t)slice);
   uint64_t *whist = reinterpret_cast<uint64_t *>(dyn + 12 * (size_t)((slice + 1) & ~1));
   const float *src = logits + (size_t)row * vocab + lo;
+  const bool stamper = row == 0 && rank == 0 && tid == 0;
+  phase_stamp(stamps, 0, stamper);
 
   for (int i = tid; i < kHistCopies * 256; i += kSThreads) whist[i] = 0;
   // ---- load the slice; this CTA's largest key --------------------------------
@@ -157,7 +170,9 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
     for (int w = 0; w < kSWarps; ++w) k = max(k, sh.wkey[w]);
     sh.cta_key = k;
   }
+  phase_stamp(stamps, 1, stamper);
   cluster.sync();  // 1: every CTA's largest key is visible
+  phase_stamp(stamps, 2, stamper);
   if (tid == 0) {
     uint32_t k = 0;
     for (unsigned r = 0; r < kSampleCluster; ++r) k = max(k, cluster.map_shared_rank(&sh.cta_key, r)[0]);
@@ -209,6 +224,7 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
     sh.prefix = 0;
     sh.above = 0;
   }
+  phase_stamp(stamps, 3, stamper);
 
   // ---- radix select of the threshold key, one byte per pass -----------------------
   for (int d = 0; d < 4; ++d) {
@@ -287,6 +303,7 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
         hist_add(myhist, (k >> (shift - 8)) & 255u, qi, i < n && qi != 0 && (k >> shift) == pre, stage, lane);
       }
     }
+    phase_stamp(stamps, 4 + d, stamper);
   }
 
   // ---- the nucleus: keys above tau, and the first r tokens at tau by id -----------
@@ -327,7 +344,9 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
     sh.seg[0] = a;
     sh.seg[1] = e;
   }
+  phase_stamp(stamps, 8, stamper);
   cluster.sync();  // 6: every CTA's segment totals are visible
+  phase_stamp(stamps, 9, stamper);
   // mass above tau and tokens at tau before this warp's segment, over the row
   uint64_t gb = 0, eb = 0;
   for (unsigned rr = 0; rr < rank; ++rr) {
@@ -365,7 +384,9 @@ top_p_kernel(const float *__restrict__ logits, int vocab, int slice, double inv_
       ties += __popc(tb);
     }
   }
+  phase_stamp(stamps, 10, stamper);
   cluster.sync();  // 7: no CTA leaves while its shared memory is being read
+  phase_stamp(stamps, 11, stamper);
 }
 
 }  // namespace
@@ -375,7 +396,7 @@ size_t sample_smem_bytes(int slice) {
 }
 
 cudaError_t launch_top_p(const float *logits, int rows, int vocab, float temperature, float top_p,
-                         const double *uniforms, int32_t *out, cudaStream_t stream) {
+                         const double *uniforms, int32_t *out, cudaStream_t stream, unsigned long long *stamps) {
   const int slice = (vocab + kSampleCluster - 1) / kSampleCluster;
   const size_t smem = sample_smem_bytes(slice);
   // the largest dynamic size set so far, per device: the attribute is set only
@@ -409,7 +430,8 @@ cudaError_t launch_top_p(const float *logits, int rows, int vocab, float tempera
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int vec4 = (vocab % 4 == 0) && (slice % 4 == 0) && ((reinterpret_cast<uintptr_t>(logits) & 15) == 0);
-  return cudaLaunchKernelEx(&cfg, top_p_kernel, logits, vocab, slice, inv_t, top_p, greedy, vec4, uniforms, out);
+  return cudaLaunchKernelEx(&cfg, top_p_kernel, logits, vocab, slice, inv_t, top_p, greedy, vec4, uniforms, out,
+                            stamps);
 }
 
 }  // namespace mk

@@ -256,6 +256,22 @@ MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *p
 MK_API int mk_sample_top_p(const float *logits, int32_t rows, int32_t vocab, float temperature,
                            float top_p, const double *uniforms, int32_t *out_tokens, void *stream);
 
+/* mk_sample_top_p, and the device clock (%globaltimer, ns) at each phase
+ * boundary of row 0's first CTA written to stamps[0 .. MK_SAMPLE_PHASES):
+ *   0 start, 1 slice loaded and its largest key found, 2 after the cluster
+ *   barrier that shares the largest key, 3 masses and first histogram done,
+ *   4..7 end of radix pass 0..3 (histogram of the next key byte included),
+ *   8 the nucleus and this CTA's segment totals done, 9 after the barrier that
+ *   shares them, 10 the draw done, 11 after the closing barrier.
+ * stamps: device uint64 [MK_SAMPLE_PHASES], caller-owned; a greedy call
+ * (temperature <= 0) writes entries 0..2 only.  A measurement aid: the
+ * sample drawn is the same as mk_sample_top_p's.  Errors as mk_sample_top_p,
+ * and MK_ERR_ARG for a NULL stamps. */
+#define MK_SAMPLE_PHASES 12
+MK_API int mk_sample_top_p_phases(const float *logits, int32_t rows, int32_t vocab, float temperature,
+                                  float top_p, const double *uniforms, int32_t *out_tokens,
+                                  unsigned long long *stamps, void *stream);
+
 /* mk_decode_step followed by mk_sample_top_p on its logits: one decode step of
  * B*T rows whose next tokens are sampled instead of taken greedily.  Arguments
  * as mk_decode_step (out_logits may be NULL: the handle's scratch holds them)

@@ -188,6 +188,12 @@ def test_sampler_checks_its_arguments_on_the_host(L):
     assert L.mk_sample_top_p(lg, 1, 10, 0.7, 0.9, None, out, None) == mk.MK_ERR_ARG
     assert L.mk_sample_top_p(lg, 1, 131073, 1.0, 0.9, u, out, None) == mk.MK_ERR_UNSUPPORTED
     assert "131072" in mk.mk_last_error()
+    st = 1024  # the phase-stamped form: the same checks, and its stamps
+    assert L.mk_sample_top_p_phases(lg, 1, 10, 1.0, 0.9, u, out, None, None) == mk.MK_ERR_ARG
+    assert "stamps" in mk.mk_last_error()
+    assert L.mk_sample_top_p_phases(None, 1, 10, 1.0, 0.9, u, out, st, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p_phases(lg, 1, 10, 0.7, 0.9, None, out, st, None) == mk.MK_ERR_ARG
+    assert L.mk_sample_top_p_phases(lg, 1, 131073, 1.0, 0.9, u, out, st, None) == mk.MK_ERR_UNSUPPORTED
     kv = mk.mk_kv_cache(None, None)
     assert L.mk_decode_step_sample(None, None, None, 1, 1, kv, None, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
 
@@ -209,6 +215,13 @@ def test_torch_wrappers_check_tensors_before_any_launch():
         mk.sample_top_p(lg.t(), 1.0, 0.9, u, out)
     with pytest.raises(ValueError, match="CUDA|cuda"):
         mk.sample_top_p(lg, 1.0, 0.9, u, out)  # CPU tensors never reach the library
+    stamps = torch.zeros(mk.MK_SAMPLE_PHASES, dtype=torch.int64)
+    with pytest.raises(ValueError, match="CUDA|cuda"):
+        mk.sample_top_p_phases(lg, 1.0, 0.9, u, out, stamps)
+    with pytest.raises(ValueError, match="dtype"):
+        mk._need(stamps.int(), torch.int64, mk.MK_SAMPLE_PHASES, "stamps")
+    with pytest.raises(ValueError, match="at least"):
+        mk._need(stamps[:5], torch.int64, mk.MK_SAMPLE_PHASES, "stamps")
     with pytest.raises(ValueError, match="dtype"):
         mk._need(u.float(), torch.float64, 4, "uniforms")
     with pytest.raises(ValueError, match="at least 4"):

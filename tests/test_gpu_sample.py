@@ -118,6 +118,26 @@ def test_repeatable():
     assert np.array_equal(a, b)
 
 
+def test_phase_stamped_sampler_draws_the_same_tokens():
+    """mk_sample_top_p_phases is the same launch with the device clock written
+    at its 12 phase boundaries: it draws the same tokens as mk_sample_top_p,
+    and its stamps are in order."""
+    dev = torch.device("cuda:0")
+    logits = make_logits(8, 64000, 1.0, seed=40).numpy()
+    u = make_uniforms(8, seed=41)
+    ref = _gpu_sample(logits, 0.8, 0.9, u)
+    lg = torch.from_numpy(np.ascontiguousarray(logits, np.float32)).to(dev)
+    uu = torch.tensor(np.asarray(u, np.float64), device=dev)
+    out = torch.full((8,), -7, dtype=torch.int32, device=dev)
+    stamps = torch.zeros(mk.MK_SAMPLE_PHASES, dtype=torch.int64, device=dev)
+    assert mk.sample_top_p_phases(lg, 0.8, 0.9, uu, out, stamps) == mk.MK_OK, mk.mk_last_error()
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), ref)
+    t = stamps.cpu().tolist()
+    assert t[0] > 0 and all(b >= a for a, b in zip(t, t[1:])), t
+    assert t[-1] - t[0] < 10_000_000, t  # well under 10 ms for one 64000-wide row
+
+
 def test_rejects_bad_arguments():
     dev = torch.device("cuda:0")
     lg = torch.zeros((2, 10), dtype=torch.float32, device=dev)
