@@ -264,7 +264,7 @@ struct mk_handle {
   cudaStream_t capture_stream;
   // wide blocks (more than kMaxRows rows): scratch of the launch sequence
   int wide_ldx, wide_lda;
-  float *w_h, *w_qkv, *w_o, *w_rlog, *w_selw, *w_gu, *w_yd, *w_gs, *w_ys, *w_part, *w_attn_o, *w_attn_ml;
+  float *w_h, *w_qkv, *w_rlog, *w_selw, *w_gu, *w_yd, *w_gs, *w_ys, *w_part, *w_attn_o, *w_attn_ml;
   long long w_part_floats;
   int32_t *w_sele, *w_tok, *w_pos;
   int *w_count, *w_off, *w_pair_row, *w_pair_slot;
@@ -480,9 +480,8 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     h->wide_lda = lda;
     HALLOC(h->w_h, sizeof(float) * (size_t)MR * D);
     HALLOC(h->w_qkv, sizeof(float) * (size_t)MR * QKVW);
-    HALLOC(h->w_o, sizeof(float) * (size_t)MR * HD);
-    {  // attention partials: per query vector (row x head) and 64-position chunk of the cache
-      const size_t slots = (size_t)MR * d.n_q_heads * ceil_div(d.kv_capacity, 64);
+    {  // attention partials: per query vector (row x head) and 128-position chunk of the cache
+      const size_t slots = (size_t)MR * d.n_q_heads * ceil_div(d.kv_capacity, 128);
       HALLOC(h->w_attn_o, sizeof(float) * slots * d.head_dim);
       HALLOC(h->w_attn_ml, sizeof(float) * slots * 2);
     }
@@ -700,7 +699,7 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
   s.dbg_hidden = h->dbg_hidden; s.dbg_ids = h->dbg_ids; s.dbg_w = h->dbg_w;
   s.ldx = h->wide_ldx; s.lda = h->wide_lda;
   s.attn_o = h->w_attn_o; s.attn_ml = h->w_attn_ml;
-  s.h = h->w_h; s.qkv = h->w_qkv; s.o = h->w_o; s.rlog = h->w_rlog; s.sel_w = h->w_selw; s.gu = h->w_gu;
+  s.h = h->w_h; s.qkv = h->w_qkv; s.rlog = h->w_rlog; s.sel_w = h->w_selw; s.gu = h->w_gu;
   s.yd = h->w_yd; s.gs = h->w_gs; s.ys = h->w_ys; s.part = h->w_part; s.part_floats = h->w_part_floats;
   s.sel_e = h->w_sele; s.count = h->w_count; s.off = h->w_off; s.pair_row = h->w_pair_row;
   s.pair_slot = h->w_pair_slot;

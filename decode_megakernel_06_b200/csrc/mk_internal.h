@@ -206,8 +206,8 @@ struct WideStep {
   float *dbg_w;
   // scratch
   int ldx, lda;
-  float *h, *qkv, *o, *rlog, *sel_w, *gu, *yd, *gs, *ys, *part;
-  float *attn_o, *attn_ml;  // attention partials: [rows * Hq * ceil(cap / 64)] x hd and x 2
+  float *h, *qkv, *rlog, *sel_w, *gu, *yd, *gs, *ys, *part;
+  float *attn_o, *attn_ml;  // attention partials: [rows * Hq * ceil(cap / 128)] x hd and x 2
   long long part_floats;
   int32_t *sel_e;
   int *count, *off, *pair_row, *pair_slot;

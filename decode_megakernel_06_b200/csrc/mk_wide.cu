@@ -6,8 +6,8 @@
 // accumulate).  Activations enter the tensor cores as a bf16 pair
 // (x = hi + lo, hi = bf16(x), lo = bf16(x - hi)), so each product keeps close
 // to fp32 accuracy; weights are bf16 already.  The remaining steps (norms,
-// rotary + cache append, attention, top-k, expert lists, SwiGLU, combine,
-// argmax) are plain CUDA-core kernels.
+// rotary + cache append, attention merge, top-k, expert lists, SwiGLU,
+// combine, argmax) are plain CUDA-core kernels.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -284,14 +284,6 @@ __global__ void wide_norm_split(const float *h, const __nv_bfloat16 *g, int d, f
   }
 }
 
-// plain split of rows [M][K] (stride lds) into the bf16 pair
-__global__ void wide_split(const float *src, int K, int lds, __nv_bfloat16 *xhi, __nv_bfloat16 *xlo, int ldx) {
-  const int m = blockIdx.x;
-  for (int c = threadIdx.x; c < K; c += blockDim.x)
-    split_store(src[static_cast<long long>(m) * lds + c], xhi + static_cast<long long>(m) * ldx + c,
-                xlo + static_cast<long long>(m) * ldx + c);
-}
-
 // Rotary embedding of k at each new row's position, k and v rounded to bf16
 // and written into the cache.  grid = (M, Hkv).
 __global__ void wide_kv_append(const float *qkv, int W3, const int32_t *positions, int T, int Hq, int Hkv, int hd,
@@ -311,136 +303,312 @@ __global__ void wide_kv_append(const float *qkv, int W3, const int32_t *position
   }
 }
 
-// Attention of a wide block, split over the KV positions: one block per
-// (sequence, KV head, chunk of kWaChunk positions) stages the chunk's K and V
-// rows in shared memory once and scores every query vector of the group
-// against them (T rows x Hq/Hkv heads, each seeing positions up to its own),
-// writing per query an unnormalised partial output with its running max and
-// sum; wide_attn_merge combines a query's chunks with the log-sum-exp rule.
-// Lane j of a warp scores positions j and j + 32 of the chunk (rows padded
-// by 8 bf16 so that the lanes' row reads fall in different banks); for P.V
-// lane l owns dims [DPL l, DPL l + DPL).
-constexpr int kWaChunk = 64;
-constexpr int kWaWarps = 8;
-constexpr int kWaPad = 8;
-template <int DPL>
-__global__ void __launch_bounds__(kWaWarps * 32) wide_attn_chunk(
-    const float *qkv, int W3, const int32_t *positions, int T, int Hq, int Hkv, const float2 *rope,
-    const __nv_bfloat16 *kc, const __nv_bfloat16 *vc, int Bmax, int cap, int layer, int nch_max, float *opart,
-    float *mlpart) {
-  constexpr int HD = 32 * DPL, HALF = HD / 2, LD = HD + kWaPad;
-  __shared__ __align__(16) __nv_bfloat16 sk[kWaChunk * LD], sv[kWaChunk * LD];
-  __shared__ __align__(16) float sq[kWaWarps][HD];
-  const int c = blockIdx.x, bg = blockIdx.y, b = bg / Hkv, g = bg % Hkv, G = Hq / Hkv;
-  const int pos0 = positions[b], last = pos0 + T - 1;  // the block's last query sees up to `last`
-  const int j0 = c * kWaChunk;
-  if (j0 > last) return;
-  const int nj = min(kWaChunk, last + 1 - j0);
-  const long long base = ((static_cast<long long>(layer) * Bmax + b) * Hkv + g) * cap;
-  // stage the chunk's rows: 16-byte pieces, HD / 8 per row
-  for (int i = threadIdx.x; i < nj * (HD / 8); i += blockDim.x) {
-    const int j = i / (HD / 8), piece = i % (HD / 8);
-    const uint4 kv4 = *reinterpret_cast<const uint4 *>(kc + (base + j0 + j) * HD + piece * 8);
-    const uint4 vv4 = *reinterpret_cast<const uint4 *>(vc + (base + j0 + j) * HD + piece * 8);
-    *reinterpret_cast<uint4 *>(sk + j * LD + piece * 8) = kv4;
-    *reinterpret_cast<uint4 *>(sv + j * LD + piece * 8) = vv4;
-  }
-  __syncthreads();
+// Attention of a wide block on the tensor cores, split over the KV positions.
+// One CTA per (chunk of kAcN cache positions, sequence x KV head, tile of up
+// to 128 query vectors) scores the group's query vectors (T rows x Hq/Hkv
+// heads, each seeing positions up to its own) against the chunk:
+//  - one thread brings the chunk's K rows by TMA (128B-swizzled, K-major: the
+//    B operand of S = Q K^T); every thread loads its share of the V rows into
+//    registers;
+//  - the rotated, scaled query vectors go into shared memory as a bf16 pair
+//    (q = hi + lo) in the same swizzled layout, the A operand (M = 128): query
+//    i of the tile in row 32 (i mod 4) + i / 4, so that each warp owns some;
+//  - S (128 x kAcN, fp32) accumulates Q_hi K^T + Q_lo K^T in tensor memory;
+//  - once S is complete, V is written transposed over the K rows (V^T is the
+//    K-major B operand of O = P V), and the thread owning a query's row of S
+//    masks the positions past the query's own and writes p = exp(s - max) as a
+//    bf16 pair over the query rows (the A operand of O = P V);
+//  - O (128 x hd) accumulates P_hi V + P_lo V; each thread writes its query's
+//    unnormalised partial output with the chunk's max and sum of p.
+// wide_attn_merge combines a query's chunks with the log-sum-exp rule.
+// ---------------------------------------------------------------------------
+constexpr int kAcN = 128;              // cache positions per chunk (N of S, K of P V)
+constexpr int kAcThreads = 128;
+constexpr int kAcTmemCols = 256;       // S: kAcN columns, then O: hd columns
+constexpr int kAcAtom = 128 * 128;     // one swizzled operand block: 128 rows x 128 bytes
+
+struct AttnArgs {
+  CUtensorMap mk;  // K cache as [L * Bmax * Hkv * cap][hd], box 64 x 128
+  const float *qkv;
+  int W3;
+  const int32_t *positions;
+  int T, Hq, Hkv;
+  const float2 *rope;
+  const __nv_bfloat16 *vc;
+  int Bmax, cap, layer, nch_max;
+  float *opart, *mlpart;  // [slot][hd], [slot][2]; slot = (bg * nch_max + chunk) * T * G + query
+  int *error;
+};
+
+// dynamic shared memory: Q (later P) in 4 blocks, K (later V^T) in hd / 64
+// blocks, + room to align them to 1024 bytes
+constexpr int attn_smem_bytes(int hd) { return (4 + hd / 64) * kAcAtom + 1024; }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);  // .x at the lower address
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// byte offset of the 16-byte piece `piece` (0..7) of row r in a swizzled block
+__device__ __forceinline__ int sw_off(int r, int piece) { return r * 128 + ((piece ^ (r & 7)) << 4); }
+
+template <int HD>
+__global__ void __launch_bounds__(kAcThreads, 2) wide_attn_tc(const __grid_constant__ AttnArgs a) {
+  constexpr int NA = HD / 64, HALF = HD / 2;
+  constexpr int NU = 64 * (HD / 8) / kAcThreads;  // (position pair, 8 dims) units of V per thread
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (sptr(smem_raw) & 1023u)) & 1023u);
+  uint8_t *sQ = smem;                // Q hi: NA blocks, Q lo: NA blocks; then P hi: 2 blocks, P lo: 2 blocks
+  uint8_t *sK = smem + 4 * kAcAtom;  // K: NA blocks of 128 positions; then V^T: 2 blocks of HD rows
+  __shared__ __align__(8) uint64_t kbar, sbar, obar;
+  __shared__ uint32_t tmem_base;
+  const int c = blockIdx.x, bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv, G = a.Hq / a.Hkv;
+  const int Q = a.T * G, q0 = blockIdx.z * 128, nq = min(128, Q - q0);
+  const int pos0 = a.positions[b], last = pos0 + a.T - 1;
+  const int j0 = c * kAcN;
+  if (j0 > last || nq <= 0) return;  // the whole CTA, before anything is allocated
+  const int nj = min(kAcN, last + 1 - j0);
+  const long long krow0 = ((static_cast<long long>(a.layer) * a.Bmax + b) * a.Hkv + g) * a.cap;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float scale = 1.0f / sqrtf(static_cast<float>(HD));
-  const int Q = T * G;
-  for (int qi = warp; qi < Q; qi += kWaWarps) {
-    const int t = qi / G, h = g * G + qi % G, m = b * T + t, lim = pos0 + t;
-    // the query vector, rotated (rotate-half pairs) and scaled, in this warp's buffer
-    const float *q = qkv + static_cast<long long>(m) * W3 + h * HD;
-    for (int i = lane; i < HALF; i += 32) {
-      const float2 cs = rope[static_cast<long long>(lim) * HALF + i];
-      const float x1 = q[i], x2 = q[i + HALF];
-      sq[warp][i] = (x1 * cs.x - x2 * cs.y) * scale;
-      sq[warp][i + HALF] = (x2 * cs.x + x1 * cs.y) * scale;
-    }
-    __syncwarp();
-    float s[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int j = lane + 32 * u;
-      float acc = 0.f;
-      if (j < nj && j0 + j <= lim) {
-        const __nv_bfloat16 *kr = sk + j * LD;
-#pragma unroll 8
-        for (int d = 0; d < HD; d += 8) {
-          const uint4 kk = *reinterpret_cast<const uint4 *>(kr + d);
-          const float4 qa = *reinterpret_cast<const float4 *>(&sq[warp][d]);
-          const float4 qb = *reinterpret_cast<const float4 *>(&sq[warp][d + 4]);
-          acc = fmaf(qa.x, __uint_as_float(kk.x << 16), acc);
-          acc = fmaf(qa.y, __uint_as_float(kk.x & 0xffff0000u), acc);
-          acc = fmaf(qa.z, __uint_as_float(kk.y << 16), acc);
-          acc = fmaf(qa.w, __uint_as_float(kk.y & 0xffff0000u), acc);
-          acc = fmaf(qb.x, __uint_as_float(kk.z << 16), acc);
-          acc = fmaf(qb.y, __uint_as_float(kk.z & 0xffff0000u), acc);
-          acc = fmaf(qb.z, __uint_as_float(kk.w << 16), acc);
-          acc = fmaf(qb.w, __uint_as_float(kk.w & 0xffff0000u), acc);
-        }
-        s[u] = acc;
-      } else {
-        s[u] = -INFINITY;
-      }
-    }
-    float mx = fmaxf(s[0], s[1]);
-    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float p[2], l = 0.f;
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      p[u] = (s[u] == -INFINITY) ? 0.f : expf(s[u] - mx);
-      l += p[u];
-    }
-    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    float acc[DPL];
-#pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) acc[dd] = 0.f;
-    if (mx != -INFINITY) {
-      for (int j = 0; j < nj; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, p[j >> 5], j & 31);
-        const __nv_bfloat16 *vr = sv + j * LD + lane * DPL;
-#pragma unroll
-        for (int dd = 0; dd < DPL; ++dd) acc[dd] = fmaf(pj, __bfloat162float(vr[dd]), acc[dd]);
-      }
-    }
-    const long long slot = (static_cast<long long>(bg) * nch_max + c) * (static_cast<long long>(T) * G) + qi;
-    float *dst = opart + slot * HD + lane * DPL;
-#pragma unroll
-    for (int dd = 0; dd < DPL; ++dd) dst[dd] = acc[dd];
-    if (lane == 0) {
-      mlpart[2 * slot] = mx;
-      mlpart[2 * slot + 1] = l;
-    }
-    __syncwarp();  // the buffer of q is rewritten by the warp's next query
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sptr(&tmem_base)),
+                 "r"(kAcTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  if (threadIdx.x == 32) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&kbar)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&sbar)) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&obar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = tmem_base;
+  if (threadIdx.x == 0) {  // K rows of the chunk (rows past the cache tensor read as zeros)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&kbar)), "r"(NA * kAcAtom)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < NA; ++i) tc_tma(sK + i * kAcAtom, &a.mk, 64 * i, static_cast<int>(krow0 + j0), &kbar);
+  }
+  // this thread's V units: positions 2 pp and 2 pp + 1, dims [8 dc, 8 dc + 8)
+  uint4 va[NU], vb[NU];
+  {
+    const __nv_bfloat16 *vbase = a.vc + (krow0 + j0) * HD;
+#pragma unroll
+    for (int i = 0; i < NU; ++i) {
+      const int u = threadIdx.x + kAcThreads * i, pp = u & 63, dc = u >> 6;
+      va[i] = 2 * pp < nj ? *reinterpret_cast<const uint4 *>(vbase + (2 * pp) * HD + 8 * dc) : make_uint4(0, 0, 0, 0);
+      vb[i] = 2 * pp + 1 < nj ? *reinterpret_cast<const uint4 *>(vbase + (2 * pp + 1) * HD + 8 * dc)
+                              : make_uint4(0, 0, 0, 0);
+    }
+  }
+  // the query vectors: rotate-half pairs at the query's position, scaled, as a bf16 pair
+  {
+    const float scale = 1.0f / sqrtf(static_cast<float>(HD));
+    for (int it = threadIdx.x; it < nq * (HALF / 8); it += kAcThreads) {
+      const int ql = it / (HALF / 8), cc = it % (HALF / 8), qi = q0 + ql;
+      const int t = qi / G, h = g * G + qi % G, m = b * a.T + t, lim = pos0 + t;
+      const float *q = a.qkv + static_cast<long long>(m) * a.W3 + h * HD + 8 * cc;
+      const float4 *cs4 = reinterpret_cast<const float4 *>(a.rope + static_cast<long long>(lim) * HALF + 8 * cc);
+      float x1[8], x2[8], cs[16];
+      *reinterpret_cast<float4 *>(&x1[0]) = *reinterpret_cast<const float4 *>(q);
+      *reinterpret_cast<float4 *>(&x1[4]) = *reinterpret_cast<const float4 *>(q + 4);
+      *reinterpret_cast<float4 *>(&x2[0]) = *reinterpret_cast<const float4 *>(q + HALF);
+      *reinterpret_cast<float4 *>(&x2[4]) = *reinterpret_cast<const float4 *>(q + HALF + 4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) *reinterpret_cast<float4 *>(&cs[4 * i]) = cs4[i];
+      uint32_t y1h[4], y1l[4], y2h[4], y2l[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        float y1[2], y2[2], r1[2], r2[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const float co = cs[2 * (e + k)], si = cs[2 * (e + k) + 1];
+          y1[k] = (x1[e + k] * co - x2[e + k] * si) * scale;
+          y2[k] = (x2[e + k] * co + x1[e + k] * si) * scale;
+          r1[k] = y1[k] - __bfloat162float(__float2bfloat16_rn(y1[k]));
+          r2[k] = y2[k] - __bfloat162float(__float2bfloat16_rn(y2[k]));
+        }
+        y1h[e / 2] = pack_bf16(y1[0], y1[1]);
+        y1l[e / 2] = pack_bf16(r1[0], r1[1]);
+        y2h[e / 2] = pack_bf16(y2[0], y2[1]);
+        y2l[e / 2] = pack_bf16(r2[0], r2[1]);
+      }
+      const int r = 32 * (ql & 3) + (ql >> 2);
+      const int d1 = 8 * cc, d2 = HALF + 8 * cc;
+      const int o1 = (d1 >> 6) * kAcAtom + sw_off(r, (d1 & 63) >> 3), o2 = (d2 >> 6) * kAcAtom + sw_off(r, (d2 & 63) >> 3);
+      *reinterpret_cast<uint4 *>(sQ + o1) = make_uint4(y1h[0], y1h[1], y1h[2], y1h[3]);
+      *reinterpret_cast<uint4 *>(sQ + NA * kAcAtom + o1) = make_uint4(y1l[0], y1l[1], y1l[2], y1l[3]);
+      *reinterpret_cast<uint4 *>(sQ + o2) = make_uint4(y2h[0], y2h[1], y2h[2], y2h[3]);
+      *reinterpret_cast<uint4 *>(sQ + NA * kAcAtom + o2) = make_uint4(y2l[0], y2l[1], y2l[2], y2l[3]);
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+  // kind::f16 instruction descriptors: fp32 accumulator, bf16 A and B, both K-major, M = 128
+  constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kAcN >> 3) << 17) | ((128 >> 4) << 24);
+  constexpr uint32_t kIdescO = (1u << 4) | (1u << 7) | (1u << 10) | ((HD >> 3) << 17) | ((128 >> 4) << 24);
+  if (threadIdx.x == 0) {
+    if (tc_wait(&kbar, 0, a.error)) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+      for (int i = 0; i < NA; ++i) {
+        const uint64_t dqh = tc_desc(sQ + i * kAcAtom), dql = tc_desc(sQ + (NA + i) * kAcAtom),
+                       dk = tc_desc(sK + i * kAcAtom);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 dims = 32 bytes = 2 descriptor units
+          tc_mma(tmem, dqh + 2 * kk, dk + 2 * kk, kIdescS, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem, dql + 2 * kk, dk + 2 * kk, kIdescS, 1u);
+        }
+      }
+    }
+    tc_commit(&sbar);
+  }
+  __syncwarp();
+  bool ok = tc_wait(&sbar, 0, a.error);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  // V^T over the K rows: row d, positions 2 pp and 2 pp + 1 in one 32-bit word
+#pragma unroll
+  for (int i = 0; i < NU; ++i) {
+    const int u = threadIdx.x + kAcThreads * i, pp = u & 63, dc = u >> 6;
+    const uint32_t wa[4] = {va[i].x, va[i].y, va[i].z, va[i].w}, wb[4] = {vb[i].x, vb[i].y, vb[i].z, vb[i].w};
+    uint8_t *blk = sK + (pp >> 5) * (HD * 128) + (pp & 3) * 4;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int d = 8 * dc + e;
+      const uint32_t word = __byte_perm(wa[e >> 1], wb[e >> 1], (e & 1) ? 0x7632 : 0x5410);
+      *reinterpret_cast<uint32_t *>(blk + sw_off(d, (pp & 31) >> 2)) = word;
+    }
+  }
+  // this thread's query row of S: mask, max, p = exp(s - max) as a bf16 pair
+  const int r = threadIdx.x, ql = 4 * lane + warp, qi = q0 + ql;
+  const bool valid = ql < nq;
+  int nv = 0;  // positions of the chunk this query sees
+  if (valid) nv = max(0, min(nj, pos0 + qi / G - j0 + 1));
+  const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+  float mx = -INFINITY, l = 0.f;
+  for (int c0 = 0; c0 < kAcN; c0 += 16) {
+    uint32_t v[16];
+    tmem_ld16(trow + c0, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (c0 + j < nv) mx = fmaxf(mx, __uint_as_float(v[j]));
+  }
+  for (int c0 = 0; c0 < kAcN; c0 += 16) {
+    uint32_t v[16];
+    tmem_ld16(trow + c0, v);
+    float pv[16], pr[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      pv[j] = c0 + j < nv ? expf(__uint_as_float(v[j]) - mx) : 0.f;
+      l += pv[j];
+      pr[j] = pv[j] - __bfloat162float(__float2bfloat16_rn(pv[j]));
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int col = c0 + 8 * hh;
+      const int off = (col >> 6) * kAcAtom + sw_off(r, (col & 63) >> 3);
+      const float *ph = pv + 8 * hh, *pl = pr + 8 * hh;
+      *reinterpret_cast<uint4 *>(sQ + off) =
+          make_uint4(pack_bf16(ph[0], ph[1]), pack_bf16(ph[2], ph[3]), pack_bf16(ph[4], ph[5]), pack_bf16(ph[6], ph[7]));
+      *reinterpret_cast<uint4 *>(sQ + 2 * kAcAtom + off) =
+          make_uint4(pack_bf16(pl[0], pl[1]), pack_bf16(pl[2], pl[3]), pack_bf16(pl[4], pl[5]), pack_bf16(pl[6], pl[7]));
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint64_t dph = tc_desc(sQ + i * kAcAtom), dpl = tc_desc(sQ + (2 + i) * kAcAtom),
+                       dv = tc_desc(sK + i * (HD * 128));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 positions per product
+          tc_mma(tmem + kAcN, dph + 2 * kk, dv + 2 * kk, kIdescO, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem + kAcN, dpl + 2 * kk, dv + 2 * kk, kIdescO, 1u);
+        }
+      }
+    }
+    tc_commit(&obar);
+  }
+  __syncwarp();
+  ok = tc_wait(&obar, 0, a.error) && ok;
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const long long slot = (static_cast<long long>(bg) * a.nch_max + c) * Q + qi;
+#pragma unroll
+  for (int c0 = 0; c0 < HD; c0 += 16) {
+    uint32_t v[16];
+    tmem_ld16(trow + kAcN + c0, v);
+    if (valid) {
+      float4 *dst = reinterpret_cast<float4 *>(a.opart + slot * HD + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = ok ? make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                                  __uint_as_float(v[4 * i + 3]))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  if (valid) {
+    a.mlpart[2 * slot] = mx;
+    a.mlpart[2 * slot + 1] = l;
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAcTmemCols) : "memory");
 }
 
-// o[m][h] = the log-sum-exp combination of query (m, h)'s chunk partials.
-// One block of HD threads per (row, head); thread i owns dim i.
+// Query (m, h)'s chunk partials combined with the log-sum-exp rule, written
+// straight into the bf16 pair that feeds the output projection (row m,
+// columns [h hd, h hd + hd)).  One block of hd threads per (row, head): warp 0
+// finds the largest chunk max and the weighted sum of the chunks' sums, then
+// thread i combines dim i.
 __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv, int hd, int nch_max,
-                                const float *opart, const float *mlpart, float *o) {
+                                const float *opart, const float *mlpart, __nv_bfloat16 *xhi, __nv_bfloat16 *xlo,
+                                int ldx) {
+  __shared__ float s_md[2];
   const int m = blockIdx.x, h = blockIdx.y, b = m / T, t = m % T, G = Hq / Hkv, g = h / G;
-  const int qi = t * G + h % G, bg = b * Hkv + g;
-  const int nch = (positions[b] + t) / kWaChunk + 1;  // chunks holding positions this query sees
-  float M = -INFINITY;
-  for (int c = 0; c < nch; ++c) {
-    const long long slot = (static_cast<long long>(bg) * nch_max + c) * (static_cast<long long>(T) * G) + qi;
-    M = fmaxf(M, mlpart[2 * slot]);
-  }
-  for (int i = threadIdx.x; i < hd; i += blockDim.x) {
-    float num = 0.f, den = 0.f;
-    for (int c = 0; c < nch; ++c) {
-      const long long slot = (static_cast<long long>(bg) * nch_max + c) * (static_cast<long long>(T) * G) + qi;
-      const float mc = mlpart[2 * slot];
-      if (mc == -INFINITY) continue;
-      const float w = expf(mc - M);
-      num = fmaf(w, opart[slot * hd + i], num);
-      den = fmaf(w, mlpart[2 * slot + 1], den);
+  const int Q = T * G, qi = t * G + h % G, bg = b * Hkv + g;
+  const int nch = (positions[b] + t) / kAcN + 1;  // chunks holding positions this query sees
+  const long long slot0 = static_cast<long long>(bg) * nch_max * Q + qi;  // chunk c: slot0 + c Q
+  if (threadIdx.x < 32) {
+    float M = -INFINITY;
+    for (int c = threadIdx.x; c < nch; c += 32) M = fmaxf(M, mlpart[2 * (slot0 + static_cast<long long>(c) * Q)]);
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+    for (int c = threadIdx.x; c < nch; c += 32) {
+      const float *ml = mlpart + 2 * (slot0 + static_cast<long long>(c) * Q);
+      den = fmaf(expf(ml[0] - M), ml[1], den);  // a chunk this query sees nothing of has max -inf: weight 0
     }
-    o[static_cast<long long>(m) * Hq * hd + h * hd + i] = num / den;
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (threadIdx.x == 0) {
+      s_md[0] = M;
+      s_md[1] = den;
+    }
+  }
+  __syncthreads();
+  const float M = s_md[0], den = s_md[1];
+  for (int i = threadIdx.x; i < hd; i += blockDim.x) {
+    float num = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < nch; ++c) {
+      const long long slot = slot0 + static_cast<long long>(c) * Q;
+      num = fmaf(expf(mlpart[2 * slot] - M), opart[slot * hd + i], num);
+    }
+    const long long at = static_cast<long long>(m) * ldx + h * hd + i;
+    split_store(num / den, xhi + at, xlo + at);
   }
 }
 
@@ -670,7 +838,9 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, int p
 }
 
 cudaError_t wide_prepare() {
-  return cudaFuncSetAttribute(wide_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes());
+  WIDE_TRY(cudaFuncSetAttribute(wide_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes()));
+  WIDE_TRY(cudaFuncSetAttribute(wide_attn_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(64)));
+  return cudaFuncSetAttribute(wide_attn_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(128));
 }
 
 cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
@@ -698,25 +868,40 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
                                                    s.vc, s.Bmax, s.cap, l);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    {
-      const int nch = (s.cap + kWaChunk - 1) / kWaChunk;
-      const dim3 grid(nch, s.B * s.Hkv);
+    {  // attention: chunk partials on the tensor cores, then the merge into the bf16 pair
+      const int G = s.Hq / s.Hkv, nch = (s.cap + kAcN - 1) / kAcN;
+      AttnArgs aa{};
+      // the kernel's TMA row coordinate is 32-bit
+      if (static_cast<uint64_t>(s.L) * s.Bmax * s.Hkv * s.cap > 0x7fffffffull ||
+          encode_2d_sw128(&aa.mk, s.kc, static_cast<uint64_t>(s.L) * s.Bmax * s.Hkv * s.cap, s.hd, s.hd, kAcN) != MK_OK)
+        return cudaErrorInvalidValue;
+      aa.qkv = s.qkv;
+      aa.W3 = W3;
+      aa.positions = s.positions_safe;
+      aa.T = s.T;
+      aa.Hq = s.Hq;
+      aa.Hkv = s.Hkv;
+      aa.rope = s.rope;
+      aa.vc = s.vc;
+      aa.Bmax = s.Bmax;
+      aa.cap = s.cap;
+      aa.layer = l;
+      aa.nch_max = nch;
+      aa.opart = s.attn_o;
+      aa.mlpart = s.attn_ml;
+      aa.error = s.error;
+      const dim3 grid(nch, s.B * s.Hkv, (s.T * G + 127) / 128);
       if (s.hd == 64)
-        wide_attn_chunk<2><<<grid, kWaWarps * 32, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.rope, s.kc,
-                                                            s.vc, s.Bmax, s.cap, l, nch, s.attn_o, s.attn_ml);
+        wide_attn_tc<64><<<grid, kAcThreads, attn_smem_bytes(64), st>>>(aa);
       else
-        wide_attn_chunk<4><<<grid, kWaWarps * 32, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.rope, s.kc,
-                                                            s.vc, s.Bmax, s.cap, l, nch, s.attn_o, s.attn_ml);
+        wide_attn_tc<128><<<grid, kAcThreads, attn_smem_bytes(128), st>>>(aa);
       WIDE_TRY(cudaGetLastError());
       ++n;
       wide_attn_merge<<<dim3(M, s.Hq), s.hd, 0, st>>>(s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
-                                                      s.attn_ml, s.o);
+                                                      s.attn_ml, s.xhi, s.xlo, ldx);
       WIDE_TRY(cudaGetLastError());
       ++n;
     }
-    wide_split<<<M, 256, 0, st>>>(s.o, HD, HD, s.xhi, s.xlo, ldx);
-    WIDE_TRY(cudaGetLastError());
-    ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), 1, d, HD, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M,
                   s.h, d, 1, st));
     // MoE block: router on the normed row, top-k, expert lists

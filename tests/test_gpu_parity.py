@@ -93,6 +93,18 @@ def test_ragged_wide_blocks(B, T):
     print(B, T, rep)
 
 
+def test_wide_block_more_query_vectors_than_one_tile():
+    """One sequence of 48 rows: 48 x 3 = 144 query vectors per KV head, more
+    than one 128-row tile of the tensor-core attention, over contexts of
+    several 128-position chunks."""
+    wl = Workload("ragged_wide_b1_t48", RAGGED, 1, 48, context=None, context_range=(200, 330), steps=3, seed=13)
+    s = Session(wl, capacity=512)
+    rep = run_verify(s, 2)
+    s.close()
+    assert rep.rows_compared >= 48
+    print(rep)
+
+
 def test_wide_block_rejects_bad_inputs_on_device():
     wl = Workload("ragged_wide_bad", RAGGED, 4, 4, context=None, context_range=(1, 40), steps=1, seed=12)
     s = Session(wl, capacity=64)
