@@ -36,7 +36,9 @@ __device__ __forceinline__ uint32_t sptr(const void *p) { return static_cast<uin
 // grid = (ceil(N / 128), ksplit, problems).  Problem p's weights are rows
 // [p * N, (p + 1) * N) of the weight map, its activation rows [row_off[p],
 // row_off[p] + row_cnt[p]) (or [0, R) when row_off is NULL); it writes the
-// same rows of Y.  With ksplit > 1 the CTA writes its K share into
+// same rows of Y.  A launch may hold two products over the same activations
+// (gate and up): problems pe .. 2 pe - 1 take the second weight map and write
+// from column ycol2 of Y on.  With ksplit > 1 the CTA writes its K share into
 // part[ks][row][n] for wide_gemm_finish.
 // ---------------------------------------------------------------------------
 constexpr int kTcM = 128;                              // weight rows per CTA (MMA M)
@@ -55,9 +57,11 @@ constexpr int kTcTmemCols = 64;                        // fp32 accumulator colum
 static_assert(kWideMaxRows <= kTcTmemCols, "one accumulator column per activation row");
 
 struct GemmArgs {
-  CUtensorMap mw;          // weights: [problems * N rows][K], box 64 x 128
+  CUtensorMap mw, mw2;     // weights: [pe * N rows][K], box 64 x 128 (mw2: the second product, if any)
   CUtensorMap mxh, mxl;    // activations hi / lo: [rows][K], box 64 x 16
   int N, K;
+  int pe;                  // problems per weight map; problem p >= pe is p - pe of mw2
+  int ycol2;               // column of Y (and part) where the second product's outputs start
   const int *row_off, *row_cnt;
   int R;
   float *Y;
@@ -122,9 +126,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
   uint8_t *smem = smem_raw + ((1024u - (sptr(smem_raw) & 1023u)) & 1023u);
   __shared__ __align__(8) uint64_t full[kTcStages], empty[kTcStages], done;
   __shared__ uint32_t tmem_base;
-  const int prob = blockIdx.z;
+  const int half = blockIdx.z >= a.pe, prob = blockIdx.z - (half ? a.pe : 0);
+  const CUtensorMap *mw = half ? &a.mw2 : &a.mw;
   const int r0 = a.row_off ? a.row_off[prob] : 0;
   const int R = a.row_off ? a.row_cnt[prob] : a.R;
+  const int ycol = half ? a.ycol2 : 0;
   if (R <= 0) return;  // the whole CTA, before anything is allocated
   const int n0 = blockIdx.x * kTcM;
   const int ksplit = gridDim.y, ks = blockIdx.y;
@@ -164,7 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
                    : "memory");
       for (int b = 0; b < kTcBoxes; ++b) {  // columns past K read as zeros
         const int x = ((kc0 + i) * kTcBoxes + b) * kTcK;
-        tc_tma(st + b * kTcWBox, &a.mw, x, prob * a.N + n0, &full[s]);
+        tc_tma(st + b * kTcWBox, mw, x, prob * a.N + n0, &full[s]);
         for (int g = 0; g < G; ++g) {
           tc_tma(st + kTcA + b * kTcXBox + g * kTcBoxBytes, &a.mxh, x, r0 + kTcRowBox * g, &full[s]);
           tc_tma(st + kTcA + kTcB + b * kTcXBox + g * kTcBoxBytes, &a.mxl, x, r0 + kTcRowBox * g, &full[s]);
@@ -211,9 +217,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       if (r >= R || n >= a.N) continue;
       const float val = ok ? __uint_as_float(v[j]) : 0.f;
       if (ksplit > 1) {
-        a.part[(static_cast<long long>(ks) * a.rows_total + r0 + r) * a.ldy + n] = val;
+        a.part[(static_cast<long long>(ks) * a.rows_total + r0 + r) * a.ldy + ycol + n] = val;
       } else {
-        float *y = a.Y + static_cast<long long>(r0 + r) * a.ldy + n;
+        float *y = a.Y + static_cast<long long>(r0 + r) * a.ldy + ycol + n;
         *y = a.accumulate ? *y + val : val;
       }
     }
@@ -661,43 +667,58 @@ __global__ void wide_topk(const float *logits, int E, int K, int32_t *sel_e, flo
   }
 }
 
-// Pairs (row m, selection j) grouped by expert, in (expert, m, j) order:
-// count[e], off[e], pair_row[q], pair_slot[m * K + j] = position q of the
-// pair.  One block; also adds the number of distinct experts to stats.
-__global__ void wide_expert_lists(const int32_t *sel_e, int M, int K, int E, int *count, int *off, int *pair_row,
-                                  int *pair_slot, unsigned long long *stats) {
-  __shared__ int cnt[kMaxExperts], start[kMaxExperts];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i < M * K; i += blockDim.x) atomicAdd(&cnt[sel_e[i]], 1);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int s = 0, nu = 0;
-    for (int e = 0; e < E; ++e) {
-      start[e] = s;
-      off[e] = s;
-      count[e] = cnt[e];
-      s += cnt[e];
-      nu += cnt[e] ? 1 : 0;
-    }
-    atomicAdd(stats, static_cast<unsigned long long>(nu));
-    // stable placement in (m, j) order
-    for (int i = 0; i < M * K; ++i) {
-      const int e = sel_e[i];
-      const int q = start[e]++;
-      pair_row[q] = i / K;
-      pair_slot[i] = q;
-    }
+// The routed (row, choice) pairs in expert-major order, and each pair's row
+// gathered there, in one launch.  Block i owns pair i = (m, j) (in (m, j)
+// order): its place is the number of pairs of a lower expert plus the earlier
+// pairs of its own expert (so the pairs of one expert keep (m, j) order), and
+// it copies row m of the bf16 pair to that place.  Block 0 also writes each
+// expert's count and first place and adds the number of experts in use to the
+// statistics.
+__global__ void wide_route_gather(const int32_t *sel_e, int M, int K, int E, const __nv_bfloat16 *xhi,
+                                  const __nv_bfloat16 *xlo, int ldx, int d, int *count, int *off, int *pair_row,
+                                  int *pair_slot, unsigned long long *stats, __nv_bfloat16 *ghi, __nv_bfloat16 *glo) {
+  __shared__ float red[32];
+  __shared__ int s_q;
+  const int i = blockIdx.x, MK = M * K, e = sel_e[i];
+  float before = 0.f;  // exact: at most a few thousand
+  for (int j = threadIdx.x; j < MK; j += blockDim.x) {
+    const int ej = sel_e[j];
+    before += (ej < e || (ej == e && j < i)) ? 1.f : 0.f;
   }
-}
-
-// rows of the bf16 pair gathered into pair order
-__global__ void wide_gather(const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, const int *pair_row, int K,
-                            __nv_bfloat16 *ghi, __nv_bfloat16 *glo) {
-  const int q = blockIdx.x, m = pair_row[q];
-  for (int c = threadIdx.x; c < K; c += blockDim.x) {
-    ghi[static_cast<long long>(q) * ldx + c] = xhi[static_cast<long long>(m) * ldx + c];
-    glo[static_cast<long long>(q) * ldx + c] = xlo[static_cast<long long>(m) * ldx + c];
+  before = block_sum(before, red);
+  if (threadIdx.x == 0) {
+    const int q = static_cast<int>(before);
+    s_q = q;
+    pair_slot[i] = q;
+    pair_row[q] = i / K;
+  }
+  if (i == 0) {
+    unsigned long long used = 0;
+    for (int x = threadIdx.x; x < E; x += blockDim.x) {
+      int c = 0, o = 0;
+      for (int j = 0; j < MK; ++j) {
+        const int ej = sel_e[j];
+        c += ej == x;
+        o += ej < x;
+      }
+      count[x] = c;
+      off[x] = o;
+      used += c > 0;
+    }
+    if (used) atomicAdd(stats, used);
+  }
+  __syncthreads();
+  const long long src = static_cast<long long>(i / K) * ldx, dst = static_cast<long long>(s_q) * ldx;
+  if ((d & 7) == 0) {  // 16-byte pieces (ldx is a multiple of 8)
+    for (int c = threadIdx.x; c < d / 8; c += blockDim.x) {
+      reinterpret_cast<uint4 *>(ghi + dst)[c] = reinterpret_cast<const uint4 *>(xhi + src)[c];
+      reinterpret_cast<uint4 *>(glo + dst)[c] = reinterpret_cast<const uint4 *>(xlo + src)[c];
+    }
+  } else {
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+      ghi[dst + c] = xhi[src + c];
+      glo[dst + c] = xlo[src + c];
+    }
   }
 }
 
@@ -712,10 +733,11 @@ __global__ void wide_swiglu(const float *gu, int F, __nv_bfloat16 *ahi, __nv_bfl
 }
 
 // h[m] += sum_j w[m][j] y[pair(m, j)] (selection order) + shared[m]
+// grid = (rows, ceil(d / blockDim)): one column per thread.
 __global__ void wide_combine(float *h, int d, int K, const float *sel_w, const int *pair_slot, const float *y,
                              const float *ys, float *dbg) {
   const int m = blockIdx.x;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+  for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < d; c += gridDim.y * blockDim.x) {
     float moe = 0.f;
     for (int j = 0; j < K; ++j)
       moe = fmaf(sel_w[m * K + j], y[static_cast<long long>(pair_slot[m * K + j]) * d + c], moe);
@@ -726,18 +748,32 @@ __global__ void wide_combine(float *h, int d, int K, const float *sel_w, const i
 }
 
 // argmax over the vocabulary per row (ties to the lowest index)
-__global__ void wide_argmax(const float *logits, int V, int32_t *out) {
+// One block per row; with V a multiple of 4 each thread reads 16-byte pieces.
+__global__ void __launch_bounds__(1024) wide_argmax(const float *logits, int V, int32_t *out) {
   __shared__ float bvs[32];
   __shared__ int bis[32];
   const int m = blockIdx.x;
+  const float *row = logits + static_cast<long long>(m) * V;
   float bv = -INFINITY;
   int bi = 0x7fffffff;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) {
-    const float x = logits[static_cast<long long>(m) * V + v];
+  auto take = [&](float x, int v) {
     if (x > bv || (x == bv && v < bi)) {
       bv = x;
       bi = v;
     }
+  };
+  if ((V & 3) == 0) {
+    const float4 *r4 = reinterpret_cast<const float4 *>(row);
+#pragma unroll 4
+    for (int v4 = threadIdx.x; v4 < V / 4; v4 += blockDim.x) {
+      const float4 x = r4[v4];
+      take(x.x, 4 * v4);
+      take(x.y, 4 * v4 + 1);
+      take(x.z, 4 * v4 + 2);
+      take(x.w, 4 * v4 + 3);
+    }
+  } else {
+    for (int v = threadIdx.x; v < V; v += blockDim.x) take(row[v], v);
   }
   for (int o = 16; o; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -799,17 +835,23 @@ int gemm_smem_bytes() { return kTcStages * kTcStage + 1024; }  // + room to alig
 // One product (or one grouped launch of per-expert products) on the tensor
 // cores: weight rows [p * N, (p + 1) * N) x K for problem p, activation rows
 // of the xrows-row buffers xhi / xlo (row stride ldx).  A single dense problem
-// whose 128-row tiles do not fill the GPU splits K.
-static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, int problems, int N, int K,
-                        const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, int xrows, const int *row_off,
-                        const int *row_cnt, int R, float *Y, int ldy, int accumulate, cudaStream_t st) {
+// whose 128-row tiles do not fill the GPU splits K, through `part` (one
+// split-K buffer per stream that runs products concurrently).
+static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const __nv_bfloat16 *W2, int pe, int N,
+                        int K, const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, int xrows,
+                        const int *row_off, const int *row_cnt, int R, float *Y, int ldy, int ycol2, int accumulate,
+                        float *part, cudaStream_t st) {
   GemmArgs a{};
-  if (encode_2d_sw128(&a.mw, W, static_cast<uint64_t>(problems) * N, K, K, kTcM) != MK_OK ||
+  const int problems = W2 ? 2 * pe : pe;
+  if (encode_2d_sw128(&a.mw, W, static_cast<uint64_t>(pe) * N, K, K, kTcM) != MK_OK ||
+      encode_2d_sw128(&a.mw2, W2 ? W2 : W, static_cast<uint64_t>(pe) * N, K, K, kTcM) != MK_OK ||
       encode_2d_sw128(&a.mxh, xhi, xrows, K, ldx, kTcRowBox) != MK_OK ||
       encode_2d_sw128(&a.mxl, xlo, xrows, K, ldx, kTcRowBox) != MK_OK)
     return cudaErrorInvalidValue;
   a.N = N;
   a.K = K;
+  a.pe = pe;
+  a.ycol2 = ycol2;
   a.row_off = row_off;
   a.row_cnt = row_cnt;
   a.R = R;
@@ -822,15 +864,15 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, int p
   int ksplit = 1;
   if (!row_off) {  // one dense problem: about one CTA per SM, at least two K stages each
     const int nkc = (K + kTcBoxes * kTcK - 1) / (kTcBoxes * kTcK);
-    ksplit = std::max(1, std::min(std::min(s.n_sm / nb, nkc / 2), 16));
+    ksplit = std::max(1, std::min(std::min(s.n_sm / (nb * problems), nkc / 2), 16));
     if (static_cast<long long>(ksplit) * R * ldy > s.part_floats) ksplit = 1;
   }
-  a.part = ksplit > 1 ? s.part : nullptr;
+  a.part = ksplit > 1 ? part : nullptr;
   wide_gemm<<<dim3(nb, ksplit, problems), kTcThreads, gemm_smem_bytes(), st>>>(a);
   WIDE_TRY(cudaGetLastError());
   ++n;
   if (ksplit > 1) {
-    wide_gemm_finish<<<2 * s.n_sm, 256, 0, st>>>(s.part, ksplit, R, N, ldy, Y, accumulate);
+    wide_gemm_finish<<<2 * s.n_sm, 256, 0, st>>>(part, ksplit, R, W2 ? ycol2 + N : N, ldy, Y, accumulate);
     WIDE_TRY(cudaGetLastError());
     ++n;
   }
@@ -862,8 +904,8 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
                                        s.xlo, ldx);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wqkv), 1, W3, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M,
-                  s.qkv, W3, 0, st));
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wqkv), nullptr, 1, W3, d, s.xhi, s.xlo, ldx, M, nullptr,
+                  nullptr, M, s.qkv, W3, 0, 0, s.part, st));
     wide_kv_append<<<dim3(M, s.Hkv), 128, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, s.rope, s.kc,
                                                    s.vc, s.Bmax, s.cap, l);
     WIDE_TRY(cudaGetLastError());
@@ -902,50 +944,51 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       WIDE_TRY(cudaGetLastError());
       ++n;
     }
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), 1, d, HD, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M,
-                  s.h, d, 1, st));
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), nullptr, 1, d, HD, s.xhi, s.xlo, ldx, M, nullptr,
+                  nullptr, M, s.h, d, 0, 1, s.part, st));
     // MoE block: router on the normed row, top-k, expert lists
     wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.ffn_norm), d, s.eps, s.xhi, s.xlo,
                                        ldx);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), 1, E, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M,
-                  s.rlog, E, 0, st));
+    // The shared expert needs only the normed rows: it runs on a second stream
+    // (a parallel branch of the graph) beside the router and the routed
+    // experts, with its own split-K buffer, and joins before the combine.
+    if (Fs > 0) {
+      cudaStream_t sd = s.side;
+      WIDE_TRY(cudaEventRecord(s.ev_fork, st));
+      WIDE_TRY(cudaStreamWaitEvent(sd, s.ev_fork, 0));
+      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_gate), static_cast<const __nv_bfloat16 *>(lw.ws_up),
+                    1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.gs, 2 * Fs, Fs, 0, s.part2, sd));
+      wide_swiglu<<<M, 256, 0, sd>>>(s.gs, Fs, s.shi, s.slo, s.lda);
+      WIDE_TRY(cudaGetLastError());
+      ++n;
+      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), nullptr, 1, d, Fs, s.shi, s.slo, s.lda, M,
+                    nullptr, nullptr, M, s.ys, d, 0, 0, s.part2, sd));
+      WIDE_TRY(cudaEventRecord(s.ev_join, sd));
+    }
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), nullptr, 1, E, d, s.xhi, s.xlo, ldx, M, nullptr,
+                  nullptr, M, s.rlog, E, 0, 0, s.part, st));
     int32_t *dbg_ids = s.dbg_ids ? s.dbg_ids + static_cast<long long>(l) * s.max_rows * K : nullptr;
     float *dbg_w = s.dbg_w ? s.dbg_w + static_cast<long long>(l) * s.max_rows * K : nullptr;
     wide_topk<<<M, 32, 0, st>>>(s.rlog, E, K, s.sel_e, s.sel_w, dbg_ids, dbg_w);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    wide_expert_lists<<<1, 256, 0, st>>>(s.sel_e, M, K, E, s.count, s.off, s.pair_row, s.pair_slot, s.stats);
+    // routed experts: expert lists + gather, gate and up over each expert's rows, SwiGLU, down
+    wide_route_gather<<<M * K, 256, 0, st>>>(s.sel_e, M, K, E, s.xhi, s.xlo, ldx, d, s.count, s.off, s.pair_row,
+                                             s.pair_slot, s.stats, s.ghi, s.glo);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    // routed experts: gate and up over each expert's rows, SwiGLU, down
-    wide_gather<<<M * K, 256, 0, st>>>(s.xhi, s.xlo, ldx, s.pair_row, d, s.ghi, s.glo);
-    WIDE_TRY(cudaGetLastError());
-    ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), E, F, d, s.ghi, s.glo, ldx, M * K, s.off, s.count,
-                  M * K, s.gu, 2 * F, 0, st));
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_up), E, F, d, s.ghi, s.glo, ldx, M * K, s.off, s.count,
-                  M * K, s.gu + F, 2 * F, 0, st));
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), static_cast<const __nv_bfloat16 *>(lw.w_up), E, F,
+                  d, s.ghi, s.glo, ldx, M * K, s.off, s.count, M * K, s.gu, 2 * F, F, 0, s.part, st));
     wide_swiglu<<<M * K, 256, 0, st>>>(s.gu, F, s.ahi, s.alo, s.lda);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), E, d, F, s.ahi, s.alo, s.lda, M * K, s.off,
-                  s.count, M * K, s.yd, d, 0, st));
-    // shared expert on every row
-    if (Fs > 0) {
-      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_gate), 1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr,
-                    nullptr, M, s.gs, 2 * Fs, 0, st));
-      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_up), 1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr,
-                    M, s.gs + Fs, 2 * Fs, 0, st));
-      wide_swiglu<<<M, 256, 0, st>>>(s.gs, Fs, s.shi, s.slo, s.lda);
-      WIDE_TRY(cudaGetLastError());
-      ++n;
-      WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), 1, d, Fs, s.shi, s.slo, s.lda, M, nullptr,
-                    nullptr, M, s.ys, d, 0, st));
-    }
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), nullptr, E, d, F, s.ahi, s.alo, s.lda, M * K,
+                  s.off, s.count, M * K, s.yd, d, 0, 0, s.part, st));
+    if (Fs > 0) WIDE_TRY(cudaStreamWaitEvent(st, s.ev_join, 0));  // the shared expert's branch
     float *dbg = s.dbg_hidden ? s.dbg_hidden + static_cast<long long>(l + 1) * s.max_rows * d : nullptr;
-    wide_combine<<<M, 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr, dbg);
+    wide_combine<<<dim3(M, (d + 255) / 256), 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr, dbg);
     WIDE_TRY(cudaGetLastError());
     ++n;
   }
@@ -953,8 +996,9 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
   wide_norm_split<<<M, 256, 0, st>>>(s.h, s.final_norm, d, s.eps, s.xhi, s.xlo, ldx);
   WIDE_TRY(cudaGetLastError());
   ++n;
-  WIDE_TRY(gemm(n, s, s.lm_head, 1, s.V, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.logits, s.V, 0, st));
-  wide_argmax<<<M, 256, 0, st>>>(s.logits, s.V, s.argmax);
+  WIDE_TRY(gemm(n, s, s.lm_head, nullptr, 1, s.V, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.logits, s.V, 0, 0, s.part,
+                st));
+  wide_argmax<<<M, 1024, 0, st>>>(s.logits, s.V, s.argmax);
   WIDE_TRY(cudaGetLastError());
   if (launches) *launches = n + 1;
   return cudaSuccess;
