@@ -266,9 +266,6 @@ struct mk_handle {
   int wide_ldx, wide_lda;
   float *w_h, *w_qkv, *w_rlog, *w_selw, *w_gu, *w_yd, *w_gs, *w_ys, *w_part, *w_attn_o, *w_attn_ml;
   long long w_part_floats;
-  float *w_part2;               // the side stream's split-K partials
-  cudaStream_t side_stream;     // second stream of the wide-block graph
-  cudaEvent_t ev_fork, ev_join;
   int32_t *w_sele, *w_tok, *w_pos;
   int *w_count, *w_off, *w_pair_row, *w_pair_slot;
   __nv_bfloat16 *w_xhi, *w_xlo, *w_ghi, *w_glo, *w_ahi, *w_alo, *w_shi, *w_slo;
@@ -366,9 +363,6 @@ MK_API void mk_destroy(mk_handle *h) {
   if (!h) return;
   for (auto &g : h->graphs) cudaGraphExecDestroy(g.exec);
   if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
-  if (h->side_stream) cudaStreamDestroy(h->side_stream);
-  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
-  if (h->ev_join) cudaEventDestroy(h->ev_join);
   for (void *p : h->allocs) cudaFree(p);
   delete h;
 }
@@ -516,13 +510,6 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     const int ld_max = std::max(std::max(QKVW, D), std::max(2 * Fs, std::max(d.n_experts, HD)));
     h->w_part_floats = 16LL * MR * ld_max;
     HALLOC(h->w_part, sizeof(float) * (size_t)h->w_part_floats);
-    HALLOC(h->w_part2, sizeof(float) * (size_t)h->w_part_floats);
-    if (cudaStreamCreateWithFlags(&h->side_stream, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
-      mk_destroy(h);
-      return fail(MK_ERR_CUDA, "wide-block stream setup failed");
-    }
     cudaError_t pe = wide_prepare();
     if (pe != cudaSuccess) {
       mk_destroy(h);
@@ -714,8 +701,6 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
   s.attn_o = h->w_attn_o; s.attn_ml = h->w_attn_ml;
   s.h = h->w_h; s.qkv = h->w_qkv; s.rlog = h->w_rlog; s.sel_w = h->w_selw; s.gu = h->w_gu;
   s.yd = h->w_yd; s.gs = h->w_gs; s.ys = h->w_ys; s.part = h->w_part; s.part_floats = h->w_part_floats;
-  s.part2 = h->w_part2;
-  s.side = h->side_stream; s.ev_fork = h->ev_fork; s.ev_join = h->ev_join;
   s.sel_e = h->w_sele; s.count = h->w_count; s.off = h->w_off; s.pair_row = h->w_pair_row;
   s.pair_slot = h->w_pair_slot;
   s.xhi = h->w_xhi; s.xlo = h->w_xlo; s.ghi = h->w_ghi; s.glo = h->w_glo; s.ahi = h->w_ahi; s.alo = h->w_alo;

@@ -209,9 +209,6 @@ struct WideStep {
   float *h, *qkv, *rlog, *sel_w, *gu, *yd, *gs, *ys, *part;
   float *attn_o, *attn_ml;  // attention partials: [rows * Hq * ceil(cap / 128)] x hd and x 2
   long long part_floats;
-  float *part2;                  // the side stream's split-K buffer (part_floats floats, like part)
-  cudaStream_t side;             // second stream of the captured graph (the shared expert)
-  cudaEvent_t ev_fork, ev_join;  // fork to / join from the side stream
   int32_t *sel_e;
   int *count, *off, *pair_row, *pair_slot;
   __nv_bfloat16 *xhi, *xlo, *ghi, *glo, *ahi, *alo, *shi, *slo;

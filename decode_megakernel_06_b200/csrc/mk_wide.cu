@@ -23,23 +23,29 @@ __device__ __forceinline__ uint32_t sptr(const void *p) { return static_cast<uin
 
 // ---------------------------------------------------------------------------
 // Y[r][n] (+)= sum_k W[n][k] * (xhi[r][k] + xlo[r][k]) on the 5th-generation
-// tensor cores.  A CTA owns 128 weight rows (the MMA's M) of one problem and
-// all of its activation rows (the MMA's N: 16 to 64), over its share of K:
-//  - warp 0 (one thread) streams K in stages of 128 columns by TMA: per 64
-//    columns a 128 x 64 weight box and the activation rows in 16-row boxes,
-//    hi and lo, all 128B-swizzled, completing on the stage's full mbarrier;
+// tensor cores.  A unit of work is 128 weight rows (the MMA's M) of one
+// problem against all of its activation rows (the MMA's N: 16 to 64), over
+// one share of K.  The kernel is persistent: CTA b takes units b, b + grid,
+// ... and streams them through one pipeline, so the set-up and the first
+// loads are paid once per CTA, not once per unit:
+//  - warp 0 (one thread) streams each unit's K in stages of 128 columns by
+//    TMA: per 64 columns a 128 x 64 weight box and the activation rows in
+//    16-row boxes, hi and lo, all 128B-swizzled, completing on the stage's
+//    full mbarrier;
 //  - warp 1 (one thread) issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
-//    K = 16 each, hi then lo into one accumulator in tensor memory, and
-//    releases the stage with tcgen05.commit on its empty mbarrier;
-//  - then every warp reads its 32 accumulator lanes (weight rows) with
-//    tcgen05.ld and writes them out.
-// grid = (ceil(N / 128), ksplit, problems).  Problem p's weights are rows
-// [p * N, (p + 1) * N) of the weight map, its activation rows [row_off[p],
-// row_off[p] + row_cnt[p]) (or [0, R) when row_off is NULL); it writes the
-// same rows of Y.  A launch may hold two products over the same activations
-// (gate and up): problems pe .. 2 pe - 1 take the second weight map and write
-// from column ycol2 of Y on.  With ksplit > 1 the CTA writes its K share into
-// part[ks][row][n] for wide_gemm_finish.
+//    K = 16 each, hi then lo into one of two accumulators in tensor memory,
+//    releases each stage with tcgen05.commit on its empty mbarrier, and marks
+//    the unit's accumulator full;
+//  - warps 2-5 read the accumulator (each its 32 lanes = weight rows) with
+//    tcgen05.ld, write the unit out and hand the accumulator back, while the
+//    next unit's products go into the other one.
+// Units: (problem, K share, 128-row tile), tile fastest.  Problem p's weights
+// are rows [p * N, (p + 1) * N) of the weight map, its activation rows
+// [row_off[p], row_off[p] + row_cnt[p]) (or [0, R) when row_off is NULL); it
+// writes the same rows of Y.  A launch may hold two products over the same
+// activations (gate and up): problems pe .. 2 pe - 1 take the second weight
+// map and write from column ycol2 of Y on.  With ksplit > 1 a unit writes its
+// K share into part[ks][row][n] for wide_gemm_finish.
 // ---------------------------------------------------------------------------
 constexpr int kTcM = 128;                              // weight rows per CTA (MMA M)
 constexpr int kTcK = 64;                               // K columns per box: one 128-byte swizzled row
@@ -52,9 +58,10 @@ constexpr int kTcXBox = kWideMaxRows * kTcK * 2;       // 8 KB: up to 64 activat
 constexpr int kTcA = kTcBoxes * kTcWBox;               // weights per stage
 constexpr int kTcB = kTcBoxes * kTcXBox;               // one activation half (hi or lo) per stage
 constexpr int kTcStage = kTcA + 2 * kTcB;
-constexpr int kTcThreads = 128;
-constexpr int kTcTmemCols = 64;                        // fp32 accumulator columns: one per activation row
-static_assert(kWideMaxRows <= kTcTmemCols, "one accumulator column per activation row");
+constexpr int kTcThreads = 192;                        // producer warp, MMA warp, 4 epilogue warps
+constexpr int kTcAccCols = 64;                         // fp32 accumulator columns: one per activation row
+constexpr int kTcTmemCols = 2 * kTcAccCols;            // two accumulators
+static_assert(kWideMaxRows <= kTcAccCols, "one accumulator column per activation row");
 
 struct GemmArgs {
   CUtensorMap mw, mw2;     // weights: [pe * N rows][K], box 64 x 128 (mw2: the second product, if any)
@@ -62,6 +69,7 @@ struct GemmArgs {
   int N, K;
   int pe;                  // problems per weight map; problem p >= pe is p - pe of mw2
   int ycol2;               // column of Y (and part) where the second product's outputs start
+  int nb, ksplit, units;   // 128-row tiles per problem, K shares, nb * ksplit * problems
   const int *row_off, *row_cnt;
   int R;
   float *Y;
@@ -120,23 +128,51 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
                : "memory");
 }
 
+// One unit's coordinates; R <= 0 marks a problem without rows (skipped by
+// every role alike).
+struct TcUnit {
+  const CUtensorMap *mw;
+  int wrow, r0, R, n0, kc0, nk, G, ycol, ks;
+};
+__device__ __forceinline__ TcUnit tc_unit(const GemmArgs &a, int u, int nkc) {
+  TcUnit t;
+  const int tile = u % a.nb, ks = (u / a.nb) % a.ksplit, pz = u / (a.nb * a.ksplit);
+  const int half = pz >= a.pe, prob = pz - (half ? a.pe : 0);
+  t.mw = half ? &a.mw2 : &a.mw;
+  t.r0 = a.row_off ? a.row_off[prob] : 0;
+  t.R = a.row_off ? a.row_cnt[prob] : a.R;
+  t.n0 = tile * kTcM;
+  t.wrow = prob * a.N + t.n0;
+  t.kc0 = (nkc * ks) / a.ksplit;
+  t.nk = (nkc * (ks + 1)) / a.ksplit - t.kc0;
+  t.G = (t.R + kTcRowBox - 1) / kTcRowBox;
+  t.ycol = half ? a.ycol2 : 0;
+  t.ks = ks;
+  return t;
+}
+
+// Bounded wait that also gives up once another role has (abort != 0).
+__device__ __forceinline__ bool tc_wait_or_abort(uint64_t *bar, uint32_t par, int *error, volatile int *abort) {
+  const uint64_t t0 = tc_now();
+  while (!tc_try_wait(bar, par)) {
+    if (*abort) return false;
+    if (tc_now() - t0 > 1000000000ull) {
+      if (atomicCAS(&error[0], 0, -5) == 0) atomicExch(&error[1], -2);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   // stages start on 1024-byte boundaries (the 128-byte swizzle repeats every 8 rows)
   uint8_t *smem = smem_raw + ((1024u - (sptr(smem_raw) & 1023u)) & 1023u);
-  __shared__ __align__(8) uint64_t full[kTcStages], empty[kTcStages], done;
+  __shared__ __align__(8) uint64_t full[kTcStages], empty[kTcStages], accf[2], acce[2];
   __shared__ uint32_t tmem_base;
-  const int half = blockIdx.z >= a.pe, prob = blockIdx.z - (half ? a.pe : 0);
-  const CUtensorMap *mw = half ? &a.mw2 : &a.mw;
-  const int r0 = a.row_off ? a.row_off[prob] : 0;
-  const int R = a.row_off ? a.row_cnt[prob] : a.R;
-  const int ycol = half ? a.ycol2 : 0;
-  if (R <= 0) return;  // the whole CTA, before anything is allocated
-  const int n0 = blockIdx.x * kTcM;
-  const int ksplit = gridDim.y, ks = blockIdx.y;
+  __shared__ int abort_flag;
   const int nkc = (a.K + kTcBoxes * kTcK - 1) / (kTcBoxes * kTcK);
-  const int kc0 = (nkc * ks) / ksplit, kc1 = (nkc * (ks + 1)) / ksplit, nk = kc1 - kc0;
-  const int G = (R + kTcRowBox - 1) / kTcRowBox, NM = kTcRowBox * G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sptr(&tmem_base)),
@@ -149,85 +185,129 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&full[s])) : "memory");
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&empty[s])) : "memory");
     }
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&done)) : "memory");
+    for (int b = 0; b < 2; ++b) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sptr(&accf[b])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(sptr(&acce[b])), "r"(32 * 4) : "memory");
+    }
+    abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = tmem_base;
-  // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
-  // K-major, N = NM, M = 128
-  const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(NM >> 3) << 17) |
-                         (static_cast<uint32_t>(kTcM >> 4) << 24);
-  if (warp == 0 && lane == 0) {  // TMA producer
-    for (int i = 0; i < nk; ++i) {
-      const int s = i % kTcStages;
-      if (i >= kTcStages && !tc_wait(&empty[s], ((i / kTcStages) & 1) ^ 1, a.error)) break;
-      uint8_t *st = smem + s * kTcStage;
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&full[s])),
-                   "r"(kTcBoxes * (kTcWBox + 2 * G * kTcBoxBytes))
-                   : "memory");
-      for (int b = 0; b < kTcBoxes; ++b) {  // columns past K read as zeros
-        const int x = ((kc0 + i) * kTcBoxes + b) * kTcK;
-        tc_tma(st + b * kTcWBox, mw, x, prob * a.N + n0, &full[s]);
-        for (int g = 0; g < G; ++g) {
-          tc_tma(st + kTcA + b * kTcXBox + g * kTcBoxBytes, &a.mxh, x, r0 + kTcRowBox * g, &full[s]);
-          tc_tma(st + kTcA + kTcB + b * kTcXBox + g * kTcBoxBytes, &a.mxl, x, r0 + kTcRowBox * g, &full[s]);
+  volatile int *abort = &abort_flag;
+  if (warp == 0) {
+    if (lane == 0) {  // TMA producer: every unit's stages through one ring
+      int it = 0;
+      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+        const TcUnit t = tc_unit(a, u, nkc);
+        if (t.R <= 0) continue;
+        for (int i = 0; i < t.nk; ++i, ++it) {
+          const int s = it % kTcStages;
+          if (it >= kTcStages && !tc_wait_or_abort(&empty[s], ((it / kTcStages) & 1) ^ 1, a.error, abort)) break;
+          uint8_t *st = smem + s * kTcStage;
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&full[s])),
+                       "r"(kTcBoxes * (kTcWBox + 2 * t.G * kTcBoxBytes))
+                       : "memory");
+          for (int b = 0; b < kTcBoxes; ++b) {  // columns past K read as zeros
+            const int x = ((t.kc0 + i) * kTcBoxes + b) * kTcK;
+            tc_tma(st + b * kTcWBox, t.mw, x, t.wrow, &full[s]);
+            for (int g = 0; g < t.G; ++g) {
+              tc_tma(st + kTcA + b * kTcXBox + g * kTcBoxBytes, &a.mxh, x, t.r0 + kTcRowBox * g, &full[s]);
+              tc_tma(st + kTcA + kTcB + b * kTcXBox + g * kTcBoxBytes, &a.mxl, x, t.r0 + kTcRowBox * g, &full[s]);
+            }
+          }
         }
       }
     }
-  }
-  if (warp == 1 && lane == 0) {  // MMA issuer
-    for (int i = 0; i < nk; ++i) {
-      const int s = i % kTcStages;
-      if (!tc_wait(&full[s], (i / kTcStages) & 1, a.error)) break;
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      int it = 0, lu = 0;
+      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x, ++lu) {
+        const TcUnit t = tc_unit(a, u, nkc);
+        if (t.R <= 0) {
+          --lu;
+          continue;
+        }
+        const int buf = lu & 1;
+        if (lu >= 2 && !tc_wait_or_abort(&acce[buf], ((lu >> 1) & 1) ^ 1, a.error, abort)) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t acc = tmem + static_cast<uint32_t>(buf * kTcAccCols);
+        // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B,
+        // both K-major, N = 16 G, M = 128
+        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                               (static_cast<uint32_t>((kTcRowBox * t.G) >> 3) << 17) |
+                               (static_cast<uint32_t>(kTcM >> 4) << 24);
+        bool ok = true;
+        for (int i = 0; i < t.nk; ++i, ++it) {
+          const int s = it % kTcStages;
+          if (!tc_wait_or_abort(&full[s], (it / kTcStages) & 1, a.error, abort)) {
+            ok = false;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const uint8_t *st = smem + s * kTcStage;
+#pragma unroll
+          for (int b = 0; b < kTcBoxes; ++b) {
+            const uint64_t da = tc_desc(st + b * kTcWBox), dh = tc_desc(st + kTcA + b * kTcXBox),
+                           dl = tc_desc(st + kTcA + kTcB + b * kTcXBox);
+#pragma unroll
+            for (int kk = 0; kk < kTcK / 16; ++kk) {  // 16 columns = 32 bytes = 2 descriptor units
+              tc_mma(acc, da + 2 * kk, dh + 2 * kk, idesc, (i > 0 || b > 0 || kk > 0) ? 1u : 0u);
+              tc_mma(acc, da + 2 * kk, dl + 2 * kk, idesc, 1u);
+            }
+          }
+          tc_commit(&empty[s]);  // the stage is free once these products have read it
+        }
+        if (!ok) break;
+        tc_commit(&accf[buf]);  // the unit's accumulator is complete
+      }
+    }
+  } else {  // epilogue: warp w reads accumulator lanes 32 (w mod 4) ..
+    const int q = warp & 3;
+    int lu = 0;
+    for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
+      const TcUnit t = tc_unit(a, u, nkc);
+      if (t.R <= 0) continue;
+      const int buf = lu & 1;
+      const bool ok = __all_sync(0xffffffffu, tc_wait_or_abort(&accf[buf], (lu >> 1) & 1, a.error, abort));
+      if (!ok) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint8_t *st = smem + s * kTcStage;
+      const int n = t.n0 + 32 * q + lane;
+      const int NM = kTcRowBox * t.G;
+      for (int c0 = 0; c0 < NM; c0 += 16) {
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * kTcAccCols + c0)));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-      for (int b = 0; b < kTcBoxes; ++b) {
-        const uint64_t da = tc_desc(st + b * kTcWBox), dh = tc_desc(st + kTcA + b * kTcXBox),
-                       dl = tc_desc(st + kTcA + kTcB + b * kTcXBox);
-#pragma unroll
-        for (int kk = 0; kk < kTcK / 16; ++kk) {  // 16 columns = 32 bytes = 2 descriptor units
-          tc_mma(tmem, da + 2 * kk, dh + 2 * kk, idesc, (i > 0 || b > 0 || kk > 0) ? 1u : 0u);
-          tc_mma(tmem, da + 2 * kk, dl + 2 * kk, idesc, 1u);
+        for (int j = 0; j < 16; ++j) {
+          const int r = c0 + j;
+          if (r >= t.R || n >= a.N) continue;
+          const float val = __uint_as_float(v[j]);
+          if (a.ksplit > 1) {
+            a.part[(static_cast<long long>(t.ks) * a.rows_total + t.r0 + r) * a.ldy + t.ycol + n] = val;
+          } else {
+            float *y = a.Y + static_cast<long long>(t.r0 + r) * a.ldy + t.ycol + n;
+            *y = a.accumulate ? *y + val : val;
+          }
         }
       }
-      tc_commit(&empty[s]);  // the stage is free once these products have read it
-    }
-    tc_commit(&done);
-  }
-  __syncwarp();
-  const bool ok = tc_wait(&done, 0, a.error) && nk > 0;
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  // warp w holds accumulator lanes 32w .. 32w + 31 = weight rows n0 + 32w + lane
-  const int n = n0 + 32 * warp + lane;
-  for (int c0 = 0; c0 < NM; c0 += 16) {
-    uint32_t v[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(tmem + (static_cast<uint32_t>(32 * warp) << 16) + static_cast<uint32_t>(c0)));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int r = c0 + j;
-      if (r >= R || n >= a.N) continue;
-      const float val = ok ? __uint_as_float(v[j]) : 0.f;
-      if (ksplit > 1) {
-        a.part[(static_cast<long long>(ks) * a.rows_total + r0 + r) * a.ldy + ycol + n] = val;
-      } else {
-        float *y = a.Y + static_cast<long long>(r0 + r) * a.ldy + ycol + n;
-        *y = a.accumulate ? *y + val : val;
-      }
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(sptr(&acce[buf])) : "memory");
+      ++lu;
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0)
+  if (warp == 0) {
+    __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols) : "memory");
+  }
 }
 
 // Y[r][n] (+)= sum over ks of part[ks][r][n], in order.
@@ -835,8 +915,7 @@ int gemm_smem_bytes() { return kTcStages * kTcStage + 1024; }  // + room to alig
 // One product (or one grouped launch of per-expert products) on the tensor
 // cores: weight rows [p * N, (p + 1) * N) x K for problem p, activation rows
 // of the xrows-row buffers xhi / xlo (row stride ldx).  A single dense problem
-// whose 128-row tiles do not fill the GPU splits K, through `part` (one
-// split-K buffer per stream that runs products concurrently).
+// whose 128-row tiles do not fill the GPU splits K, through `part`.
 static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const __nv_bfloat16 *W2, int pe, int N,
                         int K, const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, int xrows,
                         const int *row_off, const int *row_cnt, int R, float *Y, int ldy, int ycol2, int accumulate,
@@ -868,7 +947,10 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const
     if (static_cast<long long>(ksplit) * R * ldy > s.part_floats) ksplit = 1;
   }
   a.part = ksplit > 1 ? part : nullptr;
-  wide_gemm<<<dim3(nb, ksplit, problems), kTcThreads, gemm_smem_bytes(), st>>>(a);
+  a.nb = nb;
+  a.ksplit = ksplit;
+  a.units = nb * ksplit * problems;
+  wide_gemm<<<std::min(a.units, s.n_sm), kTcThreads, gemm_smem_bytes(), st>>>(a);
   WIDE_TRY(cudaGetLastError());
   ++n;
   if (ksplit > 1) {
@@ -951,21 +1033,15 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
                                        ldx);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    // The shared expert needs only the normed rows: it runs on a second stream
-    // (a parallel branch of the graph) beside the router and the routed
-    // experts, with its own split-K buffer, and joins before the combine.
+    // shared expert on every row (gate and up in one launch)
     if (Fs > 0) {
-      cudaStream_t sd = s.side;
-      WIDE_TRY(cudaEventRecord(s.ev_fork, st));
-      WIDE_TRY(cudaStreamWaitEvent(sd, s.ev_fork, 0));
       WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_gate), static_cast<const __nv_bfloat16 *>(lw.ws_up),
-                    1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.gs, 2 * Fs, Fs, 0, s.part2, sd));
-      wide_swiglu<<<M, 256, 0, sd>>>(s.gs, Fs, s.shi, s.slo, s.lda);
+                    1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.gs, 2 * Fs, Fs, 0, s.part, st));
+      wide_swiglu<<<M, 256, 0, st>>>(s.gs, Fs, s.shi, s.slo, s.lda);
       WIDE_TRY(cudaGetLastError());
       ++n;
       WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), nullptr, 1, d, Fs, s.shi, s.slo, s.lda, M,
-                    nullptr, nullptr, M, s.ys, d, 0, 0, s.part2, sd));
-      WIDE_TRY(cudaEventRecord(s.ev_join, sd));
+                    nullptr, nullptr, M, s.ys, d, 0, 0, s.part, st));
     }
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), nullptr, 1, E, d, s.xhi, s.xlo, ldx, M, nullptr,
                   nullptr, M, s.rlog, E, 0, 0, s.part, st));
@@ -986,7 +1062,6 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), nullptr, E, d, F, s.ahi, s.alo, s.lda, M * K,
                   s.off, s.count, M * K, s.yd, d, 0, 0, s.part, st));
-    if (Fs > 0) WIDE_TRY(cudaStreamWaitEvent(st, s.ev_join, 0));  // the shared expert's branch
     float *dbg = s.dbg_hidden ? s.dbg_hidden + static_cast<long long>(l + 1) * s.max_rows * d : nullptr;
     wide_combine<<<dim3(M, (d + 255) / 256), 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr, dbg);
     WIDE_TRY(cudaGetLastError());
