@@ -343,6 +343,20 @@ __device__ __forceinline__ void split_store(float x, __nv_bfloat16 *hi, __nv_bfl
   *lo = __float2bfloat16_rn(x - __bfloat162float(h));
 }
 
+// A product whose K shares are still in the split-K buffer: the consumer adds
+// part[0][r][col] + part[1][r][col] + ... in that order (as wide_gemm_finish
+// would have) instead of reading the finished value.  ks <= 1: nothing
+// deferred, the product is in its output already.
+struct Split {
+  const float *part;
+  int ks, rows, ld;
+};
+__device__ __forceinline__ float split_sum(const Split &p, int r, int col) {
+  float s = 0.f;
+  for (int k = 0; k < p.ks; ++k) s += p.part[(static_cast<long long>(k) * p.rows + r) * p.ld + col];
+  return s;
+}
+
 // h[m] = embed[token[m]]; the debug copy of the layer-0 input.
 __global__ void wide_embed(const int32_t *tokens, const __nv_bfloat16 *embed, int d, float *h, float *dbg) {
   const int m = blockIdx.x;
@@ -354,14 +368,22 @@ __global__ void wide_embed(const int32_t *tokens, const __nv_bfloat16 *embed, in
   }
 }
 
-// x = h / sqrt(mean(h^2) + eps) * g, as a bf16 pair.
-__global__ void wide_norm_split(const float *h, const __nv_bfloat16 *g, int d, float eps, __nv_bfloat16 *xhi,
-                                __nv_bfloat16 *xlo, int ldx) {
+// x = h / sqrt(mean(h^2) + eps) * g, as a bf16 pair.  With a deferred
+// product `add` (the attention output projection), h += that product first.
+__global__ void wide_norm_split(float *h, const __nv_bfloat16 *g, int d, float eps, __nv_bfloat16 *xhi,
+                                __nv_bfloat16 *xlo, int ldx, Split add) {
   __shared__ float red[32];
   const int m = blockIdx.x;
-  const float *row = h + static_cast<long long>(m) * d;
+  float *row = h + static_cast<long long>(m) * d;
   float s = 0.f;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) s = fmaf(row[c], row[c], s);
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float x = row[c];
+    if (add.ks > 1) {
+      x = x + split_sum(add, m, c);
+      row[c] = x;  // read back below by this same thread
+    }
+    s = fmaf(x, x, s);
+  }
   s = block_sum(s, red);
   const float inv = 1.0f / sqrtf(s / static_cast<float>(d) + eps);
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
@@ -371,11 +393,23 @@ __global__ void wide_norm_split(const float *h, const __nv_bfloat16 *g, int d, f
 }
 
 // Rotary embedding of k at each new row's position, k and v rounded to bf16
-// and written into the cache.  grid = (M, Hkv).
-__global__ void wide_kv_append(const float *qkv, int W3, const int32_t *positions, int T, int Hq, int Hkv, int hd,
+// and written into the cache.  grid = (M, Hkv).  With the QKV product's K
+// shares deferred, block (m, g) first finishes row m's q heads of group g
+// and its k and v heads in qkv.
+__global__ void wide_kv_append(float *qkv, int W3, const int32_t *positions, int T, int Hq, int Hkv, int hd,
                                const float2 *rope, __nv_bfloat16 *kc, __nv_bfloat16 *vc, int Bmax, int cap,
-                               int layer) {
+                               int layer, Split sp) {
   const int m = blockIdx.x, g = blockIdx.y, b = m / T, t = m % T;
+  if (sp.ks > 1) {
+    const int G = Hq / Hkv;
+    float *row = qkv + static_cast<long long>(m) * W3;
+    for (int i = threadIdx.x; i < (G + 2) * hd; i += blockDim.x) {
+      const int col = i < G * hd ? g * G * hd + i : i < (G + 1) * hd ? (Hq + g) * hd + i - G * hd
+                                                                     : (Hq + Hkv + g) * hd + i - (G + 1) * hd;
+      row[col] = split_sum(sp, m, col);
+    }
+    __syncthreads();
+  }
   const int p = positions[b] + t, half = hd / 2;
   const float *k = qkv + static_cast<long long>(m) * W3 + (Hq + g) * hd;
   const float *v = qkv + static_cast<long long>(m) * W3 + (Hq + Hkv + g) * hd;
@@ -701,14 +735,23 @@ __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv
 // Per row: softmax over the E router logits, top-k (ties to the lower id),
 // weights renormalised by their sum.  One warp per row.
 __global__ void wide_topk(const float *logits, int E, int K, int32_t *sel_e, float *sel_w, int32_t *dbg_ids,
-                          float *dbg_w) {
+                          float *dbg_w, Split sp) {
   const int m = blockIdx.x, lane = threadIdx.x;
-  const float *z = logits + static_cast<long long>(m) * E;
+  float z[kMaxExperts / 32];  // lane's logits: expert lane + 32 i (from the split-K buffer when deferred)
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i) {
+    const int e = lane + 32 * i;
+    z[i] = e < E ? (sp.ks > 1 ? split_sum(sp, m, e) : logits[static_cast<long long>(m) * E + e]) : 0.f;
+  }
   float mx = -INFINITY;
-  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, z[e]);
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i)
+    if (lane + 32 * i < E) mx = fmaxf(mx, z[i]);
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float sum = 0.f;
-  for (int e = lane; e < E; e += 32) sum += expf(z[e] - mx);
+#pragma unroll
+  for (int i = 0; i < kMaxExperts / 32; ++i)
+    if (lane + 32 * i < E) sum += expf(z[i] - mx);
   for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   uint32_t taken[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // bit e of expert e (E <= 256)
   float sel = 0.f, my_w = 0.f;
@@ -716,9 +759,11 @@ __global__ void wide_topk(const float *logits, int E, int K, int32_t *sel_e, flo
   for (int j = 0; j < K; ++j) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) {
-      if ((taken[e >> 5] >> (e & 31)) & 1u) continue;
-      const float pe = expf(z[e] - mx) / sum;
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const int e = lane + 32 * i;
+      if (e >= E || ((taken[e >> 5] >> (e & 31)) & 1u)) continue;
+      const float pe = expf(z[i] - mx) / sum;
       if (pe > bv || (pe == bv && e < bi)) {
         bv = pe;
         bi = e;
@@ -802,26 +847,30 @@ __global__ void wide_route_gather(const int32_t *sel_e, int M, int K, int E, con
   }
 }
 
-// act = silu(gate) * up for rows [rows][2F] (gate then up), as a bf16 pair
-__global__ void wide_swiglu(const float *gu, int F, __nv_bfloat16 *ahi, __nv_bfloat16 *alo, int lda) {
+// act = silu(gate) * up for rows [rows][2F] (gate then up), as a bf16 pair;
+// gate and up come from the split-K buffer when deferred.
+__global__ void wide_swiglu(const float *gu, int F, __nv_bfloat16 *ahi, __nv_bfloat16 *alo, int lda, Split sp) {
   const int q = blockIdx.x;
   for (int c = threadIdx.x; c < F; c += blockDim.x) {
-    const float gt = gu[static_cast<long long>(q) * 2 * F + c], up = gu[static_cast<long long>(q) * 2 * F + F + c];
+    const float gt = sp.ks > 1 ? split_sum(sp, q, c) : gu[static_cast<long long>(q) * 2 * F + c];
+    const float up = sp.ks > 1 ? split_sum(sp, q, F + c) : gu[static_cast<long long>(q) * 2 * F + F + c];
     split_store(gt / (1.0f + expf(-gt)) * up, ahi + static_cast<long long>(q) * lda + c,
                 alo + static_cast<long long>(q) * lda + c);
   }
 }
 
 // h[m] += sum_j w[m][j] y[pair(m, j)] (selection order) + shared[m]
-// grid = (rows, ceil(d / blockDim)): one column per thread.
+// grid = (rows, ceil(d / blockDim)): one column per thread.  The shared
+// expert's output comes from the split-K buffer when deferred.
 __global__ void wide_combine(float *h, int d, int K, const float *sel_w, const int *pair_slot, const float *y,
-                             const float *ys, float *dbg) {
+                             const float *ys, float *dbg, Split sp) {
   const int m = blockIdx.x;
   for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < d; c += gridDim.y * blockDim.x) {
     float moe = 0.f;
     for (int j = 0; j < K; ++j)
       moe = fmaf(sel_w[m * K + j], y[static_cast<long long>(pair_slot[m * K + j]) * d + c], moe);
-    const float v = h[static_cast<long long>(m) * d + c] + (ys ? moe + ys[static_cast<long long>(m) * d + c] : moe);
+    const float sh = ys ? (sp.ks > 1 ? split_sum(sp, m, c) : ys[static_cast<long long>(m) * d + c]) : 0.f;
+    const float v = h[static_cast<long long>(m) * d + c] + (ys ? moe + sh : moe);
     h[static_cast<long long>(m) * d + c] = v;
     if (dbg) dbg[static_cast<long long>(m) * d + c] = v;
   }
@@ -915,11 +964,13 @@ int gemm_smem_bytes() { return kTcStages * kTcStage + 1024; }  // + room to alig
 // One product (or one grouped launch of per-expert products) on the tensor
 // cores: weight rows [p * N, (p + 1) * N) x K for problem p, activation rows
 // of the xrows-row buffers xhi / xlo (row stride ldx).  A single dense problem
-// whose 128-row tiles do not fill the GPU splits K, through `part`.
+// whose 128-row tiles do not fill the GPU splits K, through `part`; with
+// `defer` the shares stay there for the consumer to add (no finish launch),
+// which must run before the next product that splits K.
 static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const __nv_bfloat16 *W2, int pe, int N,
                         int K, const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, int xrows,
                         const int *row_off, const int *row_cnt, int R, float *Y, int ldy, int ycol2, int accumulate,
-                        float *part, cudaStream_t st) {
+                        float *part, cudaStream_t st, Split *defer = nullptr) {
   GemmArgs a{};
   const int problems = W2 ? 2 * pe : pe;
   if (encode_2d_sw128(&a.mw, W, static_cast<uint64_t>(pe) * N, K, K, kTcM) != MK_OK ||
@@ -953,7 +1004,8 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const
   wide_gemm<<<std::min(a.units, s.n_sm), kTcThreads, gemm_smem_bytes(), st>>>(a);
   WIDE_TRY(cudaGetLastError());
   ++n;
-  if (ksplit > 1) {
+  if (defer) *defer = Split{part, ksplit > 1 ? ksplit : 0, R, ldy};
+  if (ksplit > 1 && !defer) {
     wide_gemm_finish<<<2 * s.n_sm, 256, 0, st>>>(part, ksplit, R, W2 ? ycol2 + N : N, ldy, Y, accumulate);
     WIDE_TRY(cudaGetLastError());
     ++n;
@@ -981,15 +1033,18 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
   ++n;
   for (int l = 0; l < L; ++l) {
     const mk_layer_weights &lw = s.layers[l];
+    // Products that split K leave their shares in s.part for the next kernel
+    // to add (Split), so each is consumed before the next such product.
     // attention block
     wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.attn_norm), d, s.eps, s.xhi,
-                                       s.xlo, ldx);
+                                       s.xlo, ldx, Split{});
     WIDE_TRY(cudaGetLastError());
     ++n;
+    Split sq{};
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wqkv), nullptr, 1, W3, d, s.xhi, s.xlo, ldx, M, nullptr,
-                  nullptr, M, s.qkv, W3, 0, 0, s.part, st));
+                  nullptr, M, s.qkv, W3, 0, 0, s.part, st, &sq));
     wide_kv_append<<<dim3(M, s.Hkv), 128, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, s.rope, s.kc,
-                                                   s.vc, s.Bmax, s.cap, l);
+                                                   s.vc, s.Bmax, s.cap, l, sq);
     WIDE_TRY(cudaGetLastError());
     ++n;
     {  // attention: chunk partials on the tensor cores, then the merge into the bf16 pair
@@ -1026,30 +1081,36 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       WIDE_TRY(cudaGetLastError());
       ++n;
     }
+    Split so{};
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), nullptr, 1, d, HD, s.xhi, s.xlo, ldx, M, nullptr,
-                  nullptr, M, s.h, d, 0, 1, s.part, st));
-    // MoE block: router on the normed row, top-k, expert lists
+                  nullptr, M, s.h, d, 0, 1, s.part, st, &so));
+    // MoE block: h += the output projection, norm; router, top-k
     wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.ffn_norm), d, s.eps, s.xhi, s.xlo,
-                                       ldx);
+                                       ldx, so);
     WIDE_TRY(cudaGetLastError());
     ++n;
-    // shared expert on every row (gate and up in one launch)
+    Split sr{};
+    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), nullptr, 1, E, d, s.xhi, s.xlo, ldx, M, nullptr,
+                  nullptr, M, s.rlog, E, 0, 0, s.part, st, &sr));
+    int32_t *dbg_ids = s.dbg_ids ? s.dbg_ids + static_cast<long long>(l) * s.max_rows * K : nullptr;
+    float *dbg_w = s.dbg_w ? s.dbg_w + static_cast<long long>(l) * s.max_rows * K : nullptr;
+    wide_topk<<<M, 32, 0, st>>>(s.rlog, E, K, s.sel_e, s.sel_w, dbg_ids, dbg_w, sr);
+    WIDE_TRY(cudaGetLastError());
+    ++n;
+    // shared expert on every row (gate and up in one launch); its down
+    // product's shares are added by the combine (the routed products below
+    // do not split K, so they leave s.part alone)
+    Split sd{};
     if (Fs > 0) {
+      Split sg{};
       WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_gate), static_cast<const __nv_bfloat16 *>(lw.ws_up),
-                    1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.gs, 2 * Fs, Fs, 0, s.part, st));
-      wide_swiglu<<<M, 256, 0, st>>>(s.gs, Fs, s.shi, s.slo, s.lda);
+                    1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.gs, 2 * Fs, Fs, 0, s.part, st, &sg));
+      wide_swiglu<<<M, 256, 0, st>>>(s.gs, Fs, s.shi, s.slo, s.lda, sg);
       WIDE_TRY(cudaGetLastError());
       ++n;
       WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), nullptr, 1, d, Fs, s.shi, s.slo, s.lda, M,
-                    nullptr, nullptr, M, s.ys, d, 0, 0, s.part, st));
+                    nullptr, nullptr, M, s.ys, d, 0, 0, s.part, st, &sd));
     }
-    WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), nullptr, 1, E, d, s.xhi, s.xlo, ldx, M, nullptr,
-                  nullptr, M, s.rlog, E, 0, 0, s.part, st));
-    int32_t *dbg_ids = s.dbg_ids ? s.dbg_ids + static_cast<long long>(l) * s.max_rows * K : nullptr;
-    float *dbg_w = s.dbg_w ? s.dbg_w + static_cast<long long>(l) * s.max_rows * K : nullptr;
-    wide_topk<<<M, 32, 0, st>>>(s.rlog, E, K, s.sel_e, s.sel_w, dbg_ids, dbg_w);
-    WIDE_TRY(cudaGetLastError());
-    ++n;
     // routed experts: expert lists + gather, gate and up over each expert's rows, SwiGLU, down
     wide_route_gather<<<M * K, 256, 0, st>>>(s.sel_e, M, K, E, s.xhi, s.xlo, ldx, d, s.count, s.off, s.pair_row,
                                              s.pair_slot, s.stats, s.ghi, s.glo);
@@ -1057,18 +1118,19 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), static_cast<const __nv_bfloat16 *>(lw.w_up), E, F,
                   d, s.ghi, s.glo, ldx, M * K, s.off, s.count, M * K, s.gu, 2 * F, F, 0, s.part, st));
-    wide_swiglu<<<M * K, 256, 0, st>>>(s.gu, F, s.ahi, s.alo, s.lda);
+    wide_swiglu<<<M * K, 256, 0, st>>>(s.gu, F, s.ahi, s.alo, s.lda, Split{});
     WIDE_TRY(cudaGetLastError());
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), nullptr, E, d, F, s.ahi, s.alo, s.lda, M * K,
                   s.off, s.count, M * K, s.yd, d, 0, 0, s.part, st));
     float *dbg = s.dbg_hidden ? s.dbg_hidden + static_cast<long long>(l + 1) * s.max_rows * d : nullptr;
-    wide_combine<<<dim3(M, (d + 255) / 256), 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr, dbg);
+    wide_combine<<<dim3(M, (d + 255) / 256), 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr,
+                                                           dbg, sd);
     WIDE_TRY(cudaGetLastError());
     ++n;
   }
   // final norm, lm_head, argmax
-  wide_norm_split<<<M, 256, 0, st>>>(s.h, s.final_norm, d, s.eps, s.xhi, s.xlo, ldx);
+  wide_norm_split<<<M, 256, 0, st>>>(s.h, s.final_norm, d, s.eps, s.xhi, s.xlo, ldx, Split{});
   WIDE_TRY(cudaGetLastError());
   ++n;
   WIDE_TRY(gemm(n, s, s.lm_head, nullptr, 1, s.V, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.logits, s.V, 0, 0, s.part,
