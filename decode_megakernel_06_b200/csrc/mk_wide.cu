@@ -425,27 +425,31 @@ __global__ void wide_kv_append(float *qkv, int W3, const int32_t *positions, int
 
 // Attention of a wide block on the tensor cores, split over the KV positions.
 // One CTA per (chunk of kAcN cache positions, sequence x KV head, tile of up
-// to 128 query vectors) scores the group's query vectors (T rows x Hq/Hkv
-// heads, each seeing positions up to its own) against the chunk:
+// to kAcQ query vectors) scores the group's query vectors (T rows x Hq/Hkv
+// heads, each seeing positions up to its own) against the chunk, with the
+// chunk's positions as the MMA's M and the query vectors as its N:
 //  - one thread brings the chunk's K rows by TMA (128B-swizzled, K-major: the
-//    B operand of S = Q K^T); every thread loads its share of the V rows into
-//    registers;
+//    A operand of S^T = K Q^T); every thread loads its share of the V rows and
+//    writes them transposed (V^T, K-major: the A operand of O^T = V^T P^T);
 //  - the rotated, scaled query vectors go into shared memory as a bf16 pair
-//    (q = hi + lo) in the same swizzled layout, the A operand (M = 128): query
-//    i of the tile in row 32 (i mod 4) + i / 4, so that each warp owns some;
-//  - S (128 x kAcN, fp32) accumulates Q_hi K^T + Q_lo K^T in tensor memory;
-//  - once S is complete, V is written transposed over the K rows (V^T is the
-//    K-major B operand of O = P V), and the thread owning a query's row of S
-//    masks the positions past the query's own and writes p = exp(s - max) as a
-//    bf16 pair over the query rows (the A operand of O = P V);
-//  - O (128 x hd) accumulates P_hi V + P_lo V; each thread writes its query's
-//    unnormalised partial output with the chunk's max and sum of p.
+//    (q = hi + lo), one row each (the B operand, N = kAcQ);
+//  - S^T (positions x queries, fp32) accumulates K Q_hi^T + K Q_lo^T in tensor
+//    memory; thread j reads position j's row, masks the queries that do not
+//    see position j, and the CTA reduces the max and then the sum of
+//    p = exp(s - max) over the positions of each query (a transposing shuffle
+//    reduction in each warp, then across the warps); p is written as a bf16
+//    pair, one row per query (the B operand of O^T);
+//  - O^T (hd x queries, fp32) accumulates V^T P_hi^T + V^T P_lo^T; thread d
+//    writes dim d of every query's unnormalised partial output, thread q the
+//    query's max and sum.
 // wide_attn_merge combines a query's chunks with the log-sum-exp rule.
 // ---------------------------------------------------------------------------
-constexpr int kAcN = 128;              // cache positions per chunk (N of S, K of P V)
+constexpr int kAcN = 128;             // cache positions per chunk (M of S^T, K of O^T)
+constexpr int kAcQ = 32;              // query vectors per CTA (N of both products)
 constexpr int kAcThreads = 128;
-constexpr int kAcTmemCols = 256;       // S: kAcN columns, then O: hd columns
-constexpr int kAcAtom = 128 * 128;     // one swizzled operand block: 128 rows x 128 bytes
+constexpr int kAcTmemCols = 64;       // S^T: columns [0, 32), O^T: [32, 64)
+constexpr int kAcAtom = 128 * 128;    // a swizzled block of 128 rows x 128 bytes
+constexpr int kAcQAtom = kAcQ * 128;  // a swizzled block of kAcQ rows x 128 bytes
 
 struct AttnArgs {
   CUtensorMap mk;  // K cache as [L * Bmax * Hkv * cap][hd], box 64 x 128
@@ -460,9 +464,9 @@ struct AttnArgs {
   int *error;
 };
 
-// dynamic shared memory: Q (later P) in 4 blocks, K (later V^T) in hd / 64
-// blocks, + room to align them to 1024 bytes
-constexpr int attn_smem_bytes(int hd) { return (4 + hd / 64) * kAcAtom + 1024; }
+// dynamic shared memory: K (hd / 64 blocks), V^T (2 blocks), Q then P
+// (16 KB), + room to align them to 1024 bytes
+constexpr int attn_smem_bytes(int hd) { return (hd / 64 + 2) * kAcAtom + 4 * kAcQAtom + 1024; }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);  // .x at the lower address
@@ -479,18 +483,39 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 // byte offset of the 16-byte piece `piece` (0..7) of row r in a swizzled block
 __device__ __forceinline__ int sw_off(int r, int piece) { return r * 128 + ((piece ^ (r & 7)) << 4); }
 
+// Reduces each of the 32 values over the warp's lanes: afterwards v[0] of
+// lane l holds the reduction of value l (31 shuffles; v is overwritten).
+// Each step trades half of the values with the lane `o` away and combines.
+template <bool MAX>
+__device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = upper ? v[i] : v[i + o];
+      const float keep = upper ? v[i + o] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, o);
+      v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+
 template <int HD>
-__global__ void __launch_bounds__(kAcThreads, 2) wide_attn_tc(const __grid_constant__ AttnArgs a) {
+__global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant__ AttnArgs a) {
   constexpr int NA = HD / 64, HALF = HD / 2;
   constexpr int NU = 64 * (HD / 8) / kAcThreads;  // (position pair, 8 dims) units of V per thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (sptr(smem_raw) & 1023u)) & 1023u);
-  uint8_t *sQ = smem;                // Q hi: NA blocks, Q lo: NA blocks; then P hi: 2 blocks, P lo: 2 blocks
-  uint8_t *sK = smem + 4 * kAcAtom;  // K: NA blocks of 128 positions; then V^T: 2 blocks of HD rows
+  uint8_t *sK = smem;                         // NA blocks: 128 positions x 64 dims
+  uint8_t *sVT = smem + NA * kAcAtom;         // 2 blocks: 128 dim rows (HD used) x 64 positions
+  uint8_t *sQ = sVT + 2 * kAcAtom;            // Q hi: NA blocks, Q lo: NA blocks; then P hi: 2, P lo: 2
   __shared__ __align__(8) uint64_t kbar, sbar, obar;
   __shared__ uint32_t tmem_base;
+  __shared__ __align__(16) float red[4][kAcQ], sM[kAcQ];
   const int c = blockIdx.x, bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv, G = a.Hq / a.Hkv;
-  const int Q = a.T * G, q0 = blockIdx.z * 128, nq = min(128, Q - q0);
+  const int Q = a.T * G, q0 = blockIdx.z * kAcQ, nq = min(kAcQ, Q - q0);
   const int pos0 = a.positions[b], last = pos0 + a.T - 1;
   const int j0 = c * kAcN;
   if (j0 > last || nq <= 0) return;  // the whole CTA, before anything is allocated
@@ -563,31 +588,44 @@ __global__ void __launch_bounds__(kAcThreads, 2) wide_attn_tc(const __grid_const
         y2h[e / 2] = pack_bf16(y2[0], y2[1]);
         y2l[e / 2] = pack_bf16(r2[0], r2[1]);
       }
-      const int r = 32 * (ql & 3) + (ql >> 2);
       const int d1 = 8 * cc, d2 = HALF + 8 * cc;
-      const int o1 = (d1 >> 6) * kAcAtom + sw_off(r, (d1 & 63) >> 3), o2 = (d2 >> 6) * kAcAtom + sw_off(r, (d2 & 63) >> 3);
+      const int o1 = (d1 >> 6) * kAcQAtom + sw_off(ql, (d1 & 63) >> 3),
+                o2 = (d2 >> 6) * kAcQAtom + sw_off(ql, (d2 & 63) >> 3);
       *reinterpret_cast<uint4 *>(sQ + o1) = make_uint4(y1h[0], y1h[1], y1h[2], y1h[3]);
-      *reinterpret_cast<uint4 *>(sQ + NA * kAcAtom + o1) = make_uint4(y1l[0], y1l[1], y1l[2], y1l[3]);
+      *reinterpret_cast<uint4 *>(sQ + NA * kAcQAtom + o1) = make_uint4(y1l[0], y1l[1], y1l[2], y1l[3]);
       *reinterpret_cast<uint4 *>(sQ + o2) = make_uint4(y2h[0], y2h[1], y2h[2], y2h[3]);
-      *reinterpret_cast<uint4 *>(sQ + NA * kAcAtom + o2) = make_uint4(y2l[0], y2l[1], y2l[2], y2l[3]);
+      *reinterpret_cast<uint4 *>(sQ + NA * kAcQAtom + o2) = make_uint4(y2l[0], y2l[1], y2l[2], y2l[3]);
+    }
+  }
+  // V^T: row d, positions 2 pp and 2 pp + 1 in one 32-bit word
+#pragma unroll
+  for (int i = 0; i < NU; ++i) {
+    const int u = threadIdx.x + kAcThreads * i, pp = u & 63, dc = u >> 6;
+    const uint32_t wa[4] = {va[i].x, va[i].y, va[i].z, va[i].w}, wb[4] = {vb[i].x, vb[i].y, vb[i].z, vb[i].w};
+    uint8_t *blk = sVT + (pp >> 5) * kAcAtom + (pp & 3) * 4;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int d = 8 * dc + e;
+      const uint32_t word = __byte_perm(wa[e >> 1], wb[e >> 1], (e & 1) ? 0x7632 : 0x5410);
+      *reinterpret_cast<uint32_t *>(blk + sw_off(d, (pp & 31) >> 2)) = word;
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
-  // kind::f16 instruction descriptors: fp32 accumulator, bf16 A and B, both K-major, M = 128
-  constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kAcN >> 3) << 17) | ((128 >> 4) << 24);
-  constexpr uint32_t kIdescO = (1u << 4) | (1u << 7) | (1u << 10) | ((HD >> 3) << 17) | ((128 >> 4) << 24);
+  // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
+  // K-major, N = kAcQ, M = 128 (both products)
+  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kAcQ >> 3) << 17) | ((128 >> 4) << 24);
   if (threadIdx.x == 0) {
     if (tc_wait(&kbar, 0, a.error)) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll
       for (int i = 0; i < NA; ++i) {
-        const uint64_t dqh = tc_desc(sQ + i * kAcAtom), dql = tc_desc(sQ + (NA + i) * kAcAtom),
-                       dk = tc_desc(sK + i * kAcAtom);
+        const uint64_t dk = tc_desc(sK + i * kAcAtom), dqh = tc_desc(sQ + i * kAcQAtom),
+                       dql = tc_desc(sQ + (NA + i) * kAcQAtom);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // 16 dims = 32 bytes = 2 descriptor units
-          tc_mma(tmem, dqh + 2 * kk, dk + 2 * kk, kIdescS, (i > 0 || kk > 0) ? 1u : 0u);
-          tc_mma(tmem, dql + 2 * kk, dk + 2 * kk, kIdescS, 1u);
+          tc_mma(tmem, dk + 2 * kk, dqh + 2 * kk, kIdesc, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem, dk + 2 * kk, dql + 2 * kk, kIdesc, 1u);
         }
       }
     }
@@ -596,98 +634,104 @@ __global__ void __launch_bounds__(kAcThreads, 2) wide_attn_tc(const __grid_const
   __syncwarp();
   bool ok = tc_wait(&sbar, 0, a.error);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  // V^T over the K rows: row d, positions 2 pp and 2 pp + 1 in one 32-bit word
+  // position j = this thread's accumulator lane: its scores for the kAcQ query vectors
+  const int j = threadIdx.x;
+  const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+  float sc[kAcQ];
+  {
+    uint32_t v0[16], v1[16];
+    tmem_ld16(tlane, v0);
+    tmem_ld16(tlane + 16, v1);
+    // query ql sees position j0 + j iff it exists and j0 + j <= pos0 + (q0 + ql) / G
+    const int dj = j0 + j - pos0;
 #pragma unroll
-  for (int i = 0; i < NU; ++i) {
-    const int u = threadIdx.x + kAcThreads * i, pp = u & 63, dc = u >> 6;
-    const uint32_t wa[4] = {va[i].x, va[i].y, va[i].z, va[i].w}, wb[4] = {vb[i].x, vb[i].y, vb[i].z, vb[i].w};
-    uint8_t *blk = sK + (pp >> 5) * (HD * 128) + (pp & 3) * 4;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int d = 8 * dc + e;
-      const uint32_t word = __byte_perm(wa[e >> 1], wb[e >> 1], (e & 1) ? 0x7632 : 0x5410);
-      *reinterpret_cast<uint32_t *>(blk + sw_off(d, (pp & 31) >> 2)) = word;
+    for (int ql = 0; ql < kAcQ; ++ql) {
+      const bool see = ql < nq && j < nj && (dj <= 0 || q0 + ql >= G * dj);
+      sc[ql] = see ? __uint_as_float(ql < 16 ? v0[ql] : v1[ql - 16]) : -INFINITY;
     }
   }
-  // this thread's query row of S: mask, max, p = exp(s - max) as a bf16 pair
-  const int r = threadIdx.x, ql = 4 * lane + warp, qi = q0 + ql;
-  const bool valid = ql < nq;
-  int nv = 0;  // positions of the chunk this query sees
-  if (valid) nv = max(0, min(nj, pos0 + qi / G - j0 + 1));
-  const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-  float mx = -INFINITY, l = 0.f;
-  for (int c0 = 0; c0 < kAcN; c0 += 16) {
-    uint32_t v[16];
-    tmem_ld16(trow + c0, v);
+  {
+    float t[kAcQ];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (c0 + j < nv) mx = fmaxf(mx, __uint_as_float(v[j]));
+    for (int ql = 0; ql < kAcQ; ++ql) t[ql] = sc[ql];
+    red[warp][lane] = warp_transpose_reduce<true>(t, lane);
   }
-  for (int c0 = 0; c0 < kAcN; c0 += 16) {
-    uint32_t v[16];
-    tmem_ld16(trow + c0, v);
-    float pv[16], pr[16];
+  __syncthreads();
+  if (threadIdx.x < kAcQ)
+    sM[threadIdx.x] = fmaxf(fmaxf(red[0][threadIdx.x], red[1][threadIdx.x]), fmaxf(red[2][threadIdx.x], red[3][threadIdx.x]));
+  __syncthreads();
+  float pv[kAcQ];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      pv[j] = c0 + j < nv ? expf(__uint_as_float(v[j]) - mx) : 0.f;
-      l += pv[j];
-      pr[j] = pv[j] - __bfloat162float(__float2bfloat16_rn(pv[j]));
+  for (int q4 = 0; q4 < kAcQ / 4; ++q4) {
+    const float4 m4 = *reinterpret_cast<const float4 *>(&sM[4 * q4]);
+    const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int ql = 4 * q4 + k;
+      pv[ql] = sc[ql] == -INFINITY ? 0.f : expf(sc[ql] - mm[k]);
     }
+  }
+  // p^T as a bf16 pair: row ql, K index j (the Q rows are no longer read)
+  {
+    uint8_t *base = sQ + (j >> 6) * kAcQAtom + (j & 7) * 2;
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int col = c0 + 8 * hh;
-      const int off = (col >> 6) * kAcAtom + sw_off(r, (col & 63) >> 3);
-      const float *ph = pv + 8 * hh, *pl = pr + 8 * hh;
-      *reinterpret_cast<uint4 *>(sQ + off) =
-          make_uint4(pack_bf16(ph[0], ph[1]), pack_bf16(ph[2], ph[3]), pack_bf16(ph[4], ph[5]), pack_bf16(ph[6], ph[7]));
-      *reinterpret_cast<uint4 *>(sQ + 2 * kAcAtom + off) =
-          make_uint4(pack_bf16(pl[0], pl[1]), pack_bf16(pl[2], pl[3]), pack_bf16(pl[4], pl[5]), pack_bf16(pl[6], pl[7]));
+    for (int ql = 0; ql < kAcQ; ++ql) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(pv[ql]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(pv[ql] - __bfloat162float(hi));
+      const int off = sw_off(ql, (j & 63) >> 3);
+      *reinterpret_cast<__nv_bfloat16 *>(base + off) = hi;
+      *reinterpret_cast<__nv_bfloat16 *>(base + 2 * kAcQAtom + off) = lo;
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
+  __syncthreads();  // also: every warp has read red (the maxima) before it is reused below
   if (threadIdx.x == 0) {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (ok) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const uint64_t dph = tc_desc(sQ + i * kAcAtom), dpl = tc_desc(sQ + (2 + i) * kAcAtom),
-                       dv = tc_desc(sK + i * (HD * 128));
+        const uint64_t dv = tc_desc(sVT + i * kAcAtom), dph = tc_desc(sQ + i * kAcQAtom),
+                       dpl = tc_desc(sQ + (2 + i) * kAcQAtom);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // 16 positions per product
-          tc_mma(tmem + kAcN, dph + 2 * kk, dv + 2 * kk, kIdescO, (i > 0 || kk > 0) ? 1u : 0u);
-          tc_mma(tmem + kAcN, dpl + 2 * kk, dv + 2 * kk, kIdescO, 1u);
+          tc_mma(tmem + kAcQ, dv + 2 * kk, dph + 2 * kk, kIdesc, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem + kAcQ, dv + 2 * kk, dpl + 2 * kk, kIdesc, 1u);
         }
       }
     }
     tc_commit(&obar);
   }
+  // meanwhile: the sum of p over the positions of each query
+  red[warp][lane] = warp_transpose_reduce<false>(pv, lane);
+  __syncthreads();
   __syncwarp();
   ok = tc_wait(&obar, 0, a.error) && ok;
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const long long slot = (static_cast<long long>(bg) * a.nch_max + c) * Q + qi;
+  const long long slot0 = (static_cast<long long>(bg) * a.nch_max + c) * Q + q0;
+  {
+    // dim d = this thread's accumulator lane of O^T
+    uint32_t v0[16], v1[16];
+    tmem_ld16(tlane + kAcQ, v0);
+    tmem_ld16(tlane + kAcQ + 16, v1);
+    const int d = threadIdx.x;
+    if (d < HD) {
 #pragma unroll
-  for (int c0 = 0; c0 < HD; c0 += 16) {
-    uint32_t v[16];
-    tmem_ld16(trow + kAcN + c0, v);
-    if (valid) {
-      float4 *dst = reinterpret_cast<float4 *>(a.opart + slot * HD + c0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[i] = ok ? make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
-                                  __uint_as_float(v[4 * i + 3]))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int ql = 0; ql < kAcQ; ++ql)
+        if (ql < nq) a.opart[(slot0 + ql) * HD + d] = ok ? __uint_as_float(ql < 16 ? v0[ql] : v1[ql - 16]) : 0.f;
     }
   }
-  if (valid) {
-    a.mlpart[2 * slot] = mx;
-    a.mlpart[2 * slot + 1] = l;
+  if (threadIdx.x < nq) {
+    const int ql = threadIdx.x;
+    a.mlpart[2 * (slot0 + ql)] = sM[ql];
+    a.mlpart[2 * (slot0 + ql) + 1] = ((red[0][ql] + red[1][ql]) + red[2][ql]) + red[3][ql];
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0)
+  if (warp == 0) {
+    __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAcTmemCols) : "memory");
+  }
 }
 
 // Query (m, h)'s chunk partials combined with the log-sum-exp rule, written
@@ -1069,7 +1113,7 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       aa.opart = s.attn_o;
       aa.mlpart = s.attn_ml;
       aa.error = s.error;
-      const dim3 grid(nch, s.B * s.Hkv, (s.T * G + 127) / 128);
+      const dim3 grid(nch, s.B * s.Hkv, (s.T * G + kAcQ - 1) / kAcQ);
       if (s.hd == 64)
         wide_attn_tc<64><<<grid, kAcThreads, attn_smem_bytes(64), st>>>(aa);
       else
