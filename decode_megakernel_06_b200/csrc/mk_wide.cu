@@ -13,6 +13,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "mk_internal.h"
 
@@ -20,6 +21,15 @@ namespace mk {
 namespace {
 
 __device__ __forceinline__ uint32_t sptr(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+// Programmatic dependent launch.  pdl_wait() returns once the previous
+// kernel in the stream has completed and its writes are visible; every CTA of
+// every kernel here calls it before it reads what an earlier kernel wrote or
+// writes what an earlier kernel reads (and before it exits, so that each
+// kernel completes after its predecessor).  pdl_launch() lets the next
+// kernel's CTAs be scheduled (they then wait in their own pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // Y[r][n] (+)= sum_k W[n][k] * (xhi[r][k] + xlo[r][k]) on the 5th-generation
@@ -199,6 +209,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
   volatile int *abort = &abort_flag;
   if (warp == 0) {
     if (lane == 0) {  // TMA producer: every unit's stages through one ring
+      // A dense product's rows are known without the previous kernel, and no
+      // kernel writes weights: the first unit's first stages of weights go
+      // out before the wait (a grouped product's rows come from an earlier
+      // kernel, so it waits first).
+      int pre = 0;
+      if (!a.row_off) {
+        const TcUnit t = tc_unit(a, blockIdx.x, nkc);
+        if (t.R > 0) pre = min(t.nk, kTcStages);
+        for (int i = 0; i < pre; ++i) {
+          uint8_t *st = smem + i * kTcStage;
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&full[i])),
+                       "r"(kTcBoxes * (kTcWBox + 2 * t.G * kTcBoxBytes))
+                       : "memory");
+          for (int b = 0; b < kTcBoxes; ++b)
+            tc_tma(st + b * kTcWBox, t.mw, ((t.kc0 + i) * kTcBoxes + b) * kTcK, t.wrow, &full[i]);
+        }
+      }
+      pdl_wait();
+      pdl_launch();
       int it = 0;
       for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
         const TcUnit t = tc_unit(a, u, nkc);
@@ -207,12 +236,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
           const int s = it % kTcStages;
           if (it >= kTcStages && !tc_wait_or_abort(&empty[s], ((it / kTcStages) & 1) ^ 1, a.error, abort)) break;
           uint8_t *st = smem + s * kTcStage;
-          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&full[s])),
-                       "r"(kTcBoxes * (kTcWBox + 2 * t.G * kTcBoxBytes))
-                       : "memory");
+          const bool weights_out = it < pre;  // sent before the wait, with the stage's byte count
+          if (!weights_out)
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sptr(&full[s])),
+                         "r"(kTcBoxes * (kTcWBox + 2 * t.G * kTcBoxBytes))
+                         : "memory");
           for (int b = 0; b < kTcBoxes; ++b) {  // columns past K read as zeros
             const int x = ((t.kc0 + i) * kTcBoxes + b) * kTcK;
-            tc_tma(st + b * kTcWBox, t.mw, x, t.wrow, &full[s]);
+            if (!weights_out) tc_tma(st + b * kTcWBox, t.mw, x, t.wrow, &full[s]);
             for (int g = 0; g < t.G; ++g) {
               tc_tma(st + kTcA + b * kTcXBox + g * kTcBoxBytes, &a.mxh, x, t.r0 + kTcRowBox * g, &full[s]);
               tc_tma(st + kTcA + kTcB + b * kTcXBox + g * kTcBoxBytes, &a.mxl, x, t.r0 + kTcRowBox * g, &full[s]);
@@ -222,6 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       }
     }
   } else if (warp == 1) {
+    pdl_wait();
     if (lane == 0) {  // MMA issuer
       int it = 0, lu = 0;
       for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x, ++lu) {
@@ -265,6 +297,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       }
     }
   } else {  // epilogue: warp w reads accumulator lanes 32 (w mod 4) ..
+    pdl_wait();
     const int q = warp & 3;
     int lu = 0;
     for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
@@ -312,6 +345,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
 
 // Y[r][n] (+)= sum over ks of part[ks][r][n], in order.
 __global__ void wide_gemm_finish(const float *part, int ksplit, int rows, int N, int ld, float *Y, int accumulate) {
+  pdl_wait();
+  pdl_launch();
   const long long total = static_cast<long long>(rows) * N;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -359,6 +394,8 @@ __device__ __forceinline__ float split_sum(const Split &p, int r, int col) {
 
 // h[m] = embed[token[m]]; the debug copy of the layer-0 input.
 __global__ void wide_embed(const int32_t *tokens, const __nv_bfloat16 *embed, int d, float *h, float *dbg) {
+  pdl_wait();
+  pdl_launch();
   const int m = blockIdx.x;
   const int tok = tokens[m];
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
@@ -372,6 +409,8 @@ __global__ void wide_embed(const int32_t *tokens, const __nv_bfloat16 *embed, in
 // product `add` (the attention output projection), h += that product first.
 __global__ void wide_norm_split(float *h, const __nv_bfloat16 *g, int d, float eps, __nv_bfloat16 *xhi,
                                 __nv_bfloat16 *xlo, int ldx, Split add) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float red[32];
   const int m = blockIdx.x;
   float *row = h + static_cast<long long>(m) * d;
@@ -399,6 +438,8 @@ __global__ void wide_norm_split(float *h, const __nv_bfloat16 *g, int d, float e
 __global__ void wide_kv_append(float *qkv, int W3, const int32_t *positions, int T, int Hq, int Hkv, int hd,
                                const float2 *rope, __nv_bfloat16 *kc, __nv_bfloat16 *vc, int Bmax, int cap,
                                int layer, Split sp) {
+  pdl_wait();
+  pdl_launch();
   const int m = blockIdx.x, g = blockIdx.y, b = m / T, t = m % T;
   if (sp.ks > 1) {
     const int G = Hq / Hkv;
@@ -504,6 +545,8 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane)
 
 template <int HD>
 __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant__ AttnArgs a) {
+  pdl_wait();
+  pdl_launch();
   constexpr int NA = HD / 64, HALF = HD / 2;
   constexpr int NU = 64 * (HD / 8) / kAcThreads;  // (position pair, 8 dims) units of V per thread
   extern __shared__ uint8_t smem_raw[];
@@ -742,6 +785,8 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
 __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv, int hd, int nch_max,
                                 const float *opart, const float *mlpart, __nv_bfloat16 *xhi, __nv_bfloat16 *xlo,
                                 int ldx) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float s_md[2];
   const int m = blockIdx.x, h = blockIdx.y, b = m / T, t = m % T, G = Hq / Hkv, g = h / G;
   const int Q = T * G, qi = t * G + h % G, bg = b * Hkv + g;
@@ -780,6 +825,8 @@ __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv
 // weights renormalised by their sum.  One warp per row.
 __global__ void wide_topk(const float *logits, int E, int K, int32_t *sel_e, float *sel_w, int32_t *dbg_ids,
                           float *dbg_w, Split sp) {
+  pdl_wait();
+  pdl_launch();
   const int m = blockIdx.x, lane = threadIdx.x;
   float z[kMaxExperts / 32];  // lane's logits: expert lane + 32 i (from the split-K buffer when deferred)
 #pragma unroll
@@ -846,6 +893,8 @@ __global__ void wide_topk(const float *logits, int E, int K, int32_t *sel_e, flo
 __global__ void wide_route_gather(const int32_t *sel_e, int M, int K, int E, const __nv_bfloat16 *xhi,
                                   const __nv_bfloat16 *xlo, int ldx, int d, int *count, int *off, int *pair_row,
                                   int *pair_slot, unsigned long long *stats, __nv_bfloat16 *ghi, __nv_bfloat16 *glo) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float red[32];
   __shared__ int s_q;
   const int i = blockIdx.x, MK = M * K, e = sel_e[i];
@@ -892,10 +941,13 @@ __global__ void wide_route_gather(const int32_t *sel_e, int M, int K, int E, con
 }
 
 // act = silu(gate) * up for rows [rows][2F] (gate then up), as a bf16 pair;
-// gate and up come from the split-K buffer when deferred.
+// gate and up come from the split-K buffer when deferred.  grid = (rows,
+// ceil(F / blockDim)).
 __global__ void wide_swiglu(const float *gu, int F, __nv_bfloat16 *ahi, __nv_bfloat16 *alo, int lda, Split sp) {
+  pdl_wait();
+  pdl_launch();
   const int q = blockIdx.x;
-  for (int c = threadIdx.x; c < F; c += blockDim.x) {
+  for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < F; c += gridDim.y * blockDim.x) {
     const float gt = sp.ks > 1 ? split_sum(sp, q, c) : gu[static_cast<long long>(q) * 2 * F + c];
     const float up = sp.ks > 1 ? split_sum(sp, q, F + c) : gu[static_cast<long long>(q) * 2 * F + F + c];
     split_store(gt / (1.0f + expf(-gt)) * up, ahi + static_cast<long long>(q) * lda + c,
@@ -908,6 +960,8 @@ __global__ void wide_swiglu(const float *gu, int F, __nv_bfloat16 *ahi, __nv_bfl
 // expert's output comes from the split-K buffer when deferred.
 __global__ void wide_combine(float *h, int d, int K, const float *sel_w, const int *pair_slot, const float *y,
                              const float *ys, float *dbg, Split sp) {
+  pdl_wait();
+  pdl_launch();
   const int m = blockIdx.x;
   for (int c = blockIdx.y * blockDim.x + threadIdx.x; c < d; c += gridDim.y * blockDim.x) {
     float moe = 0.f;
@@ -923,6 +977,8 @@ __global__ void wide_combine(float *h, int d, int K, const float *sel_w, const i
 // argmax over the vocabulary per row (ties to the lowest index)
 // One block per row; with V a multiple of 4 each thread reads 16-byte pieces.
 __global__ void __launch_bounds__(1024) wide_argmax(const float *logits, int V, int32_t *out) {
+  pdl_wait();
+  pdl_launch();
   __shared__ float bvs[32];
   __shared__ int bis[32];
   const int m = blockIdx.x;
@@ -978,6 +1034,8 @@ __global__ void __launch_bounds__(1024) wide_argmax(const float *logits, int V, 
 // access leaves its buffer, and the status marks the step's results invalid.
 __global__ void wide_check(const int32_t *tokens, const int32_t *positions, int B, int T, int V, int cap,
                            int32_t *tokens_safe, int32_t *positions_safe, int *error) {
+  pdl_wait();
+  pdl_launch();
   bool bad = false;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int p = positions[b];
@@ -999,6 +1057,26 @@ int gemm_smem_bytes() { return kTcStages * kTcStage + 1024; }  // + room to alig
 // ---------------------------------------------------------------------------
 // Host driver
 // ---------------------------------------------------------------------------
+// Every launch of the step may start while its predecessor in the stream
+// finishes (programmatic dependent launch, kept as such by graph capture);
+// each kernel waits for the predecessor with pdl_wait() before it touches
+// memory that kernels before it use.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 #define WIDE_TRY(x)                   \
   do {                                \
     cudaError_t e__ = (x);            \
@@ -1045,13 +1123,11 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const
   a.nb = nb;
   a.ksplit = ksplit;
   a.units = nb * ksplit * problems;
-  wide_gemm<<<std::min(a.units, s.n_sm), kTcThreads, gemm_smem_bytes(), st>>>(a);
-  WIDE_TRY(cudaGetLastError());
+  WIDE_TRY(launch(wide_gemm, dim3(std::min(a.units, s.n_sm)), dim3(kTcThreads), gemm_smem_bytes(), st, a));
   ++n;
   if (defer) *defer = Split{part, ksplit > 1 ? ksplit : 0, R, ldy};
   if (ksplit > 1 && !defer) {
-    wide_gemm_finish<<<2 * s.n_sm, 256, 0, st>>>(part, ksplit, R, W2 ? ycol2 + N : N, ldy, Y, accumulate);
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_gemm_finish, dim3(2 * s.n_sm), dim3(256), 0, st, part, ksplit, R, W2 ? ycol2 + N : N, ldy, Y, accumulate));
     ++n;
   }
   return cudaSuccess;
@@ -1068,28 +1144,24 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
   const int M = s.B * s.T, d = s.d, L = s.L, K = s.topk, E = s.E, F = s.F, Fs = s.Fs;
   const int W3 = (s.Hq + 2 * s.Hkv) * s.hd, HD = s.Hq * s.hd;
   const int ldx = s.ldx;  // >= max(d, HD), multiple of 8
-  wide_check<<<1, 256, 0, st>>>(s.tokens, s.positions, s.B, s.T, s.V, s.cap, s.tokens_safe, s.positions_safe,
-                                s.error);
-  WIDE_TRY(cudaGetLastError());
+  WIDE_TRY(launch(wide_check, dim3(1), dim3(256), 0, st, s.tokens, s.positions, s.B, s.T, s.V, s.cap, s.tokens_safe, s.positions_safe,
+                                s.error));
   ++n;
-  wide_embed<<<M, 256, 0, st>>>(s.tokens_safe, s.embed, d, s.h, s.dbg_hidden);
-  WIDE_TRY(cudaGetLastError());
+  WIDE_TRY(launch(wide_embed, dim3(M), dim3(256), 0, st, s.tokens_safe, s.embed, d, s.h, s.dbg_hidden));
   ++n;
   for (int l = 0; l < L; ++l) {
     const mk_layer_weights &lw = s.layers[l];
     // Products that split K leave their shares in s.part for the next kernel
     // to add (Split), so each is consumed before the next such product.
     // attention block
-    wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.attn_norm), d, s.eps, s.xhi,
-                                       s.xlo, ldx, Split{});
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_norm_split, dim3(M), dim3(1024), 0, st, s.h, static_cast<const __nv_bfloat16 *>(lw.attn_norm), d, s.eps, s.xhi,
+                                       s.xlo, ldx, Split{}));
     ++n;
     Split sq{};
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wqkv), nullptr, 1, W3, d, s.xhi, s.xlo, ldx, M, nullptr,
                   nullptr, M, s.qkv, W3, 0, 0, s.part, st, &sq));
-    wide_kv_append<<<dim3(M, s.Hkv), 128, 0, st>>>(s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, s.rope, s.kc,
-                                                   s.vc, s.Bmax, s.cap, l, sq);
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_kv_append, dim3(M, s.Hkv), dim3(256), 0, st, s.qkv, W3, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, s.rope, s.kc,
+                                                   s.vc, s.Bmax, s.cap, l, sq));
     ++n;
     {  // attention: chunk partials on the tensor cores, then the merge into the bf16 pair
       const int G = s.Hq / s.Hkv, nch = (s.cap + kAcN - 1) / kAcN;
@@ -1115,31 +1187,27 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       aa.error = s.error;
       const dim3 grid(nch, s.B * s.Hkv, (s.T * G + kAcQ - 1) / kAcQ);
       if (s.hd == 64)
-        wide_attn_tc<64><<<grid, kAcThreads, attn_smem_bytes(64), st>>>(aa);
+        WIDE_TRY(launch(wide_attn_tc<64>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(64), st, aa));
       else
-        wide_attn_tc<128><<<grid, kAcThreads, attn_smem_bytes(128), st>>>(aa);
-      WIDE_TRY(cudaGetLastError());
+        WIDE_TRY(launch(wide_attn_tc<128>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(128), st, aa));
       ++n;
-      wide_attn_merge<<<dim3(M, s.Hq), s.hd, 0, st>>>(s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
-                                                      s.attn_ml, s.xhi, s.xlo, ldx);
-      WIDE_TRY(cudaGetLastError());
+      WIDE_TRY(launch(wide_attn_merge, dim3(M, s.Hq), dim3(s.hd), 0, st, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
+                                                      s.attn_ml, s.xhi, s.xlo, ldx));
       ++n;
     }
     Split so{};
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.wo), nullptr, 1, d, HD, s.xhi, s.xlo, ldx, M, nullptr,
                   nullptr, M, s.h, d, 0, 1, s.part, st, &so));
     // MoE block: h += the output projection, norm; router, top-k
-    wide_norm_split<<<M, 256, 0, st>>>(s.h, static_cast<const __nv_bfloat16 *>(lw.ffn_norm), d, s.eps, s.xhi, s.xlo,
-                                       ldx, so);
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_norm_split, dim3(M), dim3(1024), 0, st, s.h, static_cast<const __nv_bfloat16 *>(lw.ffn_norm), d, s.eps, s.xhi, s.xlo,
+                                       ldx, so));
     ++n;
     Split sr{};
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.router), nullptr, 1, E, d, s.xhi, s.xlo, ldx, M, nullptr,
                   nullptr, M, s.rlog, E, 0, 0, s.part, st, &sr));
     int32_t *dbg_ids = s.dbg_ids ? s.dbg_ids + static_cast<long long>(l) * s.max_rows * K : nullptr;
     float *dbg_w = s.dbg_w ? s.dbg_w + static_cast<long long>(l) * s.max_rows * K : nullptr;
-    wide_topk<<<M, 32, 0, st>>>(s.rlog, E, K, s.sel_e, s.sel_w, dbg_ids, dbg_w, sr);
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_topk, dim3(M), dim3(32), 0, st, s.rlog, E, K, s.sel_e, s.sel_w, dbg_ids, dbg_w, sr));
     ++n;
     // shared expert on every row (gate and up in one launch); its down
     // product's shares are added by the combine (the routed products below
@@ -1149,38 +1217,32 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       Split sg{};
       WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_gate), static_cast<const __nv_bfloat16 *>(lw.ws_up),
                     1, Fs, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.gs, 2 * Fs, Fs, 0, s.part, st, &sg));
-      wide_swiglu<<<M, 256, 0, st>>>(s.gs, Fs, s.shi, s.slo, s.lda, sg);
-      WIDE_TRY(cudaGetLastError());
+      WIDE_TRY(launch(wide_swiglu, dim3(M, (Fs + 255) / 256), dim3(256), 0, st, s.gs, Fs, s.shi, s.slo, s.lda, sg));
       ++n;
       WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.ws_down), nullptr, 1, d, Fs, s.shi, s.slo, s.lda, M,
                     nullptr, nullptr, M, s.ys, d, 0, 0, s.part, st, &sd));
     }
     // routed experts: expert lists + gather, gate and up over each expert's rows, SwiGLU, down
-    wide_route_gather<<<M * K, 256, 0, st>>>(s.sel_e, M, K, E, s.xhi, s.xlo, ldx, d, s.count, s.off, s.pair_row,
-                                             s.pair_slot, s.stats, s.ghi, s.glo);
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_route_gather, dim3(M * K), dim3(256), 0, st, s.sel_e, M, K, E, s.xhi, s.xlo, ldx, d, s.count, s.off, s.pair_row,
+                                             s.pair_slot, s.stats, s.ghi, s.glo));
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), static_cast<const __nv_bfloat16 *>(lw.w_up), E, F,
                   d, s.ghi, s.glo, ldx, M * K, s.off, s.count, M * K, s.gu, 2 * F, F, 0, s.part, st));
-    wide_swiglu<<<M * K, 256, 0, st>>>(s.gu, F, s.ahi, s.alo, s.lda, Split{});
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_swiglu, dim3(M * K, (F + 255) / 256), dim3(256), 0, st, s.gu, F, s.ahi, s.alo, s.lda, Split{}));
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), nullptr, E, d, F, s.ahi, s.alo, s.lda, M * K,
                   s.off, s.count, M * K, s.yd, d, 0, 0, s.part, st));
     float *dbg = s.dbg_hidden ? s.dbg_hidden + static_cast<long long>(l + 1) * s.max_rows * d : nullptr;
-    wide_combine<<<dim3(M, (d + 255) / 256), 256, 0, st>>>(s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr,
-                                                           dbg, sd);
-    WIDE_TRY(cudaGetLastError());
+    WIDE_TRY(launch(wide_combine, dim3(M, (d + 255) / 256), dim3(256), 0, st, s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr,
+                                                           dbg, sd));
     ++n;
   }
   // final norm, lm_head, argmax
-  wide_norm_split<<<M, 256, 0, st>>>(s.h, s.final_norm, d, s.eps, s.xhi, s.xlo, ldx, Split{});
-  WIDE_TRY(cudaGetLastError());
+  WIDE_TRY(launch(wide_norm_split, dim3(M), dim3(1024), 0, st, s.h, s.final_norm, d, s.eps, s.xhi, s.xlo, ldx, Split{}));
   ++n;
   WIDE_TRY(gemm(n, s, s.lm_head, nullptr, 1, s.V, d, s.xhi, s.xlo, ldx, M, nullptr, nullptr, M, s.logits, s.V, 0, 0, s.part,
                 st));
-  wide_argmax<<<M, 1024, 0, st>>>(s.logits, s.V, s.argmax);
-  WIDE_TRY(cudaGetLastError());
+  WIDE_TRY(launch(wide_argmax, dim3(M), dim3(1024), 0, st, s.logits, s.V, s.argmax));
   if (launches) *launches = n + 1;
   return cudaSuccess;
 }
