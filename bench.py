@@ -581,17 +581,18 @@ def measure_verify_loop(device, n_steps=16, model=None, weights=None, seed=None,
             "drafter": "the model's greedy continuation with every 6th draft replaced"}
 
 
-def measure_verify_wide(device, steps=10, warmup=3, batch=8):
+def measure_verify_wide(device, steps=10, warmup=3, batch=8, model=None):
     """A speculative-verify block of 7 rows per sequence on the small model:
     8 sequences (56 rows, the wide-block tensor-core path) or 1 (7 rows, the
-    megakernel)."""
+    megakernel).  `model` names another synthetic model for the same block
+    (e.g. "small_profile", for profiler captures)."""
     import torch
 
     import decode_megakernel_06_b200 as mk
-    from synthetic import make_kv_cache, make_weights, workload
+    from synthetic import MODELS, make_kv_cache, make_weights, workload
 
     wl = workload("verify", batch)
-    m, B, T = wl.model, wl.batch, wl.tokens_per_step
+    m, B, T = (MODELS[model] if model else wl.model), wl.batch, wl.tokens_per_step
     w = make_weights(m, wl.seed, device)
     ctx = [wl.context] * B
     cap = (wl.context + (steps + warmup + 2) * T + 63) // 64 * 64
@@ -737,7 +738,10 @@ def run_mine(args):
         sweep = {}
         for bb in (1, 2, 4, 8):
             row = {}
-            for var in ("megakernel", "multikernel", "multikernel_graph"):
+            # MK_TENSORCORE: the tensor-core launch sequence for blocks of 2+ rows
+            variants = ("megakernel", "multikernel", "multikernel_graph") + (
+                ("tensorcore",) if bb >= 2 and m.n_experts > 0 else ())
+            for var in variants:
                 dec.set_variant(var)
                 n = max(5, min(args.steps, 20))
                 ctx_b = make_context_lengths(wl.__class__(wl.name, m, bb, T, wl.context,
@@ -896,7 +900,7 @@ def main():
                     choices=["large", "small", "tiny", "profile", "dense", "tiny_dense"])
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--variant", default="megakernel",
-                    choices=["megakernel", "multikernel", "multikernel_graph"])
+                    choices=["megakernel", "multikernel", "multikernel_graph", "tensorcore"])
     ap.add_argument("--sweep", action=argparse.BooleanOptionalAction, default=True)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-probe", action="store_true", help="skip the read-only HBM probe")

@@ -29,8 +29,9 @@ MK_ERR_UNSUPPORTED = -7
 MK_MEGAKERNEL = 0
 MK_MULTIKERNEL = 1
 MK_MULTIKERNEL_GRAPH = 2
+MK_TENSORCORE = 3
 VARIANTS = {"megakernel": MK_MEGAKERNEL, "multikernel": MK_MULTIKERNEL,
-            "multikernel_graph": MK_MULTIKERNEL_GRAPH}
+            "multikernel_graph": MK_MULTIKERNEL_GRAPH, "tensorcore": MK_TENSORCORE}
 
 MK_FAULT_NONE = 0
 MK_FAULT_UNREACHABLE_WAIT = 1

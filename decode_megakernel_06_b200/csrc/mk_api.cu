@@ -267,7 +267,7 @@ struct mk_handle {
   float *w_h, *w_qkv, *w_rlog, *w_selw, *w_gu, *w_yd, *w_gs, *w_ys, *w_part, *w_attn_o, *w_attn_ml;
   long long w_part_floats;
   int32_t *w_sele, *w_tok, *w_pos;
-  int *w_count, *w_off, *w_pair_row, *w_pair_slot;
+  int *w_count, *w_off, *w_pair_row, *w_pair_slot, *w_active;
   __nv_bfloat16 *w_xhi, *w_xlo, *w_ghi, *w_glo, *w_ahi, *w_alo, *w_shi, *w_slo;
 };
 
@@ -306,7 +306,7 @@ MK_API int mk_validate_desc(const mk_model_desc *d) {
   if (d->max_seqs < 1 || d->max_seqs > d->max_rows) return fail(MK_ERR_ARG, "max_seqs must be in [1, max_rows]");
   if (d->kv_capacity < 1) return fail(MK_ERR_ARG, "kv_capacity must be >= 1");
   if (!(d->rope_theta > 0.f) || !(d->rms_eps >= 0.f)) return fail(MK_ERR_ARG, "rope_theta > 0 and rms_eps >= 0 required");
-  if (d->variant < MK_MEGAKERNEL || d->variant > MK_MULTIKERNEL_GRAPH) return fail(MK_ERR_ARG, "unknown variant %d", d->variant);
+  if (d->variant < MK_MEGAKERNEL || d->variant > MK_TENSORCORE) return fail(MK_ERR_ARG, "unknown variant %d", d->variant);
   const long long kv_rows = (long long)d->n_layers * d->max_seqs * d->n_kv_heads * d->kv_capacity;
   if (kv_rows >= (1ll << 31)) return fail(MK_ERR_UNSUPPORTED, "KV cache too large");
   if ((long long)d->n_experts * d->expert_ffn >= (1ll << 31) || (long long)d->n_experts * d->d_model >= (1ll << 31))
@@ -472,7 +472,9 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     h->vbuf_ints = (cap / 2 + 1) * mr + (cap / 2 + 1) * mr + cap * mr;
     HALLOC(h->vbuf, sizeof(int32_t) * h->vbuf_ints);
   }
-  if (d.max_rows > kMaxRows) {  // buffers of the wide-block path
+  // buffers of the wide-block path: blocks above 8 rows, and MK_TENSORCORE
+  // blocks of 2 or more rows on a model with routed experts
+  if (d.max_rows > kMaxRows || (d.max_rows >= 2 && d.n_experts > 0)) {
     const int MR = d.max_rows, MK = MR * d.top_k, HD = d.n_q_heads * d.head_dim;
     const int ldx = ceil_div(std::max(D, HD), 8) * 8, lda = ceil_div(std::max(d.expert_ffn, std::max(d.shared_ffn, 1)), 8) * 8;
     const int Fs = std::max(d.shared_ffn, 1);
@@ -490,6 +492,7 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     HALLOC(h->w_sele, sizeof(int32_t) * (size_t)MK);
     HALLOC(h->w_count, sizeof(int) * (size_t)d.n_experts);
     HALLOC(h->w_off, sizeof(int) * (size_t)d.n_experts);
+    HALLOC(h->w_active, sizeof(int) * (size_t)(d.n_experts + 1));  // the list, then its length
     HALLOC(h->w_pair_row, sizeof(int) * (size_t)MK);
     HALLOC(h->w_pair_slot, sizeof(int) * (size_t)MK);
     HALLOC(h->w_tok, sizeof(int32_t) * (size_t)MR);
@@ -703,6 +706,7 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
   s.yd = h->w_yd; s.gs = h->w_gs; s.ys = h->w_ys; s.part = h->w_part; s.part_floats = h->w_part_floats;
   s.sel_e = h->w_sele; s.count = h->w_count; s.off = h->w_off; s.pair_row = h->w_pair_row;
   s.pair_slot = h->w_pair_slot;
+  s.active = h->w_active; s.n_active = h->w_active + d.n_experts;
   s.xhi = h->w_xhi; s.xlo = h->w_xlo; s.ghi = h->w_ghi; s.glo = h->w_glo; s.ahi = h->w_ahi; s.alo = h->w_alo;
   s.shi = h->w_shi; s.slo = h->w_slo;
   // The launch sequence is recorded once per (shape, buffers) into a CUDA graph
@@ -759,13 +763,16 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
 static int run_step(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T,
                     mk_kv_cache kv, float *logits, int32_t *argmax, cudaStream_t stream) {
   if (!h) return fail(MK_ERR_ARG, "handle is NULL");
-  if (B >= 1 && T >= 1 && (long long)B * T > kMaxRows) return run_wide(h, tokens, positions, B, T, kv, logits, argmax, stream);
+  if (B >= 1 && T >= 1 &&
+      ((long long)B * T > kMaxRows || (h->variant == MK_TENSORCORE && (long long)B * T >= 2 && h->desc.n_experts > 0)))
+    return run_wide(h, tokens, positions, B, T, kv, logits, argmax, stream);
   Params p;
   Plan pl;
   int rc = fill_params(h, tokens, positions, B, T, kv, logits, argmax, p, pl);
   if (rc) return rc;
   if (h->inject == MK_FAULT_UNREACHABLE_WAIT) p.inject_op = op_index(0, OP_ATTN);
   int variant = h->variant;
+  if (variant == MK_TENSORCORE) variant = MK_MEGAKERNEL;  // 1-row steps and dense models
   if (variant == MK_MULTIKERNEL_GRAPH && p.inject_op < 0) {
     uint64_t key[12] = {(uint64_t)B,
                         (uint64_t)T,
@@ -969,7 +976,7 @@ MK_API int mk_decode_step_host(mk_handle *h, const int32_t *tokens_host, const i
 
 MK_API int mk_set_variant(mk_handle *h, int32_t variant) {
   if (!h) return fail(MK_ERR_ARG, "handle is NULL");
-  if (variant < MK_MEGAKERNEL || variant > MK_MULTIKERNEL_GRAPH) return fail(MK_ERR_ARG, "unknown variant %d", variant);
+  if (variant < MK_MEGAKERNEL || variant > MK_TENSORCORE) return fail(MK_ERR_ARG, "unknown variant %d", variant);
   h->variant = variant;
   return MK_OK;
 }

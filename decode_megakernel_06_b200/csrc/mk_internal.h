@@ -211,6 +211,7 @@ struct WideStep {
   long long part_floats;
   int32_t *sel_e;
   int *count, *off, *pair_row, *pair_slot;
+  int *active, *n_active;  // experts with rows, in increasing order, and how many
   __nv_bfloat16 *xhi, *xlo, *ghi, *glo, *ahi, *alo, *shi, *slo;
 };
 

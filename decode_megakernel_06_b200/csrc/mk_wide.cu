@@ -80,6 +80,11 @@ struct GemmArgs {
   int pe;                  // problems per weight map; problem p >= pe is p - pe of mw2
   int ycol2;               // column of Y (and part) where the second product's outputs start
   int nb, ksplit, units;   // 128-row tiles per problem, K shares, nb * ksplit * problems
+  int halves;              // 2 when mw2 holds a second product, else 1
+  // grouped products: the problems that have rows, in increasing order, and
+  // how many (written by an earlier kernel); units then run over these only,
+  // so that every CTA gets an even share of the real work
+  const int *active, *n_active;
   const int *row_off, *row_cnt;
   int R;
   float *Y;
@@ -144,10 +149,10 @@ struct TcUnit {
   const CUtensorMap *mw;
   int wrow, r0, R, n0, kc0, nk, G, ycol, ks;
 };
-__device__ __forceinline__ TcUnit tc_unit(const GemmArgs &a, int u, int nkc) {
+__device__ __forceinline__ TcUnit tc_unit(const GemmArgs &a, int u, int nkc, int pe) {
   TcUnit t;
   const int tile = u % a.nb, ks = (u / a.nb) % a.ksplit, pz = u / (a.nb * a.ksplit);
-  const int half = pz >= a.pe, prob = pz - (half ? a.pe : 0);
+  const int half = pz >= pe, pi = pz - (half ? pe : 0), prob = a.active ? a.active[pi] : pi;
   t.mw = half ? &a.mw2 : &a.mw;
   t.r0 = a.row_off ? a.row_off[prob] : 0;
   t.R = a.row_off ? a.row_cnt[prob] : a.R;
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       // kernel, so it waits first).
       int pre = 0;
       if (!a.row_off) {
-        const TcUnit t = tc_unit(a, blockIdx.x, nkc);
+        const TcUnit t = tc_unit(a, blockIdx.x, nkc, a.pe);
         if (t.R > 0) pre = min(t.nk, kTcStages);
         for (int i = 0; i < pre; ++i) {
           uint8_t *st = smem + i * kTcStage;
@@ -228,9 +233,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
       }
       pdl_wait();
       pdl_launch();
+      const int pe = a.active ? *a.n_active : a.pe, units = a.active ? a.nb * a.ksplit * a.halves * pe : a.units;
       int it = 0;
-      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
-        const TcUnit t = tc_unit(a, u, nkc);
+      for (int u = blockIdx.x; u < units && !*abort; u += gridDim.x) {
+        const TcUnit t = tc_unit(a, u, nkc, pe);
         if (t.R <= 0) continue;
         for (int i = 0; i < t.nk; ++i, ++it) {
           const int s = it % kTcStages;
@@ -255,9 +261,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
   } else if (warp == 1) {
     pdl_wait();
     if (lane == 0) {  // MMA issuer
+      const int pe = a.active ? *a.n_active : a.pe, units = a.active ? a.nb * a.ksplit * a.halves * pe : a.units;
       int it = 0, lu = 0;
-      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x, ++lu) {
-        const TcUnit t = tc_unit(a, u, nkc);
+      for (int u = blockIdx.x; u < units && !*abort; u += gridDim.x, ++lu) {
+        const TcUnit t = tc_unit(a, u, nkc, pe);
         if (t.R <= 0) {
           --lu;
           continue;
@@ -299,9 +306,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) wide_gemm(const __grid_constant
   } else {  // epilogue: warp w reads accumulator lanes 32 (w mod 4) ..
     pdl_wait();
     const int q = warp & 3;
+    const int pe = a.active ? *a.n_active : a.pe, units = a.active ? a.nb * a.ksplit * a.halves * pe : a.units;
     int lu = 0;
-    for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
-      const TcUnit t = tc_unit(a, u, nkc);
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const TcUnit t = tc_unit(a, u, nkc, pe);
       if (t.R <= 0) continue;
       const int buf = lu & 1;
       const bool ok = __all_sync(0xffffffffu, tc_wait_or_abort(&accf[buf], (lu >> 1) & 1, a.error, abort));
@@ -888,11 +896,12 @@ __global__ void wide_topk(const float *logits, int E, int K, int32_t *sel_e, flo
 // order): its place is the number of pairs of a lower expert plus the earlier
 // pairs of its own expert (so the pairs of one expert keep (m, j) order), and
 // it copies row m of the bf16 pair to that place.  Block 0 also writes each
-// expert's count and first place and adds the number of experts in use to the
-// statistics.
+// expert's count and first place, the list of experts with rows, and adds
+// the number of experts in use to the statistics.
 __global__ void wide_route_gather(const int32_t *sel_e, int M, int K, int E, const __nv_bfloat16 *xhi,
                                   const __nv_bfloat16 *xlo, int ldx, int d, int *count, int *off, int *pair_row,
-                                  int *pair_slot, unsigned long long *stats, __nv_bfloat16 *ghi, __nv_bfloat16 *glo) {
+                                  int *pair_slot, unsigned long long *stats, __nv_bfloat16 *ghi, __nv_bfloat16 *glo,
+                                  int *active, int *n_active) {
   pdl_wait();
   pdl_launch();
   __shared__ float red[32];
@@ -911,6 +920,7 @@ __global__ void wide_route_gather(const int32_t *sel_e, int M, int K, int E, con
     pair_row[q] = i / K;
   }
   if (i == 0) {
+    __shared__ int s_cnt[kMaxExperts];
     unsigned long long used = 0;
     for (int x = threadIdx.x; x < E; x += blockDim.x) {
       int c = 0, o = 0;
@@ -921,9 +931,17 @@ __global__ void wide_route_gather(const int32_t *sel_e, int M, int K, int E, con
       }
       count[x] = c;
       off[x] = o;
+      s_cnt[x] = c;
       used += c > 0;
     }
     if (used) atomicAdd(stats, used);
+    __syncthreads();
+    if (threadIdx.x == 0) {  // the experts with rows, in increasing order
+      int na = 0;
+      for (int x = 0; x < E; ++x)
+        if (s_cnt[x] > 0) active[na++] = x;
+      *n_active = na;
+    }
   }
   __syncthreads();
   const long long src = static_cast<long long>(i / K) * ldx, dst = static_cast<long long>(s_q) * ldx;
@@ -1092,7 +1110,8 @@ static cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const __nv_bfloat16 *W2, int pe, int N,
                         int K, const __nv_bfloat16 *xhi, const __nv_bfloat16 *xlo, int ldx, int xrows,
                         const int *row_off, const int *row_cnt, int R, float *Y, int ldy, int ycol2, int accumulate,
-                        float *part, cudaStream_t st, Split *defer = nullptr) {
+                        float *part, cudaStream_t st, Split *defer = nullptr, const int *active = nullptr,
+                        const int *n_active = nullptr) {
   GemmArgs a{};
   const int problems = W2 ? 2 * pe : pe;
   if (encode_2d_sw128(&a.mw, W, static_cast<uint64_t>(pe) * N, K, K, kTcM) != MK_OK ||
@@ -1123,6 +1142,9 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const
   a.nb = nb;
   a.ksplit = ksplit;
   a.units = nb * ksplit * problems;
+  a.halves = W2 ? 2 : 1;
+  a.active = active;
+  a.n_active = active ? n_active : nullptr;
   WIDE_TRY(launch(wide_gemm, dim3(std::min(a.units, s.n_sm)), dim3(kTcThreads), gemm_smem_bytes(), st, a));
   ++n;
   if (defer) *defer = Split{part, ksplit > 1 ? ksplit : 0, R, ldy};
@@ -1224,14 +1246,15 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
     }
     // routed experts: expert lists + gather, gate and up over each expert's rows, SwiGLU, down
     WIDE_TRY(launch(wide_route_gather, dim3(M * K), dim3(256), 0, st, s.sel_e, M, K, E, s.xhi, s.xlo, ldx, d, s.count, s.off, s.pair_row,
-                                             s.pair_slot, s.stats, s.ghi, s.glo));
+                                             s.pair_slot, s.stats, s.ghi, s.glo, s.active, s.n_active));
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_gate), static_cast<const __nv_bfloat16 *>(lw.w_up), E, F,
-                  d, s.ghi, s.glo, ldx, M * K, s.off, s.count, M * K, s.gu, 2 * F, F, 0, s.part, st));
+                  d, s.ghi, s.glo, ldx, M * K, s.off, s.count, M * K, s.gu, 2 * F, F, 0, s.part, st, nullptr,
+                  s.active, s.n_active));
     WIDE_TRY(launch(wide_swiglu, dim3(M * K, (F + 255) / 256), dim3(256), 0, st, s.gu, F, s.ahi, s.alo, s.lda, Split{}));
     ++n;
     WIDE_TRY(gemm(n, s, static_cast<const __nv_bfloat16 *>(lw.w_down), nullptr, E, d, F, s.ahi, s.alo, s.lda, M * K,
-                  s.off, s.count, M * K, s.yd, d, 0, 0, s.part, st));
+                  s.off, s.count, M * K, s.yd, d, 0, 0, s.part, st, nullptr, s.active, s.n_active));
     float *dbg = s.dbg_hidden ? s.dbg_hidden + static_cast<long long>(l + 1) * s.max_rows * d : nullptr;
     WIDE_TRY(launch(wide_combine, dim3(M, (d + 255) / 256), dim3(256), 0, st, s.h, d, K, s.sel_w, s.pair_slot, s.yd, Fs > 0 ? s.ys : nullptr,
                                                            dbg, sd));

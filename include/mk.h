@@ -61,6 +61,10 @@ extern "C" {
 #define MK_MEGAKERNEL 0         /* one persistent cooperative launch per step    */
 #define MK_MULTIKERNEL 1        /* one launch per op, no cross-op prefetch       */
 #define MK_MULTIKERNEL_GRAPH 2  /* the per-op launches replayed from a CUDA graph */
+#define MK_TENSORCORE 3         /* blocks of 2 or more rows on the tensor-core     */
+                                /* launch sequence that blocks above 8 rows always */
+                                /* take (MoE models; 1-row steps, dense models and */
+                                /* the allocation-free entry stay on the megakernel) */
 
 /* ---- debug fault injection ---------------------------------------------------- */
 #define MK_FAULT_NONE 0
@@ -349,7 +353,10 @@ MK_API const char *mk_last_error(void);
 MK_API void mk_destroy(mk_handle *h);
 
 /* Switch the execution variant (MK_MEGAKERNEL, MK_MULTIKERNEL,
- * MK_MULTIKERNEL_GRAPH).  The math is identical across variants. */
+ * MK_MULTIKERNEL_GRAPH, MK_TENSORCORE).  The first three run the same math in
+ * the same order; MK_TENSORCORE computes the same step with tensor-core
+ * products (activations as a bf16 pair, about 2^-16 relative), so its results
+ * agree with the others within the parity tolerance, not bit for bit. */
 MK_API int mk_set_variant(mk_handle *h, int32_t variant);
 
 /* Bound for every device-side wait, in nanoseconds (default 1e9). */

@@ -84,6 +84,11 @@ LARGE = ModelConfig("large", 16, 4096, 32, 8, 128, 128, 8, 1536, 1536, 64000, si
 # weights): the same per-op shapes, small enough for a full profiler capture.
 PROFILE = ModelConfig("profile", 2, 4096, 32, 8, 128, 16, 8, 1536, 1536, 64000, sigma=0.015)
 
+# The small model's attention, dense and vocab shapes with 4 experts (under
+# 1 GB of weights): the wide-block path's kernels at their verify-block shapes,
+# small enough for a full profiler capture.
+SMALL_PROFILE = ModelConfig("small_profile", 8, 2048, 16, 4, 128, 4, 4, 1024, 1024, 32000)
+
 # Dense decoders (no router; one SwiGLU FFN per layer, held as the shared
 # expert): the tiny model's shapes, and the large model's attention, vocab and
 # a Llama-3-8B-sized FFN (about 7.5 GB read per step, like the large MoE's
@@ -91,7 +96,7 @@ PROFILE = ModelConfig("profile", 2, 4096, 32, 8, 128, 16, 8, 1536, 1536, 64000, 
 TINY_DENSE = ModelConfig("tiny_dense", 2, 256, 4, 2, 64, 0, 0, 16, 512, 1024)
 DENSE = ModelConfig("dense", 16, 4096, 32, 8, 128, 0, 0, 16, 14336, 64000, sigma=0.015)
 
-MODELS = {m.name: m for m in (TINY, SMALL, LARGE, PROFILE, TINY_DENSE, DENSE)}
+MODELS = {m.name: m for m in (TINY, SMALL, LARGE, PROFILE, SMALL_PROFILE, TINY_DENSE, DENSE)}
 
 
 def workload(kind: str, batch: int = 1) -> Workload:

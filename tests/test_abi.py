@@ -70,7 +70,7 @@ def test_validate_accepts_the_workload_models(L):
     ("shared_ffn", 8, mk.MK_ERR_ARG),
     ("max_rows", 65, mk.MK_ERR_UNSUPPORTED),
     ("max_seqs", 0, mk.MK_ERR_ARG),
-    ("variant", 3, mk.MK_ERR_ARG),
+    ("variant", 4, mk.MK_ERR_ARG),
     ("rope_theta", 0.0, mk.MK_ERR_ARG),
 ])
 def test_validate_rejects(L, field, value, code):

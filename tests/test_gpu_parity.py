@@ -105,6 +105,18 @@ def test_wide_block_more_query_vectors_than_one_tile():
     print(rep)
 
 
+@pytest.mark.parametrize("B,T", [(8, 1), (2, 3), (1, 2)])
+def test_tensorcore_variant_small_blocks(B, T):
+    """MK_TENSORCORE: blocks of 2 to 8 rows on the tensor-core launch sequence
+    (the ragged model), against the oracle."""
+    wl = Workload(f"ragged_tc_b{B}_t{T}", RAGGED, B, T, context=None, context_range=(1, 70), steps=3, seed=14)
+    s = Session(wl, variant="tensorcore", capacity=96)
+    rep = run_greedy(s, 2) if T == 1 else run_verify(s, 2)
+    s.close()
+    assert rep.rows_compared >= B * T
+    print(B, T, rep)
+
+
 def test_wide_block_rejects_bad_inputs_on_device():
     wl = Workload("ragged_wide_bad", RAGGED, 4, 4, context=None, context_range=(1, 40), steps=1, seed=12)
     s = Session(wl, capacity=64)
