@@ -478,8 +478,10 @@ __global__ void wide_kv_append(float *qkv, int W3, const int32_t *positions, int
 // heads, each seeing positions up to its own) against the chunk, with the
 // chunk's positions as the MMA's M and the query vectors as its N:
 //  - one thread brings the chunk's K rows by TMA (128B-swizzled, K-major: the
-//    A operand of S^T = K Q^T); every thread loads its share of the V rows and
-//    writes them transposed (V^T, K-major: the A operand of O^T = V^T P^T);
+//    A operand of S^T = K Q^T); every thread loads its share of the V rows,
+//    and once S^T is complete writes them transposed over the K rows (V^T,
+//    K-major: the A operand of O^T = V^T P^T), so that a CTA needs 49 KB of
+//    shared memory and four fit on an SM;
 //  - the rotated, scaled query vectors go into shared memory as a bf16 pair
 //    (q = hi + lo), one row each (the B operand, N = kAcQ);
 //  - S^T (positions x queries, fp32) accumulates K Q_hi^T + K Q_lo^T in tensor
@@ -513,9 +515,9 @@ struct AttnArgs {
   int *error;
 };
 
-// dynamic shared memory: K (hd / 64 blocks), V^T (2 blocks), Q then P
-// (16 KB), + room to align them to 1024 bytes
-constexpr int attn_smem_bytes(int hd) { return (hd / 64 + 2) * kAcAtom + 4 * kAcQAtom + 1024; }
+// dynamic shared memory: K then V^T (2 blocks), Q then P (16 KB), + room to
+// align them to 1024 bytes
+constexpr int attn_smem_bytes(int) { return 2 * kAcAtom + 4 * kAcQAtom + 1024; }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);  // .x at the lower address
@@ -559,9 +561,9 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
   constexpr int NU = 64 * (HD / 8) / kAcThreads;  // (position pair, 8 dims) units of V per thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (sptr(smem_raw) & 1023u)) & 1023u);
-  uint8_t *sK = smem;                         // NA blocks: 128 positions x 64 dims
-  uint8_t *sVT = smem + NA * kAcAtom;         // 2 blocks: 128 dim rows (HD used) x 64 positions
-  uint8_t *sQ = sVT + 2 * kAcAtom;            // Q hi: NA blocks, Q lo: NA blocks; then P hi: 2, P lo: 2
+  uint8_t *sK = smem;                         // NA blocks: 128 positions x 64 dims; then
+  uint8_t *sVT = smem;                        //   V^T, 2 blocks: 128 dim rows (HD used) x 64 positions
+  uint8_t *sQ = smem + 2 * kAcAtom;           // Q hi: NA blocks, Q lo: NA blocks; then P hi: 2, P lo: 2
   __shared__ __align__(8) uint64_t kbar, sbar, obar;
   __shared__ uint32_t tmem_base;
   __shared__ __align__(16) float red[4][kAcQ], sM[kAcQ];
@@ -648,19 +650,6 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
       *reinterpret_cast<uint4 *>(sQ + NA * kAcQAtom + o2) = make_uint4(y2l[0], y2l[1], y2l[2], y2l[3]);
     }
   }
-  // V^T: row d, positions 2 pp and 2 pp + 1 in one 32-bit word
-#pragma unroll
-  for (int i = 0; i < NU; ++i) {
-    const int u = threadIdx.x + kAcThreads * i, pp = u & 63, dc = u >> 6;
-    const uint32_t wa[4] = {va[i].x, va[i].y, va[i].z, va[i].w}, wb[4] = {vb[i].x, vb[i].y, vb[i].z, vb[i].w};
-    uint8_t *blk = sVT + (pp >> 5) * kAcAtom + (pp & 3) * 4;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int d = 8 * dc + e;
-      const uint32_t word = __byte_perm(wa[e >> 1], wb[e >> 1], (e & 1) ? 0x7632 : 0x5410);
-      *reinterpret_cast<uint32_t *>(blk + sw_off(d, (pp & 31) >> 2)) = word;
-    }
-  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
@@ -685,6 +674,20 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
   __syncwarp();
   bool ok = tc_wait(&sbar, 0, a.error);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  // V^T over the K rows (read by S^T, now complete): row d, positions 2 pp
+  // and 2 pp + 1 in one 32-bit word
+#pragma unroll
+  for (int i = 0; i < NU; ++i) {
+    const int u = threadIdx.x + kAcThreads * i, pp = u & 63, dc = u >> 6;
+    const uint32_t wa[4] = {va[i].x, va[i].y, va[i].z, va[i].w}, wb[4] = {vb[i].x, vb[i].y, vb[i].z, vb[i].w};
+    uint8_t *blk = sVT + (pp >> 5) * kAcAtom + (pp & 3) * 4;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int d = 8 * dc + e;
+      const uint32_t word = __byte_perm(wa[e >> 1], wb[e >> 1], (e & 1) ? 0x7632 : 0x5410);
+      *reinterpret_cast<uint32_t *>(blk + sw_off(d, (pp & 31) >> 2)) = word;
+    }
+  }
   // position j = this thread's accumulator lane: its scores for the kAcQ query vectors
   const int j = threadIdx.x;
   const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * warp) << 16);
