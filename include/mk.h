@@ -181,6 +181,9 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *weights, mk_ha
  *   out_logits : device fp32 [B*T][vocab], or NULL (kept in handle scratch)
  *   out_argmax : device int32 [B*T] (may alias tokens: read before written)
  *   stream     : cudaStream_t (NULL = legacy default stream)
+ * Blocks of up to 8 rows run the variant the handle is set to (with
+ * MK_TENSORCORE: the tensor-core launch sequence for 2 rows or more on a MoE
+ * model); blocks above 8 rows always run the tensor-core launch sequence.
  * Asynchronous.  Invalid token ids or positions are detected on the device:
  * the step stops and mk_get_device_status reports MK_ERR_DEVICE_CHECK. */
 MK_API int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *positions,

@@ -84,10 +84,10 @@ LARGE = ModelConfig("large", 16, 4096, 32, 8, 128, 128, 8, 1536, 1536, 64000, si
 # weights): the same per-op shapes, small enough for a full profiler capture.
 PROFILE = ModelConfig("profile", 2, 4096, 32, 8, 128, 16, 8, 1536, 1536, 64000, sigma=0.015)
 
-# The small model's attention, dense and vocab shapes with 4 experts (under
-# 1 GB of weights): the wide-block path's kernels at their verify-block shapes,
-# small enough for a full profiler capture.
-SMALL_PROFILE = ModelConfig("small_profile", 8, 2048, 16, 4, 128, 4, 4, 1024, 1024, 32000)
+# The small model's attention, dense and vocab shapes with 16 experts (about
+# 2.2 GB of weights): the wide-block path's kernels at their verify-block
+# shapes, small enough for a full profiler capture.
+SMALL_PROFILE = ModelConfig("small_profile", 8, 2048, 16, 4, 128, 16, 4, 1024, 1024, 32000)
 
 # Dense decoders (no router; one SwiGLU FFN per layer, held as the shared
 # expert): the tiny model's shapes, and the large model's attention, vocab and
