@@ -517,21 +517,22 @@ def measure_dense(device, steps=20, warmup=3):
             "launches_per_step": st.kernel_launches // steps}
 
 
-def measure_verify_loop(device, n_steps=16, model=None, weights=None, seed=None, context=None):
-    """Speculative verify on the device (mk_verify_steps): one sequence, blocks
-    of 7 rows (the last accepted token + 6 drafts), n_steps blocks in one
-    launch, on the small model (default) or on the given model and weights.
+def measure_verify_loop(device, n_steps=16, model=None, weights=None, seed=None, context=None, batch=1):
+    """Speculative verify on the device (mk_verify_steps): `batch` sequences,
+    blocks of 7 rows (the last accepted token + 6 drafts), n_steps blocks in
+    one call, on the small model (default) or on the given model and weights.
     The synthetic drafter proposes the model's own greedy continuation (taken
     from a greedy multi-step launch first) with every 6th draft replaced, so
-    that each block accepts 5 drafts plus one token: acceptance length 6.
-    Reports accepted tokens per second."""
+    that each block accepts 5 drafts plus one token: acceptance length 6 (a
+    near tie read differently by the tensor-core path above 8 rows can end a
+    block earlier).  Reports accepted tokens per second."""
     import torch
 
     import decode_megakernel_06_b200 as mk
     from synthetic import make_kv_cache, make_tokens, make_weights, workload
 
     wl = workload("verify", 1)
-    T = wl.tokens_per_step
+    T, B = wl.tokens_per_step, batch
     if model is None:
         m, seed, p0 = wl.model, wl.seed, wl.context
         w = make_weights(m, seed, device)
@@ -539,35 +540,37 @@ def measure_verify_loop(device, n_steps=16, model=None, weights=None, seed=None,
         m, w, p0 = model, weights, context
     acc_len = T - 1
     cap = (p0 + (n_steps + 2) * T + 64 + 63) // 64 * 64
-    k, v = make_kv_cache(m, 1, cap, seed, device)
-    dec = mk.Decoder(m, w, max_rows=T, max_seqs=1, kv_capacity=cap)
-    first = make_tokens(m.vocab, 1, 55)[0]
+    k, v = make_kv_cache(m, B, cap, seed, device)
+    dec = mk.Decoder(m, w, max_rows=B * T, max_seqs=B, kv_capacity=cap)
+    firsts = make_tokens(m.vocab, B, 55)
     ng = n_steps * acc_len + T
-    greedy = torch.empty((ng, 1), dtype=torch.int32, device=device)
-    assert dec.steps(torch.tensor([first], dtype=torch.int32, device=device),
-                     torch.tensor([p0], dtype=torch.int32, device=device), 1, ng, k, v, None, greedy) == 0
-    drafts = torch.empty((1, n_steps * T + T), dtype=torch.int32, device=device)
-    drafts[0, 0] = first
-    drafts[0, 1:ng + 1] = greedy[:, 0]
-    drafts[0, ng + 1:] = 0
+    greedy = torch.empty((ng, B), dtype=torch.int32, device=device)
+    assert dec.steps(torch.tensor(firsts, dtype=torch.int32, device=device),
+                     torch.tensor([p0] * B, dtype=torch.int32, device=device), B, ng, k, v, None, greedy) == 0
+    drafts = torch.empty((B, n_steps * T + T), dtype=torch.int32, device=device)
+    drafts[:, 0] = torch.tensor(firsts, dtype=torch.int32, device=device)
+    drafts[:, 1:ng + 1] = greedy.t()
+    drafts[:, ng + 1:] = 0
     for s in range(1, n_steps + 2):
         j = s * acc_len
         if j < drafts.shape[1]:
-            drafts[0, j] = (drafts[0, j] + 1) % m.vocab
-    blk = drafts[0, :T].clone()
-    pos = torch.tensor([p0], dtype=torch.int32, device=device)
-    out = torch.empty((n_steps, T), dtype=torch.int32, device=device)
-    acc = torch.empty((n_steps, 1), dtype=torch.int32, device=device)
+            drafts[:, j] = (drafts[:, j] + 1) % m.vocab
+    blk = drafts[:, :T].contiguous().view(-1).clone()
+    pos = torch.tensor([p0] * B, dtype=torch.int32, device=device)
+    out = torch.empty((n_steps, B * T), dtype=torch.int32, device=device)
+    acc = torch.empty((n_steps, B), dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream()
     for _ in range(2):
-        assert dec.verify_steps(blk, pos, 1, T, n_steps, drafts, k, v, None, out, acc) == 0
+        assert dec.verify_steps(blk, pos, B, T, n_steps, drafts, k, v, None, out, acc) == 0
     torch.cuda.synchronize()
+    dec.stats(reset=True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    assert dec.verify_steps(blk, pos, 1, T, n_steps, drafts, k, v, None, out, acc) == 0
+    assert dec.verify_steps(blk, pos, B, T, n_steps, drafts, k, v, None, out, acc) == 0
     e1.record(stream)
     torch.cuda.synchronize()
     assert dec.status() == 0
+    kernels = dec.stats(reset=True).kernel_launches
     ms = e0.elapsed_time(e1)
     accepted = int(acc.sum().item())
     dec.close()
@@ -575,9 +578,12 @@ def measure_verify_loop(device, n_steps=16, model=None, weights=None, seed=None,
     if model is None:
         del w
     torch.cuda.empty_cache()
-    return {"workload": f"verify_b1_t{T} ({m.name} model, context {p0}), {n_steps} blocks in one launch",
-            "accepted_tok_s": round(accepted / (ms / 1e3), 1), "mean_acceptance": round(accepted / n_steps, 2),
-            "ms_per_block": round(ms / n_steps, 4), "launches": 1,
+    path = ("one persistent megakernel launch" if B * T <= 8 else
+            "tensor-core launch sequence with acceptance on the device, one CUDA graph launch")
+    return {"workload": f"verify_b{B}_t{T} ({m.name} model, context {p0}), {n_steps} blocks in one call",
+            "accepted_tok_s": round(accepted / (ms / 1e3), 1),
+            "mean_acceptance": round(accepted / (n_steps * B), 2),
+            "ms_per_block": round(ms / n_steps, 4), "launches": 1, "kernels": int(kernels), "path": path,
             "drafter": "the model's greedy continuation with every 6th draft replaced"}
 
 
@@ -768,11 +774,12 @@ def run_mine(args):
     probe = measure_read_probe(device) if not args.no_probe else None
     probe_gbs = probe["gbs"] if probe else None
 
-    verify56 = vloop = vloop_large = dense = configs = None
+    verify56 = vloop = vloop_large = vloop56 = dense = configs = None
     if args.sweep and ws == 1 and args.workload == "large":
         verify56 = measure_verify_wide(device)
         vloop = measure_verify_loop(device)
         vloop_large = measure_verify_loop(device, model=m, weights=w, seed=wl.seed, context=wl.context)
+        vloop56 = measure_verify_loop(device, batch=8)
         dense = measure_dense(device)
         configs = measure_config_lines(device, peak, probe_gbs)
 
@@ -840,6 +847,8 @@ def run_mine(args):
             line["speculative"] = vloop
         if vloop_large is not None:
             line["speculative_large"] = vloop_large
+        if vloop56 is not None:
+            line["speculative_56"] = vloop56
         if dense is not None:
             line["dense"] = dense
         print(json.dumps(line), flush=True)

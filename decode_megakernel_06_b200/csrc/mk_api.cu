@@ -267,6 +267,7 @@ struct mk_handle {
   float *w_h, *w_qkv, *w_rlog, *w_selw, *w_gu, *w_yd, *w_gs, *w_ys, *w_part, *w_attn_o, *w_attn_ml;
   long long w_part_floats;
   int32_t *w_sele, *w_tok, *w_pos;
+  int32_t *w_vtok, *w_vpos, *w_vpos0, *w_vam;  // the wide verify loop: block, positions, start, argmax
   int *w_count, *w_off, *w_pair_row, *w_pair_slot, *w_active;
   __nv_bfloat16 *w_xhi, *w_xlo, *w_ghi, *w_glo, *w_ahi, *w_alo, *w_shi, *w_slo;
 };
@@ -497,6 +498,10 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
     HALLOC(h->w_pair_slot, sizeof(int) * (size_t)MK);
     HALLOC(h->w_tok, sizeof(int32_t) * (size_t)MR);
     HALLOC(h->w_pos, sizeof(int32_t) * (size_t)d.max_seqs);
+    HALLOC(h->w_vtok, sizeof(int32_t) * (size_t)MR);
+    HALLOC(h->w_vpos, sizeof(int32_t) * (size_t)d.max_seqs);
+    HALLOC(h->w_vpos0, sizeof(int32_t) * (size_t)d.max_seqs);
+    HALLOC(h->w_vam, sizeof(int32_t) * (size_t)MR);
     HALLOC(h->w_xhi, sizeof(__nv_bfloat16) * (size_t)MR * ldx);
     HALLOC(h->w_xlo, sizeof(__nv_bfloat16) * (size_t)MR * ldx);
     HALLOC(h->w_ghi, sizeof(__nv_bfloat16) * (size_t)MK * ldx);
@@ -674,15 +679,11 @@ static int launch_variant(mk_handle *h, Params &p, const Plan &pl, cudaStream_t 
 }
 
 // A block of more than kMaxRows rows: the launch sequence of mk_wide.cu.
-static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T, mk_kv_cache kv,
-                    float *logits, int32_t *argmax, cudaStream_t stream) {
+// The wide-block step's arguments: the handle's buffers and the call's.
+static void fill_wide(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T, mk_kv_cache kv,
+                      float *logits, int32_t *argmax, WideStep &s) {
   const mk_model_desc &d = h->desc;
-  if (!tokens || !positions || !argmax) return fail(MK_ERR_ARG, "tokens, positions and out_argmax are required");
-  if (!kv.k || !kv.v) return fail(MK_ERR_ARG, "kv.k and kv.v are required");
-  if (B > d.max_seqs || (long long)B * T > d.max_rows)
-    return fail(MK_ERR_CAPACITY, "B=%d T=%d exceeds max_seqs=%d / max_rows=%d", B, T, d.max_seqs, d.max_rows);
-  if (T > d.kv_capacity) return fail(MK_ERR_CAPACITY, "T=%d exceeds kv_capacity=%d", T, d.kv_capacity);
-  WideStep s{};
+  s = WideStep{};
   s.L = d.n_layers; s.d = d.d_model; s.Hq = d.n_q_heads; s.Hkv = d.n_kv_heads; s.hd = d.head_dim;
   s.E = d.n_experts; s.topk = d.top_k; s.F = d.expert_ffn; s.Fs = d.shared_ffn; s.V = d.vocab;
   s.Bmax = d.max_seqs; s.cap = d.kv_capacity; s.eps = d.rms_eps;
@@ -709,6 +710,18 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
   s.active = h->w_active; s.n_active = h->w_active + d.n_experts;
   s.xhi = h->w_xhi; s.xlo = h->w_xlo; s.ghi = h->w_ghi; s.glo = h->w_glo; s.ahi = h->w_ahi; s.alo = h->w_alo;
   s.shi = h->w_shi; s.slo = h->w_slo;
+}
+
+static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T, mk_kv_cache kv,
+                    float *logits, int32_t *argmax, cudaStream_t stream) {
+  const mk_model_desc &d = h->desc;
+  if (!tokens || !positions || !argmax) return fail(MK_ERR_ARG, "tokens, positions and out_argmax are required");
+  if (!kv.k || !kv.v) return fail(MK_ERR_ARG, "kv.k and kv.v are required");
+  if (B > d.max_seqs || (long long)B * T > d.max_rows)
+    return fail(MK_ERR_CAPACITY, "B=%d T=%d exceeds max_seqs=%d / max_rows=%d", B, T, d.max_seqs, d.max_rows);
+  if (T > d.kv_capacity) return fail(MK_ERR_CAPACITY, "T=%d exceeds kv_capacity=%d", T, d.kv_capacity);
+  WideStep s;
+  fill_wide(h, tokens, positions, B, T, kv, logits, argmax, s);
   // The launch sequence is recorded once per (shape, buffers) into a CUDA graph
   // and replayed: a graph launch issues the ~300 kernels without a host call
   // each.  Graphs live in the handle's cache next to the multi-kernel ones.
@@ -879,6 +892,80 @@ MK_API int mk_decode_step_sample(mk_handle *h, const int32_t *tokens, const int3
   return MK_OK;
 }
 
+// mk_verify_steps on the tensor-core launch sequence: the block and its
+// positions are copied into the handle, then n_steps x (wide step, then
+// acceptance on the device, which writes the next block in place) run as one
+// CUDA graph, recorded once per (shape, n_steps, buffers).
+static int run_wide_verify(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int T,
+                           int n_steps, const int32_t *drafts, int draft_len, mk_kv_cache kv, float *out_logits,
+                           int32_t *out_tokens, int32_t *out_accepted, cudaStream_t stream) {
+  const mk_model_desc &d = h->desc;
+  if (!tokens || !positions) return fail(MK_ERR_ARG, "tokens and positions are required");
+  if (!kv.k || !kv.v) return fail(MK_ERR_ARG, "kv.k and kv.v are required");
+  if (B < 1 || B > d.max_seqs || (long long)B * T > d.max_rows)
+    return fail(MK_ERR_CAPACITY, "B=%d T=%d exceeds max_seqs=%d / max_rows=%d", B, T, d.max_seqs, d.max_rows);
+  CUDA_TRY(cudaMemcpyAsync(h->w_vtok, tokens, sizeof(int32_t) * B * T, cudaMemcpyDeviceToDevice, stream));
+  CUDA_TRY(cudaMemcpyAsync(h->w_vpos, positions, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, stream));
+  CUDA_TRY(cudaMemcpyAsync(h->w_vpos0, positions, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, stream));
+  WideStep s;
+  fill_wide(h, h->w_vtok, h->w_vpos, B, T, kv, out_logits, h->w_vam, s);
+  const uint64_t key[12] = {(uint64_t)B | (0x56ull << 56),  // wide verify-loop entries
+                            (uint64_t)T | ((uint64_t)n_steps << 32),
+                            (uint64_t)(uintptr_t)drafts,
+                            (uint64_t)(uintptr_t)s.logits,
+                            (uint64_t)(uintptr_t)out_tokens,
+                            (uint64_t)(uintptr_t)out_accepted,
+                            (uint64_t)(uintptr_t)kv.k,
+                            (uint64_t)(uintptr_t)kv.v,
+                            (uint64_t)(uintptr_t)h->dbg_hidden,
+                            (uint64_t)(uintptr_t)h->dbg_ids ^ (uint64_t)(uintptr_t)h->dbg_w,
+                            (uint64_t)draft_len,
+                            0};
+  for (auto &g : h->graphs)
+    if (std::memcmp(g.key, key, sizeof key) == 0) {
+      CUDA_TRY(cudaGraphLaunch(g.exec, stream));
+      h->stats.kernel_launches += g.launches;
+      h->stats.steps += n_steps;
+      return MK_OK;
+    }
+  int launches = 0;
+  CUDA_TRY(cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal));
+  cudaError_t e = cudaSuccess;
+  for (int st = 0; st < n_steps && e == cudaSuccess; ++st) {
+    int n = 0;
+    e = wide_step(s, h->capture_stream, &n);
+    launches += n;
+    if (e == cudaSuccess)
+      e = wide_accept_step(B, T, st, h->w_vam, h->w_vtok, h->w_vpos, h->w_vpos0, drafts, draft_len, out_tokens,
+                           out_accepted, h->capture_stream);
+    ++launches;
+  }
+  cudaGraph_t graph = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(h->capture_stream, &graph);
+  if (e != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    return fail(MK_ERR_LAUNCH, "wide verify launch failed: %s", cudaGetErrorString(e));
+  }
+  if (ce != cudaSuccess) return fail(MK_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(ce));
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) return fail(MK_ERR_CUDA, "graph instantiate failed: %s", cudaGetErrorString(e));
+  if (h->graphs.size() >= 8) {
+    cudaGraphExecDestroy(h->graphs.front().exec);
+    h->graphs.erase(h->graphs.begin());
+  }
+  GraphEntry ge;
+  std::memcpy(ge.key, key, sizeof key);
+  ge.exec = exec;
+  ge.launches = launches;
+  h->graphs.push_back(ge);
+  CUDA_TRY(cudaGraphLaunch(exec, stream));
+  h->stats.kernel_launches += launches;
+  h->stats.steps += n_steps;
+  return MK_OK;
+}
+
 MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
                            int32_t T, int32_t n_steps, const int32_t *drafts, int32_t draft_len,
                            mk_kv_cache kv, float *out_logits, int32_t *out_tokens, int32_t *out_accepted,
@@ -886,12 +973,13 @@ MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *p
   if (!h) return fail(MK_ERR_ARG, "handle is NULL");
   if (n_steps < 1) return fail(MK_ERR_ARG, "n_steps must be >= 1");
   if (T < 2) return fail(MK_ERR_ARG, "a verify block has T >= 2 rows");
-  if ((long long)B * T > kMaxRows)
-    return fail(MK_ERR_UNSUPPORTED, "a verify launch serves at most %d rows per step", kMaxRows);
   if (!drafts || !out_tokens || !out_accepted) return fail(MK_ERR_ARG, "drafts, out_tokens and out_accepted are required");
   if ((long long)draft_len < (long long)n_steps * T)
     return fail(MK_ERR_ARG, "draft_len=%d is shorter than n_steps * T = %lld", draft_len, (long long)n_steps * T);
   if ((long long)n_steps * T > h->desc.kv_capacity) return fail(MK_ERR_CAPACITY, "n_steps * T exceeds kv_capacity");
+  if (B >= 1 && ((long long)B * T > kMaxRows || (h->variant == MK_TENSORCORE && h->desc.n_experts > 0)))
+    return run_wide_verify(h, tokens, positions, B, T, n_steps, drafts, draft_len, kv, out_logits, out_tokens,
+                           out_accepted, static_cast<cudaStream_t>(stream));
   const size_t need = (size_t)(n_steps + 1) * B + (size_t)(n_steps + 1) * B * T + (size_t)n_steps * B * T;
   if (need > h->vbuf_ints)  // sized at mk_create for every launch the checks above admit
     return fail(MK_ERR_CAPACITY, "verify buffers: %zu ints needed, %zu held", need, h->vbuf_ints);

@@ -219,6 +219,11 @@ cudaError_t wide_prepare();
 // A 128B-swizzled bf16 tensor map, box 64 columns x box_rows rows (mk_api.cu).
 int encode_2d_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
 cudaError_t wide_step(const WideStep &s, cudaStream_t stream, int *launches);
+// After verify block s: acceptance per sequence, and the next block written
+// over tok / pos in place (one launch).
+cudaError_t wide_accept_step(int B, int T, int s, const int32_t *argmax, int32_t *tok, int32_t *pos,
+                             const int32_t *pos0, const int32_t *drafts, int draft_len, int32_t *out_tokens,
+                             int32_t *out_accepted, cudaStream_t st);
 
 size_t step_smem_bytes(int n_ops, int xs_floats, int mmax, int e_ld);
 bool kernel_stages_x(int mmax);

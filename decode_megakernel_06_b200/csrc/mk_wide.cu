@@ -1071,6 +1071,34 @@ __global__ void wide_check(const int32_t *tokens, const int32_t *positions, int 
   if (bad && atomicCAS(&error[0], 0, -6) == 0) atomicExch(&error[1], 0);
 }
 
+// Acceptance after verify block s of the wide path (one thread per
+// sequence): the longest run of drafts that each equal the argmax of the row
+// before them, plus one token.  The accepted tokens (-1 after them) and their
+// count go out, and the next block replaces this one in place: the last
+// accepted token at the advanced position, then the drafts proposed for the
+// positions after it (drafts[b][j] is for cache position pos0[b] + j).
+__global__ void wide_accept(int B, int T, int s, const int32_t *argmax, int32_t *tok, int32_t *pos,
+                            const int32_t *pos0, const int32_t *drafts, int draft_len, int32_t *out_tokens,
+                            int32_t *out_accepted) {
+  pdl_wait();
+  pdl_launch();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  const int32_t *am = argmax + static_cast<long long>(b) * T;
+  int32_t *tb = tok + static_cast<long long>(b) * T;
+  int a = 1;
+  while (a < T && tb[a] == am[a - 1]) ++a;
+  for (int i = 0; i < T; ++i) out_tokens[(static_cast<long long>(s) * B + b) * T + i] = i < a ? am[i] : -1;
+  out_accepted[static_cast<long long>(s) * B + b] = a;
+  const int p = pos[b] + a;
+  pos[b] = p;
+  tb[0] = am[a - 1];
+  for (int t = 1; t < T; ++t) {
+    const int j = p + t - pos0[b];  // below draft_len for every block that runs
+    tb[t] = j >= 0 && j < draft_len ? drafts[static_cast<long long>(b) * draft_len + j] : 0;
+  }
+}
+
 int gemm_smem_bytes() { return kTcStages * kTcStage + 1024; }  // + room to align the stages to 1024 bytes
 
 }  // namespace
@@ -1156,6 +1184,13 @@ static cudaError_t gemm(int &n, const WideStep &s, const __nv_bfloat16 *W, const
     ++n;
   }
   return cudaSuccess;
+}
+
+cudaError_t wide_accept_step(int B, int T, int s, const int32_t *argmax, int32_t *tok, int32_t *pos,
+                             const int32_t *pos0, const int32_t *drafts, int draft_len, int32_t *out_tokens,
+                             int32_t *out_accepted, cudaStream_t st) {
+  return launch(wide_accept, dim3((B + 127) / 128), dim3(128), 0, st, B, T, s, argmax, tok, pos, pos0, drafts, draft_len,
+                out_tokens, out_accepted);
 }
 
 cudaError_t wide_prepare() {

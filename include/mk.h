@@ -223,15 +223,18 @@ MK_API int mk_decode_steps(mk_handle *h, const int32_t *tokens, const int32_t *p
  * accepted ones are overwritten by the next block before anything reads them.
  *   tokens      : device int32 [B*T], the first block (row b*T + t)
  *   positions   : device int32 [B]; positions[b] + n_steps*T <= kv_capacity
- *   B, T        : T >= 2, B*T <= min(max_rows, 8)
+ *   B, T        : T >= 2, B*T <= max_rows
  *   drafts      : device int32 [B][draft_len]: drafts[b][j] is the token proposed
  *                 for cache position positions[b] + j; draft_len >= n_steps*T
  *   out_logits  : device fp32 [B*T][vocab] of the LAST step, or NULL
  *   out_tokens  : device int32 [n_steps][B*T]: accepted tokens, -1 after the count
  *   out_accepted: device int32 [n_steps][B]: tokens accepted per step (1..T)
- * Always the megakernel.  Asynchronous; device-side errors are read with
- * mk_get_device_status.  Errors: MK_ERR_ARG, MK_ERR_CAPACITY, MK_ERR_UNSUPPORTED
- * (more than 8 rows) from the host checks. */
+ * Blocks of up to 8 rows run as ONE persistent megakernel launch.  Blocks
+ * above 8 rows (and, with MK_TENSORCORE, blocks on a MoE model) run the
+ * tensor-core launch sequence: n_steps x (the step, then the acceptance on
+ * the device, which writes the next block in place) as one CUDA graph launch.
+ * Asynchronous; device-side errors are read with mk_get_device_status.
+ * Errors: MK_ERR_ARG and MK_ERR_CAPACITY from the host checks. */
 MK_API int mk_verify_steps(mk_handle *h, const int32_t *tokens, const int32_t *positions,
                            int32_t B, int32_t T, int32_t n_steps, const int32_t *drafts,
                            int32_t draft_len, mk_kv_cache kv, float *out_logits,

@@ -140,6 +140,77 @@ def test_oracle_drafts_are_all_accepted():
     s.close()
 
 
+def _host_loop_batch(s: Session, firsts, p0s, drafts, n):
+    """n single-step verify calls of B sequences, acceptance on the host."""
+    dev, B = s.dev, len(firsts)
+    logits = torch.empty((B * T, s.m.vocab), dtype=torch.float32, device=dev)
+    am = torch.empty(B * T, dtype=torch.int32, device=dev)
+    last, p = list(firsts), list(p0s)
+    toks = np.full((n, B * T), -1, dtype=np.int64)
+    accs = np.zeros((n, B), dtype=np.int64)
+    for st in range(n):
+        blk = []
+        for b in range(B):
+            blk += [last[b]] + [int(drafts[b][p[b] - p0s[b] + t]) for t in range(1, T)]
+        rc = s.dec.step(torch.tensor(blk, dtype=torch.int32, device=dev),
+                        torch.tensor(p, dtype=torch.int32, device=dev), B, T, s.k, s.v, logits, am)
+        assert rc == mk.MK_OK, mk.mk_last_error()
+        row = am.cpu().numpy()
+        for b in range(B):
+            a = 1
+            while a < T and blk[b * T + a] == int(row[b * T + a - 1]):
+                a += 1
+            toks[st, b * T:b * T + a] = row[b * T:b * T + a]
+            accs[st, b] = a
+            last[b], p[b] = int(row[b * T + a - 1]), p[b] + a
+    assert s.dec.status() == mk.MK_OK
+    return toks, accs, logits.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,B,n", [("tiny", 2, 6), ("small", 8, 3)])
+def test_wide_launch_equals_host_loop(name, B, n):
+    """Blocks above 8 rows (2 x 7 on the tiny model, 8 x 7 on the small one):
+    the tensor-core sequence with acceptance on the device, n blocks in one
+    graph launch, against n single-step calls with host acceptance."""
+    wl = Workload("tiny_verify_b2", TINY, B, T, 127, steps=16, seed=0) if name == "tiny" else workload("verify", B)
+    s = Session(wl, capacity=wl.kv_capacity() + n * T + T)
+    s.dec.set_debug(None, None, None)
+    dev = s.dev
+    p0s = make_context_lengths(wl)
+    firsts = make_tokens(s.m.vocab, B, wl.seed)
+    drafts = np.stack([np.array(make_tokens(s.m.vocab, n * T + T, wl.seed + b, name="drafts"), dtype=np.int64)
+                       for b in range(B)])
+    k0, v0 = s.k.clone(), s.v.clone()
+    probe, _, _ = _host_loop_batch(s, firsts, p0s, drafts, 1)
+    s.k.copy_(k0)
+    s.v.copy_(v0)
+    for b in range(B):  # each sequence's first draft matches the model's first prediction
+        drafts[b][1] = probe[0][b * T]
+    ref_tok, ref_acc, ref_logits = _host_loop_batch(s, firsts, p0s, drafts, n)
+    k1, v1 = s.k.clone(), s.v.clone()
+    s.k.copy_(k0)
+    s.v.copy_(v0)
+    blk = []
+    for b in range(B):
+        blk += [firsts[b]] + [int(drafts[b][t]) for t in range(1, T)]
+    logits = torch.empty((B * T, s.m.vocab), dtype=torch.float32, device=dev)
+    out = torch.empty((n, B * T), dtype=torch.int32, device=dev)
+    acc = torch.empty((n, B), dtype=torch.int32, device=dev)
+    rc = s.dec.verify_steps(torch.tensor(blk, dtype=torch.int32, device=dev),
+                            torch.tensor(p0s, dtype=torch.int32, device=dev), B, T, n,
+                            torch.tensor(drafts, dtype=torch.int32, device=dev), s.k, s.v, logits, out, acc)
+    assert rc == mk.MK_OK, mk.mk_last_error()
+    assert s.dec.status() == mk.MK_OK, mk.mk_last_error()
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref_acc)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref_tok)
+    assert np.array_equal(logits.cpu().numpy().view(np.uint32), ref_logits.view(np.uint32)), "final logits differ"
+    assert torch.equal(s.k.view(torch.int16), k1.view(torch.int16)), "K cache differs"
+    assert torch.equal(s.v.view(torch.int16), v1.view(torch.int16)), "V cache differs"
+    assert (ref_acc[0] >= 2).all(), ref_acc
+    s.close()
+    print(name, B, "accepted", acc.cpu().numpy().tolist())
+
+
 def test_verify_launch_rejects_bad_arguments():
     wl = _verify_workload("tiny")
     s = Session(wl, capacity=wl.kv_capacity() + 64)
