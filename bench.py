@@ -483,10 +483,33 @@ def measure_sampled(dec, m, k, v, B, ctx, device, steps=20, warmup=3, temperatur
     phases["total (first stamp to last)"] = round(sum(med), 2)
     phases["how"] = ("%globaltimer at each phase boundary of row 0's first CTA, median of 21 calls; the "
                      "device clock advances in steps of a few hundred ns")
+    # the same sampled decode, 32 steps as one graph launch (mk_decode_steps_sample)
+    nl = 32
+    ul = torch.tensor(make_uniforms(nl * B, 59), dtype=torch.float64, device=device).view(nl, B)
+    outl = torch.empty((nl, B), dtype=torch.int32, device=device)
+    p0 = torch.tensor([ctx[b] for b in range(B)], dtype=torch.int32, device=device)
+    for _ in range(2):
+        assert dec.steps_sample(bufs[0], p0, B, nl, k, v, None, temperature, top_p, ul, outl) == 0, mk.mk_last_error()
+    torch.cuda.synchronize()
+    dec.stats(reset=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    assert dec.steps_sample(bufs[0], p0, B, nl, k, v, None, temperature, top_p, ul, outl) == 0
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    sts = dec.stats(reset=True)
+    lms = e0.elapsed_time(e1) / nl
+    loop = {"steps_per_call": nl, "ms_per_step": round(lms, 4), "tok_s": round(B / (lms / 1e3), 1),
+            "graph_launches": int(sts.graph_launches), "kernels": int(sts.kernel_launches),
+            "path": ("mk_decode_steps_sample: 32 x (megakernel step, sampler) as one CUDA graph launch"
+                     if sts.graph_launches == 1 else
+                     "mk_decode_steps_sample: 32 x (megakernel step, sampler) enqueued one by one")}
     return {"batch": B, "temperature": temperature, "top_p": top_p, "ms_per_step": round(ms, 4),
             "tok_s": round(B / (ms / 1e3), 1), "launches_per_step": 2,
             "sampler_alone": alone, "sampler_phases_rows1_us": phases, "vocab": m.vocab,
-            "path": "mk_decode_step_sample: the megakernel step, then the cluster top-p sampler on its logits"}
+            "path": "mk_decode_step_sample: the megakernel step, then the cluster top-p sampler on its logits",
+            "loop": loop}
 
 
 def measure_dense(device, steps=20, warmup=3):

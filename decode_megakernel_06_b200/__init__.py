@@ -68,7 +68,7 @@ class mk_kv_cache(ctypes.Structure):
 
 class mk_stats(ctypes.Structure):
     _fields_ = [("steps", ctypes.c_uint64), ("expert_union_total", ctypes.c_uint64),
-                ("kernel_launches", ctypes.c_uint64)]
+                ("kernel_launches", ctypes.c_uint64), ("graph_launches", ctypes.c_uint64)]
 
 
 class mk_plan_info(ctypes.Structure):
@@ -107,6 +107,8 @@ def lib():
         "mk_sample_top_p_phases": (i32, [vp, i32, i32, ctypes.c_float, ctypes.c_float, vp, vp, vp, vp]),
         "mk_decode_step_sample": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, ctypes.c_float,
                                         ctypes.c_float, vp, vp, vp]),
+        "mk_decode_steps_sample": (i32, [vp, vp, vp, i32, i32, mk_kv_cache, vp, ctypes.c_float,
+                                         ctypes.c_float, vp, vp, vp]),
         "mk_get_device_status": (i32, [vp, vp]),
         "mk_last_device_error_op": (i32, [vp]),
         "mk_last_error": (ctypes.c_char_p, []),
@@ -210,6 +212,14 @@ def mk_decode_step_sample(h, tokens: int, positions: int, B: int, T: int, kv: mk
                           out_tokens: int, stream: int) -> int:
     return lib().mk_decode_step_sample(h, tokens, positions, B, T, kv, out_logits, temperature, top_p,
                                        uniforms, out_tokens, stream)
+
+
+def mk_decode_steps_sample(h, tokens: int, positions: int, B: int, n_steps: int, kv: mk_kv_cache,
+                           out_logits: int, temperature: float, top_p: float, uniforms: int,
+                           out_tokens: int, stream: int) -> int:
+    """n_steps sampled steps as one graph launch (see include/mk.h)."""
+    return lib().mk_decode_steps_sample(h, tokens, positions, B, n_steps, kv, out_logits, temperature, top_p,
+                                        uniforms, out_tokens, stream)
 
 
 def _need(t, dtype, min_numel: int, name: str, device=None, dims: Optional[int] = None):
@@ -417,6 +427,21 @@ class Decoder:
         return mk_decode_step_sample(self.h, tokens.data_ptr(), positions.data_ptr(), B, T, kv,
                                      _ptr(logits), temperature, top_p, _ptr(uniforms),
                                      out_tokens.data_ptr(), s.cuda_stream)
+
+    def steps_sample(self, tokens, positions, B: int, n_steps: int, k_cache, v_cache, logits,
+                     temperature: float, top_p: float, uniforms, out_tokens, stream=None) -> int:
+        """n_steps sampled steps as one graph launch; uniforms is fp64
+        [n_steps, B] (None for greedy), out_tokens int32 [n_steps, B] on the
+        device.  Returns the launch status code."""
+        dev = self._io(tokens, positions, B, B, k_cache, v_cache, logits)
+        if uniforms is not None:
+            _need(uniforms, self._torch.float64, n_steps * B, "uniforms", dev)
+        _need(out_tokens, self._torch.int32, n_steps * B, "out_tokens", dev)
+        s = stream if stream is not None else self._torch.cuda.current_stream()
+        kv = mk_kv_cache(k_cache.data_ptr(), v_cache.data_ptr())
+        return mk_decode_steps_sample(self.h, tokens.data_ptr(), positions.data_ptr(), B, n_steps, kv,
+                                      _ptr(logits), temperature, top_p, _ptr(uniforms),
+                                      out_tokens.data_ptr(), s.cuda_stream)
 
     def steps(self, tokens, positions, B: int, n_steps: int, k_cache, v_cache, logits, out_tokens,
               stream=None) -> int:

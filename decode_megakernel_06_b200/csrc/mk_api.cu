@@ -268,6 +268,7 @@ struct mk_handle {
   long long w_part_floats;
   int32_t *w_sele, *w_tok, *w_pos;
   int32_t *w_vtok, *w_vpos, *w_vpos0, *w_vam;  // the wide verify loop: block, positions, start, argmax
+  int32_t *sp_pos;  // the sampled multi-step loop's positions: [kv_capacity][min(max_seqs, 8)]
   int *w_count, *w_off, *w_pair_row, *w_pair_slot, *w_active;
   __nv_bfloat16 *w_xhi, *w_xlo, *w_ghi, *w_glo, *w_ahi, *w_alo, *w_shi, *w_slo;
 };
@@ -447,6 +448,7 @@ MK_API int mk_create(const mk_model_desc *desc, const mk_weights *w, mk_handle *
   h->racc_bytes = sizeof(long long) * (size_t)L * kMaxRows * (ceil_div(std::max(d.n_experts, 1), 4) * 4);
   HALLOC(h->racc, h->racc_bytes);
   HALLOC(h->ssq, sizeof(long long) * 2 * kMaxRows);
+  HALLOC(h->sp_pos, sizeof(int32_t) * (size_t)d.kv_capacity * std::min(d.max_seqs, kMaxRows));
   HALLOC(h->qkv, sizeof(float) * 2 * (size_t)kMaxRows * QKVW);  // [K half][row][QKVW]
   HALLOC(h->o, sizeof(float) * (size_t)kMaxRows * panel_ld(d.n_q_heads * d.head_dim));
   HALLOC(h->attn_o, sizeof(float) * s.attn_o);
@@ -740,6 +742,7 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
   for (auto &g : h->graphs)
     if (std::memcmp(g.key, key, sizeof key) == 0) {
       CUDA_TRY(cudaGraphLaunch(g.exec, stream));
+      h->stats.graph_launches += 1;
       h->stats.kernel_launches += g.launches;
       h->stats.steps += 1;
       return MK_OK;
@@ -768,6 +771,7 @@ static int run_wide(mk_handle *h, const int32_t *tokens, const int32_t *position
   ge.launches = launches;
   h->graphs.push_back(ge);
   CUDA_TRY(cudaGraphLaunch(exec, stream));
+  h->stats.graph_launches += 1;
   h->stats.kernel_launches += launches;
   h->stats.steps += 1;
   return MK_OK;
@@ -827,6 +831,7 @@ static int run_step(mk_handle *h, const int32_t *tokens, const int32_t *position
       h->stats.kernel_launches -= pl.n_ops;  // counted again below on replay
     }
     CUDA_TRY(cudaGraphLaunch(exec, stream));
+    h->stats.graph_launches += 1;
     h->stats.kernel_launches += pl.n_ops;
   } else {
     if (variant == MK_MULTIKERNEL_GRAPH) variant = MK_MULTIKERNEL;
@@ -892,6 +897,110 @@ MK_API int mk_decode_step_sample(mk_handle *h, const int32_t *tokens, const int3
   return MK_OK;
 }
 
+// positions of step s of a sampled loop: out[s][b] = positions[b] + s
+__global__ void sp_positions(const int32_t *positions, int B, int n_steps, int32_t *out) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B * n_steps; i += gridDim.x * blockDim.x)
+    out[i] = positions[i % B] + i / B;
+}
+
+// The sampled loop's launches on stream s: the positions, then per step the
+// megakernel (tokens: the previous step's samples) and the sampler.
+static int enqueue_sampled_loop(mk_handle *h, const int32_t *tokens, const int32_t *positions, int B, int n_steps,
+                                mk_kv_cache kv, float *logits, float temperature, float top_p,
+                                const double *uniforms, int32_t *out_tokens, cudaStream_t s, int *launches) {
+  sp_positions<<<std::max(1, std::min(ceil_div(B * n_steps, 256), 64)), 256, 0, s>>>(positions, B, n_steps, h->sp_pos);
+  CUDA_TRY(cudaGetLastError());
+  int n = 1;
+  for (int st = 0; st < n_steps; ++st) {
+    Params p;
+    Plan pl;
+    int rc = fill_params(h, st == 0 ? tokens : out_tokens + (size_t)(st - 1) * B, h->sp_pos + (size_t)st * B, B, 1, kv,
+                         logits, out_tokens + (size_t)st * B, p, pl);
+    if (rc) return rc;
+    int e = launch_step_any(p, pl.mmax, true, s);
+    if (e) return fail(MK_ERR_LAUNCH, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
+    CUDA_TRY(launch_top_p(logits, B, h->desc.vocab, temperature, top_p, uniforms ? uniforms + (size_t)st * B : nullptr,
+                          out_tokens + (size_t)st * B, s));
+    n += 2;
+  }
+  *launches = n;
+  return MK_OK;
+}
+
+MK_API int mk_decode_steps_sample(mk_handle *h, const int32_t *tokens, const int32_t *positions, int32_t B,
+                                  int32_t n_steps, mk_kv_cache kv, float *out_logits, float temperature,
+                                  float top_p, const double *uniforms, int32_t *out_tokens, void *stream) {
+  if (!h) return fail(MK_ERR_ARG, "handle is NULL");
+  if (n_steps < 1) return fail(MK_ERR_ARG, "n_steps must be >= 1");
+  if (B < 1 || B > kMaxRows) return fail(MK_ERR_UNSUPPORTED, "a sampled loop serves 1 to %d sequences", kMaxRows);
+  if (n_steps > h->desc.kv_capacity) return fail(MK_ERR_CAPACITY, "n_steps=%d exceeds kv_capacity", n_steps);
+  if (!tokens || !positions) return fail(MK_ERR_ARG, "tokens and positions are required");
+  int rc = check_sample_args(h, B, h->desc.vocab, temperature, top_p, uniforms, out_tokens);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *logits = out_logits ? out_logits : h->logits;
+  uint32_t tb, pb;
+  std::memcpy(&tb, &temperature, 4);
+  std::memcpy(&pb, &top_p, 4);
+  const uint64_t key[12] = {(uint64_t)B | (0x53ull << 56),  // sampled-loop entries
+                            (uint64_t)n_steps,
+                            (uint64_t)(uintptr_t)tokens,
+                            (uint64_t)(uintptr_t)positions,
+                            (uint64_t)(uintptr_t)logits,
+                            (uint64_t)(uintptr_t)uniforms,
+                            (uint64_t)(uintptr_t)out_tokens,
+                            (uint64_t)(uintptr_t)kv.k,
+                            (uint64_t)(uintptr_t)kv.v,
+                            (uint64_t)tb | ((uint64_t)pb << 32),
+                            (uint64_t)(uintptr_t)h->dbg_hidden ^ (uint64_t)(uintptr_t)h->dbg_ids ^
+                                (uint64_t)(uintptr_t)h->dbg_w,
+                            h->timeout_ns};
+  for (auto &g : h->graphs)
+    if (std::memcmp(g.key, key, sizeof key) == 0) {
+      CUDA_TRY(cudaGraphLaunch(g.exec, s));
+      h->stats.graph_launches += 1;
+      h->stats.kernel_launches += g.launches;
+      h->stats.steps += n_steps;
+      return MK_OK;
+    }
+  int launches = 0;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  bool captured = false;
+  if (cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
+    rc = enqueue_sampled_loop(h, tokens, positions, B, n_steps, kv, logits, temperature, top_p, uniforms, out_tokens,
+                              h->capture_stream, &launches);
+    const cudaError_t ce = cudaStreamEndCapture(h->capture_stream, &graph);
+    if (rc == MK_OK && ce == cudaSuccess && graph && cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess)
+      captured = true;
+    if (graph) cudaGraphDestroy(graph);
+    if (rc != MK_OK && rc != MK_ERR_LAUNCH && rc != MK_ERR_CUDA) return rc;  // an argument error, not the capture
+  }
+  if (!captured) {  // enqueue the same launches one by one
+    (void)cudaGetLastError();
+    rc = enqueue_sampled_loop(h, tokens, positions, B, n_steps, kv, logits, temperature, top_p, uniforms, out_tokens, s,
+                              &launches);
+    if (rc) return rc;
+    h->stats.kernel_launches += launches;
+    h->stats.steps += n_steps;
+    return MK_OK;
+  }
+  if (h->graphs.size() >= 8) {
+    cudaGraphExecDestroy(h->graphs.front().exec);
+    h->graphs.erase(h->graphs.begin());
+  }
+  GraphEntry ge;
+  std::memcpy(ge.key, key, sizeof key);
+  ge.exec = exec;
+  ge.launches = launches;
+  h->graphs.push_back(ge);
+  CUDA_TRY(cudaGraphLaunch(exec, s));
+  h->stats.graph_launches += 1;
+  h->stats.kernel_launches += launches;
+  h->stats.steps += n_steps;
+  return MK_OK;
+}
+
 // mk_verify_steps on the tensor-core launch sequence: the block and its
 // positions are copied into the handle, then n_steps x (wide step, then
 // acceptance on the device, which writes the next block in place) run as one
@@ -924,6 +1033,7 @@ static int run_wide_verify(mk_handle *h, const int32_t *tokens, const int32_t *p
   for (auto &g : h->graphs)
     if (std::memcmp(g.key, key, sizeof key) == 0) {
       CUDA_TRY(cudaGraphLaunch(g.exec, stream));
+      h->stats.graph_launches += 1;
       h->stats.kernel_launches += g.launches;
       h->stats.steps += n_steps;
       return MK_OK;
@@ -961,6 +1071,7 @@ static int run_wide_verify(mk_handle *h, const int32_t *tokens, const int32_t *p
   ge.launches = launches;
   h->graphs.push_back(ge);
   CUDA_TRY(cudaGraphLaunch(exec, stream));
+  h->stats.graph_launches += 1;
   h->stats.kernel_launches += launches;
   h->stats.steps += n_steps;
   return MK_OK;

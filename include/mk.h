@@ -127,6 +127,8 @@ typedef struct mk_stats {
   uint64_t expert_union_total; /* sum over steps and layers of the number of
                                   distinct routed experts (device-counted)  */
   uint64_t kernel_launches;    /* kernels launched by the library           */
+  uint64_t graph_launches;     /* CUDA graphs launched by the library (their
+                                  kernels are counted in kernel_launches)   */
 } mk_stats;
 
 /* Schedule summary for a shape (host-only planning; see mk_plan_describe). */
@@ -291,6 +293,30 @@ MK_API int mk_decode_step_sample(mk_handle *h, const int32_t *tokens, const int3
                                  int32_t B, int32_t T, mk_kv_cache kv, float *out_logits,
                                  float temperature, float top_p, const double *uniforms,
                                  int32_t *out_tokens, void *stream);
+
+/* n_steps sampled decode steps of B sequences (one row each) as ONE CUDA graph
+ * launch: step s runs the megakernel at positions[b] + s on the tokens
+ * sampled by step s-1 (step 0: tokens), then mk_sample_top_p on its logits
+ * with uniforms[s][B] into out_tokens[s][B].  Passage: the pages' serving
+ * loop offers greedy or temperature / top-p generation (tpu-megakernels
+ * README, serving paragraph); this is the sampled form of mk_decode_steps.
+ *   tokens     : device int32 [B], the first step's tokens
+ *   positions  : device int32 [B]; positions[b] + n_steps <= kv_capacity
+ *   B          : 1 <= B <= min(max_seqs, 8)
+ *   out_logits : device fp32 [B][vocab]: the LAST step's logits, or NULL
+ *   uniforms   : device fp64 [n_steps][B] in [0, 1) (may be NULL when
+ *                temperature <= 0: greedy)
+ *   out_tokens : device int32 [n_steps][B]
+ * The graph is recorded once per (B, n_steps, buffers, temperature, top_p)
+ * and replayed; where a cooperative launch cannot be captured, the same
+ * 2 * n_steps launches are enqueued one by one.  Asynchronous; device-side
+ * errors are read with mk_get_device_status.  Errors: MK_ERR_ARG,
+ * MK_ERR_CAPACITY, MK_ERR_UNSUPPORTED (B > 8, vocab above the sampler's
+ * limit) from the host checks. */
+MK_API int mk_decode_steps_sample(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                                  int32_t B, int32_t n_steps, mk_kv_cache kv, float *out_logits,
+                                  float temperature, float top_p, const double *uniforms,
+                                  int32_t *out_tokens, void *stream);
 
 /* The same step driven from HOST buffers: copies tokens [B*T] and positions
  * [B] to the device, runs the step, copies argmax [B*T] back to

@@ -196,6 +196,7 @@ def test_sampler_checks_its_arguments_on_the_host(L):
     assert L.mk_sample_top_p_phases(lg, 1, 131073, 1.0, 0.9, u, out, st, None) == mk.MK_ERR_UNSUPPORTED
     kv = mk.mk_kv_cache(None, None)
     assert L.mk_decode_step_sample(None, None, None, 1, 1, kv, None, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
+    assert L.mk_decode_steps_sample(None, None, None, 1, 2, kv, None, 1.0, 0.9, u, out, None) == mk.MK_ERR_ARG
 
 
 def test_torch_wrappers_check_tensors_before_any_launch():

@@ -198,3 +198,43 @@ def test_decode_step_sample_against_oracle():
     s.close()
     assert checked >= total // 2, (checked, total)
     print("decode+sample checked", checked, "of", total)
+
+
+def test_sampled_loop_equals_single_sampled_steps():
+    """mk_decode_steps_sample (n sampled steps as one graph launch) against n
+    mk_decode_step_sample calls, each fed the previous call's tokens: the same
+    tokens, final logits and caches, bit for bit; the graph's replay too."""
+    wl = Workload("tiny_b4_sample_loop", TINY, 4, 1, context=None, context_range=(20, 120), steps=8, seed=22)
+    n, B = 6, 4
+    s = Session(wl)
+    s.dec.set_debug(None, None, None)
+    dev = s.dev
+    p0 = make_context_lengths(wl)
+    tok0 = torch.tensor(make_tokens(s.m.vocab, B, wl.seed), dtype=torch.int32, device=dev)
+    u = torch.tensor(make_uniforms(n * B, seed=77), dtype=torch.float64, device=dev).view(n, B)
+    T, top_p = 0.8, 0.9
+    k0, v0 = s.k.clone(), s.v.clone()
+    ref = torch.empty((n, B), dtype=torch.int32, device=dev)
+    tok = tok0.clone()
+    for st in range(n):
+        pos = torch.tensor([p + st for p in p0], dtype=torch.int32, device=dev)
+        assert s.dec.step_sample(tok, pos, B, 1, s.k, s.v, s.logits, T, top_p, u[st].contiguous(), ref[st]) == mk.MK_OK
+        tok = ref[st].clone()
+    assert s.dec.status() == mk.MK_OK
+    ref_logits = s.logits.clone()
+    k1, v1 = s.k.clone(), s.v.clone()
+    for rep in range(2):  # the first call records the graph, the second replays it
+        s.k.copy_(k0)
+        s.v.copy_(v0)
+        out = torch.full((n, B), -7, dtype=torch.int32, device=dev)
+        pos0 = torch.tensor(p0, dtype=torch.int32, device=dev)
+        s.dec.stats(reset=True)
+        assert s.dec.steps_sample(tok0, pos0, B, n, s.k, s.v, s.logits, T, top_p, u, out) == mk.MK_OK, mk.mk_last_error()
+        assert s.dec.status() == mk.MK_OK
+        st = s.dec.stats(reset=True)
+        print("graph launches", st.graph_launches, "kernels", st.kernel_launches)
+        assert torch.equal(out, ref), (rep, out, ref)
+        assert torch.equal(s.logits.view(torch.int32), ref_logits.view(torch.int32)), "final logits differ"
+        assert torch.equal(s.k.view(torch.int16), k1.view(torch.int16)), "K cache differs"
+        assert torch.equal(s.v.view(torch.int16), v1.view(torch.int16)), "V cache differs"
+    s.close()
