@@ -933,6 +933,7 @@ MK_API int mk_decode_steps_sample(mk_handle *h, const int32_t *tokens, const int
   if (!h) return fail(MK_ERR_ARG, "handle is NULL");
   if (n_steps < 1) return fail(MK_ERR_ARG, "n_steps must be >= 1");
   if (B < 1 || B > kMaxRows) return fail(MK_ERR_UNSUPPORTED, "a sampled loop serves 1 to %d sequences", kMaxRows);
+  if (B > h->desc.max_seqs) return fail(MK_ERR_CAPACITY, "B=%d exceeds max_seqs=%d", B, h->desc.max_seqs);
   if (n_steps > h->desc.kv_capacity) return fail(MK_ERR_CAPACITY, "n_steps=%d exceeds kv_capacity", n_steps);
   if (!tokens || !positions) return fail(MK_ERR_ARG, "tokens and positions are required");
   int rc = check_sample_args(h, B, h->desc.vocab, temperature, top_p, uniforms, out_tokens);

@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(128) probe_bulk_kernel(const uint8_t *buf, siz
         ++issued;
       }
     }
-    // thread 0 waits (bounded) for the slot; the block follows its verdict
+    // thread 0 waits (bounded) for the slot; the block follows its decision
     const int s = static_cast<int>(done % kBulkSlots);
     if (threadIdx.x == 0) {
       const uint32_t par = static_cast<uint32_t>((done / kBulkSlots) & 1);
