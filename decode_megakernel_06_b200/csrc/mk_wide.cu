@@ -496,11 +496,11 @@ __global__ void wide_kv_append(float *qkv, int W3, const int32_t *positions, int
 // wide_attn_merge combines a query's chunks with the log-sum-exp rule.
 // ---------------------------------------------------------------------------
 constexpr int kAcN = 128;             // cache positions per chunk (M of S^T, K of O^T)
-constexpr int kAcQ = 32;              // query vectors per CTA (N of both products)
+constexpr int kAcQ = 32;              // query vectors per CTA (N of both products): 32, or 16 for
+                                      // groups of at most 16 (one row per sequence, say)
 constexpr int kAcThreads = 128;
 constexpr int kAcTmemCols = 64;       // S^T: columns [0, 32), O^T: [32, 64)
 constexpr int kAcAtom = 128 * 128;    // a swizzled block of 128 rows x 128 bytes
-constexpr int kAcQAtom = kAcQ * 128;  // a swizzled block of kAcQ rows x 128 bytes
 
 struct AttnArgs {
   CUtensorMap mk;  // K cache as [L * Bmax * Hkv * cap][hd], box 64 x 128
@@ -515,9 +515,9 @@ struct AttnArgs {
   int *error;
 };
 
-// dynamic shared memory: K then V^T (2 blocks), Q then P (16 KB), + room to
-// align them to 1024 bytes
-constexpr int attn_smem_bytes(int) { return 2 * kAcAtom + 4 * kAcQAtom + 1024; }
+// dynamic shared memory: K then V^T (2 blocks), Q then P (4 blocks of qn rows
+// x 128 bytes), + room to align them to 1024 bytes
+constexpr int attn_smem_bytes(int qn) { return 2 * kAcAtom + 4 * qn * 128 + 1024; }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);  // .x at the lower address
@@ -534,13 +534,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 // byte offset of the 16-byte piece `piece` (0..7) of row r in a swizzled block
 __device__ __forceinline__ int sw_off(int r, int piece) { return r * 128 + ((piece ^ (r & 7)) << 4); }
 
-// Reduces each of the 32 values over the warp's lanes: afterwards v[0] of
-// lane l holds the reduction of value l (31 shuffles; v is overwritten).
-// Each step trades half of the values with the lane `o` away and combines.
-template <bool MAX>
-__device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane) {
+// Reduces each of the NV values over the warp's lanes: afterwards lane l
+// holds the reduction of value l mod NV (NV - 1 shuffles, then one per
+// remaining lane bit; v is overwritten).  Each step trades half of the
+// values with the lane `o` away and combines.
+template <bool MAX, int NV>
+__device__ __forceinline__ float warp_transpose_reduce(float (&v)[NV], int lane) {
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
+  for (int o = NV / 2; o >= 1; o >>= 1) {
     const bool upper = (lane & o) != 0;
 #pragma unroll
     for (int i = 0; i < o; ++i) {
@@ -550,14 +551,22 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane)
       v[i] = MAX ? fmaxf(keep, got) : keep + got;
     }
   }
-  return v[0];
+  float r = v[0];
+#pragma unroll
+  for (int o = NV; o < 32; o <<= 1) {  // lanes l and l ^ o hold the same value's partials
+    const float got = __shfl_xor_sync(0xffffffffu, r, o);
+    r = MAX ? fmaxf(r, got) : r + got;
+  }
+  return r;
 }
 
-template <int HD>
+template <int HD, int QN>
 __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant__ AttnArgs a) {
   pdl_wait();
   pdl_launch();
   constexpr int NA = HD / 64, HALF = HD / 2;
+  constexpr int QA = QN * 128;  // a swizzled block of QN rows x 128 bytes
+  static_assert(QN == 16 || QN == 32, "N of the products: 16 or 32 query vectors");
   constexpr int NU = 64 * (HD / 8) / kAcThreads;  // (position pair, 8 dims) units of V per thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (sptr(smem_raw) & 1023u)) & 1023u);
@@ -566,9 +575,9 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
   uint8_t *sQ = smem + 2 * kAcAtom;           // Q hi: NA blocks, Q lo: NA blocks; then P hi: 2, P lo: 2
   __shared__ __align__(8) uint64_t kbar, sbar, obar;
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(16) float red[4][kAcQ], sM[kAcQ];
+  __shared__ __align__(16) float red[4][QN], sM[QN];
   const int c = blockIdx.x, bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv, G = a.Hq / a.Hkv;
-  const int Q = a.T * G, q0 = blockIdx.z * kAcQ, nq = min(kAcQ, Q - q0);
+  const int Q = a.T * G, q0 = blockIdx.z * QN, nq = min(QN, Q - q0);
   const int pos0 = a.positions[b], last = pos0 + a.T - 1;
   const int j0 = c * kAcN;
   if (j0 > last || nq <= 0) return;  // the whole CTA, before anything is allocated
@@ -642,26 +651,26 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
         y2l[e / 2] = pack_bf16(r2[0], r2[1]);
       }
       const int d1 = 8 * cc, d2 = HALF + 8 * cc;
-      const int o1 = (d1 >> 6) * kAcQAtom + sw_off(ql, (d1 & 63) >> 3),
-                o2 = (d2 >> 6) * kAcQAtom + sw_off(ql, (d2 & 63) >> 3);
+      const int o1 = (d1 >> 6) * QA + sw_off(ql, (d1 & 63) >> 3),
+                o2 = (d2 >> 6) * QA + sw_off(ql, (d2 & 63) >> 3);
       *reinterpret_cast<uint4 *>(sQ + o1) = make_uint4(y1h[0], y1h[1], y1h[2], y1h[3]);
-      *reinterpret_cast<uint4 *>(sQ + NA * kAcQAtom + o1) = make_uint4(y1l[0], y1l[1], y1l[2], y1l[3]);
+      *reinterpret_cast<uint4 *>(sQ + NA * QA + o1) = make_uint4(y1l[0], y1l[1], y1l[2], y1l[3]);
       *reinterpret_cast<uint4 *>(sQ + o2) = make_uint4(y2h[0], y2h[1], y2h[2], y2h[3]);
-      *reinterpret_cast<uint4 *>(sQ + NA * kAcQAtom + o2) = make_uint4(y2l[0], y2l[1], y2l[2], y2l[3]);
+      *reinterpret_cast<uint4 *>(sQ + NA * QA + o2) = make_uint4(y2l[0], y2l[1], y2l[2], y2l[3]);
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
-  // K-major, N = kAcQ, M = 128 (both products)
-  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kAcQ >> 3) << 17) | ((128 >> 4) << 24);
+  // K-major, N = QN, M = 128 (both products)
+  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((QN >> 3) << 17) | ((128 >> 4) << 24);
   if (threadIdx.x == 0) {
     if (tc_wait(&kbar, 0, a.error)) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll
       for (int i = 0; i < NA; ++i) {
-        const uint64_t dk = tc_desc(sK + i * kAcAtom), dqh = tc_desc(sQ + i * kAcQAtom),
-                       dql = tc_desc(sQ + (NA + i) * kAcQAtom);
+        const uint64_t dk = tc_desc(sK + i * kAcAtom), dqh = tc_desc(sQ + i * QA),
+                       dql = tc_desc(sQ + (NA + i) * QA);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // 16 dims = 32 bytes = 2 descriptor units
           tc_mma(tmem, dk + 2 * kk, dqh + 2 * kk, kIdesc, (i > 0 || kk > 0) ? 1u : 0u);
@@ -688,35 +697,36 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
       *reinterpret_cast<uint32_t *>(blk + sw_off(d, (pp & 31) >> 2)) = word;
     }
   }
-  // position j = this thread's accumulator lane: its scores for the kAcQ query vectors
+  // position j = this thread's accumulator lane: its scores for the QN query vectors
   const int j = threadIdx.x;
   const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-  float sc[kAcQ];
+  float sc[QN];
   {
     uint32_t v0[16], v1[16];
     tmem_ld16(tlane, v0);
-    tmem_ld16(tlane + 16, v1);
+    if constexpr (QN == 32) tmem_ld16(tlane + 16, v1);
     // query ql sees position j0 + j iff it exists and j0 + j <= pos0 + (q0 + ql) / G
     const int dj = j0 + j - pos0;
 #pragma unroll
-    for (int ql = 0; ql < kAcQ; ++ql) {
+    for (int ql = 0; ql < QN; ++ql) {
       const bool see = ql < nq && j < nj && (dj <= 0 || q0 + ql >= G * dj);
       sc[ql] = see ? __uint_as_float(ql < 16 ? v0[ql] : v1[ql - 16]) : -INFINITY;
     }
   }
   {
-    float t[kAcQ];
+    float t[QN];
 #pragma unroll
-    for (int ql = 0; ql < kAcQ; ++ql) t[ql] = sc[ql];
-    red[warp][lane] = warp_transpose_reduce<true>(t, lane);
+    for (int ql = 0; ql < QN; ++ql) t[ql] = sc[ql];
+    const float r = warp_transpose_reduce<true, QN>(t, lane);
+    if (lane < QN) red[warp][lane] = r;
   }
   __syncthreads();
-  if (threadIdx.x < kAcQ)
+  if (threadIdx.x < QN)
     sM[threadIdx.x] = fmaxf(fmaxf(red[0][threadIdx.x], red[1][threadIdx.x]), fmaxf(red[2][threadIdx.x], red[3][threadIdx.x]));
   __syncthreads();
-  float pv[kAcQ];
+  float pv[QN];
 #pragma unroll
-  for (int q4 = 0; q4 < kAcQ / 4; ++q4) {
+  for (int q4 = 0; q4 < QN / 4; ++q4) {
     const float4 m4 = *reinterpret_cast<const float4 *>(&sM[4 * q4]);
     const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
@@ -727,14 +737,14 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
   }
   // p^T as a bf16 pair: row ql, K index j (the Q rows are no longer read)
   {
-    uint8_t *base = sQ + (j >> 6) * kAcQAtom + (j & 7) * 2;
+    uint8_t *base = sQ + (j >> 6) * QA + (j & 7) * 2;
 #pragma unroll
-    for (int ql = 0; ql < kAcQ; ++ql) {
+    for (int ql = 0; ql < QN; ++ql) {
       const __nv_bfloat16 hi = __float2bfloat16_rn(pv[ql]);
       const __nv_bfloat16 lo = __float2bfloat16_rn(pv[ql] - __bfloat162float(hi));
       const int off = sw_off(ql, (j & 63) >> 3);
       *reinterpret_cast<__nv_bfloat16 *>(base + off) = hi;
-      *reinterpret_cast<__nv_bfloat16 *>(base + 2 * kAcQAtom + off) = lo;
+      *reinterpret_cast<__nv_bfloat16 *>(base + 2 * QA + off) = lo;
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -745,19 +755,22 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
     if (ok) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const uint64_t dv = tc_desc(sVT + i * kAcAtom), dph = tc_desc(sQ + i * kAcQAtom),
-                       dpl = tc_desc(sQ + (2 + i) * kAcQAtom);
+        const uint64_t dv = tc_desc(sVT + i * kAcAtom), dph = tc_desc(sQ + i * QA),
+                       dpl = tc_desc(sQ + (2 + i) * QA);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // 16 positions per product
-          tc_mma(tmem + kAcQ, dv + 2 * kk, dph + 2 * kk, kIdesc, (i > 0 || kk > 0) ? 1u : 0u);
-          tc_mma(tmem + kAcQ, dv + 2 * kk, dpl + 2 * kk, kIdesc, 1u);
+          tc_mma(tmem + QN, dv + 2 * kk, dph + 2 * kk, kIdesc, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_mma(tmem + QN, dv + 2 * kk, dpl + 2 * kk, kIdesc, 1u);
         }
       }
     }
     tc_commit(&obar);
   }
   // meanwhile: the sum of p over the positions of each query
-  red[warp][lane] = warp_transpose_reduce<false>(pv, lane);
+  {
+    const float r = warp_transpose_reduce<false, QN>(pv, lane);
+    if (lane < QN) red[warp][lane] = r;
+  }
   __syncthreads();
   __syncwarp();
   ok = tc_wait(&obar, 0, a.error) && ok;
@@ -766,12 +779,12 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
   {
     // dim d = this thread's accumulator lane of O^T
     uint32_t v0[16], v1[16];
-    tmem_ld16(tlane + kAcQ, v0);
-    tmem_ld16(tlane + kAcQ + 16, v1);
+    tmem_ld16(tlane + QN, v0);
+    if constexpr (QN == 32) tmem_ld16(tlane + QN + 16, v1);
     const int d = threadIdx.x;
     if (d < HD) {
 #pragma unroll
-      for (int ql = 0; ql < kAcQ; ++ql)
+      for (int ql = 0; ql < QN; ++ql)
         if (ql < nq) a.opart[(slot0 + ql) * HD + d] = ok ? __uint_as_float(ql < 16 ? v0[ql] : v1[ql - 16]) : 0.f;
     }
   }
@@ -1195,8 +1208,10 @@ cudaError_t wide_accept_step(int B, int T, int s, const int32_t *argmax, int32_t
 
 cudaError_t wide_prepare() {
   WIDE_TRY(cudaFuncSetAttribute(wide_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes()));
-  WIDE_TRY(cudaFuncSetAttribute(wide_attn_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(64)));
-  return cudaFuncSetAttribute(wide_attn_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(128));
+  WIDE_TRY(cudaFuncSetAttribute(wide_attn_tc<64, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(16)));
+  WIDE_TRY(cudaFuncSetAttribute(wide_attn_tc<64, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(32)));
+  WIDE_TRY(cudaFuncSetAttribute(wide_attn_tc<128, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(16)));
+  return cudaFuncSetAttribute(wide_attn_tc<128, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes(32));
 }
 
 cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
@@ -1245,11 +1260,16 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       aa.opart = s.attn_o;
       aa.mlpart = s.attn_ml;
       aa.error = s.error;
-      const dim3 grid(nch, s.B * s.Hkv, (s.T * G + kAcQ - 1) / kAcQ);
-      if (s.hd == 64)
-        WIDE_TRY(launch(wide_attn_tc<64>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(64), st, aa));
+      const int qn = s.T * G <= 16 ? 16 : kAcQ;  // N of the products: the group's query vectors
+      const dim3 grid(nch, s.B * s.Hkv, (s.T * G + qn - 1) / qn);
+      if (s.hd == 64 && qn == 16)
+        WIDE_TRY(launch(wide_attn_tc<64, 16>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(16), st, aa));
+      else if (s.hd == 64)
+        WIDE_TRY(launch(wide_attn_tc<64, 32>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(32), st, aa));
+      else if (qn == 16)
+        WIDE_TRY(launch(wide_attn_tc<128, 16>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(16), st, aa));
       else
-        WIDE_TRY(launch(wide_attn_tc<128>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(128), st, aa));
+        WIDE_TRY(launch(wide_attn_tc<128, 32>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(32), st, aa));
       ++n;
       WIDE_TRY(launch(wide_attn_merge, dim3(M, s.Hq), dim3(s.hd), 0, st, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
                                                       s.attn_ml, s.xhi, s.xlo, ldx));
