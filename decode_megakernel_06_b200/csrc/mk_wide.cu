@@ -396,7 +396,10 @@ struct Split {
 };
 __device__ __forceinline__ float split_sum(const Split &p, int r, int col) {
   float s = 0.f;
-  for (int k = 0; k < p.ks; ++k) s += p.part[(static_cast<long long>(k) * p.rows + r) * p.ld + col];
+  const float *q = p.part + static_cast<long long>(r) * p.ld + col;
+  const long long step = static_cast<long long>(p.rows) * p.ld;
+#pragma unroll 4
+  for (int k = 0; k < p.ks; ++k) s += __ldcg(q + k * step);  // the loads go out together, the sum stays in order
   return s;
 }
 
