@@ -806,29 +806,40 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
 
 // Query (m, h)'s chunk partials combined with the log-sum-exp rule, written
 // straight into the bf16 pair that feeds the output projection (row m,
-// columns [h hd, h hd + hd)).  One block of hd threads per (row, head): warp 0
-// finds the largest chunk max and the weighted sum of the chunks' sums, then
-// thread i combines dim i.
+// columns [h hd, h hd + hd)).  One block of kMgGroups x hd threads per
+// (row, head).  Warp 0 folds the chunks' (max, sum) pairs into the overall
+// max and the weighted sum in one pass: each lane keeps a running pair over
+// its chunks, then the lanes' pairs are folded by shuffles.  Then thread group
+// r adds chunks r, r + kMgGroups, ... for dim i, and group 0 adds the groups'
+// sums in order and writes the result.
+constexpr int kMgGroups = 4;
 __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv, int hd, int nch_max,
                                 const float *opart, const float *mlpart, __nv_bfloat16 *xhi, __nv_bfloat16 *xlo,
                                 int ldx) {
   pdl_wait();
   pdl_launch();
   __shared__ float s_md[2];
+  __shared__ float s_num[kMgGroups - 1][128];
   const int m = blockIdx.x, h = blockIdx.y, b = m / T, t = m % T, G = Hq / Hkv, g = h / G;
   const int Q = T * G, qi = t * G + h % G, bg = b * Hkv + g;
   const int nch = (positions[b] + t) / kAcN + 1;  // chunks holding positions this query sees
   const long long slot0 = static_cast<long long>(bg) * nch_max * Q + qi;  // chunk c: slot0 + c Q
   if (threadIdx.x < 32) {
-    float M = -INFINITY;
-    for (int c = threadIdx.x; c < nch; c += 32) M = fmaxf(M, mlpart[2 * (slot0 + static_cast<long long>(c) * Q)]);
-    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float den = 0.f;
+    float M = -INFINITY, den = 0.f;
     for (int c = threadIdx.x; c < nch; c += 32) {
       const float *ml = mlpart + 2 * (slot0 + static_cast<long long>(c) * Q);
-      den = fmaf(expf(ml[0] - M), ml[1], den);  // a chunk this query sees nothing of has max -inf: weight 0
+      const float mc = ml[0];
+      if (mc == -INFINITY) continue;  // a chunk this query sees nothing of
+      const float nm = fmaxf(M, mc);
+      den = den * expf(M - nm) + ml[1] * expf(mc - nm);
+      M = nm;
     }
-    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    for (int o = 16; o; o >>= 1) {
+      const float oM = __shfl_xor_sync(0xffffffffu, M, o), od = __shfl_xor_sync(0xffffffffu, den, o);
+      const float nm = fmaxf(M, oM);
+      den = nm == -INFINITY ? 0.f : den * expf(M - nm) + od * expf(oM - nm);
+      M = nm;
+    }
     if (threadIdx.x == 0) {
       s_md[0] = M;
       s_md[1] = den;
@@ -836,13 +847,18 @@ __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv
   }
   __syncthreads();
   const float M = s_md[0], den = s_md[1];
-  for (int i = threadIdx.x; i < hd; i += blockDim.x) {
-    float num = 0.f;
+  const int grp = threadIdx.x / hd, i = threadIdx.x % hd;
+  float num = 0.f;
 #pragma unroll 4
-    for (int c = 0; c < nch; ++c) {
-      const long long slot = slot0 + static_cast<long long>(c) * Q;
-      num = fmaf(expf(mlpart[2 * slot] - M), opart[slot * hd + i], num);
-    }
+  for (int c = grp; c < nch; c += kMgGroups) {
+    const long long slot = slot0 + static_cast<long long>(c) * Q;
+    num = fmaf(expf(mlpart[2 * slot] - M), opart[slot * hd + i], num);
+  }
+  if (grp > 0) s_num[grp - 1][i] = num;
+  __syncthreads();
+  if (grp == 0) {
+#pragma unroll
+    for (int r = 0; r < kMgGroups - 1; ++r) num += s_num[r][i];
     const long long at = static_cast<long long>(m) * ldx + h * hd + i;
     split_store(num / den, xhi + at, xlo + at);
   }
@@ -1277,7 +1293,7 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       else
         WIDE_TRY(launch(wide_attn_tc<128, 32>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(32), st, aa));
       ++n;
-      WIDE_TRY(launch(wide_attn_merge, dim3(M, s.Hq), dim3(s.hd), 0, st, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
+      WIDE_TRY(launch(wide_attn_merge, dim3(M, s.Hq), dim3(kMgGroups * s.hd), 0, st, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
                                                       s.attn_ml, s.xhi, s.xlo, ldx));
       ++n;
     }
