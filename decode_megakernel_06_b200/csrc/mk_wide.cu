@@ -806,11 +806,11 @@ __global__ void __launch_bounds__(kAcThreads) wide_attn_tc(const __grid_constant
 
 // Query (m, h)'s chunk partials combined with the log-sum-exp rule, written
 // straight into the bf16 pair that feeds the output projection (row m,
-// columns [h hd, h hd + hd)).  One block of kMgGroups x hd threads per
-// (row, head).  Warp 0 folds the chunks' (max, sum) pairs into the overall
+// columns [h hd, h hd + hd)).  One block of groups x hd threads per (row,
+// head), groups = blockDim / hd (up to kMgGroups, more for longer caches).  Warp 0 folds the chunks' (max, sum) pairs into the overall
 // max and the weighted sum in one pass: each lane keeps a running pair over
 // its chunks, then the lanes' pairs are folded by shuffles.  Then thread group
-// r adds chunks r, r + kMgGroups, ... for dim i, and group 0 adds the groups'
+// r adds chunks r, r + groups, ... for dim i, and group 0 adds the groups'
 // sums in order and writes the result.
 constexpr int kMgGroups = 4;
 __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv, int hd, int nch_max,
@@ -847,18 +847,17 @@ __global__ void wide_attn_merge(const int32_t *positions, int T, int Hq, int Hkv
   }
   __syncthreads();
   const float M = s_md[0], den = s_md[1];
-  const int grp = threadIdx.x / hd, i = threadIdx.x % hd;
+  const int groups = blockDim.x / hd, grp = threadIdx.x / hd, i = threadIdx.x % hd;
   float num = 0.f;
 #pragma unroll 4
-  for (int c = grp; c < nch; c += kMgGroups) {
+  for (int c = grp; c < nch; c += groups) {
     const long long slot = slot0 + static_cast<long long>(c) * Q;
     num = fmaf(expf(mlpart[2 * slot] - M), opart[slot * hd + i], num);
   }
   if (grp > 0) s_num[grp - 1][i] = num;
   __syncthreads();
   if (grp == 0) {
-#pragma unroll
-    for (int r = 0; r < kMgGroups - 1; ++r) num += s_num[r][i];
+    for (int r = 0; r < groups - 1; ++r) num += s_num[r][i];
     const long long at = static_cast<long long>(m) * ldx + h * hd + i;
     split_store(num / den, xhi + at, xlo + at);
   }
@@ -1293,7 +1292,9 @@ cudaError_t wide_step(const WideStep &s, cudaStream_t st, int *launches) {
       else
         WIDE_TRY(launch(wide_attn_tc<128, 32>, dim3(grid), dim3(kAcThreads), attn_smem_bytes(32), st, aa));
       ++n;
-      WIDE_TRY(launch(wide_attn_merge, dim3(M, s.Hq), dim3(kMgGroups * s.hd), 0, st, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
+      // chunk groups per block: enough threads for long caches, few blocks' worth for short ones
+      const int mg = nch >= 32 ? kMgGroups : nch >= 16 ? 2 : 1;
+      WIDE_TRY(launch(wide_attn_merge, dim3(M, s.Hq), dim3(mg * s.hd), 0, st, s.positions_safe, s.T, s.Hq, s.Hkv, s.hd, nch, s.attn_o,
                                                       s.attn_ml, s.xhi, s.xlo, ldx));
       ++n;
     }
